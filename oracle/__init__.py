@@ -1,0 +1,161 @@
+"""fp64 CPU oracle for the Mamba mixer core -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, the smoke check and the benchmark's CPU-baseline leg use this
+package.  The product path (the CUDA library and its binding) never imports
+it, and the two share no code.
+
+The arithmetic lives in ``mixer_oracle.c`` (plain C, double precision, libm);
+this module compiles it with gcc on first use and marshals numpy arrays to it.
+Channels (or decode rows) are independent, so ``threads > 1`` only splits the
+channel range across threads; each thread runs the same sequential loop.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "mixer_oracle.c")
+_BUILD_DIR = os.path.join(_HERE, "_build")
+LIB_PATH = os.path.join(_BUILD_DIR, "libmixer_oracle.so")
+
+CFLAGS = ["-O2", "-fPIC", "-shared", "-std=c11", "-ffp-contract=off", "-fno-fast-math"]
+
+_lock = threading.Lock()
+_lib = None
+
+
+def compile_source(src: str, out: str) -> str:
+    """Compile one oracle C source into a shared library at ``out``."""
+    os.makedirs(os.path.dirname(out), exist_ok=True)
+    tmp = out + f".tmp{os.getpid()}"
+    subprocess.run(["gcc", *CFLAGS, "-o", tmp, src, "-lm"], check=True)
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    """Build the oracle library if it is missing or older than its source."""
+    if force or not os.path.exists(LIB_PATH) or os.path.getmtime(LIB_PATH) < os.path.getmtime(SOURCE):
+        compile_source(SOURCE, LIB_PATH)
+    return LIB_PATH
+
+
+def _declare(lib):
+    P = ctypes.c_void_p
+    I = ctypes.c_int64
+    lib.oracle_mixer_fwd.restype = ctypes.c_int
+    lib.oracle_mixer_fwd.argtypes = [P] * 17 + [I] * 7
+    lib.oracle_state_update.restype = ctypes.c_int
+    lib.oracle_state_update.argtypes = [P] * 13 + [I] * 7
+    return lib
+
+
+def load_library(path: str):
+    return _declare(ctypes.CDLL(path))
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = load_library(build())
+    return _lib
+
+
+def _f64(a):
+    if a is None:
+        return None
+    if hasattr(a, "detach"):  # torch tensor
+        a = a.detach().to("cpu")
+        import torch
+
+        a = a.to(torch.float64).numpy()
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _ranges(total: int, parts: int):
+    parts = max(1, min(parts, total)) if total > 0 else 1
+    bounds = [total * i // parts for i in range(parts + 1)]
+    return [(bounds[i], bounds[i + 1]) for i in range(parts)]
+
+
+def mixer_fwd(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, conv_state_in=None,
+              threads: int = 1, traces: bool = False, library=None):
+    """Run the oracle forward.  Arrays may be numpy or torch (any dtype; they are
+    widened to float64).  Returns a dict of float64 arrays: y [B,L,D],
+    h_last [B,D,N], conv_state_out [B,D,W-1] and, with ``traces``, u, delta
+    and pre (the conv output before SiLU), each [B,L,D]."""
+    L_ = library or lib()
+    xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0, conv_state_in = map(
+        _f64, (xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0, conv_state_in))
+    Bsz, L, twoD = xz.shape
+    D = twoD // 2
+    N = A.shape[-1]
+    W = conv_w.shape[-1]
+    assert A.shape == (D, N) and conv_w.shape == (D, W)
+    assert dt.shape == (Bsz, L, D) and Bm.shape == (Bsz, L, N) and Cm.shape == (Bsz, L, N)
+    y = np.zeros((Bsz, L, D))
+    h_last = np.zeros((Bsz, D, N))
+    cs_out = np.zeros((Bsz, D, max(W - 1, 0)))
+    tr = [np.zeros((Bsz, L, D)) for _ in range(3)] if traces else [None, None, None]
+
+    def run(rng):
+        rc = L_.oracle_mixer_fwd(_p(xz), _p(conv_w), _p(conv_b), _p(dt), _p(dt_bias), _p(A),
+                                 _p(Bm), _p(Cm), _p(Dskip), _p(h0), _p(conv_state_in),
+                                 _p(y), _p(h_last), _p(cs_out), _p(tr[0]), _p(tr[1]), _p(tr[2]),
+                                 Bsz, L, D, N, W, rng[0], rng[1])
+        if rc != 0:
+            raise ValueError(f"oracle_mixer_fwd rejected its arguments (rc={rc})")
+
+    parts = _ranges(D, threads)
+    if len(parts) == 1:
+        run(parts[0])
+    else:
+        with ThreadPoolExecutor(max_workers=len(parts)) as ex:
+            list(ex.map(run, parts))
+    out = {"y": y, "h_last": h_last, "conv_state_out": cs_out}
+    if traces:
+        out.update(u=tr[0], delta=tr[1], pre=tr[2])
+    return out
+
+
+def state_update(x, z, dt, conv_w, conv_b, dt_bias, Dskip, A, Bm, Cm, ssm_state, conv_state,
+                 threads: int = 1, library=None):
+    """Run the oracle decode step on copies of the carried state.  Returns a dict
+    with the new ssm_state [NL,B,D,N], conv_state [NL,B,D,W-1] and y [NL,B,D]."""
+    L_ = library or lib()
+    x, z, dt, conv_w, conv_b, dt_bias, Dskip, A, Bm, Cm = map(
+        _f64, (x, z, dt, conv_w, conv_b, dt_bias, Dskip, A, Bm, Cm))
+    ssm = _f64(ssm_state).copy()
+    cs = _f64(conv_state).copy() if conv_state is not None else None
+    NL, Bsz, D = x.shape
+    N = A.shape[-1]
+    W = conv_w.shape[-1]
+    y = np.zeros((NL, Bsz, D))
+    rows = NL * Bsz * D
+
+    def run(rng):
+        rc = L_.oracle_state_update(_p(x), _p(z), _p(dt), _p(conv_w), _p(conv_b), _p(dt_bias),
+                                    _p(Dskip), _p(A), _p(Bm), _p(Cm), _p(ssm), _p(cs), _p(y),
+                                    NL, Bsz, D, N, W, rng[0], rng[1])
+        if rc != 0:
+            raise ValueError(f"oracle_state_update rejected its arguments (rc={rc})")
+
+    parts = _ranges(rows, threads)
+    if len(parts) == 1:
+        run(parts[0])
+    else:
+        with ThreadPoolExecutor(max_workers=len(parts)) as ex:
+            list(ex.map(run, parts))
+    return {"ssm_state": ssm, "conv_state": cs, "y": y}

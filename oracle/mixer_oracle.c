@@ -1,0 +1,189 @@
+/*
+ * fp64 reference ("oracle") for the Mamba mixer core and its one-token decode
+ * step.  TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the
+ * benchmark's CPU-baseline leg call it; no product code links or calls it, and
+ * it shares no source with the CUDA library.
+ *
+ * It is the plain definition, written out as a sequential loop in double
+ * precision with libm exp/log1p, with no blocking, chunking or reordering:
+ *
+ *   Jamba hybrid SSM-Transformer lesson, section "SSM in one page":
+ *       h_t = A h_{t-1} + B x_t,   y_t = C h_t
+ *     (the output at t needs only h_{t-1} and x_t: constant memory, O(1) per
+ *     token), with A, B, C made data-dependent per token as in Mamba (the
+ *     "selective" part) and, for Mamba, a convolution applied to x_t before
+ *     the recurrence (section "Mamba-3", on the outer convolution it replaces).
+ *   Step size: the reproduction blog's profile section names Delta as the
+ *     parameter that sets how fast the state decays.
+ *   The discretised form, conv width, activations, skip and gate follow the
+ *   problem statement of the mixer core:
+ *       u_t   = SiLU(conv_b + sum_k conv_w[k] * x_{t-W+1+k})   (causal, depthwise)
+ *       Delta = softplus(dt_t + dt_bias)
+ *       h_t[n] = exp(Delta * A[n]) * h_{t-1}[n] + Delta * B_t[n] * u_t
+ *       y_t   = (sum_n C_t[n] h_t[n] + D * u_t) * SiLU(z_t)
+ *
+ * Readings taken where the sources are silent (each is listed with its reason
+ * in the design notes):
+ *   - conv_w[d, W-1] multiplies the current token (cross-correlation with W-1
+ *     tokens of left context), the left context being conv_state_in (raw,
+ *     pre-conv x, oldest first) or zeros;
+ *   - the skip term D multiplies u, the same conv+SiLU output that enters B x;
+ *   - the gate multiplies the sum (C h + D u) by SiLU(z); no norm on the path;
+ *   - A is given directly as a (negative) fp32 [D, N] matrix, not as log(-A);
+ *   - one B/C group shared by all channels of a sequence;
+ *   - softplus(v) = max(v, 0) + log1p(exp(-|v|)), exact for every v.
+ *
+ * Inputs are the exact values the GPU receives, widened to double; outputs
+ * stay unrounded in double.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#define OR_OK 0
+#define OR_ERR_ARG 1
+
+static double or_silu(double v) { return v / (1.0 + exp(-v)); }
+
+static double or_softplus(double v) { return fmax(v, 0.0) + log1p(exp(-fabs(v))); }
+
+/*
+ * Mixer forward over a whole sequence (prefill).
+ *
+ *   xz            [B, L, 2D]   x = xz[..., 0:D], z = xz[..., D:2D]
+ *   conv_w        [D, W]       conv_b [D] or NULL (= 0)
+ *   dt            [B, L, D]    pre-bias step input; dt_bias [D] or NULL (= 0)
+ *   A             [D, N]
+ *   Bm, Cm        [B, L, N]
+ *   Dskip         [D] or NULL (= 0)
+ *   h0            [B, D, N] or NULL (= 0)
+ *   conv_state_in [B, D, W-1] or NULL (= 0)
+ * Outputs (only channels d in [d_begin, d_end) are written):
+ *   y             [B, L, D]
+ *   h_last        [B, D, N]    state after token L-1
+ *   conv_state_out[B, D, W-1]  the last W-1 raw x, oldest first
+ *   u_trace, delta_trace [B, L, D] or NULL: u_t and Delta_t, for the checks
+ *   pre_trace     [B, L, D] or NULL: the conv output before SiLU
+ */
+int oracle_mixer_fwd(const double* xz, const double* conv_w, const double* conv_b,
+                     const double* dt, const double* dt_bias, const double* A,
+                     const double* Bm, const double* Cm, const double* Dskip,
+                     const double* h0, const double* conv_state_in,
+                     double* y, double* h_last, double* conv_state_out,
+                     double* u_trace, double* delta_trace, double* pre_trace,
+                     int64_t Bsz, int64_t L, int64_t D, int64_t N, int64_t W,
+                     int64_t d_begin, int64_t d_end)
+{
+    if (Bsz < 0 || L < 0 || D < 1 || N < 1 || N > 256 || W < 1 || W > 64) return OR_ERR_ARG;
+    if (d_begin < 0 || d_end > D || d_begin > d_end) return OR_ERR_ARG;
+    if (!xz && L > 0) return OR_ERR_ARG;
+    if (!conv_w || !dt || !A || !Bm || !Cm || !y || !h_last || !conv_state_out) return OR_ERR_ARG;
+
+    double h[256];
+    double win[64]; /* win[0..W-2]: the W-1 previous raw x, oldest first */
+
+    for (int64_t b = 0; b < Bsz; ++b) {
+        for (int64_t d = d_begin; d < d_end; ++d) {
+            for (int64_t j = 0; j < W - 1; ++j)
+                win[j] = conv_state_in ? conv_state_in[(b * D + d) * (W - 1) + j] : 0.0;
+            for (int64_t n = 0; n < N; ++n)
+                h[n] = h0 ? h0[(b * D + d) * N + n] : 0.0;
+
+            for (int64_t t = 0; t < L; ++t) {
+                const int64_t row = b * L + t;
+                const double x = xz[row * 2 * D + d];
+                const double z = xz[row * 2 * D + D + d];
+
+                /* causal depthwise conv, then SiLU */
+                double pre = conv_b ? conv_b[d] : 0.0;
+                for (int64_t k = 0; k < W - 1; ++k)
+                    pre += conv_w[d * W + k] * win[k];
+                pre += conv_w[d * W + (W - 1)] * x;
+                const double u = or_silu(pre);
+
+                /* step size */
+                const double delta = or_softplus(dt[row * D + d] + (dt_bias ? dt_bias[d] : 0.0));
+
+                /* selective recurrence and readout */
+                double acc = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    const double dA = exp(delta * A[d * N + n]);
+                    const double dBx = delta * Bm[row * N + n] * u;
+                    h[n] = dA * h[n] + dBx;
+                    acc += Cm[row * N + n] * h[n];
+                }
+                const double yv = acc + (Dskip ? Dskip[d] : 0.0) * u;
+                y[row * D + d] = yv * or_silu(z);
+
+                if (u_trace) u_trace[row * D + d] = u;
+                if (delta_trace) delta_trace[row * D + d] = delta;
+                if (pre_trace) pre_trace[row * D + d] = pre;
+
+                /* slide the window: drop the oldest, append this token's raw x */
+                for (int64_t j = 0; j + 1 < W - 1; ++j) win[j] = win[j + 1];
+                if (W > 1) win[W - 2] = x;
+            }
+
+            for (int64_t n = 0; n < N; ++n) h_last[(b * D + d) * N + n] = h[n];
+            for (int64_t j = 0; j < W - 1; ++j) conv_state_out[(b * D + d) * (W - 1) + j] = win[j];
+        }
+    }
+    return OR_OK;
+}
+
+/*
+ * One-token state update (decode) for NL independent stacked layers, in place.
+ * Written out on its own (not through the forward above) so the two can be
+ * checked against each other.
+ *
+ *   x, z, dt      [NL, B, D]
+ *   conv_w        [NL, D, W]; conv_b, dt_bias, Dskip [NL, D] (each may be NULL = 0)
+ *   A             [NL, D, N]
+ *   Bm, Cm        [NL, B, N]
+ *   ssm_state     [NL, B, D, N]   read, then overwritten with the new state
+ *   conv_state    [NL, B, D, W-1] read, then overwritten with the shifted window
+ *   y             [NL, B, D]
+ * Only rows r = (l * B + b) * D + d with r in [r_begin, r_end) are touched.
+ */
+int oracle_state_update(const double* x, const double* z, const double* dt,
+                        const double* conv_w, const double* conv_b,
+                        const double* dt_bias, const double* Dskip,
+                        const double* A, const double* Bm, const double* Cm,
+                        double* ssm_state, double* conv_state, double* y,
+                        int64_t NL, int64_t Bsz, int64_t D, int64_t N, int64_t W,
+                        int64_t r_begin, int64_t r_end)
+{
+    if (NL < 0 || Bsz < 0 || D < 1 || N < 1 || W < 1) return OR_ERR_ARG;
+    const int64_t rows = NL * Bsz * D;
+    if (r_begin < 0 || r_end > rows || r_begin > r_end) return OR_ERR_ARG;
+    if (!x || !z || !dt || !conv_w || !A || !Bm || !Cm || !ssm_state || !y) return OR_ERR_ARG;
+    if (W > 1 && !conv_state) return OR_ERR_ARG;
+
+    for (int64_t r = r_begin; r < r_end; ++r) {
+        const int64_t d = r % D;
+        const int64_t lb = r / D;          /* l * B + b */
+        const int64_t l = lb / Bsz;
+        const int64_t ld = l * D + d;      /* parameter row */
+
+        double* cs = conv_state ? conv_state + r * (W - 1) : NULL;
+        double pre = conv_b ? conv_b[ld] : 0.0;
+        for (int64_t k = 0; k < W - 1; ++k) pre += conv_w[ld * W + k] * cs[k];
+        pre += conv_w[ld * W + (W - 1)] * x[r];
+        const double u = or_silu(pre);
+
+        const double delta = or_softplus(dt[r] + (dt_bias ? dt_bias[ld] : 0.0));
+
+        double* h = ssm_state + r * N;
+        double acc = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+            const double dA = exp(delta * A[ld * N + n]);
+            h[n] = dA * h[n] + delta * Bm[lb * N + n] * u;
+            acc += Cm[lb * N + n] * h[n];
+        }
+        y[r] = (acc + (Dskip ? Dskip[ld] : 0.0) * u) * or_silu(z[r]);
+
+        for (int64_t k = 0; k + 1 < W - 1; ++k) cs[k] = cs[k + 1];
+        if (W > 1) cs[W - 2] = x[r];
+    }
+    return OR_OK;
+}

@@ -1,0 +1,353 @@
+"""Pins for the fp64 oracle: checks against facts that do not come from the
+oracle itself (closed forms, library routines, brute force, invariants).
+
+Every pin takes the oracle's ctypes library as an argument so the same pins
+can be run against deliberately broken copies of the oracle (see
+test_oracle_mutants.py): a plausible mistake anywhere in the oracle must make
+at least one pin fail.
+
+Where the passages come from:
+  * Jamba hybrid SSM-Transformer lesson, section "SSM in one page": the
+    recurrence h_t = A h_{t-1} + B x_t, y_t = C h_t; constant memory and O(1)
+    per token (only h_{t-1} and x_t are needed); S4's structured A evaluated as
+    a long convolution; Mamba makes A, B, C data-dependent.
+  * the mixer-core problem statement: conv width 4 + SiLU, Delta = softplus(dt +
+    dt_bias), dA = exp(Delta A), h_t = dA h_{t-1} + Delta B_t x_t, y_t = C_t h_t +
+    D x_t gated by SiLU(z), and the one-token decode step.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import scipy.signal
+import scipy.special
+
+import oracle
+
+W = 4
+
+
+def lib_silu(v):
+    """SiLU through scipy's logistic function (library routine)."""
+    return v * scipy.special.expit(v)
+
+
+def lib_softplus(v):
+    """softplus through numpy's logaddexp (library routine)."""
+    return np.logaddexp(0.0, v)
+
+
+def _rand_case(rng, B, L, D, N, *, h0=True, cs=True, conv_b=True, dskip=True):
+    xz = rng.standard_normal((B, L, 2 * D))
+    dt = 0.3 * rng.standard_normal((B, L, D))
+    conv_w = rng.uniform(-0.6, 0.6, (D, W))
+    cb = 0.2 * rng.standard_normal(D) if conv_b else None
+    dt_bias = rng.uniform(-4.0, 0.5, D)
+    A = -np.exp(rng.uniform(np.log(0.3), np.log(5.0), (D, N)))
+    Bm = rng.standard_normal((B, L, N))
+    Cm = rng.standard_normal((B, L, N))
+    Dsk = rng.normal(1.0, 0.3, D) if dskip else None
+    h0 = 0.5 * rng.standard_normal((B, D, N)) if h0 else None
+    csi = rng.standard_normal((B, D, W - 1)) if cs else None
+    return dict(xz=xz, conv_w=conv_w, conv_b=cb, dt=dt, dt_bias=dt_bias, A=A, Bm=Bm, Cm=Cm,
+                Dskip=Dsk, h0=h0, conv_state_in=csi)
+
+
+def _fwd(lib, case, **kw):
+    return oracle.mixer_fwd(case["xz"], case["conv_w"], case["conv_b"], case["dt"], case["dt_bias"],
+                            case["A"], case["Bm"], case["Cm"], case["Dskip"], case["h0"],
+                            case["conv_state_in"], library=lib, **kw)
+
+
+def _lib_conv(case):
+    """Pre-activation conv through numpy.convolve with the reversed kernel:
+    pre_t = conv_b + sum_k w[k] * xpad[t + k], xpad = (left context, x)."""
+    xz = case["xz"]
+    B, L, twoD = xz.shape
+    D = twoD // 2
+    pre = np.zeros((B, L, D))
+    for b in range(B):
+        for d in range(D):
+            left = case["conv_state_in"][b, d] if case["conv_state_in"] is not None else np.zeros(W - 1)
+            xp = np.concatenate([left, xz[b, :, d]])
+            pre[b, :, d] = np.convolve(xp, case["conv_w"][d][::-1], mode="valid")
+            if case["conv_b"] is not None:
+                pre[b, :, d] += case["conv_b"][d]
+    return pre
+
+
+def _lib_u_delta(case):
+    pre = _lib_conv(case)
+    u = lib_silu(pre)
+    bias = case["dt_bias"] if case["dt_bias"] is not None else 0.0
+    delta = lib_softplus(case["dt"] + bias)
+    return pre, u, delta
+
+
+def _gate_z(case):
+    D = case["xz"].shape[2] // 2
+    return lib_silu(case["xz"][:, :, D:])
+
+
+# --------------------------------------------------------------------------- P1
+def pin_lti_closed_form(lib):
+    """Constant Delta and time-invariant B, C: the recurrence is an LTI system,
+    so y equals the long convolution of u with K_k = sum_n C_n a_n^k Delta B_n,
+    plus the free response of h0 (S4 evaluated as a long convolution)."""
+    rng = np.random.default_rng(101)
+    B, L, D, N = 2, 48, 3, 6
+    case = _rand_case(rng, B, L, D, N)
+    case["dt"] = np.zeros((B, L, D))                         # Delta constant per channel
+    bvec = rng.standard_normal((B, N))
+    cvec = rng.standard_normal((B, N))
+    case["Bm"] = np.repeat(bvec[:, None, :], L, axis=1)
+    case["Cm"] = np.repeat(cvec[:, None, :], L, axis=1)
+    got = _fwd(lib, case)
+
+    _, u, _ = _lib_u_delta(case)
+    g = _gate_z(case)
+    for b in range(B):
+        for d in range(D):
+            dlt = lib_softplus(case["dt_bias"][d])
+            a = np.exp(dlt * case["A"][d])                     # [N]
+            k = np.arange(L)
+            K = (cvec[b][None, :] * a[None, :] ** k[:, None] * dlt * bvec[b][None, :]).sum(1)
+            free = (cvec[b][None, :] * a[None, :] ** (k[:, None] + 1) * case["h0"][b, d][None, :]).sum(1)
+            ssm = np.convolve(u[b, :, d], K)[:L] + free
+            y = (ssm + case["Dskip"][d] * u[b, :, d]) * g[b, :, d]
+            np.testing.assert_allclose(got["y"][b, :, d], y, rtol=1e-10, atol=1e-12)
+            hl = np.array([sum(a[n] ** j * dlt * bvec[b, n] * u[b, L - 1 - j, d] for j in range(L))
+                           + a[n] ** L * case["h0"][b, d, n] for n in range(N)])
+            np.testing.assert_allclose(got["h_last"][b, d], hl, rtol=1e-10, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- P2
+def pin_brute_force_selective(lib):
+    """Selective case on tiny inputs against the materialised sum
+    y_t = sum_{s<=t} C_t (prod_{r=s+1..t} dA_r) Delta_s B_s u_s
+          + C_t (prod_{r=0..t} dA_r) h0 + D u_t, gated by SiLU(z_t)."""
+    rng = np.random.default_rng(202)
+    B, L, D, N = 2, 14, 3, 5
+    case = _rand_case(rng, B, L, D, N)
+    got = _fwd(lib, case)
+    _, u, delta = _lib_u_delta(case)
+    g = _gate_z(case)
+    for b in range(B):
+        for d in range(D):
+            dA = np.exp(delta[b, :, d][:, None] * case["A"][d][None, :])   # [L, N]
+            hs = np.zeros((L, N))
+            for t in range(L):
+                acc = np.prod(dA[0:t + 1], axis=0) * case["h0"][b, d]
+                for s in range(t + 1):
+                    acc = acc + np.prod(dA[s + 1:t + 1], axis=0) * delta[b, s, d] * case["Bm"][b, s] * u[b, s, d]
+                hs[t] = acc
+            y = ((case["Cm"][b] * hs).sum(1) + case["Dskip"][d] * u[b, :, d]) * g[b, :, d]
+            np.testing.assert_allclose(got["y"][b, :, d], y, rtol=1e-10, atol=1e-12)
+            np.testing.assert_allclose(got["h_last"][b, d], hs[-1], rtol=1e-10, atol=1e-12)
+            np.testing.assert_allclose(got["conv_state_out"][b, d], case["xz"][b, L - (W - 1):, d], rtol=0, atol=0)
+
+
+# --------------------------------------------------------------------------- P3
+def pin_zero_input(lib):
+    """x = 0, conv_b = 0, h0 = 0, zero conv context => y = 0 and h_last = 0."""
+    rng = np.random.default_rng(303)
+    B, L, D, N = 2, 17, 4, 16
+    case = _rand_case(rng, B, L, D, N, h0=False, cs=False, conv_b=False)
+    case["xz"][:, :, :D] = 0.0
+    got = _fwd(lib, case)
+    assert np.all(got["y"] == 0.0)
+    assert np.all(got["h_last"] == 0.0)
+    assert np.all(got["conv_state_out"] == 0.0)
+    # and the output is not identically zero once x is not
+    case["xz"][:, 3, :D] = 1.0
+    got = _fwd(lib, case)
+    assert np.abs(got["y"][:, 3:]).max() > 1e-3
+
+
+# --------------------------------------------------------------------------- P4
+def pin_split_equals_unsplit(lib):
+    """Running the sequence in pieces, carrying (h_last, conv_state_out) into
+    (h0, conv_state_in), equals the single run exactly: the state is all the
+    history the next token needs.  Pieces shorter than the conv window included."""
+    rng = np.random.default_rng(404)
+    B, L, D, N = 2, 37, 3, 16
+    case = _rand_case(rng, B, L, D, N)
+    full = _fwd(lib, case)
+    cuts = [0, 1, 3, 4, 20, 37]
+    h, cs = case["h0"], case["conv_state_in"]
+    ys = []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        piece = dict(case)
+        piece.update(xz=case["xz"][:, a:b], dt=case["dt"][:, a:b], Bm=case["Bm"][:, a:b],
+                     Cm=case["Cm"][:, a:b], h0=h, conv_state_in=cs)
+        out = _fwd(lib, piece)
+        ys.append(out["y"])
+        h, cs = out["h_last"], out["conv_state_out"]
+    assert np.array_equal(np.concatenate(ys, axis=1), full["y"])
+    assert np.array_equal(h, full["h_last"])
+    assert np.array_equal(cs, full["conv_state_out"])
+
+
+# --------------------------------------------------------------------------- P5
+def _decode_case_from_scan(case, t, layers):
+    """The decode-step arguments for token t of a stack of independent scans,
+    one per layer (layer l uses scan case layers[l])."""
+    D = case[0]["xz"].shape[2] // 2
+    get = lambda k: np.stack([c[k] for c in case])  # noqa: E731
+    x = np.stack([c["xz"][:, t, :D] for c in case])
+    z = np.stack([c["xz"][:, t, D:] for c in case])
+    dt = np.stack([c["dt"][:, t] for c in case])
+    Bm = np.stack([c["Bm"][:, t] for c in case])
+    Cm = np.stack([c["Cm"][:, t] for c in case])
+    return dict(x=x, z=z, dt=dt, conv_w=get("conv_w"), conv_b=get("conv_b"), dt_bias=get("dt_bias"),
+                Dskip=get("Dskip"), A=get("A"), Bm=Bm, Cm=Cm)
+
+
+def pin_decode_equals_last_scan_step(lib):
+    """The one-token state update applied to the state after L-1 tokens equals
+    the scan's token L-1 (output, state, window); and k successive decode steps
+    equal a k-token scan.  Two stacked layers with different parameters."""
+    rng = np.random.default_rng(505)
+    B, L, D, N, NL = 3, 9, 4, 16, 2
+    cases = [_rand_case(rng, B, L, D, N) for _ in range(NL)]
+    fulls = [_fwd(lib, c) for c in cases]
+    # state after L-1 tokens, from the scan
+    heads = []
+    for c in cases:
+        p = dict(c)
+        p.update(xz=c["xz"][:, :L - 1], dt=c["dt"][:, :L - 1], Bm=c["Bm"][:, :L - 1], Cm=c["Cm"][:, :L - 1])
+        heads.append(_fwd(lib, p))
+    args = _decode_case_from_scan(cases, L - 1, NL)
+    ssm = np.stack([hd["h_last"] for hd in heads])
+    cs = np.stack([hd["conv_state_out"] for hd in heads])
+    out = oracle.state_update(**args, ssm_state=ssm, conv_state=cs, library=lib)
+    for l in range(NL):
+        np.testing.assert_allclose(out["y"][l], fulls[l]["y"][:, L - 1], rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(out["ssm_state"][l], fulls[l]["h_last"], rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(out["conv_state"][l], fulls[l]["conv_state_out"], rtol=0, atol=0)
+    # k decode steps from the initial state == k-token scan
+    ssm = np.stack([c["h0"] for c in cases])
+    cs = np.stack([c["conv_state_in"] for c in cases])
+    for t in range(L):
+        args = _decode_case_from_scan(cases, t, NL)
+        out = oracle.state_update(**args, ssm_state=ssm, conv_state=cs, library=lib)
+        for l in range(NL):
+            np.testing.assert_allclose(out["y"][l], fulls[l]["y"][:, t], rtol=1e-12, atol=1e-13)
+        ssm, cs = out["ssm_state"], out["conv_state"]
+    for l in range(NL):
+        np.testing.assert_allclose(ssm[l], fulls[l]["h_last"], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(cs[l], fulls[l]["conv_state_out"], rtol=0, atol=0)
+
+
+# --------------------------------------------------------------------------- P6
+def pin_conv_stage(lib):
+    """The conv stage equals numpy.convolve with the reversed kernel over the
+    sequence left-padded by the carried window, and u = SiLU of it."""
+    rng = np.random.default_rng(606)
+    for with_cs in (True, False):
+        case = _rand_case(rng, 2, 11, 5, 4, cs=with_cs)
+        got = _fwd(lib, case, traces=True)
+        pre, u, delta = _lib_u_delta(case)
+        np.testing.assert_allclose(got["pre"], pre, rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(got["u"], u, rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(got["delta"], delta, rtol=1e-13, atol=1e-15)
+
+
+# --------------------------------------------------------------------------- P7
+def pin_first_order_iir(lib):
+    """N = 1 with constant decay a: h_t = a h_{t-1} + b_t is the first-order IIR
+    filter 1 / (1 - a z^-1); compare with scipy.signal.lfilter."""
+    rng = np.random.default_rng(707)
+    B, L, D, N = 1, 40, 3, 1
+    case = _rand_case(rng, B, L, D, N, conv_b=False)
+    case["dt"] = np.zeros((B, L, D))
+    case["conv_w"] = np.tile(np.array([0.0, 0.0, 0.0, 1.0]), (D, 1))  # pre = x_t
+    case["Cm"] = np.ones((B, L, N))
+    case["Dskip"] = np.zeros(D)
+    got = _fwd(lib, case)
+    x = case["xz"][0, :, :D]
+    g = _gate_z(case)[0]
+    for d in range(D):
+        dlt = lib_softplus(case["dt_bias"][d])
+        a = np.exp(dlt * case["A"][d, 0])
+        drive = dlt * case["Bm"][0, :, 0] * lib_silu(x[:, d])
+        h, _ = scipy.signal.lfilter([1.0], [1.0, -a], drive, zi=[a * case["h0"][0, d, 0]])
+        np.testing.assert_allclose(got["y"][0, :, d], h * g[:, d], rtol=1e-11, atol=1e-13)
+        np.testing.assert_allclose(got["h_last"][0, d, 0], h[-1], rtol=1e-11, atol=1e-13)
+
+
+# --------------------------------------------------------------------------- P8
+def pin_A_zero(lib):
+    """A = 0: no decay, h_t = h0 + prefix sum of Delta u B."""
+    rng = np.random.default_rng(808)
+    B, L, D, N = 2, 25, 3, 7
+    case = _rand_case(rng, B, L, D, N)
+    case["A"] = np.zeros((D, N))
+    got = _fwd(lib, case)
+    _, u, delta = _lib_u_delta(case)
+    g = _gate_z(case)
+    for b in range(B):
+        for d in range(D):
+            hs = case["h0"][b, d][None, :] + np.cumsum((delta[b, :, d] * u[b, :, d])[:, None] * case["Bm"][b], axis=0)
+            y = ((case["Cm"][b] * hs).sum(1) + case["Dskip"][d] * u[b, :, d]) * g[b, :, d]
+            np.testing.assert_allclose(got["y"][b, :, d], y, rtol=1e-11, atol=1e-13)
+            np.testing.assert_allclose(got["h_last"][b, d], hs[-1], rtol=1e-11, atol=1e-13)
+
+
+# --------------------------------------------------------------------------- P9
+def pin_softplus_roundtrip(lib):
+    """dt = 0 and dt_bias = inverse-softplus(v) give Delta = v; softplus is
+    exact far into both tails."""
+    rng = np.random.default_rng(909)
+    D = 8
+    v = np.exp(rng.uniform(np.log(1e-3), np.log(1e-1), D))
+    case = _rand_case(rng, 1, 3, D, 2)
+    case["dt"] = np.zeros((1, 3, D))
+    case["dt_bias"] = np.log(np.expm1(v))
+    got = _fwd(lib, case, traces=True)
+    np.testing.assert_allclose(got["delta"][0], np.tile(v, (3, 1)), rtol=1e-13, atol=0)
+    case["dt_bias"] = np.array([-60.0, -30.0, -1.0, 0.0, 1.0, 30.0, 60.0, 700.0])
+    got = _fwd(lib, case, traces=True)
+    expect = np.array([np.exp(-60.0), np.log1p(np.exp(-30.0)), np.log1p(np.exp(-1.0)), np.log(2.0),
+                       1.0 + np.log1p(np.exp(-1.0)), 30.0 + np.exp(-30.0), 60.0, 700.0])
+    np.testing.assert_allclose(got["delta"][0, 0], expect, rtol=1e-14, atol=0)
+
+
+# --------------------------------------------------------------------------- P10
+def pin_skip_and_gate(lib):
+    """C = 0 removes the state from the output: y = D u SiLU(z); the gate
+    is SiLU of z (not of x), applied after the skip is added."""
+    rng = np.random.default_rng(1010)
+    B, L, D, N = 2, 9, 4, 3
+    case = _rand_case(rng, B, L, D, N)
+    case["Cm"] = np.zeros((B, L, N))
+    got = _fwd(lib, case)
+    _, u, _ = _lib_u_delta(case)
+    np.testing.assert_allclose(got["y"], case["Dskip"][None, None, :] * u * _gate_z(case), rtol=1e-13, atol=1e-15)
+
+
+# --------------------------------------------------------------------------- P11
+def pin_channel_split(lib):
+    """Channels are independent: splitting the channel range across threads
+    gives bit-identical results."""
+    rng = np.random.default_rng(1111)
+    case = _rand_case(rng, 2, 13, 7, 16)
+    a = _fwd(lib, case, threads=1)
+    b = _fwd(lib, case, threads=3)
+    for k in a:
+        assert np.array_equal(a[k], b[k])
+
+
+ALL_PINS = [
+    pin_lti_closed_form,
+    pin_brute_force_selective,
+    pin_zero_input,
+    pin_split_equals_unsplit,
+    pin_decode_equals_last_scan_step,
+    pin_conv_stage,
+    pin_first_order_iir,
+    pin_A_zero,
+    pin_softplus_roundtrip,
+    pin_skip_and_gate,
+    pin_channel_split,
+]

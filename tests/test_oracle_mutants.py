@@ -1,0 +1,75 @@
+"""Plants plausible mistakes in copies of the oracle (on the CPU) and checks
+that each one makes at least one pin fail, so the pins really constrain every
+step of the oracle: conv, SiLU, softplus, discretisation, recurrence, readout,
+skip, gate, carried state and the decode step."""
+
+import os
+
+import pytest
+
+import oracle
+from pins import ALL_PINS
+
+# (name, exact text in the oracle source, replacement)
+MUTANTS = [
+    ("drop_skip", "const double yv = acc + (Dskip ? Dskip[d] : 0.0) * u;", "const double yv = acc;"),
+    ("gate_by_z", "y[row * D + d] = yv * or_silu(z);", "y[row * D + d] = yv * z;"),
+    ("gate_by_x", "y[row * D + d] = yv * or_silu(z);", "y[row * D + d] = yv * or_silu(x);"),
+    ("conv_current_tap", "pre += conv_w[d * W + (W - 1)] * x;", "pre += conv_w[d * W + 0] * x;"),
+    ("conv_window_tap", "pre += conv_w[d * W + k] * win[k];", "pre += conv_w[d * W + k + 1] * win[k];"),
+    ("conv_bias_dropped", "double pre = conv_b ? conv_b[d] : 0.0;\n                for", "double pre = 0.0;\n                for"),
+    ("silu_sign", "return v / (1.0 + exp(-v));", "return v / (1.0 + exp(v));"),
+    ("softplus_no_log", "log1p(exp(-fabs(v)))", "exp(-fabs(v))"),
+    ("dt_bias_dropped", "dt[row * D + d] + (dt_bias ? dt_bias[d] : 0.0)", "dt[row * D + d]"),
+    ("A_sign", "const double dA = exp(delta * A[d * N + n]);", "const double dA = exp(-delta * A[d * N + n]);"),
+    ("A_transposed", "const double dA = exp(delta * A[d * N + n]);", "const double dA = exp(delta * A[n * D + d]);"),
+    ("dA_not_exp", "const double dA = exp(delta * A[d * N + n]);", "const double dA = 1.0 + delta * A[d * N + n];"),
+    ("dBx_no_delta", "const double dBx = delta * Bm[row * N + n] * u;", "const double dBx = Bm[row * N + n] * u;"),
+    ("dBx_raw_x", "const double dBx = delta * Bm[row * N + n] * u;", "const double dBx = delta * Bm[row * N + n] * x;"),
+    ("B_previous_token", "const double dBx = delta * Bm[row * N + n] * u;",
+     "const double dBx = delta * Bm[(t > 0 ? row - 1 : row) * N + n] * u;"),
+    ("C_as_B", "acc += Cm[row * N + n] * h[n];", "acc += Bm[row * N + n] * h[n];"),
+    ("readout_before_update",
+     "h[n] = dA * h[n] + dBx;\n                    acc += Cm[row * N + n] * h[n];",
+     "acc += Cm[row * N + n] * h[n];\n                    h[n] = dA * h[n] + dBx;"),
+    ("h0_ignored", "h[n] = h0 ? h0[(b * D + d) * N + n] : 0.0;", "h[n] = 0.0;"),
+    ("conv_state_ignored", "win[j] = conv_state_in ? conv_state_in[(b * D + d) * (W - 1) + j] : 0.0;", "win[j] = 0.0;"),
+    ("window_not_appended", "if (W > 1) win[W - 2] = x;", "if (W > 1) win[W - 2] = 0.0;"),
+    ("window_order", "for (int64_t j = 0; j + 1 < W - 1; ++j) win[j] = win[j + 1];",
+     "for (int64_t j = W - 3; j >= 0; --j) win[j + 1] = win[j];"),
+    ("h_last_not_written", "for (int64_t n = 0; n < N; ++n) h_last[(b * D + d) * N + n] = h[n];",
+     "for (int64_t n = 0; n < N; ++n) h_last[(b * D + d) * N + n] = 0.0;"),
+    ("decode_A_sign", "const double dA = exp(delta * A[ld * N + n]);", "const double dA = exp(-delta * A[ld * N + n]);"),
+    ("decode_readout_before_update",
+     "h[n] = dA * h[n] + delta * Bm[lb * N + n] * u;\n            acc += Cm[lb * N + n] * h[n];",
+     "acc += Cm[lb * N + n] * h[n];\n            h[n] = dA * h[n] + delta * Bm[lb * N + n] * u;"),
+    ("decode_window_not_shifted", "for (int64_t k = 0; k + 1 < W - 1; ++k) cs[k] = cs[k + 1];", ""),
+    ("decode_params_of_layer0", "const int64_t ld = l * D + d;", "const int64_t ld = d;"),
+    ("decode_no_skip", "y[r] = (acc + (Dskip ? Dskip[ld] : 0.0) * u) * or_silu(z[r]);", "y[r] = acc * or_silu(z[r]);"),
+]
+
+
+def _run_pins(lib):
+    failed = []
+    for pin in ALL_PINS:
+        try:
+            pin(lib)
+        except (AssertionError, ValueError, FloatingPointError):
+            failed.append(pin.__name__)
+    return failed
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(tmp_path, name, old, new):
+    src = open(oracle.SOURCE).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    mutated = tmp_path / f"mut_{name}.c"
+    mutated.write_text(src.replace(old, new))
+    so = oracle.compile_source(str(mutated), str(tmp_path / f"libmut_{name}.so"))
+    lib = oracle.load_library(so)
+    failed = _run_pins(lib)
+    assert failed, f"mutant {name} passed every pin"
+
+
+def test_unmutated_passes_all_pins():
+    assert _run_pins(oracle.lib()) == []
