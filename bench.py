@@ -1,0 +1,487 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 Mamba mixer core.
+
+One step = one fused selective-scan forward (conv + SiLU, softplus step,
+discretisation, fp32 recurrence, readout, D-skip, SiLU(z) gate, carried state
+out) over one Jamba-shaped layer's prefill: batch 1, 4096 tokens, d_inner 8192
+(hidden 4096 x expand 2), d_state 16, conv width 4, bf16 activations and fp32
+state.  The one-token decode update across 28 stacked layers at batch 128 is
+measured in the same run and reported under "decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+N > 1 is launched with torchrun (one process per GPU).  The path has no data
+exchange between GPUs, so every rank runs the same independent workload
+(replicas, weak scaling) and rank 0 prints one JSON line with the whole-job
+throughput over the slowest rank's device time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from workloads import CONFIGS, make_decode_inputs, make_mixer_inputs  # noqa: E402
+
+METRIC = "Mamba mixer tokens/s per layer (d_inner 8192) and % of B200 HBM roofline"
+PREFILL = CONFIGS["jamba_prefill"]
+DECODE = CONFIGS["decode_28x128"]
+
+SMS = 148
+FP32_LANES_PER_SM = 128
+SM_MAX_MHZ_FALLBACK = 1965.0
+HBM_FALLBACK_GBS = 6650.0
+
+# Algorithmic fp32-pipe work of the forward per (token, channel): for each of
+# the 16 states a decay factor, the Delta*u*B product, the state FMA and the
+# readout FMA (4 x 16), plus the 4 conv taps, Delta*u, the skip FMA and the
+# gate product.  Transcendentals (softplus, SiLU x2, one exp per token-channel
+# at least) run on the MUFU pipe and are not counted.
+FWD_FP32_OPS_PER_TOKEN_CHANNEL = 16 * 4 + 4 + 1 + 1 + 1
+
+
+def prefill_bytes(B, L, D, N=16, W=4, es=2, h0=False, cs_in=False):
+    """Algorithmic HBM bytes of one forward call: xz, dt, B, C in and y out
+    per token; parameters once; carried state in (if given) and out."""
+    per_token = 2 * D * es + D * es + 2 * N * es + D * es
+    params = D * (W * 4 + 4 + 4 + N * 4 + 4)
+    state = B * D * (N * 4 + (W - 1) * es) * (1 + (1 if h0 else 0))
+    if cs_in and not h0:
+        state += B * D * (W - 1) * es
+    return B * L * per_token + params + state
+
+
+def decode_bytes(NL, B, D, N=16, W=4, es=2):
+    per_row = D * (2 * 4 * N + 2 * es * (W - 1) + 3 * es + es) + 2 * N * es
+    params = D * (W * 4 + 4 + 4 + 4 + N * 4)
+    return NL * B * per_row + NL * params
+
+
+def _measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f)
+    except (OSError, ValueError):
+        return None
+
+
+def _kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mamba_selective_scan_core_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _ncu_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel_key)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_sha") != _kernel_source_sha():
+        return None
+    return rec.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "sw_power_cap": 0x4,
+    }
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.index = index
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM))
+            self.ok = True
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(float(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- distributed
+def _dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return rank, local, world
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def _max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- GPU arm
+def _fwd_call(mm, d, out):
+    mm.mixer_fwd(d["xz"], d["conv_w"], d["conv_b"], d["dt"], d["dt_bias"], d["A"], d["Bm"], d["Cm"], d["Dskip"],
+                 d["h0"], d["conv_state_in"], y=out[0], h_last=out[1], conv_state_out=out[2])
+
+
+def run_gpu(args):
+    rank, local, world = _dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    import mamba_selective_scan_core_b200 as mm
+
+    mm.lib()
+    cfg = PREFILL
+    B, L, D = cfg.batch, cfg.seqlen, cfg.d_inner
+    host = make_mixer_inputs(cfg)
+    nsets = 2   # rotate input sets so no step finds the previous step's data in L2
+    sets = [{k: (v.cuda() if v is not None else None) for k, v in host.items()} for _ in range(nsets)]
+    outs = [(torch.empty((B, L, D), dtype=torch.bfloat16, device="cuda"),
+             torch.empty((B, D, 16), device="cuda"),
+             torch.empty((B, D, 3), dtype=torch.bfloat16, device="cuda")) for _ in range(nsets)]
+    stream = torch.cuda.current_stream()
+
+    for i in range(args.warmup):
+        _fwd_call(mm, sets[i % nsets], outs[i % nsets])
+    torch.cuda.synchronize()
+
+    # ---- device-timed region: exactly K steps
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    clk = ClockSampler(local)
+    clk.start()
+    _barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        _fwd_call(mm, sets[i % nsets], outs[i % nsets])
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    _barrier(world)
+    clk.stop()
+    region_ms = t0.elapsed_time(t1)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    region_ms_max = _max_over_ranks(region_ms, world)
+    tokens = B * L
+    value = world * tokens * K / (region_ms_max * 1e-3)
+    avg_launch_s = statistics.mean(launch_ms) * 1e-3
+
+    # ---- roofline of the forward kernel
+    peaks = _measured_peaks()
+    hbm_peak = float(peaks["hbm_gbs"]) if peaks and "hbm_gbs" in peaks else HBM_FALLBACK_GBS
+    hbm_src = "measured" if peaks and "hbm_gbs" in peaks else "fallback"
+    nbytes = prefill_bytes(B, L, D, h0=host["h0"] is not None, cs_in=host["conv_state_in"] is not None)
+    hbm_gbs = nbytes / avg_launch_s / 1e9
+    sm_max = clk.max_mhz or SM_MAX_MHZ_FALLBACK
+    alu_peak = SMS * FP32_LANES_PER_SM * sm_max * 1e6 / 1e12       # T fp32 lane-ops/s
+    alu_ops = FWD_FP32_OPS_PER_TOKEN_CHANNEL * tokens * D
+    alu_ach = alu_ops / avg_launch_s / 1e12
+    traffic = _ncu_traffic("mixer_fwd_kernel/jamba_prefill")
+    hbm_part = {"bound": "hbm", "achieved": round(hbm_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(hbm_gbs / hbm_peak, 4), "traffic": traffic,
+                "algorithmic_bytes": nbytes, "peak_source": hbm_src}
+    alu_part = {"bound": "alu", "achieved": round(alu_ach, 3), "peak": round(alu_peak, 3),
+                "unit": "T fp32-pipe ops/s", "frac": round(alu_ach / alu_peak, 4), "traffic": traffic,
+                "ops_per_token_channel": FWD_FP32_OPS_PER_TOKEN_CHANNEL,
+                "peak_source": "148 SMs x 128 fp32 lanes x max SM clock"}
+    roofline, other = (alu_part, hbm_part) if alu_part["frac"] >= hbm_part["frac"] else (hbm_part, alu_part)
+
+    # ---- end to end through the public API with host buffers
+    e2e = run_e2e(mm, host, args, world)
+
+    # ---- decode state update (28 layers x batch 128)
+    dec = run_decode(mm, args, world, hbm_peak, hbm_src)
+
+    result = None
+    if rank == 0:
+        cpu = cpu_baseline(host, cfg) if world == 1 and not args.no_cpu_baseline else None
+        result = {
+            "metric": METRIC,
+            "value": round(value, 1),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": round(region_ms_max / K, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) x/z/B/C, 0.1 N(0,1) dt, log-uniform softplus(dt_bias), "
+                    "A[d,n] = -(n+1), D ~ N(1, 0.1), fp32 state",
+            "config": {"workload": cfg.name, "batch": B, "seq_len": L, "d_inner": D, "d_state": 16, "d_conv": 4,
+                       "act": "bf16", "parallelism": f"replicas x{world}",
+                       "l2": "inputs (270 MB/step) larger than L2, rotated over 2 buffer sets"},
+            "roofline": roofline,
+            "roofline_other": other,
+            "hbm_frac": hbm_part["frac"],
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": K,
+            "clocks": clk.summary(),
+            "decode": dec,
+            "launch_ms": {"mean": round(statistics.mean(launch_ms), 5), "min": round(min(launch_ms), 5),
+                          "max": round(max(launch_ms), 5)},
+        }
+    return result, world
+
+
+def run_e2e(mm, host, args, world):
+    """Same metric through the public API with host buffers: every step copies
+    its inputs from pinned host memory, runs the forward and reads y and the
+    carried state back."""
+    cfg = PREFILL
+    B, L, D = cfg.batch, cfg.seqlen, cfg.d_inner
+    keys_in = ["xz", "dt", "Bm", "Cm"]
+    pinned = {k: host[k].pin_memory() for k in keys_in}
+    params = {k: (host[k].cuda() if host[k] is not None else None)
+              for k in ("conv_w", "conv_b", "dt_bias", "A", "Dskip", "h0", "conv_state_in")}
+    dev = {k: torch.empty_like(pinned[k], device="cuda") for k in keys_in}
+    y_h = torch.empty((B, L, D), dtype=torch.bfloat16).pin_memory()
+    h_h = torch.empty((B, D, 16)).pin_memory()
+    cs_h = torch.empty((B, D, 3), dtype=torch.bfloat16).pin_memory()
+    outs = (torch.empty((B, L, D), dtype=torch.bfloat16, device="cuda"), torch.empty((B, D, 16), device="cuda"),
+            torch.empty((B, D, 3), dtype=torch.bfloat16, device="cuda"))
+    h2d = sum(pinned[k].numel() * pinned[k].element_size() for k in keys_in)
+    d2h = sum(t.numel() * t.element_size() for t in (y_h, h_h, cs_h))
+
+    def step():
+        for k in keys_in:
+            dev[k].copy_(pinned[k], non_blocking=True)
+        d = dict(params)
+        d.update(dev)
+        _fwd_call(mm, d, outs)
+        y_h.copy_(outs[0], non_blocking=True)
+        h_h.copy_(outs[1], non_blocking=True)
+        cs_h.copy_(outs[2], non_blocking=True)
+
+    K = max(3, min(args.steps, 200))
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    _barrier(world)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(K):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = _max_over_ranks(a.elapsed_time(b), world)
+    return {"value": round(world * B * L * K / (ms * 1e-3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
+            "ms_per_step": round(ms / K, 4)}
+
+
+def run_decode(mm, args, world, hbm_peak, hbm_src):
+    cfg = DECODE
+    NL, B, D = cfg.layers, cfg.batch, cfg.d_inner
+    host = make_decode_inputs(cfg)
+    d = {k: (v.cuda() if v is not None else None) for k, v in host.items()}
+    y = torch.empty((NL, B, D), dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        mm.state_update(d["x"], d["z"], d["dt"], d["conv_w"], d["conv_b"], d["dt_bias"], d["Dskip"], d["A"],
+                        d["Bm"], d["Cm"], d["ssm_state"], d["conv_state"], y=y)
+
+    for _ in range(max(3, args.warmup // 10)):
+        step()
+    torch.cuda.synchronize()
+    K = max(3, min(args.steps, 200))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    _barrier(world)
+    for i in range(K):
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    avg_ms = _max_over_ranks(statistics.mean(ms), world)
+    nbytes = decode_bytes(NL, B, D)
+    gbs = nbytes / (avg_ms * 1e-3) / 1e9
+    traffic = _ncu_traffic("state_update_kernel/decode_28x128")
+    return {
+        "workload": cfg.name, "layers": NL, "batch": B, "d_inner": D, "steps": K,
+        "ms_per_step": round(avg_ms, 5),
+        "value": round(world * NL * B / (avg_ms * 1e-3), 1), "unit": "layer-tokens/s",
+        "per_layer_tokens_per_s": round(world * B / (avg_ms * 1e-3), 1),
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(gbs / hbm_peak, 4), "traffic": traffic, "algorithmic_bytes": nbytes,
+                     "peak_source": hbm_src},
+        "l2": "state (1.88 GB) larger than L2",
+    }
+
+
+# ---------------------------------------------------------------- CPU oracle
+def cpu_baseline(host, cfg, target_s=12.0, sample_override=None):
+    """The fp64 oracle as it stands, on all host cores, on a channel sample of
+    the same workload; tokens/s scaled from the sample's channel count to
+    d_inner (channels are independent given the shared B/C)."""
+    import oracle
+    from workloads import sample_channels, subset_channels as subset
+
+    threads = os.cpu_count() or 1
+    D = cfg.d_inner
+
+    def timed(nch):
+        chans = sample_channels(D, nch)
+        sub = subset(host, chans)
+        t = time.perf_counter()
+        oracle.mixer_fwd(sub["xz"], sub["conv_w"], sub["conv_b"], sub["dt"], sub["dt_bias"], sub["A"], sub["Bm"],
+                         sub["Cm"], sub["Dskip"], sub["h0"], sub["conv_state_in"], threads=threads)
+        return time.perf_counter() - t, len(chans)
+
+    if sample_override:
+        el, n = timed(sample_override)
+    else:
+        probe = max(threads, 16)
+        el, n = timed(probe)
+        want = int(min(D, max(probe, probe * target_s / max(el, 1e-3))))
+        want = max(threads, want // threads * threads)
+        el, n = timed(want)
+    tokens = cfg.batch * cfg.seqlen
+    value = tokens * n / D / el
+    return {"value": round(value, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} of {D} channels x {tokens} tokens ({cfg.name}), {el:.2f} s; "
+                      f"tokens/s scaled by {n}/{D}"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None, world
+    cfg = PREFILL
+    host = make_mixer_inputs(cfg)
+    threads = os.cpu_count() or 1
+    # size each step's channel sample so the whole run stays near 2 minutes
+    probe = cpu_baseline(host, cfg, sample_override=threads)
+    per_chan_s = (cfg.batch * cfg.seqlen / probe["value"]) / cfg.d_inner     # wall s per channel, all cores
+    step_budget = 120.0 / max(1, args.steps + args.warmup)
+    nch = int(max(1, min(cfg.d_inner, step_budget / max(per_chan_s, 1e-9))))
+    for _ in range(args.warmup):
+        cpu_baseline(host, cfg, sample_override=nch)
+    vals = []
+    t_all = time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(host, cfg, sample_override=nch)["value"])
+    total = time.perf_counter() - t_all
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / max(1, args.steps) * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (same seeded workload as the GPU arm)",
+        "config": {"workload": cfg.name, "batch": cfg.batch, "seq_len": cfg.seqlen, "d_inner": cfg.d_inner,
+                   "d_state": 16, "d_conv": 4, "act": "bf16 inputs widened to f64", "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{nch} of {cfg.d_inner} channels x {cfg.batch * cfg.seqlen} tokens per step; "
+                                   "tokens/s scaled by the channel fraction"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line, world
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        line, world = run_reference(args)
+    else:
+        line, world = run_gpu(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    if world > 1 and args.impl != "reference":
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

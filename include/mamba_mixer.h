@@ -1,0 +1,153 @@
+/*
+ * mamba_mixer.h -- C ABI of the B200 (sm_100a) Mamba mixer core.
+ *
+ * Two operations, both on device memory the caller owns, both asynchronous on
+ * a CUDA stream the caller chooses:
+ *
+ *   mamba_mixer_fwd      selective-scan forward over a whole sequence (prefill)
+ *   mamba_state_update   the one-token state update used in decode
+ *
+ * What they compute.  The Jamba hybrid SSM-Transformer lesson (section "SSM in
+ * one page") gives the recurrence h_t = A h_{t-1} + B x_t, y_t = C h_t, notes
+ * that y_t needs only h_{t-1} and x_t (constant memory, O(1) per token), and
+ * that Mamba makes A, B and C data-dependent ("selective").  Its "Mamba-3"
+ * section describes Mamba's convolution as an outer convolution on x_t ahead of
+ * the recurrence; the reproduction blog's kernel-profile section names Delta as
+ * the parameter that sets the state's decay.  The mixer-core problem statement
+ * fixes the remaining form, which this library implements per channel d and
+ * state index n:
+ *
+ *   u_t      = SiLU(conv_b[d] + sum_{k<W} conv_w[d,k] * x_{t-W+1+k})
+ *   Delta_t  = softplus(dt_t + dt_bias[d])
+ *   h_t[n]   = exp(Delta_t * A[d,n]) * h_{t-1}[n] + Delta_t * B_t[n] * u_t
+ *   y_t      = (sum_n C_t[n] * h_t[n] + Dskip[d] * u_t) * SiLU(z_t)
+ *
+ * with x_{t<0} taken from the carried conv window, conv_w[d, W-1] applied to
+ * the current token, one (B_t, C_t) group shared by all channels of a
+ * sequence, and A passed directly (negative entries), not as log(-A).
+ *
+ * Conventions for every entry point:
+ *   - Pointers are device (or managed) addresses, 16-byte aligned, dense
+ *     row-major with the last dimension contiguous.  Host pointers are not
+ *     accepted; the caller copies host data in first.
+ *   - "act" tensors hold MM_F32 floats or MM_BF16 bfloat16 values; parameters
+ *     and the SSM state are always fp32.
+ *   - Supported sizes: d_state == 16, d_conv == 4, d_inner a multiple of 8.
+ *   - Validation happens on the host before anything is launched; a rejected
+ *     call launches nothing and writes nothing.  A launch failure reported by
+ *     the CUDA runtime returns MM_ERR_CUDA (the runtime's error is cleared).
+ *   - The library allocates no memory and keeps no state between calls.
+ *     Calls only enqueue work: results are valid once the stream reaches them.
+ *   - Kernels never assert or trap.
+ */
+#ifndef MAMBA_MIXER_H
+#define MAMBA_MIXER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mm_status {
+    MM_OK = 0,
+    MM_ERR_NULL = 1,        /* a required pointer is NULL                            */
+    MM_ERR_SHAPE = 2,       /* a size is negative, zero where it must not be, or too big */
+    MM_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                      */
+    MM_ERR_DTYPE = 4,       /* unknown activation dtype                              */
+    MM_ERR_ALIAS = 5,       /* an output overlaps an input or another output         */
+    MM_ERR_UNSUPPORTED = 6, /* d_state != 16, d_conv != 4, or d_inner % 8 != 0       */
+    MM_ERR_CUDA = 7,        /* the CUDA runtime reported an error at launch          */
+    MM_ERR_DEVICE = 8       /* no usable sm_100 device is current                    */
+} mm_status;
+
+typedef enum mm_dtype {
+    MM_F32 = 0,   /* IEEE binary32 */
+    MM_BF16 = 1   /* bfloat16      */
+} mm_dtype;
+
+/*
+ * Selective-scan forward (prefill) for `batch` sequences of `seqlen` tokens.
+ *
+ * Inputs (act = activation dtype):
+ *   xz             [batch, seqlen, 2*d_inner] act   x = xz[..., :d_inner], z = xz[..., d_inner:]
+ *   conv_w         [d_inner, d_conv]          fp32  conv_w[d, d_conv-1] multiplies the current token
+ *   conv_b         [d_inner]                  fp32  or NULL (= 0)
+ *   dt             [batch, seqlen, d_inner]   act   step input before the bias
+ *   dt_bias        [d_inner]                  fp32
+ *   A              [d_inner, d_state]         fp32  (negative for a decaying state)
+ *   Bm, Cm         [batch, seqlen, d_state]   act   shared by all channels of a sequence
+ *   Dskip          [d_inner]                  fp32  or NULL (= 0)
+ *   h0             [batch, d_inner, d_state]  fp32  initial state, or NULL (= 0)
+ *   conv_state_in  [batch, d_inner, d_conv-1] act   the d_conv-1 raw x preceding token 0,
+ *                                                   oldest first, or NULL (= 0)
+ * Outputs:
+ *   y              [batch, seqlen, d_inner]   act   rounded to nearest even for bf16
+ *   h_last         [batch, d_inner, d_state]  fp32  state after the last token (h0 if seqlen == 0)
+ *   conv_state_out [batch, d_inner, d_conv-1] act   the last d_conv-1 raw x, oldest first
+ *                                                   (shifted in from conv_state_in when
+ *                                                   seqlen < d_conv-1)
+ * Passing (h_last, conv_state_out) of one call as (h0, conv_state_in) of the
+ * next continues the sequence exactly; outputs may not overlap inputs, so
+ * carry through two buffer sets (MM_ERR_ALIAS otherwise).
+ *
+ * workspace / workspace_bytes: device scratch of at least
+ * mamba_mixer_workspace_size(...) bytes (may be NULL when that is 0).
+ * stream: a cudaStream_t (NULL = the legacy default stream).
+ * batch == 0 is a no-op.  seqlen == 0 writes h_last and conv_state_out only.
+ */
+mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv_b,
+                          const void* dt, const float* dt_bias, const float* A,
+                          const void* Bm, const void* Cm, const float* Dskip,
+                          const float* h0, const void* conv_state_in,
+                          void* y, float* h_last, void* conv_state_out,
+                          int64_t batch, int64_t seqlen, int64_t d_inner,
+                          int64_t d_state, int64_t d_conv, mm_dtype act,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device scratch mamba_mixer_fwd needs for these sizes (0 = none). */
+size_t mamba_mixer_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner,
+                                  int64_t d_state, int64_t d_conv, mm_dtype act);
+
+/*
+ * One-token state update (decode) for n_layers independent stacked Mamba
+ * layers at batch `batch`, updating the carried state in place.
+ *
+ *   x, z, dt       [n_layers, batch, d_inner]          act   the new token's inputs
+ *   conv_w         [n_layers, d_inner, d_conv]         fp32
+ *   conv_b         [n_layers, d_inner]                 fp32  or NULL (= 0)
+ *   dt_bias        [n_layers, d_inner]                 fp32
+ *   Dskip          [n_layers, d_inner]                 fp32  or NULL (= 0)
+ *   A              [n_layers, d_inner, d_state]        fp32
+ *   Bm, Cm         [n_layers, batch, d_state]          act
+ *   ssm_state      [n_layers, batch, d_inner, d_state] fp32  in: h_{t-1}; out: h_t
+ *   conv_state     [n_layers, batch, d_inner, d_conv-1] act  in: the d_conv-1 previous raw x,
+ *                                                            oldest first; out: shifted by one
+ *                                                            with x appended
+ *   y              [n_layers, batch, d_inner]          act
+ * This is the forward's step for one token (same arithmetic), so a prefill
+ * followed by decode steps equals one longer prefill.  In-place by contract;
+ * y may not overlap any other argument (MM_ERR_ALIAS).
+ */
+mm_status mamba_state_update(const void* x, const void* z, const void* dt,
+                             const float* conv_w, const float* conv_b,
+                             const float* dt_bias, const float* Dskip, const float* A,
+                             const void* Bm, const void* Cm,
+                             float* ssm_state, void* conv_state, void* y,
+                             int64_t n_layers, int64_t batch, int64_t d_inner,
+                             int64_t d_state, int64_t d_conv, mm_dtype act, void* stream);
+
+/* A static, human-readable name for a status code. */
+const char* mamba_status_string(mm_status status);
+
+/* ABI version of this header (incremented on any signature change). */
+int mamba_mixer_abi_version(void);
+
+#define MAMBA_MIXER_ABI_VERSION 1
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MAMBA_MIXER_H */

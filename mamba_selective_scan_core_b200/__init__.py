@@ -1,0 +1,210 @@
+"""Python binding of the B200 Mamba mixer core library (libmamba_mixer.so).
+
+Argument marshalling only: tensors are checked (device, dtype, shape,
+contiguity), output tensors are allocated with torch when not given, and the
+data pointers plus the current CUDA stream go through ctypes to the C ABI of
+``include/mamba_mixer.h``.  Every step of the computation runs in the
+library's kernels; there is no fallback path.  If the compiled library is
+missing, loading fails with an error that says how to build it.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "MM_F32", "MM_BF16", "MixerError", "lib", "library_path", "mixer_fwd", "state_update",
+    "workspace_size", "status_string", "abi_version", "EXPORTED_SYMBOLS",
+]
+
+MM_F32 = 0
+MM_BF16 = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libmamba_mixer.so"
+_lib = None
+
+EXPORTED_SYMBOLS = (
+    "mamba_mixer_fwd",
+    "mamba_mixer_workspace_size",
+    "mamba_state_update",
+    "mamba_status_string",
+    "mamba_mixer_abi_version",
+)
+
+
+class MixerError(RuntimeError):
+    """A non-zero mm_status returned by the library."""
+
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (mm_status {status})")
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, _LIB_NAME)
+
+
+def _declare(L):
+    P = ctypes.c_void_p
+    I64 = ctypes.c_int64
+    L.mamba_mixer_fwd.restype = ctypes.c_int
+    L.mamba_mixer_fwd.argtypes = [P] * 14 + [I64] * 5 + [ctypes.c_int, P, ctypes.c_size_t, P]
+    L.mamba_mixer_workspace_size.restype = ctypes.c_size_t
+    L.mamba_mixer_workspace_size.argtypes = [I64] * 5 + [ctypes.c_int]
+    L.mamba_state_update.restype = ctypes.c_int
+    L.mamba_state_update.argtypes = [P] * 13 + [I64] * 5 + [ctypes.c_int, P]
+    L.mamba_status_string.restype = ctypes.c_char_p
+    L.mamba_status_string.argtypes = [ctypes.c_int]
+    L.mamba_mixer_abi_version.restype = ctypes.c_int
+    L.mamba_mixer_abi_version.argtypes = []
+    return L
+
+
+def lib():
+    """The loaded C library (ctypes.CDLL).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise ImportError(
+                f"{path} is missing: build the CUDA library first "
+                "(python -m mamba_selective_scan_core_b200.build, or __graft_entry__.build())")
+        _lib = _declare(ctypes.CDLL(path))
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().mamba_status_string(int(status)).decode()
+
+
+def abi_version() -> int:
+    return int(lib().mamba_mixer_abi_version())
+
+
+def _act_code(dtype):
+    import torch
+
+    if dtype == torch.bfloat16:
+        return MM_BF16
+    if dtype == torch.float32:
+        return MM_F32
+    raise TypeError(f"activation dtype must be bfloat16 or float32, got {dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(t, name, dtype, shape, device):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream_handle(stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def workspace_size(batch, seqlen, d_inner, d_state=16, d_conv=4, act=MM_BF16) -> int:
+    return int(lib().mamba_mixer_workspace_size(batch, seqlen, d_inner, d_state, d_conv, act))
+
+
+def mixer_fwd(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, conv_state_in=None, *,
+              y=None, h_last=None, conv_state_out=None, workspace=None, stream=None):
+    """Selective-scan forward.  Shapes: xz [B,L,2D], dt [B,L,D], Bm/Cm [B,L,N]
+    (act dtype: bf16 or fp32); conv_w [D,W], conv_b/dt_bias/Dskip [D], A [D,N],
+    h0 [B,D,N] (fp32); conv_state_in [B,D,W-1] (act).  conv_b, Dskip, h0 and
+    conv_state_in may be None.  Returns (y [B,L,D], h_last [B,D,N],
+    conv_state_out [B,D,W-1]), allocating any output not given."""
+    import torch
+
+    act = _act_code(xz.dtype)
+    Bsz, L, twoD = xz.shape
+    D = twoD // 2
+    N = A.shape[-1]
+    W = conv_w.shape[-1]
+    dev = xz.device
+    f32 = torch.float32
+    _check(xz, "xz", xz.dtype, (Bsz, L, 2 * D), dev)
+    _check(conv_w, "conv_w", f32, (D, W), dev)
+    _check(conv_b, "conv_b", f32, (D,), dev)
+    _check(dt, "dt", xz.dtype, (Bsz, L, D), dev)
+    _check(dt_bias, "dt_bias", f32, (D,), dev)
+    _check(A, "A", f32, (D, N), dev)
+    _check(Bm, "Bm", xz.dtype, (Bsz, L, N), dev)
+    _check(Cm, "Cm", xz.dtype, (Bsz, L, N), dev)
+    _check(Dskip, "Dskip", f32, (D,), dev)
+    _check(h0, "h0", f32, (Bsz, D, N), dev)
+    _check(conv_state_in, "conv_state_in", xz.dtype, (Bsz, D, W - 1), dev)
+    if y is None:
+        y = torch.empty((Bsz, L, D), dtype=xz.dtype, device=dev)
+    if h_last is None:
+        h_last = torch.empty((Bsz, D, N), dtype=f32, device=dev)
+    if conv_state_out is None:
+        conv_state_out = torch.empty((Bsz, D, W - 1), dtype=xz.dtype, device=dev)
+    _check(y, "y", xz.dtype, (Bsz, L, D), dev)
+    _check(h_last, "h_last", f32, (Bsz, D, N), dev)
+    _check(conv_state_out, "conv_state_out", xz.dtype, (Bsz, D, W - 1), dev)
+    ws_bytes = workspace_size(Bsz, L, D, N, W, act)
+    if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        st = lib().mamba_mixer_fwd(
+            _ptr(xz), _ptr(conv_w), _ptr(conv_b), _ptr(dt), _ptr(dt_bias), _ptr(A), _ptr(Bm), _ptr(Cm),
+            _ptr(Dskip), _ptr(h0), _ptr(conv_state_in), _ptr(y), _ptr(h_last), _ptr(conv_state_out),
+            Bsz, L, D, N, W, act, _ptr(workspace) if ws_bytes else None, ws_bytes, _stream_handle(stream))
+    if st != 0:
+        raise MixerError(st, "mamba_mixer_fwd")
+    return y, h_last, conv_state_out
+
+
+def state_update(x, z, dt, conv_w, conv_b, dt_bias, Dskip, A, Bm, Cm, ssm_state, conv_state, *,
+                 y=None, stream=None):
+    """One-token decode step for NL stacked layers, in place on ssm_state
+    [NL,B,D,N] (fp32) and conv_state [NL,B,D,W-1] (act).  x/z/dt [NL,B,D] and
+    Bm/Cm [NL,B,N] in the act dtype; conv_w [NL,D,W], conv_b/dt_bias/Dskip
+    [NL,D], A [NL,D,N] in fp32 (conv_b, Dskip may be None).  Returns y [NL,B,D]."""
+    import torch
+
+    act = _act_code(x.dtype)
+    NL, Bsz, D = x.shape
+    N = A.shape[-1]
+    W = conv_w.shape[-1]
+    dev = x.device
+    f32 = torch.float32
+    for t, name in ((x, "x"), (z, "z"), (dt, "dt")):
+        _check(t, name, x.dtype, (NL, Bsz, D), dev)
+    _check(conv_w, "conv_w", f32, (NL, D, W), dev)
+    for t, name in ((conv_b, "conv_b"), (dt_bias, "dt_bias"), (Dskip, "Dskip")):
+        _check(t, name, f32, (NL, D), dev)
+    _check(A, "A", f32, (NL, D, N), dev)
+    _check(Bm, "Bm", x.dtype, (NL, Bsz, N), dev)
+    _check(Cm, "Cm", x.dtype, (NL, Bsz, N), dev)
+    _check(ssm_state, "ssm_state", f32, (NL, Bsz, D, N), dev)
+    _check(conv_state, "conv_state", x.dtype, (NL, Bsz, D, W - 1), dev)
+    if y is None:
+        y = torch.empty((NL, Bsz, D), dtype=x.dtype, device=dev)
+    _check(y, "y", x.dtype, (NL, Bsz, D), dev)
+    with torch.cuda.device(dev):
+        st = lib().mamba_state_update(
+            _ptr(x), _ptr(z), _ptr(dt), _ptr(conv_w), _ptr(conv_b), _ptr(dt_bias), _ptr(Dskip), _ptr(A),
+            _ptr(Bm), _ptr(Cm), _ptr(ssm_state), _ptr(conv_state), _ptr(y), NL, Bsz, D, N, W, act,
+            _stream_handle(stream))
+    if st != 0:
+        raise MixerError(st, "mamba_state_update")
+    return y

@@ -1,0 +1,259 @@
+// Host side of the C ABI declared in include/mamba_mixer.h: argument
+// validation (before anything is launched), launch-shape selection and the
+// launches themselves.  No allocation, no global state.
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+
+#include "mamba_mixer.h"
+#include "mixer_decode.cuh"
+#include "mixer_prefill.cuh"
+
+namespace {
+
+using mm::PrefillLayout;
+using mm::PrefillParams;
+
+constexpr int kTile = 32;
+constexpr int kMaxThreads = 256;
+constexpr int kSmemBudget = 200 * 1024;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Span {
+    uintptr_t lo = 0, hi = 0;   // [lo, hi); empty when lo == hi
+};
+Span span(const void* p, int64_t bytes) {
+    Span s;
+    if (p && bytes > 0) {
+        s.lo = reinterpret_cast<uintptr_t>(p);
+        s.hi = s.lo + static_cast<uintptr_t>(bytes);
+    }
+    return s;
+}
+bool overlaps(const Span& a, const Span& b) { return a.lo < a.hi && b.lo < b.hi && a.lo < b.hi && b.lo < a.hi; }
+
+// a * b with overflow detection on non-negative operands
+bool mul_ok(int64_t a, int64_t b, int64_t* out) {
+    if (a < 0 || b < 0) return false;
+    if (a != 0 && b > INT64_MAX / a) return false;
+    *out = a * b;
+    return true;
+}
+
+mm_status check_device(int* sm_count) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return MM_ERR_DEVICE; }
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MM_ERR_DEVICE;
+    }
+    if (major != 10) return MM_ERR_DEVICE;
+    return MM_OK;
+}
+
+// Lanes per channel: the fewest (cheapest per state element) that still give
+// about 6 warps per SM; overridable for tuning with MAMBA_MIXER_LPC=1|2|4.
+int choose_lpc(int64_t channels, int sm_count) {
+    if (const char* e = std::getenv("MAMBA_MIXER_LPC")) {
+        const int v = std::atoi(e);
+        if (v == 1 || v == 2 || v == 4) return v;
+    }
+    const int64_t want_warps = static_cast<int64_t>(sm_count) * 6;
+    if (channels / 32 >= want_warps) return 1;
+    if (channels * 2 / 32 >= want_warps) return 2;
+    return 4;
+}
+
+template <typename T, typename M, int LPC, int STAGES>
+cudaError_t launch_prefill(const PrefillParams& p, int64_t batch, int threads, cudaStream_t s) {
+    auto kern = mm::mixer_fwd_kernel<T, M, LPC, kTile, STAGES>;
+    const int smem = PrefillLayout<T>::smem_bytes(kTile, STAGES, p.octets);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = batch * p.ctas_per_seq;
+    kern<<<static_cast<unsigned>(grid), threads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename T, typename M, int LPC>
+cudaError_t launch_prefill_stages(const PrefillParams& p, int64_t batch, int threads, cudaStream_t s) {
+    // as deep a copy ring as fits the shared-memory budget (4, else 3, else 2)
+    if (PrefillLayout<T>::smem_bytes(kTile, 4, p.octets) <= kSmemBudget)
+        return launch_prefill<T, M, LPC, 4>(p, batch, threads, s);
+    if (PrefillLayout<T>::smem_bytes(kTile, 3, p.octets) <= kSmemBudget)
+        return launch_prefill<T, M, LPC, 3>(p, batch, threads, s);
+    return launch_prefill<T, M, LPC, 2>(p, batch, threads, s);
+}
+
+template <typename T, typename M>
+cudaError_t dispatch_prefill(PrefillParams p, int64_t batch, int sm_count, cudaStream_t s) {
+    const int64_t octets_per_seq = p.D / 8;
+    const int lpc = choose_lpc(batch * p.D, sm_count);
+    // octets per CTA: spread all channels over about one CTA per SM, capped by
+    // the CTA size and the shared-memory budget; then even out the CTAs of a
+    // sequence so that none is a small remainder.
+    int max_oct = kMaxThreads / (8 * lpc);
+    while (max_oct > 1 && PrefillLayout<T>::smem_bytes(kTile, 2, max_oct) > kSmemBudget) --max_oct;
+    int64_t oct = (batch * octets_per_seq + sm_count - 1) / sm_count;
+    if (oct < 1) oct = 1;
+    if (oct > max_oct) oct = max_oct;
+    if (oct > octets_per_seq) oct = octets_per_seq;
+    const int64_t ctas = (octets_per_seq + oct - 1) / oct;
+    oct = (octets_per_seq + ctas - 1) / ctas;
+    p.octets = static_cast<int>(oct);
+    p.ctas_per_seq = static_cast<int>(ctas);
+    const int threads = static_cast<int>(((oct * 8 * lpc) + 31) / 32 * 32);
+    switch (lpc) {
+        case 1: return launch_prefill_stages<T, M, 1>(p, batch, threads, s);
+        case 2: return launch_prefill_stages<T, M, 2>(p, batch, threads, s);
+        default: return launch_prefill_stages<T, M, 4>(p, batch, threads, s);
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+int mamba_mixer_abi_version(void) { return MAMBA_MIXER_ABI_VERSION; }
+
+const char* mamba_status_string(mm_status status) {
+    switch (status) {
+        case MM_OK: return "ok";
+        case MM_ERR_NULL: return "a required pointer is NULL";
+        case MM_ERR_SHAPE: return "invalid size (negative, zero where not allowed, or too large)";
+        case MM_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+        case MM_ERR_DTYPE: return "unknown activation dtype";
+        case MM_ERR_ALIAS: return "an output overlaps an input or another output";
+        case MM_ERR_UNSUPPORTED: return "unsupported size (need d_state == 16, d_conv == 4, d_inner % 8 == 0)";
+        case MM_ERR_CUDA: return "CUDA runtime error at launch";
+        case MM_ERR_DEVICE: return "no usable sm_100 device is current";
+    }
+    return "unknown status";
+}
+
+size_t mamba_mixer_workspace_size(int64_t, int64_t, int64_t, int64_t, int64_t, mm_dtype) {
+    // the forward keeps its whole state in registers and shared memory
+    return 0;
+}
+
+mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv_b,
+                          const void* dt, const float* dt_bias, const float* A,
+                          const void* Bm, const void* Cm, const float* Dskip,
+                          const float* h0, const void* conv_state_in,
+                          void* y, float* h_last, void* conv_state_out,
+                          int64_t batch, int64_t seqlen, int64_t d_inner,
+                          int64_t d_state, int64_t d_conv, mm_dtype act,
+                          void* workspace, size_t workspace_bytes, void* stream)
+{
+    (void)workspace;
+    (void)workspace_bytes;
+    if (act != MM_F32 && act != MM_BF16) return MM_ERR_DTYPE;
+    if (batch < 0 || seqlen < 0 || d_inner <= 0 || d_state <= 0 || d_conv <= 0) return MM_ERR_SHAPE;
+    if (d_state != 16 || d_conv != 4 || d_inner % 8 != 0) return MM_ERR_UNSUPPORTED;
+    if (d_inner > (1 << 24) || batch > (1 << 24)) return MM_ERR_SHAPE;
+    const int64_t es = act == MM_F32 ? 4 : 2;
+    int64_t tokens, xz_bytes, dt_bytes, bc_bytes, st_bytes;
+    if (!mul_ok(batch, seqlen, &tokens) || !mul_ok(tokens, 2 * d_inner * es, &xz_bytes) ||
+        !mul_ok(tokens, d_inner * es, &dt_bytes) || !mul_ok(tokens, d_state * es, &bc_bytes) ||
+        !mul_ok(batch, d_inner * d_state * 4, &st_bytes))
+        return MM_ERR_SHAPE;
+    const int64_t cs_bytes = batch * d_inner * (d_conv - 1) * es;
+    if (batch == 0) return MM_OK;
+
+    // required pointers
+    if (!conv_w || !dt_bias || !A || !h_last || !conv_state_out) return MM_ERR_NULL;
+    if (seqlen > 0 && (!xz || !dt || !Bm || !Cm || !y)) return MM_ERR_NULL;
+    const void* all[] = {xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0, conv_state_in,
+                         y, h_last, conv_state_out};
+    for (const void* q : all)
+        if (q && !aligned16(q)) return MM_ERR_ALIGN;
+
+    const Span in[] = {span(xz, xz_bytes), span(conv_w, d_inner * d_conv * 4), span(conv_b, d_inner * 4),
+                       span(dt, dt_bytes), span(dt_bias, d_inner * 4), span(A, d_inner * d_state * 4),
+                       span(Bm, bc_bytes), span(Cm, bc_bytes), span(Dskip, d_inner * 4),
+                       span(h0, st_bytes), span(conv_state_in, cs_bytes)};
+    const Span out[] = {span(y, dt_bytes), span(h_last, st_bytes), span(conv_state_out, cs_bytes)};
+    for (const Span& o : out)
+        for (const Span& i : in)
+            if (overlaps(o, i)) return MM_ERR_ALIAS;
+    if (overlaps(out[0], out[1]) || overlaps(out[0], out[2]) || overlaps(out[1], out[2])) return MM_ERR_ALIAS;
+
+    int sm_count = 0;
+    if (mm_status st = check_device(&sm_count); st != MM_OK) return st;
+
+    PrefillParams p{};
+    p.xz = xz; p.conv_w = conv_w; p.conv_b = conv_b; p.dt = dt; p.dt_bias = dt_bias; p.A = A;
+    p.Bm = Bm; p.Cm = Cm; p.Dskip = Dskip; p.h0 = h0; p.cs_in = conv_state_in;
+    p.y = y; p.h_last = h_last; p.cs_out = conv_state_out;
+    p.L = seqlen;
+    p.D = static_cast<int>(d_inner);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = act == MM_BF16 ? dispatch_prefill<__nv_bfloat16, mm::MathFast>(p, batch, sm_count, s)
+                                   : dispatch_prefill<float, mm::MathExact>(p, batch, sm_count, s);
+    if (e != cudaSuccess) { cudaGetLastError(); return MM_ERR_CUDA; }
+    return MM_OK;
+}
+
+mm_status mamba_state_update(const void* x, const void* z, const void* dt,
+                             const float* conv_w, const float* conv_b,
+                             const float* dt_bias, const float* Dskip, const float* A,
+                             const void* Bm, const void* Cm,
+                             float* ssm_state, void* conv_state, void* y,
+                             int64_t n_layers, int64_t batch, int64_t d_inner,
+                             int64_t d_state, int64_t d_conv, mm_dtype act, void* stream)
+{
+    if (act != MM_F32 && act != MM_BF16) return MM_ERR_DTYPE;
+    if (n_layers < 0 || batch < 0 || d_inner <= 0 || d_state <= 0 || d_conv <= 0) return MM_ERR_SHAPE;
+    if (d_state != 16 || d_conv != 4 || d_inner % 8 != 0) return MM_ERR_UNSUPPORTED;
+    if (d_inner > (1 << 24) || batch > (1 << 24) || n_layers > (1 << 24)) return MM_ERR_SHAPE;
+    const int64_t es = act == MM_F32 ? 4 : 2;
+    int64_t lb, rows, st_bytes;
+    if (!mul_ok(n_layers, batch, &lb) || !mul_ok(lb, d_inner, &rows) || !mul_ok(rows, d_state * 4, &st_bytes))
+        return MM_ERR_SHAPE;
+    if (rows == 0) return MM_OK;
+    if ((rows + 255) / 256 > INT32_MAX) return MM_ERR_SHAPE;
+
+    if (!x || !z || !dt || !conv_w || !dt_bias || !A || !Bm || !Cm || !ssm_state || !conv_state || !y)
+        return MM_ERR_NULL;
+    const void* all[] = {x, z, dt, conv_w, conv_b, dt_bias, Dskip, A, Bm, Cm, ssm_state, conv_state, y};
+    for (const void* q : all)
+        if (q && !aligned16(q)) return MM_ERR_ALIGN;
+
+    const int64_t tok_bytes = rows * es;
+    const int64_t par = n_layers * d_inner * 4;
+    const Span in[] = {span(x, tok_bytes), span(z, tok_bytes), span(dt, tok_bytes),
+                       span(conv_w, par * d_conv), span(conv_b, par), span(dt_bias, par), span(Dskip, par),
+                       span(A, par * d_state), span(Bm, lb * d_state * es), span(Cm, lb * d_state * es)};
+    const Span io[] = {span(ssm_state, st_bytes), span(conv_state, rows * (d_conv - 1) * es), span(y, tok_bytes)};
+    for (const Span& o : io)
+        for (const Span& i : in)
+            if (overlaps(o, i)) return MM_ERR_ALIAS;
+    if (overlaps(io[0], io[1]) || overlaps(io[0], io[2]) || overlaps(io[1], io[2])) return MM_ERR_ALIAS;
+
+    int sm_count = 0;
+    if (mm_status st = check_device(&sm_count); st != MM_OK) return st;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const unsigned grid = static_cast<unsigned>((rows + 255) / 256);
+    if (act == MM_BF16) {
+        using T = __nv_bfloat16;
+        mm::state_update_kernel<T, mm::MathFast><<<grid, 256, 0, s>>>(
+            static_cast<const T*>(x), static_cast<const T*>(z), static_cast<const T*>(dt), conv_w, conv_b,
+            dt_bias, Dskip, A, static_cast<const T*>(Bm), static_cast<const T*>(Cm), ssm_state,
+            static_cast<T*>(conv_state), static_cast<T*>(y), rows, static_cast<int>(batch),
+            static_cast<int>(d_inner));
+    } else {
+        mm::state_update_kernel<float, mm::MathExact><<<grid, 256, 0, s>>>(
+            static_cast<const float*>(x), static_cast<const float*>(z), static_cast<const float*>(dt), conv_w,
+            conv_b, dt_bias, Dskip, A, static_cast<const float*>(Bm), static_cast<const float*>(Cm), ssm_state,
+            static_cast<float*>(conv_state), static_cast<float*>(y), rows, static_cast<int>(batch),
+            static_cast<int>(d_inner));
+    }
+    if (cudaGetLastError() != cudaSuccess) return MM_ERR_CUDA;
+    return MM_OK;
+}
+
+}  // extern "C"

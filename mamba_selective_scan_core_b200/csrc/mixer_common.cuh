@@ -1,0 +1,108 @@
+// Device helpers shared by the prefill and decode kernels of the Mamba mixer
+// core: activation loads/stores, the two math flavours (exact and fast), and
+// small packed-fp32 helpers for sm_100a.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace mm {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr unsigned kFull = 0xffffffffu;
+
+// ---------------------------------------------------------------- act dtype
+template <typename T> struct Act;
+template <> struct Act<float> {
+    using storage = float;
+    static constexpr int kBytes = 4;
+    __device__ __forceinline__ static float load(const float* p) { return *p; }
+    __device__ __forceinline__ static float to_f32(float v) { return v; }
+    __device__ __forceinline__ static float from_f32(float v) { return v; }
+};
+template <> struct Act<__nv_bfloat16> {
+    using storage = __nv_bfloat16;
+    static constexpr int kBytes = 2;
+    __device__ __forceinline__ static float to_f32(__nv_bfloat16 v) {
+        return __uint_as_float(static_cast<uint32_t>(__bfloat16_as_ushort(v)) << 16);
+    }
+    __device__ __forceinline__ static float load(const __nv_bfloat16* p) { return to_f32(*p); }
+    __device__ __forceinline__ static __nv_bfloat16 from_f32(float v) { return __float2bfloat16_rn(v); }
+};
+
+// ---------------------------------------------------------------- fast math
+// Single MUFU instructions (inline PTX); used by the bf16 path, whose
+// tolerance is set by bf16 rounding of the inputs and outputs.
+__device__ __forceinline__ float ex2_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2_fast(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_fast(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Math policy.  kExact: CUDA's correctly-rounded-ish libm (expf/log1pf, IEEE
+// division) in natural units.  kFast: MUFU ex2/lg2/rcp in log2 units.
+//
+// Both compute, for the pre-bias step input v = dt + dt_bias:
+//   step(v)   : a scaled step size "l" such that Delta = l * step_scale
+//   decay(l,a): exp(Delta * a) for a state coefficient a (= A[d, n])
+// kExact: l = Delta, step_scale = 1, decay = expf(l * a).
+// kFast : l = Delta / ln 2 (log2 of 1 + 2^(v log2 e)), step_scale = ln 2,
+//         decay = 2^(l * a)   (= e^(Delta a), since Delta log2(e) = l).
+struct MathExact {
+    static constexpr float step_scale = 1.0f;
+    __device__ __forceinline__ static float silu(float v) { return v / (1.0f + expf(-v)); }
+    __device__ __forceinline__ static float step(float dt, float bias) {
+        const float v = dt + bias;
+        return fmaxf(v, 0.0f) + log1pf(expf(-fabsf(v)));
+    }
+    __device__ __forceinline__ static float decay(float l, float a) { return expf(l * a); }
+};
+
+struct MathFast {
+    static constexpr float step_scale = kLn2;
+    __device__ __forceinline__ static float silu(float v) {
+        return v * rcp_fast(1.0f + ex2_fast(-kLog2e * v));
+    }
+    // bias2 = dt_bias * log2(e), precomputed per channel.
+    __device__ __forceinline__ static float step2(float dt, float bias2) {
+        const float v2 = fmaf(dt, kLog2e, bias2);
+        // log2(1 + 2^v2), exact enough for v2 <= 126; beyond that 2^v2 would
+        // overflow and the answer is v2 itself.
+        const float l = lg2_fast(1.0f + ex2_fast(fminf(v2, 126.0f)));
+        return fmaxf(l, v2);
+    }
+    __device__ __forceinline__ static float decay(float l, float a) { return ex2_fast(l * a); }
+};
+
+// ---------------------------------------------------------------- packed fp32
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+
+// ---------------------------------------------------------------- async copy
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+// 16-byte global -> shared copy; src_bytes == 0 zero-fills the destination
+// without reading (src must still be a valid address form).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n"
+                 :: "r"(smem_addr(dst)), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" :: "n"(N) : "memory"); }
+
+}  // namespace mm

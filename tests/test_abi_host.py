@@ -1,0 +1,212 @@
+"""The C-ABI library on the host, without a GPU: it loads, exports every
+function the public header declares, and rejects bad arguments with the
+documented status before touching the device.  Pointers here are fake
+addresses; validation never dereferences them."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import mamba_selective_scan_core_b200 as mm
+from mamba_selective_scan_core_b200 import build as mmbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mamba_mixer.h")
+
+OK, ENULL, ESHAPE, EALIGN, EDTYPE, EALIAS, EUNSUP, ECUDA, EDEVICE = range(9)
+
+
+@pytest.fixture(scope="module")
+def L():
+    mmbuild.build()
+    return mm.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mamba_\w+)\s*\(", src)))
+
+
+def test_header_declares_expected_api():
+    assert set(declared_functions()) == set(mm.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), f"{name} missing from {mm.library_path()}"
+
+
+def test_exported_symbols_are_c_linkage():
+    out = os.popen(f"nm -D --defined-only {mm.library_path()}").read()
+    names = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_functions():
+        assert name in names
+
+
+def test_version_and_strings(L):
+    assert mm.abi_version() == 1
+    for code in range(9):
+        s = mm.status_string(code)
+        assert s and s != "unknown status"
+    assert mm.status_string(99) == "unknown status"
+    assert mm.workspace_size(1, 4096, 8192) == 0
+
+
+# ---------------------------------------------------------------- mixer_fwd validation
+BASE = 0x7F0000000000   # a fake, 16-byte-aligned device address region
+
+
+def fwd_args(B=1, Lq=64, D=64, N=16, W=4, act=1, **over):
+    es = 4 if act == 0 else 2
+    sizes = dict(xz=B * Lq * 2 * D * es, conv_w=D * W * 4, conv_b=D * 4, dt=B * Lq * D * es, dt_bias=D * 4,
+                 A=D * N * 4, Bm=B * Lq * N * es, Cm=B * Lq * N * es, Dskip=D * 4, h0=B * D * N * 4,
+                 cs_in=B * D * (W - 1) * es, y=B * Lq * D * es, h_last=B * D * N * 4,
+                 cs_out=B * D * (W - 1) * es)
+    ptrs = {}
+    addr = BASE
+    for k, v in sizes.items():
+        ptrs[k] = addr
+        addr += (v + 4095) // 4096 * 4096 + 4096
+    ptrs.update(over)
+    order = ["xz", "conv_w", "conv_b", "dt", "dt_bias", "A", "Bm", "Cm", "Dskip", "h0", "cs_in",
+             "y", "h_last", "cs_out"]
+    return [ptrs[k] for k in order] + [B, Lq, D, N, W, act, None, 0, None]
+
+
+def call_fwd(L, **kw):
+    return L.mamba_mixer_fwd(*fwd_args(**kw))
+
+
+def test_fwd_valid_arguments_reach_the_device_check(L):
+    # everything valid: validation passes and the call stops at the device check
+    st = call_fwd(L)
+    assert st in (EDEVICE, OK, ECUDA)
+
+
+def test_fwd_batch_zero_is_a_noop(L):
+    assert call_fwd(L, B=0) == OK
+
+
+@pytest.mark.parametrize("act", [2, -1])
+def test_fwd_bad_dtype(L, act):
+    assert call_fwd(L, act=act) == EDTYPE
+
+
+@pytest.mark.parametrize("kw", [dict(B=-1), dict(Lq=-1), dict(D=0), dict(D=-8), dict(N=0), dict(W=0)])
+def test_fwd_bad_shape(L, kw):
+    assert call_fwd(L, **kw) == ESHAPE
+
+
+@pytest.mark.parametrize("kw", [dict(N=8), dict(N=32), dict(W=3), dict(W=2), dict(D=12), dict(D=65)])
+def test_fwd_unsupported(L, kw):
+    assert call_fwd(L, **kw) == EUNSUP
+
+
+def test_fwd_overflowing_sizes(L):
+    assert call_fwd(L, B=1 << 20, Lq=1 << 40) == ESHAPE
+
+
+@pytest.mark.parametrize("name", ["xz", "conv_w", "dt", "dt_bias", "A", "Bm", "Cm", "y", "h_last", "cs_out"])
+def test_fwd_required_null(L, name):
+    assert call_fwd(L, **{name: None}) == ENULL
+
+
+@pytest.mark.parametrize("name", ["conv_b", "Dskip", "h0", "cs_in"])
+def test_fwd_optional_null_passes_validation(L, name):
+    assert call_fwd(L, **{name: None}) in (EDEVICE, OK, ECUDA)
+
+
+def test_fwd_seqlen_zero_needs_no_token_buffers(L):
+    assert call_fwd(L, Lq=0, xz=None, dt=None, Bm=None, Cm=None, y=None) in (EDEVICE, OK, ECUDA)
+
+
+@pytest.mark.parametrize("name", ["xz", "conv_w", "conv_b", "dt", "A", "Bm", "h0", "cs_in", "y", "h_last", "cs_out"])
+def test_fwd_misaligned(L, name):
+    args = fwd_args()
+    base = dict(zip(["xz", "conv_w", "conv_b", "dt", "dt_bias", "A", "Bm", "Cm", "Dskip", "h0", "cs_in",
+                     "y", "h_last", "cs_out"], args[:14]))
+    assert call_fwd(L, **{name: base[name] + 8}) == EALIGN
+
+
+@pytest.mark.parametrize("out,inp", [("y", "xz"), ("y", "dt"), ("h_last", "h0"), ("cs_out", "cs_in"),
+                                     ("y", "Bm"), ("h_last", "A"), ("y", "h_last"), ("cs_out", "y")])
+def test_fwd_alias(L, out, inp):
+    args = fwd_args()
+    names = ["xz", "conv_w", "conv_b", "dt", "dt_bias", "A", "Bm", "Cm", "Dskip", "h0", "cs_in",
+             "y", "h_last", "cs_out"]
+    base = dict(zip(names, args[:14]))
+    assert call_fwd(L, **{out: base[inp]}) == EALIAS
+
+
+def test_fwd_partial_overlap_is_alias(L):
+    args = fwd_args()
+    names = ["xz", "conv_w", "conv_b", "dt", "dt_bias", "A", "Bm", "Cm", "Dskip", "h0", "cs_in",
+             "y", "h_last", "cs_out"]
+    base = dict(zip(names, args[:14]))
+    # y starting 16 bytes before the end of dt
+    dt_bytes = 1 * 64 * 64 * 2
+    assert call_fwd(L, y=base["dt"] + dt_bytes - 16) == EALIAS
+
+
+# ---------------------------------------------------------------- state_update validation
+def upd_args(NL=2, B=3, D=64, N=16, W=4, act=1, **over):
+    es = 4 if act == 0 else 2
+    rows = NL * B * D
+    sizes = dict(x=rows * es, z=rows * es, dt=rows * es, conv_w=NL * D * W * 4, conv_b=NL * D * 4,
+                 dt_bias=NL * D * 4, Dskip=NL * D * 4, A=NL * D * N * 4, Bm=NL * B * N * es,
+                 Cm=NL * B * N * es, ssm=rows * N * 4, cs=rows * (W - 1) * es, y=rows * es)
+    ptrs = {}
+    addr = BASE
+    for k, v in sizes.items():
+        ptrs[k] = addr
+        addr += (v + 4095) // 4096 * 4096 + 4096
+    ptrs.update(over)
+    order = ["x", "z", "dt", "conv_w", "conv_b", "dt_bias", "Dskip", "A", "Bm", "Cm", "ssm", "cs", "y"]
+    return [ptrs[k] for k in order] + [NL, B, D, N, W, act, None]
+
+
+def call_upd(L, **kw):
+    return L.mamba_state_update(*upd_args(**kw))
+
+
+def test_update_valid_reaches_device_check(L):
+    assert call_upd(L) in (EDEVICE, OK, ECUDA)
+
+
+def test_update_empty_is_noop(L):
+    assert call_upd(L, NL=0) == OK
+    assert call_upd(L, B=0) == OK
+
+
+@pytest.mark.parametrize("name", ["x", "z", "dt", "conv_w", "dt_bias", "A", "Bm", "Cm", "ssm", "cs", "y"])
+def test_update_required_null(L, name):
+    assert call_upd(L, **{name: None}) == ENULL
+
+
+@pytest.mark.parametrize("kw,code", [(dict(act=3), EDTYPE), (dict(N=4), EUNSUP), (dict(W=5), EUNSUP),
+                                     (dict(D=20), EUNSUP), (dict(NL=-1), ESHAPE)])
+def test_update_bad_sizes(L, kw, code):
+    assert call_upd(L, **kw) == code
+
+
+def test_update_alias(L):
+    args = upd_args()
+    assert call_upd(L, y=args[0]) == EALIAS          # y over x
+    assert call_upd(L, cs=args[10]) == EALIAS        # conv_state over ssm_state
+    assert call_upd(L, ssm=args[7]) == EALIAS        # state over A
+
+
+def test_update_misaligned(L):
+    args = upd_args()
+    assert call_upd(L, ssm=args[10] + 4) == EALIGN
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    # the binding never falls back: a missing library is an ImportError
+    monkeypatch.setattr(mm, "_lib", None)
+    monkeypatch.setattr(mm, "library_path", lambda: str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        mm.lib()

@@ -14,4 +14,5 @@ from .synth import (  # noqa: F401
     make_mixer_inputs_custom,
     make_decode_inputs_custom,
     sample_channels,
+    subset_channels,
 )

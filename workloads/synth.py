@@ -262,8 +262,27 @@ def sample_channels(d_inner: int, count: int = 256) -> np.ndarray:
     last 8 channels plus an even stride through the rest."""
     if d_inner <= count:
         return np.arange(d_inner)
+    if count <= 32:
+        return np.unique(np.linspace(0, d_inner - 1, count).round().astype(np.int64))
     edge = list(range(8)) + list(range(d_inner - 8, d_inner))
     stride = max(1, d_inner // (count - 16))
     mid = [d for d in range(3, d_inner, stride) if 8 <= d < d_inner - 8][: count - 16]
     sel = sorted(set(edge + mid))
     return np.array(sel, dtype=np.int64)
+
+
+def subset_channels(inp: dict, chans) -> dict:
+    """Mixer-forward inputs restricted to the channels ``chans`` (a copy).
+    Channels are independent given the shared B/C, so a computation on the
+    subset equals the full computation restricted to those channels."""
+    S = torch.as_tensor(np.asarray(chans), dtype=torch.long)
+    D = inp["dt"].shape[-1]
+    xz = inp["xz"]
+    out = dict(inp)
+    out["xz"] = torch.cat([xz[..., :D].index_select(-1, S), xz[..., D:].index_select(-1, S)], dim=-1)
+    out["dt"] = inp["dt"].index_select(-1, S)
+    for k in ("conv_w", "conv_b", "dt_bias", "A", "Dskip"):
+        out[k] = inp[k].index_select(0, S) if inp.get(k) is not None else None
+    for k in ("h0", "conv_state_in"):
+        out[k] = inp[k].index_select(1, S) if inp.get(k) is not None else None
+    return out
