@@ -59,7 +59,8 @@ typedef enum mm_status {
     MM_ERR_ALIAS = 5,       /* an output overlaps an input or another output         */
     MM_ERR_UNSUPPORTED = 6, /* d_state != 16, d_conv != 4, or d_inner % 8 != 0       */
     MM_ERR_CUDA = 7,        /* the CUDA runtime reported an error at launch          */
-    MM_ERR_DEVICE = 8       /* no usable sm_100 device is current                    */
+    MM_ERR_DEVICE = 8,      /* no usable sm_100 device is current                    */
+    MM_ERR_WORKSPACE = 9    /* workspace missing or smaller than the size this call needs */
 } mm_status;
 
 typedef enum mm_dtype {
@@ -93,7 +94,14 @@ typedef enum mm_dtype {
  * carry through two buffer sets (MM_ERR_ALIAS otherwise).
  *
  * workspace / workspace_bytes: device scratch of at least
- * mamba_mixer_workspace_size(...) bytes (may be NULL when that is 0).
+ * mamba_mixer_workspace_size(...) bytes for the same sizes (may be NULL when
+ * that is 0; MM_ERR_WORKSPACE when missing or smaller).  When a sequence has
+ * too few channels to fill the GPU, the forward splits it into time chunks:
+ * a first launch stores each chunk's end state (run from a zero state) and
+ * total step size there, and a second launch starts every chunk from the
+ * exact carried state.  The caller owns the workspace; its contents are not
+ * needed after the call and calls that share one must not overlap in time.
+ * It may not overlap any input or output (MM_ERR_ALIAS).
  * stream: a cudaStream_t (NULL = the legacy default stream).
  * batch == 0 is a no-op.  seqlen == 0 writes h_last and conv_state_out only.
  */
@@ -106,7 +114,10 @@ mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv
                           int64_t d_state, int64_t d_conv, mm_dtype act,
                           void* workspace, size_t workspace_bytes, void* stream);
 
-/* Bytes of device scratch mamba_mixer_fwd needs for these sizes (0 = none). */
+/* Bytes of device scratch mamba_mixer_fwd needs for these sizes (0 = none).
+ * A pure function of its arguments (and of the MAMBA_MIXER_LPC /
+ * MAMBA_MIXER_CHUNKS tuning variables, which must not change between this
+ * call and the forward that uses the result). */
 size_t mamba_mixer_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner,
                                   int64_t d_state, int64_t d_conv, mm_dtype act);
 

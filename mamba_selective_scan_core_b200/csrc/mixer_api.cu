@@ -1,6 +1,7 @@
 // Host side of the C ABI declared in include/mamba_mixer.h: argument
 // validation (before anything is launched), launch-shape selection and the
 // launches themselves.  No allocation, no global state.
+#include <algorithm>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -54,62 +55,119 @@ mm_status check_device(int* sm_count) {
     return MM_OK;
 }
 
-// Lanes per channel: the fewest (cheapest per state element) that still give
-// about 6 warps per SM; overridable for tuning with MAMBA_MIXER_LPC=1|2|4.
-int choose_lpc(int64_t channels, int sm_count) {
-    if (const char* e = std::getenv("MAMBA_MIXER_LPC")) {
+// Launch plan of a forward call: lanes per channel, time chunks and the
+// workspace they need.  A pure function of the sizes (and the two tuning
+// variables), so that mamba_mixer_workspace_size() and the call agree.
+struct FwdPlan {
+    int lpc = 1;
+    int chunks = 1;
+    int64_t chunk_len = 0;
+    size_t ws_bytes = 0;
+};
+
+constexpr int kPlanSMs = 148;            // B200: 2 dies x 74 SMs
+#ifndef MM_WARPS_PER_SM
+#define MM_WARPS_PER_SM 6
+#endif
+#ifndef MM_CTAS_PER_SM
+#define MM_CTAS_PER_SM 1
+#endif
+constexpr int kWarpsPerSM = MM_WARPS_PER_SM;   // resident warps wanted per SM
+constexpr int kCtasPerSM = MM_CTAS_PER_SM;     // resident CTAs the grid is shaped for
+constexpr int kMinChunkTiles = 4;        // shortest chunk worth a summary pass
+constexpr int kMaxChunks = 16;
+
+int env_int(const char* name, int lo, int hi) {
+    if (const char* e = std::getenv(name)) {
         const int v = std::atoi(e);
-        if (v == 1 || v == 2 || v == 4) return v;
+        if (v >= lo && v <= hi) return v;
     }
-    const int64_t want_warps = static_cast<int64_t>(sm_count) * 6;
-    if (channels / 32 >= want_warps) return 1;
-    if (channels * 2 / 32 >= want_warps) return 2;
-    return 4;
+    return 0;
 }
 
-template <typename T, typename M, int LPC, int STAGES>
-cudaError_t launch_prefill(const PrefillParams& p, int64_t batch, int threads, cudaStream_t s) {
-    auto kern = mm::mixer_fwd_kernel<T, M, LPC, kTile, STAGES>;
+FwdPlan plan_fwd(int64_t batch, int64_t seqlen, int64_t d_inner) {
+    FwdPlan pl;
+    const int lpc = env_int("MAMBA_MIXER_LPC", 1, 4);
+    pl.lpc = (lpc == 1 || lpc == 2 || lpc == 4) ? lpc : 1;
+    const int64_t channels = batch * d_inner;
+    const int64_t warps = channels * pl.lpc / 32;
+    const int64_t want = static_cast<int64_t>(kPlanSMs) * kWarpsPerSM;
+    const int64_t tiles = (seqlen + kTile - 1) / kTile;
+    int64_t k = 1;
+    if (const int forced = env_int("MAMBA_MIXER_CHUNKS", 1, 1 << 20)) {
+        k = forced;
+    } else if (warps < want) {
+        k = (want + std::max<int64_t>(warps, 1) - 1) / std::max<int64_t>(warps, 1);
+        k = std::min<int64_t>(k, std::max<int64_t>(1, tiles / kMinChunkTiles));
+        k = std::min<int64_t>(k, kMaxChunks);
+    }
+    k = std::max<int64_t>(1, std::min<int64_t>(k, std::max<int64_t>(tiles, 1)));
+    const int64_t tiles_per_chunk = (tiles + k - 1) / k;
+    pl.chunk_len = std::max<int64_t>(1, tiles_per_chunk) * kTile;
+    pl.chunks = static_cast<int>(seqlen > 0 ? (seqlen + pl.chunk_len - 1) / pl.chunk_len : 1);
+    if (pl.chunks > 1)
+        pl.ws_bytes = static_cast<size_t>(pl.chunks - 1) * batch * d_inner * (16 + 1) * sizeof(float);
+    return pl;
+}
+
+template <typename T, typename M, int LPC, int STAGES, bool SUMMARY>
+cudaError_t launch_prefill(const PrefillParams& p, int64_t batch, int chunks, int threads, cudaStream_t s) {
+    auto kern = mm::mixer_fwd_kernel<T, M, LPC, kTile, STAGES, SUMMARY>;
     const int smem = PrefillLayout<T>::smem_bytes(kTile, STAGES, p.octets);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const int64_t grid = batch * p.ctas_per_seq;
-    kern<<<static_cast<unsigned>(grid), threads, smem, s>>>(p);
+    const dim3 grid(static_cast<unsigned>(batch * p.ctas_per_seq), static_cast<unsigned>(chunks));
+    kern<<<grid, threads, smem, s>>>(p);
     return cudaGetLastError();
 }
 
-template <typename T, typename M, int LPC>
-cudaError_t launch_prefill_stages(const PrefillParams& p, int64_t batch, int threads, cudaStream_t s) {
-    // as deep a copy ring as fits the shared-memory budget (4, else 3, else 2)
-    if (PrefillLayout<T>::smem_bytes(kTile, 4, p.octets) <= kSmemBudget)
-        return launch_prefill<T, M, LPC, 4>(p, batch, threads, s);
-    if (PrefillLayout<T>::smem_bytes(kTile, 3, p.octets) <= kSmemBudget)
-        return launch_prefill<T, M, LPC, 3>(p, batch, threads, s);
-    return launch_prefill<T, M, LPC, 2>(p, batch, threads, s);
-}
-
-template <typename T, typename M>
-cudaError_t dispatch_prefill(PrefillParams p, int64_t batch, int sm_count, cudaStream_t s) {
+// Octets per CTA: spread the (channel octet, chunk) units over about one CTA
+// per SM, capped by the CTA size and the shared-memory budget; then even out
+// the CTAs of a sequence so that none is a small remainder.
+template <typename T>
+void shape_ctas(PrefillParams& p, int64_t batch, int64_t units_per_octet, int lpc, int sm_count, int* threads) {
     const int64_t octets_per_seq = p.D / 8;
-    const int lpc = choose_lpc(batch * p.D, sm_count);
-    // octets per CTA: spread all channels over about one CTA per SM, capped by
-    // the CTA size and the shared-memory budget; then even out the CTAs of a
-    // sequence so that none is a small remainder.
     int max_oct = kMaxThreads / (8 * lpc);
     while (max_oct > 1 && PrefillLayout<T>::smem_bytes(kTile, 2, max_oct) > kSmemBudget) --max_oct;
-    int64_t oct = (batch * octets_per_seq + sm_count - 1) / sm_count;
-    if (oct < 1) oct = 1;
-    if (oct > max_oct) oct = max_oct;
-    if (oct > octets_per_seq) oct = octets_per_seq;
+    const int64_t slots = static_cast<int64_t>(sm_count) * kCtasPerSM;
+    int64_t oct = (batch * octets_per_seq * units_per_octet + slots - 1) / slots;
+    oct = std::max<int64_t>(1, std::min<int64_t>({oct, max_oct, octets_per_seq}));
     const int64_t ctas = (octets_per_seq + oct - 1) / oct;
     oct = (octets_per_seq + ctas - 1) / ctas;
     p.octets = static_cast<int>(oct);
     p.ctas_per_seq = static_cast<int>(ctas);
-    const int threads = static_cast<int>(((oct * 8 * lpc) + 31) / 32 * 32);
-    switch (lpc) {
-        case 1: return launch_prefill_stages<T, M, 1>(p, batch, threads, s);
-        case 2: return launch_prefill_stages<T, M, 2>(p, batch, threads, s);
-        default: return launch_prefill_stages<T, M, 4>(p, batch, threads, s);
+    *threads = static_cast<int>(((oct * 8 * lpc) + 31) / 32 * 32);
+}
+
+template <typename T, typename M, int LPC, bool SUMMARY>
+cudaError_t launch_pass(PrefillParams p, int64_t batch, int chunks, int sm_count, cudaStream_t s) {
+    int threads = 0;
+    shape_ctas<T>(p, batch, chunks, LPC, sm_count, &threads);
+    // as deep a copy ring as fits the shared-memory budget (4, else 3, else 2)
+    if (PrefillLayout<T>::smem_bytes(kTile, 4, p.octets) <= kSmemBudget)
+        return launch_prefill<T, M, LPC, 4, SUMMARY>(p, batch, chunks, threads, s);
+    if (PrefillLayout<T>::smem_bytes(kTile, 3, p.octets) <= kSmemBudget)
+        return launch_prefill<T, M, LPC, 3, SUMMARY>(p, batch, chunks, threads, s);
+    return launch_prefill<T, M, LPC, 2, SUMMARY>(p, batch, chunks, threads, s);
+}
+
+template <typename T, typename M, int LPC>
+cudaError_t run_fwd(const PrefillParams& p, int64_t batch, int chunks, int sm_count, cudaStream_t s) {
+    if (chunks > 1) {
+        cudaError_t e = launch_pass<T, M, LPC, true>(p, batch, chunks - 1, sm_count, s);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_pass<T, M, LPC, false>(p, batch, chunks, sm_count, s);
+}
+
+template <typename T, typename M>
+cudaError_t dispatch_prefill(PrefillParams p, int64_t batch, const FwdPlan& pl, int sm_count, cudaStream_t s) {
+    p.chunk_len = pl.chunk_len;
+    p.n_chunks = pl.chunks;
+    switch (pl.lpc) {
+        case 1: return run_fwd<T, M, 1>(p, batch, pl.chunks, sm_count, s);
+        case 2: return run_fwd<T, M, 2>(p, batch, pl.chunks, sm_count, s);
+        default: return run_fwd<T, M, 4>(p, batch, pl.chunks, sm_count, s);
     }
 }
 
@@ -130,13 +188,17 @@ const char* mamba_status_string(mm_status status) {
         case MM_ERR_UNSUPPORTED: return "unsupported size (need d_state == 16, d_conv == 4, d_inner % 8 == 0)";
         case MM_ERR_CUDA: return "CUDA runtime error at launch";
         case MM_ERR_DEVICE: return "no usable sm_100 device is current";
+        case MM_ERR_WORKSPACE: return "workspace missing or smaller than mamba_mixer_workspace_size()";
     }
     return "unknown status";
 }
 
-size_t mamba_mixer_workspace_size(int64_t, int64_t, int64_t, int64_t, int64_t, mm_dtype) {
-    // the forward keeps its whole state in registers and shared memory
-    return 0;
+size_t mamba_mixer_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state,
+                                  int64_t d_conv, mm_dtype act) {
+    if ((act != MM_F32 && act != MM_BF16) || batch <= 0 || seqlen <= 0 || d_inner <= 0 || d_state != 16 ||
+        d_conv != 4 || d_inner % 8 != 0 || d_inner > (1 << 24) || batch > (1 << 24))
+        return 0;
+    return plan_fwd(batch, seqlen, d_inner).ws_bytes;
 }
 
 mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv_b,
@@ -148,8 +210,6 @@ mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv
                           int64_t d_state, int64_t d_conv, mm_dtype act,
                           void* workspace, size_t workspace_bytes, void* stream)
 {
-    (void)workspace;
-    (void)workspace_bytes;
     if (act != MM_F32 && act != MM_BF16) return MM_ERR_DTYPE;
     if (batch < 0 || seqlen < 0 || d_inner <= 0 || d_state <= 0 || d_conv <= 0) return MM_ERR_SHAPE;
     if (d_state != 16 || d_conv != 4 || d_inner % 8 != 0) return MM_ERR_UNSUPPORTED;
@@ -181,6 +241,17 @@ mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv
             if (overlaps(o, i)) return MM_ERR_ALIAS;
     if (overlaps(out[0], out[1]) || overlaps(out[0], out[2]) || overlaps(out[1], out[2])) return MM_ERR_ALIAS;
 
+    const FwdPlan pl = plan_fwd(batch, seqlen, d_inner);
+    if (pl.ws_bytes > 0) {
+        if (!workspace || workspace_bytes < pl.ws_bytes) return MM_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return MM_ERR_ALIGN;
+        const Span ws = span(workspace, static_cast<int64_t>(pl.ws_bytes));
+        for (const Span& i : in)
+            if (overlaps(ws, i)) return MM_ERR_ALIAS;
+        for (const Span& o : out)
+            if (overlaps(ws, o)) return MM_ERR_ALIAS;
+    }
+
     int sm_count = 0;
     if (mm_status st = check_device(&sm_count); st != MM_OK) return st;
 
@@ -190,9 +261,12 @@ mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv
     p.y = y; p.h_last = h_last; p.cs_out = conv_state_out;
     p.L = seqlen;
     p.D = static_cast<int>(d_inner);
+    p.batch = static_cast<int>(batch);
+    p.ws_state = static_cast<float*>(workspace);
+    p.ws_lsum = pl.ws_bytes ? p.ws_state + static_cast<int64_t>(pl.chunks - 1) * batch * d_inner * 16 : nullptr;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = act == MM_BF16 ? dispatch_prefill<__nv_bfloat16, mm::MathFast>(p, batch, sm_count, s)
-                                   : dispatch_prefill<float, mm::MathExact>(p, batch, sm_count, s);
+    cudaError_t e = act == MM_BF16 ? dispatch_prefill<__nv_bfloat16, mm::MathFast>(p, batch, pl, sm_count, s)
+                                   : dispatch_prefill<float, mm::MathExact>(p, batch, pl, sm_count, s);
     if (e != cudaSuccess) { cudaGetLastError(); return MM_ERR_CUDA; }
     return MM_OK;
 }

@@ -15,7 +15,7 @@ from mamba_selective_scan_core_b200 import build as mmbuild
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "mamba_mixer.h")
 
-OK, ENULL, ESHAPE, EALIGN, EDTYPE, EALIAS, EUNSUP, ECUDA, EDEVICE = range(9)
+OK, ENULL, ESHAPE, EALIGN, EDTYPE, EALIAS, EUNSUP, ECUDA, EDEVICE, EWORKSPACE = range(10)
 
 
 @pytest.fixture(scope="module")
@@ -48,11 +48,15 @@ def test_exported_symbols_are_c_linkage():
 
 def test_version_and_strings(L):
     assert mm.abi_version() == 1
-    for code in range(9):
+    for code in range(10):
         s = mm.status_string(code)
         assert s and s != "unknown status"
     assert mm.status_string(99) == "unknown status"
-    assert mm.workspace_size(1, 4096, 8192) == 0
+    # one 8192-channel sequence is split into 4 time chunks: 3 carried states
+    assert mm.workspace_size(1, 4096, 8192) == 3 * 8192 * 17 * 4
+    # four sequences fill the GPU without time chunks
+    assert mm.workspace_size(4, 32768, 8192) == 0
+    assert mm.workspace_size(1, 4096, 8192, act=5) == 0
 
 
 # ---------------------------------------------------------------- mixer_fwd validation
@@ -78,6 +82,29 @@ def fwd_args(B=1, Lq=64, D=64, N=16, W=4, act=1, **over):
 
 def call_fwd(L, **kw):
     return L.mamba_mixer_fwd(*fwd_args(**kw))
+
+
+def test_fwd_workspace_rules(L):
+    # B1 L4096 D64 has 2 warps of channels: the plan splits time and needs scratch
+    need = mm.workspace_size(1, 4096, 64)
+    assert need > 0
+    args = fwd_args(B=1, Lq=4096, D=64)
+    ws_addr = BASE + (1 << 36)
+    ok = list(args)
+    ok[-3], ok[-2] = ws_addr, need
+    assert L.mamba_mixer_fwd(*ok) in (EDEVICE, OK, ECUDA)
+    missing = list(args)
+    missing[-3], missing[-2] = None, need
+    assert L.mamba_mixer_fwd(*missing) == 9
+    small = list(args)
+    small[-3], small[-2] = ws_addr, need - 4
+    assert L.mamba_mixer_fwd(*small) == 9
+    mis = list(args)
+    mis[-3], mis[-2] = ws_addr + 4, need
+    assert L.mamba_mixer_fwd(*mis) == EALIGN
+    alias = list(args)
+    alias[-3], alias[-2] = args[11], need          # workspace over y
+    assert L.mamba_mixer_fwd(*alias) == EALIAS
 
 
 def test_fwd_valid_arguments_reach_the_device_check(L):

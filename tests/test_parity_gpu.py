@@ -23,12 +23,14 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(autouse=True)
-def _lpc_env():
-    old = os.environ.pop("MAMBA_MIXER_LPC", None)
+def _tuning_env():
+    names = ("MAMBA_MIXER_LPC", "MAMBA_MIXER_CHUNKS")
+    old = {n: os.environ.pop(n, None) for n in names}
     yield
-    os.environ.pop("MAMBA_MIXER_LPC", None)
-    if old is not None:
-        os.environ["MAMBA_MIXER_LPC"] = old
+    for n in names:
+        os.environ.pop(n, None)
+        if old[n] is not None:
+            os.environ[n] = old[n]
 
 
 def check_fwd(inp, act, chans=None, **kw):
@@ -65,6 +67,21 @@ def test_small_shapes(act, lpc, B, L, D, A_mode):
     os.environ["MAMBA_MIXER_LPC"] = str(lpc)
     inp = make_mixer_inputs_custom(B, L, D, act=act, seed=1000 + L * 7 + D + B, h0_std=0.5, conv_state_std=1.0,
                                    conv_b_std=0.2, A_mode=A_mode, dt_std=0.5)
+    check_fwd(inp, act)
+
+
+CHUNKED = [(act, lpc, k, A_mode) for act in ("bf16", "f32") for lpc in (1, 2, 4) for k in (2, 5)
+           for A_mode in ("structured", "general")]
+
+
+@pytest.mark.parametrize("act,lpc,chunks,A_mode", CHUNKED)
+def test_time_chunked(act, lpc, chunks, A_mode):
+    """The two-pass time-chunked forward (summary pass + seeded full pass),
+    ragged last chunk included."""
+    os.environ["MAMBA_MIXER_LPC"] = str(lpc)
+    os.environ["MAMBA_MIXER_CHUNKS"] = str(chunks)
+    inp = make_mixer_inputs_custom(2, 333, 40, act=act, seed=900 + chunks * 10 + lpc, h0_std=0.5,
+                                   conv_state_std=1.0, conv_b_std=0.2, A_mode=A_mode, dt_std=0.5)
     check_fwd(inp, act)
 
 
@@ -118,13 +135,8 @@ def test_batched_prefill_workload_sampled():
     check_fwd(inp, "bf16", chans=sample_channels(cfg.d_inner, 128))
 
 
-def test_long_256k_carried_chunks_sampled():
-    """256K tokens as 8 carried 32768-token calls: equal (bit for bit) to one
-    unsplit call, and within tolerance of the unsplit oracle."""
-    cfg = CONFIGS["long_256k"]
-    inp = make_mixer_inputs(cfg)
-    dev = to_dev(inp)
-    L, D, n = cfg.seqlen, cfg.d_inner, cfg.chunks
+def _run_carried(dev, n, D):
+    L = dev["xz"].shape[1]
     step = L // n
     y = torch.empty((1, L, D), dtype=torch.bfloat16, device="cuda")
     bufs = [(torch.empty((1, D, 16), device="cuda"), torch.empty((1, D, 3), dtype=torch.bfloat16, device="cuda"))
@@ -139,17 +151,33 @@ def test_long_256k_carried_chunks_sampled():
         yi, h, cs = gpu_fwd(part, h_last=hout, conv_state_out=csout)
         y[:, sl] = yi
         del part
+    return y, h.clone(), cs.clone()
+
+
+def test_long_256k_carried_chunks_sampled():
+    """256K tokens as 8 carried 32768-token calls (the launch plan the
+    benchmark uses) against the unsplit oracle; and, with one time chunk per
+    call, bit-identical to a single unsplit call."""
+    cfg = CONFIGS["long_256k"]
+    inp = make_mixer_inputs(cfg)
+    dev = to_dev(inp)
+    L, D, n = cfg.seqlen, cfg.d_inner, cfg.chunks
+    y, h, cs = _run_carried(dev, n, D)
     torch.cuda.synchronize()
-    y1, h1, cs1 = gpu_fwd(dev)
-    torch.cuda.synchronize()
-    assert torch.equal(y, y1)
-    assert torch.equal(h, h1)
-    assert torch.equal(cs, cs1)
     chans = sample_channels(D, 64)
     ref = oracle_fwd(subset(inp, chans))
     S = torch.as_tensor(chans, device="cuda")
     assert_close(np64(y.index_select(-1, S)), ref["y"], "bf16", "y", stored_bf16=True)
     assert_close(np64(h.index_select(1, S)), ref["h_last"], "bf16", "h_last")
+    np.testing.assert_array_equal(np64(cs.index_select(1, S)), ref["conv_state_out"])
+    del y
+    os.environ["MAMBA_MIXER_CHUNKS"] = "1"
+    y8, h8, cs8 = _run_carried(dev, n, D)
+    y1, h1, cs1 = gpu_fwd(dev)
+    torch.cuda.synchronize()
+    assert torch.equal(y8, y1)
+    assert torch.equal(h8, h1)
+    assert torch.equal(cs8, cs1)
 
 
 # ------------------------------------------------------------------ decode

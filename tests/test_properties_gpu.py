@@ -26,7 +26,9 @@ def _slice(dev, a, b, h0, cs):
 @pytest.mark.parametrize("act", ["bf16", "f32"])
 @pytest.mark.parametrize("lpc", ["1", "2", "4"])
 def test_split_equals_unsplit_bitwise(act, lpc):
+    # one time chunk per call, so both runs apply the same per-token arithmetic
     os.environ["MAMBA_MIXER_LPC"] = lpc
+    os.environ["MAMBA_MIXER_CHUNKS"] = "1"
     try:
         inp = make_mixer_inputs_custom(2, 300, 48, act=act, seed=31, h0_std=0.3, conv_state_std=1.0)
         dev = to_dev(inp)
@@ -43,6 +45,27 @@ def test_split_equals_unsplit_bitwise(act, lpc):
         assert torch.equal(cs, cs_full)
     finally:
         os.environ.pop("MAMBA_MIXER_LPC", None)
+        os.environ.pop("MAMBA_MIXER_CHUNKS", None)
+
+
+@pytest.mark.parametrize("act", ["bf16", "f32"])
+@pytest.mark.parametrize("chunks", ["2", "3", "7"])
+def test_time_chunks_match_one_chunk(act, chunks):
+    """The two-pass time-chunked forward equals the single-chunk forward up to
+    rounding (it is an exact re-association of the recurrence)."""
+    inp = make_mixer_inputs_custom(2, 500, 24, act=act, seed=57, h0_std=0.4, conv_state_std=1.0, conv_b_std=0.1)
+    dev = to_dev(inp)
+    try:
+        os.environ["MAMBA_MIXER_CHUNKS"] = "1"
+        y1, h1, c1 = gpu_fwd(dev)
+        os.environ["MAMBA_MIXER_CHUNKS"] = chunks
+        yk, hk, ck = gpu_fwd(dev)
+        torch.cuda.synchronize()
+    finally:
+        os.environ.pop("MAMBA_MIXER_CHUNKS", None)
+    assert_close(np64(yk), np64(y1), act, "y", stored_bf16=True)
+    assert_close(np64(hk), np64(h1), act, "h_last")
+    assert torch.equal(ck, c1)
 
 
 def _decode_from_prefill(dev, t, h, cs):
