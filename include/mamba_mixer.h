@@ -115,9 +115,9 @@ mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv
                           void* workspace, size_t workspace_bytes, void* stream);
 
 /* Bytes of device scratch mamba_mixer_fwd needs for these sizes (0 = none).
- * A pure function of its arguments (and of the MAMBA_MIXER_LPC /
- * MAMBA_MIXER_CHUNKS tuning variables, which must not change between this
- * call and the forward that uses the result). */
+ * A pure function of its arguments (and of the MAMBA_MIXER_CHUNKS tuning
+ * variable, which must not change between this call and the forward that
+ * uses the result). */
 size_t mamba_mixer_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner,
                                   int64_t d_state, int64_t d_conv, mm_dtype act);
 

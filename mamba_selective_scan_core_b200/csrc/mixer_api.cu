@@ -55,25 +55,17 @@ mm_status check_device(int* sm_count) {
     return MM_OK;
 }
 
-// Launch plan of a forward call: lanes per channel, time chunks and the
-// workspace they need.  A pure function of the sizes (and the two tuning
-// variables), so that mamba_mixer_workspace_size() and the call agree.
+// Launch plan of a forward call: time chunks and the workspace they need.
+// A pure function of the sizes (and of the MAMBA_MIXER_CHUNKS tuning
+// variable), so that mamba_mixer_workspace_size() and the call agree.
 struct FwdPlan {
-    int lpc = 1;
     int chunks = 1;
     int64_t chunk_len = 0;
     size_t ws_bytes = 0;
 };
 
 constexpr int kPlanSMs = 148;            // B200: 2 dies x 74 SMs
-#ifndef MM_WARPS_PER_SM
-#define MM_WARPS_PER_SM 6
-#endif
-#ifndef MM_CTAS_PER_SM
-#define MM_CTAS_PER_SM 1
-#endif
-constexpr int kWarpsPerSM = MM_WARPS_PER_SM;   // resident warps wanted per SM
-constexpr int kCtasPerSM = MM_CTAS_PER_SM;     // resident CTAs the grid is shaped for
+constexpr int kWarpsPerSM = 8;           // resident warps per SM at the forward's register use
 constexpr int kMinChunkTiles = 4;        // shortest chunk worth a summary pass
 constexpr int kMaxChunks = 16;
 
@@ -85,19 +77,18 @@ int env_int(const char* name, int lo, int hi) {
     return 0;
 }
 
+// Time chunks: the fewest that bring the resident warps (two channels per
+// thread) to ~80% of what the SMs hold.
 FwdPlan plan_fwd(int64_t batch, int64_t seqlen, int64_t d_inner) {
     FwdPlan pl;
-    const int lpc = env_int("MAMBA_MIXER_LPC", 1, 4);
-    pl.lpc = (lpc == 1 || lpc == 2 || lpc == 4) ? lpc : 1;
-    const int64_t channels = batch * d_inner;
-    const int64_t warps = channels * pl.lpc / 32;
-    const int64_t want = static_cast<int64_t>(kPlanSMs) * kWarpsPerSM;
+    const int64_t warps = std::max<int64_t>(1, batch * d_inner / 2 / 32);
+    const int64_t want = static_cast<int64_t>(kPlanSMs) * kWarpsPerSM * 4 / 5;
     const int64_t tiles = (seqlen + kTile - 1) / kTile;
     int64_t k = 1;
     if (const int forced = env_int("MAMBA_MIXER_CHUNKS", 1, 1 << 20)) {
         k = forced;
     } else if (warps < want) {
-        k = (want + std::max<int64_t>(warps, 1) - 1) / std::max<int64_t>(warps, 1);
+        k = (want + warps - 1) / warps;
         k = std::min<int64_t>(k, std::max<int64_t>(1, tiles / kMinChunkTiles));
         k = std::min<int64_t>(k, kMaxChunks);
     }
@@ -110,9 +101,9 @@ FwdPlan plan_fwd(int64_t batch, int64_t seqlen, int64_t d_inner) {
     return pl;
 }
 
-template <typename T, typename M, int LPC, int STAGES, bool SUMMARY>
+template <typename T, typename M, int STAGES, bool SUMMARY>
 cudaError_t launch_prefill(const PrefillParams& p, int64_t batch, int chunks, int threads, cudaStream_t s) {
-    auto kern = mm::mixer_fwd_kernel<T, M, LPC, kTile, STAGES, SUMMARY>;
+    auto kern = mm::mixer_fwd_kernel<T, M, kTile, STAGES, SUMMARY>;
     const int smem = PrefillLayout<T>::smem_bytes(kTile, STAGES, p.octets);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -121,54 +112,66 @@ cudaError_t launch_prefill(const PrefillParams& p, int64_t batch, int chunks, in
     return cudaGetLastError();
 }
 
-// Octets per CTA: spread the (channel octet, chunk) units over about one CTA
-// per SM, capped by the CTA size and the shared-memory budget; then even out
-// the CTAs of a sequence so that none is a small remainder.
+// Octets per CTA (4 threads per octet) and copy-ring depth.  Every warp of
+// a pass does the same work, so the pass takes about one warp's time per
+// wave: pick the shape with the fewest waves, counting how many CTAs an SM
+// holds under both its register file (8 warps at the forward's register use)
+// and its shared memory; among equals prefer the wider CTA (B/C staging is
+// shared by a CTA's channels), then the deeper ring.
+constexpr int kSmemPerSM = 227 * 1024;
+
 template <typename T>
-void shape_ctas(PrefillParams& p, int64_t batch, int64_t units_per_octet, int lpc, int sm_count, int* threads) {
-    const int64_t octets_per_seq = p.D / 8;
-    int max_oct = kMaxThreads / (8 * lpc);
-    while (max_oct > 1 && PrefillLayout<T>::smem_bytes(kTile, 2, max_oct) > kSmemBudget) --max_oct;
-    const int64_t slots = static_cast<int64_t>(sm_count) * kCtasPerSM;
-    int64_t oct = (batch * octets_per_seq * units_per_octet + slots - 1) / slots;
-    oct = std::max<int64_t>(1, std::min<int64_t>({oct, max_oct, octets_per_seq}));
-    const int64_t ctas = (octets_per_seq + oct - 1) / oct;
-    oct = (octets_per_seq + ctas - 1) / ctas;
-    p.octets = static_cast<int>(oct);
-    p.ctas_per_seq = static_cast<int>(ctas);
-    *threads = static_cast<int>(((oct * 8 * lpc) + 31) / 32 * 32);
+int ring_depth(int oct) {
+    for (int st = 4; st >= 2; --st)
+        if (PrefillLayout<T>::smem_bytes(kTile, st, oct) <= kSmemBudget) return st;
+    return 0;
 }
 
-template <typename T, typename M, int LPC, bool SUMMARY>
+template <typename T>
+int shape_ctas(PrefillParams& p, int64_t batch, int64_t chunks, int sm_count, int* threads) {
+    const int64_t octets_per_seq = p.D / 8;
+    const int max_oct = static_cast<int>(std::min<int64_t>(kMaxThreads / 4, octets_per_seq));
+    int64_t best_waves = INT64_MAX;
+    int best = 1, best_stages = 2;
+    for (int oct = 1; oct <= max_oct; ++oct) {
+        const int64_t per_seq = (octets_per_seq + oct - 1) / oct;
+        if (per_seq * oct - octets_per_seq >= oct) continue;        // same CTA count as a smaller oct
+        const int warps = (oct * 4 + 31) / 32;
+        for (int st = ring_depth<T>(oct); st >= 2; --st) {
+            const int smem = PrefillLayout<T>::smem_bytes(kTile, st, oct);
+            const int per_sm = std::max(1, std::min(kWarpsPerSM / warps, kSmemPerSM / smem));
+            const int64_t slots = static_cast<int64_t>(sm_count) * per_sm;
+            const int64_t waves = (batch * per_seq * chunks + slots - 1) / slots;
+            if (waves < best_waves || (waves == best_waves && (oct > best || (oct == best && st > best_stages)))) {
+                best_waves = waves; best = oct; best_stages = st;
+            }
+        }
+    }
+    const int64_t ctas = (octets_per_seq + best - 1) / best;
+    p.octets = static_cast<int>((octets_per_seq + ctas - 1) / ctas);
+    p.ctas_per_seq = static_cast<int>(ctas);
+    *threads = ((p.octets * 4) + 31) / 32 * 32;
+    return std::min(best_stages, std::max(2, ring_depth<T>(p.octets)));
+}
+
+template <typename T, typename M, bool SUMMARY>
 cudaError_t launch_pass(PrefillParams p, int64_t batch, int chunks, int sm_count, cudaStream_t s) {
     int threads = 0;
-    shape_ctas<T>(p, batch, chunks, LPC, sm_count, &threads);
-    // as deep a copy ring as fits the shared-memory budget (4, else 3, else 2)
-    if (PrefillLayout<T>::smem_bytes(kTile, 4, p.octets) <= kSmemBudget)
-        return launch_prefill<T, M, LPC, 4, SUMMARY>(p, batch, chunks, threads, s);
-    if (PrefillLayout<T>::smem_bytes(kTile, 3, p.octets) <= kSmemBudget)
-        return launch_prefill<T, M, LPC, 3, SUMMARY>(p, batch, chunks, threads, s);
-    return launch_prefill<T, M, LPC, 2, SUMMARY>(p, batch, chunks, threads, s);
-}
-
-template <typename T, typename M, int LPC>
-cudaError_t run_fwd(const PrefillParams& p, int64_t batch, int chunks, int sm_count, cudaStream_t s) {
-    if (chunks > 1) {
-        cudaError_t e = launch_pass<T, M, LPC, true>(p, batch, chunks - 1, sm_count, s);
-        if (e != cudaSuccess) return e;
-    }
-    return launch_pass<T, M, LPC, false>(p, batch, chunks, sm_count, s);
+    const int stages = shape_ctas<T>(p, batch, chunks, sm_count, &threads);
+    if (stages >= 4) return launch_prefill<T, M, 4, SUMMARY>(p, batch, chunks, threads, s);
+    if (stages == 3) return launch_prefill<T, M, 3, SUMMARY>(p, batch, chunks, threads, s);
+    return launch_prefill<T, M, 2, SUMMARY>(p, batch, chunks, threads, s);
 }
 
 template <typename T, typename M>
 cudaError_t dispatch_prefill(PrefillParams p, int64_t batch, const FwdPlan& pl, int sm_count, cudaStream_t s) {
     p.chunk_len = pl.chunk_len;
     p.n_chunks = pl.chunks;
-    switch (pl.lpc) {
-        case 1: return run_fwd<T, M, 1>(p, batch, pl.chunks, sm_count, s);
-        case 2: return run_fwd<T, M, 2>(p, batch, pl.chunks, sm_count, s);
-        default: return run_fwd<T, M, 4>(p, batch, pl.chunks, sm_count, s);
+    if (pl.chunks > 1) {
+        cudaError_t e = launch_pass<T, M, true>(p, batch, pl.chunks - 1, sm_count, s);
+        if (e != cudaSuccess) return e;
     }
+    return launch_pass<T, M, false>(p, batch, pl.chunks, sm_count, s);
 }
 
 }  // namespace

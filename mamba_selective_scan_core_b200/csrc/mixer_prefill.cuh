@@ -13,71 +13,51 @@
 // each of the 16 states, a decay, a Delta*u*B product, the state FMA and the
 // readout FMA -- at least 64 fp32 pipe operations against 8 bytes of HBM
 // traffic (x, z, dt in, y out; B/C are shared by all channels).  At 128 fp32
-// lanes per SM per clock that is the binding limit, not HBM, so the kernel is
-// laid out to spend as few fp32/issue slots as possible per state element:
-//   * the state lives in registers (no re-scan of a chunk from its carried
-//     state, nothing re-read from HBM);
-//   * state pairs use packed f32x2 FMA/MUL (one issue slot per two lanes);
+// lanes per SM per clock that, not HBM, is the binding limit, so the kernel is
+// laid out to spend as few fp32-pipe and issue slots as possible:
+//   * a thread owns two adjacent channels and keeps their 2 x 16 states in
+//     registers for its whole stretch of the sequence; every state operation,
+//     and the per-token conv / softplus / SiLU / gate arithmetic, is a packed
+//     f32x2 instruction over the two channels, and x, z, dt, y move as 32-bit
+//     bf16 pairs;
 //   * when a channel's A row is A[n] = (n+1) A[0] (detected on the device, per
-//     warp), the 16 decays are powers of q = exp(Delta A[0]): one ex2 plus one
-//     packed multiply per state pair, instead of 16 ex2 on the 16/clk MUFU;
-//   * the per-token work shared by a channel's states (conv, softplus, SiLU,
-//     gate) runs once per (token, channel).
+//     warp), the 16 decays are powers of q = exp(Delta A[0]): one ex2 and one
+//     packed multiply per state instead of 16 ex2 on the 16/clk MUFU pipe;
+//   * B_t/C_t, shared by every channel of a sequence, are staged once per CTA
+//     and tile in shared memory, each value duplicated into a pair, so one
+//     16-byte load feeds two states of both channels.
 //
-// Parallelism.  The recurrence is sequential in t per channel, and a single
-// 8192-channel sequence is only 256 warps at one lane per channel -- under 2
-// per SM.  Two ways to get more, both exact re-associations of the linear
-// recurrence h_t = a_t h_{t-1} + b_t:
-//   * time chunks (two passes): a summary pass runs each of chunks 0..K-2
-//     from a zero state and keeps only its end state e_c and the sum of its
-//     step sizes (whose exponential is the chunk's total decay P_c); the full
-//     pass then starts chunk c from h0 combined with (P_0, e_0) .. (P_{c-1},
-//     e_{c-1}), i.e. the true state at the chunk boundary, and runs the fused
-//     forward.  The summary pass skips the readout, gate and z/C traffic.
-//   * state splitting: a channel's 16 states are spread over LPC = 2 or 4
-//     lanes that take turns doing the per-token work and exchange (decay
-//     base, Delta*u) and the partial readouts with warp shuffles.
+// Parallelism.  The recurrence is sequential in t per channel: a single
+// 8192-channel sequence is only 4096 channel pairs, 128 warps.  Time chunks
+// supply the rest, as an exact re-association of h_t = a_t h_{t-1} + b_t:
+// a summary pass runs each of chunks 0..K-2 from a zero state and keeps its
+// end state e_c and the sum of its step sizes (whose exponential is the
+// chunk's total decay P_c); the full pass starts chunk c from h0 carried
+// through (P_0, e_0) .. (P_{c-1}, e_{c-1}) -- the true state at the chunk
+// boundary -- and runs the fused forward.  The summary pass skips the
+// readout, the gate and the z/C traffic.
 //
-// Latency: each tile of TILE tokens is processed in sub-tiles of SUB tokens
-// in three phases, so that the long per-token chains (conv -> SiLU ->
-// softplus -> exp) of SUB tokens are independent and overlap:
-//   A. per-token work for the SUB tokens (each lane owns every LPC-th token);
-//   B. the state update for the SUB tokens (the only serial dependency is
-//      one FMA per token on each state; decay powers by repeated squaring,
-//      readout over two accumulators);
-//   C. transpose-reduce of the partial readouts over the LPC lanes, skip,
-//      gate and store, again for all SUB tokens at once.
+// Latency: each tile is processed in sub-tiles of SUB tokens in three phases
+// so that the long per-token chains (conv -> SiLU -> softplus -> exp) of SUB
+// tokens are independent and overlap: A. per-token work, B. the state update
+// (the only serial dependency is one FMA per token on each state; decay
+// powers by repeated squaring), C. skip, gate and store.
 //
 // Data movement: each CTA owns a contiguous block of channels of one sequence
 // and one time chunk, and walks it in tiles of TILE tokens.  x (with 3 rows
 // of left context), z, dt rows of the block and the B_t/C_t rows are staged
 // in shared memory by cp.async 16-byte copies in a STAGES-deep ring (rows
 // outside the chunk are zero-filled; the left context of token 0 comes from
-// the carried conv window); B/C are converted once per tile to fp32, permuted
-// so each lane's states are contiguous, and shared by every channel of the
-// CTA.
+// the carried conv window).
 #pragma once
 
 #include <type_traits>
 
 #include "mixer_common.cuh"
 
-// Scheduling knobs of the forward kernel (compile-time; the defaults are the
-// measured best on B200).
-#ifndef MM_SUB1
-#define MM_SUB1 8              // tokens per sub-tile at one lane per channel
+#ifndef MM_SUB
+#define MM_SUB 8               // tokens per sub-tile
 #endif
-#ifndef MM_SUBTILE_UNROLL
-#define MM_SUBTILE_UNROLL 1    // sub-tiles unrolled together (lets phases overlap)
-#endif
-#ifndef MM_TOKENS_OUTER
-#define MM_TOKENS_OUTER 0      // phase B loop order: 0 = state pairs outer, 1 = tokens outer
-#endif
-#ifndef MM_MIN_BLOCKS
-#define MM_MIN_BLOCKS 1        // resident CTAs per SM the register budget must allow
-#endif
-#define MM_PRAGMA_(x) _Pragma(#x)
-#define MM_PRAGMA(x) MM_PRAGMA_(x)
 
 namespace mm {
 
@@ -98,7 +78,7 @@ struct PrefillParams {
     void* cs_out;
     int64_t L;          // tokens per sequence
     int D;              // d_inner
-    int octets;         // channel octets (8 channels) per CTA
+    int octets;         // channel octets (8 channels, 4 threads) per CTA
     int ctas_per_seq;   // CTAs per sequence
     int64_t chunk_len;  // tokens per time chunk (a multiple of the tile)
     int n_chunks;       // time chunks K (blockIdx.y of the full pass)
@@ -118,10 +98,9 @@ struct PrefillLayout {
     __host__ __device__ static int stage_bytes(int tile, int octets) {
         return (3 * tile + kHalo) * row_bytes(octets) + 2 * tile * bc_row_bytes();
     }
-    // plus the tile's B/C in fp32, [lane j][pair k][token r][B0 B1 C0 C1], each
-    // lane class's block padded by 16 bytes so the LPC classes hit different banks
+    // plus the tile's B/C in fp32, each value duplicated: [token][B0 B0 B1 B1 .. C15 C15]
     __host__ __device__ static int smem_bytes(int tile, int stages, int octets) {
-        return stages * stage_bytes(tile, octets) + tile * 32 * 4 + 4 * 16;
+        return stages * stage_bytes(tile, octets) + tile * 64 * 4;
     }
 };
 
@@ -139,36 +118,61 @@ struct GridWalk {
     }
 };
 
+// A pair of adjacent activations <-> float2.
+template <typename T> struct Pair;
+template <> struct Pair<float> {
+    __device__ __forceinline__ static float2 load(const float* p) { return *reinterpret_cast<const float2*>(p); }
+    __device__ __forceinline__ static void store(float* p, float2 v) { *reinterpret_cast<float2*>(p) = v; }
+};
+template <> struct Pair<__nv_bfloat16> {
+    __device__ __forceinline__ static float2 load(const __nv_bfloat16* p) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+    __device__ __forceinline__ static void store(__nv_bfloat16* p, float2 v) {
+        *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v.x, v.y);
+    }
+};
+
+// Packed forms of the math policy's per-channel functions.
+template <typename M>
+__device__ __forceinline__ float2 silu2(float2 v) { return f2(M::silu(v.x), M::silu(v.y)); }
+
+template <typename M>
+__device__ __forceinline__ float2 step_pair(float2 dt, float2 bias) {
+    if constexpr (M::step_scale == 1.0f) return f2(M::step(dt.x, bias.x), M::step(dt.y, bias.y));
+    else return f2(M::step2(dt.x, bias.x), M::step2(dt.y, bias.y));
+}
+
+template <typename M>
+__device__ __forceinline__ float2 decay2(float2 l, float2 a) {
+    return f2(M::decay(l.x, a.x), M::decay(l.y, a.y));
+}
+
 // SUMMARY = true: the summary pass (chunk end state from zero + sum of l).
 // SUMMARY = false: the full fused forward over one chunk.
-template <typename T, typename M, int LPC, int TILE, int STAGES, bool SUMMARY>
-__global__ void __launch_bounds__(256, MM_MIN_BLOCKS)
+template <typename T, typename M, int TILE, int STAGES, bool SUMMARY>
+__global__ void __launch_bounds__(256, 1)
 mixer_fwd_kernel(const PrefillParams p)
 {
-    static_assert(LPC == 1 || LPC == 2 || LPC == 4, "lanes per channel");
-    constexpr int NS = 16 / LPC;          // states per lane
-    constexpr int NP = NS / 2;            // packed state pairs per lane
-    constexpr int SUB = LPC == 1 ? MM_SUB1 : 16;  // tokens per sub-tile
-    constexpr int OWN = SUB / LPC;        // tokens of a sub-tile this lane owns
-    constexpr int XW = SUB - LPC + 4;     // x window a lane reads per sub-tile
+    constexpr int SUB = MM_SUB;
     static_assert(TILE % SUB == 0, "tile");
     constexpr bool kFast = (M::step_scale != 1.0f);
     using A_ = Act<T>;
+    using P_ = Pair<T>;
 
     extern __shared__ __align__(16) unsigned char smem[];
 
     const int tid = threadIdx.x;
-    const int lane = tid & 31;
-    const int j = tid % LPC;                  // lane within the channel
-    const int cl = tid / LPC;                 // channel within the CTA
     const int seq = blockIdx.x / p.ctas_per_seq;
     const int blk = blockIdx.x - seq * p.ctas_per_seq;
     const int chunk = blockIdx.y;
     const int d0 = blk * p.octets * 8;
     const int nch = min(p.octets * 8, p.D - d0);
+    const int cl = 2 * tid;                      // first of my two channels, within the CTA
     const bool active = cl < nch;
     const int d = d0 + (active ? cl : 0);
-    const int cls = min(cl, p.octets * 8 - 1);   // staged column (padding lanes read a real one)
+    const int cls = min(cl, p.octets * 8 - 2);   // staged column (padding threads read a real one)
     const int64_t L = p.L;
     const int D = p.D;
     const int nthreads = blockDim.x;
@@ -181,15 +185,14 @@ mixer_fwd_kernel(const PrefillParams p)
     const int offZ = (TILE + kHalo) * rowB;
     const int offDT = offZ + TILE * rowB;
     const int offBC = offDT + TILE * rowB;
-    float* bcf = reinterpret_cast<float*>(smem + STAGES * stageB);   // [LPC][NP][TILE][4] (+pad)
-    constexpr int JSTRIDE = NP * TILE * 4 + 4;                         // floats per lane class
+    float* bcf = reinterpret_cast<float*>(smem + STAGES * stageB);   // [TILE][64]
 
     const T* xz = static_cast<const T*>(p.xz);
     const T* dtg = static_cast<const T*>(p.dt);
     const T* Bg = static_cast<const T*>(p.Bm);
     const T* Cg = static_cast<const T*>(p.Cm);
     const int64_t seq_row0 = static_cast<int64_t>(seq) * L;
-    const int64_t chan = static_cast<int64_t>(seq) * D + d;           // (sequence, channel) row
+    const int64_t chan = static_cast<int64_t>(seq) * D + d;           // (sequence, first channel) row
 
     // ---------------------------------------------------------- tile loader
     constexpr int kEPC = 16 / sizeof(T);              // elements per 16-byte chunk
@@ -234,42 +237,44 @@ mixer_fwd_kernel(const PrefillParams p)
         cp_async_commit();
     };
 
-    // ---------------------------------------------------------- per-lane setup
-    float w[4] = {0.f, 0.f, 0.f, 0.f};
-    float cb = 0.f, bias = 0.f, dsk = 0.f;
-    float a_row[NS];                // A[d, j + LPC*i]
-    float A0 = 0.f;
-    float h[NS];
+    // ---------------------------------------------------------- per-thread setup
+    float2 w2[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) w2[k] = f2(0.f, 0.f);
+    float2 cb2 = f2(0.f, 0.f), bias2 = f2(0.f, 0.f), dsk2 = f2(0.f, 0.f), A02 = f2(0.f, 0.f);
     if (active) {
-        const float4 wv = *reinterpret_cast<const float4*>(p.conv_w + static_cast<int64_t>(d) * 4);
-        w[0] = wv.x; w[1] = wv.y; w[2] = wv.z; w[3] = wv.w;
-        cb = p.conv_b ? p.conv_b[d] : 0.f;
-        bias = p.dt_bias[d];
-        dsk = p.Dskip ? p.Dskip[d] : 0.f;
+        const float4 wa = *reinterpret_cast<const float4*>(p.conv_w + static_cast<int64_t>(d) * 4);
+        const float4 wb = *reinterpret_cast<const float4*>(p.conv_w + static_cast<int64_t>(d + 1) * 4);
+        w2[0] = f2(wa.x, wb.x); w2[1] = f2(wa.y, wb.y); w2[2] = f2(wa.z, wb.z); w2[3] = f2(wa.w, wb.w);
+        if (p.conv_b) cb2 = *reinterpret_cast<const float2*>(p.conv_b + d);
+        bias2 = *reinterpret_cast<const float2*>(p.dt_bias + d);
+        if (p.Dskip) dsk2 = *reinterpret_cast<const float2*>(p.Dskip + d);
+        A02 = f2(p.A[static_cast<int64_t>(d) * 16], p.A[static_cast<int64_t>(d + 1) * 16]);
     }
-    if constexpr (kFast) bias *= kLog2e;
-    {
-        const float* arow = p.A + static_cast<int64_t>(d) * 16;
-        A0 = active ? arow[0] : 0.f;
+    if constexpr (kFast) bias2 = mul2(bias2, f2(kLog2e, kLog2e));
+    const float* arow0 = p.A + static_cast<int64_t>(d) * 16;
+    const float* arow1 = arow0 + 16;
+
+    // state pairs h[n] = (h_d[n], h_{d+1}[n]), at the start of this chunk
+    float2 h[16];
+    if constexpr (SUMMARY) {
 #pragma unroll
-        for (int i = 0; i < NS; ++i) a_row[i] = active ? arow[j + LPC * i] : 0.f;
-        if constexpr (SUMMARY) {
+        for (int n = 0; n < 16; ++n) h[n] = f2(0.f, 0.f);
+    } else {
+        const float* h0 = (p.h0 && active) ? p.h0 + chan * 16 : nullptr;
 #pragma unroll
-            for (int i = 0; i < NS; ++i) h[i] = 0.f;
-        } else {
-            // state at the chunk boundary: h0 carried through the summaries of
-            // the chunks before this one, h <- exp(A * sum Delta) h + e
-            const float* h0 = p.h0 ? p.h0 + chan * 16 : nullptr;
-#pragma unroll
-            for (int i = 0; i < NS; ++i) h[i] = (active && h0) ? h0[j + LPC * i] : 0.f;
+        for (int n = 0; n < 16; ++n) h[n] = h0 ? f2(h0[n], h0[16 + n]) : f2(0.f, 0.f);
+        // carry h0 through the summaries of the chunks before this one:
+        // h <- exp(A sum Delta) h + e
+        if (active && chunk > 0) {
             const int64_t stride = static_cast<int64_t>(p.batch) * D;
 #pragma unroll 1
             for (int c = 0; c < chunk; ++c) {
-                const float ls = active ? p.ws_lsum[c * stride + chan] : 0.f;
-                const float* e = p.ws_state + (c * stride + chan) * 16;
+                const float2 ls = *reinterpret_cast<const float2*>(p.ws_lsum + c * stride + chan);
+                const float* e0 = p.ws_state + (c * stride + chan) * 16;
 #pragma unroll
-                for (int i = 0; i < NS; ++i)
-                    h[i] = fmaf(M::decay(ls, a_row[i]), h[i], active ? e[j + LPC * i] : 0.f);
+                for (int n = 0; n < 16; ++n)
+                    h[n] = fma2(decay2<M>(ls, f2(arow0[n], arow1[n])), h[n], f2(e0[n], e0[16 + n]));
             }
         }
     }
@@ -279,9 +284,12 @@ mixer_fwd_kernel(const PrefillParams p)
     bool structured = false;
     if constexpr (kFast) {
         bool mine = true;
+        if (active) {
 #pragma unroll
-        for (int i = 0; i < NS; ++i) mine = mine && (a_row[i] == static_cast<float>(j + LPC * i + 1) * A0);
-        structured = __all_sync(kFull, mine || !active);
+            for (int n = 0; n < 16; ++n)
+                mine = mine && arow0[n] == static_cast<float>(n + 1) * A02.x && arow1[n] == static_cast<float>(n + 1) * A02.y;
+        }
+        structured = __all_sync(kFull, mine);
     }
 
     // ---------------------------------------------------------- pipeline prologue
@@ -289,242 +297,155 @@ mixer_fwd_kernel(const PrefillParams p)
     for (int s = 0; s < STAGES - 1; ++s) load_tile(s);
 
     T* yg = static_cast<T*>(p.y);
-    const int lane_base = lane & ~(LPC - 1);
-    float lsum = 0.f;                   // summary pass: sum of l over my tokens
+    float2 lsum = f2(0.f, 0.f);           // summary pass: sum of l over the chunk
 
     // One sub-tile of SUB tokens starting at staged row r0 (token t0).
-    auto run_sub = [&](const unsigned char* st, int r0, int64_t t0, auto structured_tag) {
+    // a2 (general A only): the 16 A pairs of my channels.
+    auto run_sub = [&](const unsigned char* st, int r0, int64_t t0, auto structured_tag, const float2* a2) {
         constexpr bool kStruct = decltype(structured_tag)::value;
         const T* xs = reinterpret_cast<const T*>(st);          // row rho = token - 3 (tile-relative)
         const T* zs = reinterpret_cast<const T*>(st + offZ);
         const T* ds = reinterpret_cast<const T*>(st + offDT);
+        const int nvalid = static_cast<int>(min(static_cast<int64_t>(SUB), t_end - t0));   // tokens of the chunk here
 
-        // ---- A: per-token work of my tokens r0 + LPC*i + j
-        float xw[XW];                                        // x of staged rows r0+j .. r0+j+XW-1
+        // ---- A: per-token work (conv, SiLU, step, Delta*u), both channels packed
+        float2 xw[SUB + 3];
 #pragma unroll
-        for (int k = 0; k < XW; ++k) xw[k] = A_::to_f32(xs[(r0 + j + k) * rs + cls]);
-        float ea[OWN], sa[OWN], ua[OWN];
-#pragma unroll
-        for (int i = 0; i < OWN; ++i) {
-            const int r = r0 + LPC * i + j;                  // tile row of this token
-            float pre = cb;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) pre = fmaf(w[k], xw[LPC * i + k], pre);
-            const float u = M::silu(pre);
-            const float dtv = A_::to_f32(ds[r * rs + cls]);
-            float l;
-            if constexpr (kFast) l = M::step2(dtv, bias);
-            else l = M::step(dtv, bias);
-            float s = l * u;                                 // Delta*u in B' units (B' = B * step_scale)
-            const bool valid = t0 + LPC * i + j < t_end;
-            if (!valid) { l = 0.f; s = 0.f; }
-            if constexpr (SUMMARY) lsum += l;
-            if constexpr (kStruct) ea[i] = ex2_fast(l * A0);  // q = exp(Delta A[0])
-            else ea[i] = l;
-            sa[i] = s;
-            ua[i] = u;
-        }
-
-        // ---- B: state update over the SUB tokens.  Pairs of states outer,
-        // tokens inner: each pair is a chain of SUB dependent FMAs, and the
-        // NP pairs are independent of each other.
-        float em[SUB], sm[SUB];
+        for (int k = 0; k < SUB + 3; ++k) xw[k] = P_::load(xs + (r0 + k) * rs + cls);
+        float2 ea[SUB], sa[SUB], ua[SUB];
 #pragma unroll
         for (int m = 0; m < SUB; ++m) {
-            const int i = m / LPC, o = m % LPC;
-            em[m] = (LPC == 1) ? ea[i] : __shfl_sync(kFull, ea[i], lane_base + o);
-            sm[m] = (LPC == 1) ? sa[i] : __shfl_sync(kFull, sa[i], lane_base + o);
-        }
-        // structured decays q^(n+1), n = j + LPC*i: per token a running pair
-        // (b Q^(2k), b Q^(2k+1)) with base b = q^(j+1) and stride Q = q^LPC
-        float2 pw[SUB];
-        float qq[SUB];
-        if constexpr (kStruct) {
+            float2 pre = cb2;
 #pragma unroll
-            for (int m = 0; m < SUB; ++m) {
-                const float q1 = em[m];
-                float b, Q;
-                if constexpr (LPC == 1) { b = q1; Q = q1; }
-                else if constexpr (LPC == 2) { const float q2 = q1 * q1; b = j ? q2 : q1; Q = q2; }
-                else {
-                    const float q2 = q1 * q1, q3 = q2 * q1, q4 = q2 * q2;
-                    b = (j & 2) ? ((j & 1) ? q4 : q3) : ((j & 1) ? q2 : q1);
-                    Q = q4;
-                }
-                pw[m] = f2(b, b * Q);
-                qq[m] = Q * Q;
-            }
+            for (int k = 0; k < 4; ++k) pre = fma2(w2[k], xw[m + k], pre);
+            const float2 u = silu2<M>(pre);
+            float2 l = step_pair<M>(P_::load(ds + (r0 + m) * rs + cls), bias2);
+            if (m >= nvalid) l = f2(0.f, 0.f);                  // past the chunk: no step
+            const float2 s = mul2(l, u);                         // Delta*u in B' units (B' = B * step_scale)
+            if constexpr (SUMMARY) lsum = __fadd2_rn(lsum, l);
+            if constexpr (kStruct) ea[m] = f2(ex2_fast(l.x * A02.x), ex2_fast(l.y * A02.y));   // q
+            else ea[m] = l;
+            sa[m] = s;
+            ua[m] = u;
         }
-#if MM_TOKENS_OUTER
+
+        // ---- B: state update (and readout) over the SUB tokens
         float2 yacc[SUB];
-        const float* bj = bcf + j * JSTRIDE + r0 * 4;
 #pragma unroll
         for (int m = 0; m < SUB; ++m) {
-            float2 P[NP];
+            float2 P[16];
             if constexpr (kStruct) {
-                P[0] = pw[m];
-                float st2 = qq[m];
+                // P[n] = q^(n+1) by repeated squaring: depth 4, 15 packed multiplies
+                P[0] = ea[m];
+                P[1] = mul2(P[0], P[0]);
+                P[2] = mul2(P[1], P[0]);
+                P[3] = mul2(P[1], P[1]);
 #pragma unroll
-                for (int len = 1; len < NP; len *= 2) {
-                    const float2 sv = f2(st2, st2);
+                for (int n = 0; n < 4; ++n) P[4 + n] = mul2(P[n], P[3]);
 #pragma unroll
-                    for (int k = 0; k < len; ++k)
-                        if (k + len < NP) P[k + len] = mul2(P[k], sv);
-                    st2 = st2 * st2;
-                }
+                for (int n = 0; n < 8; ++n) P[8 + n] = mul2(P[n], P[7]);
             } else {
 #pragma unroll
-                for (int k = 0; k < NP; ++k)
-                    P[k] = f2(M::decay(em[m], a_row[2 * k]), M::decay(em[m], a_row[2 * k + 1]));
+                for (int n = 0; n < 16; ++n) P[n] = decay2<M>(ea[m], a2[n]);
             }
-            float2 acc[2];
+            const float* row = bcf + (r0 + m) * 64;
+            const float2 s = sa[m];
+            float2 acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
 #pragma unroll
-            for (int k = 0; k < NP; ++k) {
-                const float* slot = bj + (k * TILE + m) * 4;
-                float2 hh = f2(h[2 * k], h[2 * k + 1]);
-                if constexpr (SUMMARY) {
-                    const float2 bb = *reinterpret_cast<const float2*>(slot);
-                    hh = fma2(P[k], hh, mul2(f2(sm[m], sm[m]), bb));
-                } else {
-                    const float4 bc = *reinterpret_cast<const float4*>(slot);
-                    hh = fma2(P[k], hh, mul2(f2(sm[m], sm[m]), f2(bc.x, bc.y)));
-                    acc[k & 1] = (k < 2) ? mul2(f2(bc.z, bc.w), hh) : fma2(f2(bc.z, bc.w), hh, acc[k & 1]);
+            for (int n = 0; n < 16; n += 2) {
+                const float4 bb = *reinterpret_cast<const float4*>(row + 2 * n);        // (Bn, Bn, Bn+1, Bn+1)
+                h[n] = fma2(P[n], h[n], mul2(s, f2(bb.x, bb.y)));
+                h[n + 1] = fma2(P[n + 1], h[n + 1], mul2(s, f2(bb.z, bb.w)));
+                if constexpr (!SUMMARY) {
+                    const float4 cc = *reinterpret_cast<const float4*>(row + 32 + 2 * n);   // (Cn, Cn, Cn+1, Cn+1)
+                    acc0 = fma2(f2(cc.x, cc.y), h[n], acc0);
+                    acc1 = fma2(f2(cc.z, cc.w), h[n + 1], acc1);
                 }
-                h[2 * k] = hh.x; h[2 * k + 1] = hh.y;
             }
-            if constexpr (!SUMMARY) yacc[m] = __fadd2_rn(acc[0], acc[1]);
+            if constexpr (!SUMMARY) yacc[m] = __fadd2_rn(acc0, acc1);
         }
-#else
-        float2 yacc[SUB];
-        const float* bj = bcf + j * JSTRIDE + r0 * 4;
-#pragma unroll
-        for (int k = 0; k < NP; ++k) {
-            float2 hh = f2(h[2 * k], h[2 * k + 1]);
+
+        // ---- C: skip, gate, store
+        if constexpr (!SUMMARY) {
 #pragma unroll
             for (int m = 0; m < SUB; ++m) {
-                const float* slot = bj + (k * TILE + m) * 4;
-                float2 P;
-                if constexpr (kStruct) {
-                    P = pw[m];
-                    if (k + 1 < NP) pw[m] = mul2(pw[m], f2(qq[m], qq[m]));
-                } else {
-                    P = f2(M::decay(em[m], a_row[2 * k]), M::decay(em[m], a_row[2 * k + 1]));
-                }
-                if constexpr (SUMMARY) {
-                    const float2 bb = *reinterpret_cast<const float2*>(slot);
-                    hh = fma2(P, hh, mul2(f2(sm[m], sm[m]), bb));
-                } else {
-                    const float4 bc = *reinterpret_cast<const float4*>(slot);
-                    hh = fma2(P, hh, mul2(f2(sm[m], sm[m]), f2(bc.x, bc.y)));
-                    yacc[m] = (k == 0) ? mul2(f2(bc.z, bc.w), hh) : fma2(f2(bc.z, bc.w), hh, yacc[m]);
-                }
-            }
-            h[2 * k] = hh.x; h[2 * k + 1] = hh.y;
-        }
-#endif
-        float yp[SUB];
-        if constexpr (!SUMMARY) {
-#pragma unroll
-            for (int m = 0; m < SUB; ++m) yp[m] = yacc[m].x + yacc[m].y;
-        }
-        if constexpr (!SUMMARY) {
-            // ---- C: transpose-reduce each group of LPC tokens (lane j ends with
-            // token LPC*i + j), then skip, gate, store
-#pragma unroll
-            for (int i = 0; i < OWN; ++i) {
-                float* v = yp + LPC * i;
-#pragma unroll
-                for (int bit = LPC / 2; bit >= 1; bit >>= 1) {
-                    const bool upper = (j & bit) != 0;
-#pragma unroll
-                    for (int q = 0; q < bit; ++q) {
-                        const float send = upper ? v[q] : v[q + bit];
-                        const float keep = upper ? v[q + bit] : v[q];
-                        v[q] = keep + __shfl_xor_sync(kFull, send, bit);
-                    }
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < OWN; ++i) {
-                const int r = r0 + LPC * i + j;
-                const int64_t t = t0 + LPC * i + j;
-                const float zv = A_::to_f32(zs[r * rs + cls]);
-                if (t < t_end && active) {
-                    const float yv = fmaf(dsk, ua[i], yp[LPC * i]) * M::silu(zv);
-                    yg[(seq_row0 + t) * D + d] = A_::from_f32(yv);
-                }
+                const float2 g = silu2<M>(P_::load(zs + (r0 + m) * rs + cls));
+                const float2 yv = mul2(fma2(dsk2, ua[m], yacc[m]), g);
+                if (m < nvalid && active) P_::store(yg + (seq_row0 + t0 + m) * D + d, yv);
             }
         }
     };
 
     // ---------------------------------------------------------- main loop
-    const T* csi = p.cs_in ? static_cast<const T*>(p.cs_in) + chan * 3 : nullptr;
+    const T* csi = (p.cs_in && active) ? static_cast<const T*>(p.cs_in) + chan * 3 : nullptr;
+    auto main_loop = [&](auto structured_tag, const float2* a2) {
 #pragma unroll 1
-    for (int64_t k = 0; k < ntiles; ++k) {
-        cp_async_wait<STAGES - 2>();
-        __syncthreads();
-        unsigned char* st = smem + (k % STAGES) * stageB;
-        if (t_begin == 0 && k == 0 && j == 0 && cl < p.octets * 8) {
-            // left context of token 0: the carried conv window (zeros if none)
-            T* xs = reinterpret_cast<T*>(st);
+        for (int64_t k = 0; k < ntiles; ++k) {
+            cp_async_wait<STAGES - 2>();
+            __syncthreads();
+            unsigned char* st = smem + (k % STAGES) * stageB;
+            if (t_begin == 0 && k == 0 && cl < p.octets * 8) {
+                // left context of token 0: the carried conv window (zeros if none)
+                T* xs = reinterpret_cast<T*>(st);
 #pragma unroll
-            for (int q = 0; q < kHalo; ++q)
-                xs[q * rs + cl] = (active && csi) ? csi[q] : A_::from_f32(0.f);
-        }
-        // B (and C) of this tile -> fp32, permuted to [r][B|C][lane j][i], B scaled
-        {
-            const T* bs = reinterpret_cast<const T*>(st + offBC);
-            for (int i = tid; i < TILE * 16 * kBC; i += nthreads) {
-                const int r = i / (16 * kBC);
-                const int e = i - r * 16 * kBC;
-                const int which = e >> 4;
-                const int n = e & 15;
-                float v = A_::to_f32(bs[which * TILE * 16 + r * 16 + n]);
-                if (which == 0) v *= M::step_scale;
-                const int jj = n % LPC, ii = n / LPC;      // lane class, state within lane
-                bcf[jj * JSTRIDE + ((ii >> 1) * TILE + r) * 4 + which * 2 + (ii & 1)] = v;
+                for (int q = 0; q < kHalo; ++q) {
+                    xs[q * rs + cl] = csi ? csi[q] : A_::from_f32(0.f);
+                    xs[q * rs + cl + 1] = csi ? csi[3 + q] : A_::from_f32(0.f);
+                }
             }
-        }
-        load_tile(k + STAGES - 1);
-        __syncthreads();
-        const int64_t tile_t0 = t_begin + k * TILE;
-        if (structured) {
-MM_PRAGMA(unroll MM_SUBTILE_UNROLL)
+            // B (and C) of this tile -> fp32, each value duplicated, B scaled
+            {
+                const T* bs = reinterpret_cast<const T*>(st + offBC);
+                for (int i = tid; i < TILE * 16 * kBC; i += nthreads) {
+                    const int r = i / (16 * kBC);
+                    const int e = i - r * 16 * kBC;               // 0..15 B, 16..31 C
+                    float v = A_::to_f32(bs[(e >> 4) * TILE * 16 + r * 16 + (e & 15)]);
+                    if (e < 16) v *= M::step_scale;
+                    *reinterpret_cast<float2*>(bcf + r * 64 + 2 * e) = f2(v, v);
+                }
+            }
+            load_tile(k + STAGES - 1);
+            __syncthreads();
+            const int64_t tile_t0 = t_begin + k * TILE;
+#pragma unroll 1
             for (int r0 = 0; r0 < TILE; r0 += SUB)
-                run_sub(st, r0, tile_t0 + r0, std::true_type{});
-        } else {
-MM_PRAGMA(unroll MM_SUBTILE_UNROLL)
-            for (int r0 = 0; r0 < TILE; r0 += SUB)
-                run_sub(st, r0, tile_t0 + r0, std::false_type{});
+                run_sub(st, r0, tile_t0 + r0, structured_tag, a2);
         }
+    };
+    if (structured) {
+        main_loop(std::true_type{}, nullptr);
+    } else {
+        float2 a2[16];
+#pragma unroll
+        for (int n = 0; n < 16; ++n) a2[n] = active ? f2(arow0[n], arow1[n]) : f2(0.f, 0.f);
+        main_loop(std::false_type{}, a2);
     }
     cp_async_wait<0>();
 
     // ---------------------------------------------------------- carried state out
     if constexpr (SUMMARY) {
-#pragma unroll
-        for (int bit = LPC / 2; bit >= 1; bit >>= 1) lsum += __shfl_xor_sync(kFull, lsum, bit);
         if (active) {
             const int64_t stride = static_cast<int64_t>(p.batch) * D;
             float* e = p.ws_state + (chunk * stride + chan) * 16;
 #pragma unroll
-            for (int i = 0; i < NS; ++i) e[j + LPC * i] = h[i];
-            if (j == 0) p.ws_lsum[chunk * stride + chan] = lsum;
+            for (int n = 0; n < 16; ++n) { e[n] = h[n].x; e[16 + n] = h[n].y; }
+            *reinterpret_cast<float2*>(p.ws_lsum + chunk * stride + chan) = lsum;
         }
     } else if (active && chunk == p.n_chunks - 1) {
         float* hl = p.h_last + chan * 16;
 #pragma unroll
-        for (int i = 0; i < NS; ++i) hl[j + LPC * i] = h[i];
-        if (j == 0) {
-            // the last 3 raw x, shifted in from the incoming window when L < 3
-            T* cso = static_cast<T*>(p.cs_out) + chan * 3;
+        for (int n = 0; n < 16; ++n) { hl[n] = h[n].x; hl[16 + n] = h[n].y; }
+        // the last 3 raw x of both channels, shifted in from the incoming window when L < 3
+        T* cso = static_cast<T*>(p.cs_out) + chan * 3;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
 #pragma unroll
             for (int q = 0; q < 3; ++q) {
                 const int64_t tpos = L - 3 + q;
                 T v;
-                if (tpos >= 0) v = xz[(seq_row0 + tpos) * 2 * D + d];
-                else v = csi ? csi[tpos + 3] : A_::from_f32(0.f);
-                cso[q] = v;
+                if (tpos >= 0) v = xz[(seq_row0 + tpos) * 2 * D + d + c];
+                else v = csi ? csi[3 * c + tpos + 3] : A_::from_f32(0.f);
+                cso[3 * c + q] = v;
             }
         }
     }
