@@ -60,7 +60,8 @@ typedef enum mm_status {
     MM_ERR_UNSUPPORTED = 6, /* d_state != 16, d_conv != 4, or d_inner % 8 != 0       */
     MM_ERR_CUDA = 7,        /* the CUDA runtime reported an error at launch          */
     MM_ERR_DEVICE = 8,      /* no usable sm_100 device is current                    */
-    MM_ERR_WORKSPACE = 9    /* workspace missing or smaller than the size this call needs */
+    MM_ERR_WORKSPACE = 9,   /* workspace missing or smaller than the size this call needs */
+    MM_ERR_SCRATCH_LIMIT = 10 /* mamba_mixer_fwd_noalloc: sizes need more than its built-in scratch */
 } mm_status;
 
 typedef enum mm_dtype {
@@ -113,6 +114,42 @@ mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv
                           int64_t batch, int64_t seqlen, int64_t d_inner,
                           int64_t d_state, int64_t d_conv, mm_dtype act,
                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * mamba_mixer_fwd without a workspace argument, for callers that cannot
+ * allocate device memory.  No counterpart in the paper: it is a calling
+ * convenience of this library, not part of the method.
+ *
+ * Who needs it: a host program that links only this C library and has no
+ * device allocator of its own, and serving processes whose device memory is
+ * planned in full before they start (weights, per-sequence SSM and conv
+ * state) and that do not allocate on the request path.  Both can still pass
+ * the inputs and outputs they already own; only the forward's scratch (the
+ * carried chunk states of a time-split sequence) has nowhere to come from.
+ *
+ * The scratch is a fixed MAMBA_MIXER_NOALLOC_SCRATCH_BYTES array in the
+ * library's device image: every GPU that loads the library holds it until
+ * the process exits.  Sizes whose scratch would not fit (see
+ * mamba_mixer_workspace_size) return MM_ERR_SCRATCH_LIMIT before anything is
+ * launched; with the default launch plan every size fits.
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current) and keeps it; make that first call before any stream
+ * capture.  All calls on a device share the one array and nothing in it is
+ * kept between calls (each call writes every scratch value it later reads),
+ * but calls that overlap on the GPU -- on different streams, or from
+ * different threads -- race on it and give wrong results: serialise them.
+ * Arguments, outputs, validation and errors are otherwise those of
+ * mamba_mixer_fwd.
+ */
+#define MAMBA_MIXER_NOALLOC_SCRATCH_BYTES (8u << 20)
+mm_status mamba_mixer_fwd_noalloc(const void* xz, const float* conv_w, const float* conv_b,
+                                  const void* dt, const float* dt_bias, const float* A,
+                                  const void* Bm, const void* Cm, const float* Dskip,
+                                  const float* h0, const void* conv_state_in,
+                                  void* y, float* h_last, void* conv_state_out,
+                                  int64_t batch, int64_t seqlen, int64_t d_inner,
+                                  int64_t d_state, int64_t d_conv, mm_dtype act, void* stream);
 
 /* Bytes of device scratch mamba_mixer_fwd needs for these sizes (0 = none).
  * A pure function of its arguments (and of the MAMBA_MIXER_CHUNKS tuning

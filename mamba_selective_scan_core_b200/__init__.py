@@ -14,7 +14,7 @@ import ctypes
 import os
 
 __all__ = [
-    "MM_F32", "MM_BF16", "MixerError", "lib", "library_path", "mixer_fwd", "state_update",
+    "MM_F32", "MM_BF16", "MixerError", "lib", "library_path", "mixer_fwd", "mixer_fwd_noalloc", "state_update",
     "workspace_size", "status_string", "abi_version", "EXPORTED_SYMBOLS",
 ]
 
@@ -27,6 +27,7 @@ _lib = None
 
 EXPORTED_SYMBOLS = (
     "mamba_mixer_fwd",
+    "mamba_mixer_fwd_noalloc",
     "mamba_mixer_workspace_size",
     "mamba_state_update",
     "mamba_status_string",
@@ -51,6 +52,8 @@ def _declare(L):
     I64 = ctypes.c_int64
     L.mamba_mixer_fwd.restype = ctypes.c_int
     L.mamba_mixer_fwd.argtypes = [P] * 14 + [I64] * 5 + [ctypes.c_int, P, ctypes.c_size_t, P]
+    L.mamba_mixer_fwd_noalloc.restype = ctypes.c_int
+    L.mamba_mixer_fwd_noalloc.argtypes = [P] * 14 + [I64] * 5 + [ctypes.c_int, P]
     L.mamba_mixer_workspace_size.restype = ctypes.c_size_t
     L.mamba_mixer_workspace_size.argtypes = [I64] * 5 + [ctypes.c_int]
     L.mamba_state_update.restype = ctypes.c_int
@@ -170,6 +173,39 @@ def mixer_fwd(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, conv_s
             Bsz, L, D, N, W, act, _ptr(workspace) if ws_bytes else None, ws_bytes, _stream_handle(stream))
     if st != 0:
         raise MixerError(st, "mamba_mixer_fwd")
+    return y, h_last, conv_state_out
+
+
+def mixer_fwd_noalloc(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, conv_state_in=None, *,
+                      y, h_last, conv_state_out, stream=None):
+    """mixer_fwd through the entry point that takes no workspace and allocates
+    nothing (its scratch is a fixed array inside the library).  The caller
+    passes the output tensors; calls that overlap on the GPU race on the
+    shared scratch, so serialise them."""
+    import torch
+
+    act = _act_code(xz.dtype)
+    Bsz, L, twoD = xz.shape
+    D = twoD // 2
+    N = A.shape[-1]
+    W = conv_w.shape[-1]
+    dev = xz.device
+    f32 = torch.float32
+    for t, name, dtype, shape in (
+            (xz, "xz", xz.dtype, (Bsz, L, 2 * D)), (conv_w, "conv_w", f32, (D, W)), (conv_b, "conv_b", f32, (D,)),
+            (dt, "dt", xz.dtype, (Bsz, L, D)), (dt_bias, "dt_bias", f32, (D,)), (A, "A", f32, (D, N)),
+            (Bm, "Bm", xz.dtype, (Bsz, L, N)), (Cm, "Cm", xz.dtype, (Bsz, L, N)), (Dskip, "Dskip", f32, (D,)),
+            (h0, "h0", f32, (Bsz, D, N)), (conv_state_in, "conv_state_in", xz.dtype, (Bsz, D, W - 1)),
+            (y, "y", xz.dtype, (Bsz, L, D)), (h_last, "h_last", f32, (Bsz, D, N)),
+            (conv_state_out, "conv_state_out", xz.dtype, (Bsz, D, W - 1))):
+        _check(t, name, dtype, shape, dev)
+    with torch.cuda.device(dev):
+        st = lib().mamba_mixer_fwd_noalloc(
+            _ptr(xz), _ptr(conv_w), _ptr(conv_b), _ptr(dt), _ptr(dt_bias), _ptr(A), _ptr(Bm), _ptr(Cm),
+            _ptr(Dskip), _ptr(h0), _ptr(conv_state_in), _ptr(y), _ptr(h_last), _ptr(conv_state_out),
+            Bsz, L, D, N, W, act, _stream_handle(stream))
+    if st != 0:
+        raise MixerError(st, "mamba_mixer_fwd_noalloc")
     return y, h_last, conv_state_out
 
 

@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "mamba_mixer.h"
 #include "mixer_decode.cuh"
@@ -176,6 +177,38 @@ cudaError_t dispatch_prefill(PrefillParams p, int64_t batch, const FwdPlan& pl, 
 
 }  // namespace
 
+// Scratch of mamba_mixer_fwd_noalloc: one fixed array per device in the
+// library's device image, for callers that cannot allocate.  Host code only
+// ever passes its device address (looked up per device, below) to kernels.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MAMBA_MIXER_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 256;
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (with that device current) and kept.
+mm_status noalloc_scratch(void** out) {
+    static std::mutex mu;
+    static void* addr[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return MM_ERR_DEVICE; }
+    if (dev < 0 || dev >= kMaxDevices) return MM_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return MM_ERR_CUDA;
+        }
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return MM_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int mamba_mixer_abi_version(void) { return MAMBA_MIXER_ABI_VERSION; }
@@ -192,6 +225,9 @@ const char* mamba_status_string(mm_status status) {
         case MM_ERR_CUDA: return "CUDA runtime error at launch";
         case MM_ERR_DEVICE: return "no usable sm_100 device is current";
         case MM_ERR_WORKSPACE: return "workspace missing or smaller than mamba_mixer_workspace_size()";
+        case MM_ERR_SCRATCH_LIMIT:
+            return "sizes need more scratch than mamba_mixer_fwd_noalloc's built-in 8 MiB; pass a workspace to "
+                   "mamba_mixer_fwd instead";
     }
     return "unknown status";
 }
@@ -331,6 +367,25 @@ mm_status mamba_state_update(const void* x, const void* z, const void* dt,
     }
     if (cudaGetLastError() != cudaSuccess) return MM_ERR_CUDA;
     return MM_OK;
+}
+
+mm_status mamba_mixer_fwd_noalloc(const void* xz, const float* conv_w, const float* conv_b,
+                                  const void* dt, const float* dt_bias, const float* A,
+                                  const void* Bm, const void* Cm, const float* Dskip,
+                                  const float* h0, const void* conv_state_in,
+                                  void* y, float* h_last, void* conv_state_out,
+                                  int64_t batch, int64_t seqlen, int64_t d_inner,
+                                  int64_t d_state, int64_t d_conv, mm_dtype act, void* stream)
+{
+    const size_t need = mamba_mixer_workspace_size(batch, seqlen, d_inner, d_state, d_conv, act);
+    if (need > MAMBA_MIXER_NOALLOC_SCRATCH_BYTES) return MM_ERR_SCRATCH_LIMIT;
+    void* scratch = nullptr;
+    if (need > 0) {
+        if (mm_status st = noalloc_scratch(&scratch); st != MM_OK) return st;
+    }
+    return mamba_mixer_fwd(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0, conv_state_in, y, h_last,
+                           conv_state_out, batch, seqlen, d_inner, d_state, d_conv, act, scratch,
+                           need > 0 ? MAMBA_MIXER_NOALLOC_SCRATCH_BYTES : 0, stream);
 }
 
 }  // extern "C"

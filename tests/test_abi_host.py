@@ -15,7 +15,7 @@ from mamba_selective_scan_core_b200 import build as mmbuild
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "mamba_mixer.h")
 
-OK, ENULL, ESHAPE, EALIGN, EDTYPE, EALIAS, EUNSUP, ECUDA, EDEVICE, EWORKSPACE = range(10)
+OK, ENULL, ESHAPE, EALIGN, EDTYPE, EALIAS, EUNSUP, ECUDA, EDEVICE, EWORKSPACE, ESCRATCH = range(11)
 
 
 @pytest.fixture(scope="module")
@@ -48,7 +48,7 @@ def test_exported_symbols_are_c_linkage():
 
 def test_version_and_strings(L):
     assert mm.abi_version() == 1
-    for code in range(10):
+    for code in range(11):
         s = mm.status_string(code)
         assert s and s != "unknown status"
     assert mm.status_string(99) == "unknown status"
@@ -240,3 +240,22 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(mm, "library_path", lambda: str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         mm.lib()
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch(L, monkeypatch):
+    # 16 forced time chunks over 65536 channels need 15 * 65536 * 68 bytes of
+    # scratch, more than the built-in 8 MiB: rejected before any launch
+    monkeypatch.setenv("MAMBA_MIXER_CHUNKS", "16")
+    args = fwd_args(B=8, Lq=4096, D=8192)
+    assert mm.workspace_size(8, 4096, 8192) > 8 << 20
+    noalloc = args[:-3] + [args[-1]]          # same arguments without workspace and its size
+    assert L.mamba_mixer_fwd_noalloc(*noalloc) == ESCRATCH
+
+
+def test_noalloc_validates_like_the_forward(L):
+    args = fwd_args()
+    noalloc = args[:-3] + [args[-1]]
+    bad = list(noalloc)
+    bad[0] = None                             # xz
+    assert L.mamba_mixer_fwd_noalloc(*bad) == ENULL
+    assert L.mamba_mixer_fwd_noalloc(*noalloc) in (EDEVICE, OK, ECUDA)
