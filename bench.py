@@ -80,9 +80,12 @@ def _measured_peaks():
 
 
 def _kernel_source_sha():
+    """Hash of the device code (the kernel headers) the traffic figures depend on."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mamba_selective_scan_core_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
+        if not name.endswith(".cuh"):
+            continue
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -256,7 +259,7 @@ def run_gpu(args):
     alu_peak = SMS * FP32_LANES_PER_SM * sm_max * 1e6 / 1e12       # T fp32 lane-ops/s
     alu_ops = FWD_FP32_OPS_PER_TOKEN_CHANNEL * tokens * D
     alu_ach = alu_ops / avg_launch_s / 1e12
-    traffic = _ncu_traffic("mixer_fwd_kernel/jamba_prefill")
+    traffic = _ncu_traffic("mixer_fwd/jamba_prefill")
     hbm_part = {"bound": "hbm", "achieved": round(hbm_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(hbm_gbs / hbm_peak, 4), "traffic": traffic,
                 "algorithmic_bytes": nbytes, "peak_source": hbm_src}
