@@ -465,6 +465,42 @@ def run_reference(args):
     return line, world
 
 
+def run_only(args):
+    """One kernel's warm-up and timed loop on the benchmark's inputs, for
+    profiler captures (ncu -k ... -s ... -c ...); prints the mean time only."""
+    import mamba_selective_scan_core_b200 as mm
+
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    mm.lib()
+    if args.only == "forward":
+        cfg = PREFILL
+        d = {k: (v.cuda() if v is not None else None) for k, v in make_mixer_inputs(cfg).items()}
+        out = (torch.empty((cfg.batch, cfg.seqlen, cfg.d_inner), dtype=torch.bfloat16, device="cuda"),
+               torch.empty((cfg.batch, cfg.d_inner, 16), device="cuda"),
+               torch.empty((cfg.batch, cfg.d_inner, 3), dtype=torch.bfloat16, device="cuda"))
+        step = lambda: _fwd_call(mm, d, out)  # noqa: E731
+    else:
+        cfg = DECODE
+        nl = args.decode_layers or cfg.layers
+        from workloads import make_decode_inputs_custom
+
+        d = {k: (v.cuda() if v is not None else None)
+             for k, v in make_decode_inputs_custom(nl, cfg.batch, cfg.d_inner, seed=cfg.seed).items()}
+        y = torch.empty((nl, cfg.batch, cfg.d_inner), dtype=torch.bfloat16, device="cuda")
+        step = lambda: mm.state_update(d["x"], d["z"], d["dt"], d["conv_w"], d["conv_b"], d["dt_bias"],  # noqa: E731
+                                       d["Dskip"], d["A"], d["Bm"], d["Cm"], d["ssm_state"], d["conv_state"], y=y)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    print(f"{args.only}: {a.elapsed_time(b) / max(1, args.steps) * 1e3:.1f} us per call", flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -472,9 +508,16 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["forward", "decode"], default=None,
+                    help="run one kernel's timed loop only (for profiler captures); prints no JSON line")
+    ap.add_argument("--decode-layers", type=int, default=None,
+                    help="with --only decode: stacked layers (default: the workload's 28)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.only:
+        run_only(args)
+        return
     if args.impl == "reference":
         line, world = run_reference(args)
     else:
