@@ -61,7 +61,8 @@ typedef enum mm_status {
     MM_ERR_CUDA = 7,        /* the CUDA runtime reported an error at launch          */
     MM_ERR_DEVICE = 8,      /* no usable sm_100 device is current                    */
     MM_ERR_WORKSPACE = 9,   /* workspace missing or smaller than the size this call needs */
-    MM_ERR_SCRATCH_LIMIT = 10 /* mamba_mixer_fwd_noalloc: sizes need more than its built-in scratch */
+    MM_ERR_SCRATCH_LIMIT = 10, /* mamba_mixer_fwd_noalloc: sizes need more than its built-in scratch */
+    MM_ERR_TIMEOUT = 11     /* mamba_mixer_fault_status: a kernel gave up waiting for its copies */
 } mm_status;
 
 typedef enum mm_dtype {
@@ -185,6 +186,18 @@ mm_status mamba_state_update(const void* x, const void* z, const void* dt,
                              float* ssm_state, void* conv_state, void* y,
                              int64_t n_layers, int64_t batch, int64_t d_inner,
                              int64_t d_state, int64_t d_conv, mm_dtype act, void* stream);
+
+/*
+ * Device fault word of the library on the current device.  Every wait of a
+ * kernel on its own bulk copies is bounded; a kernel that gives up (a copy
+ * that never lands -- not expected on working hardware) sets this word,
+ * skips its remaining work and exits instead of hanging.  Returns
+ * MM_ERR_TIMEOUT if the word is set, MM_OK if not; clears it when `reset` is
+ * non-zero.  Synchronises with the device (reads device memory).
+ * Test hook: the environment variable MAMBA_MIXER_WAIT_LIMIT sets the number
+ * of wait attempts (0 makes the forward give up at once).
+ */
+mm_status mamba_mixer_fault_status(int reset);
 
 /* A static, human-readable name for a status code. */
 const char* mamba_status_string(mm_status status);

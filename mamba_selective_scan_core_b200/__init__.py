@@ -15,7 +15,7 @@ import os
 
 __all__ = [
     "MM_F32", "MM_BF16", "MixerError", "lib", "library_path", "mixer_fwd", "mixer_fwd_noalloc", "state_update",
-    "workspace_size", "status_string", "abi_version", "EXPORTED_SYMBOLS",
+    "workspace_size", "status_string", "abi_version", "fault_status", "EXPORTED_SYMBOLS",
 ]
 
 MM_F32 = 0
@@ -32,6 +32,7 @@ EXPORTED_SYMBOLS = (
     "mamba_state_update",
     "mamba_status_string",
     "mamba_mixer_abi_version",
+    "mamba_mixer_fault_status",
 )
 
 
@@ -62,6 +63,8 @@ def _declare(L):
     L.mamba_status_string.argtypes = [ctypes.c_int]
     L.mamba_mixer_abi_version.restype = ctypes.c_int
     L.mamba_mixer_abi_version.argtypes = []
+    L.mamba_mixer_fault_status.restype = ctypes.c_int
+    L.mamba_mixer_fault_status.argtypes = [ctypes.c_int]
     return L
 
 
@@ -84,6 +87,12 @@ def status_string(status: int) -> str:
 
 def abi_version() -> int:
     return int(lib().mamba_mixer_abi_version())
+
+
+def fault_status(reset: bool = False) -> int:
+    """0 if no kernel gave up waiting for its bulk copies on the current
+    device, else MM_ERR_TIMEOUT (11); clears the flag when reset is set."""
+    return int(lib().mamba_mixer_fault_status(1 if reset else 0))
 
 
 def _act_code(dtype):

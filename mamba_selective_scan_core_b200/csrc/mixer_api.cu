@@ -2,6 +2,7 @@
 // validation (before anything is launched), launch-shape selection and the
 // launches themselves.  No allocation, no global state.
 #include <algorithm>
+#include <cudaTypedefs.h>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -80,6 +81,18 @@ int env_int(const char* name, int lo, int hi) {
 
 // Time chunks: the fewest that bring the resident warps (two channels per
 // thread) to ~80% of what the SMs hold.
+// Tries per wait on a bulk copy (each try waits a bounded time in hardware):
+// about a second by default; MAMBA_MIXER_WAIT_LIMIT overrides it (tests use 0
+// to make the wait give up at once).
+unsigned copy_wait_limit() {
+    if (const char* e = std::getenv("MAMBA_MIXER_WAIT_LIMIT")) {
+        char* end = nullptr;
+        const long v = std::strtol(e, &end, 10);
+        if (end != e && v >= 0 && v <= (1L << 30)) return static_cast<unsigned>(v);
+    }
+    return 1u << 20;
+}
+
 FwdPlan plan_fwd(int64_t batch, int64_t seqlen, int64_t d_inner) {
     FwdPlan pl;
     const int64_t warps = std::max<int64_t>(1, batch * d_inner / 2 / 32);
@@ -102,14 +115,67 @@ FwdPlan plan_fwd(int64_t batch, int64_t seqlen, int64_t d_inner) {
     return pl;
 }
 
+// ---------------------------------------------------------------- tensor maps
+// The driver's tensor-map encoder, fetched through the runtime (no link
+// against libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+struct TensorMaps {
+    CUtensorMap x, z, dt, b, c;
+};
+
+// 3-D map over a [batch][rows][cols] tensor with a [1][box_rows][box_cols] box.
+bool encode_3d(CUtensorMap* m, const void* base, bool bf16, int64_t cols, int64_t rows, int64_t batch,
+               int box_cols, int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const int64_t es = bf16 ? 2 : 4;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                                static_cast<cuuint64_t>(batch)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols * es), static_cast<cuuint64_t>(rows * cols * es)};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T>
+bool make_maps(const PrefillParams& p, int64_t batch, TensorMaps* m) {
+    std::memset(m, 0, sizeof(*m));
+    if (p.L == 0) return true;                 // no tiles: the maps are never read
+    constexpr bool bf16 = sizeof(T) == 2;
+    const int boxc = p.octets * 8;
+    return encode_3d(&m->x, p.xz, bf16, 2 * int64_t(p.D), p.L, batch, boxc, kTile + mm::kHalo) &&
+           encode_3d(&m->z, p.xz, bf16, 2 * int64_t(p.D), p.L, batch, boxc, kTile) &&
+           encode_3d(&m->dt, p.dt, bf16, p.D, p.L, batch, boxc, kTile) &&
+           encode_3d(&m->b, p.Bm, bf16, 16, p.L, batch, 16, kTile) &&
+           encode_3d(&m->c, p.Cm, bf16, 16, p.L, batch, 16, kTile);
+}
+
 template <typename T, typename M, int STAGES, bool SUMMARY>
 cudaError_t launch_prefill(const PrefillParams& p, int64_t batch, int chunks, int threads, cudaStream_t s) {
     auto kern = mm::mixer_fwd_kernel<T, M, kTile, STAGES, SUMMARY>;
+    TensorMaps maps;
+    if (!make_maps<T>(p, batch, &maps)) return cudaErrorInvalidValue;
     const int smem = PrefillLayout<T>::smem_bytes(kTile, STAGES, p.octets);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const dim3 grid(static_cast<unsigned>(batch * p.ctas_per_seq), static_cast<unsigned>(chunks));
-    kern<<<grid, threads, smem, s>>>(p);
+    kern<<<grid, threads, smem, s>>>(p, maps.x, maps.z, maps.dt, maps.b, maps.c);
     return cudaGetLastError();
 }
 
@@ -131,7 +197,8 @@ int ring_depth(int oct) {
 template <typename T>
 int shape_ctas(PrefillParams& p, int64_t batch, int64_t chunks, int sm_count, int* threads) {
     const int64_t octets_per_seq = p.D / 8;
-    const int max_oct = static_cast<int>(std::min<int64_t>(kMaxThreads / 4, octets_per_seq));
+    // a copy box spans at most 256 channels: 32 octets
+    const int max_oct = static_cast<int>(std::min<int64_t>({kMaxThreads / 4, 32, octets_per_seq}));
     int64_t best_waves = INT64_MAX;
     int best = 1, best_stages = 2;
     for (int oct = 1; oct <= max_oct; ++oct) {
@@ -225,11 +292,22 @@ const char* mamba_status_string(mm_status status) {
         case MM_ERR_CUDA: return "CUDA runtime error at launch";
         case MM_ERR_DEVICE: return "no usable sm_100 device is current";
         case MM_ERR_WORKSPACE: return "workspace missing or smaller than mamba_mixer_workspace_size()";
+        case MM_ERR_TIMEOUT: return "a kernel gave up waiting for its bulk copies (see mamba_mixer_fault_status)";
         case MM_ERR_SCRATCH_LIMIT:
             return "sizes need more scratch than mamba_mixer_fwd_noalloc's built-in 8 MiB; pass a workspace to "
                    "mamba_mixer_fwd instead";
     }
     return "unknown status";
+}
+
+mm_status mamba_mixer_fault_status(int reset) {
+    unsigned v = 0;
+    if (cudaMemcpyFromSymbol(&v, mm::g_mm_fault, sizeof(v)) != cudaSuccess) { cudaGetLastError(); return MM_ERR_CUDA; }
+    if (reset && v) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(mm::g_mm_fault, &zero, sizeof(zero)) != cudaSuccess) { cudaGetLastError(); return MM_ERR_CUDA; }
+    }
+    return v ? MM_ERR_TIMEOUT : MM_OK;
 }
 
 size_t mamba_mixer_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state,
@@ -301,6 +379,7 @@ mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv
     p.L = seqlen;
     p.D = static_cast<int>(d_inner);
     p.batch = static_cast<int>(batch);
+    p.wait_limit = copy_wait_limit();
     p.ws_state = static_cast<float*>(workspace);
     p.ws_lsum = pl.ws_bytes ? p.ws_state + static_cast<int64_t>(pl.chunks - 1) * batch * d_inner * 16 : nullptr;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

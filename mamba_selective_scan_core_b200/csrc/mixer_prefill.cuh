@@ -43,12 +43,16 @@
 // (the only serial dependency is one FMA per token on each state; decay
 // powers by repeated squaring), C. skip, gate and store.
 //
-// Data movement: each CTA owns a contiguous block of channels of one sequence
-// and one time chunk, and walks it in tiles of TILE tokens.  x (with 3 rows
-// of left context), z, dt rows of the block and the B_t/C_t rows are staged
-// in shared memory by cp.async 16-byte copies in a STAGES-deep ring (rows
-// outside the chunk are zero-filled; the left context of token 0 comes from
-// the carried conv window).
+// Data movement: each CTA owns a contiguous block of up to 256 channels of
+// one sequence and one time chunk, and walks it in tiles of TILE tokens.  One
+// thread stages each tile with five 3-D tiled bulk tensor copies (TMA): x
+// with 3 rows of left context, z, dt, and the B_t/C_t rows, into a
+// STAGES-deep ring of shared-memory buffers, each completing on its own
+// mbarrier.  Rows before token 0 or past the sequence are zero-filled by the
+// copy engine; the left context of token 0 is then overwritten with the
+// carried conv window.  Every wait on a copy is bounded: a copy that never
+// lands sets a fault word the host can read (mamba_mixer_fault_status)
+// instead of hanging the GPU.
 #pragma once
 
 #include <type_traits>
@@ -85,36 +89,28 @@ struct PrefillParams {
     float* ws_state;    // [K-1][batch][D][16]: end state of chunk c run from zero
     float* ws_lsum;     // [K-1][batch][D]:     sum over chunk c of the step size l
     int batch;
+    unsigned wait_limit;  // tries per wait on a bulk copy before giving up (fault)
 };
 
 constexpr int kHalo = 3;   // conv left context rows (d_conv - 1)
 
 template <typename T>
 struct PrefillLayout {
-    // one staged tile for a CTA of `octets` channel octets:
+    // one staged tile for a CTA of `octets` channel octets, each region
+    // 128-byte aligned:
     //   x [TILE+3][ch], z [TILE][ch], dt [TILE][ch], B [TILE][16], C [TILE][16]
+    __host__ __device__ static constexpr int a128(int b) { return (b + 127) & ~127; }
     __host__ __device__ static constexpr int row_bytes(int octets) { return octets * 8 * static_cast<int>(sizeof(T)); }
-    __host__ __device__ static constexpr int bc_row_bytes() { return 16 * static_cast<int>(sizeof(T)); }
+    __host__ __device__ static constexpr int x_bytes(int tile, int octets) { return a128((tile + kHalo) * row_bytes(octets)); }
+    __host__ __device__ static constexpr int zdt_bytes(int tile, int octets) { return a128(tile * row_bytes(octets)); }
+    __host__ __device__ static constexpr int bc_bytes(int tile) { return a128(tile * 16 * static_cast<int>(sizeof(T))); }
     __host__ __device__ static int stage_bytes(int tile, int octets) {
-        return (3 * tile + kHalo) * row_bytes(octets) + 2 * tile * bc_row_bytes();
+        return x_bytes(tile, octets) + 2 * zdt_bytes(tile, octets) + 2 * bc_bytes(tile);
     }
-    // plus the tile's B/C in fp32, each value duplicated: [token][B0 B0 B1 B1 .. C15 C15]
+    // plus the tile's B/C in fp32, each value duplicated ([token][B0 B0 .. C15
+    // C15]), and one mbarrier per stage
     __host__ __device__ static int smem_bytes(int tile, int stages, int octets) {
-        return stages * stage_bytes(tile, octets) + tile * 64 * 4;
-    }
-};
-
-// Walk the chunk indices i = tid, tid + nthreads, ... of a [rows][cols] grid
-// without a division per step.
-struct GridWalk {
-    int r, c, dr, dc, cols;
-    __device__ GridWalk(int tid, int nthreads, int cols_) : cols(cols_) {
-        r = tid / cols; c = tid - r * cols;
-        dr = nthreads / cols; dc = nthreads - dr * cols;
-    }
-    __device__ void next() {
-        r += dr; c += dc;
-        if (c >= cols) { c -= cols; ++r; }
+        return stages * stage_bytes(tile, octets) + tile * 64 * 4 + stages * 8;
     }
 };
 
@@ -153,7 +149,9 @@ __device__ __forceinline__ float2 decay2(float2 l, float2 a) {
 // SUMMARY = false: the full fused forward over one chunk.
 template <typename T, typename M, int TILE, int STAGES, bool SUMMARY>
 __global__ void __launch_bounds__(256, 1)
-mixer_fwd_kernel(const PrefillParams p)
+mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x,
+                 const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_dt,
+                 const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c)
 {
     constexpr int SUB = MM_SUB;
     static_assert(TILE % SUB == 0, "tile");
@@ -161,7 +159,7 @@ mixer_fwd_kernel(const PrefillParams p)
     using A_ = Act<T>;
     using P_ = Pair<T>;
 
-    extern __shared__ __align__(16) unsigned char smem[];
+    extern __shared__ __align__(128) unsigned char smem[];
 
     const int tid = threadIdx.x;
     const int seq = blockIdx.x / p.ctas_per_seq;
@@ -179,13 +177,14 @@ mixer_fwd_kernel(const PrefillParams p)
     const int64_t t_begin = static_cast<int64_t>(chunk) * p.chunk_len;
     const int64_t t_end = min(L, t_begin + p.chunk_len);
 
-    const int rowB = PrefillLayout<T>::row_bytes(p.octets);
-    const int rs = p.octets * 8;                 // elements per staged row
-    const int stageB = PrefillLayout<T>::stage_bytes(TILE, p.octets);
-    const int offZ = (TILE + kHalo) * rowB;
-    const int offDT = offZ + TILE * rowB;
-    const int offBC = offDT + TILE * rowB;
+    using Lay = PrefillLayout<T>;
+    const int rs = p.octets * 8;                 // elements per staged row (the copy box width)
+    const int stageB = Lay::stage_bytes(TILE, p.octets);
+    const int offZ = Lay::x_bytes(TILE, p.octets);
+    const int offDT = offZ + Lay::zdt_bytes(TILE, p.octets);
+    const int offBC = offDT + Lay::zdt_bytes(TILE, p.octets);
     float* bcf = reinterpret_cast<float*>(smem + STAGES * stageB);   // [TILE][64]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * stageB + TILE * 64 * 4);
 
     const T* xz = static_cast<const T*>(p.xz);
     const T* dtg = static_cast<const T*>(p.dt);
@@ -195,46 +194,27 @@ mixer_fwd_kernel(const PrefillParams p)
     const int64_t chan = static_cast<int64_t>(seq) * D + d;           // (sequence, first channel) row
 
     // ---------------------------------------------------------- tile loader
-    constexpr int kEPC = 16 / sizeof(T);              // elements per 16-byte chunk
-    const int cpr = rowB / 16;                        // chunks per x/z/dt row
-    constexpr int bcr = 16 * sizeof(T) / 16;          // chunks per B or C row
     const int64_t ntiles = t_end > t_begin ? (t_end - t_begin + TILE - 1) / TILE : 0;
-    constexpr int kZDT = SUMMARY ? 1 : 2;             // the summary pass needs dt but not z
-    constexpr int kBC = SUMMARY ? 1 : 2;              // ... and B but not C
+    constexpr int kBC = SUMMARY ? 1 : 2;              // the summary pass needs B but not C (nor z)
+    const unsigned rowb = static_cast<unsigned>(rs * sizeof(T));
+    const unsigned stage_tx = (TILE + kHalo) * rowb + TILE * rowb * (SUMMARY ? 1 : 2) +
+                              kBC * TILE * 16 * static_cast<unsigned>(sizeof(T));
 
-    auto load_tile = [&](int64_t k) {
-        if (k < ntiles) {
-            unsigned char* st = smem + (k % STAGES) * stageB;
-            const int64_t tbase = t_begin + k * TILE;
-            // x with 3 rows of left context: staged row rho holds token tbase - 3 + rho
-            for (GridWalk g(tid, nthreads, cpr); g.r < TILE + kHalo; g.next()) {
-                const int64_t t = tbase - kHalo + g.r;
-                const bool ok = t >= 0 && t < t_end && g.c * kEPC < nch;
-                const T* src = xz + (seq_row0 + (ok ? t : 0)) * 2 * D + d0 + g.c * kEPC;
-                cp_async16(st + g.r * rowB + g.c * 16, ok ? src : p.xz, ok ? 16u : 0u);
-            }
-            // dt (and z for the full pass)
-            for (GridWalk g(tid, nthreads, kZDT * cpr); g.r < TILE; g.next()) {
-                const int64_t t = tbase + g.r;
-                const bool isdt = SUMMARY || g.c >= cpr;
-                const int cc = (SUMMARY || !isdt) ? g.c : g.c - cpr;
-                const bool ok = t < t_end && cc * kEPC < nch;
-                const int64_t row = seq_row0 + (ok ? t : 0);
-                const T* src = isdt ? dtg + row * D + d0 + cc * kEPC : xz + row * 2 * D + D + d0 + cc * kEPC;
-                cp_async16(st + (isdt ? offDT : offZ) + g.r * rowB + cc * 16, ok ? src : p.xz, ok ? 16u : 0u);
-            }
-            // B (and C for the full pass)
-            for (GridWalk g(tid, nthreads, kBC * bcr); g.r < TILE; g.next()) {
-                const int64_t t = tbase + g.r;
-                const bool isC = g.c >= bcr;
-                const int part = isC ? g.c - bcr : g.c;
-                const bool ok = t < t_end;
-                const T* src = (isC ? Cg : Bg) + (seq_row0 + (ok ? t : 0)) * 16 + part * kEPC;
-                cp_async16(st + offBC + (isC ? TILE * 16 * sizeof(T) : 0) + g.r * 16 * sizeof(T) + part * 16,
-                           ok ? src : p.xz, ok ? 16u : 0u);
-            }
+    // one thread: stage tile k (tokens t_begin + k*TILE ..) into ring slot k % STAGES
+    auto issue_tile = [&](int64_t k) {
+        if (k >= ntiles) return;
+        const int slot = static_cast<int>(k % STAGES);
+        unsigned char* st = smem + slot * stageB;
+        const int tb = static_cast<int>(t_begin + k * TILE);
+        uint64_t* bar = &bars[slot];
+        mbar_arrive_expect_tx(bar, stage_tx);
+        tma_load_3d(st, &tm_x, d0, tb - kHalo, seq, bar);
+        tma_load_3d(st + offDT, &tm_dt, d0, tb, seq, bar);
+        tma_load_3d(st + offBC, &tm_b, 0, tb, seq, bar);
+        if constexpr (!SUMMARY) {
+            tma_load_3d(st + offZ, &tm_z, D + d0, tb, seq, bar);
+            tma_load_3d(st + offBC + Lay::bc_bytes(TILE), &tm_c, 0, tb, seq, bar);
         }
-        cp_async_commit();
     };
 
     // ---------------------------------------------------------- per-thread setup
@@ -293,8 +273,16 @@ mixer_fwd_kernel(const PrefillParams p)
     }
 
     // ---------------------------------------------------------- pipeline prologue
+    if (tid == 0) {
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s) mbar_init(&bars[s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
 #pragma unroll 1
-    for (int s = 0; s < STAGES - 1; ++s) load_tile(s);
+        for (int s = 0; s < STAGES - 1; ++s) issue_tile(s);
+    }
 
     T* yg = static_cast<T*>(p.y);
     float2 lsum = f2(0.f, 0.f);           // summary pass: sum of l over the chunk
@@ -378,12 +366,20 @@ mixer_fwd_kernel(const PrefillParams p)
 
     // ---------------------------------------------------------- main loop
     const T* csi = (p.cs_in && active) ? static_cast<const T*>(p.cs_in) + chan * 3 : nullptr;
-    auto main_loop = [&](auto structured_tag, const float2* a2) {
+    // returns false when a copy did not land (fault set; the caller exits)
+    auto main_loop = [&](auto structured_tag, const float2* a2) -> bool {
 #pragma unroll 1
         for (int64_t k = 0; k < ntiles; ++k) {
-            cp_async_wait<STAGES - 2>();
-            __syncthreads();
-            unsigned char* st = smem + (k % STAGES) * stageB;
+            const int slot = static_cast<int>(k % STAGES);
+            const bool landed = mbar_wait_bounded(&bars[slot], static_cast<unsigned>((k / STAGES) & 1), p.wait_limit);
+            if (__syncthreads_or(!landed)) {
+                if (tid == 0) atomicOr(&g_mm_fault, 1u);
+                // let the copies already issued land before the CTA's shared memory goes away
+                for (int64_t j = k; j < min(ntiles, k + STAGES - 1); ++j)
+                    mbar_wait_bounded(&bars[j % STAGES], static_cast<unsigned>((j / STAGES) & 1), 1u << 20);
+                return false;
+            }
+            unsigned char* st = smem + slot * stageB;
             if (t_begin == 0 && k == 0 && cl < p.octets * 8) {
                 // left context of token 0: the carried conv window (zeros if none)
                 T* xs = reinterpret_cast<T*>(st);
@@ -396,31 +392,38 @@ mixer_fwd_kernel(const PrefillParams p)
             // B (and C) of this tile -> fp32, each value duplicated, B scaled
             {
                 const T* bs = reinterpret_cast<const T*>(st + offBC);
+                constexpr int cstride = Lay::bc_bytes(TILE) / static_cast<int>(sizeof(T));   // elements from B to C
                 for (int i = tid; i < TILE * 16 * kBC; i += nthreads) {
                     const int r = i / (16 * kBC);
                     const int e = i - r * 16 * kBC;               // 0..15 B, 16..31 C
-                    float v = A_::to_f32(bs[(e >> 4) * TILE * 16 + r * 16 + (e & 15)]);
+                    float v = A_::to_f32(bs[(e >> 4) * cstride + r * 16 + (e & 15)]);
                     if (e < 16) v *= M::step_scale;
                     *reinterpret_cast<float2*>(bcf + r * 64 + 2 * e) = f2(v, v);
                 }
             }
-            load_tile(k + STAGES - 1);
+            if (tid == 0) {
+                // the slot refilled next held tile k-1, which every thread has finished with
+                fence_proxy_async_smem();
+                issue_tile(k + STAGES - 1);
+            }
             __syncthreads();
             const int64_t tile_t0 = t_begin + k * TILE;
 #pragma unroll 1
             for (int r0 = 0; r0 < TILE; r0 += SUB)
                 run_sub(st, r0, tile_t0 + r0, structured_tag, a2);
         }
+        return true;
     };
+    bool completed;
     if (structured) {
-        main_loop(std::true_type{}, nullptr);
+        completed = main_loop(std::true_type{}, nullptr);
     } else {
         float2 a2[16];
 #pragma unroll
         for (int n = 0; n < 16; ++n) a2[n] = active ? f2(arow0[n], arow1[n]) : f2(0.f, 0.f);
-        main_loop(std::false_type{}, a2);
+        completed = main_loop(std::false_type{}, a2);
     }
-    cp_async_wait<0>();
+    if (!completed) return;
 
     // ---------------------------------------------------------- carried state out
     if constexpr (SUMMARY) {
