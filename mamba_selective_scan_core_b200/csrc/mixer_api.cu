@@ -406,7 +406,10 @@ mm_status mamba_state_update(const void* x, const void* z, const void* dt,
     if (!mul_ok(n_layers, batch, &lb) || !mul_ok(lb, d_inner, &rows) || !mul_ok(rows, d_state * 4, &st_bytes))
         return MM_ERR_SHAPE;
     if (rows == 0) return MM_OK;
-    if ((rows + 255) / 256 > INT32_MAX) return MM_ERR_SHAPE;
+    // one warp per (layer, 32-channel block, chunk of batch rows); warps <= rows
+    const int64_t warps = n_layers * ((d_inner + 31) / 32) *
+                          ((batch + mm::kDecodeBatchChunk - 1) / mm::kDecodeBatchChunk);
+    if ((warps + 7) / 8 > INT32_MAX) return MM_ERR_SHAPE;
 
     if (!x || !z || !dt || !conv_w || !dt_bias || !A || !Bm || !Cm || !ssm_state || !conv_state || !y)
         return MM_ERR_NULL;
@@ -429,20 +432,20 @@ mm_status mamba_state_update(const void* x, const void* z, const void* dt,
     if (mm_status st = check_device(&sm_count); st != MM_OK) return st;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const unsigned grid = static_cast<unsigned>((rows + 255) / 256);
+    const unsigned grid = static_cast<unsigned>((warps + 7) / 8);
     if (act == MM_BF16) {
         using T = __nv_bfloat16;
         mm::state_update_kernel<T, mm::MathFast><<<grid, 256, 0, s>>>(
             static_cast<const T*>(x), static_cast<const T*>(z), static_cast<const T*>(dt), conv_w, conv_b,
             dt_bias, Dskip, A, static_cast<const T*>(Bm), static_cast<const T*>(Cm), ssm_state,
-            static_cast<T*>(conv_state), static_cast<T*>(y), rows, static_cast<int>(batch),
+            static_cast<T*>(conv_state), static_cast<T*>(y), static_cast<int>(n_layers), static_cast<int>(batch),
             static_cast<int>(d_inner));
     } else {
         mm::state_update_kernel<float, mm::MathExact><<<grid, 256, 0, s>>>(
             static_cast<const float*>(x), static_cast<const float*>(z), static_cast<const float*>(dt), conv_w,
             conv_b, dt_bias, Dskip, A, static_cast<const float*>(Bm), static_cast<const float*>(Cm), ssm_state,
-            static_cast<float*>(conv_state), static_cast<float*>(y), rows, static_cast<int>(batch),
-            static_cast<int>(d_inner));
+            static_cast<float*>(conv_state), static_cast<float*>(y), static_cast<int>(n_layers),
+            static_cast<int>(batch), static_cast<int>(d_inner));
     }
     if (cudaGetLastError() != cudaSuccess) return MM_ERR_CUDA;
     return MM_OK;

@@ -12,20 +12,29 @@
 //
 // It is a single streaming pass over HBM: per (layer, batch, channel) row,
 // 64 B of state in and out, the 3-value window in and out, x/z/dt in and y
-// out.  Work decomposition, chosen so every global access of a warp is one
-// contiguous span:
-//   * a warp owns 32 consecutive rows; in the row phase lane i does the
-//     per-row work of row i (window, conv, SiLU, softplus, SiLU(z)) with
-//     coalesced 2-byte accesses;
+// out; the per-layer parameters and B/C are shared and stay in L2.
+//
+// Work decomposition, chosen so every global access of a warp is one
+// contiguous span and the shared per-layer data is read once per warp:
+//   * a warp owns one layer's block of 32 channels and walks a chunk of 16
+//     batch rows for it; A and the per-channel parameters are read from
+//     HBM/L2 once and from L1 for the other rows (A is not held in registers:
+//     that would cost 16 of them and force spills or lower occupancy);
+//   * in the row phase lane i does the per-row work of channel i (window, conv,
+//     SiLU, softplus, SiLU(z)) with coalesced 2-byte accesses;
 //   * in four state passes, pass p covers rows 8p..8p+7 with 4 lanes per row
 //     and 4 states per lane, so the warp's 16-byte state and A accesses form
 //     one contiguous 512-byte span; (Delta, Delta*u) arrive from the row's
 //     lane by shuffle and the partial readouts go back the same way.
-// State loads and stores are marked streaming (evict-first) so the per-layer
+// State loads and stores are marked streaming (evict-first) so the
 // parameters, reused by every batch row, stay in L2.
 #pragma once
 
 #include "mixer_common.cuh"
+
+#ifndef MM_DECODE_MIN_BLOCKS
+#define MM_DECODE_MIN_BLOCKS 4     // CTAs of 256 threads per SM: 64 registers, no spills
+#endif
 
 namespace mm {
 
@@ -41,84 +50,114 @@ template <> struct Vec4Act<__nv_bfloat16> {
     }
 };
 
+// Batch rows a warp walks for one (layer, 32-channel block).  A and the
+// per-channel parameters come from HBM/L2 once per warp and from L1 for the
+// other rows, so the per-layer data costs 1/16 of a row's traffic.
+constexpr int kDecodeBatchChunk = 16;
+
+// The fp32 path's libm calls need more registers; it keeps 3 CTAs per SM.
 template <typename T, typename M>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, sizeof(T) == 4 ? 3 : MM_DECODE_MIN_BLOCKS)
 state_update_kernel(const T* __restrict__ x, const T* __restrict__ z, const T* __restrict__ dt,
                     const float* __restrict__ conv_w, const float* __restrict__ conv_b,
                     const float* __restrict__ dt_bias, const float* __restrict__ Dskip,
                     const float* __restrict__ A, const T* __restrict__ Bm, const T* __restrict__ Cm,
                     float* __restrict__ ssm_state, T* __restrict__ conv_state, T* __restrict__ y,
-                    int64_t rows, int batch, int D)
+                    int n_layers, int batch, int D)
 {
     const int lane = threadIdx.x & 31;
-    const int64_t warp_row0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31));
-    if (warp_row0 >= rows) return;                      // whole warp past the end
+    const int q = lane & 3;            // which 4 states of a row
+    const int rr = lane >> 2;          // row within a pass
+    const int cblocks = (D + 31) / 32;
+    const int bchunks = (batch + kDecodeBatchChunk - 1) / kDecodeBatchChunk;
+    const int64_t warp = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
+    if (warp >= static_cast<int64_t>(n_layers) * cblocks * bchunks) return;
+    const int bc = static_cast<int>(warp % bchunks);
+    const int cb = static_cast<int>((warp / bchunks) % cblocks);
+    const int layer = static_cast<int>(warp / (static_cast<int64_t>(bchunks) * cblocks));
+    const int d0 = cb * 32;
+    const int b_begin = bc * kDecodeBatchChunk;
+    const int b_end = min(batch, b_begin + kDecodeBatchChunk);
 
-    // ---------------------------------------------------------- row phase
-    const int64_t r = warp_row0 + lane;
-    const bool live = r < rows;
-    float l = 0.f, s = 0.f, u = 0.f, gz = 0.f, dsk = 0.f;
-    if (live) {
-        const int64_t lb = r / D;
-        const int d = static_cast<int>(r - lb * D);
-        const int64_t ld = (lb / batch) * D + d;       // parameter row (layer, d)
-        const float4 w = *reinterpret_cast<const float4*>(conv_w + ld * 4);
-        const float cb = conv_b ? conv_b[ld] : 0.0f;
-        const float bias = dt_bias[ld];
+    // ---- per-(layer, channel) values shared by every batch row
+    const float* Aw = A + (static_cast<int64_t>(layer) * D + d0 + rr) * 16 + q * 4;  // pass 0's slice
+    const int dl = d0 + lane;          // this lane's channel in the row phase
+    const bool lok = dl < D;
+    float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+    float cbias = 0.f, bias2 = 0.f, dsk = 0.f;
+    if (lok) {
+        const int64_t ld = static_cast<int64_t>(layer) * D + dl;
+        w = *reinterpret_cast<const float4*>(conv_w + ld * 4);
+        cbias = conv_b ? conv_b[ld] : 0.0f;
+        bias2 = dt_bias[ld];
+        if constexpr (M::step_scale != 1.0f) bias2 *= kLog2e;
         dsk = Dskip ? Dskip[ld] : 0.0f;
-        T* cs = conv_state + r * 3;
-        const T c0 = cs[0], c1 = cs[1], c2 = cs[2];
-        const T xr = x[r];
-        float pre = fmaf(w.x, Act<T>::to_f32(c0), cb);
-        pre = fmaf(w.y, Act<T>::to_f32(c1), pre);
-        pre = fmaf(w.z, Act<T>::to_f32(c2), pre);
-        pre = fmaf(w.w, Act<T>::to_f32(xr), pre);
-        u = M::silu(pre);
-        const float dtv = Act<T>::load(dt + r);
-        if constexpr (M::step_scale == 1.0f) l = M::step(dtv, bias);
-        else l = M::step2(dtv, bias * kLog2e);
-        s = l * M::step_scale * u;                      // Delta * u
-        gz = M::silu(Act<T>::load(z + r));
-        // slide the window: drop the oldest, append this token's raw x
-        cs[0] = c1;
-        cs[1] = c2;
-        cs[2] = xr;
     }
 
-    // ---------------------------------------------------------- state passes
-    const int q = lane & 3;            // which 4 states of the row
-    const int rr = lane >> 2;          // row within the pass
-    float ysum = 0.f;                  // lane i ends with row i's readout
+#pragma unroll 1
+    for (int b = b_begin; b < b_end; ++b) {
+        const int64_t lb = static_cast<int64_t>(layer) * batch + b;
+        const int64_t rowbase = lb * D + d0;
+        // the row's whole 2 KB of state first, so it is in flight during the row phase
+        float4 hv[4];
 #pragma unroll
-    for (int pass = 0; pass < 4; ++pass) {
-        const int src = pass * 8 + rr;                  // lane holding this row's per-row values
-        const float lr = __shfl_sync(kFull, l, src);
-        const float sr = __shfl_sync(kFull, s, src);
-        const int64_t row = warp_row0 + src;
-        float part = 0.f;
-        if (row < rows) {
-            const int64_t lb = row / D;
-            const int d = static_cast<int>(row - lb * D);
-            const int64_t ld = (lb / batch) * D + d;
-            float4* hp = reinterpret_cast<float4*>(ssm_state + row * 16 + q * 4);
-            float4 h = __ldcs(hp);
-            const float4 a = *reinterpret_cast<const float4*>(A + ld * 16 + q * 4);
-            const float4 bv = Vec4Act<T>::load(Bm + lb * 16 + q * 4);
-            const float4 cv = Vec4Act<T>::load(Cm + lb * 16 + q * 4);
-            h.x = fmaf(M::decay(lr, a.x), h.x, sr * bv.x);
-            h.y = fmaf(M::decay(lr, a.y), h.y, sr * bv.y);
-            h.z = fmaf(M::decay(lr, a.z), h.z, sr * bv.z);
-            h.w = fmaf(M::decay(lr, a.w), h.w, sr * bv.w);
-            __stcs(hp, h);
-            part = fmaf(cv.x, h.x, fmaf(cv.y, h.y, fmaf(cv.z, h.z, cv.w * h.w)));
+        for (int pass = 0; pass < 4; ++pass)
+            hv[pass] = d0 + pass * 8 + rr < D
+                           ? __ldcs(reinterpret_cast<const float4*>(ssm_state + (rowbase + pass * 8 + rr) * 16 + q * 4))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 bq = Vec4Act<T>::load(Bm + lb * 16 + q * 4);
+        const float4 cq = Vec4Act<T>::load(Cm + lb * 16 + q * 4);
+
+        // ---- row phase: lane i does the per-row work of channel d0 + i
+        float l = 0.f, s = 0.f, u = 0.f, gz = 0.f;
+        if (lok) {
+            const int64_t r = rowbase + lane;
+            T* cs = conv_state + r * 3;
+            const T w0 = cs[0], w1 = cs[1], w2 = cs[2];
+            const T xr = x[r];
+            const float dtv = Act<T>::load(dt + r);
+            const float zv = Act<T>::load(z + r);
+            float pre = fmaf(w.x, Act<T>::to_f32(w0), cbias);
+            pre = fmaf(w.y, Act<T>::to_f32(w1), pre);
+            pre = fmaf(w.z, Act<T>::to_f32(w2), pre);
+            pre = fmaf(w.w, Act<T>::to_f32(xr), pre);
+            u = M::silu(pre);
+            if constexpr (M::step_scale == 1.0f) l = M::step(dtv, bias2);
+            else l = M::step2(dtv, bias2);
+            s = l * M::step_scale * u;                  // Delta * u
+            gz = M::silu(zv);
+            // slide the window: drop the oldest, append this token's raw x
+            cs[0] = w1;
+            cs[1] = w2;
+            cs[2] = xr;
         }
-        part += __shfl_xor_sync(kFull, part, 1);
-        part += __shfl_xor_sync(kFull, part, 2);
-        // every lane of the quad now holds row src's readout; lane src takes it
-        const float got = __shfl_sync(kFull, part, ((lane - pass * 8) & 7) * 4);
-        if ((lane >> 3) == pass) ysum = got;
+
+        // ---- state passes: 4 lanes per row, 4 states per lane
+        float ysum = 0.f;              // lane i ends with channel d0 + i's readout
+#pragma unroll
+        for (int pass = 0; pass < 4; ++pass) {
+            const int src = pass * 8 + rr;              // lane holding this row's per-row values
+            const float lr = __shfl_sync(kFull, l, src);
+            const float sr = __shfl_sync(kFull, s, src);
+            float part = 0.f;
+            if (d0 + src < D) {
+                float4 h = hv[pass];
+                const float4 a = __ldg(reinterpret_cast<const float4*>(Aw + pass * 8 * 16));  // L1 after row 0
+                h.x = fmaf(M::decay(lr, a.x), h.x, sr * bq.x);
+                h.y = fmaf(M::decay(lr, a.y), h.y, sr * bq.y);
+                h.z = fmaf(M::decay(lr, a.z), h.z, sr * bq.z);
+                h.w = fmaf(M::decay(lr, a.w), h.w, sr * bq.w);
+                __stcs(reinterpret_cast<float4*>(ssm_state + (rowbase + src) * 16 + q * 4), h);
+                part = fmaf(cq.x, h.x, fmaf(cq.y, h.y, fmaf(cq.z, h.z, cq.w * h.w)));
+            }
+            part += __shfl_xor_sync(kFull, part, 1);
+            part += __shfl_xor_sync(kFull, part, 2);
+            // every lane of the quad now holds row src's readout; lane src takes it
+            const float got = __shfl_sync(kFull, part, ((lane - pass * 8) & 7) * 4);
+            if ((lane >> 3) == pass) ysum = got;
+        }
+        if (lok) y[rowbase + lane] = Act<T>::from_f32(fmaf(dsk, u, ysum) * gz);
     }
-    if (live) y[r] = Act<T>::from_f32(fmaf(dsk, u, ysum) * gz);
 }
 
 }  // namespace mm

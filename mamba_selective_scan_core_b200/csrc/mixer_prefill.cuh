@@ -187,9 +187,6 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * stageB + TILE * 64 * 4);
 
     const T* xz = static_cast<const T*>(p.xz);
-    const T* dtg = static_cast<const T*>(p.dt);
-    const T* Bg = static_cast<const T*>(p.Bm);
-    const T* Cg = static_cast<const T*>(p.Cm);
     const int64_t seq_row0 = static_cast<int64_t>(seq) * L;
     const int64_t chan = static_cast<int64_t>(seq) * D + d;           // (sequence, first channel) row
 
@@ -292,7 +289,7 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
     auto run_sub = [&](const unsigned char* st, int r0, int64_t t0, auto structured_tag, const float2* a2) {
         constexpr bool kStruct = decltype(structured_tag)::value;
         const T* xs = reinterpret_cast<const T*>(st);          // row rho = token - 3 (tile-relative)
-        const T* zs = reinterpret_cast<const T*>(st + offZ);
+        [[maybe_unused]] const T* zs = reinterpret_cast<const T*>(st + offZ);   // full pass only
         const T* ds = reinterpret_cast<const T*>(st + offDT);
         const int nvalid = static_cast<int>(min(static_cast<int64_t>(SUB), t_end - t0));   // tokens of the chunk here
 
@@ -318,7 +315,7 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
         }
 
         // ---- B: state update (and readout) over the SUB tokens
-        float2 yacc[SUB];
+        [[maybe_unused]] float2 yacc[SUB];                 // full pass only
 #pragma unroll
         for (int m = 0; m < SUB; ++m) {
             float2 P[16];
