@@ -18,7 +18,7 @@ using mm::PrefillLayout;
 using mm::PrefillParams;
 
 constexpr int kTile = 32;
-constexpr int kMaxThreads = 256;
+constexpr int kMaxThreads = 128;
 constexpr int kSmemBudget = 200 * 1024;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -67,7 +67,7 @@ struct FwdPlan {
 };
 
 constexpr int kPlanSMs = 148;            // B200: 2 dies x 74 SMs
-constexpr int kWarpsPerSM = 8;           // resident warps per SM at the forward's register use
+constexpr int kWarpsPerSM = 4 * MM_FWD_MIN_BLOCKS;   // resident warps per SM at the forward's register use
 constexpr int kMinChunkTiles = 4;        // shortest chunk worth a summary pass
 constexpr int kMaxChunks = 16;
 
@@ -79,8 +79,6 @@ int env_int(const char* name, int lo, int hi) {
     return 0;
 }
 
-// Time chunks: the fewest that bring the resident warps (two channels per
-// thread) to ~80% of what the SMs hold.
 // Tries per wait on a bulk copy (each try waits a bounded time in hardware):
 // about a second by default; MAMBA_MIXER_WAIT_LIMIT overrides it (tests use 0
 // to make the wait give up at once).
@@ -93,16 +91,19 @@ unsigned copy_wait_limit() {
     return 1u << 20;
 }
 
+// Time chunks: as many as the SMs' resident warp slots hold in one wave
+// (two channels per thread, so a sequence of D channels is D/64 warps per
+// chunk); a second, partial wave would cost more than the idle slots.
 FwdPlan plan_fwd(int64_t batch, int64_t seqlen, int64_t d_inner) {
     FwdPlan pl;
     const int64_t warps = std::max<int64_t>(1, batch * d_inner / 2 / 32);
-    const int64_t want = static_cast<int64_t>(kPlanSMs) * kWarpsPerSM * 4 / 5;
+    const int64_t slots = static_cast<int64_t>(kPlanSMs) * kWarpsPerSM;
     const int64_t tiles = (seqlen + kTile - 1) / kTile;
     int64_t k = 1;
     if (const int forced = env_int("MAMBA_MIXER_CHUNKS", 1, 1 << 20)) {
         k = forced;
-    } else if (warps < want) {
-        k = (want + warps - 1) / warps;
+    } else if (2 * warps <= slots) {
+        k = slots / warps;
         k = std::min<int64_t>(k, std::max<int64_t>(1, tiles / kMinChunkTiles));
         k = std::min<int64_t>(k, kMaxChunks);
     }

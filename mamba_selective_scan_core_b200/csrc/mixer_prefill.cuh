@@ -62,6 +62,9 @@
 #ifndef MM_SUB
 #define MM_SUB 8               // tokens per sub-tile
 #endif
+#ifndef MM_FWD_MIN_BLOCKS
+#define MM_FWD_MIN_BLOCKS 2    // resident CTAs of 128 threads per SM the register budget must allow
+#endif
 
 namespace mm {
 
@@ -132,7 +135,14 @@ template <> struct Pair<__nv_bfloat16> {
 
 // Packed forms of the math policy's per-channel functions.
 template <typename M>
-__device__ __forceinline__ float2 silu2(float2 v) { return f2(M::silu(v.x), M::silu(v.y)); }
+__device__ __forceinline__ float2 silu2(float2 v) {
+    if constexpr (M::step_scale != 1.0f) {
+        // fast path: SiLU(v) = h + h tanh(h), h = v/2, with the halving and the FMA packed
+        const float2 h = mul2(v, f2(0.5f, 0.5f));
+        return fma2(h, f2(tanh_fast(h.x), tanh_fast(h.y)), h);
+    }
+    return f2(M::silu(v.x), M::silu(v.y));
+}
 
 template <typename M>
 __device__ __forceinline__ float2 step_pair(float2 dt, float2 bias) {
@@ -148,7 +158,7 @@ __device__ __forceinline__ float2 decay2(float2 l, float2 a) {
 // SUMMARY = true: the summary pass (chunk end state from zero + sum of l).
 // SUMMARY = false: the full fused forward over one chunk.
 template <typename T, typename M, int TILE, int STAGES, bool SUMMARY>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(128, MM_FWD_MIN_BLOCKS)
 mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x,
                  const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_dt,
                  const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c)

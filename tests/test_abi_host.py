@@ -52,9 +52,10 @@ def test_version_and_strings(L):
         s = mm.status_string(code)
         assert s and s != "unknown status"
     assert mm.status_string(99) == "unknown status"
-    # one 8192-channel sequence (128 warps of channel pairs) is split into 8
-    # time chunks to fill the SMs: 7 carried states of 17 floats per channel
-    assert mm.workspace_size(1, 4096, 8192) == 7 * 8192 * 17 * 4
+    # one 8192-channel sequence (128 warps of channel pairs) is split into as
+    # many time chunks as 148 SMs x 8 warps hold at once: 9 chunks of 480
+    # tokens, 8 carried states of 17 floats per channel
+    assert mm.workspace_size(1, 4096, 8192) == 8 * 8192 * 17 * 4
     # four such sequences into 2 chunks
     assert mm.workspace_size(4, 32768, 8192) == 1 * 4 * 8192 * 17 * 4
     # enough sequences need no time chunks and no workspace
