@@ -80,11 +80,11 @@ def _measured_peaks():
 
 
 def _kernel_source_sha():
-    """Hash of the device code (the kernel headers) the traffic figures depend on."""
+    """Hash of the CUDA sources (kernels and launch plan) the traffic figures depend on."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mamba_selective_scan_core_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if not name.endswith(".cuh"):
+        if not name.endswith((".cuh", ".cu")):
             continue
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
