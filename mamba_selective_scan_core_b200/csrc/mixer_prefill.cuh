@@ -30,12 +30,15 @@
 // Parallelism.  The recurrence is sequential in t per channel: a single
 // 8192-channel sequence is only 4096 channel pairs, 128 warps.  Time chunks
 // supply the rest, as an exact re-association of h_t = a_t h_{t-1} + b_t:
-// a summary pass runs each of chunks 0..K-2 from a zero state and keeps its
-// end state e_c and the sum of its step sizes (whose exponential is the
-// chunk's total decay P_c); the full pass starts chunk c from h0 carried
-// through (P_0, e_0) .. (P_{c-1}, e_{c-1}) -- the true state at the chunk
-// boundary -- and runs the fused forward.  The summary pass skips the
-// readout, the gate and the z/C traffic.
+// a summary pass finds, for each of chunks 0..K-2, its end state e_c from a
+// zero start and the sum of its step sizes (whose exponential is the chunk's
+// total decay P_c); the full pass starts chunk c from h0 carried through
+// (P_0, e_0) .. (P_{c-1}, e_{c-1}) -- the true state at the chunk boundary --
+// and runs the fused forward.  The summary pass skips the readout, the gate
+// and the z/C traffic, and walks its chunk backward: e_c[n] is the sum over
+// tokens of s_t B_t[n] exp(A[n] R_t), R_t the steps after token t, so with
+// structured A a token costs a 16-step multiply chain and 16 FMAs instead of
+// the forward recurrence's 15 decay powers, 16 products and 16 FMAs.
 //
 // Latency: each tile is processed in sub-tiles of SUB tokens in three phases
 // so that the long per-token chains (conv -> SiLU -> softplus -> exp) of SUB
@@ -207,12 +210,17 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
     const unsigned stage_tx = (TILE + kHalo) * rowb + TILE * rowb * (SUMMARY ? 1 : 2) +
                               kBC * TILE * 16 * static_cast<unsigned>(sizeof(T));
 
-    // one thread: stage tile k (tokens t_begin + k*TILE ..) into ring slot k % STAGES
+    // The full pass walks its chunk forward; the summary pass walks it
+    // backward (its end state is accumulated from the last token down).
+    auto tile_of = [&](int64_t k) -> int64_t { return SUMMARY ? ntiles - 1 - k : k; };
+
+    // one thread: stage the k-th tile walked (tokens t_begin + tile_of(k)*TILE ..)
+    // into ring slot k % STAGES
     auto issue_tile = [&](int64_t k) {
         if (k >= ntiles) return;
         const int slot = static_cast<int>(k % STAGES);
         unsigned char* st = smem + slot * stageB;
-        const int tb = static_cast<int>(t_begin + k * TILE);
+        const int tb = static_cast<int>(t_begin + tile_of(k) * TILE);
         uint64_t* bar = &bars[slot];
         mbar_arrive_expect_tx(bar, stage_tx);
         tma_load_3d(st, &tm_x, d0, tb - kHalo, seq, bar);
@@ -292,7 +300,7 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
     }
 
     T* yg = static_cast<T*>(p.y);
-    float2 lsum = f2(0.f, 0.f);           // summary pass: sum of l over the chunk
+    float2 lsum = f2(0.f, 0.f);           // summary pass: sum of l over the tokens walked so far
 
     // One sub-tile of SUB tokens starting at staged row r0 (token t0).
     // a2 (general A only): the 16 A pairs of my channels.
@@ -317,51 +325,95 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
             float2 l = step_pair<M>(P_::load(ds + (r0 + m) * rs + cls), bias2);
             if (m >= nvalid) l = f2(0.f, 0.f);                  // past the chunk: no step
             const float2 s = mul2(l, u);                         // Delta*u in B' units (B' = B * step_scale)
-            if constexpr (SUMMARY) lsum = __fadd2_rn(lsum, l);
-            if constexpr (kStruct) ea[m] = f2(ex2_fast(l.x * A02.x), ex2_fast(l.y * A02.y));   // q
+            if constexpr (!SUMMARY && kStruct) ea[m] = f2(ex2_fast(l.x * A02.x), ex2_fast(l.y * A02.y));   // q
             else ea[m] = l;
             sa[m] = s;
             ua[m] = u;
         }
 
-        // ---- B: state update (and readout) over the SUB tokens
-        [[maybe_unused]] float2 yacc[SUB];                 // full pass only
+        if constexpr (SUMMARY) {
+            // ---- B (summary pass, tokens walked last to first): the chunk's end
+            // state from zero is e[n] = sum_t s_t B'_t[n] exp(A[n] R_t), with
+            // R_t the sum of the steps after token t.  With R carried in lsum
+            // (the steps of the tokens walked so far), a token's 16 weights are
+            // s r^(n+1), r = exp(A[0] R): 18 packed multiplies, no exp per state.
+            float2 R[SUB];
+            R[SUB - 1] = lsum;
 #pragma unroll
-        for (int m = 0; m < SUB; ++m) {
-            float2 P[16];
-            if constexpr (kStruct) {
-                // P[n] = q^(n+1) by repeated squaring: depth 4, 15 packed multiplies
-                P[0] = ea[m];
-                P[1] = mul2(P[0], P[0]);
-                P[2] = mul2(P[1], P[0]);
-                P[3] = mul2(P[1], P[1]);
+            for (int m = SUB - 2; m >= 0; --m) R[m] = __fadd2_rn(R[m + 1], ea[m + 1]);
+            lsum = __fadd2_rn(R[0], ea[0]);
 #pragma unroll
-                for (int n = 0; n < 4; ++n) P[4 + n] = mul2(P[n], P[3]);
+            for (int m = SUB - 1; m >= 0; --m) {
+                const float* row = bcf + (r0 + m) * 64;
+                if constexpr (kStruct) {
+                    // weights w[n] = s r^(n+1) as four interleaved chains (step r^4),
+                    // so no chain is longer than six multiplies
+                    const float2 r = f2(ex2_fast(R[m].x * A02.x), ex2_fast(R[m].y * A02.y));
+                    const float2 r2 = mul2(r, r);
+                    const float2 r4 = mul2(r2, r2);
+                    float2 w[4];
+                    w[0] = mul2(sa[m], r);
+                    w[1] = mul2(w[0], r);
+                    w[2] = mul2(w[0], r2);
+                    w[3] = mul2(w[1], r2);
 #pragma unroll
-                for (int n = 0; n < 8; ++n) P[8 + n] = mul2(P[n], P[7]);
-            } else {
+                    for (int g = 0; g < 4; ++g) {
+                        const float4 b01 = *reinterpret_cast<const float4*>(row + 8 * g);       // (B,B) of states 4g, 4g+1
+                        const float4 b23 = *reinterpret_cast<const float4*>(row + 8 * g + 4);
+                        h[4 * g] = fma2(w[0], f2(b01.x, b01.y), h[4 * g]);
+                        h[4 * g + 1] = fma2(w[1], f2(b01.z, b01.w), h[4 * g + 1]);
+                        h[4 * g + 2] = fma2(w[2], f2(b23.x, b23.y), h[4 * g + 2]);
+                        h[4 * g + 3] = fma2(w[3], f2(b23.z, b23.w), h[4 * g + 3]);
+                        if (g < 3) {
 #pragma unroll
-                for (int n = 0; n < 16; ++n) P[n] = decay2<M>(ea[m], a2[n]);
+                            for (int i = 0; i < 4; ++i) w[i] = mul2(w[i], r4);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int n = 0; n < 16; n += 2) {
+                        const float4 bb = *reinterpret_cast<const float4*>(row + 2 * n);
+                        h[n] = fma2(mul2(sa[m], decay2<M>(R[m], a2[n])), f2(bb.x, bb.y), h[n]);
+                        h[n + 1] = fma2(mul2(sa[m], decay2<M>(R[m], a2[n + 1])), f2(bb.z, bb.w), h[n + 1]);
+                    }
+                }
             }
-            const float* row = bcf + (r0 + m) * 64;
-            const float2 s = sa[m];
-            float2 acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
+        } else {
+            // ---- B: state update and readout over the SUB tokens
+            float2 yacc[SUB];
 #pragma unroll
-            for (int n = 0; n < 16; n += 2) {
-                const float4 bb = *reinterpret_cast<const float4*>(row + 2 * n);        // (Bn, Bn, Bn+1, Bn+1)
-                h[n] = fma2(P[n], h[n], mul2(s, f2(bb.x, bb.y)));
-                h[n + 1] = fma2(P[n + 1], h[n + 1], mul2(s, f2(bb.z, bb.w)));
-                if constexpr (!SUMMARY) {
+            for (int m = 0; m < SUB; ++m) {
+                float2 P[16];
+                if constexpr (kStruct) {
+                    // P[n] = q^(n+1) by repeated squaring: depth 4, 15 packed multiplies
+                    P[0] = ea[m];
+                    P[1] = mul2(P[0], P[0]);
+                    P[2] = mul2(P[1], P[0]);
+                    P[3] = mul2(P[1], P[1]);
+#pragma unroll
+                    for (int n = 0; n < 4; ++n) P[4 + n] = mul2(P[n], P[3]);
+#pragma unroll
+                    for (int n = 0; n < 8; ++n) P[8 + n] = mul2(P[n], P[7]);
+                } else {
+#pragma unroll
+                    for (int n = 0; n < 16; ++n) P[n] = decay2<M>(ea[m], a2[n]);
+                }
+                const float* row = bcf + (r0 + m) * 64;
+                const float2 s = sa[m];
+                float2 acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
+#pragma unroll
+                for (int n = 0; n < 16; n += 2) {
+                    const float4 bb = *reinterpret_cast<const float4*>(row + 2 * n);        // (Bn, Bn, Bn+1, Bn+1)
+                    h[n] = fma2(P[n], h[n], mul2(s, f2(bb.x, bb.y)));
+                    h[n + 1] = fma2(P[n + 1], h[n + 1], mul2(s, f2(bb.z, bb.w)));
                     const float4 cc = *reinterpret_cast<const float4*>(row + 32 + 2 * n);   // (Cn, Cn, Cn+1, Cn+1)
                     acc0 = fma2(f2(cc.x, cc.y), h[n], acc0);
                     acc1 = fma2(f2(cc.z, cc.w), h[n + 1], acc1);
                 }
+                yacc[m] = __fadd2_rn(acc0, acc1);
             }
-            if constexpr (!SUMMARY) yacc[m] = __fadd2_rn(acc0, acc1);
-        }
 
-        // ---- C: skip, gate, store
-        if constexpr (!SUMMARY) {
+            // ---- C: skip, gate, store
 #pragma unroll
             for (int m = 0; m < SUB; ++m) {
                 const float2 g = silu2<M>(P_::load(zs + (r0 + m) * rs + cls));
@@ -387,7 +439,7 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
                 return false;
             }
             unsigned char* st = smem + slot * stageB;
-            if (t_begin == 0 && k == 0 && cl < p.octets * 8) {
+            if (t_begin == 0 && tile_of(k) == 0 && cl < p.octets * 8) {
                 // left context of token 0: the carried conv window (zeros if none)
                 T* xs = reinterpret_cast<T*>(st);
 #pragma unroll
@@ -414,10 +466,12 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
                 issue_tile(k + STAGES - 1);
             }
             __syncthreads();
-            const int64_t tile_t0 = t_begin + k * TILE;
+            const int64_t tile_t0 = t_begin + tile_of(k) * TILE;
 #pragma unroll 1
-            for (int r0 = 0; r0 < TILE; r0 += SUB)
+            for (int j = 0; j < TILE / SUB; ++j) {
+                const int r0 = (SUMMARY ? TILE / SUB - 1 - j : j) * SUB;
                 run_sub(st, r0, tile_t0 + r0, structured_tag, a2);
+            }
         }
         return true;
     };
