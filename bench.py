@@ -310,33 +310,29 @@ def run_gpu(args):
 
 
 def run_e2e(mm, host, args, world):
-    """Same metric through the public API with host buffers: every step copies
-    its inputs from pinned host memory, runs the forward and reads y and the
-    carried state back."""
+    """Same metric through the public API with host buffers: every step calls
+    the host-memory forward (mamba_mixer_fwd_host) on pinned inputs; it copies
+    them in, runs the forward and copies y and the carried state back,
+    overlapping the copies of one piece of the sequence with the compute of
+    its neighbours."""
     cfg = PREFILL
     B, L, D = cfg.batch, cfg.seqlen, cfg.d_inner
     keys_in = ["xz", "dt", "Bm", "Cm"]
     pinned = {k: host[k].pin_memory() for k in keys_in}
     params = {k: (host[k].cuda() if host[k] is not None else None)
-              for k in ("conv_w", "conv_b", "dt_bias", "A", "Dskip", "h0", "conv_state_in")}
-    dev = {k: torch.empty_like(pinned[k], device="cuda") for k in keys_in}
+              for k in ("conv_w", "conv_b", "dt_bias", "A", "Dskip")}
+    carry_in = {k: (host[k].pin_memory() if host[k] is not None else None) for k in ("h0", "conv_state_in")}
     y_h = torch.empty((B, L, D), dtype=torch.bfloat16).pin_memory()
     h_h = torch.empty((B, D, 16)).pin_memory()
     cs_h = torch.empty((B, D, 3), dtype=torch.bfloat16).pin_memory()
-    outs = (torch.empty((B, L, D), dtype=torch.bfloat16, device="cuda"), torch.empty((B, D, 16), device="cuda"),
-            torch.empty((B, D, 3), dtype=torch.bfloat16, device="cuda"))
-    h2d = sum(pinned[k].numel() * pinned[k].element_size() for k in keys_in)
+    ws = torch.empty(max(16, mm.host_workspace_size(B, L, D)), dtype=torch.uint8, device="cuda")
+    h2d = sum(t.numel() * t.element_size() for t in list(pinned.values()) + [v for v in carry_in.values() if v is not None])
     d2h = sum(t.numel() * t.element_size() for t in (y_h, h_h, cs_h))
 
     def step():
-        for k in keys_in:
-            dev[k].copy_(pinned[k], non_blocking=True)
-        d = dict(params)
-        d.update(dev)
-        _fwd_call(mm, d, outs)
-        y_h.copy_(outs[0], non_blocking=True)
-        h_h.copy_(outs[1], non_blocking=True)
-        cs_h.copy_(outs[2], non_blocking=True)
+        mm.mixer_fwd_host(pinned["xz"], params["conv_w"], params["conv_b"], pinned["dt"], params["dt_bias"],
+                          params["A"], pinned["Bm"], pinned["Cm"], params["Dskip"], carry_in["h0"],
+                          carry_in["conv_state_in"], y=y_h, h_last=h_h, conv_state_out=cs_h, workspace=ws)
 
     K = max(3, min(args.steps, 200))
     for _ in range(3):

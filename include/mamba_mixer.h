@@ -160,6 +160,49 @@ size_t mamba_mixer_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner
                                   int64_t d_state, int64_t d_conv, mm_dtype act);
 
 /*
+ * The forward (mamba_mixer_fwd) on activations held in HOST memory, for a
+ * caller whose sequence is not yet on the device.  The per-channel
+ * parameters (conv_w, conv_b, dt_bias, A, Dskip) are DEVICE pointers, as in
+ * mamba_mixer_fwd; everything else is a HOST pointer with the same shape and
+ * meaning:
+ *   in : xz, dt, Bm, Cm; h0 and conv_state_in (or NULL = zeros)
+ *   out: y, h_last, conv_state_out
+ * The sequence is cut into pieces along L.  Each piece's inputs are copied
+ * to the device on `h2d_stream`, the forward runs on it on `stream` with the
+ * state (h and the conv window) carried from the previous piece on the
+ * device, and its y is copied back on `d2h_stream`; two staging slots let the
+ * copies of one piece overlap the compute of its neighbours.  The result is
+ * the forward of the whole sequence (it differs from one mamba_mixer_fwd
+ * call only by where the time is split, i.e. by fp32 rounding).
+ *
+ * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister) for
+ * the copies to overlap; pageable memory is correct but serialises.
+ * `workspace` is DEVICE memory of at least
+ * mamba_mixer_host_workspace_size(...) bytes, 16-byte aligned; it holds the
+ * staging slots, the carried state and the forward's own scratch.  The
+ * library allocates no memory.  The three streams may be the same stream
+ * (no overlap) and may be NULL (the legacy default stream).
+ * Asynchronous: when it returns, all work is queued and `stream` waits for
+ * the last copy back, so synchronising `stream` makes every output valid.
+ * Host buffers must stay alive and unmodified until then.  Errors as
+ * mamba_mixer_fwd; sizes are validated before anything is queued.
+ */
+mm_status mamba_mixer_fwd_host(const void* xz, const float* conv_w, const float* conv_b,
+                               const void* dt, const float* dt_bias, const float* A,
+                               const void* Bm, const void* Cm, const float* Dskip,
+                               const float* h0, const void* conv_state_in,
+                               void* y, float* h_last, void* conv_state_out,
+                               int64_t batch, int64_t seqlen, int64_t d_inner,
+                               int64_t d_state, int64_t d_conv, mm_dtype act,
+                               void* workspace, size_t workspace_bytes,
+                               void* stream, void* h2d_stream, void* d2h_stream);
+
+/* Bytes of device workspace mamba_mixer_fwd_host needs for these sizes (0 for
+ * invalid sizes). */
+size_t mamba_mixer_host_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner,
+                                       int64_t d_state, int64_t d_conv, mm_dtype act);
+
+/*
  * One-token state update (decode) for n_layers independent stacked Mamba
  * layers at batch `batch`, updating the carried state in place.
  *

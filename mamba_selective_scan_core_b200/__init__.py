@@ -14,8 +14,9 @@ import ctypes
 import os
 
 __all__ = [
-    "MM_F32", "MM_BF16", "MixerError", "lib", "library_path", "mixer_fwd", "mixer_fwd_noalloc", "state_update",
-    "workspace_size", "status_string", "abi_version", "fault_status", "EXPORTED_SYMBOLS",
+    "MM_F32", "MM_BF16", "MixerError", "lib", "library_path", "mixer_fwd", "mixer_fwd_noalloc", "mixer_fwd_host",
+    "state_update", "workspace_size", "host_workspace_size", "status_string", "abi_version", "fault_status",
+    "EXPORTED_SYMBOLS",
 ]
 
 MM_F32 = 0
@@ -28,7 +29,9 @@ _lib = None
 EXPORTED_SYMBOLS = (
     "mamba_mixer_fwd",
     "mamba_mixer_fwd_noalloc",
+    "mamba_mixer_fwd_host",
     "mamba_mixer_workspace_size",
+    "mamba_mixer_host_workspace_size",
     "mamba_state_update",
     "mamba_status_string",
     "mamba_mixer_abi_version",
@@ -55,8 +58,12 @@ def _declare(L):
     L.mamba_mixer_fwd.argtypes = [P] * 14 + [I64] * 5 + [ctypes.c_int, P, ctypes.c_size_t, P]
     L.mamba_mixer_fwd_noalloc.restype = ctypes.c_int
     L.mamba_mixer_fwd_noalloc.argtypes = [P] * 14 + [I64] * 5 + [ctypes.c_int, P]
+    L.mamba_mixer_fwd_host.restype = ctypes.c_int
+    L.mamba_mixer_fwd_host.argtypes = [P] * 14 + [I64] * 5 + [ctypes.c_int, P, ctypes.c_size_t, P, P, P]
     L.mamba_mixer_workspace_size.restype = ctypes.c_size_t
     L.mamba_mixer_workspace_size.argtypes = [I64] * 5 + [ctypes.c_int]
+    L.mamba_mixer_host_workspace_size.restype = ctypes.c_size_t
+    L.mamba_mixer_host_workspace_size.argtypes = [I64] * 5 + [ctypes.c_int]
     L.mamba_state_update.restype = ctypes.c_int
     L.mamba_state_update.argtypes = [P] * 13 + [I64] * 5 + [ctypes.c_int, P]
     L.mamba_status_string.restype = ctypes.c_char_p
@@ -182,6 +189,89 @@ def mixer_fwd(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, conv_s
             Bsz, L, D, N, W, act, _ptr(workspace) if ws_bytes else None, ws_bytes, _stream_handle(stream))
     if st != 0:
         raise MixerError(st, "mamba_mixer_fwd")
+    return y, h_last, conv_state_out
+
+
+def host_workspace_size(batch, seqlen, d_inner, d_state=16, d_conv=4, act=MM_BF16) -> int:
+    return int(lib().mamba_mixer_host_workspace_size(batch, seqlen, d_inner, d_state, d_conv, act))
+
+
+def _check_host(t, name, dtype, shape):
+    if t is None:
+        return
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+_side_streams = {}
+
+
+def _copy_streams(dev):
+    """Two side streams per device for the host path's copies (created once)."""
+    import torch
+
+    key = torch.device(dev).index
+    if key not in _side_streams:
+        with torch.cuda.device(dev):
+            _side_streams[key] = (torch.cuda.Stream(), torch.cuda.Stream())
+    return _side_streams[key]
+
+
+def mixer_fwd_host(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, conv_state_in=None, *,
+                   y=None, h_last=None, conv_state_out=None, workspace=None, stream=None):
+    """mixer_fwd on activations in host memory (mamba_mixer_fwd_host): xz, dt,
+    Bm, Cm, h0, conv_state_in and the outputs are CPU tensors (page-locked for
+    the copies to overlap the compute; outputs are allocated pinned when not
+    given); conv_w, conv_b, dt_bias, A, Dskip are CUDA tensors on the device
+    that runs it.  Copies go on two side streams, the forward on `stream`
+    (default: the current stream), which waits for the copies back: the
+    outputs are valid once `stream` is synchronised."""
+    import torch
+
+    act = _act_code(xz.dtype)
+    Bsz, L, twoD = xz.shape
+    D = twoD // 2
+    N = A.shape[-1]
+    W = conv_w.shape[-1]
+    dev = conv_w.device
+    f32 = torch.float32
+    for t, name, dtype, shape in ((xz, "xz", xz.dtype, (Bsz, L, 2 * D)), (dt, "dt", xz.dtype, (Bsz, L, D)),
+                                  (Bm, "Bm", xz.dtype, (Bsz, L, N)), (Cm, "Cm", xz.dtype, (Bsz, L, N)),
+                                  (h0, "h0", f32, (Bsz, D, N)),
+                                  (conv_state_in, "conv_state_in", xz.dtype, (Bsz, D, W - 1))):
+        _check_host(t, name, dtype, shape)
+    _check(conv_w, "conv_w", f32, (D, W), dev)
+    _check(conv_b, "conv_b", f32, (D,), dev)
+    _check(dt_bias, "dt_bias", f32, (D,), dev)
+    _check(A, "A", f32, (D, N), dev)
+    _check(Dskip, "Dskip", f32, (D,), dev)
+    if y is None:
+        y = torch.empty((Bsz, L, D), dtype=xz.dtype).pin_memory()
+    if h_last is None:
+        h_last = torch.empty((Bsz, D, N), dtype=f32).pin_memory()
+    if conv_state_out is None:
+        conv_state_out = torch.empty((Bsz, D, W - 1), dtype=xz.dtype).pin_memory()
+    _check_host(y, "y", xz.dtype, (Bsz, L, D))
+    _check_host(h_last, "h_last", f32, (Bsz, D, N))
+    _check_host(conv_state_out, "conv_state_out", xz.dtype, (Bsz, D, W - 1))
+    ws_bytes = host_workspace_size(Bsz, L, D, N, W, act)
+    if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    s_in, s_out = _copy_streams(dev)
+    with torch.cuda.device(dev):
+        st = lib().mamba_mixer_fwd_host(
+            _ptr(xz), _ptr(conv_w), _ptr(conv_b), _ptr(dt), _ptr(dt_bias), _ptr(A), _ptr(Bm), _ptr(Cm),
+            _ptr(Dskip), _ptr(h0), _ptr(conv_state_in), _ptr(y), _ptr(h_last), _ptr(conv_state_out),
+            Bsz, L, D, N, W, act, _ptr(workspace), ws_bytes, _stream_handle(stream),
+            ctypes.c_void_p(s_in.cuda_stream), ctypes.c_void_p(s_out.cuda_stream))
+    if st != 0:
+        raise MixerError(st, "mamba_mixer_fwd_host")
     return y, h_last, conv_state_out
 
 

@@ -243,6 +243,62 @@ cudaError_t dispatch_prefill(PrefillParams p, int64_t batch, const FwdPlan& pl, 
     return launch_pass<T, M, false>(p, batch, pl.chunks, sm_count, s);
 }
 
+// ---------------------------------------------------------------- host-memory forward
+// Piece plan of mamba_mixer_fwd_host: the sequence is cut into about
+// kHostPieces pieces (whole tiles, at least kHostMinPiece tokens) and the
+// device workspace holds two staging slots, two carried states (ping-pong)
+// and the piece forward's own scratch, each region 256-byte aligned.
+constexpr int64_t kHostPieces = 8;
+constexpr int64_t kHostMinPiece = 256;
+
+struct HostPlan {
+    int64_t piece = 0, pieces = 0;
+    size_t off_dt = 0, off_b = 0, off_c = 0, off_y = 0, slot = 0;   // within a staging slot
+    size_t carry_h = 0, carry = 0;                                  // within a carried state
+    size_t fwd_ws = 0, total = 0;
+};
+
+size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+HostPlan plan_host(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t es) {
+    HostPlan hp;
+    int64_t piece = (seqlen + kHostPieces - 1) / kHostPieces;
+    piece = (piece + kTile - 1) / kTile * kTile;
+    piece = std::max(piece, kHostMinPiece);
+    hp.piece = std::max<int64_t>(1, std::min(piece, seqlen));
+    hp.pieces = seqlen > 0 ? (seqlen + hp.piece - 1) / hp.piece : 1;   // L = 0: one empty piece
+    const size_t tok = static_cast<size_t>(batch) * static_cast<size_t>(hp.piece);
+    const size_t D = static_cast<size_t>(d_inner), e = static_cast<size_t>(es);
+    hp.off_dt = align256(tok * 2 * D * e);
+    hp.off_b = hp.off_dt + align256(tok * D * e);
+    hp.off_c = hp.off_b + align256(tok * 16 * e);
+    hp.off_y = hp.off_c + align256(tok * 16 * e);
+    hp.slot = hp.off_y + align256(tok * D * e);
+    hp.carry_h = align256(static_cast<size_t>(batch) * D * 16 * 4);
+    hp.carry = hp.carry_h + align256(static_cast<size_t>(batch) * D * 3 * e);
+    // every piece but the last has hp.piece tokens; the scratch must fit both plans
+    const int64_t last = seqlen - (hp.pieces - 1) * hp.piece;
+    hp.fwd_ws = align256(std::max(plan_fwd(batch, hp.piece, d_inner).ws_bytes,
+                                  plan_fwd(batch, std::max<int64_t>(last, 0), d_inner).ws_bytes));
+    hp.total = 2 * hp.slot + 2 * hp.carry + hp.fwd_ws;
+    return hp;
+}
+
+// Events of one mamba_mixer_fwd_host call, destroyed when it returns (the
+// driver releases an event still pending once it completes).
+struct HostEvents {
+    cudaEvent_t ev[8] = {};
+    int n = 0;
+    cudaEvent_t make() {
+        cudaEvent_t e = nullptr;
+        if (n < 8 && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess) ev[n++] = e;
+        return e;
+    }
+    ~HostEvents() {
+        for (int i = 0; i < n; ++i) cudaEventDestroy(ev[i]);
+    }
+};
+
 }  // namespace
 
 // Scratch of mamba_mixer_fwd_noalloc: one fixed array per device in the
@@ -469,6 +525,153 @@ mm_status mamba_mixer_fwd_noalloc(const void* xz, const float* conv_w, const flo
     return mamba_mixer_fwd(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0, conv_state_in, y, h_last,
                            conv_state_out, batch, seqlen, d_inner, d_state, d_conv, act, scratch,
                            need > 0 ? MAMBA_MIXER_NOALLOC_SCRATCH_BYTES : 0, stream);
+}
+
+size_t mamba_mixer_host_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state,
+                                       int64_t d_conv, mm_dtype act) {
+    if ((act != MM_F32 && act != MM_BF16) || batch <= 0 || seqlen < 0 || d_inner <= 0 || d_state != 16 ||
+        d_conv != 4 || d_inner % 8 != 0 || d_inner > (1 << 24) || batch > (1 << 24))
+        return 0;
+    int64_t tokens, bytes;
+    if (!mul_ok(batch, seqlen, &tokens) || !mul_ok(tokens, 2 * d_inner * 4, &bytes)) return 0;
+    return plan_host(batch, seqlen, d_inner, act == MM_F32 ? 4 : 2).total;
+}
+
+mm_status mamba_mixer_fwd_host(const void* xz, const float* conv_w, const float* conv_b,
+                               const void* dt, const float* dt_bias, const float* A,
+                               const void* Bm, const void* Cm, const float* Dskip,
+                               const float* h0, const void* conv_state_in,
+                               void* y, float* h_last, void* conv_state_out,
+                               int64_t batch, int64_t seqlen, int64_t d_inner,
+                               int64_t d_state, int64_t d_conv, mm_dtype act,
+                               void* workspace, size_t workspace_bytes,
+                               void* stream, void* h2d_stream, void* d2h_stream)
+{
+    if (act != MM_F32 && act != MM_BF16) return MM_ERR_DTYPE;
+    if (batch < 0 || seqlen < 0 || d_inner <= 0 || d_state <= 0 || d_conv <= 0) return MM_ERR_SHAPE;
+    if (d_state != 16 || d_conv != 4 || d_inner % 8 != 0) return MM_ERR_UNSUPPORTED;
+    if (d_inner > (1 << 24) || batch > (1 << 24)) return MM_ERR_SHAPE;
+    const int64_t es = act == MM_F32 ? 4 : 2;
+    int64_t tokens, xz_bytes, dt_bytes, bc_bytes, st_bytes;
+    if (!mul_ok(batch, seqlen, &tokens) || !mul_ok(tokens, 2 * d_inner * es, &xz_bytes) ||
+        !mul_ok(tokens, d_inner * es, &dt_bytes) || !mul_ok(tokens, d_state * es, &bc_bytes) ||
+        !mul_ok(batch, d_inner * d_state * 4, &st_bytes))
+        return MM_ERR_SHAPE;
+    const int64_t cs_bytes = batch * d_inner * (d_conv - 1) * es;
+    if (batch == 0) return MM_OK;
+
+    if (!conv_w || !dt_bias || !A || !h_last || !conv_state_out) return MM_ERR_NULL;
+    if (seqlen > 0 && (!xz || !dt || !Bm || !Cm || !y)) return MM_ERR_NULL;
+    // device pointers and the workspace: 16-byte aligned (host buffers need not be)
+    const void* dev_ptrs[] = {conv_w, conv_b, dt_bias, A, Dskip};
+    for (const void* q : dev_ptrs)
+        if (q && !aligned16(q)) return MM_ERR_ALIGN;
+    // host outputs may not overlap host inputs
+    const Span in[] = {span(xz, xz_bytes), span(dt, dt_bytes), span(Bm, bc_bytes), span(Cm, bc_bytes),
+                       span(h0, st_bytes), span(conv_state_in, cs_bytes)};
+    const Span out[] = {span(y, dt_bytes), span(h_last, st_bytes), span(conv_state_out, cs_bytes)};
+    for (const Span& o : out)
+        for (const Span& i : in)
+            if (overlaps(o, i)) return MM_ERR_ALIAS;
+    if (overlaps(out[0], out[1]) || overlaps(out[0], out[2]) || overlaps(out[1], out[2])) return MM_ERR_ALIAS;
+
+    const HostPlan hp = plan_host(batch, seqlen, d_inner, es);
+    if (!workspace || workspace_bytes < hp.total) return MM_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MM_ERR_ALIGN;
+    int sm_count = 0;
+    if (mm_status st = check_device(&sm_count); st != MM_OK) return st;
+
+    cudaStream_t sc = static_cast<cudaStream_t>(stream);
+    cudaStream_t s_in = static_cast<cudaStream_t>(h2d_stream);
+    cudaStream_t s_out = static_cast<cudaStream_t>(d2h_stream);
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    unsigned char* slot[2] = {ws, ws + hp.slot};
+    unsigned char* carry[2] = {ws + 2 * hp.slot, ws + 2 * hp.slot + hp.carry};
+    void* fwd_ws = hp.fwd_ws ? ws + 2 * hp.slot + 2 * hp.carry : nullptr;
+
+    HostEvents evs;
+    cudaEvent_t ev_start = evs.make(), ev_final = evs.make();
+    cudaEvent_t ev_in[2] = {evs.make(), evs.make()};
+    cudaEvent_t ev_done[2] = {evs.make(), evs.make()};
+    cudaEvent_t ev_free[2] = {evs.make(), evs.make()};
+    if (evs.n != 8) { cudaGetLastError(); return MM_ERR_CUDA; }
+
+    bool ok = true;
+    mm_status fwd_status = MM_OK;
+    auto chk = [&](cudaError_t e) { ok = ok && e == cudaSuccess; };
+    const size_t B = static_cast<size_t>(batch), D = static_cast<size_t>(d_inner), e = static_cast<size_t>(es);
+    const size_t L = static_cast<size_t>(seqlen);
+    const unsigned char* xz_h = static_cast<const unsigned char*>(xz);
+    const unsigned char* dt_h = static_cast<const unsigned char*>(dt);
+    const unsigned char* b_h = static_cast<const unsigned char*>(Bm);
+    const unsigned char* c_h = static_cast<const unsigned char*>(Cm);
+    unsigned char* y_h = static_cast<unsigned char*>(y);
+
+    // the copies touch the workspace, which the caller's earlier work on `stream` may still use
+    chk(cudaEventRecord(ev_start, sc));
+    chk(cudaStreamWaitEvent(s_in, ev_start, 0));
+    chk(cudaStreamWaitEvent(s_out, ev_start, 0));
+    if (h0) chk(cudaMemcpyAsync(carry[0], h0, static_cast<size_t>(st_bytes), cudaMemcpyHostToDevice, s_in));
+    if (conv_state_in)
+        chk(cudaMemcpyAsync(carry[0] + hp.carry_h, conv_state_in, static_cast<size_t>(cs_bytes),
+                            cudaMemcpyHostToDevice, s_in));
+
+    for (int64_t i = 0; ok && i < hp.pieces; ++i) {
+        const int j = static_cast<int>(i & 1);
+        const size_t t0 = static_cast<size_t>(i * hp.piece);
+        const size_t n = static_cast<size_t>(std::min<int64_t>(hp.piece, seqlen - i * hp.piece));
+        unsigned char* sl = slot[j];
+        // inputs of piece i -> slot j, once the piece that used the slot has been copied out
+        if (i >= 2) chk(cudaStreamWaitEvent(s_in, ev_free[j], 0));
+        if (n > 0) {
+            chk(cudaMemcpy2DAsync(sl, n * 2 * D * e, xz_h + t0 * 2 * D * e, L * 2 * D * e, n * 2 * D * e, B,
+                                  cudaMemcpyHostToDevice, s_in));
+            chk(cudaMemcpy2DAsync(sl + hp.off_dt, n * D * e, dt_h + t0 * D * e, L * D * e, n * D * e, B,
+                                  cudaMemcpyHostToDevice, s_in));
+            chk(cudaMemcpy2DAsync(sl + hp.off_b, n * 16 * e, b_h + t0 * 16 * e, L * 16 * e, n * 16 * e, B,
+                                  cudaMemcpyHostToDevice, s_in));
+            chk(cudaMemcpy2DAsync(sl + hp.off_c, n * 16 * e, c_h + t0 * 16 * e, L * 16 * e, n * 16 * e, B,
+                                  cudaMemcpyHostToDevice, s_in));
+        }
+        chk(cudaEventRecord(ev_in[j], s_in));
+        // the forward of piece i, carrying the state from piece i-1
+        chk(cudaStreamWaitEvent(sc, ev_in[j], 0));
+        unsigned char* cin = carry[i & 1];
+        unsigned char* cout = carry[(i + 1) & 1];
+        const bool first = i == 0;
+        const float* h_in = (first && !h0) ? nullptr : reinterpret_cast<const float*>(cin);
+        const void* cs_in = (first && !conv_state_in) ? nullptr : cin + hp.carry_h;
+        if (!ok) break;
+        fwd_status = mamba_mixer_fwd(sl, conv_w, conv_b, sl + hp.off_dt, dt_bias, A, sl + hp.off_b,
+                                             sl + hp.off_c, Dskip, h_in, cs_in, sl + hp.off_y,
+                                             reinterpret_cast<float*>(cout), cout + hp.carry_h, batch,
+                                             static_cast<int64_t>(n), d_inner, d_state, d_conv, act, fwd_ws,
+                                             hp.fwd_ws, sc);
+        if (fwd_status != MM_OK) break;
+        chk(cudaEventRecord(ev_done[j], sc));
+        // y of piece i -> host; the slot is free again after this copy
+        chk(cudaStreamWaitEvent(s_out, ev_done[j], 0));
+        if (n > 0)
+            chk(cudaMemcpy2DAsync(y_h + t0 * D * e, L * D * e, sl + hp.off_y, n * D * e, n * D * e, B,
+                                  cudaMemcpyDeviceToHost, s_out));
+        chk(cudaEventRecord(ev_free[j], s_out));
+    }
+    // the carried state after the last piece -> host; `stream` then waits for every
+    // copy queued so far (also after a failure, so the caller can sync `stream`
+    // before releasing its buffers)
+    if (ok && fwd_status == MM_OK) {
+        unsigned char* cl = carry[hp.pieces & 1];
+        chk(cudaMemcpyAsync(h_last, cl, static_cast<size_t>(st_bytes), cudaMemcpyDeviceToHost, s_out));
+        chk(cudaMemcpyAsync(conv_state_out, cl + hp.carry_h, static_cast<size_t>(cs_bytes),
+                            cudaMemcpyDeviceToHost, s_out));
+    }
+    const bool fenced = cudaEventRecord(ev_final, s_out) == cudaSuccess &&
+                        cudaEventRecord(ev_in[0], s_in) == cudaSuccess &&
+                        cudaStreamWaitEvent(sc, ev_final, 0) == cudaSuccess &&
+                        cudaStreamWaitEvent(sc, ev_in[0], 0) == cudaSuccess;
+    if (fwd_status != MM_OK) return fwd_status;
+    if (!ok || !fenced) { cudaGetLastError(); return MM_ERR_CUDA; }
+    return MM_OK;
 }
 
 }  // extern "C"

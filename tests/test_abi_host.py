@@ -260,3 +260,44 @@ def test_noalloc_validates_like_the_forward(L):
     bad[0] = None                             # xz
     assert L.mamba_mixer_fwd_noalloc(*bad) == ENULL
     assert L.mamba_mixer_fwd_noalloc(*noalloc) in (EDEVICE, OK, ECUDA)
+
+
+# ---------------------------------------------------------------- host-memory forward
+def host_args(B=1, Lq=64, D=64, ws=None, ws_bytes=0, **over):
+    """mamba_mixer_fwd_host arguments over fake addresses (the same layout as
+    fwd_args, reused for host and device buffers alike)."""
+    a = fwd_args(B=B, Lq=Lq, D=D, **over)
+    return a[:-3] + [ws, ws_bytes, None, None, None]
+
+
+def test_host_workspace_size_rules():
+    need = mm.host_workspace_size(1, 4096, 8192)
+    # two staging slots of one 512-token piece (xz, dt, B, C, y in bf16) plus
+    # two carried states and the piece forward's scratch
+    piece_bytes = 512 * (2 * 8192 + 8192 + 16 + 16 + 8192) * 2
+    assert need >= 2 * piece_bytes + 2 * 8192 * (16 * 4 + 3 * 2)
+    assert need < 2 * piece_bytes + (16 << 20)
+    assert mm.host_workspace_size(1, 0, 64) > 0           # an empty sequence still carries its state
+    assert mm.host_workspace_size(1, 4096, 60) == 0       # d_inner % 8 != 0
+    assert mm.host_workspace_size(0, 4096, 64) == 0
+    assert mm.host_workspace_size(1, 4096, 64, act=7) == 0
+
+
+def test_host_fwd_validates_before_any_copy(L):
+    need = mm.host_workspace_size(2, 1000, 64)
+    ws = BASE + (1 << 36)
+    assert L.mamba_mixer_fwd_host(*host_args(B=2, Lq=1000, ws=ws, ws_bytes=need, xz=None)) == ENULL
+    assert L.mamba_mixer_fwd_host(*host_args(B=2, Lq=1000, ws=ws, ws_bytes=need, act=5)) == EDTYPE
+    assert L.mamba_mixer_fwd_host(*host_args(B=2, Lq=1000, ws=ws, ws_bytes=need - 1)) == EWORKSPACE
+    assert L.mamba_mixer_fwd_host(*host_args(B=2, Lq=1000, ws=None, ws_bytes=0)) == EWORKSPACE
+    assert L.mamba_mixer_fwd_host(*host_args(B=2, Lq=1000, ws=ws + 8, ws_bytes=need)) == EALIGN
+    # device parameters must be aligned; host activations need not be
+    assert L.mamba_mixer_fwd_host(*host_args(B=2, Lq=1000, ws=ws, ws_bytes=need, A=BASE + 4)) == EALIGN
+    args = host_args(B=2, Lq=1000, ws=ws, ws_bytes=need)
+    args[0] += 2                                          # unaligned host xz: still accepted
+    assert L.mamba_mixer_fwd_host(*args) in (EDEVICE, OK, ECUDA)
+    # a host output overlapping a host input
+    args = host_args(B=2, Lq=1000, ws=ws, ws_bytes=need)
+    args[11] = args[0]                                    # y over xz
+    assert L.mamba_mixer_fwd_host(*args) == EALIAS
+    assert L.mamba_mixer_fwd_host(*host_args(B=0, Lq=1000, ws=None, ws_bytes=0)) == OK
