@@ -149,8 +149,15 @@ __device__ __forceinline__ float2 silu2(float2 v) {
 
 template <typename M>
 __device__ __forceinline__ float2 step_pair(float2 dt, float2 bias) {
-    if constexpr (M::step_scale == 1.0f) return f2(M::step(dt.x, bias.x), M::step(dt.y, bias.y));
-    else return f2(M::step2(dt.x, bias.x), M::step2(dt.y, bias.y));
+    if constexpr (M::step_scale == 1.0f) {
+        return f2(M::step(dt.x, bias.x), M::step(dt.y, bias.y));
+    } else {
+        // MathFast::step2 on both channels, with the affine steps packed:
+        // v2 = dt log2(e) + bias2, l = max(log2(1 + 2^min(v2, 126)), v2)
+        const float2 v2 = fma2(dt, f2(kLog2e, kLog2e), bias);
+        const float2 e = __fadd2_rn(f2(ex2_fast(fminf(v2.x, 126.0f)), ex2_fast(fminf(v2.y, 126.0f))), f2(1.f, 1.f));
+        return f2(fmaxf(lg2_fast(e.x), v2.x), fmaxf(lg2_fast(e.y), v2.y));
+    }
 }
 
 template <typename M>
@@ -325,7 +332,10 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
             float2 l = step_pair<M>(P_::load(ds + (r0 + m) * rs + cls), bias2);
             if (m >= nvalid) l = f2(0.f, 0.f);                  // past the chunk: no step
             const float2 s = mul2(l, u);                         // Delta*u in B' units (B' = B * step_scale)
-            if constexpr (!SUMMARY && kStruct) ea[m] = f2(ex2_fast(l.x * A02.x), ex2_fast(l.y * A02.y));   // q
+            if constexpr (!SUMMARY && kStruct) {
+                const float2 la = mul2(l, A02);
+                ea[m] = f2(ex2_fast(la.x), ex2_fast(la.y));   // q
+            }
             else ea[m] = l;
             sa[m] = s;
             ua[m] = u;
@@ -348,7 +358,8 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
                 if constexpr (kStruct) {
                     // weights w[n] = s r^(n+1) as four interleaved chains (step r^4),
                     // so no chain is longer than six multiplies
-                    const float2 r = f2(ex2_fast(R[m].x * A02.x), ex2_fast(R[m].y * A02.y));
+                    const float2 ra = mul2(R[m], A02);
+                    const float2 r = f2(ex2_fast(ra.x), ex2_fast(ra.y));
                     const float2 r2 = mul2(r, r);
                     const float2 r4 = mul2(r2, r2);
                     float2 w[4];
@@ -414,11 +425,12 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
             }
 
             // ---- C: skip, gate, store
+            T* yrow = yg + (seq_row0 + t0) * D + d;
 #pragma unroll
             for (int m = 0; m < SUB; ++m) {
                 const float2 g = silu2<M>(P_::load(zs + (r0 + m) * rs + cls));
                 const float2 yv = mul2(fma2(dsk2, ua[m], yacc[m]), g);
-                if (m < nvalid && active) P_::store(yg + (seq_row0 + t0 + m) * D + d, yv);
+                if (m < nvalid && active) P_::store(yrow + m * D, yv);
             }
         }
     };
