@@ -63,7 +63,10 @@
 #include "mixer_common.cuh"
 
 #ifndef MM_SUB
-#define MM_SUB 8               // tokens per sub-tile
+#define MM_SUB 8               // tokens per sub-tile (full pass)
+#endif
+#ifndef MM_SUB_SUMMARY
+#define MM_SUB_SUMMARY 16      // tokens per sub-tile (summary pass: fewer live arrays, more chains)
 #endif
 #ifndef MM_FWD_MIN_BLOCKS
 #define MM_FWD_MIN_BLOCKS 2    // resident CTAs of 128 threads per SM the register budget must allow
@@ -173,7 +176,7 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
                  const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_dt,
                  const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c)
 {
-    constexpr int SUB = MM_SUB;
+    constexpr int SUB = SUMMARY ? MM_SUB_SUMMARY : MM_SUB;
     static_assert(TILE % SUB == 0, "tile");
     constexpr bool kFast = (M::step_scale != 1.0f);
     using A_ = Act<T>;
@@ -253,7 +256,13 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
         if (p.Dskip) dsk2 = *reinterpret_cast<const float2*>(p.Dskip + d);
         A02 = f2(p.A[static_cast<int64_t>(d) * 16], p.A[static_cast<int64_t>(d + 1) * 16]);
     }
-    if constexpr (kFast) bias2 = mul2(bias2, f2(kLog2e, kLog2e));
+    if constexpr (kFast) {
+        bias2 = mul2(bias2, f2(kLog2e, kLog2e));
+        // the conv yields v/2, the argument SiLU's tanh form needs (exact: a power-of-2 scale)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) w2[k] = mul2(w2[k], f2(0.5f, 0.5f));
+        cb2 = mul2(cb2, f2(0.5f, 0.5f));
+    }
     const float* arow0 = p.A + static_cast<int64_t>(d) * 16;
     const float* arow1 = arow0 + 16;
 
@@ -328,7 +337,9 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
             float2 pre = cb2;
 #pragma unroll
             for (int k = 0; k < 4; ++k) pre = fma2(w2[k], xw[m + k], pre);
-            const float2 u = silu2<M>(pre);
+            float2 u;
+            if constexpr (kFast) u = fma2(pre, f2(tanh_fast(pre.x), tanh_fast(pre.y)), pre);   // pre = v/2
+            else u = silu2<M>(pre);
             float2 l = step_pair<M>(P_::load(ds + (r0 + m) * rs + cls), bias2);
             if (m >= nvalid) l = f2(0.f, 0.f);                  // past the chunk: no step
             const float2 s = mul2(l, u);                         // Delta*u in B' units (B' = B * step_scale)
