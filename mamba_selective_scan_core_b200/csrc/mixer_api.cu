@@ -91,25 +91,43 @@ unsigned copy_wait_limit() {
     return 1u << 20;
 }
 
-// Time chunks: as many as the SMs' resident warp slots hold in one wave
-// (two channels per thread, so a sequence of D channels is D/64 warps per
-// chunk); a second, partial wave would cost more than the idle slots.
+// Time chunks.  More chunks put more warps on the SMs but add a summary pass
+// over (K-1)/K of the tokens, so K minimises a measured cost model: a pass
+// takes about (tokens per chunk) x (time of its busiest SM), an SM running
+// 8 warps (two CTAs) taking ~1.85x as long as one running 4, and a summary
+// token costing ~0.55 of a full-pass token (B200 measurements of both
+// kernels), among splits that fit one wave.  It picks 9 chunks for one
+// 8192-channel sequence and a single chunk once a batch fills the SMs on
+// its own.
+double busiest_sm(int64_t warps) {
+    const int64_t m = (warps + kPlanSMs - 1) / kPlanSMs;        // warps on the busiest SM
+    const int64_t waves = m / kWarpsPerSM, rest = m % kWarpsPerSM;
+    return 1.85 * static_cast<double>(waves) + (rest == 0 ? 0.0 : rest * 2 <= kWarpsPerSM ? 1.0 : 1.85);
+}
+
 FwdPlan plan_fwd(int64_t batch, int64_t seqlen, int64_t d_inner) {
     FwdPlan pl;
-    const int64_t warps = std::max<int64_t>(1, batch * d_inner / 2 / 32);
-    const int64_t slots = static_cast<int64_t>(kPlanSMs) * kWarpsPerSM;
-    const int64_t tiles = (seqlen + kTile - 1) / kTile;
+    const int64_t warps = std::max<int64_t>(1, batch * ((d_inner / 2 + 31) / 32));   // per chunk
+    const int64_t tiles = std::max<int64_t>(1, (seqlen + kTile - 1) / kTile);
+    auto chunk_tiles = [&](int64_t k) { return (tiles + k - 1) / k; };
     int64_t k = 1;
     if (const int forced = env_int("MAMBA_MIXER_CHUNKS", 1, 1 << 20)) {
-        k = forced;
-    } else if (2 * warps <= slots) {
-        k = slots / warps;
-        k = std::min<int64_t>(k, std::max<int64_t>(1, tiles / kMinChunkTiles));
-        k = std::min<int64_t>(k, kMaxChunks);
+        k = std::min<int64_t>(forced, tiles);
+    } else {
+        double best = 0.0;
+        const int64_t kmax = std::min<int64_t>(kMaxChunks, std::max<int64_t>(1, tiles / kMinChunkTiles));
+        for (int64_t c = 1; c <= kmax; ++c) {
+            const int64_t ct = chunk_tiles(c);
+            const int64_t chunks = (tiles + ct - 1) / ct;            // chunks the split really makes
+            // a split stays within one wave of resident warps (the model does not
+            // charge what grows with the chunk count: carry chains, pipeline fills)
+            if (chunks > 1 && chunks * warps > static_cast<int64_t>(kPlanSMs) * kWarpsPerSM) break;
+            const double cost = static_cast<double>(ct) *
+                                (busiest_sm(chunks * warps) + (chunks > 1 ? 0.55 * busiest_sm((chunks - 1) * warps) : 0.0));
+            if (c == 1 || cost < best) { best = cost; k = c; }
+        }
     }
-    k = std::max<int64_t>(1, std::min<int64_t>(k, std::max<int64_t>(tiles, 1)));
-    const int64_t tiles_per_chunk = (tiles + k - 1) / k;
-    pl.chunk_len = std::max<int64_t>(1, tiles_per_chunk) * kTile;
+    pl.chunk_len = chunk_tiles(k) * kTile;
     pl.chunks = static_cast<int>(seqlen > 0 ? (seqlen + pl.chunk_len - 1) / pl.chunk_len : 1);
     if (pl.chunks > 1)
         pl.ws_bytes = static_cast<size_t>(pl.chunks - 1) * batch * d_inner * (16 + 1) * sizeof(float);

@@ -52,12 +52,15 @@ def test_version_and_strings(L):
         s = mm.status_string(code)
         assert s and s != "unknown status"
     assert mm.status_string(99) == "unknown status"
-    # one 8192-channel sequence (128 warps of channel pairs) is split into as
-    # many time chunks as 148 SMs x 8 warps hold at once: 9 chunks of 480
-    # tokens, 8 carried states of 17 floats per channel
+    # one 8192-channel sequence (128 warps of channel pairs) is split into 9
+    # time chunks of 480 tokens: 8 carried states of 17 floats per channel
     assert mm.workspace_size(1, 4096, 8192) == 8 * 8192 * 17 * 4
-    # four such sequences into 2 chunks
-    assert mm.workspace_size(4, 32768, 8192) == 1 * 4 * 8192 * 17 * 4
+    # two such sequences: 4 chunks; three: 3 chunks
+    assert mm.workspace_size(2, 4096, 8192) == 3 * 2 * 8192 * 17 * 4
+    assert mm.workspace_size(3, 4096, 8192) == 2 * 3 * 8192 * 17 * 4
+    # four: one chunk (their 512 warps fill the SMs well enough that a summary
+    # pass over half the tokens would cost more than it gains)
+    assert mm.workspace_size(4, 32768, 8192) == 0
     # enough sequences need no time chunks and no workspace
     assert mm.workspace_size(8, 4096, 8192) == 0
     assert mm.workspace_size(1, 4096, 8192, act=5) == 0
