@@ -266,7 +266,7 @@ cudaError_t dispatch_prefill(PrefillParams p, int64_t batch, const FwdPlan& pl, 
 // kHostPieces pieces (whole tiles, at least kHostMinPiece tokens) and the
 // device workspace holds two staging slots, two carried states (ping-pong)
 // and the piece forward's own scratch, each region 256-byte aligned.
-constexpr int64_t kHostPieces = 16;
+constexpr int64_t kHostPieces = 8;
 constexpr int64_t kHostMinPiece = 256;
 
 struct HostPlan {

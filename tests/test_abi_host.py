@@ -275,9 +275,9 @@ def host_args(B=1, Lq=64, D=64, ws=None, ws_bytes=0, **over):
 
 def test_host_workspace_size_rules():
     need = mm.host_workspace_size(1, 4096, 8192)
-    # two staging slots of one 256-token piece (xz, dt, B, C, y in bf16) plus
+    # two staging slots of one 512-token piece (xz, dt, B, C, y in bf16) plus
     # two carried states and the piece forward's scratch
-    piece_bytes = 256 * (2 * 8192 + 8192 + 16 + 16 + 8192) * 2
+    piece_bytes = 512 * (2 * 8192 + 8192 + 16 + 16 + 8192) * 2
     assert need >= 2 * piece_bytes + 2 * 8192 * (16 * 4 + 3 * 2)
     assert need < 2 * piece_bytes + (16 << 20)
     assert mm.host_workspace_size(1, 0, 64) > 0           # an empty sequence still carries its state
