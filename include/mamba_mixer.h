@@ -1,11 +1,15 @@
 /*
  * mamba_mixer.h -- C ABI of the B200 (sm_100a) Mamba mixer core.
  *
- * Two operations, both on device memory the caller owns, both asynchronous on
- * a CUDA stream the caller chooses:
+ * Two operations, both asynchronous on a CUDA stream the caller chooses:
  *
  *   mamba_mixer_fwd      selective-scan forward over a whole sequence (prefill)
  *   mamba_state_update   the one-token state update used in decode
+ *
+ * and three ways into the forward beyond the plain call:
+ *   mamba_mixer_fwd_noalloc  no workspace argument (a fixed scratch array inside the library)
+ *   mamba_mixer_fwd_host     activations in host memory, copies overlapped with the compute
+ *   mamba_mixer_fault_status the device word a kernel sets if it gives up on a bounded wait
  *
  * What they compute.  The Jamba hybrid SSM-Transformer lesson (section "SSM in
  * one page") gives the recurrence h_t = A h_{t-1} + B x_t, y_t = C h_t, notes
@@ -28,15 +32,17 @@
  *
  * Conventions for every entry point:
  *   - Pointers are device (or managed) addresses, 16-byte aligned, dense
- *     row-major with the last dimension contiguous.  Host pointers are not
- *     accepted; the caller copies host data in first.
+ *     row-major with the last dimension contiguous -- except the activations
+ *     of mamba_mixer_fwd_host, which are host addresses.
  *   - "act" tensors hold MM_F32 floats or MM_BF16 bfloat16 values; parameters
  *     and the SSM state are always fp32.
  *   - Supported sizes: d_state == 16, d_conv == 4, d_inner a multiple of 8.
  *   - Validation happens on the host before anything is launched; a rejected
  *     call launches nothing and writes nothing.  A launch failure reported by
  *     the CUDA runtime returns MM_ERR_CUDA (the runtime's error is cleared).
- *   - The library allocates no memory and keeps no state between calls.
+ *   - The library allocates no device memory; the caller passes every buffer
+ *     and scratch area.  Its only state between calls is the device fault
+ *     word and the fixed scratch array of mamba_mixer_fwd_noalloc.
  *     Calls only enqueue work: results are valid once the stream reaches them.
  *   - Kernels never assert or trap.
  */

@@ -25,7 +25,9 @@
 //     packed multiply per state instead of 16 ex2 on the 16/clk MUFU pipe;
 //   * B_t/C_t, shared by every channel of a sequence, are staged once per CTA
 //     and tile in shared memory, each value duplicated into a pair, so one
-//     16-byte load feeds two states of both channels.
+//     16-byte load feeds two states of both channels;
+//   * in the bf16 path SiLU is h + h tanh(h) with h = v/2 (one MUFU op), and
+//     the conv weights are halved once so the conv yields v/2 directly.
 //
 // Parallelism.  The recurrence is sequential in t per channel: a single
 // 8192-channel sequence is only 4096 channel pairs, 128 warps.  Time chunks
@@ -37,8 +39,9 @@
 // and runs the fused forward.  The summary pass skips the readout, the gate
 // and the z/C traffic, and walks its chunk backward: e_c[n] is the sum over
 // tokens of s_t B_t[n] exp(A[n] R_t), R_t the steps after token t, so with
-// structured A a token costs a 16-step multiply chain and 16 FMAs instead of
-// the forward recurrence's 15 decay powers, 16 products and 16 FMAs.
+// structured A a token's weights s r^(n+1) cost 18 packed multiplies (four
+// short chains) and 16 FMAs instead of the forward recurrence's 15 decay
+// powers, 16 products and 16 FMAs.
 //
 // Latency: each tile is processed in sub-tiles of SUB tokens in three phases
 // so that the long per-token chains (conv -> SiLU -> softplus -> exp) of SUB
