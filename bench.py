@@ -80,15 +80,23 @@ def _measured_peaks():
 
 
 def _kernel_source_sha():
-    """Hash of the CUDA sources (kernels and launch plan) the traffic figures depend on."""
+    """Hash of the CUDA sources (kernels and launch plan) the traffic figures
+    depend on, with comments and blank space stripped so that only code
+    changes invalidate a capture."""
+    import re
+
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mamba_selective_scan_core_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if not name.endswith((".cuh", ".cu")):
             continue
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode())
-            h.update(f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            src = f.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        src = "\n".join(line.strip() for line in src.splitlines() if line.strip())
+        h.update(name.encode())
+        h.update(src.encode())
     return h.hexdigest()[:16]
 
 
