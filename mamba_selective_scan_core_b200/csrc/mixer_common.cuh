@@ -1,6 +1,7 @@
 // Device helpers shared by the prefill and decode kernels of the Mamba mixer
-// core: activation loads/stores, the two math flavours (exact and fast), and
-// small packed-fp32 helpers for sm_100a.
+// core: activation loads/stores, the two math flavours (exact and fast),
+// small packed-fp32 helpers, and the mbarrier / bulk-tensor-copy wrappers the
+// forward stages its tiles with.
 #pragma once
 
 #include <cstdint>
@@ -94,19 +95,10 @@ __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 
-// ---------------------------------------------------------------- async copy
+// ---------------------------------------------------------------- shared memory
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-// 16-byte global -> shared copy; src_bytes == 0 zero-fills the destination
-// without reading (src must still be a valid address form).
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n"
-                 :: "r"(smem_addr(dst)), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" :: "n"(N) : "memory"); }
 
 }  // namespace mm
 
