@@ -132,6 +132,25 @@ def test_batched_prefill_workload_sampled():
     check_fwd(inp, "bf16", chans=sample_channels(cfg.d_inner, 128))
 
 
+@pytest.mark.parametrize("B,chunks", [(2, 4), (3, 3)])
+def test_multi_sequence_chunk_plans_sampled(B, chunks):
+    """Two and three Jamba-shaped sequences at full size, with the launch
+    plans the planner picks for them (4 and 3 time chunks: the carried state
+    crosses chunk boundaries inside every sequence of the batch)."""
+    assert mm.workspace_size(B, 4096, 8192) == (chunks - 1) * B * 8192 * 17 * 4
+    inp = make_mixer_inputs_custom(B, 4096, 8192, act="bf16", seed=80 + B, h0_std=0.1, conv_state_std=1.0)
+    check_fwd(inp, "bf16", chans=sample_channels(8192, 64))
+
+
+@pytest.mark.parametrize("act", ["bf16", "f32"])
+def test_narrow_sequence_sixteen_chunks(act):
+    """64 channels x 4096 tokens: the default plan takes the maximum 16 time
+    chunks (a 15-step carry chain), checked against the oracle in full."""
+    assert mm.workspace_size(1, 4096, 64) == 15 * 64 * 17 * 4
+    inp = make_mixer_inputs_custom(1, 4096, 64, act=act, seed=91, h0_std=0.3, conv_state_std=1.0)
+    check_fwd(inp, act)
+
+
 def _run_carried(dev, n, D):
     L = dev["xz"].shape[1]
     step = L // n
