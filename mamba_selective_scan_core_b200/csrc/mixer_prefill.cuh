@@ -98,7 +98,7 @@ struct PrefillParams {
     int ctas_per_seq;   // CTAs per sequence
     int64_t chunk_len;  // tokens per time chunk (a multiple of the tile)
     int n_chunks;       // time chunks K (blockIdx.y of the full pass)
-    float* ws_state;    // [K-1][batch][D][16]: end state of chunk c run from zero
+    float* ws_state;    // [K-1][batch][16][D]: end state of chunk c run from zero (state-major)
     float* ws_lsum;     // [K-1][batch][D]:     sum over chunk c of the step size l
     int batch;
     unsigned wait_limit;  // tries per wait on a bulk copy before giving up (fault)
@@ -245,6 +245,18 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
         }
     };
 
+    // ---------------------------------------------------------- pipeline prologue (the first tiles stream in during the setup)
+    if (tid == 0) {
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s) mbar_init(&bars[s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+#pragma unroll 1
+        for (int s = 0; s < STAGES - 1; ++s) issue_tile(s);
+    }
+
     // ---------------------------------------------------------- per-thread setup
     float2 w2[4];
 #pragma unroll
@@ -257,7 +269,6 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
         if (p.conv_b) cb2 = *reinterpret_cast<const float2*>(p.conv_b + d);
         bias2 = *reinterpret_cast<const float2*>(p.dt_bias + d);
         if (p.Dskip) dsk2 = *reinterpret_cast<const float2*>(p.Dskip + d);
-        A02 = f2(p.A[static_cast<int64_t>(d) * 16], p.A[static_cast<int64_t>(d + 1) * 16]);
     }
     if constexpr (kFast) {
         bias2 = mul2(bias2, f2(kLog2e, kLog2e));
@@ -266,8 +277,21 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
         for (int k = 0; k < 4; ++k) w2[k] = mul2(w2[k], f2(0.5f, 0.5f));
         cb2 = mul2(cb2, f2(0.5f, 0.5f));
     }
-    const float* arow0 = p.A + static_cast<int64_t>(d) * 16;
-    const float* arow1 = arow0 + 16;
+    // A pairs a2[n] = (A[d][n], A[d+1][n]): my two A rows are 128 contiguous
+    // bytes, read in 16-byte loads (a warp-wide scalar load here would touch
+    // 32 lines per instruction)
+    float2 a2[16];
+    {
+        float av[32];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4*>(av + 4 * q) =
+                active ? __ldg(reinterpret_cast<const float4*>(p.A + static_cast<int64_t>(d) * 16) + q)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int n = 0; n < 16; ++n) a2[n] = f2(av[n], av[16 + n]);
+    }
+    A02 = a2[0];
 
     // state pairs h[n] = (h_d[n], h_{d+1}[n]), at the start of this chunk
     float2 h[16];
@@ -275,20 +299,31 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
 #pragma unroll
         for (int n = 0; n < 16; ++n) h[n] = f2(0.f, 0.f);
     } else {
-        const float* h0 = (p.h0 && active) ? p.h0 + chan * 16 : nullptr;
+        if (p.h0 && active) {
+            float hv[32];   // my two channels' rows of h0: 128 contiguous bytes
 #pragma unroll
-        for (int n = 0; n < 16; ++n) h[n] = h0 ? f2(h0[n], h0[16 + n]) : f2(0.f, 0.f);
+            for (int q = 0; q < 8; ++q)
+                *reinterpret_cast<float4*>(hv + 4 * q) = reinterpret_cast<const float4*>(p.h0 + chan * 16)[q];
+#pragma unroll
+            for (int n = 0; n < 16; ++n) h[n] = f2(hv[n], hv[16 + n]);
+        } else {
+#pragma unroll
+            for (int n = 0; n < 16; ++n) h[n] = f2(0.f, 0.f);
+        }
         // carry h0 through the summaries of the chunks before this one:
-        // h <- exp(A sum Delta) h + e
+        // h <- exp(A sum Delta) h + e, the summaries read state-major so that
+        // a warp's loads of one state are contiguous
         if (active && chunk > 0) {
             const int64_t stride = static_cast<int64_t>(p.batch) * D;
 #pragma unroll 1
             for (int c = 0; c < chunk; ++c) {
                 const float2 ls = *reinterpret_cast<const float2*>(p.ws_lsum + c * stride + chan);
-                const float* e0 = p.ws_state + (c * stride + chan) * 16;
+                const float* e = p.ws_state + (c * stride + static_cast<int64_t>(seq) * D) * 16 + d;
+                float2 ev[16];
 #pragma unroll
-                for (int n = 0; n < 16; ++n)
-                    h[n] = fma2(decay2<M>(ls, f2(arow0[n], arow1[n])), h[n], f2(e0[n], e0[16 + n]));
+                for (int n = 0; n < 16; ++n) ev[n] = *reinterpret_cast<const float2*>(e + static_cast<int64_t>(n) * D);
+#pragma unroll
+                for (int n = 0; n < 16; ++n) h[n] = fma2(decay2<M>(ls, a2[n]), h[n], ev[n]);
             }
         }
     }
@@ -301,21 +336,9 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
         if (active) {
 #pragma unroll
             for (int n = 0; n < 16; ++n)
-                mine = mine && arow0[n] == static_cast<float>(n + 1) * A02.x && arow1[n] == static_cast<float>(n + 1) * A02.y;
+                mine &= (a2[n].x == static_cast<float>(n + 1) * A02.x) & (a2[n].y == static_cast<float>(n + 1) * A02.y);
         }
         structured = __all_sync(kFull, mine);
-    }
-
-    // ---------------------------------------------------------- pipeline prologue
-    if (tid == 0) {
-#pragma unroll
-        for (int s = 0; s < STAGES; ++s) mbar_init(&bars[s], 1);
-        fence_mbar_init();
-    }
-    __syncthreads();
-    if (tid == 0) {
-#pragma unroll 1
-        for (int s = 0; s < STAGES - 1; ++s) issue_tile(s);
     }
 
     T* yg = static_cast<T*>(p.y);
@@ -505,9 +528,6 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
     if (structured) {
         completed = main_loop(std::true_type{}, nullptr);
     } else {
-        float2 a2[16];
-#pragma unroll
-        for (int n = 0; n < 16; ++n) a2[n] = active ? f2(arow0[n], arow1[n]) : f2(0.f, 0.f);
         completed = main_loop(std::false_type{}, a2);
     }
     if (!completed) return;
@@ -516,15 +536,19 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
     if constexpr (SUMMARY) {
         if (active) {
             const int64_t stride = static_cast<int64_t>(p.batch) * D;
-            float* e = p.ws_state + (chunk * stride + chan) * 16;
+            float* e = p.ws_state + (chunk * stride + static_cast<int64_t>(seq) * D) * 16 + d;
 #pragma unroll
-            for (int n = 0; n < 16; ++n) { e[n] = h[n].x; e[16 + n] = h[n].y; }
+            for (int n = 0; n < 16; ++n) *reinterpret_cast<float2*>(e + static_cast<int64_t>(n) * D) = h[n];
             *reinterpret_cast<float2*>(p.ws_lsum + chunk * stride + chan) = lsum;
         }
     } else if (active && chunk == p.n_chunks - 1) {
-        float* hl = p.h_last + chan * 16;
+        // my two channels' rows of h_last: 128 contiguous bytes, in 16-byte stores
+        float4* hl = reinterpret_cast<float4*>(p.h_last + chan * 16);
 #pragma unroll
-        for (int n = 0; n < 16; ++n) { hl[n] = h[n].x; hl[16 + n] = h[n].y; }
+        for (int q = 0; q < 4; ++q) {
+            hl[q] = make_float4(h[4 * q].x, h[4 * q + 1].x, h[4 * q + 2].x, h[4 * q + 3].x);
+            hl[4 + q] = make_float4(h[4 * q].y, h[4 * q + 1].y, h[4 * q + 2].y, h[4 * q + 3].y);
+        }
         // the last 3 raw x of both channels, shifted in from the incoming window when L < 3
         T* cso = static_cast<T*>(p.cs_out) + chan * 3;
 #pragma unroll
