@@ -44,6 +44,9 @@
  *     and scratch area.  Its only state between calls is the device fault
  *     word and the fixed scratch array of mamba_mixer_fwd_noalloc.
  *     Calls only enqueue work: results are valid once the stream reaches them.
+ *     A call starts after all earlier work in its stream and is complete
+ *     before later work starts.  Within a time-chunked forward call, the
+ *     second launch overlaps the first's tail (programmatic dependent launch).
  *   - Kernels never assert or trap.
  */
 #ifndef MAMBA_MIXER_H

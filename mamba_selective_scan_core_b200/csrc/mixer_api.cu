@@ -185,16 +185,29 @@ bool make_maps(const PrefillParams& p, int64_t batch, TensorMaps* m) {
            encode_3d(&m->c, p.Cm, bf16, 16, p.L, batch, 16, kTile);
 }
 
+// `dependent`: launch as a programmatic dependent of the kernel before it in
+// the stream (the summary pass of the same call), see mixer_fwd_kernel.
 template <typename T, typename M, int STAGES, bool SUMMARY>
-cudaError_t launch_prefill(const PrefillParams& p, int64_t batch, int chunks, int threads, cudaStream_t s) {
+cudaError_t launch_prefill(const PrefillParams& p, int64_t batch, int chunks, int threads, bool dependent,
+                           cudaStream_t s) {
     auto kern = mm::mixer_fwd_kernel<T, M, kTile, STAGES, SUMMARY>;
     TensorMaps maps;
     if (!make_maps<T>(p, batch, &maps)) return cudaErrorInvalidValue;
     const int smem = PrefillLayout<T>::smem_bytes(kTile, STAGES, p.octets);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const dim3 grid(static_cast<unsigned>(batch * p.ctas_per_seq), static_cast<unsigned>(chunks));
-    kern<<<grid, threads, smem, s>>>(p, maps.x, maps.z, maps.dt, maps.b, maps.c);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(batch * p.ctas_per_seq), static_cast<unsigned>(chunks));
+    cfg.blockDim = dim3(static_cast<unsigned>(threads));
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = dependent ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kern, p, maps.x, maps.z, maps.dt, maps.b, maps.c);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -242,23 +255,28 @@ int shape_ctas(PrefillParams& p, int64_t batch, int64_t chunks, int sm_count, in
 }
 
 template <typename T, typename M, bool SUMMARY>
-cudaError_t launch_pass(PrefillParams p, int64_t batch, int chunks, int sm_count, cudaStream_t s) {
+cudaError_t launch_pass(PrefillParams p, int64_t batch, int chunks, int sm_count, bool dependent, cudaStream_t s) {
     int threads = 0;
     const int stages = shape_ctas<T>(p, batch, chunks, sm_count, &threads);
-    if (stages >= 4) return launch_prefill<T, M, 4, SUMMARY>(p, batch, chunks, threads, s);
-    if (stages == 3) return launch_prefill<T, M, 3, SUMMARY>(p, batch, chunks, threads, s);
-    return launch_prefill<T, M, 2, SUMMARY>(p, batch, chunks, threads, s);
+    if (stages >= 4) return launch_prefill<T, M, 4, SUMMARY>(p, batch, chunks, threads, dependent, s);
+    if (stages == 3) return launch_prefill<T, M, 3, SUMMARY>(p, batch, chunks, threads, dependent, s);
+    return launch_prefill<T, M, 2, SUMMARY>(p, batch, chunks, threads, dependent, s);
 }
 
 template <typename T, typename M>
 cudaError_t dispatch_prefill(PrefillParams p, int64_t batch, const FwdPlan& pl, int sm_count, cudaStream_t s) {
     p.chunk_len = pl.chunk_len;
     p.n_chunks = pl.chunks;
+    // The summary pass is launched normally: it starts after everything
+    // before it in the stream, the producers of the inputs included.  The
+    // full pass follows it as a programmatic dependent; its CTAs read the
+    // inputs freely (they were complete before the summary pass started) and
+    // wait for the summary grid before reading its results.
     if (pl.chunks > 1) {
-        cudaError_t e = launch_pass<T, M, true>(p, batch, pl.chunks - 1, sm_count, s);
+        cudaError_t e = launch_pass<T, M, true>(p, batch, pl.chunks - 1, sm_count, false, s);
         if (e != cudaSuccess) return e;
     }
-    return launch_pass<T, M, false>(p, batch, pl.chunks, sm_count, s);
+    return launch_pass<T, M, false>(p, batch, pl.chunks, sm_count, pl.chunks > 1, s);
 }
 
 // ---------------------------------------------------------------- host-memory forward

@@ -139,6 +139,14 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity
         if (mbar_try_wait(bar, parity)) return true;
     return false;
 }
+// Programmatic dependent launch.  launch_dependents lets the next kernel in
+// the stream, when launched as a programmatic dependent, start once every CTA
+// of this grid has executed it (or exited).  grid_dependency_wait returns once
+// the grid this one depends on has completed and its writes are visible; with
+// no such dependency it returns at once.
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
 // 3-D tiled bulk tensor copy global -> this CTA's shared memory; completion
 // is signalled on `bar` as transferred bytes.  No multicast.
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, uint64_t* bar) {

@@ -41,7 +41,10 @@
 // tokens of s_t B_t[n] exp(A[n] R_t), R_t the steps after token t, so with
 // structured A a token's weights s r^(n+1) cost 18 packed multiplies (four
 // short chains) and 16 FMAs instead of the forward recurrence's 15 decay
-// powers, 16 products and 16 FMAs.
+// powers, 16 products and 16 FMAs.  The full pass is launched as a
+// programmatic dependent of the summary pass: its CTAs start on SMs the
+// summary leaves free, and only those of chunks 1.. wait for the summary grid
+// before the carry; the inputs were complete before the summary pass began.
 //
 // Latency: each tile is processed in sub-tiles of SUB tokens in three phases
 // so that the long per-token chains (conv -> SiLU -> softplus -> exp) of SUB
@@ -245,6 +248,11 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
         }
     };
 
+    // The full pass may be launched as a programmatic dependent of this
+    // summary pass: its CTAs can then be placed on free SMs, run their setup
+    // and chunk 0 meanwhile, and wait only before reading the summaries.
+    if constexpr (SUMMARY) launch_dependents();
+
     // ---------------------------------------------------------- pipeline prologue (the first tiles stream in during the setup)
     if (tid == 0) {
 #pragma unroll
@@ -313,6 +321,7 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
         // carry h0 through the summaries of the chunks before this one:
         // h <- exp(A sum Delta) h + e, the summaries read state-major so that
         // a warp's loads of one state are contiguous
+        if (chunk > 0) grid_dependency_wait();   // the summaries of chunks 0..chunk-1 (no-op when launched normally)
         if (active && chunk > 0) {
             const int64_t stride = static_cast<int64_t>(p.batch) * D;
 #pragma unroll 1
