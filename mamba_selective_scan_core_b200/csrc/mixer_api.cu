@@ -283,12 +283,17 @@ cudaError_t dispatch_prefill(PrefillParams p, int64_t batch, const FwdPlan& pl, 
 // Piece plan of mamba_mixer_fwd_host: the sequence is cut into about
 // kHostPieces pieces (whole tiles, at least kHostMinPiece tokens) and the
 // device workspace holds two staging slots, two carried states (ping-pong)
-// and the piece forward's own scratch, each region 256-byte aligned.
+// and the piece forward's own scratch, each region 256-byte aligned.  What
+// follows the last input copy -- the last piece's forward and the copy back
+// of its y -- is the call's tail, so a last piece of at least kHostMinPiece
+// tokens is cut once more, in two.
 constexpr int64_t kHostPieces = 8;
 constexpr int64_t kHostMinPiece = 256;
 
 struct HostPlan {
     int64_t piece = 0, pieces = 0;
+    int64_t head = 0;     // pieces 0..head-1 hold `piece` tokens each
+    int64_t tail1 = 0;    // the rest: one piece, or (tail1 > 0) tail1 tokens then the remainder
     size_t off_dt = 0, off_b = 0, off_c = 0, off_y = 0, slot = 0;   // within a staging slot
     size_t carry_h = 0, carry = 0;                                  // within a carried state
     size_t fwd_ws = 0, total = 0;
@@ -296,13 +301,25 @@ struct HostPlan {
 
 size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
 
+// First token and length of piece i of a plan over `seqlen` tokens.
+void piece_range(const HostPlan& hp, int64_t i, int64_t seqlen, int64_t* t0, int64_t* n) {
+    const int64_t tail = hp.head * hp.piece;
+    if (i < hp.head) { *t0 = i * hp.piece; *n = hp.piece; }
+    else if (hp.tail1 == 0) { *t0 = tail; *n = seqlen - tail; }
+    else if (i == hp.head) { *t0 = tail; *n = hp.tail1; }
+    else { *t0 = tail + hp.tail1; *n = seqlen - tail - hp.tail1; }
+}
+
 HostPlan plan_host(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t es) {
     HostPlan hp;
     int64_t piece = (seqlen + kHostPieces - 1) / kHostPieces;
     piece = (piece + kTile - 1) / kTile * kTile;
     piece = std::max(piece, kHostMinPiece);
     hp.piece = std::max<int64_t>(1, std::min(piece, seqlen));
-    hp.pieces = seqlen > 0 ? (seqlen + hp.piece - 1) / hp.piece : 1;   // L = 0: one empty piece
+    hp.head = seqlen > 0 ? (seqlen + hp.piece - 1) / hp.piece - 1 : 0;   // L = 0: one empty piece
+    const int64_t rest = seqlen - hp.head * hp.piece;
+    hp.tail1 = rest >= kHostMinPiece ? ((rest + 1) / 2 + kTile - 1) / kTile * kTile : 0;
+    hp.pieces = hp.head + (hp.tail1 > 0 ? 2 : 1);
     const size_t tok = static_cast<size_t>(batch) * static_cast<size_t>(hp.piece);
     const size_t D = static_cast<size_t>(d_inner), e = static_cast<size_t>(es);
     hp.off_dt = align256(tok * 2 * D * e);
@@ -312,10 +329,11 @@ HostPlan plan_host(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t es) {
     hp.slot = hp.off_y + align256(tok * D * e);
     hp.carry_h = align256(static_cast<size_t>(batch) * D * 16 * 4);
     hp.carry = hp.carry_h + align256(static_cast<size_t>(batch) * D * 3 * e);
-    // every piece but the last has hp.piece tokens; the scratch must fit both plans
-    const int64_t last = seqlen - (hp.pieces - 1) * hp.piece;
-    hp.fwd_ws = align256(std::max(plan_fwd(batch, hp.piece, d_inner).ws_bytes,
-                                  plan_fwd(batch, std::max<int64_t>(last, 0), d_inner).ws_bytes));
+    // the scratch must fit the plan of every piece length used
+    size_t ws = plan_fwd(batch, hp.tail1 > 0 ? hp.tail1 : rest, d_inner).ws_bytes;
+    if (hp.head > 0) ws = std::max(ws, plan_fwd(batch, hp.piece, d_inner).ws_bytes);
+    if (hp.tail1 > 0) ws = std::max(ws, plan_fwd(batch, rest - hp.tail1, d_inner).ws_bytes);
+    hp.fwd_ws = align256(ws);
     hp.total = 2 * hp.slot + 2 * hp.carry + hp.fwd_ws;
     return hp;
 }
@@ -654,8 +672,9 @@ mm_status mamba_mixer_fwd_host(const void* xz, const float* conv_w, const float*
 
     for (int64_t i = 0; ok && i < hp.pieces; ++i) {
         const int j = static_cast<int>(i & 1);
-        const size_t t0 = static_cast<size_t>(i * hp.piece);
-        const size_t n = static_cast<size_t>(std::min<int64_t>(hp.piece, seqlen - i * hp.piece));
+        int64_t pt0 = 0, pn = 0;
+        piece_range(hp, i, seqlen, &pt0, &pn);
+        const size_t t0 = static_cast<size_t>(pt0), n = static_cast<size_t>(pn);
         unsigned char* sl = slot[j];
         // inputs of piece i -> slot j, once the piece that used the slot has been copied out
         if (i >= 2) chk(cudaStreamWaitEvent(s_in, ev_free[j], 0));
