@@ -101,3 +101,21 @@ def test_host_path_empty_sequence_passes_state():
     assert y.shape == (2, 0, 64)
     assert torch.equal(h, inp["h0"])
     assert torch.equal(cs, inp["conv_state_in"])
+
+
+def test_host_path_jamba_prefill_workload_sampled():
+    """The end-to-end leg's call at full size: the Jamba-shaped prefill
+    (1 x 4096 x 8192, bf16) from pinned host memory, in its default piece
+    plan, against the oracle on a deterministic channel sample."""
+    from gpu_util import subset
+    from workloads import CONFIGS, make_mixer_inputs, sample_channels
+
+    cfg = CONFIGS["jamba_prefill"]
+    inp = make_mixer_inputs(cfg)
+    y, h, cs = host_fwd(inp)
+    chans = sample_channels(cfg.d_inner, 256)
+    ref = oracle_fwd(subset(inp, chans))
+    S = torch.as_tensor(chans)
+    assert_close(np64(y.index_select(-1, S)), ref["y"], "bf16", "y", stored_bf16=True)
+    assert_close(np64(h.index_select(1, S)), ref["h_last"], "bf16", "h_last")
+    np.testing.assert_array_equal(np64(cs.index_select(1, S)), ref["conv_state_out"])
