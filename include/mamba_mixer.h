@@ -115,6 +115,11 @@ typedef enum mm_dtype {
  * It may not overlap any input or output (MM_ERR_ALIAS).
  * stream: a cudaStream_t (NULL = the legacy default stream).
  * batch == 0 is a no-op.  seqlen == 0 writes h_last and conv_state_out only.
+ * Length bound (MM_ERR_SHAPE, and a workspace size of 0, beyond it): one
+ * sequence's xz rows, seqlen x 2 d_inner elements, must span less than 2^40
+ * bytes (the bulk tensor copy's stride limit), and seqlen <= 2^30.  In bf16
+ * at d_inner 8192 that is up to 2^25 - 1 tokens; run longer sequences as
+ * several calls, carrying (h_last, conv_state_out).
  */
 mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv_b,
                           const void* dt, const float* dt_bias, const float* A,
@@ -194,7 +199,9 @@ size_t mamba_mixer_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner
  * Asynchronous: when it returns, all work is queued and `stream` waits for
  * the last copy back, so synchronising `stream` makes every output valid.
  * Host buffers must stay alive and unmodified until then.  Errors as
- * mamba_mixer_fwd; sizes are validated before anything is queued.
+ * mamba_mixer_fwd; sizes are validated before anything is queued.  The
+ * length bound of mamba_mixer_fwd applies to each piece (about an eighth of
+ * the sequence), not to the whole sequence.
  */
 mm_status mamba_mixer_fwd_host(const void* xz, const float* conv_w, const float* conv_b,
                                const void* dt, const float* dt_bias, const float* A,

@@ -1,6 +1,8 @@
 // Host side of the C ABI declared in include/mamba_mixer.h: argument
 // validation (before anything is launched), launch-shape selection and the
-// launches themselves.  No allocation, no global state.
+// launches themselves.  No allocation.  The only state is the device fault
+// word, the fixed scratch array of mamba_mixer_fwd_noalloc with its
+// per-device address, and the tensor-map encoder's entry point.
 #include <algorithm>
 #include <cudaTypedefs.h>
 #include <cstdint>
@@ -42,6 +44,15 @@ bool mul_ok(int64_t a, int64_t b, int64_t* out) {
     if (a != 0 && b > INT64_MAX / a) return false;
     *out = a * b;
     return true;
+}
+
+// Sequence lengths the forward's bulk tensor copies can address: token
+// coordinates are 32-bit, and the copy engine takes strides below 2^40 bytes,
+// which bounds one sequence's xz rows (seqlen x 2 d_inner elements).  Longer
+// sequences are run as several calls with the state carried.
+constexpr int64_t kMaxSeqlen = int64_t(1) << 30;
+bool seqlen_ok(int64_t seqlen, int64_t d_inner, int64_t es) {
+    return seqlen <= kMaxSeqlen && seqlen * 2 * d_inner * es < (int64_t(1) << 40);
 }
 
 mm_status check_device(int* sm_count) {
@@ -424,7 +435,8 @@ mm_status mamba_mixer_fault_status(int reset) {
 size_t mamba_mixer_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state,
                                   int64_t d_conv, mm_dtype act) {
     if ((act != MM_F32 && act != MM_BF16) || batch <= 0 || seqlen <= 0 || d_inner <= 0 || d_state != 16 ||
-        d_conv != 4 || d_inner % 8 != 0 || d_inner > (1 << 24) || batch > (1 << 24))
+        d_conv != 4 || d_inner % 8 != 0 || d_inner > (1 << 24) || batch > (1 << 24) ||
+        !seqlen_ok(seqlen, d_inner, act == MM_F32 ? 4 : 2))
         return 0;
     return plan_fwd(batch, seqlen, d_inner).ws_bytes;
 }
@@ -443,6 +455,7 @@ mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv
     if (d_state != 16 || d_conv != 4 || d_inner % 8 != 0) return MM_ERR_UNSUPPORTED;
     if (d_inner > (1 << 24) || batch > (1 << 24)) return MM_ERR_SHAPE;
     const int64_t es = act == MM_F32 ? 4 : 2;
+    if (!seqlen_ok(seqlen, d_inner, es)) return MM_ERR_SHAPE;
     int64_t tokens, xz_bytes, dt_bytes, bc_bytes, st_bytes;
     if (!mul_ok(batch, seqlen, &tokens) || !mul_ok(tokens, 2 * d_inner * es, &xz_bytes) ||
         !mul_ok(tokens, d_inner * es, &dt_bytes) || !mul_ok(tokens, d_state * es, &bc_bytes) ||
@@ -588,7 +601,9 @@ size_t mamba_mixer_host_workspace_size(int64_t batch, int64_t seqlen, int64_t d_
         return 0;
     int64_t tokens, bytes;
     if (!mul_ok(batch, seqlen, &tokens) || !mul_ok(tokens, 2 * d_inner * 4, &bytes)) return 0;
-    return plan_host(batch, seqlen, d_inner, act == MM_F32 ? 4 : 2).total;
+    const int64_t es = act == MM_F32 ? 4 : 2;
+    const HostPlan hp = plan_host(batch, seqlen, d_inner, es);
+    return seqlen_ok(hp.piece, d_inner, es) ? hp.total : 0;
 }
 
 mm_status mamba_mixer_fwd_host(const void* xz, const float* conv_w, const float* conv_b,
@@ -630,6 +645,7 @@ mm_status mamba_mixer_fwd_host(const void* xz, const float* conv_w, const float*
     if (overlaps(out[0], out[1]) || overlaps(out[0], out[2]) || overlaps(out[1], out[2])) return MM_ERR_ALIAS;
 
     const HostPlan hp = plan_host(batch, seqlen, d_inner, es);
+    if (!seqlen_ok(hp.piece, d_inner, es)) return MM_ERR_SHAPE;   // each piece is one device call
     if (!workspace || workspace_bytes < hp.total) return MM_ERR_WORKSPACE;
     if (!aligned16(workspace)) return MM_ERR_ALIGN;
     int sm_count = 0;

@@ -143,6 +143,20 @@ def test_fwd_overflowing_sizes(L):
     assert call_fwd(L, B=1 << 20, Lq=1 << 40) == ESHAPE
 
 
+def test_fwd_sequence_length_bound(L):
+    # one sequence's xz rows (seqlen x 2 d_inner elements) must span less than
+    # 2^40 bytes, the bulk copy engine's stride limit: 2^25 tokens at d_inner
+    # 8192 in bf16 is exactly 2^40
+    assert call_fwd(L, Lq=1 << 25, D=8192) == ESHAPE
+    assert mm.workspace_size(1, 1 << 25, 8192) == 0
+    assert call_fwd(L, Lq=(1 << 25) - 32, D=8192) != ESHAPE
+    assert mm.workspace_size(1, (1 << 25) - 32, 8192) > 0
+    assert call_fwd(L, Lq=(1 << 30) + 1, D=8) == ESHAPE
+    # the host-memory forward bounds each piece (about an eighth of the sequence) instead
+    assert mm.host_workspace_size(1, 1 << 25, 8192) > 0
+    assert mm.host_workspace_size(1, 1 << 29, 8192) == 0
+
+
 @pytest.mark.parametrize("name", ["xz", "conv_w", "dt", "dt_bias", "A", "Bm", "Cm", "y", "h_last", "cs_out"])
 def test_fwd_required_null(L, name):
     assert call_fwd(L, **{name: None}) == ENULL
