@@ -524,7 +524,8 @@ def run_only(args):
     mm.lib()
     if args.only == "forward":
         cfg = PREFILL
-        d = {k: (v.cuda() if v is not None else None) for k, v in make_mixer_inputs(cfg).items()}
+        d = {k: (v.cuda() if v is not None else None)
+             for k, v in make_mixer_inputs(cfg, A_mode=args.a_mode).items()}
         out = (torch.empty((cfg.batch, cfg.seqlen, cfg.d_inner), dtype=torch.bfloat16, device="cuda"),
                torch.empty((cfg.batch, cfg.d_inner, 16), device="cuda"),
                torch.empty((cfg.batch, cfg.d_inner, 3), dtype=torch.bfloat16, device="cuda"))
@@ -562,6 +563,9 @@ def main():
                     help="run one kernel's timed loop only (for profiler captures); prints no JSON line")
     ap.add_argument("--decode-layers", type=int, default=None,
                     help="with --only decode: stacked layers (default: the workload's 28)")
+    ap.add_argument("--a-mode", choices=["structured", "general"], default="structured",
+                    help="with --only forward: A[d,n] = -(n+1) (the workload's) or per-state rows, "
+                         "as trained weights have")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
