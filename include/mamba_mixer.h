@@ -169,7 +169,10 @@ mm_status mamba_mixer_fwd_noalloc(const void* xz, const float* conv_w, const flo
 /* Bytes of device scratch mamba_mixer_fwd needs for these sizes (0 = none).
  * A pure function of its arguments (and of the MAMBA_MIXER_CHUNKS tuning
  * variable, which must not change between this call and the forward that
- * uses the result). */
+ * uses the result).  MAMBA_MIXER_CHUNKS=K (a positive integer) forces K time
+ * chunks per sequence instead of the launch plan's choice, capped at one
+ * chunk per 32-token tile; the result is the same up to fp32 rounding.  It is
+ * a tuning and test knob. */
 size_t mamba_mixer_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner,
                                   int64_t d_state, int64_t d_conv, mm_dtype act);
 
