@@ -126,6 +126,15 @@ def test_jamba_prefill_workload_sampled():
     check_fwd(inp, "bf16", chans=sample_channels(cfg.d_inner, 256))
 
 
+def test_jamba_prefill_general_A_sampled():
+    """The Jamba-shaped prefill with per-state A rows (as trained weights
+    have): the general path at full size, in the launch plan the bench's
+    general_a leg times."""
+    cfg = CONFIGS["jamba_prefill"]
+    inp = make_mixer_inputs(cfg, A_mode="general")
+    check_fwd(inp, "bf16", chans=sample_channels(cfg.d_inner, 256))
+
+
 def test_batched_prefill_workload_sampled():
     cfg = CONFIGS["batched_prefill"]
     inp = make_mixer_inputs(cfg)
