@@ -318,3 +318,44 @@ def test_host_fwd_validates_before_any_copy(L):
     args[11] = args[0]                                    # y over xz
     assert L.mamba_mixer_fwd_host(*args) == EALIAS
     assert L.mamba_mixer_fwd_host(*host_args(B=0, Lq=1000, ws=None, ws_bytes=0)) == OK
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "mamba_mixer.h"
+
+int main(void) {
+    /* host-only entry points: no device is needed */
+    if (mamba_mixer_abi_version() != MAMBA_MIXER_ABI_VERSION) return 1;
+    size_t ws = mamba_mixer_workspace_size(1, 4096, 8192, 16, 4, MM_BF16);
+    if (ws != (size_t)8 * 8192 * 17 * 4) return 2;
+    if (strcmp(mamba_status_string(MM_OK), "ok") != 0) return 3;
+    /* a rejected call: NULL required pointers, caught before any launch */
+    mm_status st = mamba_mixer_fwd(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL,
+                                   NULL, NULL, NULL, 1, 64, 64, 16, 4, MM_BF16, NULL, 0, NULL);
+    if (st != MM_ERR_NULL) return 4;
+    printf("%zu\n", ws);
+    return 0;
+}
+"""
+
+
+def test_plain_c_program_uses_the_abi(L, tmp_path):
+    """The boundary is a C ABI: a C11 program (no C++, no torch) includes the
+    header, links the library and calls its host-only entry points."""
+    import shutil
+    import subprocess
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_abi.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "use_abi"
+    libdir = os.path.dirname(mm.library_path())
+    subprocess.run([cc, "-std=c11", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), "-L", libdir, "-lmamba_mixer", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, (out.returncode, out.stderr)
+    assert out.stdout.strip() == str(8 * 8192 * 17 * 4)
