@@ -59,9 +59,13 @@
 // STAGES-deep ring of shared-memory buffers, each completing on its own
 // mbarrier.  Rows before token 0 or past the sequence are zero-filled by the
 // copy engine; the left context of token 0 is then overwritten with the
-// carried conv window.  Every wait on a copy is bounded: a copy that never
-// lands sets a fault word the host can read (mamba_mixer_fault_status)
-// instead of hanging the GPU.
+// carried conv window.  The first tiles' copies are issued before the
+// per-thread setup (parameters, A rows, h0, the chunk carry), so they land
+// while it runs; the setup's own global accesses move each thread's 128
+// contiguous bytes in 16-byte pieces, and the chunk summaries are stored
+// state-major so that a warp's access to one state is one contiguous span.
+// Every wait on a copy is bounded: a copy that never lands sets a fault word
+// the host can read (mamba_mixer_fault_status) instead of hanging the GPU.
 #pragma once
 
 #include <type_traits>
