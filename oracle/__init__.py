@@ -1,7 +1,7 @@
 """fp64 CPU oracle for the Mamba mixer core -- TEST INFRASTRUCTURE ONLY.
 
-Only the tests, the smoke check and the benchmark's CPU-baseline leg use this
-package.  The product path (the CUDA library and its binding) never imports
+Only the tests, the smoke check and the benchmark's CPU-baseline and
+reference legs use this package.  The product path (the CUDA library and its binding) never imports
 it, and the two share no code.
 
 The arithmetic lives in ``mixer_oracle.c`` (plain C, double precision, libm);

@@ -1,8 +1,8 @@
 /*
  * fp64 reference ("oracle") for the Mamba mixer core and its one-token decode
  * step.  TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the
- * benchmark's CPU-baseline leg call it; no product code links or calls it, and
- * it shares no source with the CUDA library.
+ * benchmark's CPU-baseline and reference legs call it; no product code links
+ * or calls it, and it shares no source with the CUDA library.
  *
  * It is the plain definition, written out as a sequential loop in double
  * precision with libm exp/log1p, with no blocking, chunking or reordering:
