@@ -139,6 +139,17 @@ def _stream_handle(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+def _keep_alive_on(tensors, streams):
+    """Tell torch's caching allocator that device tensors this module
+    allocated are used by work queued on `streams` (besides the stream current
+    at allocation), so their memory is not handed out again before that work
+    has finished."""
+    for t in tensors:
+        for s in streams:
+            if s is not None:
+                t.record_stream(s)
+
+
 def workspace_size(batch, seqlen, d_inner, d_state=16, d_conv=4, act=MM_BF16) -> int:
     return int(lib().mamba_mixer_workspace_size(batch, seqlen, d_inner, d_state, d_conv, act))
 
@@ -159,6 +170,7 @@ def mixer_fwd(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, conv_s
     W = conv_w.shape[-1]
     dev = xz.device
     f32 = torch.float32
+    made = []
     _check(xz, "xz", xz.dtype, (Bsz, L, 2 * D), dev)
     _check(conv_w, "conv_w", f32, (D, W), dev)
     _check(conv_b, "conv_b", f32, (D,), dev)
@@ -172,16 +184,20 @@ def mixer_fwd(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, conv_s
     _check(conv_state_in, "conv_state_in", xz.dtype, (Bsz, D, W - 1), dev)
     if y is None:
         y = torch.empty((Bsz, L, D), dtype=xz.dtype, device=dev)
+        made.append(y)
     if h_last is None:
         h_last = torch.empty((Bsz, D, N), dtype=f32, device=dev)
+        made.append(h_last)
     if conv_state_out is None:
         conv_state_out = torch.empty((Bsz, D, W - 1), dtype=xz.dtype, device=dev)
+        made.append(conv_state_out)
     _check(y, "y", xz.dtype, (Bsz, L, D), dev)
     _check(h_last, "h_last", f32, (Bsz, D, N), dev)
     _check(conv_state_out, "conv_state_out", xz.dtype, (Bsz, D, W - 1), dev)
     ws_bytes = workspace_size(Bsz, L, D, N, W, act)
     if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        made.append(workspace)
     with torch.cuda.device(dev):
         st = lib().mamba_mixer_fwd(
             _ptr(xz), _ptr(conv_w), _ptr(conv_b), _ptr(dt), _ptr(dt_bias), _ptr(A), _ptr(Bm), _ptr(Cm),
@@ -189,6 +205,7 @@ def mixer_fwd(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, conv_s
             Bsz, L, D, N, W, act, _ptr(workspace) if ws_bytes else None, ws_bytes, _stream_handle(stream))
     if st != 0:
         raise MixerError(st, "mamba_mixer_fwd")
+    _keep_alive_on(made, (stream,))
     return y, h_last, conv_state_out
 
 
@@ -261,8 +278,10 @@ def mixer_fwd_host(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, c
     _check_host(h_last, "h_last", f32, (Bsz, D, N))
     _check_host(conv_state_out, "conv_state_out", xz.dtype, (Bsz, D, W - 1))
     ws_bytes = host_workspace_size(Bsz, L, D, N, W, act)
+    made = []
     if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
         workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+        made.append(workspace)
     s_in, s_out = _copy_streams(dev)
     with torch.cuda.device(dev):
         st = lib().mamba_mixer_fwd_host(
@@ -272,6 +291,7 @@ def mixer_fwd_host(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, c
             ctypes.c_void_p(s_in.cuda_stream), ctypes.c_void_p(s_out.cuda_stream))
     if st != 0:
         raise MixerError(st, "mamba_mixer_fwd_host")
+    _keep_alive_on(made, (stream, s_in, s_out))
     return y, h_last, conv_state_out
 
 
@@ -332,8 +352,10 @@ def state_update(x, z, dt, conv_w, conv_b, dt_bias, Dskip, A, Bm, Cm, ssm_state,
     _check(Cm, "Cm", x.dtype, (NL, Bsz, N), dev)
     _check(ssm_state, "ssm_state", f32, (NL, Bsz, D, N), dev)
     _check(conv_state, "conv_state", x.dtype, (NL, Bsz, D, W - 1), dev)
+    made = []
     if y is None:
         y = torch.empty((NL, Bsz, D), dtype=x.dtype, device=dev)
+        made.append(y)
     _check(y, "y", x.dtype, (NL, Bsz, D), dev)
     with torch.cuda.device(dev):
         st = lib().mamba_state_update(
@@ -342,4 +364,5 @@ def state_update(x, z, dt, conv_w, conv_b, dt_bias, Dskip, A, Bm, Cm, ssm_state,
             _stream_handle(stream))
     if st != 0:
         raise MixerError(st, "mamba_state_update")
+    _keep_alive_on(made, (stream,))
     return y

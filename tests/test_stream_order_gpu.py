@@ -98,3 +98,35 @@ def test_back_to_back_repeats_are_deterministic():
     b = run(True)
     for u, v in zip(a, b):
         assert torch.equal(u, v)
+
+
+def test_calls_on_a_side_stream_with_binding_allocations():
+    """mixer_fwd and state_update on a side stream, with the outputs and the
+    scratch workspace allocated by the binding (on the current stream and
+    recorded on the side stream): the same bits as on the current stream."""
+    import mamba_selective_scan_core_b200 as mm
+    from gpu_util import decode_args
+    from workloads import make_decode_inputs_custom
+
+    dev = to_dev(make_mixer_inputs_custom(1, 2048, 1032, act="bf16", seed=96, h0_std=0.3, conv_state_std=1.0))
+    assert mm.workspace_size(1, 2048, 1032) > 0          # a chunked plan: the binding allocates scratch
+    ref = gpu_fwd(dev)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    out = gpu_fwd(dev, stream=side)
+    side.synchronize()
+    for a, b in zip(out, ref):
+        assert torch.equal(a, b)
+
+    dinp = to_dev(make_decode_inputs_custom(2, 8, 256, act="bf16", seed=97))
+    st, cs = dinp["ssm_state"].clone(), dinp["conv_state"].clone()
+    y_ref = mm.state_update(*decode_args(dinp), st, cs)
+    torch.cuda.synchronize()
+    st2, cs2 = dinp["ssm_state"].clone(), dinp["conv_state"].clone()
+    side.wait_stream(torch.cuda.current_stream())
+    y = mm.state_update(*decode_args(dinp), st2, cs2, stream=side)
+    side.synchronize()
+    assert torch.equal(y, y_ref)
+    assert torch.equal(st2, st)
+    assert torch.equal(cs2, cs)
