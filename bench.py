@@ -284,13 +284,20 @@ def run_gpu(args):
                 "frac": round(hbm_gbs / hbm_peak, 4), "traffic": traffic,
                 "algorithmic_bytes": nbytes, "peak_source": hbm_src}
     alu_part = {"bound": "alu", "achieved": round(alu_ach, 3), "peak": round(alu_peak, 3),
-                "unit": "T fp32-pipe ops/s", "frac": round(alu_ach / alu_peak, 4), "traffic": traffic,
+                "unit": "T fp32-pipe ops/s", "frac": round(alu_ach / alu_peak, 4),
                 "ops_per_token_channel": FWD_FP32_OPS_PER_TOKEN_CHANNEL,
-                "peak_source": "148 SMs x 128 fp32 lanes x max SM clock"}
-    roofline, other = (alu_part, hbm_part) if alu_part["frac"] >= hbm_part["frac"] else (hbm_part, alu_part)
+                "peak_source": "derived, nominal: 148 SMs x 128 fp32 lanes x max SM clock (not measured)"}
 
+    del sets, outs
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(mm, host, args, world)
+
+    # ---- the other prefill workloads: 4 x 32768 tokens with h0, and 262,144
+    # tokens run as 8 carried calls of 32768
+    legs = {}
+    if not args.no_extra_prefill:
+        for name in ("batched_prefill", "long_256k"):
+            legs[name] = run_prefill_leg(mm, CONFIGS[name], args, world, hbm_peak, hbm_src, alu_peak)
 
     # ---- decode state update (28 layers x batch 128)
     dec = run_decode(mm, args, world, hbm_peak, hbm_src)
@@ -301,6 +308,7 @@ def run_gpu(args):
     result = None
     if rank == 0:
         cpu = cpu_baseline(host, cfg) if world == 1 and not args.no_cpu_baseline else None
+        cpu1 = cpu_baseline(host, cfg, target_s=6.0, threads=1) if world == 1 and not args.no_cpu_baseline else None
         result = {
             "metric": METRIC,
             "value": round(value, 1),
@@ -320,15 +328,18 @@ def run_gpu(args):
             "config": {"workload": cfg.name, "batch": B, "seq_len": L, "d_inner": D, "d_state": 16, "d_conv": 4,
                        "act": "bf16", "state": "f32", "parallelism": f"replicas x{world}",
                        "l2": "inputs (270 MB/step) larger than L2, rotated over 2 buffer sets"},
-            "roofline": roofline,
-            "roofline_other": other,
+            "roofline": hbm_part,
+            "roofline_alu": alu_part,
             "hbm_frac": hbm_part["frac"],
+            "fp32_pipe_frac": alu_part["frac"],
             "cpu_baseline": cpu,
+            "cpu_baseline_1core": cpu1,
             "e2e": e2e,
             "gpu_launches": K * launches_per_step,
             "clocks": clk.summary(),
             "decode": dec,
             "general_a": gen,
+            **legs,
             "launch_ms": {"mean": round(statistics.mean(launch_ms), 5), "min": round(min(launch_ms), 5),
                           "max": round(max(launch_ms), 5)},
         }
@@ -376,6 +387,70 @@ def run_e2e(mm, host, args, world):
     return {"value": round(_job_rate(world, B * L * K, ms), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
             "ms_per_step": round(ms / K, 4)}
+
+
+def run_prefill_leg(mm, cfg, args, world, hbm_peak, hbm_src, alu_peak):
+    """A prefill workload besides the headline one, through mixer_fwd with
+    device-resident inputs.  A workload with `chunks` > 1 (262,144 tokens) is
+    run as that many sequential calls of L/chunks tokens, each starting from
+    the previous call's (h_last, conv_state_out); one step is the whole
+    sequence.  Its inputs (8.6 and 17.2 GB) are far larger than L2."""
+    B, L, D = cfg.batch, cfg.seqlen, cfg.d_inner
+    host = make_mixer_inputs(cfg)
+    d = {k: (v.cuda() if v is not None else None) for k, v in host.items()}
+    del host
+    n = max(1, getattr(cfg, "chunks", 1) or 1)
+    step_len = L // n
+    y = torch.empty((B, L, D), dtype=torch.bfloat16, device="cuda")
+    carry = [(torch.empty((B, D, 16), device="cuda"), torch.empty((B, D, 3), dtype=torch.bfloat16, device="cuda"))
+             for _ in range(2)]
+    ws = torch.empty(mm.workspace_size(B, step_len, D), dtype=torch.uint8, device="cuda")
+    pieces = []
+    for i in range(n):
+        sl = slice(i * step_len, (i + 1) * step_len)
+        pieces.append({k: (d[k][:, sl] if B == 1 or n == 1 else d[k][:, sl].contiguous())
+                       for k in ("xz", "dt", "Bm", "Cm")})
+    ys = [y[:, i * step_len:(i + 1) * step_len] for i in range(n)]
+
+    def step():
+        h, cs = d["h0"], d["conv_state_in"]
+        for i in range(n):
+            pc = pieces[i]
+            hout, csout = carry[i % 2]
+            mm.mixer_fwd(pc["xz"], d["conv_w"], d["conv_b"], pc["dt"], d["dt_bias"], d["A"], pc["Bm"], pc["Cm"],
+                         d["Dskip"], h, cs, y=ys[i], h_last=hout, conv_state_out=csout, workspace=ws)
+            h, cs = hout, csout
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    K = max(3, min(args.steps, 20))
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(K):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = _max_over_ranks(a.elapsed_time(b) / K, world)
+    nbytes = sum(prefill_bytes(B, step_len, D, h0=(i > 0 or d["h0"] is not None),
+                               cs_in=(i > 0 or d["conv_state_in"] is not None)) for i in range(n))
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    ops = FWD_FP32_OPS_PER_TOKEN_CHANNEL * B * L * D
+    out = {
+        "workload": cfg.name, "batch": B, "seq_len": L, "d_inner": D, "calls_per_step": n,
+        "h0": d["h0"] is not None, "steps": K, "ms_per_step": round(ms, 4),
+        "value": round(_job_rate(world, B * L, ms), 1), "unit": "tokens/s",
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(gbs / hbm_peak, 4), "traffic": None, "algorithmic_bytes": nbytes,
+                     "peak_source": hbm_src},
+        "fp32_pipe_frac": round(ops / (ms * 1e-3) / 1e12 / alu_peak, 4),
+        "l2": f"inputs ({nbytes / 1e9:.1f} GB/step) larger than L2",
+    }
+    del d, y, carry, ws, pieces, ys
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_decode(mm, args, world, hbm_peak, hbm_src):
@@ -454,14 +529,15 @@ def run_general_a(mm, args, world, alu_peak):
 
 
 # ---------------------------------------------------------------- CPU oracle
-def cpu_baseline(host, cfg, target_s=12.0, sample_override=None):
-    """The fp64 oracle as it stands, on all host cores, on a channel sample of
-    the same workload; tokens/s scaled from the sample's channel count to
-    d_inner (channels are independent given the shared B/C)."""
+def cpu_baseline(host, cfg, target_s=12.0, sample_override=None, threads=None):
+    """The fp64 oracle as it stands, on all host cores (or `threads` of
+    them), on a channel sample of the same workload; tokens/s scaled from the
+    sample's channel count to d_inner (channels are independent given the
+    shared B/C)."""
     import oracle
     from workloads import sample_channels, subset_channels as subset
 
-    threads = os.cpu_count() or 1
+    threads = threads or os.cpu_count() or 1
     D = cfg.d_inner
 
     def timed(nch):
@@ -599,6 +675,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra-prefill", action="store_true",
+                    help="skip the 4 x 32768 and 262,144-token prefill legs")
     ap.add_argument("--only", choices=["forward", "decode"], default=None,
                     help="run one kernel's timed loop only (for profiler captures); prints no JSON line")
     ap.add_argument("--decode-layers", type=int, default=None,

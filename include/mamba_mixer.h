@@ -6,10 +6,12 @@
  *   mamba_mixer_fwd      selective-scan forward over a whole sequence (prefill)
  *   mamba_state_update   the one-token state update used in decode
  *
- * and three ways into the forward beyond the plain call:
+ * two more ways into the forward beyond the plain call:
  *   mamba_mixer_fwd_noalloc  no workspace argument (a fixed scratch array inside the library)
  *   mamba_mixer_fwd_host     activations in host memory, copies overlapped with the compute
- *   mamba_mixer_fault_status the device word a kernel sets if it gives up on a bounded wait
+ * and two status readers:
+ *   mamba_check_status       did the last forward on this workspace complete? (per call)
+ *   mamba_mixer_fault_status has any kernel on this device given up a bounded wait? (sticky)
  *
  * What they compute.  The Jamba hybrid SSM-Transformer lesson (section "SSM in
  * one page") gives the recurrence h_t = A h_{t-1} + B x_t, y_t = C h_t, notes
@@ -41,8 +43,8 @@
  *     call launches nothing and writes nothing.  A launch failure reported by
  *     the CUDA runtime returns MM_ERR_CUDA (the runtime's error is cleared).
  *   - The library allocates no device memory; the caller passes every buffer
- *     and scratch area.  Its only state between calls is the device fault
- *     word and the fixed scratch array of mamba_mixer_fwd_noalloc.
+ *     and scratch area.  Its only device state between calls is the device
+ *     fault word and the fixed scratch array of mamba_mixer_fwd_noalloc.
  *     Calls only enqueue work: results are valid once the stream reaches them.
  *     A call starts after all earlier work in its stream and is complete
  *     before later work starts.  Within a time-chunked forward call, the
@@ -71,7 +73,8 @@ typedef enum mm_status {
     MM_ERR_DEVICE = 8,      /* no usable sm_100 device is current                    */
     MM_ERR_WORKSPACE = 9,   /* workspace missing or smaller than the size this call needs */
     MM_ERR_SCRATCH_LIMIT = 10, /* mamba_mixer_fwd_noalloc: sizes need more than its built-in scratch */
-    MM_ERR_TIMEOUT = 11     /* mamba_mixer_fault_status: a kernel gave up waiting for its copies */
+    MM_ERR_TIMEOUT = 11     /* mamba_check_status / mamba_mixer_fault_status: a kernel gave up a
+                               bounded wait (its bulk copies, or a chunk summary never written) */
 } mm_status;
 
 typedef enum mm_dtype {
@@ -105,14 +108,16 @@ typedef enum mm_dtype {
  * carry through two buffer sets (MM_ERR_ALIAS otherwise).
  *
  * workspace / workspace_bytes: device scratch of at least
- * mamba_mixer_workspace_size(...) bytes for the same sizes (may be NULL when
- * that is 0; MM_ERR_WORKSPACE when missing or smaller).  When a sequence has
- * too few channels to fill the GPU, the forward splits it into time chunks:
- * a first launch stores each chunk's end state (run from a zero state) and
- * total step size there, and a second launch starts every chunk from the
- * exact carried state.  The caller owns the workspace; its contents are not
- * needed after the call and calls that share one must not overlap in time.
- * It may not overlap any input or output (MM_ERR_ALIAS).
+ * mamba_mixer_workspace_size(...) bytes for the same sizes, 16-byte aligned
+ * (MM_ERR_WORKSPACE when missing or smaller).  Its first 256 bytes hold the
+ * call's status, which mamba_check_status reads.  When a sequence has too few
+ * channels to fill the GPU, the forward splits it into time chunks: a first
+ * launch stores each chunk's end state (run from a zero state) and total step
+ * size there, and a second launch starts every chunk from the exact carried
+ * state.  The caller owns the workspace; its contents need not be initialised
+ * and are not needed after the call, except for the status; calls that share
+ * one must not overlap in time.  It may not overlap any input or output
+ * (MM_ERR_ALIAS).
  * stream: a cudaStream_t (NULL = the legacy default stream).
  * batch == 0 is a no-op.  seqlen == 0 writes h_last and conv_state_out only.
  * Length bound (MM_ERR_SHAPE, and a workspace size of 0, beyond it): one
@@ -148,14 +153,17 @@ mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv
  * mamba_mixer_workspace_size) return MM_ERR_SCRATCH_LIMIT before anything is
  * launched; with the default launch plan every size fits.
  *
- * The first call on each device looks up the array's device address (with
- * that device current) and keeps it; make that first call before any stream
- * capture.  All calls on a device share the one array and nothing in it is
- * kept between calls (each call writes every scratch value it later reads),
- * but calls that overlap on the GPU -- on different streams, or from
+ * The first call in each CUDA context (a device's primary context, or one
+ * the caller made current) looks up the array's device address in that
+ * context and keeps it, keyed by the context's unique id, so a context made
+ * after cudaDeviceReset gets a lookup of its own; make that first call before
+ * any stream capture.  All calls on a device share the one array and nothing
+ * in it is kept between calls (each call writes every scratch value it later
+ * reads), but calls that overlap on the GPU -- on different streams, or from
  * different threads -- race on it and give wrong results: serialise them.
- * Arguments, outputs, validation and errors are otherwise those of
- * mamba_mixer_fwd.
+ * The status of the last call is read with mamba_check_status(NULL, stream).
+ * Arguments, outputs and errors are otherwise those of mamba_mixer_fwd, and
+ * every argument check of mamba_mixer_fwd comes before the scratch-size check.
  */
 #define MAMBA_MIXER_NOALLOC_SCRATCH_BYTES (8u << 20)
 mm_status mamba_mixer_fwd_noalloc(const void* xz, const float* conv_w, const float* conv_b,
@@ -166,13 +174,14 @@ mm_status mamba_mixer_fwd_noalloc(const void* xz, const float* conv_w, const flo
                                   int64_t batch, int64_t seqlen, int64_t d_inner,
                                   int64_t d_state, int64_t d_conv, mm_dtype act, void* stream);
 
-/* Bytes of device scratch mamba_mixer_fwd needs for these sizes (0 = none).
- * A pure function of its arguments (and of the MAMBA_MIXER_CHUNKS tuning
- * variable, which must not change between this call and the forward that
- * uses the result).  MAMBA_MIXER_CHUNKS=K (a positive integer) forces K time
- * chunks per sequence instead of the launch plan's choice, capped at one
- * chunk per 32-token tile; the result is the same up to fp32 rounding.  It is
- * a tuning and test knob. */
+/* Bytes of device workspace mamba_mixer_fwd needs for these sizes: at least
+ * 256 (the status) for every valid size, 0 for invalid sizes.  A function of
+ * its arguments, of the SM count of the current device (148, a B200's, when
+ * no device is usable) and of the MAMBA_MIXER_CHUNKS tuning variable; none of
+ * these may change between this call and the forward that uses the result.
+ * MAMBA_MIXER_CHUNKS=K (a positive integer) forces K time chunks per sequence
+ * instead of the launch plan's choice, capped at one chunk per 32-token tile;
+ * the result is the same up to fp32 rounding.  It is a tuning and test knob. */
 size_t mamba_mixer_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner,
                                   int64_t d_state, int64_t d_conv, mm_dtype act);
 
@@ -204,7 +213,11 @@ size_t mamba_mixer_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner
  * Host buffers must stay alive and unmodified until then.  Errors as
  * mamba_mixer_fwd; sizes are validated before anything is queued.  The
  * length bound of mamba_mixer_fwd applies to each piece (about an eighth of
- * the sequence), not to the whole sequence.
+ * the sequence), not to the whole sequence.  Every piece records a failure
+ * in the workspace's status under the call's one epoch:
+ * mamba_check_status(workspace, stream) after the call reports whether any
+ * piece gave up.  The device parameters may not overlap the workspace
+ * (MM_ERR_ALIAS).
  */
 mm_status mamba_mixer_fwd_host(const void* xz, const float* conv_w, const float* conv_b,
                                const void* dt, const float* dt_bias, const float* A,
@@ -250,14 +263,34 @@ mm_status mamba_state_update(const void* x, const void* z, const void* dt,
                              int64_t d_state, int64_t d_conv, mm_dtype act, void* stream);
 
 /*
+ * Status of the last forward call that ran on `workspace` (the workspace of
+ * mamba_mixer_fwd or mamba_mixer_fwd_host; NULL = the fixed scratch of
+ * mamba_mixer_fwd_noalloc in the current context).  Waits for `stream` to
+ * finish (the status is device memory written by the call's kernels), so it
+ * cannot be recorded in a stream capture.  Returns MM_ERR_TIMEOUT if a kernel
+ * of that call gave up a bounded wait -- on its own bulk copies, or because a
+ * chunk summary it starts from was never written (the kernel then writes no
+ * output, so y and the carried state of that call are not valid) -- MM_OK if
+ * it completed, MM_ERR_CUDA if the status could not be read, MM_ERR_ALIGN for
+ * a workspace that is not 16-byte aligned.  The status belongs to one call:
+ * a later call on the same workspace replaces it.
+ */
+mm_status mamba_check_status(const void* workspace, void* stream);
+
+/*
  * Device fault word of the library on the current device.  Every wait of a
  * kernel on its own bulk copies is bounded; a kernel that gives up (a copy
  * that never lands -- not expected on working hardware) sets this word,
  * skips its remaining work and exits instead of hanging.  Returns
  * MM_ERR_TIMEOUT if the word is set, MM_OK if not; clears it when `reset` is
  * non-zero.  Synchronises with the device (reads device memory).
- * Test hook: the environment variable MAMBA_MIXER_WAIT_LIMIT sets the number
- * of wait attempts (0 makes the forward give up at once).
+ * Test hooks: the environment variable MAMBA_MIXER_WAIT_LIMIT sets the number
+ * of wait attempts (0 makes the forward give up at once) and
+ * MAMBA_MIXER_SUMMARY_WAIT_LIMIT the same for the summary pass of a
+ * time-chunked forward alone (its chunk summaries then go missing);
+ * MAMBA_MIXER_TEST_LAUNCH_FAIL=1 makes every forward launch ask for more
+ * shared memory than a CTA may have, so the runtime rejects it on the host
+ * and the call returns MM_ERR_CUDA (nothing reaches the GPU).
  */
 mm_status mamba_mixer_fault_status(int reset);
 
@@ -267,7 +300,7 @@ const char* mamba_status_string(mm_status status);
 /* ABI version of this header (incremented on any signature change). */
 int mamba_mixer_abi_version(void);
 
-#define MAMBA_MIXER_ABI_VERSION 1
+#define MAMBA_MIXER_ABI_VERSION 2
 
 #ifdef __cplusplus
 }

@@ -16,7 +16,7 @@ import os
 __all__ = [
     "MM_F32", "MM_BF16", "MixerError", "lib", "library_path", "mixer_fwd", "mixer_fwd_noalloc", "mixer_fwd_host",
     "state_update", "workspace_size", "host_workspace_size", "status_string", "abi_version", "fault_status",
-    "EXPORTED_SYMBOLS",
+    "check_status", "EXPORTED_SYMBOLS",
 ]
 
 MM_F32 = 0
@@ -36,6 +36,7 @@ EXPORTED_SYMBOLS = (
     "mamba_status_string",
     "mamba_mixer_abi_version",
     "mamba_mixer_fault_status",
+    "mamba_check_status",
 )
 
 
@@ -72,6 +73,8 @@ def _declare(L):
     L.mamba_mixer_abi_version.argtypes = []
     L.mamba_mixer_fault_status.restype = ctypes.c_int
     L.mamba_mixer_fault_status.argtypes = [ctypes.c_int]
+    L.mamba_check_status.restype = ctypes.c_int
+    L.mamba_check_status.argtypes = [P, P]
     return L
 
 
@@ -100,6 +103,18 @@ def fault_status(reset: bool = False) -> int:
     """0 if no kernel gave up waiting for its bulk copies on the current
     device, else MM_ERR_TIMEOUT (11); clears the flag when reset is set."""
     return int(lib().mamba_mixer_fault_status(1 if reset else 0))
+
+
+def check_status(workspace=None, stream=None) -> int:
+    """Status of the last forward that ran on `workspace` (a CUDA uint8
+    tensor given to mixer_fwd or mixer_fwd_host; None = the fixed scratch of
+    mixer_fwd_noalloc): 0 if it completed, MM_ERR_TIMEOUT (11) if one of its
+    kernels gave up a bounded wait.  Waits for `stream` (default: current)."""
+    import torch
+
+    dev = workspace.device if workspace is not None else torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        return int(lib().mamba_check_status(_ptr(workspace), _stream_handle(stream)))
 
 
 def _act_code(dtype):
@@ -195,14 +210,15 @@ def mixer_fwd(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, conv_s
     _check(h_last, "h_last", f32, (Bsz, D, N), dev)
     _check(conv_state_out, "conv_state_out", xz.dtype, (Bsz, D, W - 1), dev)
     ws_bytes = workspace_size(Bsz, L, D, N, W, act)
-    if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
         made.append(workspace)
     with torch.cuda.device(dev):
         st = lib().mamba_mixer_fwd(
             _ptr(xz), _ptr(conv_w), _ptr(conv_b), _ptr(dt), _ptr(dt_bias), _ptr(A), _ptr(Bm), _ptr(Cm),
             _ptr(Dskip), _ptr(h0), _ptr(conv_state_in), _ptr(y), _ptr(h_last), _ptr(conv_state_out),
-            Bsz, L, D, N, W, act, _ptr(workspace) if ws_bytes else None, ws_bytes, _stream_handle(stream))
+            Bsz, L, D, N, W, act, _ptr(workspace), workspace.numel() * workspace.element_size(),
+            _stream_handle(stream))
     if st != 0:
         raise MixerError(st, "mamba_mixer_fwd")
     _keep_alive_on(made, (stream,))

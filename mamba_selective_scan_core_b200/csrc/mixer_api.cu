@@ -1,9 +1,12 @@
 // Host side of the C ABI declared in include/mamba_mixer.h: argument
-// validation (before anything is launched), launch-shape selection and the
-// launches themselves.  No allocation.  The only state is the device fault
-// word, the fixed scratch array of mamba_mixer_fwd_noalloc with its
-// per-device address, and the tensor-map encoder's entry point.
+// validation (before anything is launched), launch-plan and CTA-shape
+// selection, and the launches themselves.  No allocation.  The library's
+// state is the device fault word, the fixed scratch array of
+// mamba_mixer_fwd_noalloc with its per-context address, a call counter, and
+// host-side caches (SM counts, kernel attributes already set, recent tensor
+// maps) that only save repeated work.
 #include <algorithm>
+#include <atomic>
 #include <cudaTypedefs.h>
 #include <cstdint>
 #include <cstdlib>
@@ -22,6 +25,7 @@ using mm::PrefillParams;
 constexpr int kTile = 32;
 constexpr int kMaxThreads = 128;
 constexpr int kSmemBudget = 200 * 1024;
+constexpr int kMaxDevices = 256;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -55,33 +59,6 @@ bool seqlen_ok(int64_t seqlen, int64_t d_inner, int64_t es) {
     return seqlen <= kMaxSeqlen && seqlen * 2 * d_inner * es < (int64_t(1) << 40);
 }
 
-mm_status check_device(int* sm_count) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return MM_ERR_DEVICE; }
-    int major = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-        cudaGetLastError();
-        return MM_ERR_DEVICE;
-    }
-    if (major != 10) return MM_ERR_DEVICE;
-    return MM_OK;
-}
-
-// Launch plan of a forward call: time chunks and the workspace they need.
-// A pure function of the sizes (and of the MAMBA_MIXER_CHUNKS tuning
-// variable), so that mamba_mixer_workspace_size() and the call agree.
-struct FwdPlan {
-    int chunks = 1;
-    int64_t chunk_len = 0;
-    size_t ws_bytes = 0;
-};
-
-constexpr int kPlanSMs = 148;            // B200: 2 dies x 74 SMs
-constexpr int kWarpsPerSM = 4 * MM_FWD_MIN_BLOCKS;   // resident warps per SM at the forward's register use
-constexpr int kMinChunkTiles = 4;        // shortest chunk worth a summary pass
-constexpr int kMaxChunks = 16;
-
 int env_int(const char* name, int lo, int hi) {
     if (const char* e = std::getenv(name)) {
         const int v = std::atoi(e);
@@ -90,17 +67,85 @@ int env_int(const char* name, int lo, int hi) {
     return 0;
 }
 
+// ---------------------------------------------------------------- devices
+// SM count of the current device, queried once per device.  Without a usable
+// device the plan falls back to a B200's 148 SMs, so that sizes computed on a
+// machine without a GPU describe the B200 plan.
+constexpr int kB200SMs = 148;
+
+int plan_sms() {
+    static std::atomic<int> cache[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return kB200SMs;
+    }
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n > 0) return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return kB200SMs;
+    }
+    cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+// The current device must be an sm_100 part (B200).
+mm_status check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return MM_ERR_DEVICE; }
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MM_ERR_DEVICE;
+    }
+    return major == 10 ? MM_OK : MM_ERR_DEVICE;
+}
+
+// Ids of launch pairs and per-call status epochs: unique in the process,
+// never 0, below 2^56 (the status word keeps 8 bits for the code).
+std::atomic<unsigned long long> g_call_counter{0};
+unsigned long long next_call_id() { return (g_call_counter.fetch_add(1) + 1) & ((1ull << 56) - 1); }
+
+// ---------------------------------------------------------------- launch plan
+// Launch plan of a forward call: time chunks, and the workspace they need.
+// A function of the sizes, the current device's SM count and the
+// MAMBA_MIXER_CHUNKS tuning variable, so that mamba_mixer_workspace_size()
+// and the call agree.
+//
+// Workspace layout (every region 256-byte aligned):
+//   header  [256 B]                   the call status (PrefillParams::ws_hdr)
+//   tags    [K-1][batch][D/8] u64     who wrote each summary (PrefillParams::ws_tags)
+//   state   [K-1][batch][16][D] f32   chunk end states from zero
+//   lsum    [K-1][batch][D] f32       chunk step-size sums
+struct FwdPlan {
+    int chunks = 1;
+    int64_t chunk_len = 0;
+    size_t off_tags = 0, off_state = 0, off_lsum = 0, ws_bytes = 0;
+};
+
+constexpr size_t kWsHeader = 256;
+constexpr int kMinBlocksFwd = MM_FWD_MIN_BLOCKS;
+constexpr int kWarpsPerSM = 4 * kMinBlocksFwd;   // resident warps per SM at the forward's register use
+constexpr int kMinChunkTiles = 4;        // shortest chunk worth a summary pass
+constexpr int kMaxChunks = 16;
+
+size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
 // Tries per wait on a bulk copy (each try waits a bounded time in hardware):
 // about a second by default; MAMBA_MIXER_WAIT_LIMIT overrides it (tests use 0
 // to make the wait give up at once).
-unsigned copy_wait_limit() {
-    if (const char* e = std::getenv("MAMBA_MIXER_WAIT_LIMIT")) {
+// MAMBA_MIXER_SUMMARY_WAIT_LIMIT applies to the summary pass alone (tests use
+// it to make only the summaries go missing).
+unsigned env_wait_limit(const char* name, unsigned dflt) {
+    if (const char* e = std::getenv(name)) {
         char* end = nullptr;
         const long v = std::strtol(e, &end, 10);
         if (end != e && v >= 0 && v <= (1L << 30)) return static_cast<unsigned>(v);
     }
-    return 1u << 20;
+    return dflt;
 }
+unsigned copy_wait_limit() { return env_wait_limit("MAMBA_MIXER_WAIT_LIMIT", 1u << 20); }
 
 // Time chunks.  More chunks put more warps on the SMs but add a summary pass
 // over (K-1)/K of the tokens, so K minimises a measured cost model: a pass
@@ -108,15 +153,15 @@ unsigned copy_wait_limit() {
 // 8 warps (two CTAs) taking ~1.85x as long as one running 4, and a summary
 // token costing ~0.55 of a full-pass token (B200 measurements of both
 // kernels), among splits that fit one wave.  It picks 9 chunks for one
-// 8192-channel sequence and a single chunk once a batch fills the SMs on
-// its own.
-double busiest_sm(int64_t warps) {
-    const int64_t m = (warps + kPlanSMs - 1) / kPlanSMs;        // warps on the busiest SM
+// 8192-channel sequence on 148 SMs and a single chunk once a batch fills the
+// SMs on its own.
+double busiest_sm(int64_t warps, int sms) {
+    const int64_t m = (warps + sms - 1) / sms;        // warps on the busiest SM
     const int64_t waves = m / kWarpsPerSM, rest = m % kWarpsPerSM;
     return 1.85 * static_cast<double>(waves) + (rest == 0 ? 0.0 : rest * 2 <= kWarpsPerSM ? 1.0 : 1.85);
 }
 
-FwdPlan plan_fwd(int64_t batch, int64_t seqlen, int64_t d_inner) {
+FwdPlan plan_fwd(int64_t batch, int64_t seqlen, int64_t d_inner, int sms) {
     FwdPlan pl;
     const int64_t warps = std::max<int64_t>(1, batch * ((d_inner / 2 + 31) / 32));   // per chunk
     const int64_t tiles = std::max<int64_t>(1, (seqlen + kTile - 1) / kTile);
@@ -132,16 +177,21 @@ FwdPlan plan_fwd(int64_t batch, int64_t seqlen, int64_t d_inner) {
             const int64_t chunks = (tiles + ct - 1) / ct;            // chunks the split really makes
             // a split stays within one wave of resident warps (the model does not
             // charge what grows with the chunk count: carry chains, pipeline fills)
-            if (chunks > 1 && chunks * warps > static_cast<int64_t>(kPlanSMs) * kWarpsPerSM) break;
+            if (chunks > 1 && chunks * warps > static_cast<int64_t>(sms) * kWarpsPerSM) break;
             const double cost = static_cast<double>(ct) *
-                                (busiest_sm(chunks * warps) + (chunks > 1 ? 0.55 * busiest_sm((chunks - 1) * warps) : 0.0));
+                                (busiest_sm(chunks * warps, sms) +
+                                 (chunks > 1 ? 0.55 * busiest_sm((chunks - 1) * warps, sms) : 0.0));
             if (c == 1 || cost < best) { best = cost; k = c; }
         }
     }
     pl.chunk_len = chunk_tiles(k) * kTile;
     pl.chunks = static_cast<int>(seqlen > 0 ? (seqlen + pl.chunk_len - 1) / pl.chunk_len : 1);
-    if (pl.chunks > 1)
-        pl.ws_bytes = static_cast<size_t>(pl.chunks - 1) * batch * d_inner * (16 + 1) * sizeof(float);
+    const size_t c1 = static_cast<size_t>(pl.chunks - 1), B = static_cast<size_t>(batch);
+    const size_t D = static_cast<size_t>(d_inner);
+    pl.off_tags = kWsHeader;
+    pl.off_state = pl.off_tags + align256(c1 * B * (D / 8) * sizeof(unsigned long long));
+    pl.off_lsum = pl.off_state + align256(c1 * B * 16 * D * sizeof(float));
+    pl.ws_bytes = pl.off_lsum + align256(c1 * B * D * sizeof(float));
     return pl;
 }
 
@@ -166,9 +216,34 @@ struct TensorMaps {
     CUtensorMap x, z, dt, b, c;
 };
 
+// A map is a pure function of its base address, sizes and box; each host
+// thread keeps its most recent ones, so repeated calls on the same buffers
+// (a serving loop, a benchmark) skip the encoder.
+struct MapKey {
+    const void* base;
+    int64_t cols, rows, batch;
+    int box_cols, box_rows;
+    bool bf16;
+    bool operator==(const MapKey& o) const {
+        return base == o.base && cols == o.cols && rows == o.rows && batch == o.batch && box_cols == o.box_cols &&
+               box_rows == o.box_rows && bf16 == o.bf16;
+    }
+};
+constexpr int kMapCache = 20;
+struct MapCache {
+    MapKey key[kMapCache];
+    CUtensorMap map[kMapCache];
+    int n = 0, next = 0;
+};
+thread_local MapCache t_maps;
+
 // 3-D map over a [batch][rows][cols] tensor with a [1][box_rows][box_cols] box.
 bool encode_3d(CUtensorMap* m, const void* base, bool bf16, int64_t cols, int64_t rows, int64_t batch,
                int box_cols, int box_rows) {
+    const MapKey k{base, cols, rows, batch, box_cols, box_rows, bf16};
+    MapCache& c = t_maps;
+    for (int i = 0; i < c.n; ++i)
+        if (c.key[i] == k) { *m = c.map[i]; return true; }
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     const int64_t es = bf16 ? 2 : 4;
@@ -177,10 +252,16 @@ bool encode_3d(CUtensorMap* m, const void* base, bool bf16, int64_t cols, int64_
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols * es), static_cast<cuuint64_t>(rows * cols * es)};
     const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
-               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+            const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    const int slot = c.n < kMapCache ? c.n++ : c.next;
+    c.next = (slot + 1) % kMapCache;
+    c.key[slot] = k;
+    c.map[slot] = *m;
+    return true;
 }
 
 template <typename T>
@@ -196,6 +277,27 @@ bool make_maps(const PrefillParams& p, int64_t batch, TensorMaps* m) {
            encode_3d(&m->c, p.Cm, bf16, 16, p.L, batch, 16, kTile);
 }
 
+// Every launch asks for at most kSmemBudget bytes of dynamic shared memory
+// (ring_depth guarantees it); each kernel is allowed that much once per device
+// (the attribute belongs to the kernel in that device's context).  `done` is
+// the per-kernel record of devices already set.
+template <typename Kern>
+cudaError_t allow_smem(Kern kern, std::atomic<unsigned long long>& done) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaGetLastError();
+    const unsigned long long bit = dev < 64 ? 1ull << dev : 0;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
+
+// Test hook: MAMBA_MIXER_TEST_LAUNCH_FAIL=1 makes every forward launch ask
+// for more dynamic shared memory than any CTA may have, so the runtime
+// rejects it on the host (nothing reaches the GPU) and the call returns
+// MM_ERR_CUDA; the next call without it runs normally.
+bool forced_launch_failure() { return env_int("MAMBA_MIXER_TEST_LAUNCH_FAIL", 1, 1) == 1; }
+
 // `dependent`: launch as a programmatic dependent of the kernel before it in
 // the stream (the summary pass of the same call), see mixer_fwd_kernel.
 template <typename T, typename M, int STAGES, bool SUMMARY>
@@ -205,12 +307,13 @@ cudaError_t launch_prefill(const PrefillParams& p, int64_t batch, int chunks, in
     TensorMaps maps;
     if (!make_maps<T>(p, batch, &maps)) return cudaErrorInvalidValue;
     const int smem = PrefillLayout<T>::smem_bytes(kTile, STAGES, p.octets);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    static std::atomic<unsigned long long> smem_allowed{0};   // one record per kernel instance
+    cudaError_t e = allow_smem(kern, smem_allowed);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(batch * p.ctas_per_seq), static_cast<unsigned>(chunks));
     cfg.blockDim = dim3(static_cast<unsigned>(threads));
-    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.dynamicSmemBytes = forced_launch_failure() ? size_t(1) << 20 : static_cast<size_t>(smem);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -237,9 +340,13 @@ int ring_depth(int oct) {
     return 0;
 }
 
+struct CtaShape {
+    int octets = 1, ctas_per_seq = 1, threads = 32, stages = 2;
+};
+
 template <typename T>
-int shape_ctas(PrefillParams& p, int64_t batch, int64_t chunks, int sm_count, int* threads) {
-    const int64_t octets_per_seq = p.D / 8;
+CtaShape shape_ctas(int64_t d_inner, int64_t batch, int64_t chunks, int sm_count) {
+    const int64_t octets_per_seq = d_inner / 8;
     // a copy box spans at most 256 channels: 32 octets
     const int max_oct = static_cast<int>(std::min<int64_t>({kMaxThreads / 4, 32, octets_per_seq}));
     int64_t best_waves = INT64_MAX;
@@ -258,46 +365,148 @@ int shape_ctas(PrefillParams& p, int64_t batch, int64_t chunks, int sm_count, in
             }
         }
     }
+    CtaShape sh;
     const int64_t ctas = (octets_per_seq + best - 1) / best;
-    p.octets = static_cast<int>((octets_per_seq + ctas - 1) / ctas);
-    p.ctas_per_seq = static_cast<int>(ctas);
-    *threads = ((p.octets * 4) + 31) / 32 * 32;
-    return std::min(best_stages, std::max(2, ring_depth<T>(p.octets)));
+    sh.octets = static_cast<int>((octets_per_seq + ctas - 1) / ctas);
+    sh.ctas_per_seq = static_cast<int>(ctas);
+    sh.threads = ((sh.octets * 4) + 31) / 32 * 32;
+    sh.stages = std::min(best_stages, std::max(2, ring_depth<T>(sh.octets)));
+    return sh;
 }
 
 template <typename T, typename M, bool SUMMARY>
-cudaError_t launch_pass(PrefillParams p, int64_t batch, int chunks, int sm_count, bool dependent, cudaStream_t s) {
-    int threads = 0;
-    const int stages = shape_ctas<T>(p, batch, chunks, sm_count, &threads);
-    if (stages >= 4) return launch_prefill<T, M, 4, SUMMARY>(p, batch, chunks, threads, dependent, s);
-    if (stages == 3) return launch_prefill<T, M, 3, SUMMARY>(p, batch, chunks, threads, dependent, s);
-    return launch_prefill<T, M, 2, SUMMARY>(p, batch, chunks, threads, dependent, s);
+cudaError_t launch_pass(PrefillParams p, const CtaShape& sh, int64_t batch, int chunks, bool dependent,
+                        cudaStream_t s) {
+    p.octets = sh.octets;
+    p.ctas_per_seq = sh.ctas_per_seq;
+    if (sh.stages >= 4) return launch_prefill<T, M, 4, SUMMARY>(p, batch, chunks, sh.threads, dependent, s);
+    if (sh.stages == 3) return launch_prefill<T, M, 3, SUMMARY>(p, batch, chunks, sh.threads, dependent, s);
+    return launch_prefill<T, M, 2, SUMMARY>(p, batch, chunks, sh.threads, dependent, s);
 }
 
 template <typename T, typename M>
 cudaError_t dispatch_prefill(PrefillParams p, int64_t batch, const FwdPlan& pl, int sm_count, cudaStream_t s) {
     p.chunk_len = pl.chunk_len;
     p.n_chunks = pl.chunks;
+    const CtaShape full = shape_ctas<T>(p.D, batch, pl.chunks, sm_count);
     // The summary pass is launched normally: it starts after everything
     // before it in the stream, the producers of the inputs included.  The
     // full pass follows it as a programmatic dependent; its CTAs read the
     // inputs freely (they were complete before the summary pass started) and
     // wait for the summary grid before reading its results.
     if (pl.chunks > 1) {
-        cudaError_t e = launch_pass<T, M, true>(p, batch, pl.chunks - 1, sm_count, false, s);
+        const CtaShape sum = shape_ctas<T>(p.D, batch, pl.chunks - 1, sm_count);
+        p.sum_octets = sum.octets;
+        PrefillParams ps = p;
+        ps.wait_limit = env_wait_limit("MAMBA_MIXER_SUMMARY_WAIT_LIMIT", p.wait_limit);
+        cudaError_t e = launch_pass<T, M, true>(ps, sum, batch, pl.chunks - 1, false, s);
         if (e != cudaSuccess) return e;
     }
-    return launch_pass<T, M, false>(p, batch, pl.chunks, sm_count, pl.chunks > 1, s);
+    return launch_pass<T, M, false>(p, full, batch, pl.chunks, pl.chunks > 1, s);
+}
+
+// ---------------------------------------------------------------- forward calls
+// The arguments of a forward call, as the entry points receive them.
+struct FwdArgs {
+    const void* xz; const float* conv_w; const float* conv_b; const void* dt; const float* dt_bias;
+    const float* A; const void* Bm; const void* Cm; const float* Dskip; const float* h0;
+    const void* cs_in; void* y; float* h_last; void* cs_out;
+    int64_t batch, seqlen, d_inner, d_state, d_conv;
+    mm_dtype act;
+};
+
+struct FwdBytes {
+    int64_t es = 0, xz = 0, dt = 0, bc = 0, st = 0, cs = 0;
+};
+
+// Sizes and dtype: the checks shared by every forward entry point.
+mm_status check_sizes(const FwdArgs& a, FwdBytes* nb) {
+    if (a.act != MM_F32 && a.act != MM_BF16) return MM_ERR_DTYPE;
+    if (a.batch < 0 || a.seqlen < 0 || a.d_inner <= 0 || a.d_state <= 0 || a.d_conv <= 0) return MM_ERR_SHAPE;
+    if (a.d_state != 16 || a.d_conv != 4 || a.d_inner % 8 != 0) return MM_ERR_UNSUPPORTED;
+    if (a.d_inner > (1 << 24) || a.batch > (1 << 24)) return MM_ERR_SHAPE;
+    nb->es = a.act == MM_F32 ? 4 : 2;
+    int64_t tokens;
+    if (!mul_ok(a.batch, a.seqlen, &tokens) || !mul_ok(tokens, 2 * a.d_inner * nb->es, &nb->xz) ||
+        !mul_ok(tokens, a.d_inner * nb->es, &nb->dt) || !mul_ok(tokens, a.d_state * nb->es, &nb->bc) ||
+        !mul_ok(a.batch, a.d_inner * a.d_state * 4, &nb->st))
+        return MM_ERR_SHAPE;
+    nb->cs = a.batch * a.d_inner * (a.d_conv - 1) * nb->es;
+    return MM_OK;
+}
+
+// Every check of a device-memory forward call except the workspace.
+mm_status validate_fwd(const FwdArgs& a, FwdBytes* nb) {
+    if (mm_status st = check_sizes(a, nb); st != MM_OK) return st;
+    if (!seqlen_ok(a.seqlen, a.d_inner, nb->es)) return MM_ERR_SHAPE;
+    if (a.batch == 0) return MM_OK;
+    if (!a.conv_w || !a.dt_bias || !a.A || !a.h_last || !a.cs_out) return MM_ERR_NULL;
+    if (a.seqlen > 0 && (!a.xz || !a.dt || !a.Bm || !a.Cm || !a.y)) return MM_ERR_NULL;
+    const void* all[] = {a.xz, a.conv_w, a.conv_b, a.dt, a.dt_bias, a.A, a.Bm, a.Cm, a.Dskip, a.h0, a.cs_in,
+                         a.y, a.h_last, a.cs_out};
+    for (const void* q : all)
+        if (q && !aligned16(q)) return MM_ERR_ALIGN;
+    const int64_t D = a.d_inner;
+    const Span in[] = {span(a.xz, nb->xz), span(a.conv_w, D * a.d_conv * 4), span(a.conv_b, D * 4),
+                       span(a.dt, nb->dt), span(a.dt_bias, D * 4), span(a.A, D * a.d_state * 4),
+                       span(a.Bm, nb->bc), span(a.Cm, nb->bc), span(a.Dskip, D * 4),
+                       span(a.h0, nb->st), span(a.cs_in, nb->cs)};
+    const Span out[] = {span(a.y, nb->dt), span(a.h_last, nb->st), span(a.cs_out, nb->cs)};
+    for (const Span& o : out)
+        for (const Span& i : in)
+            if (overlaps(o, i)) return MM_ERR_ALIAS;
+    if (overlaps(out[0], out[1]) || overlaps(out[0], out[2]) || overlaps(out[1], out[2])) return MM_ERR_ALIAS;
+    return MM_OK;
+}
+
+// The workspace (or scratch) may overlap no input or output.
+bool workspace_overlaps(const FwdArgs& a, const FwdBytes& nb, const void* ws, size_t bytes) {
+    const int64_t D = a.d_inner;
+    const Span w = span(ws, static_cast<int64_t>(bytes));
+    const Span all[] = {span(a.xz, nb.xz), span(a.conv_w, D * a.d_conv * 4), span(a.conv_b, D * 4),
+                        span(a.dt, nb.dt), span(a.dt_bias, D * 4), span(a.A, D * a.d_state * 4),
+                        span(a.Bm, nb.bc), span(a.Cm, nb.bc), span(a.Dskip, D * 4), span(a.h0, nb.st),
+                        span(a.cs_in, nb.cs), span(a.y, nb.dt), span(a.h_last, nb.st), span(a.cs_out, nb.cs)};
+    for (const Span& s : all)
+        if (overlaps(w, s)) return true;
+    return false;
+}
+
+// Launch a validated forward (batch > 0) on `ws`, laid out as `pl` says.
+// Its failures are recorded in ws's header under `status_epoch`.
+mm_status run_fwd(const FwdArgs& a, const FwdPlan& pl, int sm_count, void* ws, unsigned long long status_epoch,
+                  cudaStream_t s) {
+    unsigned char* w = static_cast<unsigned char*>(ws);
+    PrefillParams p{};
+    p.xz = a.xz; p.conv_w = a.conv_w; p.conv_b = a.conv_b; p.dt = a.dt; p.dt_bias = a.dt_bias; p.A = a.A;
+    p.Bm = a.Bm; p.Cm = a.Cm; p.Dskip = a.Dskip; p.h0 = a.h0; p.cs_in = a.cs_in;
+    p.y = a.y; p.h_last = a.h_last; p.cs_out = a.cs_out;
+    p.L = a.seqlen;
+    p.D = static_cast<int>(a.d_inner);
+    p.batch = static_cast<int>(a.batch);
+    p.wait_limit = copy_wait_limit();
+    p.ws_hdr = reinterpret_cast<unsigned long long*>(w);
+    p.ws_tags = reinterpret_cast<unsigned long long*>(w + pl.off_tags);
+    p.ws_state = reinterpret_cast<float*>(w + pl.off_state);
+    p.ws_lsum = reinterpret_cast<float*>(w + pl.off_lsum);
+    p.call_id = next_call_id();
+    p.status_epoch = status_epoch;
+    p.sum_octets = 1;
+    cudaError_t e = a.act == MM_BF16 ? dispatch_prefill<__nv_bfloat16, mm::MathFast>(p, a.batch, pl, sm_count, s)
+                                     : dispatch_prefill<float, mm::MathExact>(p, a.batch, pl, sm_count, s);
+    if (e != cudaSuccess) { cudaGetLastError(); return MM_ERR_CUDA; }
+    return MM_OK;
 }
 
 // ---------------------------------------------------------------- host-memory forward
 // Piece plan of mamba_mixer_fwd_host: the sequence is cut into about
 // kHostPieces pieces (whole tiles, at least kHostMinPiece tokens) and the
-// device workspace holds two staging slots, two carried states (ping-pong)
-// and the piece forward's own scratch, each region 256-byte aligned.  What
-// follows the last input copy -- the last piece's forward and the copy back
-// of its y -- is the call's tail, so a last piece of at least kHostMinPiece
-// tokens is cut once more, in two.
+// device workspace holds the piece forward's own workspace first (so that
+// mamba_check_status reads the call's status from the workspace's start),
+// then two staging slots and two carried states (ping-pong), each region
+// 256-byte aligned.  What follows the last input copy -- the last piece's
+// forward and the copy back of its y -- is the call's tail, so a last piece of
+// at least kHostMinPiece tokens is cut once more, in two.
 constexpr int64_t kHostPieces = 8;
 constexpr int64_t kHostMinPiece = 256;
 
@@ -310,8 +519,6 @@ struct HostPlan {
     size_t fwd_ws = 0, total = 0;
 };
 
-size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
-
 // First token and length of piece i of a plan over `seqlen` tokens.
 void piece_range(const HostPlan& hp, int64_t i, int64_t seqlen, int64_t* t0, int64_t* n) {
     const int64_t tail = hp.head * hp.piece;
@@ -321,7 +528,7 @@ void piece_range(const HostPlan& hp, int64_t i, int64_t seqlen, int64_t* t0, int
     else { *t0 = tail + hp.tail1; *n = seqlen - tail - hp.tail1; }
 }
 
-HostPlan plan_host(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t es) {
+HostPlan plan_host(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t es, int sms) {
     HostPlan hp;
     int64_t piece = (seqlen + kHostPieces - 1) / kHostPieces;
     piece = (piece + kTile - 1) / kTile * kTile;
@@ -340,12 +547,12 @@ HostPlan plan_host(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t es) {
     hp.slot = hp.off_y + align256(tok * D * e);
     hp.carry_h = align256(static_cast<size_t>(batch) * D * 16 * 4);
     hp.carry = hp.carry_h + align256(static_cast<size_t>(batch) * D * 3 * e);
-    // the scratch must fit the plan of every piece length used
-    size_t ws = plan_fwd(batch, hp.tail1 > 0 ? hp.tail1 : rest, d_inner).ws_bytes;
-    if (hp.head > 0) ws = std::max(ws, plan_fwd(batch, hp.piece, d_inner).ws_bytes);
-    if (hp.tail1 > 0) ws = std::max(ws, plan_fwd(batch, rest - hp.tail1, d_inner).ws_bytes);
+    // the piece workspace must fit the plan of every piece length used
+    size_t ws = plan_fwd(batch, hp.tail1 > 0 ? hp.tail1 : rest, d_inner, sms).ws_bytes;
+    if (hp.head > 0) ws = std::max(ws, plan_fwd(batch, hp.piece, d_inner, sms).ws_bytes);
+    if (hp.tail1 > 0) ws = std::max(ws, plan_fwd(batch, rest - hp.tail1, d_inner, sms).ws_bytes);
     hp.fwd_ws = align256(ws);
-    hp.total = 2 * hp.slot + 2 * hp.carry + hp.fwd_ws;
+    hp.total = hp.fwd_ws + 2 * hp.slot + 2 * hp.carry;
     return hp;
 }
 
@@ -368,31 +575,72 @@ struct HostEvents {
 
 // Scratch of mamba_mixer_fwd_noalloc: one fixed array per device in the
 // library's device image, for callers that cannot allocate.  Host code only
-// ever passes its device address (looked up per device, below) to kernels.
+// ever passes its device address (looked up per context, below) to kernels.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[MAMBA_MIXER_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 
-constexpr int kMaxDevices = 256;
+// The driver's context queries, fetched through the runtime like the
+// tensor-map encoder (no link against libcuda).
+using PfnCtxGetCurrent = CUresult (*)(CUcontext*);
+using PfnCtxGetId = CUresult (*)(CUcontext, unsigned long long*);
 
-// Device address of g_noalloc_scratch on the current device, looked up once
-// per device (with that device current) and kept.
+struct CtxApi {
+    PfnCtxGetCurrent get_current = nullptr;
+    PfnCtxGetId get_id = nullptr;
+};
+const CtxApi& ctx_api() {
+    static std::once_flag once;
+    static CtxApi api;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            api.get_current = reinterpret_cast<PfnCtxGetCurrent>(f);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            api.get_id = reinterpret_cast<PfnCtxGetId>(f);
+        cudaGetLastError();
+    });
+    return api;
+}
+
+// Device address of g_noalloc_scratch in the current CUDA context.  The
+// address belongs to the module image loaded in one context: a context the
+// caller made current, or the primary context created again after
+// cudaDeviceReset, has its own.  So it is looked up once per context, keyed
+// by the context's process-unique id, and kept; without the id query it is
+// looked up on every call.
 mm_status noalloc_scratch(void** out) {
+    // the lookup itself makes the runtime's context current if none is yet
+    void* p = nullptr;
+    const CtxApi& api = ctx_api();
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    const bool keyed = api.get_current && api.get_id && api.get_current(&ctx) == CUDA_SUCCESS && ctx &&
+                       api.get_id(ctx, &id) == CUDA_SUCCESS;
     static std::mutex mu;
-    static void* addr[kMaxDevices] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return MM_ERR_DEVICE; }
-    if (dev < 0 || dev >= kMaxDevices) return MM_ERR_DEVICE;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
-            cudaGetLastError();
-            return MM_ERR_CUDA;
-        }
-        addr[dev] = p;
+    constexpr int kSlots = 64;
+    static unsigned long long ids[kSlots] = {};
+    static void* addrs[kSlots] = {};
+    static int next = 0;
+    if (keyed) {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < kSlots; ++i)
+            if (ids[i] == id && addrs[i]) { *out = addrs[i]; return MM_OK; }
     }
-    *out = addr[dev];
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+        cudaGetLastError();
+        return MM_ERR_CUDA;
+    }
+    if (keyed) {
+        std::lock_guard<std::mutex> lock(mu);
+        ids[next] = id;
+        addrs[next] = p;
+        next = (next + 1) % kSlots;
+    }
+    *out = p;
     return MM_OK;
 }
 
@@ -414,7 +662,9 @@ const char* mamba_status_string(mm_status status) {
         case MM_ERR_CUDA: return "CUDA runtime error at launch";
         case MM_ERR_DEVICE: return "no usable sm_100 device is current";
         case MM_ERR_WORKSPACE: return "workspace missing or smaller than mamba_mixer_workspace_size()";
-        case MM_ERR_TIMEOUT: return "a kernel gave up waiting for its bulk copies (see mamba_mixer_fault_status)";
+        case MM_ERR_TIMEOUT:
+            return "a kernel of the call gave up waiting (for its bulk copies, or for a chunk summary that was "
+                   "never written); its outputs are not valid";
         case MM_ERR_SCRATCH_LIMIT:
             return "sizes need more scratch than mamba_mixer_fwd_noalloc's built-in 8 MiB; pass a workspace to "
                    "mamba_mixer_fwd instead";
@@ -432,13 +682,31 @@ mm_status mamba_mixer_fault_status(int reset) {
     return v ? MM_ERR_TIMEOUT : MM_OK;
 }
 
+mm_status mamba_check_status(const void* workspace, void* stream) {
+    const void* ws = workspace;
+    if (!ws) {
+        void* p = nullptr;
+        if (mm_status st = noalloc_scratch(&p); st != MM_OK) return st;
+        ws = p;
+    }
+    if (!aligned16(ws)) return MM_ERR_ALIGN;
+    unsigned long long hdr[2] = {0, 0};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(hdr, ws, sizeof(hdr), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
+        cudaGetLastError();
+        return MM_ERR_CUDA;
+    }
+    return (hdr[0] & 0xff) != 0 && (hdr[0] >> 8) == hdr[1] ? MM_ERR_TIMEOUT : MM_OK;
+}
+
 size_t mamba_mixer_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state,
                                   int64_t d_conv, mm_dtype act) {
-    if ((act != MM_F32 && act != MM_BF16) || batch <= 0 || seqlen <= 0 || d_inner <= 0 || d_state != 16 ||
+    if ((act != MM_F32 && act != MM_BF16) || batch <= 0 || seqlen < 0 || d_inner <= 0 || d_state != 16 ||
         d_conv != 4 || d_inner % 8 != 0 || d_inner > (1 << 24) || batch > (1 << 24) ||
         !seqlen_ok(seqlen, d_inner, act == MM_F32 ? 4 : 2))
         return 0;
-    return plan_fwd(batch, seqlen, d_inner).ws_bytes;
+    return plan_fwd(batch, seqlen, d_inner, plan_sms()).ws_bytes;
 }
 
 mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv_b,
@@ -450,67 +718,18 @@ mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv
                           int64_t d_state, int64_t d_conv, mm_dtype act,
                           void* workspace, size_t workspace_bytes, void* stream)
 {
-    if (act != MM_F32 && act != MM_BF16) return MM_ERR_DTYPE;
-    if (batch < 0 || seqlen < 0 || d_inner <= 0 || d_state <= 0 || d_conv <= 0) return MM_ERR_SHAPE;
-    if (d_state != 16 || d_conv != 4 || d_inner % 8 != 0) return MM_ERR_UNSUPPORTED;
-    if (d_inner > (1 << 24) || batch > (1 << 24)) return MM_ERR_SHAPE;
-    const int64_t es = act == MM_F32 ? 4 : 2;
-    if (!seqlen_ok(seqlen, d_inner, es)) return MM_ERR_SHAPE;
-    int64_t tokens, xz_bytes, dt_bytes, bc_bytes, st_bytes;
-    if (!mul_ok(batch, seqlen, &tokens) || !mul_ok(tokens, 2 * d_inner * es, &xz_bytes) ||
-        !mul_ok(tokens, d_inner * es, &dt_bytes) || !mul_ok(tokens, d_state * es, &bc_bytes) ||
-        !mul_ok(batch, d_inner * d_state * 4, &st_bytes))
-        return MM_ERR_SHAPE;
-    const int64_t cs_bytes = batch * d_inner * (d_conv - 1) * es;
+    const FwdArgs a{xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0, conv_state_in, y, h_last,
+                    conv_state_out, batch, seqlen, d_inner, d_state, d_conv, act};
+    FwdBytes nb;
+    if (mm_status st = validate_fwd(a, &nb); st != MM_OK) return st;
     if (batch == 0) return MM_OK;
-
-    // required pointers
-    if (!conv_w || !dt_bias || !A || !h_last || !conv_state_out) return MM_ERR_NULL;
-    if (seqlen > 0 && (!xz || !dt || !Bm || !Cm || !y)) return MM_ERR_NULL;
-    const void* all[] = {xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0, conv_state_in,
-                         y, h_last, conv_state_out};
-    for (const void* q : all)
-        if (q && !aligned16(q)) return MM_ERR_ALIGN;
-
-    const Span in[] = {span(xz, xz_bytes), span(conv_w, d_inner * d_conv * 4), span(conv_b, d_inner * 4),
-                       span(dt, dt_bytes), span(dt_bias, d_inner * 4), span(A, d_inner * d_state * 4),
-                       span(Bm, bc_bytes), span(Cm, bc_bytes), span(Dskip, d_inner * 4),
-                       span(h0, st_bytes), span(conv_state_in, cs_bytes)};
-    const Span out[] = {span(y, dt_bytes), span(h_last, st_bytes), span(conv_state_out, cs_bytes)};
-    for (const Span& o : out)
-        for (const Span& i : in)
-            if (overlaps(o, i)) return MM_ERR_ALIAS;
-    if (overlaps(out[0], out[1]) || overlaps(out[0], out[2]) || overlaps(out[1], out[2])) return MM_ERR_ALIAS;
-
-    const FwdPlan pl = plan_fwd(batch, seqlen, d_inner);
-    if (pl.ws_bytes > 0) {
-        if (!workspace || workspace_bytes < pl.ws_bytes) return MM_ERR_WORKSPACE;
-        if (!aligned16(workspace)) return MM_ERR_ALIGN;
-        const Span ws = span(workspace, static_cast<int64_t>(pl.ws_bytes));
-        for (const Span& i : in)
-            if (overlaps(ws, i)) return MM_ERR_ALIAS;
-        for (const Span& o : out)
-            if (overlaps(ws, o)) return MM_ERR_ALIAS;
-    }
-
-    int sm_count = 0;
-    if (mm_status st = check_device(&sm_count); st != MM_OK) return st;
-
-    PrefillParams p{};
-    p.xz = xz; p.conv_w = conv_w; p.conv_b = conv_b; p.dt = dt; p.dt_bias = dt_bias; p.A = A;
-    p.Bm = Bm; p.Cm = Cm; p.Dskip = Dskip; p.h0 = h0; p.cs_in = conv_state_in;
-    p.y = y; p.h_last = h_last; p.cs_out = conv_state_out;
-    p.L = seqlen;
-    p.D = static_cast<int>(d_inner);
-    p.batch = static_cast<int>(batch);
-    p.wait_limit = copy_wait_limit();
-    p.ws_state = static_cast<float*>(workspace);
-    p.ws_lsum = pl.ws_bytes ? p.ws_state + static_cast<int64_t>(pl.chunks - 1) * batch * d_inner * 16 : nullptr;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = act == MM_BF16 ? dispatch_prefill<__nv_bfloat16, mm::MathFast>(p, batch, pl, sm_count, s)
-                                   : dispatch_prefill<float, mm::MathExact>(p, batch, pl, sm_count, s);
-    if (e != cudaSuccess) { cudaGetLastError(); return MM_ERR_CUDA; }
-    return MM_OK;
+    const int sms = plan_sms();
+    const FwdPlan pl = plan_fwd(batch, seqlen, d_inner, sms);
+    if (!workspace || workspace_bytes < pl.ws_bytes) return MM_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MM_ERR_ALIGN;
+    if (workspace_overlaps(a, nb, workspace, pl.ws_bytes)) return MM_ERR_ALIAS;
+    if (mm_status st = check_device(); st != MM_OK) return st;
+    return run_fwd(a, pl, sms, workspace, next_call_id(), static_cast<cudaStream_t>(stream));
 }
 
 mm_status mamba_state_update(const void* x, const void* z, const void* dt,
@@ -552,8 +771,7 @@ mm_status mamba_state_update(const void* x, const void* z, const void* dt,
             if (overlaps(o, i)) return MM_ERR_ALIAS;
     if (overlaps(io[0], io[1]) || overlaps(io[0], io[2]) || overlaps(io[1], io[2])) return MM_ERR_ALIAS;
 
-    int sm_count = 0;
-    if (mm_status st = check_device(&sm_count); st != MM_OK) return st;
+    if (mm_status st = check_device(); st != MM_OK) return st;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const unsigned grid = static_cast<unsigned>((warps + 7) / 8);
@@ -583,15 +801,18 @@ mm_status mamba_mixer_fwd_noalloc(const void* xz, const float* conv_w, const flo
                                   int64_t batch, int64_t seqlen, int64_t d_inner,
                                   int64_t d_state, int64_t d_conv, mm_dtype act, void* stream)
 {
-    const size_t need = mamba_mixer_workspace_size(batch, seqlen, d_inner, d_state, d_conv, act);
-    if (need > MAMBA_MIXER_NOALLOC_SCRATCH_BYTES) return MM_ERR_SCRATCH_LIMIT;
+    const FwdArgs a{xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0, conv_state_in, y, h_last,
+                    conv_state_out, batch, seqlen, d_inner, d_state, d_conv, act};
+    FwdBytes nb;
+    if (mm_status st = validate_fwd(a, &nb); st != MM_OK) return st;
+    if (batch == 0) return MM_OK;
+    const int sms = plan_sms();
+    const FwdPlan pl = plan_fwd(batch, seqlen, d_inner, sms);
+    if (pl.ws_bytes > MAMBA_MIXER_NOALLOC_SCRATCH_BYTES) return MM_ERR_SCRATCH_LIMIT;
+    if (mm_status st = check_device(); st != MM_OK) return st;
     void* scratch = nullptr;
-    if (need > 0) {
-        if (mm_status st = noalloc_scratch(&scratch); st != MM_OK) return st;
-    }
-    return mamba_mixer_fwd(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0, conv_state_in, y, h_last,
-                           conv_state_out, batch, seqlen, d_inner, d_state, d_conv, act, scratch,
-                           need > 0 ? MAMBA_MIXER_NOALLOC_SCRATCH_BYTES : 0, stream);
+    if (mm_status st = noalloc_scratch(&scratch); st != MM_OK) return st;
+    return run_fwd(a, pl, sms, scratch, next_call_id(), static_cast<cudaStream_t>(stream));
 }
 
 size_t mamba_mixer_host_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state,
@@ -602,7 +823,7 @@ size_t mamba_mixer_host_workspace_size(int64_t batch, int64_t seqlen, int64_t d_
     int64_t tokens, bytes;
     if (!mul_ok(batch, seqlen, &tokens) || !mul_ok(tokens, 2 * d_inner * 4, &bytes)) return 0;
     const int64_t es = act == MM_F32 ? 4 : 2;
-    const HostPlan hp = plan_host(batch, seqlen, d_inner, es);
+    const HostPlan hp = plan_host(batch, seqlen, d_inner, es, plan_sms());
     return seqlen_ok(hp.piece, d_inner, es) ? hp.total : 0;
 }
 
@@ -616,17 +837,10 @@ mm_status mamba_mixer_fwd_host(const void* xz, const float* conv_w, const float*
                                void* workspace, size_t workspace_bytes,
                                void* stream, void* h2d_stream, void* d2h_stream)
 {
-    if (act != MM_F32 && act != MM_BF16) return MM_ERR_DTYPE;
-    if (batch < 0 || seqlen < 0 || d_inner <= 0 || d_state <= 0 || d_conv <= 0) return MM_ERR_SHAPE;
-    if (d_state != 16 || d_conv != 4 || d_inner % 8 != 0) return MM_ERR_UNSUPPORTED;
-    if (d_inner > (1 << 24) || batch > (1 << 24)) return MM_ERR_SHAPE;
-    const int64_t es = act == MM_F32 ? 4 : 2;
-    int64_t tokens, xz_bytes, dt_bytes, bc_bytes, st_bytes;
-    if (!mul_ok(batch, seqlen, &tokens) || !mul_ok(tokens, 2 * d_inner * es, &xz_bytes) ||
-        !mul_ok(tokens, d_inner * es, &dt_bytes) || !mul_ok(tokens, d_state * es, &bc_bytes) ||
-        !mul_ok(batch, d_inner * d_state * 4, &st_bytes))
-        return MM_ERR_SHAPE;
-    const int64_t cs_bytes = batch * d_inner * (d_conv - 1) * es;
+    const FwdArgs a{xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0, conv_state_in, y, h_last,
+                    conv_state_out, batch, seqlen, d_inner, d_state, d_conv, act};
+    FwdBytes nb;
+    if (mm_status st = check_sizes(a, &nb); st != MM_OK) return st;
     if (batch == 0) return MM_OK;
 
     if (!conv_w || !dt_bias || !A || !h_last || !conv_state_out) return MM_ERR_NULL;
@@ -636,28 +850,40 @@ mm_status mamba_mixer_fwd_host(const void* xz, const float* conv_w, const float*
     for (const void* q : dev_ptrs)
         if (q && !aligned16(q)) return MM_ERR_ALIGN;
     // host outputs may not overlap host inputs
-    const Span in[] = {span(xz, xz_bytes), span(dt, dt_bytes), span(Bm, bc_bytes), span(Cm, bc_bytes),
-                       span(h0, st_bytes), span(conv_state_in, cs_bytes)};
-    const Span out[] = {span(y, dt_bytes), span(h_last, st_bytes), span(conv_state_out, cs_bytes)};
+    const Span in[] = {span(xz, nb.xz), span(dt, nb.dt), span(Bm, nb.bc), span(Cm, nb.bc),
+                       span(h0, nb.st), span(conv_state_in, nb.cs)};
+    const Span out[] = {span(y, nb.dt), span(h_last, nb.st), span(conv_state_out, nb.cs)};
     for (const Span& o : out)
         for (const Span& i : in)
             if (overlaps(o, i)) return MM_ERR_ALIAS;
     if (overlaps(out[0], out[1]) || overlaps(out[0], out[2]) || overlaps(out[1], out[2])) return MM_ERR_ALIAS;
 
-    const HostPlan hp = plan_host(batch, seqlen, d_inner, es);
+    const int64_t es = nb.es;
+    const int sms = plan_sms();
+    const HostPlan hp = plan_host(batch, seqlen, d_inner, es, sms);
     if (!seqlen_ok(hp.piece, d_inner, es)) return MM_ERR_SHAPE;   // each piece is one device call
     if (!workspace || workspace_bytes < hp.total) return MM_ERR_WORKSPACE;
     if (!aligned16(workspace)) return MM_ERR_ALIGN;
-    int sm_count = 0;
-    if (mm_status st = check_device(&sm_count); st != MM_OK) return st;
+    // the device parameters may not overlap the workspace the pieces are staged in
+    {
+        const Span w = span(workspace, static_cast<int64_t>(hp.total));
+        const Span par[] = {span(conv_w, d_inner * d_conv * 4), span(conv_b, d_inner * 4),
+                            span(dt_bias, d_inner * 4), span(A, d_inner * d_state * 4), span(Dskip, d_inner * 4)};
+        for (const Span& q : par)
+            if (overlaps(w, q)) return MM_ERR_ALIAS;
+    }
+    if (mm_status st = check_device(); st != MM_OK) return st;
 
     cudaStream_t sc = static_cast<cudaStream_t>(stream);
     cudaStream_t s_in = static_cast<cudaStream_t>(h2d_stream);
     cudaStream_t s_out = static_cast<cudaStream_t>(d2h_stream);
     unsigned char* ws = static_cast<unsigned char*>(workspace);
-    unsigned char* slot[2] = {ws, ws + hp.slot};
-    unsigned char* carry[2] = {ws + 2 * hp.slot, ws + 2 * hp.slot + hp.carry};
-    void* fwd_ws = hp.fwd_ws ? ws + 2 * hp.slot + 2 * hp.carry : nullptr;
+    void* fwd_ws = ws;
+    unsigned char* slot[2] = {ws + hp.fwd_ws, ws + hp.fwd_ws + hp.slot};
+    unsigned char* carry[2] = {ws + hp.fwd_ws + 2 * hp.slot, ws + hp.fwd_ws + 2 * hp.slot + hp.carry};
+    // every piece records its failures under the call's one epoch, so the
+    // workspace's status reports a failure of any piece
+    const unsigned long long epoch = next_call_id();
 
     HostEvents evs;
     cudaEvent_t ev_start = evs.make(), ev_final = evs.make();
@@ -681,9 +907,9 @@ mm_status mamba_mixer_fwd_host(const void* xz, const float* conv_w, const float*
     chk(cudaEventRecord(ev_start, sc));
     chk(cudaStreamWaitEvent(s_in, ev_start, 0));
     chk(cudaStreamWaitEvent(s_out, ev_start, 0));
-    if (h0) chk(cudaMemcpyAsync(carry[0], h0, static_cast<size_t>(st_bytes), cudaMemcpyHostToDevice, s_in));
+    if (h0) chk(cudaMemcpyAsync(carry[0], h0, static_cast<size_t>(nb.st), cudaMemcpyHostToDevice, s_in));
     if (conv_state_in)
-        chk(cudaMemcpyAsync(carry[0] + hp.carry_h, conv_state_in, static_cast<size_t>(cs_bytes),
+        chk(cudaMemcpyAsync(carry[0] + hp.carry_h, conv_state_in, static_cast<size_t>(nb.cs),
                             cudaMemcpyHostToDevice, s_in));
 
     for (int64_t i = 0; ok && i < hp.pieces; ++i) {
@@ -710,14 +936,13 @@ mm_status mamba_mixer_fwd_host(const void* xz, const float* conv_w, const float*
         unsigned char* cin = carry[i & 1];
         unsigned char* cout = carry[(i + 1) & 1];
         const bool first = i == 0;
-        const float* h_in = (first && !h0) ? nullptr : reinterpret_cast<const float*>(cin);
-        const void* cs_in = (first && !conv_state_in) ? nullptr : cin + hp.carry_h;
         if (!ok) break;
-        fwd_status = mamba_mixer_fwd(sl, conv_w, conv_b, sl + hp.off_dt, dt_bias, A, sl + hp.off_b,
-                                             sl + hp.off_c, Dskip, h_in, cs_in, sl + hp.off_y,
-                                             reinterpret_cast<float*>(cout), cout + hp.carry_h, batch,
-                                             static_cast<int64_t>(n), d_inner, d_state, d_conv, act, fwd_ws,
-                                             hp.fwd_ws, sc);
+        const FwdArgs pa{sl, conv_w, conv_b, sl + hp.off_dt, dt_bias, A, sl + hp.off_b, sl + hp.off_c, Dskip,
+                         (first && !h0) ? nullptr : reinterpret_cast<const float*>(cin),
+                         (first && !conv_state_in) ? nullptr : cin + hp.carry_h, sl + hp.off_y,
+                         reinterpret_cast<float*>(cout), cout + hp.carry_h, batch, static_cast<int64_t>(n),
+                         d_inner, d_state, d_conv, act};
+        fwd_status = run_fwd(pa, plan_fwd(batch, static_cast<int64_t>(n), d_inner, sms), sms, fwd_ws, epoch, sc);
         if (fwd_status != MM_OK) break;
         chk(cudaEventRecord(ev_done[j], sc));
         // y of piece i -> host; the slot is free again after this copy
@@ -732,8 +957,8 @@ mm_status mamba_mixer_fwd_host(const void* xz, const float* conv_w, const float*
     // before releasing its buffers)
     if (ok && fwd_status == MM_OK) {
         unsigned char* cl = carry[hp.pieces & 1];
-        chk(cudaMemcpyAsync(h_last, cl, static_cast<size_t>(st_bytes), cudaMemcpyDeviceToHost, s_out));
-        chk(cudaMemcpyAsync(conv_state_out, cl + hp.carry_h, static_cast<size_t>(cs_bytes),
+        chk(cudaMemcpyAsync(h_last, cl, static_cast<size_t>(nb.st), cudaMemcpyDeviceToHost, s_out));
+        chk(cudaMemcpyAsync(conv_state_out, cl + hp.carry_h, static_cast<size_t>(nb.cs),
                             cudaMemcpyDeviceToHost, s_out));
     }
     const bool fenced = cudaEventRecord(ev_final, s_out) == cudaSuccess &&

@@ -107,9 +107,24 @@ struct PrefillParams {
     int n_chunks;       // time chunks K (blockIdx.y of the full pass)
     float* ws_state;    // [K-1][batch][16][D]: end state of chunk c run from zero (state-major)
     float* ws_lsum;     // [K-1][batch][D]:     sum over chunk c of the step size l
+    // Per-call status, in the caller's workspace.  hdr[0] = (epoch << 8) |
+    // code of a failure (kStatusCopyTimeout, kStatusNoSummary), written by any
+    // CTA that fails; hdr[1] = the epoch of the last call that ran on this
+    // workspace.  The call failed iff hdr[0] >> 8 == hdr[1] and its code is set.
+    unsigned long long* ws_hdr;
+    // [K-1][batch][D/8]: for chunk c, sequence b and each summary-pass CTA
+    // (indexed by its first channel octet), the id of the call whose summary
+    // pass stored that CTA's chunk summaries.  A CTA that gave up writes none.
+    unsigned long long* ws_tags;
+    unsigned long long call_id;       // unique per launch pair (summary + full pass)
+    unsigned long long status_epoch;  // the epoch hdr[] is written with
+    int sum_octets;     // channel octets per summary-pass CTA (its tag stride)
     int batch;
     unsigned wait_limit;  // tries per wait on a bulk copy before giving up (fault)
 };
+
+constexpr unsigned long long kStatusCopyTimeout = 1;  // a wait on the CTA's own bulk copies gave up
+constexpr unsigned long long kStatusNoSummary = 2;    // a chunk summary this CTA starts from was not written
 
 constexpr int kHalo = 3;   // conv left context rows (d_conv - 1)
 
@@ -256,6 +271,21 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
     // summary pass: its CTAs can then be placed on free SMs, run their setup
     // and chunk 0 meanwhile, and wait only before reading the summaries.
     if constexpr (SUMMARY) launch_dependents();
+    // this call is the last one to run on the workspace
+    if (!SUMMARY && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) p.ws_hdr[1] = p.status_epoch;
+    // record a failure of this CTA in the call's status and the device fault word
+    auto fail = [&](unsigned long long code) {
+        if (tid == 0) {
+            atomicOr(&g_mm_fault, 1u);
+            atomicExch(p.ws_hdr, (p.status_epoch << 8) | code);
+        }
+    };
+    // let the copies issued for walked tiles k0 .. k0+STAGES-2 land before the
+    // CTA's shared memory goes away (each wait bounded)
+    auto drain = [&](int64_t k0) {
+        for (int64_t j = k0; j < min(ntiles, k0 + STAGES - 1); ++j)
+            mbar_wait_bounded(&bars[j % STAGES], static_cast<unsigned>((j / STAGES) & 1), 1u << 20);
+    };
 
     // ---------------------------------------------------------- pipeline prologue (the first tiles stream in during the setup)
     if (tid == 0) {
@@ -325,7 +355,26 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
         // carry h0 through the summaries of the chunks before this one:
         // h <- exp(A sum Delta) h + e, the summaries read state-major so that
         // a warp's loads of one state are contiguous
-        if (chunk > 0) grid_dependency_wait();   // the summaries of chunks 0..chunk-1 (no-op when launched normally)
+        if (chunk > 0) {
+            grid_dependency_wait();   // the summaries of chunks 0..chunk-1 (no-op when launched normally)
+            // every summary-pass CTA covering my channels must have stored its
+            // summaries of chunks 0..chunk-1 in this call; else the carry would
+            // read stale values: record the failure and write nothing
+            bool ok = true;
+            if (tid == 0) {
+                const int span = 8 * p.sum_octets;
+                const int64_t octs = D / 8;
+                for (int c = 0; c < chunk; ++c)
+                    for (int sb = d0 / span; sb <= (d0 + nch - 1) / span; ++sb)
+                        ok &= p.ws_tags[(static_cast<int64_t>(c) * p.batch + seq) * octs +
+                                        static_cast<int64_t>(sb) * p.sum_octets] == p.call_id;
+            }
+            if (__syncthreads_or(!ok)) {
+                fail(kStatusNoSummary);
+                drain(0);
+                return;
+            }
+        }
         if (active && chunk > 0) {
             const int64_t stride = static_cast<int64_t>(p.batch) * D;
 #pragma unroll 1
@@ -494,10 +543,8 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
             const int slot = static_cast<int>(k % STAGES);
             const bool landed = mbar_wait_bounded(&bars[slot], static_cast<unsigned>((k / STAGES) & 1), p.wait_limit);
             if (__syncthreads_or(!landed)) {
-                if (tid == 0) atomicOr(&g_mm_fault, 1u);
-                // let the copies already issued land before the CTA's shared memory goes away
-                for (int64_t j = k; j < min(ntiles, k + STAGES - 1); ++j)
-                    mbar_wait_bounded(&bars[j % STAGES], static_cast<unsigned>((j / STAGES) & 1), 1u << 20);
+                fail(kStatusCopyTimeout);
+                drain(k);
                 return false;
             }
             unsigned char* st = smem + slot * stageB;
@@ -554,6 +601,11 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
             for (int n = 0; n < 16; ++n) *reinterpret_cast<float2*>(e + static_cast<int64_t>(n) * D) = h[n];
             *reinterpret_cast<float2*>(p.ws_lsum + chunk * stride + chan) = lsum;
         }
+        // this CTA's summaries are stored (the full pass reads them only after
+        // this grid has completed, so no fence is needed)
+        __syncthreads();
+        if (tid == 0)
+            p.ws_tags[(static_cast<int64_t>(chunk) * p.batch + seq) * (D / 8) + d0 / 8] = p.call_id;
     } else if (active && chunk == p.n_chunks - 1) {
         // my two channels' rows of h_last: 128 contiguous bytes, in 16-byte stores
         float4* hl = reinterpret_cast<float4*>(p.h_last + chan * 16);

@@ -47,6 +47,17 @@ def np64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu").to(torch.float64).numpy()
 
 
+# Worst error / bound of every comparison made in this session, printed in
+# pytest's terminal summary (conftest.py) so a drift toward the tolerance shows
+# before it fails: (test id, tensor name, elements compared, margin).
+MARGINS = []
+
+
+def _record(name, n, margin):
+    test = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    MARGINS.append((test, name, int(n), float(margin)))
+
+
 def assert_close(got, ref, act: str, name: str, stored_bf16: bool = False):
     """fp32: |err| <= 1e-4 (1 + |ref|) elementwise.
 
@@ -64,17 +75,22 @@ def assert_close(got, ref, act: str, name: str, stored_bf16: bool = False):
     err = np.abs(got - ref)
     if act == "f32":
         bound = F32_RTOL * (1.0 + np.abs(ref))
-        worst = np.max(err / bound) if err.size else 0.0
+        worst = float(np.max(err / bound)) if err.size else 0.0
+        _record(name, err.size, worst)
         assert worst <= 1.0, f"{name}: max err/bound {worst:.3g} (max err {err.max():.3g})"
-        return
+        return worst
     if not err.size:
-        return
+        return 0.0
     rms = float(np.sqrt(np.mean(ref ** 2)))
     excess = err - (BF16_HALF_ULP * np.abs(ref) if stored_bf16 else 0.0)
     mx = float(excess.max())
-    assert mx <= BF16_FRAC * rms + 1e-30, f"{name}: max err beyond output rounding {mx:.3g} > {BF16_FRAC} * rms {rms:.3g}"
     rerr = float(np.sqrt(np.mean(err ** 2)))
-    assert rerr <= BF16_FRAC * rms + 1e-30, f"{name}: rms err {rerr:.3g} > {BF16_FRAC} * rms {rms:.3g}"
+    bound = BF16_FRAC * rms + 1e-30
+    worst = max(mx, rerr) / bound
+    _record(name, err.size, worst)
+    assert mx <= bound, f"{name}: max err beyond output rounding {mx:.3g} > {BF16_FRAC} * rms {rms:.3g}"
+    assert rerr <= bound, f"{name}: rms err {rerr:.3g} > {BF16_FRAC} * rms {rms:.3g}"
+    return worst
 
 
 def decode_args(inp: dict):

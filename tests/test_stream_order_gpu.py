@@ -109,7 +109,7 @@ def test_calls_on_a_side_stream_with_binding_allocations():
     from workloads import make_decode_inputs_custom
 
     dev = to_dev(make_mixer_inputs_custom(1, 2048, 1032, act="bf16", seed=96, h0_std=0.3, conv_state_std=1.0))
-    assert mm.workspace_size(1, 2048, 1032) > 0          # a chunked plan: the binding allocates scratch
+    assert mm.workspace_size(1, 2048, 1032) > 256        # a chunked plan: the binding allocates scratch
     ref = gpu_fwd(dev)
     torch.cuda.synchronize()
     side = torch.cuda.Stream()
