@@ -54,6 +54,8 @@ def _declare(lib):
     lib.oracle_mixer_fwd.argtypes = [P] * 17 + [I] * 7
     lib.oracle_state_update.restype = ctypes.c_int
     lib.oracle_state_update.argtypes = [P] * 13 + [I] * 7
+    lib.oracle_rmsnorm_rows.restype = ctypes.c_int
+    lib.oracle_rmsnorm_rows.argtypes = [P, P, ctypes.c_double, P, I, I]
     return lib
 
 
@@ -159,3 +161,44 @@ def state_update(x, z, dt, conv_w, conv_b, dt_bias, Dskip, A, Bm, Cm, ssm_state,
         with ThreadPoolExecutor(max_workers=len(parts)) as ex:
             list(ex.map(run, parts))
     return {"ssm_state": ssm, "conv_state": cs, "y": y}
+
+
+def rmsnorm_rows(x, w, eps: float, library=None):
+    """RMSNorm over the last axis with one weight per entry of that axis:
+    x * w / sqrt(mean(x^2) + eps), in float64 (oracle_rmsnorm_rows)."""
+    L_ = library or lib()
+    x = _f64(x)
+    w = _f64(w)
+    n = x.shape[-1]
+    assert w.shape == (n,)
+    out = np.zeros_like(x)
+    rc = L_.oracle_rmsnorm_rows(_p(x), _p(w), float(eps), _p(out), x.size // n, n)
+    if rc != 0:
+        raise ValueError(f"oracle_rmsnorm_rows rejected its arguments (rc={rc})")
+    return out
+
+
+def mixer_fwd_normed(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, conv_state_in=None,
+                     b_norm_w=None, c_norm_w=None, norm_eps: float = 1e-6, threads: int = 1, library=None):
+    """The forward with B_t and C_t each RMS-normalised over d_state first
+    (a weight of None leaves that input as it is)."""
+    Bn = rmsnorm_rows(Bm, b_norm_w, norm_eps, library) if b_norm_w is not None else Bm
+    Cn = rmsnorm_rows(Cm, c_norm_w, norm_eps, library) if c_norm_w is not None else Cm
+    return mixer_fwd(xz, conv_w, conv_b, dt, dt_bias, A, Bn, Cn, Dskip, h0, conv_state_in, threads=threads,
+                     library=library)
+
+
+def state_update_normed(x, z, dt, conv_w, conv_b, dt_bias, Dskip, A, Bm, Cm, ssm_state, conv_state,
+                        b_norm_w=None, c_norm_w=None, norm_eps: float = 1e-6, threads: int = 1, library=None):
+    """The decode step with each layer's B and C rows RMS-normalised over
+    d_state first, with that layer's weights ([NL, N]; None = not normalised)."""
+    def per_layer(M, w):
+        if w is None:
+            return M
+        M = _f64(M)
+        w = _f64(w)
+        return np.stack([rmsnorm_rows(M[l], w[l], norm_eps, library) for l in range(M.shape[0])])
+
+    return state_update(x, z, dt, conv_w, conv_b, dt_bias, Dskip, A, per_layer(Bm, b_norm_w),
+                        per_layer(Cm, c_norm_w), ssm_state, conv_state, threads=threads, library=library)
+

@@ -28,7 +28,10 @@
  *     tokens of left context), the left context being conv_state_in (raw,
  *     pre-conv x, oldest first) or zeros;
  *   - the skip term D multiplies u, the same conv+SiLU output that enters B x;
- *   - the gate multiplies the sum (C h + D u) by SiLU(z); no norm on the path;
+ *   - the gate multiplies the sum (C h + D u) by SiLU(z); no norm between the
+ *     readout and the gate.  The RMSNorm the pages place inside the Mamba
+ *     layer is taken to act on B_t and C_t before the recurrence
+ *     (oracle_rmsnorm_rows, at the end of this file), and is optional;
  *   - A is given directly as a (negative) fp32 [D, N] matrix, not as log(-A);
  *   - one B/C group shared by all channels of a sequence;
  *   - softplus(v) = max(v, 0) + log1p(exp(-|v|)), exact for every v.
@@ -187,3 +190,26 @@ int oracle_state_update(const double* x, const double* z, const double* dt,
     }
     return OR_OK;
 }
+
+/*
+ * RMSNorm of each row of a [rows, n] matrix, with one weight per column.
+ * Jamba deep-dive report, "standard components" list: RMSNorm sits inside the
+ * Mamba layer; large-scale-stability section: it is applied to the layer's
+ * internal activations.  Reading taken (the pages do not say which
+ * activations): the selective parameters B_t and C_t, each normalised over
+ * its d_state entries before it enters the recurrence:
+ *
+ *     out[r, i] = x[r, i] * w[i] / sqrt(mean_j x[r, j]^2 + eps)
+ */
+int oracle_rmsnorm_rows(const double* x, const double* w, double eps, double* out, int64_t rows, int64_t n)
+{
+    if (rows < 0 || n < 1 || !x || !w || !out || !(eps >= 0.0)) return OR_ERR_ARG;
+    for (int64_t r = 0; r < rows; ++r) {
+        double ss = 0.0;
+        for (int64_t i = 0; i < n; ++i) ss += x[r * n + i] * x[r * n + i];
+        const double inv = 1.0 / sqrt(ss / (double)n + eps);
+        for (int64_t i = 0; i < n; ++i) out[r * n + i] = x[r * n + i] * inv * w[i];
+    }
+    return OR_OK;
+}
+

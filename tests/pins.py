@@ -338,7 +338,71 @@ def pin_channel_split(lib):
         assert np.array_equal(a[k], b[k])
 
 
+def pin_rmsnorm_constant_rows(lib):
+    """A row of n equal entries c with unit weights normalises to
+    c / sqrt(c^2 + eps) in every entry (closed form)."""
+    n = 16
+    for c, eps in ((3.0, 0.25), (-0.5, 1e-6), (0.0, 0.5), (1e-3, 1e-6)):
+        out = oracle.rmsnorm_rows(np.full((2, n), c), np.ones(n), eps, library=lib)
+        np.testing.assert_allclose(out, c / np.sqrt(c * c + eps), rtol=1e-14, atol=1e-300)
+
+
+def pin_rmsnorm_library(lib):
+    """Random rows and per-column weights against torch's rms_norm in float64
+    (library routine), with a small and a large eps."""
+    import torch
+
+    rng = np.random.default_rng(41)
+    x = rng.standard_normal((37, 16)) * rng.uniform(0.1, 5.0, (37, 1))
+    w = rng.uniform(0.2, 2.0, 16)
+    for eps in (1e-6, 0.3):
+        ref = torch.nn.functional.rms_norm(torch.from_numpy(x), (16,), torch.from_numpy(w), eps).numpy()
+        np.testing.assert_allclose(oracle.rmsnorm_rows(x, w, eps, library=lib), ref, rtol=1e-12, atol=1e-15)
+
+
+def pin_rmsnorm_homogeneity(lib):
+    """Scaling a row by a and eps by a^2 leaves the result unchanged; scaling
+    the weights by k scales it by k; the normalised row/weight has mean square
+    ms / (ms + eps)."""
+    rng = np.random.default_rng(42)
+    x = rng.standard_normal((9, 16))
+    w = rng.uniform(0.5, 1.5, 16)
+    base = oracle.rmsnorm_rows(x, w, 0.1, library=lib)
+    np.testing.assert_allclose(oracle.rmsnorm_rows(7.0 * x, w, 0.1 * 49.0, library=lib), base, rtol=1e-13)
+    np.testing.assert_allclose(oracle.rmsnorm_rows(x, 3.0 * w, 0.1, library=lib), 3.0 * base, rtol=1e-13)
+    ms = np.mean(x ** 2, axis=-1)
+    np.testing.assert_allclose(np.mean((base / w) ** 2, axis=-1), ms / (ms + 0.1), rtol=1e-13)
+
+
+def pin_normed_forward_uses_normalised_B_and_C(lib):
+    """With every B_t (and C_t) row constant, RMSNorm with weights w turns it
+    into w * c / sqrt(c^2 + eps): the normed forward equals the plain forward
+    on those values, and a weight of None leaves the input untouched."""
+    rng = np.random.default_rng(43)
+    case = _rand_case(rng, 1, 12, 3, 16)
+    cb = rng.uniform(0.5, 2.0, (1, 12, 1))
+    cc = rng.uniform(-2.0, -0.5, (1, 12, 1))
+    case["Bm"] = np.repeat(cb, 16, axis=-1)
+    case["Cm"] = np.repeat(cc, 16, axis=-1)
+    wb, wc, eps = rng.uniform(0.5, 1.5, 16), rng.uniform(0.5, 1.5, 16), 0.2
+    got = oracle.mixer_fwd_normed(case["xz"], case["conv_w"], case["conv_b"], case["dt"], case["dt_bias"],
+                                  case["A"], case["Bm"], case["Cm"], case["Dskip"], case["h0"],
+                                  case["conv_state_in"], b_norm_w=wb, c_norm_w=wc, norm_eps=eps, library=lib)
+    want_case = dict(case, Bm=wb * cb / np.sqrt(cb * cb + eps), Cm=wc * cc / np.sqrt(cc * cc + eps))
+    want = _fwd(lib, want_case)
+    for k in ("y", "h_last"):
+        np.testing.assert_allclose(got[k], want[k], rtol=1e-12, atol=1e-14)
+    plain = oracle.mixer_fwd_normed(case["xz"], case["conv_w"], case["conv_b"], case["dt"], case["dt_bias"],
+                                    case["A"], case["Bm"], case["Cm"], case["Dskip"], case["h0"],
+                                    case["conv_state_in"], library=lib)
+    np.testing.assert_array_equal(plain["y"], _fwd(lib, case)["y"])
+
+
 ALL_PINS = [
+    pin_rmsnorm_constant_rows,
+    pin_rmsnorm_library,
+    pin_rmsnorm_homogeneity,
+    pin_normed_forward_uses_normalised_B_and_C,
     pin_lti_closed_form,
     pin_brute_force_selective,
     pin_zero_input,

@@ -1,7 +1,7 @@
 """Plants plausible mistakes in copies of the oracle (on the CPU) and checks
 that each one makes at least one pin fail, so the pins really constrain every
 step of the oracle: conv, SiLU, softplus, discretisation, recurrence, readout,
-skip, gate, carried state and the decode step."""
+skip, gate, carried state, the decode step and the RMSNorm of B and C."""
 
 import os
 
@@ -46,6 +46,16 @@ MUTANTS = [
     ("decode_window_not_shifted", "for (int64_t k = 0; k + 1 < W - 1; ++k) cs[k] = cs[k + 1];", ""),
     ("decode_params_of_layer0", "const int64_t ld = l * D + d;", "const int64_t ld = d;"),
     ("decode_no_skip", "y[r] = (acc + (Dskip ? Dskip[ld] : 0.0) * u) * or_silu(z[r]);", "y[r] = acc * or_silu(z[r]);"),
+    ("rms_no_sqrt", "const double inv = 1.0 / sqrt(ss / (double)n + eps);",
+     "const double inv = 1.0 / (ss / (double)n + eps);"),
+    ("rms_sum_not_mean", "const double inv = 1.0 / sqrt(ss / (double)n + eps);",
+     "const double inv = 1.0 / sqrt(ss + eps);"),
+    ("rms_eps_outside", "const double inv = 1.0 / sqrt(ss / (double)n + eps);",
+     "const double inv = 1.0 / (sqrt(ss / (double)n) + eps);"),
+    ("rms_weight_dropped", "out[r * n + i] = x[r * n + i] * inv * w[i];", "out[r * n + i] = x[r * n + i] * inv;"),
+    ("rms_weight_reversed", "out[r * n + i] = x[r * n + i] * inv * w[i];",
+     "out[r * n + i] = x[r * n + i] * inv * w[n - 1 - i];"),
+    ("rms_abs_not_square", "ss += x[r * n + i] * x[r * n + i];", "ss += fabs(x[r * n + i]);"),
 ]
 
 
