@@ -56,6 +56,8 @@ def _declare(lib):
     lib.oracle_state_update.argtypes = [P] * 13 + [I] * 7
     lib.oracle_rmsnorm_rows.restype = ctypes.c_int
     lib.oracle_rmsnorm_rows.argtypes = [P, P, ctypes.c_double, P, I, I]
+    lib.oracle_matmul_nt.restype = ctypes.c_int
+    lib.oracle_matmul_nt.argtypes = [P, P, P, I, I, I, I, I]
     return lib
 
 
@@ -201,4 +203,70 @@ def state_update_normed(x, z, dt, conv_w, conv_b, dt_bias, Dskip, A, Bm, Cm, ssm
 
     return state_update(x, z, dt, conv_w, conv_b, dt_bias, Dskip, A, per_layer(Bm, b_norm_w),
                         per_layer(Cm, c_norm_w), ssm_state, conv_state, threads=threads, library=library)
+
+
+def matmul_nt(A, Bw, threads: int = 1, library=None):
+    """C = A @ Bw^T in float64 with Bw stored [N, K] (oracle_matmul_nt); A may
+    have leading batch dimensions, which are flattened into rows."""
+    L_ = library or lib()
+    A = _f64(A)
+    Bw = _f64(Bw)
+    K = A.shape[-1]
+    N = Bw.shape[0]
+    assert Bw.shape == (N, K)
+    M = int(np.prod(A.shape[:-1]))
+    A2 = A.reshape(M, K)
+    C = np.zeros((M, N))
+
+    def run(rng):
+        rc = L_.oracle_matmul_nt(_p(A2), _p(Bw), _p(C), M, N, K, rng[0], rng[1])
+        if rc != 0:
+            raise ValueError(f"oracle_matmul_nt rejected its arguments (rc={rc})")
+
+    parts = _ranges(M, threads)
+    if len(parts) == 1:
+        run(parts[0])
+    else:
+        with ThreadPoolExecutor(max_workers=len(parts)) as ex:
+            list(ex.map(run, parts))
+    return C.reshape(A.shape[:-1] + (N,))
+
+
+def projected_fwd(xz, conv_w, conv_b, W_x, W_dt, dt_bias, A, Dskip, h0=None, conv_state_in=None,
+                  dt_norm_w=None, b_norm_w=None, c_norm_w=None, norm_eps: float = 1e-6,
+                  threads: int = 1, library=None):
+    """The mixer with its producers, in the order the method runs them:
+        u      = SiLU(causal conv(x))                        [B, L, D]
+        x_dbl  = u @ W_x^T, W_x [R + 2N, D]                  [B, L, R + 2N]
+        dt_low, B, C = x_dbl[..., :R], [..., R:R+N], [..., R+N:]
+        (each optionally RMS-normalised over its own width)
+        dt     = dt_low @ W_dt^T, W_dt [D, R]                [B, L, D]
+        y, h_last, conv_state_out = the selective scan on (x, z, dt, B, C)
+    Returns the scan's outputs plus the intermediates u, dt_low, Bm, Cm, dt."""
+    L_ = library or lib()
+    xz_ = _f64(xz)
+    Bsz, Lq, twoD = xz_.shape
+    D = twoD // 2
+    N = _f64(A).shape[-1]
+    W_x = _f64(W_x)
+    R = W_x.shape[0] - 2 * N
+    # u: the scan's own conv + SiLU output, taken from its trace (B, C and dt do
+    # not enter u, so zeros stand in for them)
+    zeros_bc = np.zeros((Bsz, Lq, N))
+    tr = mixer_fwd(xz_, conv_w, conv_b, np.zeros((Bsz, Lq, D)), None, A, zeros_bc, zeros_bc, None, None,
+                   conv_state_in, threads=threads, traces=True, library=L_)
+    u = tr["u"]
+    x_dbl = matmul_nt(u, W_x, threads=threads, library=L_)
+    dt_low, Bm, Cm = x_dbl[..., :R], x_dbl[..., R:R + N], x_dbl[..., R + N:]
+    if dt_norm_w is not None:
+        dt_low = rmsnorm_rows(dt_low, dt_norm_w, norm_eps, L_)
+    if b_norm_w is not None:
+        Bm = rmsnorm_rows(Bm, b_norm_w, norm_eps, L_)
+    if c_norm_w is not None:
+        Cm = rmsnorm_rows(Cm, c_norm_w, norm_eps, L_)
+    dt = matmul_nt(dt_low, W_dt, threads=threads, library=L_)
+    out = mixer_fwd(xz_, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0, conv_state_in, threads=threads,
+                    library=L_)
+    out.update(u=u, dt_low=dt_low, Bm=Bm, Cm=Cm, dt=dt)
+    return out
 

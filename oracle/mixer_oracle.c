@@ -213,3 +213,31 @@ int oracle_rmsnorm_rows(const double* x, const double* w, double eps, double* ou
     return OR_OK;
 }
 
+/*
+ * Dense product with the second operand stored row-major as [N, K] (the
+ * layout of a projection's weight, one row per output feature):
+ *
+ *     C[m, n] = sum_k A[m, k] * Bw[n, k]
+ *
+ * The projections on either side of the selective scan are such products:
+ * x_proj maps the conv output u_t (d_inner) to the low-rank step input, B_t
+ * and C_t; dt_proj maps the low-rank step input back to d_inner (the Jamba
+ * reproduction blog's LoRA section names the low-rank Delta projection, and
+ * the JAMBA hybrid-model blog names x_proj and dt_proj).  Only rows m in
+ * [m_begin, m_end) are written.
+ */
+int oracle_matmul_nt(const double* A, const double* Bw, double* C, int64_t M, int64_t N, int64_t K,
+                     int64_t m_begin, int64_t m_end)
+{
+    if (M < 0 || N < 0 || K < 0 || !A || !Bw || !C) return OR_ERR_ARG;
+    if (m_begin < 0 || m_end > M || m_begin > m_end) return OR_ERR_ARG;
+    for (int64_t m = m_begin; m < m_end; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc += A[m * K + k] * Bw[n * K + k];
+            C[m * N + n] = acc;
+        }
+    }
+    return OR_OK;
+}
+

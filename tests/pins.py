@@ -398,7 +398,71 @@ def pin_normed_forward_uses_normalised_B_and_C(lib):
     np.testing.assert_array_equal(plain["y"], _fwd(lib, case)["y"])
 
 
+def pin_matmul_library(lib):
+    """The projection product against numpy's matmul on random operands
+    (library routine), including an empty K and a single row."""
+    rng = np.random.default_rng(51)
+    for M, N, K in ((7, 5, 33), (1, 288, 64), (4, 3, 0)):
+        A = rng.standard_normal((M, K))
+        Bw = rng.standard_normal((N, K))
+        np.testing.assert_allclose(oracle.matmul_nt(A, Bw, threads=2, library=lib), A @ Bw.T, rtol=1e-12,
+                                   atol=1e-12)
+
+
+def pin_matmul_selection(lib):
+    """Rows of Bw that are unit vectors select columns of A (closed form), and
+    a rank-one product a b^T times (c d^T)^T is (b . d) a c^T."""
+    rng = np.random.default_rng(52)
+    A = rng.standard_normal((6, 10))
+    sel = np.array([3, 0, 9, 3])
+    E = np.eye(10)[sel]
+    np.testing.assert_array_equal(oracle.matmul_nt(A, E, library=lib), A[:, sel])
+    a, b, c, d = (rng.standard_normal(n) for n in (6, 10, 4, 10))
+    got = oracle.matmul_nt(np.outer(a, b), np.outer(c, d), library=lib)
+    np.testing.assert_allclose(got, np.dot(b, d) * np.outer(a, c), rtol=1e-12, atol=1e-12)
+
+
+def pin_projected_forward_wiring(lib):
+    """The mixer with its projections: u from the conv + SiLU (checked against
+    scipy's logistic and numpy's convolve), then x_proj's output split as
+    [dt_low | B | C], optional norms, dt = dt_low W_dt^T, and the scan on those
+    -- recomputed here with numpy's matmul and the plain forward."""
+    rng = np.random.default_rng(53)
+    Bsz, Lq, D, N, R = 2, 9, 6, 16, 5
+    case = _rand_case(rng, Bsz, Lq, D, N)
+    W_x = rng.standard_normal((R + 2 * N, D)) * 0.4
+    W_dt = rng.standard_normal((D, R)) * 0.4
+    wd, wb, wc = rng.uniform(0.5, 1.5, R), rng.uniform(0.5, 1.5, N), rng.uniform(0.5, 1.5, N)
+    got = oracle.projected_fwd(case["xz"], case["conv_w"], case["conv_b"], W_x, W_dt, case["dt_bias"], case["A"],
+                               case["Dskip"], case["h0"], case["conv_state_in"], dt_norm_w=wd, b_norm_w=wb,
+                               c_norm_w=wc, norm_eps=0.1, library=lib)
+    # u by library routines: the causal conv over [window, x] and x * logistic(x)
+    x = case["xz"][..., :D]
+    u = np.zeros((Bsz, Lq, D))
+    for b in range(Bsz):
+        for d in range(D):
+            seq = np.concatenate([case["conv_state_in"][b, d], x[b, :, d]])
+            pre = np.convolve(seq, case["conv_w"][d, ::-1], mode="valid") + case["conv_b"][d]
+            u[b, :, d] = lib_silu(pre)
+    np.testing.assert_allclose(got["u"], u, rtol=1e-12, atol=1e-12)
+
+    def rms(v, w):
+        return v * w / np.sqrt(np.mean(v * v, axis=-1, keepdims=True) + 0.1)
+
+    x_dbl = u @ W_x.T
+    dt_low, Bm, Cm = rms(x_dbl[..., :R], wd), rms(x_dbl[..., R:R + N], wb), rms(x_dbl[..., R + N:], wc)
+    dt = dt_low @ W_dt.T
+    for k, v in (("dt_low", dt_low), ("Bm", Bm), ("Cm", Cm), ("dt", dt)):
+        np.testing.assert_allclose(got[k], v, rtol=1e-11, atol=1e-12)
+    want = _fwd(lib, dict(case, dt=dt, Bm=Bm, Cm=Cm))
+    for k in ("y", "h_last", "conv_state_out"):
+        np.testing.assert_allclose(got[k], want[k], rtol=1e-10, atol=1e-12)
+
+
 ALL_PINS = [
+    pin_matmul_library,
+    pin_matmul_selection,
+    pin_projected_forward_wiring,
     pin_rmsnorm_constant_rows,
     pin_rmsnorm_library,
     pin_rmsnorm_homogeneity,

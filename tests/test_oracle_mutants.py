@@ -1,7 +1,7 @@
 """Plants plausible mistakes in copies of the oracle (on the CPU) and checks
 that each one makes at least one pin fail, so the pins really constrain every
 step of the oracle: conv, SiLU, softplus, discretisation, recurrence, readout,
-skip, gate, carried state, the decode step and the RMSNorm of B and C."""
+skip, gate, carried state, the decode step, the RMSNorm of B and C and the projection product."""
 
 import os
 
@@ -56,6 +56,11 @@ MUTANTS = [
     ("rms_weight_reversed", "out[r * n + i] = x[r * n + i] * inv * w[i];",
      "out[r * n + i] = x[r * n + i] * inv * w[n - 1 - i];"),
     ("rms_abs_not_square", "ss += x[r * n + i] * x[r * n + i];", "ss += fabs(x[r * n + i]);"),
+    ("matmul_weight_transposed", "acc += A[m * K + k] * Bw[n * K + k];", "acc += A[m * K + k] * Bw[k * N + n];"),
+    ("matmul_last_term_dropped", "for (int64_t k = 0; k < K; ++k) acc += A[m * K + k] * Bw[n * K + k];",
+     "for (int64_t k = 0; k + 1 < K; ++k) acc += A[m * K + k] * Bw[n * K + k];"),
+    ("matmul_no_accumulate", "acc += A[m * K + k] * Bw[n * K + k];", "acc = A[m * K + k] * Bw[n * K + k];"),
+    ("matmul_row_of_A", "acc += A[m * K + k] * Bw[n * K + k];", "acc += A[n * K + k] * Bw[n * K + k];"),
 ]
 
 
