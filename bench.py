@@ -44,6 +44,7 @@ SMS = 148
 FP32_LANES_PER_SM = 128
 SM_MAX_MHZ_FALLBACK = 1965.0
 HBM_FALLBACK_GBS = 6650.0
+BF16_FALLBACK_TFLOPS = 1590.0
 
 # Algorithmic fp32-pipe work of the forward per (token, channel): for each of
 # the 16 states a decay factor, the Delta*u*B product, the state FMA and the
@@ -305,6 +306,13 @@ def run_gpu(args):
     # ---- the same forward with per-state A rows (as trained weights have)
     gen = run_general_a(mm, args, world, alu_peak)
 
+    # ---- the same forward with the RMSNorm of B and C fused in
+    normed = run_normed(mm, args, world, hbm_peak, hbm_src, statistics.mean(launch_ms))
+
+    # ---- the projections either side of the scan on the tensor cores, and the
+    # mixer with its producers (conv -> x_proj -> norms -> dt_proj -> scan)
+    proj = run_projections(mm, args, world, hbm_peak, hbm_src, peaks)
+
     result = None
     if rank == 0:
         cpu = cpu_baseline(host, cfg) if world == 1 and not args.no_cpu_baseline else None
@@ -339,6 +347,8 @@ def run_gpu(args):
             "clocks": clk.summary(),
             "decode": dec,
             "general_a": gen,
+            "bc_rmsnorm": normed,
+            "projections": proj,
             **legs,
             "launch_ms": {"mean": round(statistics.mean(launch_ms), 5), "min": round(min(launch_ms), 5),
                           "max": round(max(launch_ms), 5)},
@@ -528,6 +538,134 @@ def run_general_a(mm, args, world, alu_peak):
     }
 
 
+def run_normed(mm, args, world, hbm_peak, hbm_src, plain_ms):
+    """The Jamba-shaped forward through mamba_mixer_fwd_normed (RMSNorm of
+    B_t and C_t over d_state, fused into the tile staging), with the same
+    timing rules as the main loop.  Its extra HBM traffic is the two 64-byte
+    weight rows."""
+    from workloads import make_norm_weights
+
+    cfg = PREFILL
+    B, L, D = cfg.batch, cfg.seqlen, cfg.d_inner
+    host = make_mixer_inputs(cfg)
+    wb, wc = (w.cuda() for w in make_norm_weights(seed=cfg.seed))
+    nsets = 2
+    sets = [{k: (v.cuda() if v is not None else None) for k, v in host.items()} for _ in range(nsets)]
+    outs = [(torch.empty((B, L, D), dtype=torch.bfloat16, device="cuda"),
+             torch.empty((B, D, 16), device="cuda"),
+             torch.empty((B, D, 3), dtype=torch.bfloat16, device="cuda")) for _ in range(nsets)]
+    ws = torch.empty(mm.workspace_size(B, L, D), dtype=torch.uint8, device="cuda")
+
+    def call(i):
+        d, o = sets[i % nsets], outs[i % nsets]
+        mm.mixer_fwd(d["xz"], d["conv_w"], d["conv_b"], d["dt"], d["dt_bias"], d["A"], d["Bm"], d["Cm"],
+                     d["Dskip"], d["h0"], d["conv_state_in"], y=o[0], h_last=o[1], conv_state_out=o[2],
+                     workspace=ws, b_norm_w=wb, c_norm_w=wc, norm_eps=1e-6)
+
+    for i in range(max(3, args.warmup // 10)):
+        call(i)
+    torch.cuda.synchronize()
+    K = max(3, min(args.steps, 400))
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize()
+    a.record()
+    for i in range(K):
+        call(i)
+    b.record()
+    torch.cuda.synchronize()
+    ms = _max_over_ranks(a.elapsed_time(b) / K, world)
+    nbytes = prefill_bytes(B, L, D) + 2 * 16 * 4
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {
+        "workload": cfg.name, "norm": "RMSNorm of B_t and C_t over d_state, eps 1e-6", "steps": K,
+        "ms_per_step": round(ms, 5), "value": round(_job_rate(world, B * L, ms), 1), "unit": "tokens/s",
+        "vs_plain_forward": round(ms / plain_ms, 4),
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(gbs / hbm_peak, 4), "traffic": None, "algorithmic_bytes": nbytes,
+                     "peak_source": hbm_src},
+    }
+
+
+def _time_loop(fn, K, world):
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(K):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return _max_over_ranks(a.elapsed_time(b) / K, world)
+
+
+def run_projections(mm, args, world, hbm_peak, hbm_src, peaks):
+    """x_proj (tokens x 8192 -> 288) and dt_proj (tokens x 256 -> 8192) as
+    tensor-core products at the Jamba size, and the whole mixer with its
+    producers (dt_rank 256, the three RMSNorms on).  The products' roofline is
+    the measured dense bf16 rate (burst figure: each is timed alone)."""
+    from workloads import make_norm_weights, make_projection_weights
+
+    cfg = PREFILL
+    B, L, D, R = cfg.batch, cfg.seqlen, cfg.d_inner, 256
+    M = B * L
+    if peaks and "bf16_tflops" in peaks:
+        tpeak, tsrc = float(peaks["bf16_tflops"]), "measured"
+    else:
+        tpeak, tsrc = BF16_FALLBACK_TFLOPS, "fallback"
+    K = max(3, min(args.steps, 200))
+    g = torch.Generator(device="cuda").manual_seed(7)
+    u = torch.randn((M, D), device="cuda", generator=g).to(torch.bfloat16)
+    W_x, W_dt, wd = (t.cuda() for t in make_projection_weights(D, R, seed=cfg.seed))
+    dtl = torch.randn((M, R), device="cuda", generator=g).to(torch.bfloat16)
+    xdbl = torch.empty((M, R + 32), device="cuda")
+    dt = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+
+    def leg(name, fn, flops, nbytes, ms):
+        return {"ms_per_call": round(ms, 5), "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
+                "roofline": {"bound": "tensor", "achieved": round(flops / (ms * 1e-3) / 1e12, 1), "peak": tpeak,
+                             "unit": "TFLOP/s", "frac": round(flops / (ms * 1e-3) / 1e12 / tpeak, 4),
+                             "traffic": None, "peak_source": tsrc},
+                "hbm_gbs": round(nbytes / (ms * 1e-3) / 1e9, 1), "shape": name}
+
+    ms_x = _time_loop(lambda: mm.proj_matmul(u, W_x, out=xdbl, workspace=ws), K, world)
+    ms_d = _time_loop(lambda: mm.proj_matmul(dtl, W_dt, out=dt, workspace=ws), K, world)
+    out = {
+        "x_proj": leg(f"{M} x {R + 32} x {D}, bf16 -> fp32", None, 2.0 * M * (R + 32) * D,
+                      M * D * 2 + (R + 32) * D * 2 + M * (R + 32) * 4, ms_x),
+        "dt_proj": leg(f"{M} x {D} x {R}, bf16 -> bf16", None, 2.0 * M * D * R, M * R * 2 + D * R * 2 + M * D * 2,
+                       ms_d),
+    }
+    del u, dtl, xdbl, dt
+    host = make_mixer_inputs(cfg)
+    d = {k: (v.cuda() if v is not None else None) for k, v in host.items()}
+    wb, wc = (w.cuda() for w in make_norm_weights(seed=cfg.seed))
+    y = torch.empty((B, L, D), dtype=torch.bfloat16, device="cuda")
+    h = torch.empty((B, D, 16), device="cuda")
+    cs = torch.empty((B, D, 3), dtype=torch.bfloat16, device="cuda")
+    pws = torch.empty(mm.projected_workspace_size(B, L, D, R), dtype=torch.uint8, device="cuda")
+
+    def chain():
+        mm.mixer_fwd_projected(d["xz"], d["conv_w"], d["conv_b"], W_x, W_dt, d["dt_bias"], d["A"], d["Dskip"],
+                               d["h0"], d["conv_state_in"], dt_norm_w=wd, b_norm_w=wb, c_norm_w=wc,
+                               y=y, h_last=h, conv_state_out=cs, workspace=pws)
+
+    ms_c = _time_loop(chain, K, world)
+    out["projected_forward"] = {
+        "workload": cfg.name, "dt_rank": R, "norms": "dt_low, B, C", "ms_per_step": round(ms_c, 5),
+        "value": round(_job_rate(world, M, ms_c), 1), "unit": "tokens/s",
+        "kernels": "conv+SiLU, x_proj (tcgen05, split-K), x_proj epilogue (sum, split, RMSNorm), "
+                   "dt_proj (tcgen05), scan (summary + full pass)",
+    }
+    del d, y, h, cs, pws
+    torch.cuda.empty_cache()
+    return out
+
+
 # ---------------------------------------------------------------- CPU oracle
 def cpu_baseline(host, cfg, target_s=12.0, sample_override=None, threads=None):
     """The fp64 oracle as it stands, on all host cores (or `threads` of
@@ -638,7 +776,23 @@ def run_only(args):
 
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
     mm.lib()
-    if args.only == "forward":
+    if args.only in ("xproj", "dtproj"):
+        from workloads import make_projection_weights
+
+        cfg = PREFILL
+        M, D, R = cfg.batch * cfg.seqlen, cfg.d_inner, 256
+        W_x, W_dt, _ = (t.cuda() for t in make_projection_weights(D, R, seed=cfg.seed))
+        g = torch.Generator(device="cuda").manual_seed(7)
+        ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+        if args.only == "xproj":
+            a = torch.randn((M, D), device="cuda", generator=g).to(torch.bfloat16)
+            o = torch.empty((M, R + 32), device="cuda")
+            step = lambda: mm.proj_matmul(a, W_x, out=o, workspace=ws)  # noqa: E731
+        else:
+            a = torch.randn((M, R), device="cuda", generator=g).to(torch.bfloat16)
+            o = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
+            step = lambda: mm.proj_matmul(a, W_dt, out=o, workspace=ws)  # noqa: E731
+    elif args.only == "forward":
         cfg = PREFILL
         d = {k: (v.cuda() if v is not None else None)
              for k, v in make_mixer_inputs(cfg, A_mode=args.a_mode).items()}
@@ -677,7 +831,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra-prefill", action="store_true",
                     help="skip the 4 x 32768 and 262,144-token prefill legs")
-    ap.add_argument("--only", choices=["forward", "decode"], default=None,
+    ap.add_argument("--only", choices=["forward", "decode", "xproj", "dtproj"], default=None,
                     help="run one kernel's timed loop only (for profiler captures); prints no JSON line")
     ap.add_argument("--decode-layers", type=int, default=None,
                     help="with --only decode: stacked layers (default: the workload's 28)")

@@ -6,9 +6,16 @@
  *   mamba_mixer_fwd      selective-scan forward over a whole sequence (prefill)
  *   mamba_state_update   the one-token state update used in decode
  *
+ * the same two with the RMSNorm of B_t and C_t fused in:
+ *   mamba_mixer_fwd_normed, mamba_state_update_normed
+ *
  * two more ways into the forward beyond the plain call:
  *   mamba_mixer_fwd_noalloc  no workspace argument (a fixed scratch array inside the library)
  *   mamba_mixer_fwd_host     activations in host memory, copies overlapped with the compute
+ * the producers either side of the scan, on the tensor cores (tcgen05):
+ *   mamba_proj_matmul           out = A W^T, a projection (bf16 operands, fp32 accumulation)
+ *   mamba_mixer_fwd_projected   conv -> x_proj -> [dt_low | B | C] (+RMSNorm) -> dt_proj -> scan
+ *
  * and two status readers:
  *   mamba_check_status       did the last forward on this workspace complete? (per call)
  *   mamba_mixer_fault_status has any kernel on this device given up a bounded wait? (sticky)
@@ -73,8 +80,9 @@ typedef enum mm_status {
     MM_ERR_DEVICE = 8,      /* no usable sm_100 device is current                    */
     MM_ERR_WORKSPACE = 9,   /* workspace missing or smaller than the size this call needs */
     MM_ERR_SCRATCH_LIMIT = 10, /* mamba_mixer_fwd_noalloc: sizes need more than its built-in scratch */
-    MM_ERR_TIMEOUT = 11     /* mamba_check_status / mamba_mixer_fault_status: a kernel gave up a
+    MM_ERR_TIMEOUT = 11,    /* mamba_check_status / mamba_mixer_fault_status: a kernel gave up a
                                bounded wait (its bulk copies, or a chunk summary never written) */
+    MM_ERR_ARG = 12         /* an argument value out of range (norm_eps not positive and finite) */
 } mm_status;
 
 typedef enum mm_dtype {
@@ -134,6 +142,33 @@ mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv
                           int64_t batch, int64_t seqlen, int64_t d_inner,
                           int64_t d_state, int64_t d_conv, mm_dtype act,
                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * mamba_mixer_fwd with an RMSNorm of the selective parameters fused in.
+ * The Jamba deep-dive report lists RMSNorm inside the Mamba layer among its
+ * standard components, and its large-scale-stability section applies it to
+ * the layer's internal activations; the pages do not say which.  This library
+ * takes B_t and C_t, the activations that enter the recurrence, and
+ * normalises each over its d_state entries before it is used:
+ *
+ *   B_t[n] <- B_t[n] * b_norm_w[n] / sqrt(mean_n B_t[n]^2 + norm_eps)
+ *   C_t[n] <- C_t[n] * c_norm_w[n] / sqrt(mean_n C_t[n]^2 + norm_eps)
+ *
+ * b_norm_w, c_norm_w: [d_state] fp32 device weights, 16-byte aligned; NULL =
+ * that input is used as it is (both NULL = mamba_mixer_fwd).  norm_eps must
+ * be positive and finite when a weight is given (MM_ERR_ARG otherwise).  The
+ * norm is computed in fp32 as each tile of B/C is staged; the inputs are not
+ * modified.  Everything else is as mamba_mixer_fwd, including the workspace.
+ */
+mm_status mamba_mixer_fwd_normed(const void* xz, const float* conv_w, const float* conv_b,
+                                 const void* dt, const float* dt_bias, const float* A,
+                                 const void* Bm, const void* Cm, const float* Dskip,
+                                 const float* h0, const void* conv_state_in,
+                                 void* y, float* h_last, void* conv_state_out,
+                                 int64_t batch, int64_t seqlen, int64_t d_inner,
+                                 int64_t d_state, int64_t d_conv, mm_dtype act,
+                                 const float* b_norm_w, const float* c_norm_w, float norm_eps,
+                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * mamba_mixer_fwd without a workspace argument, for callers that cannot
@@ -263,6 +298,22 @@ mm_status mamba_state_update(const void* x, const void* z, const void* dt,
                              int64_t d_state, int64_t d_conv, mm_dtype act, void* stream);
 
 /*
+ * mamba_state_update with each (layer, batch) row's B and C normalised as in
+ * mamba_mixer_fwd_normed, so decode continues a normed prefill exactly.
+ * b_norm_w, c_norm_w: [n_layers, d_state] fp32 (one weight row per layer), or
+ * NULL; norm_eps positive and finite when a weight is given (MM_ERR_ARG).
+ */
+mm_status mamba_state_update_normed(const void* x, const void* z, const void* dt,
+                                    const float* conv_w, const float* conv_b,
+                                    const float* dt_bias, const float* Dskip, const float* A,
+                                    const void* Bm, const void* Cm,
+                                    float* ssm_state, void* conv_state, void* y,
+                                    int64_t n_layers, int64_t batch, int64_t d_inner,
+                                    int64_t d_state, int64_t d_conv, mm_dtype act,
+                                    const float* b_norm_w, const float* c_norm_w, float norm_eps,
+                                    void* stream);
+
+/*
  * Status of the last forward call that ran on `workspace` (the workspace of
  * mamba_mixer_fwd or mamba_mixer_fwd_host; NULL = the fixed scratch of
  * mamba_mixer_fwd_noalloc in the current context).  Waits for `stream` to
@@ -294,13 +345,73 @@ mm_status mamba_check_status(const void* workspace, void* stream);
  */
 mm_status mamba_mixer_fault_status(int reset);
 
+/*
+ * Projection product on the tensor cores: out[m, n] = sum_k A[m, k] W[n, k],
+ * bf16 operands, fp32 accumulation (tcgen05.mma, operands staged by TMA,
+ * accumulator in tensor memory).  The projections either side of the scan
+ * are such products: the JAMBA hybrid-model blog names x_proj and dt_proj,
+ * and the Jamba reproduction blog's LoRA section the low-rank Delta
+ * projection.
+ *   A    [M, K] bf16, row-major          W   [N, K] bf16 (one row per output feature)
+ *   out  [M, N] fp32 (out_dtype MM_F32) or bf16 (MM_BF16, rounded to nearest even)
+ * K and N must be multiples of 8 (16-byte rows; MM_ERR_UNSUPPORTED), M, N, K
+ * below 2^31.  workspace: at least mamba_proj_matmul_workspace_size(M, N, K)
+ * bytes (the call's status, read by mamba_check_status).  M == 0 is a no-op.
+ * out may not overlap A, W or the workspace (MM_ERR_ALIAS).
+ */
+mm_status mamba_proj_matmul(const void* A, const void* W, void* out, int64_t M, int64_t N, int64_t K,
+                            mm_dtype out_dtype, void* workspace, size_t workspace_bytes, void* stream);
+size_t mamba_proj_matmul_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/*
+ * The mixer with its producers, in the order the method runs them (bf16
+ * activations only: the products run on the tensor cores):
+ *
+ *   u      = SiLU(conv_b + causal depthwise conv(x))                [B, L, D]
+ *   x_dbl  = u W_x^T                        W_x [R + 2 N, D] bf16   [B, L, R + 2N]
+ *   dt_low, B_t, C_t = x_dbl[:R], x_dbl[R:R+N], x_dbl[R+N:]
+ *            each RMS-normalised over its own width when its weight is given
+ *            (dt_norm_w [R], b_norm_w / c_norm_w [N] fp32; NULL = not normalised)
+ *   dt     = dt_low W_dt^T                  W_dt [D, R] bf16        [B, L, D]
+ *   y, h_last, conv_state_out = the selective scan of mamba_mixer_fwd on
+ *            (x, z, dt, B, C) with conv_w, conv_b, dt_bias, A, Dskip, h0,
+ *            conv_state_in as there.
+ *
+ * R = dt_rank, a multiple of 32 up to 1024; d_state == 16; d_conv == 4;
+ * d_inner a multiple of 64.  The pages name the projections (JAMBA hybrid-model
+ * blog: x_proj, dt_proj; reproduction blog: the low-rank Delta projection)
+ * but give no rank; the standard choice, ceil(hidden / 16) = 256 at hidden
+ * 4096, is what the tests and the benchmark use.  workspace: at least
+ * mamba_mixer_projected_workspace_size(...) bytes; it holds the scan's own
+ * workspace (with the call's status, first) and the intermediates u, x_proj's
+ * split-K partials, dt_low, B, C and dt.  The weights and every caller buffer
+ * may not overlap it (MM_ERR_ALIAS).  Errors otherwise as mamba_mixer_fwd.
+ */
+mm_status mamba_mixer_fwd_projected(const void* xz, const float* conv_w, const float* conv_b,
+                                    const void* W_x, const void* W_dt, const float* dt_bias, const float* A,
+                                    const float* Dskip, const float* h0, const void* conv_state_in,
+                                    const float* dt_norm_w, const float* b_norm_w, const float* c_norm_w,
+                                    float norm_eps, void* y, float* h_last, void* conv_state_out,
+                                    int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state,
+                                    int64_t dt_rank, int64_t d_conv, mm_dtype act,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+size_t mamba_mixer_projected_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state,
+                                            int64_t dt_rank, int64_t d_conv, mm_dtype act);
+/* Byte offsets, within that workspace, of the intermediates a call leaves
+ * there (valid once its stream has reached the end of the call): offsets[0]
+ * u [B, L, D], [1] dt_low [B, L, R], [2] B_t [B, L, N], [3] C_t [B, L, N],
+ * [4] dt [B, L, D], all bf16 row-major.  For inspection and tests; the
+ * forward itself does not need them afterwards. */
+mm_status mamba_mixer_projected_layout(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state,
+                                       int64_t dt_rank, int64_t d_conv, size_t offsets[5]);
+
 /* A static, human-readable name for a status code. */
 const char* mamba_status_string(mm_status status);
 
 /* ABI version of this header (incremented on any signature change). */
 int mamba_mixer_abi_version(void);
 
-#define MAMBA_MIXER_ABI_VERSION 2
+#define MAMBA_MIXER_ABI_VERSION 4
 
 #ifdef __cplusplus
 }

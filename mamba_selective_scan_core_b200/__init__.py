@@ -16,7 +16,8 @@ import os
 __all__ = [
     "MM_F32", "MM_BF16", "MixerError", "lib", "library_path", "mixer_fwd", "mixer_fwd_noalloc", "mixer_fwd_host",
     "state_update", "workspace_size", "host_workspace_size", "status_string", "abi_version", "fault_status",
-    "check_status", "EXPORTED_SYMBOLS",
+    "check_status", "proj_matmul", "proj_matmul_workspace_size", "mixer_fwd_projected",
+    "projected_workspace_size", "EXPORTED_SYMBOLS",
 ]
 
 MM_F32 = 0
@@ -37,6 +38,13 @@ EXPORTED_SYMBOLS = (
     "mamba_mixer_abi_version",
     "mamba_mixer_fault_status",
     "mamba_check_status",
+    "mamba_mixer_fwd_normed",
+    "mamba_state_update_normed",
+    "mamba_proj_matmul",
+    "mamba_proj_matmul_workspace_size",
+    "mamba_mixer_fwd_projected",
+    "mamba_mixer_projected_workspace_size",
+    "mamba_mixer_projected_layout",
 )
 
 
@@ -75,6 +83,22 @@ def _declare(L):
     L.mamba_mixer_fault_status.argtypes = [ctypes.c_int]
     L.mamba_check_status.restype = ctypes.c_int
     L.mamba_check_status.argtypes = [P, P]
+    L.mamba_mixer_fwd_normed.restype = ctypes.c_int
+    L.mamba_mixer_fwd_normed.argtypes = [P] * 14 + [I64] * 5 + [ctypes.c_int, P, P, ctypes.c_float, P,
+                                                                 ctypes.c_size_t, P]
+    L.mamba_state_update_normed.restype = ctypes.c_int
+    L.mamba_state_update_normed.argtypes = [P] * 13 + [I64] * 5 + [ctypes.c_int, P, P, ctypes.c_float, P]
+    L.mamba_proj_matmul.restype = ctypes.c_int
+    L.mamba_proj_matmul.argtypes = [P, P, P, I64, I64, I64, ctypes.c_int, P, ctypes.c_size_t, P]
+    L.mamba_proj_matmul_workspace_size.restype = ctypes.c_size_t
+    L.mamba_proj_matmul_workspace_size.argtypes = [I64, I64, I64]
+    L.mamba_mixer_fwd_projected.restype = ctypes.c_int
+    L.mamba_mixer_fwd_projected.argtypes = [P] * 13 + [ctypes.c_float] + [P] * 3 + [I64] * 6 + [
+        ctypes.c_int, P, ctypes.c_size_t, P]
+    L.mamba_mixer_projected_workspace_size.restype = ctypes.c_size_t
+    L.mamba_mixer_projected_workspace_size.argtypes = [I64] * 6 + [ctypes.c_int]
+    L.mamba_mixer_projected_layout.restype = ctypes.c_int
+    L.mamba_mixer_projected_layout.argtypes = [I64] * 6 + [P]
     return L
 
 
@@ -170,12 +194,15 @@ def workspace_size(batch, seqlen, d_inner, d_state=16, d_conv=4, act=MM_BF16) ->
 
 
 def mixer_fwd(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, conv_state_in=None, *,
-              y=None, h_last=None, conv_state_out=None, workspace=None, stream=None):
+              y=None, h_last=None, conv_state_out=None, workspace=None, stream=None,
+              b_norm_w=None, c_norm_w=None, norm_eps=1e-6):
     """Selective-scan forward.  Shapes: xz [B,L,2D], dt [B,L,D], Bm/Cm [B,L,N]
     (act dtype: bf16 or fp32); conv_w [D,W], conv_b/dt_bias/Dskip [D], A [D,N],
     h0 [B,D,N] (fp32); conv_state_in [B,D,W-1] (act).  conv_b, Dskip, h0 and
-    conv_state_in may be None.  Returns (y [B,L,D], h_last [B,D,N],
-    conv_state_out [B,D,W-1]), allocating any output not given."""
+    conv_state_in may be None.  b_norm_w / c_norm_w ([N] fp32) switch on the
+    fused RMSNorm of B / C (mamba_mixer_fwd_normed).  Returns (y [B,L,D],
+    h_last [B,D,N], conv_state_out [B,D,W-1]), allocating any output not
+    given."""
     import torch
 
     act = _act_code(xz.dtype)
@@ -197,6 +224,9 @@ def mixer_fwd(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, conv_s
     _check(Dskip, "Dskip", f32, (D,), dev)
     _check(h0, "h0", f32, (Bsz, D, N), dev)
     _check(conv_state_in, "conv_state_in", xz.dtype, (Bsz, D, W - 1), dev)
+    _check(b_norm_w, "b_norm_w", f32, (N,), dev)
+    _check(c_norm_w, "c_norm_w", f32, (N,), dev)
+    normed = b_norm_w is not None or c_norm_w is not None
     if y is None:
         y = torch.empty((Bsz, L, D), dtype=xz.dtype, device=dev)
         made.append(y)
@@ -213,14 +243,17 @@ def mixer_fwd(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, conv_s
     if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
         made.append(workspace)
-    with torch.cuda.device(dev):
-        st = lib().mamba_mixer_fwd(
-            _ptr(xz), _ptr(conv_w), _ptr(conv_b), _ptr(dt), _ptr(dt_bias), _ptr(A), _ptr(Bm), _ptr(Cm),
+    args = (_ptr(xz), _ptr(conv_w), _ptr(conv_b), _ptr(dt), _ptr(dt_bias), _ptr(A), _ptr(Bm), _ptr(Cm),
             _ptr(Dskip), _ptr(h0), _ptr(conv_state_in), _ptr(y), _ptr(h_last), _ptr(conv_state_out),
-            Bsz, L, D, N, W, act, _ptr(workspace), workspace.numel() * workspace.element_size(),
-            _stream_handle(stream))
+            Bsz, L, D, N, W, act)
+    tail = (_ptr(workspace), workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    with torch.cuda.device(dev):
+        if normed:
+            st = lib().mamba_mixer_fwd_normed(*args, _ptr(b_norm_w), _ptr(c_norm_w), float(norm_eps), *tail)
+        else:
+            st = lib().mamba_mixer_fwd(*args, *tail)
     if st != 0:
-        raise MixerError(st, "mamba_mixer_fwd")
+        raise MixerError(st, "mamba_mixer_fwd_normed" if normed else "mamba_mixer_fwd")
     _keep_alive_on(made, (stream,))
     return y, h_last, conv_state_out
 
@@ -345,11 +378,13 @@ def mixer_fwd_noalloc(xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0=None
 
 
 def state_update(x, z, dt, conv_w, conv_b, dt_bias, Dskip, A, Bm, Cm, ssm_state, conv_state, *,
-                 y=None, stream=None):
+                 y=None, stream=None, b_norm_w=None, c_norm_w=None, norm_eps=1e-6):
     """One-token decode step for NL stacked layers, in place on ssm_state
     [NL,B,D,N] (fp32) and conv_state [NL,B,D,W-1] (act).  x/z/dt [NL,B,D] and
     Bm/Cm [NL,B,N] in the act dtype; conv_w [NL,D,W], conv_b/dt_bias/Dskip
-    [NL,D], A [NL,D,N] in fp32 (conv_b, Dskip may be None).  Returns y [NL,B,D]."""
+    [NL,D], A [NL,D,N] in fp32 (conv_b, Dskip may be None).  b_norm_w /
+    c_norm_w ([NL,N] fp32) switch on the fused RMSNorm of B / C
+    (mamba_state_update_normed).  Returns y [NL,B,D]."""
     import torch
 
     act = _act_code(x.dtype)
@@ -368,17 +403,137 @@ def state_update(x, z, dt, conv_w, conv_b, dt_bias, Dskip, A, Bm, Cm, ssm_state,
     _check(Cm, "Cm", x.dtype, (NL, Bsz, N), dev)
     _check(ssm_state, "ssm_state", f32, (NL, Bsz, D, N), dev)
     _check(conv_state, "conv_state", x.dtype, (NL, Bsz, D, W - 1), dev)
+    _check(b_norm_w, "b_norm_w", f32, (NL, N), dev)
+    _check(c_norm_w, "c_norm_w", f32, (NL, N), dev)
+    normed = b_norm_w is not None or c_norm_w is not None
     made = []
     if y is None:
         y = torch.empty((NL, Bsz, D), dtype=x.dtype, device=dev)
         made.append(y)
     _check(y, "y", x.dtype, (NL, Bsz, D), dev)
+    args = (_ptr(x), _ptr(z), _ptr(dt), _ptr(conv_w), _ptr(conv_b), _ptr(dt_bias), _ptr(Dskip), _ptr(A),
+            _ptr(Bm), _ptr(Cm), _ptr(ssm_state), _ptr(conv_state), _ptr(y), NL, Bsz, D, N, W, act)
     with torch.cuda.device(dev):
-        st = lib().mamba_state_update(
-            _ptr(x), _ptr(z), _ptr(dt), _ptr(conv_w), _ptr(conv_b), _ptr(dt_bias), _ptr(Dskip), _ptr(A),
-            _ptr(Bm), _ptr(Cm), _ptr(ssm_state), _ptr(conv_state), _ptr(y), NL, Bsz, D, N, W, act,
-            _stream_handle(stream))
+        if normed:
+            st = lib().mamba_state_update_normed(*args, _ptr(b_norm_w), _ptr(c_norm_w), float(norm_eps),
+                                                 _stream_handle(stream))
+        else:
+            st = lib().mamba_state_update(*args, _stream_handle(stream))
     if st != 0:
-        raise MixerError(st, "mamba_state_update")
+        raise MixerError(st, "mamba_state_update_normed" if normed else "mamba_state_update")
     _keep_alive_on(made, (stream,))
     return y
+
+
+def proj_matmul_workspace_size(M, N, K) -> int:
+    return int(lib().mamba_proj_matmul_workspace_size(M, N, K))
+
+
+def proj_matmul(A, W, *, out=None, out_dtype=None, workspace=None, stream=None):
+    """out = A @ W^T on the tensor cores (mamba_proj_matmul): A [M, K] and W
+    [N, K] bf16 CUDA tensors, out [M, N] fp32 (default) or bf16."""
+    import torch
+
+    M, K = A.shape
+    N = W.shape[0]
+    dev = A.device
+    _check(A, "A", torch.bfloat16, (M, K), dev)
+    _check(W, "W", torch.bfloat16, (N, K), dev)
+    dtype = out_dtype or (out.dtype if out is not None else torch.float32)
+    if out is None:
+        out = torch.empty((M, N), dtype=dtype, device=dev)
+    _check(out, "out", dtype, (M, N), dev)
+    code = MM_BF16 if dtype == torch.bfloat16 else MM_F32
+    ws_bytes = proj_matmul_workspace_size(M, N, K)
+    made = []
+    if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+        made.append(workspace)
+    with torch.cuda.device(dev):
+        st = lib().mamba_proj_matmul(_ptr(A), _ptr(W), _ptr(out), M, N, K, code, _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    if st != 0:
+        raise MixerError(st, "mamba_proj_matmul")
+    _keep_alive_on(made, (stream,))
+    return out
+
+
+def projected_workspace_size(batch, seqlen, d_inner, dt_rank, d_state=16, d_conv=4, act=MM_BF16) -> int:
+    return int(lib().mamba_mixer_projected_workspace_size(batch, seqlen, d_inner, d_state, dt_rank, d_conv, act))
+
+
+def projected_intermediates(workspace, batch, seqlen, d_inner, dt_rank, d_state=16, d_conv=4):
+    """Views of the intermediates a mixer_fwd_projected call left in its
+    workspace (u, dt_low, Bm, Cm, dt; bf16), by mamba_mixer_projected_layout."""
+    import torch
+
+    offs = (ctypes.c_size_t * 5)()
+    st = lib().mamba_mixer_projected_layout(batch, seqlen, d_inner, d_state, dt_rank, d_conv, offs)
+    if st != 0:
+        raise MixerError(st, "mamba_mixer_projected_layout")
+    shapes = ((batch, seqlen, d_inner), (batch, seqlen, dt_rank), (batch, seqlen, d_state), (batch, seqlen, d_state),
+              (batch, seqlen, d_inner))
+    out = []
+    for off, shp in zip(offs, shapes):
+        n = 1
+        for v in shp:
+            n *= v
+        out.append(workspace[off:off + 2 * n].view(torch.bfloat16).view(shp))
+    return dict(zip(("u", "dt_low", "Bm", "Cm", "dt"), out))
+
+
+def mixer_fwd_projected(xz, conv_w, conv_b, W_x, W_dt, dt_bias, A, Dskip, h0=None, conv_state_in=None, *,
+                        dt_norm_w=None, b_norm_w=None, c_norm_w=None, norm_eps=1e-6, y=None, h_last=None,
+                        conv_state_out=None, workspace=None, stream=None):
+    """The mixer with its producers (mamba_mixer_fwd_projected): u = SiLU(conv
+    x), x_proj (W_x [R + 2N, D] bf16) split into dt_low | B | C with optional
+    RMSNorms (dt_norm_w [R], b_norm_w / c_norm_w [N] fp32), dt_proj (W_dt
+    [D, R] bf16), then the selective scan.  bf16 activations only.  Returns
+    (y, h_last, conv_state_out)."""
+    import torch
+
+    Bsz, L, twoD = xz.shape
+    D = twoD // 2
+    N = A.shape[-1]
+    W = conv_w.shape[-1]
+    R = W_dt.shape[-1]
+    dev = xz.device
+    f32, bf = torch.float32, torch.bfloat16
+    _check(xz, "xz", bf, (Bsz, L, 2 * D), dev)
+    _check(conv_w, "conv_w", f32, (D, W), dev)
+    _check(conv_b, "conv_b", f32, (D,), dev)
+    _check(W_x, "W_x", bf, (R + 2 * N, D), dev)
+    _check(W_dt, "W_dt", bf, (D, R), dev)
+    _check(dt_bias, "dt_bias", f32, (D,), dev)
+    _check(A, "A", f32, (D, N), dev)
+    _check(Dskip, "Dskip", f32, (D,), dev)
+    _check(h0, "h0", f32, (Bsz, D, N), dev)
+    _check(conv_state_in, "conv_state_in", bf, (Bsz, D, W - 1), dev)
+    _check(dt_norm_w, "dt_norm_w", f32, (R,), dev)
+    _check(b_norm_w, "b_norm_w", f32, (N,), dev)
+    _check(c_norm_w, "c_norm_w", f32, (N,), dev)
+    made = []
+    if y is None:
+        y = torch.empty((Bsz, L, D), dtype=bf, device=dev)
+        made.append(y)
+    if h_last is None:
+        h_last = torch.empty((Bsz, D, N), dtype=f32, device=dev)
+        made.append(h_last)
+    if conv_state_out is None:
+        conv_state_out = torch.empty((Bsz, D, W - 1), dtype=bf, device=dev)
+        made.append(conv_state_out)
+    ws_bytes = projected_workspace_size(Bsz, L, D, R, N, W)
+    if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+        made.append(workspace)
+    with torch.cuda.device(dev):
+        st = lib().mamba_mixer_fwd_projected(
+            _ptr(xz), _ptr(conv_w), _ptr(conv_b), _ptr(W_x), _ptr(W_dt), _ptr(dt_bias), _ptr(A), _ptr(Dskip),
+            _ptr(h0), _ptr(conv_state_in), _ptr(dt_norm_w), _ptr(b_norm_w), _ptr(c_norm_w), float(norm_eps),
+            _ptr(y), _ptr(h_last), _ptr(conv_state_out), Bsz, L, D, N, R, W, MM_BF16, _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    if st != 0:
+        raise MixerError(st, "mamba_mixer_fwd_projected")
+    _keep_alive_on(made, (stream,))
+    return y, h_last, conv_state_out
+

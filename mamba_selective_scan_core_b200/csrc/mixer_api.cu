@@ -16,6 +16,8 @@
 #include "mamba_mixer.h"
 #include "mixer_decode.cuh"
 #include "mixer_prefill.cuh"
+#include "proj_gemm.cuh"
+#include "proj_ops.cuh"
 
 namespace {
 
@@ -120,7 +122,8 @@ unsigned long long next_call_id() { return (g_call_counter.fetch_add(1) + 1) & (
 //   lsum    [K-1][batch][D] f32       chunk step-size sums
 struct FwdPlan {
     int chunks = 1;
-    int64_t chunk_len = 0;
+    int64_t chunk0_len = 0;   // tokens of chunk 0
+    int64_t chunk_len = 0;    // tokens of every later chunk (the last one may be shorter)
     size_t off_tags = 0, off_state = 0, off_lsum = 0, ws_bytes = 0;
 };
 
@@ -185,7 +188,27 @@ FwdPlan plan_fwd(int64_t batch, int64_t seqlen, int64_t d_inner, int sms) {
         }
     }
     pl.chunk_len = chunk_tiles(k) * kTile;
+    pl.chunk0_len = pl.chunk_len;
     pl.chunks = static_cast<int>(seqlen > 0 ? (seqlen + pl.chunk_len - 1) / pl.chunk_len : 1);
+    // Chunk 0 needs no carried state, so its full pass runs while the summary
+    // pass runs; chunks 1.. start once every summary is stored.  The call then
+    // takes about max(l0, (1 + 0.55) l1) in tile units, with l0 the tiles of
+    // chunk 0 and l1 those of every other chunk: a longer chunk 0 and even
+    // chunks after it (instead of equal chunks and a short last one).
+    if (pl.chunks > 1 && !env_int("MAMBA_MIXER_CHUNKS", 1, 1 << 20)) {
+        const int64_t K = pl.chunks;
+        double best = 1e300;
+        int64_t best_l1 = 0;
+        for (int64_t l1 = 1; l1 * (K - 1) < tiles; ++l1) {
+            const int64_t l0 = tiles - l1 * (K - 1);
+            const double t = std::max(static_cast<double>(l0), 1.55 * static_cast<double>(l1));
+            if (t < best) { best = t; best_l1 = l1; }
+        }
+        if (best_l1 > 0) {
+            pl.chunk_len = best_l1 * kTile;
+            pl.chunk0_len = (tiles - best_l1 * (K - 1)) * kTile;
+        }
+    }
     const size_t c1 = static_cast<size_t>(pl.chunks - 1), B = static_cast<size_t>(batch);
     const size_t D = static_cast<size_t>(d_inner);
     pl.off_tags = kWsHeader;
@@ -387,6 +410,7 @@ cudaError_t launch_pass(PrefillParams p, const CtaShape& sh, int64_t batch, int 
 template <typename T, typename M>
 cudaError_t dispatch_prefill(PrefillParams p, int64_t batch, const FwdPlan& pl, int sm_count, cudaStream_t s) {
     p.chunk_len = pl.chunk_len;
+    p.chunk0_len = pl.chunk0_len;
     p.n_chunks = pl.chunks;
     const CtaShape full = shape_ctas<T>(p.D, batch, pl.chunks, sm_count);
     // The summary pass is launched normally: it starts after everything
@@ -413,6 +437,9 @@ struct FwdArgs {
     const void* cs_in; void* y; float* h_last; void* cs_out;
     int64_t batch, seqlen, d_inner, d_state, d_conv;
     mm_dtype act;
+    const float* b_norm_w = nullptr;   // optional RMSNorm of B_t / C_t ([d_state] each)
+    const float* c_norm_w = nullptr;
+    float norm_eps = 0.0f;
 };
 
 struct FwdBytes {
@@ -442,15 +469,17 @@ mm_status validate_fwd(const FwdArgs& a, FwdBytes* nb) {
     if (a.batch == 0) return MM_OK;
     if (!a.conv_w || !a.dt_bias || !a.A || !a.h_last || !a.cs_out) return MM_ERR_NULL;
     if (a.seqlen > 0 && (!a.xz || !a.dt || !a.Bm || !a.Cm || !a.y)) return MM_ERR_NULL;
+    if ((a.b_norm_w || a.c_norm_w) && !(a.norm_eps > 0.0f && a.norm_eps < 1e30f)) return MM_ERR_ARG;
     const void* all[] = {a.xz, a.conv_w, a.conv_b, a.dt, a.dt_bias, a.A, a.Bm, a.Cm, a.Dskip, a.h0, a.cs_in,
-                         a.y, a.h_last, a.cs_out};
+                         a.y, a.h_last, a.cs_out, a.b_norm_w, a.c_norm_w};
     for (const void* q : all)
         if (q && !aligned16(q)) return MM_ERR_ALIGN;
     const int64_t D = a.d_inner;
     const Span in[] = {span(a.xz, nb->xz), span(a.conv_w, D * a.d_conv * 4), span(a.conv_b, D * 4),
                        span(a.dt, nb->dt), span(a.dt_bias, D * 4), span(a.A, D * a.d_state * 4),
                        span(a.Bm, nb->bc), span(a.Cm, nb->bc), span(a.Dskip, D * 4),
-                       span(a.h0, nb->st), span(a.cs_in, nb->cs)};
+                       span(a.h0, nb->st), span(a.cs_in, nb->cs), span(a.b_norm_w, a.d_state * 4),
+                       span(a.c_norm_w, a.d_state * 4)};
     const Span out[] = {span(a.y, nb->dt), span(a.h_last, nb->st), span(a.cs_out, nb->cs)};
     for (const Span& o : out)
         for (const Span& i : in)
@@ -466,7 +495,8 @@ bool workspace_overlaps(const FwdArgs& a, const FwdBytes& nb, const void* ws, si
     const Span all[] = {span(a.xz, nb.xz), span(a.conv_w, D * a.d_conv * 4), span(a.conv_b, D * 4),
                         span(a.dt, nb.dt), span(a.dt_bias, D * 4), span(a.A, D * a.d_state * 4),
                         span(a.Bm, nb.bc), span(a.Cm, nb.bc), span(a.Dskip, D * 4), span(a.h0, nb.st),
-                        span(a.cs_in, nb.cs), span(a.y, nb.dt), span(a.h_last, nb.st), span(a.cs_out, nb.cs)};
+                        span(a.cs_in, nb.cs), span(a.y, nb.dt), span(a.h_last, nb.st), span(a.cs_out, nb.cs),
+                        span(a.b_norm_w, a.d_state * 4), span(a.c_norm_w, a.d_state * 4)};
     for (const Span& s : all)
         if (overlaps(w, s)) return true;
     return false;
@@ -492,6 +522,9 @@ mm_status run_fwd(const FwdArgs& a, const FwdPlan& pl, int sm_count, void* ws, u
     p.call_id = next_call_id();
     p.status_epoch = status_epoch;
     p.sum_octets = 1;
+    p.b_norm_w = a.b_norm_w;
+    p.c_norm_w = a.c_norm_w;
+    p.norm_eps = a.norm_eps;
     cudaError_t e = a.act == MM_BF16 ? dispatch_prefill<__nv_bfloat16, mm::MathFast>(p, a.batch, pl, sm_count, s)
                                      : dispatch_prefill<float, mm::MathExact>(p, a.batch, pl, sm_count, s);
     if (e != cudaSuccess) { cudaGetLastError(); return MM_ERR_CUDA; }
@@ -665,6 +698,7 @@ const char* mamba_status_string(mm_status status) {
         case MM_ERR_TIMEOUT:
             return "a kernel of the call gave up waiting (for its bulk copies, or for a chunk summary that was "
                    "never written); its outputs are not valid";
+        case MM_ERR_ARG: return "an argument value is out of range (norm_eps must be positive and finite)";
         case MM_ERR_SCRATCH_LIMIT:
             return "sizes need more scratch than mamba_mixer_fwd_noalloc's built-in 8 MiB; pass a workspace to "
                    "mamba_mixer_fwd instead";
@@ -709,17 +743,13 @@ size_t mamba_mixer_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner
     return plan_fwd(batch, seqlen, d_inner, plan_sms()).ws_bytes;
 }
 
-mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv_b,
-                          const void* dt, const float* dt_bias, const float* A,
-                          const void* Bm, const void* Cm, const float* Dskip,
-                          const float* h0, const void* conv_state_in,
-                          void* y, float* h_last, void* conv_state_out,
-                          int64_t batch, int64_t seqlen, int64_t d_inner,
-                          int64_t d_state, int64_t d_conv, mm_dtype act,
-                          void* workspace, size_t workspace_bytes, void* stream)
-{
-    const FwdArgs a{xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0, conv_state_in, y, h_last,
-                    conv_state_out, batch, seqlen, d_inner, d_state, d_conv, act};
+}  // extern "C"
+
+namespace {
+
+// mamba_mixer_fwd and mamba_mixer_fwd_normed: validate, check the workspace, launch.
+mm_status fwd_with_workspace(const FwdArgs& a, void* workspace, size_t workspace_bytes, void* stream) {
+    const int64_t batch = a.batch, seqlen = a.seqlen, d_inner = a.d_inner;
     FwdBytes nb;
     if (mm_status st = validate_fwd(a, &nb); st != MM_OK) return st;
     if (batch == 0) return MM_OK;
@@ -732,13 +762,54 @@ mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv
     return run_fwd(a, pl, sms, workspace, next_call_id(), static_cast<cudaStream_t>(stream));
 }
 
-mm_status mamba_state_update(const void* x, const void* z, const void* dt,
-                             const float* conv_w, const float* conv_b,
-                             const float* dt_bias, const float* Dskip, const float* A,
-                             const void* Bm, const void* Cm,
-                             float* ssm_state, void* conv_state, void* y,
-                             int64_t n_layers, int64_t batch, int64_t d_inner,
-                             int64_t d_state, int64_t d_conv, mm_dtype act, void* stream)
+}  // namespace
+
+extern "C" {
+
+mm_status mamba_mixer_fwd(const void* xz, const float* conv_w, const float* conv_b,
+                          const void* dt, const float* dt_bias, const float* A,
+                          const void* Bm, const void* Cm, const float* Dskip,
+                          const float* h0, const void* conv_state_in,
+                          void* y, float* h_last, void* conv_state_out,
+                          int64_t batch, int64_t seqlen, int64_t d_inner,
+                          int64_t d_state, int64_t d_conv, mm_dtype act,
+                          void* workspace, size_t workspace_bytes, void* stream)
+{
+    const FwdArgs a{xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0, conv_state_in, y, h_last,
+                    conv_state_out, batch, seqlen, d_inner, d_state, d_conv, act};
+    return fwd_with_workspace(a, workspace, workspace_bytes, stream);
+}
+
+mm_status mamba_mixer_fwd_normed(const void* xz, const float* conv_w, const float* conv_b,
+                                 const void* dt, const float* dt_bias, const float* A,
+                                 const void* Bm, const void* Cm, const float* Dskip,
+                                 const float* h0, const void* conv_state_in,
+                                 void* y, float* h_last, void* conv_state_out,
+                                 int64_t batch, int64_t seqlen, int64_t d_inner,
+                                 int64_t d_state, int64_t d_conv, mm_dtype act,
+                                 const float* b_norm_w, const float* c_norm_w, float norm_eps,
+                                 void* workspace, size_t workspace_bytes, void* stream)
+{
+    FwdArgs a{xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0, conv_state_in, y, h_last,
+              conv_state_out, batch, seqlen, d_inner, d_state, d_conv, act};
+    a.b_norm_w = b_norm_w;
+    a.c_norm_w = c_norm_w;
+    a.norm_eps = norm_eps;
+    return fwd_with_workspace(a, workspace, workspace_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+mm_status state_update_impl(const void* x, const void* z, const void* dt,
+                            const float* conv_w, const float* conv_b,
+                            const float* dt_bias, const float* Dskip, const float* A,
+                            const void* Bm, const void* Cm,
+                            float* ssm_state, void* conv_state, void* y,
+                            int64_t n_layers, int64_t batch, int64_t d_inner,
+                            int64_t d_state, int64_t d_conv, mm_dtype act,
+                            const float* b_norm_w, const float* c_norm_w, float norm_eps, void* stream)
 {
     if (act != MM_F32 && act != MM_BF16) return MM_ERR_DTYPE;
     if (n_layers < 0 || batch < 0 || d_inner <= 0 || d_state <= 0 || d_conv <= 0) return MM_ERR_SHAPE;
@@ -756,7 +827,9 @@ mm_status mamba_state_update(const void* x, const void* z, const void* dt,
 
     if (!x || !z || !dt || !conv_w || !dt_bias || !A || !Bm || !Cm || !ssm_state || !conv_state || !y)
         return MM_ERR_NULL;
-    const void* all[] = {x, z, dt, conv_w, conv_b, dt_bias, Dskip, A, Bm, Cm, ssm_state, conv_state, y};
+    if ((b_norm_w || c_norm_w) && !(norm_eps > 0.0f && norm_eps < 1e30f)) return MM_ERR_ARG;
+    const void* all[] = {x, z, dt, conv_w, conv_b, dt_bias, Dskip, A, Bm, Cm, ssm_state, conv_state, y,
+                         b_norm_w, c_norm_w};
     for (const void* q : all)
         if (q && !aligned16(q)) return MM_ERR_ALIGN;
 
@@ -764,7 +837,8 @@ mm_status mamba_state_update(const void* x, const void* z, const void* dt,
     const int64_t par = n_layers * d_inner * 4;
     const Span in[] = {span(x, tok_bytes), span(z, tok_bytes), span(dt, tok_bytes),
                        span(conv_w, par * d_conv), span(conv_b, par), span(dt_bias, par), span(Dskip, par),
-                       span(A, par * d_state), span(Bm, lb * d_state * es), span(Cm, lb * d_state * es)};
+                       span(A, par * d_state), span(Bm, lb * d_state * es), span(Cm, lb * d_state * es),
+                       span(b_norm_w, n_layers * d_state * 4), span(c_norm_w, n_layers * d_state * 4)};
     const Span io[] = {span(ssm_state, st_bytes), span(conv_state, rows * (d_conv - 1) * es), span(y, tok_bytes)};
     for (const Span& o : io)
         for (const Span& i : in)
@@ -775,22 +849,54 @@ mm_status mamba_state_update(const void* x, const void* z, const void* dt,
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const unsigned grid = static_cast<unsigned>((warps + 7) / 8);
-    if (act == MM_BF16) {
-        using T = __nv_bfloat16;
-        mm::state_update_kernel<T, mm::MathFast><<<grid, 256, 0, s>>>(
+    auto launch = [&](auto tag_t, auto math, auto norm) {
+        using T = decltype(tag_t);
+        constexpr bool NORM = decltype(norm)::value;
+        mm::state_update_kernel<T, decltype(math), NORM><<<grid, 256, 0, s>>>(
             static_cast<const T*>(x), static_cast<const T*>(z), static_cast<const T*>(dt), conv_w, conv_b,
             dt_bias, Dskip, A, static_cast<const T*>(Bm), static_cast<const T*>(Cm), ssm_state,
             static_cast<T*>(conv_state), static_cast<T*>(y), static_cast<int>(n_layers), static_cast<int>(batch),
-            static_cast<int>(d_inner));
+            static_cast<int>(d_inner), b_norm_w, c_norm_w, norm_eps);
+    };
+    const bool norm = b_norm_w || c_norm_w;
+    if (act == MM_BF16) {
+        if (norm) launch(__nv_bfloat16{}, mm::MathFast{}, std::true_type{});
+        else launch(__nv_bfloat16{}, mm::MathFast{}, std::false_type{});
     } else {
-        mm::state_update_kernel<float, mm::MathExact><<<grid, 256, 0, s>>>(
-            static_cast<const float*>(x), static_cast<const float*>(z), static_cast<const float*>(dt), conv_w,
-            conv_b, dt_bias, Dskip, A, static_cast<const float*>(Bm), static_cast<const float*>(Cm), ssm_state,
-            static_cast<float*>(conv_state), static_cast<float*>(y), static_cast<int>(n_layers),
-            static_cast<int>(batch), static_cast<int>(d_inner));
+        if (norm) launch(float{}, mm::MathExact{}, std::true_type{});
+        else launch(float{}, mm::MathExact{}, std::false_type{});
     }
     if (cudaGetLastError() != cudaSuccess) return MM_ERR_CUDA;
     return MM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mm_status mamba_state_update(const void* x, const void* z, const void* dt,
+                             const float* conv_w, const float* conv_b,
+                             const float* dt_bias, const float* Dskip, const float* A,
+                             const void* Bm, const void* Cm,
+                             float* ssm_state, void* conv_state, void* y,
+                             int64_t n_layers, int64_t batch, int64_t d_inner,
+                             int64_t d_state, int64_t d_conv, mm_dtype act, void* stream)
+{
+    return state_update_impl(x, z, dt, conv_w, conv_b, dt_bias, Dskip, A, Bm, Cm, ssm_state, conv_state, y,
+                             n_layers, batch, d_inner, d_state, d_conv, act, nullptr, nullptr, 0.0f, stream);
+}
+
+mm_status mamba_state_update_normed(const void* x, const void* z, const void* dt,
+                                    const float* conv_w, const float* conv_b,
+                                    const float* dt_bias, const float* Dskip, const float* A,
+                                    const void* Bm, const void* Cm,
+                                    float* ssm_state, void* conv_state, void* y,
+                                    int64_t n_layers, int64_t batch, int64_t d_inner,
+                                    int64_t d_state, int64_t d_conv, mm_dtype act,
+                                    const float* b_norm_w, const float* c_norm_w, float norm_eps, void* stream)
+{
+    return state_update_impl(x, z, dt, conv_w, conv_b, dt_bias, Dskip, A, Bm, Cm, ssm_state, conv_state, y,
+                             n_layers, batch, d_inner, d_state, d_conv, act, b_norm_w, c_norm_w, norm_eps, stream);
 }
 
 mm_status mamba_mixer_fwd_noalloc(const void* xz, const float* conv_w, const float* conv_b,
@@ -971,3 +1077,280 @@ mm_status mamba_mixer_fwd_host(const void* xz, const float* conv_w, const float*
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- projections (tcgen05 GEMM)
+namespace {
+
+// 2-D map over a row-major [rows][cols] bf16 matrix, [box_rows][64] boxes,
+// 128-byte swizzle (the layout the MMA's shared-memory descriptor reads).
+bool encode_gemm_2d(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * 2)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(mm::kGemmBK), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tile width of the GEMM for N output columns: one tile up to 144 columns
+// (x_proj's 288 = 2 x 144), else 256-column tiles.
+int gemm_bn(int64_t N) { return N <= 64 ? 64 : N <= 128 ? 128 : (N <= 144 || N == 288) ? 144 : 256; }
+
+template <int BN, int STAGES, bool OUT_BF16>
+cudaError_t launch_gemm_t(const mm::GemmParams& gp, const void* A, const void* W, int ksplit, cudaStream_t s) {
+    CUtensorMap ta, tw;
+    if (!encode_gemm_2d(&ta, A, gp.K, gp.M, mm::kGemmBM) || !encode_gemm_2d(&tw, W, gp.K, gp.N, BN))
+        return cudaErrorInvalidValue;
+    auto kern = mm::proj_gemm_kernel<BN, STAGES, OUT_BF16>;
+    const int smem = mm::GemmLayout<BN>::smem_bytes(STAGES);
+    static std::atomic<unsigned long long> smem_allowed{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaGetLastError();
+    const unsigned long long bit = dev < 64 ? 1ull << dev : 0;
+    if (!(bit && (smem_allowed.load() & bit))) {
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        if (bit) smem_allowed.fetch_or(bit);
+    }
+    const dim3 grid(static_cast<unsigned>((gp.M + mm::kGemmBM - 1) / mm::kGemmBM),
+                    static_cast<unsigned>((gp.N + BN - 1) / BN), static_cast<unsigned>(ksplit));
+    kern<<<grid, mm::kGemmThreads, forced_launch_failure() ? (1 << 20) : smem, s>>>(gp, ta, tw);
+    return cudaGetLastError();
+}
+
+template <bool OUT_BF16>
+cudaError_t launch_gemm(mm::GemmParams gp, const void* A, const void* W, int ksplit, cudaStream_t s) {
+    switch (gemm_bn(gp.N)) {
+        case 64: return launch_gemm_t<64, 8, OUT_BF16>(gp, A, W, ksplit, s);
+        case 128: return launch_gemm_t<128, 6, OUT_BF16>(gp, A, W, ksplit, s);
+        case 144: return launch_gemm_t<144, 6, OUT_BF16>(gp, A, W, ksplit, s);
+        default: return launch_gemm_t<256, 4, OUT_BF16>(gp, A, W, ksplit, s);
+    }
+}
+
+// Plan of the mixer with its projections: regions of its workspace (each
+// 256-byte aligned; the scan's own workspace first, so mamba_check_status
+// reads the call's status at the workspace's start) and x_proj's split.
+struct ProjPlan {
+    FwdPlan scan;
+    int64_t M = 0;          // tokens (batch x seqlen)
+    int R = 0, NC = 0;      // dt_rank, x_proj's output width R + 2 d_state
+    int ksplit = 1;
+    size_t off_u = 0, off_part = 0, off_dtlow = 0, off_b = 0, off_c = 0, off_dt = 0, total = 0;
+};
+
+ProjPlan plan_projected(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t dt_rank, int sms) {
+    ProjPlan pp;
+    pp.scan = plan_fwd(batch, seqlen, d_inner, sms);
+    pp.M = batch * seqlen;
+    pp.R = static_cast<int>(dt_rank);
+    pp.NC = pp.R + 32;
+    const int64_t m_tiles = (pp.M + mm::kGemmBM - 1) / mm::kGemmBM;
+    const int64_t n_tiles = (pp.NC + gemm_bn(pp.NC) - 1) / gemm_bn(pp.NC);
+    const int64_t k_tiles = (d_inner + mm::kGemmBK - 1) / mm::kGemmBK;
+    // split K until the x_proj grid covers the SMs once (one CTA per SM: its ring fills shared memory)
+    int64_t split = std::max<int64_t>(1, sms / std::max<int64_t>(1, m_tiles * n_tiles));
+    pp.ksplit = static_cast<int>(std::min<int64_t>({split, k_tiles, 16}));
+    const size_t M = static_cast<size_t>(pp.M), D = static_cast<size_t>(d_inner);
+    pp.off_u = align256(pp.scan.ws_bytes);
+    pp.off_part = pp.off_u + align256(M * D * 2);
+    pp.off_dtlow = pp.off_part + align256(static_cast<size_t>(pp.ksplit) * M * pp.NC * 4);
+    pp.off_b = pp.off_dtlow + align256(M * pp.R * 2);
+    pp.off_c = pp.off_b + align256(M * 16 * 2);
+    pp.off_dt = pp.off_c + align256(M * 16 * 2);
+    pp.total = pp.off_dt + align256(M * D * 2);
+    return pp;
+}
+
+bool proj_sizes_ok(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state, int64_t dt_rank,
+                   int64_t d_conv) {
+    int64_t tokens;
+    return batch >= 0 && seqlen >= 0 && d_inner > 0 && d_state == 16 && d_conv == 4 && d_inner % 64 == 0 &&
+           d_inner <= (1 << 20) && dt_rank > 0 && dt_rank % 32 == 0 && dt_rank <= 1024 &&
+           mul_ok(batch, seqlen, &tokens) && tokens < (int64_t(1) << 31) && seqlen_ok(seqlen, d_inner, 2);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mamba_proj_matmul_workspace_size(int64_t M, int64_t N, int64_t K) {
+    if (M <= 0 || N <= 0 || K <= 0 || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+        return 0;
+    return kWsHeader;
+}
+
+mm_status mamba_proj_matmul(const void* A, const void* W, void* out, int64_t M, int64_t N, int64_t K,
+                            mm_dtype out_dtype, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (out_dtype != MM_F32 && out_dtype != MM_BF16) return MM_ERR_DTYPE;
+    if (M < 0 || N <= 0 || K <= 0 || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+        return MM_ERR_SHAPE;
+    if (K % 8 != 0 || N % 8 != 0) return MM_ERR_UNSUPPORTED;
+    if (M == 0) return MM_OK;
+    if (!A || !W || !out) return MM_ERR_NULL;
+    if (!aligned16(A) || !aligned16(W) || !aligned16(out)) return MM_ERR_ALIGN;
+    const int64_t es = out_dtype == MM_F32 ? 4 : 2;
+    const Span a = span(A, M * K * 2), w = span(W, N * K * 2), o = span(out, M * N * es);
+    if (overlaps(o, a) || overlaps(o, w)) return MM_ERR_ALIAS;
+    if (!workspace || workspace_bytes < kWsHeader) return MM_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MM_ERR_ALIGN;
+    const Span ws = span(workspace, kWsHeader);
+    if (overlaps(ws, a) || overlaps(ws, w) || overlaps(ws, o)) return MM_ERR_ALIAS;
+    if (mm_status st = check_device(); st != MM_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the call's status: hdr[1] = epoch, written before the GEMM in stream order
+    const unsigned long long epoch = next_call_id();
+    unsigned long long* hdr = static_cast<unsigned long long*>(workspace);
+    if (cudaMemcpyAsync(hdr + 1, &epoch, sizeof(epoch), cudaMemcpyHostToDevice, s) != cudaSuccess) {
+        cudaGetLastError();
+        return MM_ERR_CUDA;
+    }
+    mm::GemmParams gp{};
+    gp.out = out;
+    gp.ldo = N;
+    gp.split_stride = 0;
+    gp.M = static_cast<int>(M);
+    gp.N = static_cast<int>(N);
+    gp.K = static_cast<int>(K);
+    gp.k_tiles_per_split = static_cast<int>((K + mm::kGemmBK - 1) / mm::kGemmBK);
+    gp.wait_limit = copy_wait_limit();
+    gp.status = hdr;
+    gp.status_epoch = epoch;
+    const cudaError_t e = out_dtype == MM_BF16 ? launch_gemm<true>(gp, A, W, 1, s) : launch_gemm<false>(gp, A, W, 1, s);
+    if (e != cudaSuccess) { cudaGetLastError(); return MM_ERR_CUDA; }
+    return MM_OK;
+}
+
+mm_status mamba_mixer_projected_layout(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state,
+                                       int64_t dt_rank, int64_t d_conv, size_t offsets[5]) {
+    if (!offsets) return MM_ERR_NULL;
+    if (batch <= 0 || !proj_sizes_ok(batch, seqlen, d_inner, d_state, dt_rank, d_conv)) return MM_ERR_SHAPE;
+    const ProjPlan pp = plan_projected(batch, seqlen, d_inner, dt_rank, plan_sms());
+    offsets[0] = pp.off_u;
+    offsets[1] = pp.off_dtlow;
+    offsets[2] = pp.off_b;
+    offsets[3] = pp.off_c;
+    offsets[4] = pp.off_dt;
+    return MM_OK;
+}
+
+size_t mamba_mixer_projected_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state,
+                                            int64_t dt_rank, int64_t d_conv, mm_dtype act) {
+    if (act != MM_BF16 || batch <= 0 || !proj_sizes_ok(batch, seqlen, d_inner, d_state, dt_rank, d_conv)) return 0;
+    return plan_projected(batch, seqlen, d_inner, dt_rank, plan_sms()).total;
+}
+
+mm_status mamba_mixer_fwd_projected(const void* xz, const float* conv_w, const float* conv_b,
+                                    const void* W_x, const void* W_dt, const float* dt_bias, const float* A,
+                                    const float* Dskip, const float* h0, const void* conv_state_in,
+                                    const float* dt_norm_w, const float* b_norm_w, const float* c_norm_w,
+                                    float norm_eps, void* y, float* h_last, void* conv_state_out,
+                                    int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state,
+                                    int64_t dt_rank, int64_t d_conv, mm_dtype act,
+                                    void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (act != MM_F32 && act != MM_BF16) return MM_ERR_DTYPE;
+    if (act != MM_BF16) return MM_ERR_UNSUPPORTED;        // the tensor-core products take bf16 operands
+    if (batch < 0 || seqlen < 0 || d_inner <= 0 || d_state <= 0 || dt_rank <= 0 || d_conv <= 0) return MM_ERR_SHAPE;
+    if (!proj_sizes_ok(batch, seqlen, d_inner, d_state, dt_rank, d_conv)) {
+        if (d_state != 16 || d_conv != 4 || d_inner % 64 != 0 || dt_rank % 32 != 0) return MM_ERR_UNSUPPORTED;
+        return MM_ERR_SHAPE;
+    }
+    if (batch == 0) return MM_OK;
+    if (!W_x || !W_dt) return MM_ERR_NULL;
+    if (!aligned16(W_x) || !aligned16(W_dt)) return MM_ERR_ALIGN;
+    if ((dt_norm_w || b_norm_w || c_norm_w) && !(norm_eps > 0.0f && norm_eps < 1e30f)) return MM_ERR_ARG;
+    for (const void* q : {static_cast<const void*>(dt_norm_w), static_cast<const void*>(b_norm_w),
+                          static_cast<const void*>(c_norm_w)})
+        if (q && !aligned16(q)) return MM_ERR_ALIGN;
+    const int sms = plan_sms();
+    const ProjPlan pp = plan_projected(batch, seqlen, d_inner, dt_rank, sms);
+    if (!workspace || workspace_bytes < pp.total) return MM_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MM_ERR_ALIGN;
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    __nv_bfloat16* u = reinterpret_cast<__nv_bfloat16*>(ws + pp.off_u);
+    float* part = reinterpret_cast<float*>(ws + pp.off_part);
+    __nv_bfloat16* dtlow = reinterpret_cast<__nv_bfloat16*>(ws + pp.off_dtlow);
+    __nv_bfloat16* Bm = reinterpret_cast<__nv_bfloat16*>(ws + pp.off_b);
+    __nv_bfloat16* Cm = reinterpret_cast<__nv_bfloat16*>(ws + pp.off_c);
+    __nv_bfloat16* dt = reinterpret_cast<__nv_bfloat16*>(ws + pp.off_dt);
+    // the scan's arguments, validated as one mamba_mixer_fwd_normed call on the
+    // workspace's intermediates (B and C are already normalised by x_proj's epilogue)
+    const FwdArgs a{xz, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0, conv_state_in, y, h_last,
+                    conv_state_out, batch, seqlen, d_inner, d_state, d_conv, act};
+    FwdBytes nb;
+    if (mm_status st = validate_fwd(a, &nb); st != MM_OK) return st;
+    // the weights and the caller's buffers may not overlap the workspace
+    {
+        const Span w = span(workspace, static_cast<int64_t>(pp.total));
+        const int64_t NC = pp.NC;
+        const Span ins[] = {span(xz, nb.xz), span(conv_w, d_inner * d_conv * 4), span(conv_b, d_inner * 4),
+                            span(W_x, NC * d_inner * 2), span(W_dt, d_inner * dt_rank * 2), span(dt_bias, d_inner * 4),
+                            span(A, d_inner * d_state * 4), span(Dskip, d_inner * 4), span(h0, nb.st),
+                            span(conv_state_in, nb.cs), span(dt_norm_w, dt_rank * 4), span(b_norm_w, 64),
+                            span(c_norm_w, 64), span(y, nb.dt), span(h_last, nb.st), span(conv_state_out, nb.cs)};
+        for (const Span& q : ins)
+            if (overlaps(w, q)) return MM_ERR_ALIAS;
+        const Span outs[] = {span(y, nb.dt), span(h_last, nb.st), span(conv_state_out, nb.cs)};
+        for (const Span& o : outs)
+            if (overlaps(o, span(W_x, NC * d_inner * 2)) || overlaps(o, span(W_dt, d_inner * dt_rank * 2)) ||
+                overlaps(o, span(dt_norm_w, dt_rank * 4)))
+                return MM_ERR_ALIAS;
+    }
+    if (mm_status st = check_device(); st != MM_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const unsigned long long epoch = next_call_id();
+    unsigned long long* hdr = reinterpret_cast<unsigned long long*>(ws);
+    if (seqlen > 0) {
+        const int64_t M = pp.M;
+        // u = SiLU(conv(x))
+        {
+            const dim3 grid(static_cast<unsigned>((d_inner / 8 + 127) / 128),
+                            static_cast<unsigned>((seqlen + mm::kConvTokens - 1) / mm::kConvTokens),
+                            static_cast<unsigned>(batch));
+            mm::conv_silu_kernel<<<grid, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(xz), conv_w, conv_b,
+                                                      static_cast<const __nv_bfloat16*>(conv_state_in), u, seqlen,
+                                                      static_cast<int>(d_inner));
+            if (cudaGetLastError() != cudaSuccess) return MM_ERR_CUDA;
+        }
+        // x_proj partials: [ksplit][M][R + 32] fp32
+        mm::GemmParams gp{};
+        gp.out = part;
+        gp.ldo = pp.NC;
+        gp.split_stride = M * pp.NC;
+        gp.M = static_cast<int>(M);
+        gp.N = pp.NC;
+        gp.K = static_cast<int>(d_inner);
+        const int k_tiles = static_cast<int>((d_inner + mm::kGemmBK - 1) / mm::kGemmBK);
+        gp.k_tiles_per_split = (k_tiles + pp.ksplit - 1) / pp.ksplit;
+        gp.wait_limit = copy_wait_limit();
+        gp.status = hdr;
+        gp.status_epoch = epoch;
+        if (launch_gemm<false>(gp, u, W_x, pp.ksplit, s) != cudaSuccess) { cudaGetLastError(); return MM_ERR_CUDA; }
+        // sum the partials; split into dt_low | B | C, normalised, bf16
+        mm::xproj_epilogue_kernel<<<static_cast<unsigned>((M + 7) / 8), 256, 0, s>>>(
+            part, pp.ksplit, gp.split_stride, M, pp.R, dt_norm_w, b_norm_w, c_norm_w, norm_eps, dtlow, Bm, Cm);
+        if (cudaGetLastError() != cudaSuccess) return MM_ERR_CUDA;
+        // dt = dt_low W_dt^T: [M][d_inner] bf16
+        mm::GemmParams gd{};
+        gd.out = dt;
+        gd.ldo = d_inner;
+        gd.M = static_cast<int>(M);
+        gd.N = static_cast<int>(d_inner);
+        gd.K = pp.R;
+        gd.k_tiles_per_split = (pp.R + mm::kGemmBK - 1) / mm::kGemmBK;
+        gd.wait_limit = gp.wait_limit;
+        gd.status = hdr;
+        gd.status_epoch = epoch;
+        if (launch_gemm<true>(gd, dtlow, W_dt, 1, s) != cudaSuccess) { cudaGetLastError(); return MM_ERR_CUDA; }
+    }
+    // the selective scan on (x, z, dt, B, C)
+    return run_fwd(a, pp.scan, sms, workspace, epoch, s);
+}
+
+}  // extern "C"
+

@@ -50,20 +50,34 @@ template <> struct Vec4Act<__nv_bfloat16> {
     }
 };
 
+// RMSNorm of a 16-entry row held as 4 values in each lane of a quad: the
+// sum of squares is combined across the quad by two shuffles.
+__device__ __forceinline__ float4 rms_scale4(float4 v, const float* w, float eps) {
+    float ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, v.w * v.w)));
+    ss += __shfl_xor_sync(kFull, ss, 1);
+    ss += __shfl_xor_sync(kFull, ss, 2);
+    const float sc = rsqrtf(fmaf(ss, 1.0f / 16.0f, eps));
+    const float4 wv = __ldg(reinterpret_cast<const float4*>(w));
+    return make_float4(v.x * sc * wv.x, v.y * sc * wv.y, v.z * sc * wv.z, v.w * sc * wv.w);
+}
+
 // Batch rows a warp walks for one (layer, 32-channel block).  A and the
 // per-channel parameters come from HBM/L2 once per warp and from L1 for the
 // other rows, so the per-layer data costs 1/16 of a row's traffic.
 constexpr int kDecodeBatchChunk = 16;
 
 // The fp32 path's libm calls need more registers; it keeps 3 CTAs per SM.
-template <typename T, typename M>
-__global__ void __launch_bounds__(256, sizeof(T) == 4 ? 3 : MM_DECODE_MIN_BLOCKS)
+// NORM: the RMSNorm of each row's B and C is applied (a separate instance at 3
+// CTAs per SM, so the plain step keeps its register budget and occupancy).
+template <typename T, typename M, bool NORM>
+__global__ void __launch_bounds__(256, (sizeof(T) == 4 || NORM) ? 3 : MM_DECODE_MIN_BLOCKS)
 state_update_kernel(const T* __restrict__ x, const T* __restrict__ z, const T* __restrict__ dt,
                     const float* __restrict__ conv_w, const float* __restrict__ conv_b,
                     const float* __restrict__ dt_bias, const float* __restrict__ Dskip,
                     const float* __restrict__ A, const T* __restrict__ Bm, const T* __restrict__ Cm,
                     float* __restrict__ ssm_state, T* __restrict__ conv_state, T* __restrict__ y,
-                    int n_layers, int batch, int D)
+                    int n_layers, int batch, int D,
+                    const float* __restrict__ b_norm_w, const float* __restrict__ c_norm_w, float norm_eps)
 {
     const int lane = threadIdx.x & 31;
     const int q = lane & 3;            // which 4 states of a row
@@ -105,8 +119,13 @@ state_update_kernel(const T* __restrict__ x, const T* __restrict__ z, const T* _
             hv[pass] = d0 + pass * 8 + rr < D
                            ? __ldcs(reinterpret_cast<const float4*>(ssm_state + (rowbase + pass * 8 + rr) * 16 + q * 4))
                            : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 bq = Vec4Act<T>::load(Bm + lb * 16 + q * 4);
-        const float4 cq = Vec4Act<T>::load(Cm + lb * 16 + q * 4);
+        float4 bq = Vec4Act<T>::load(Bm + lb * 16 + q * 4);
+        float4 cq = Vec4Act<T>::load(Cm + lb * 16 + q * 4);
+        // optional RMSNorm of the row's B and C over their 16 entries (4 lanes x 4)
+        if constexpr (NORM) {
+            if (b_norm_w) bq = rms_scale4(bq, b_norm_w + static_cast<int64_t>(layer) * 16 + q * 4, norm_eps);
+            if (c_norm_w) cq = rms_scale4(cq, c_norm_w + static_cast<int64_t>(layer) * 16 + q * 4, norm_eps);
+        }
 
         // ---- row phase: lane i does the per-row work of channel d0 + i
         float l = 0.f, s = 0.f, u = 0.f, gz = 0.f;

@@ -103,7 +103,8 @@ struct PrefillParams {
     int D;              // d_inner
     int octets;         // channel octets (8 channels, 4 threads) per CTA
     int ctas_per_seq;   // CTAs per sequence
-    int64_t chunk_len;  // tokens per time chunk (a multiple of the tile)
+    int64_t chunk0_len; // tokens of time chunk 0
+    int64_t chunk_len;  // tokens of every later time chunk (the last one may end early)
     int n_chunks;       // time chunks K (blockIdx.y of the full pass)
     float* ws_state;    // [K-1][batch][16][D]: end state of chunk c run from zero (state-major)
     float* ws_lsum;     // [K-1][batch][D]:     sum over chunk c of the step size l
@@ -119,6 +120,12 @@ struct PrefillParams {
     unsigned long long call_id;       // unique per launch pair (summary + full pass)
     unsigned long long status_epoch;  // the epoch hdr[] is written with
     int sum_octets;     // channel octets per summary-pass CTA (its tag stride)
+    // Optional RMSNorm of B_t and C_t over their 16 entries before the
+    // recurrence: B_t[n] * b_norm_w[n] / sqrt(mean(B_t^2) + norm_eps), the same
+    // for C.  NULL = that input is used as it is.
+    const float* b_norm_w;
+    const float* c_norm_w;
+    float norm_eps;
     int batch;
     unsigned wait_limit;  // tries per wait on a bulk copy before giving up (fault)
 };
@@ -222,8 +229,8 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
     const int64_t L = p.L;
     const int D = p.D;
     const int nthreads = blockDim.x;
-    const int64_t t_begin = static_cast<int64_t>(chunk) * p.chunk_len;
-    const int64_t t_end = min(L, t_begin + p.chunk_len);
+    const int64_t t_begin = chunk == 0 ? 0 : p.chunk0_len + static_cast<int64_t>(chunk - 1) * p.chunk_len;
+    const int64_t t_end = min(L, chunk == 0 ? p.chunk0_len : t_begin + p.chunk_len);
 
     using Lay = PrefillLayout<T>;
     const int rs = p.octets * 8;                 // elements per staged row (the copy box width)
@@ -561,10 +568,21 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
             {
                 const T* bs = reinterpret_cast<const T*>(st + offBC);
                 constexpr int cstride = Lay::bc_bytes(TILE) / static_cast<int>(sizeof(T));   // elements from B to C
+                const bool normed = p.b_norm_w != nullptr || p.c_norm_w != nullptr;
+                // The loop's trip count and thread count are multiples of 32, so each
+                // half-warp holds one 16-entry row (one token's B or C) in every pass:
+                // the RMSNorm's sum of squares is four shuffles within it.
                 for (int i = tid; i < TILE * 16 * kBC; i += nthreads) {
                     const int r = i / (16 * kBC);
                     const int e = i - r * 16 * kBC;               // 0..15 B, 16..31 C
                     float v = A_::to_f32(bs[(e >> 4) * cstride + r * 16 + (e & 15)]);
+                    if (normed) {
+                        float ss = v * v;
+#pragma unroll
+                        for (int o = 1; o < 16; o <<= 1) ss += __shfl_xor_sync(kFull, ss, o);
+                        const float* w = (e >> 4) ? p.c_norm_w : p.b_norm_w;
+                        if (w) v *= rsqrtf(fmaf(ss, 1.0f / 16.0f, p.norm_eps)) * __ldg(w + (e & 15));
+                    }
                     if (e < 16) v *= M::step_scale;
                     *reinterpret_cast<float2*>(bcf + r * 64 + 2 * e) = f2(v, v);
                 }

@@ -232,8 +232,20 @@ def matmul_nt(A, Bw, threads: int = 1, library=None):
     return C.reshape(A.shape[:-1] + (N,))
 
 
+def _store(a, store):
+    """An intermediate as a bf16 implementation stores it: rounded to nearest
+    even (torch's cast), then widened back; store=None keeps it exact."""
+    if store is None:
+        return a
+    if store != "bf16":
+        raise ValueError(f"unknown storage dtype {store!r}")
+    import torch
+
+    return torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
 def projected_fwd(xz, conv_w, conv_b, W_x, W_dt, dt_bias, A, Dskip, h0=None, conv_state_in=None,
-                  dt_norm_w=None, b_norm_w=None, c_norm_w=None, norm_eps: float = 1e-6,
+                  dt_norm_w=None, b_norm_w=None, c_norm_w=None, norm_eps: float = 1e-6, store=None,
                   threads: int = 1, library=None):
     """The mixer with its producers, in the order the method runs them:
         u      = SiLU(causal conv(x))                        [B, L, D]
@@ -242,6 +254,9 @@ def projected_fwd(xz, conv_w, conv_b, W_x, W_dt, dt_bias, A, Dskip, h0=None, con
         (each optionally RMS-normalised over its own width)
         dt     = dt_low @ W_dt^T, W_dt [D, R]                [B, L, D]
         y, h_last, conv_state_out = the selective scan on (x, z, dt, B, C)
+    With store="bf16" the intermediates an implementation keeps in memory
+    between these steps (u, dt_low, B, C, dt) are rounded to bf16 where they are
+    stored, as the bf16 activations they are; the arithmetic stays fp64.
     Returns the scan's outputs plus the intermediates u, dt_low, Bm, Cm, dt."""
     L_ = library or lib()
     xz_ = _f64(xz)
@@ -255,7 +270,7 @@ def projected_fwd(xz, conv_w, conv_b, W_x, W_dt, dt_bias, A, Dskip, h0=None, con
     zeros_bc = np.zeros((Bsz, Lq, N))
     tr = mixer_fwd(xz_, conv_w, conv_b, np.zeros((Bsz, Lq, D)), None, A, zeros_bc, zeros_bc, None, None,
                    conv_state_in, threads=threads, traces=True, library=L_)
-    u = tr["u"]
+    u = _store(tr["u"], store)
     x_dbl = matmul_nt(u, W_x, threads=threads, library=L_)
     dt_low, Bm, Cm = x_dbl[..., :R], x_dbl[..., R:R + N], x_dbl[..., R + N:]
     if dt_norm_w is not None:
@@ -264,7 +279,8 @@ def projected_fwd(xz, conv_w, conv_b, W_x, W_dt, dt_bias, A, Dskip, h0=None, con
         Bm = rmsnorm_rows(Bm, b_norm_w, norm_eps, L_)
     if c_norm_w is not None:
         Cm = rmsnorm_rows(Cm, c_norm_w, norm_eps, L_)
-    dt = matmul_nt(dt_low, W_dt, threads=threads, library=L_)
+    dt_low, Bm, Cm = _store(dt_low, store), _store(Bm, store), _store(Cm, store)
+    dt = _store(matmul_nt(dt_low, W_dt, threads=threads, library=L_), store)
     out = mixer_fwd(xz_, conv_w, conv_b, dt, dt_bias, A, Bm, Cm, Dskip, h0, conv_state_in, threads=threads,
                     library=L_)
     out.update(u=u, dt_low=dt_low, Bm=Bm, Cm=Cm, dt=dt)

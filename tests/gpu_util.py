@@ -58,7 +58,7 @@ def _record(name, n, margin):
     MARGINS.append((test, name, int(n), float(margin)))
 
 
-def assert_close(got, ref, act: str, name: str, stored_bf16: bool = False):
+def assert_close(got, ref, act: str, name: str, stored_bf16: bool = False, rounded_steps: int = 0):
     """fp32: |err| <= 1e-4 (1 + |ref|) elementwise.
 
     bf16 inputs / fp32 state: max |err| <= 2e-2 rms(ref), applied to the
@@ -67,7 +67,14 @@ def assert_close(got, ref, act: str, name: str, stored_bf16: bool = False):
     differ by a further 2^-8 |ref| (half a bf16 ulp), because even the exact
     result rounded to bf16 differs from the unrounded oracle by that much and
     these outputs reach 10-20x their rms.  The rms of the error must also stay
-    within 2e-2 rms(ref)."""
+    within 2e-2 rms(ref).
+
+    rounded_steps: for a chain that stores that many intermediates in bf16
+    between its kernels, each may round one step (2^-8 relative, half an ulp
+    either side) differently on the GPU's fp32 sums than on the oracle's fp64
+    ones; each such step moves the output by up to that much of its own
+    magnitude, so the max-error budget excludes a further rounded_steps *
+    2^-8 |ref|.  The rms budget is unchanged."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert got.shape == ref.shape, (name, got.shape, ref.shape)
@@ -82,7 +89,7 @@ def assert_close(got, ref, act: str, name: str, stored_bf16: bool = False):
     if not err.size:
         return 0.0
     rms = float(np.sqrt(np.mean(ref ** 2)))
-    excess = err - (BF16_HALF_ULP * np.abs(ref) if stored_bf16 else 0.0)
+    excess = err - ((BF16_HALF_ULP if stored_bf16 else 0.0) + rounded_steps * BF16_HALF_ULP) * np.abs(ref)
     mx = float(excess.max())
     rerr = float(np.sqrt(np.mean(err ** 2)))
     bound = BF16_FRAC * rms + 1e-30

@@ -457,6 +457,26 @@ def pin_projected_forward_wiring(lib):
     want = _fwd(lib, dict(case, dt=dt, Bm=Bm, Cm=Cm))
     for k in ("y", "h_last", "conv_state_out"):
         np.testing.assert_allclose(got[k], want[k], rtol=1e-10, atol=1e-12)
+    # stored as bf16: each intermediate is the exact one rounded by torch's cast
+    import torch
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).to(torch.float64).numpy()
+
+    got_b = oracle.projected_fwd(case["xz"], case["conv_w"], case["conv_b"], W_x, W_dt, case["dt_bias"], case["A"],
+                                 case["Dskip"], case["h0"], case["conv_state_in"], dt_norm_w=wd, b_norm_w=wb,
+                                 c_norm_w=wc, norm_eps=0.1, store="bf16", library=lib)
+    ub = bf(u)
+    xb = ub @ W_x.T
+    dlb, Bb, Cb = bf(rms(xb[..., :R], wd)), bf(rms(xb[..., R:R + N], wb)), bf(rms(xb[..., R + N:], wc))
+    dtb = bf(dlb @ W_dt.T)
+    np.testing.assert_array_equal(got_b["u"], ub)
+    # the products are summed in another order than numpy's: a value next to a
+    # rounding boundary may land one bf16 step (2^-7 relative) away
+    for k, v in (("dt_low", dlb), ("Bm", Bb), ("Cm", Cb), ("dt", dtb)):
+        np.testing.assert_allclose(got_b[k], v, rtol=2.0 ** -7, atol=1e-12)
+    want_b = _fwd(lib, dict(case, dt=dtb, Bm=Bb, Cm=Cb))
+    np.testing.assert_allclose(got_b["y"], want_b["y"], rtol=1e-6, atol=1e-9)
 
 
 ALL_PINS = [

@@ -20,7 +20,7 @@ from mamba_selective_scan_core_b200 import build as mmbuild
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "mamba_mixer.h")
 
-OK, ENULL, ESHAPE, EALIGN, EDTYPE, EALIAS, EUNSUP, ECUDA, EDEVICE, EWORKSPACE, ESCRATCH = range(11)
+OK, ENULL, ESHAPE, EALIGN, EDTYPE, EALIAS, EUNSUP, ECUDA, EDEVICE, EWORKSPACE, ESCRATCH, ETIMEOUT, EARG = range(13)
 
 
 @pytest.fixture(scope="module")
@@ -59,8 +59,8 @@ def test_exported_symbols_are_c_linkage():
 
 def test_version_and_strings():
     mmbuild.build()
-    assert mm.abi_version() == 2
-    for code in range(12):
+    assert mm.abi_version() == 4
+    for code in range(13):
         s = mm.status_string(code)
         assert s and s != "unknown status"
     assert mm.status_string(99) == "unknown status"
@@ -214,6 +214,42 @@ def test_fwd_partial_overlap_is_alias(L):
     # y starting 16 bytes before the end of dt
     dt_bytes = 1 * 64 * 64 * 2
     assert call_fwd(L, y=base["dt"] + dt_bytes - 16) == EALIAS
+
+
+# ---------------------------------------------------------------- fused RMSNorm of B and C
+def normed_args(wb=None, wc=None, eps=1e-6, **kw):
+    a = fwd_args(**kw)
+    return a[:-3] + [wb, wc, eps] + a[-3:]
+
+
+NORM_W = BASE + (1 << 39)    # fake weight rows, clear of every buffer
+
+
+def test_normed_fwd_validation(L):
+    # valid: stops at the device check; no weight at all is the plain forward
+    assert L.mamba_mixer_fwd_normed(*normed_args(NORM_W, NORM_W + 256)) == EDEVICE
+    assert L.mamba_mixer_fwd_normed(*normed_args(None, None, eps=0.0)) == EDEVICE
+    # eps must be positive and finite once a weight is given
+    for eps in (0.0, -1.0, float("inf"), float("nan")):
+        assert L.mamba_mixer_fwd_normed(*normed_args(NORM_W, None, eps=eps)) == EARG
+        assert L.mamba_mixer_fwd_normed(*normed_args(None, NORM_W, eps=eps)) == EARG
+    assert L.mamba_mixer_fwd_normed(*normed_args(NORM_W + 4, None)) == EALIGN
+    # a weight under an output
+    y_addr = fwd_args()[11]
+    assert L.mamba_mixer_fwd_normed(*normed_args(y_addr, None)) == EALIAS
+    # the same argument checks as the plain forward come first
+    assert L.mamba_mixer_fwd_normed(*normed_args(NORM_W, None, xz=None)) == ENULL
+
+
+def test_normed_decode_validation(L):
+    def args(wb, wc, eps=1e-6, **kw):
+        a = upd_args(**kw)
+        return a[:-1] + [wb, wc, eps, a[-1]]
+
+    assert L.mamba_state_update_normed(*args(NORM_W, NORM_W + 4096)) == EDEVICE
+    assert L.mamba_state_update_normed(*args(NORM_W, None, eps=0.0)) == EARG
+    assert L.mamba_state_update_normed(*args(NORM_W + 8, None)) == EALIGN
+    assert L.mamba_state_update_normed(*args(upd_args()[12], None)) == EALIAS     # weight under y
 
 
 # ---------------------------------------------------------------- state_update validation

@@ -13,6 +13,8 @@ from .synth import (  # noqa: F401
     make_decode_inputs,
     make_mixer_inputs_custom,
     make_decode_inputs_custom,
+    make_norm_weights,
+    make_projection_weights,
     sample_channels,
     subset_channels,
 )

@@ -42,6 +42,7 @@ _BLOCK = 1 << 22  # elements per independently seeded block
 
 # fixed stream ids, one per tensor
 _T_XZ, _T_DT, _T_B, _T_C, _T_CONVW, _T_DTB, _T_D, _T_H0, _T_SSM, _T_CONVS, _T_X, _T_Z, _T_CONVB, _T_A = range(14)
+_T_BNORM, _T_CNORM, _T_WX, _T_WDT, _T_DTNORM = 14, 15, 16, 17, 18
 
 
 def _threads() -> int:
@@ -286,3 +287,26 @@ def subset_channels(inp: dict, chans) -> dict:
     for k in ("h0", "conv_state_in"):
         out[k] = inp[k].index_select(1, S) if inp.get(k) is not None else None
     return out
+
+
+def make_norm_weights(d_state: int = 16, layers=None, seed: int = 0):
+    """Per-state weights of the RMSNorm of B and C: U(0.5, 1.5) fp32, shape
+    [d_state] (forward) or [layers, d_state] (decode).  Returns (b_norm_w,
+    c_norm_w)."""
+    shape = (d_state,) if layers is None else (layers, d_state)
+    wb = _uniform(shape, seed, _T_BNORM, 0.5, 1.5)
+    wc = _uniform(shape, seed, _T_CNORM, 0.5, 1.5)
+    return torch.from_numpy(wb), torch.from_numpy(wc)
+
+
+def make_projection_weights(d_inner: int, dt_rank: int = 256, d_state: int = 16, seed: int = 0):
+    """Weights of the projections either side of the scan, bf16 (RNE):
+    W_x [dt_rank + 2 d_state, d_inner] ~ N(0, 1/d_inner) (so x_proj keeps the
+    scale of u), W_dt [d_inner, dt_rank] ~ N(0, 0.01/dt_rank) (so dt keeps the
+    workloads' 0.1 N(0, 1) scale for unit-rms dt_low), and the RMSNorm weight
+    of dt_low [dt_rank] ~ U(0.5, 1.5) fp32.  Returns (W_x, W_dt, dt_norm_w)."""
+    wx = _normal((dt_rank + 2 * d_state, d_inner), seed, _T_WX, std=1.0 / math.sqrt(d_inner))
+    wdt = _normal((d_inner, dt_rank), seed, _T_WDT, std=0.1 / math.sqrt(dt_rank))
+    wn = _uniform((dt_rank,), seed, _T_DTNORM, 0.5, 1.5)
+    return _act(wx, "bf16"), _act(wdt, "bf16"), torch.from_numpy(wn)
+
