@@ -623,7 +623,8 @@ def run_projections(mm, args, world, hbm_peak, hbm_src, peaks):
     dtl = torch.randn((M, R), device="cuda", generator=g).to(torch.bfloat16)
     xdbl = torch.empty((M, R + 32), device="cuda")
     dt = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(max(mm.proj_matmul_workspace_size(M, R + 32, D), mm.proj_matmul_workspace_size(M, D, R)),
+                     dtype=torch.uint8, device="cuda")
 
     def leg(name, fn, flops, nbytes, ms):
         return {"ms_per_call": round(ms, 5), "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
@@ -635,8 +636,8 @@ def run_projections(mm, args, world, hbm_peak, hbm_src, peaks):
     ms_x = _time_loop(lambda: mm.proj_matmul(u, W_x, out=xdbl, workspace=ws), K, world)
     ms_d = _time_loop(lambda: mm.proj_matmul(dtl, W_dt, out=dt, workspace=ws), K, world)
     out = {
-        "x_proj": leg(f"{M} x {R + 32} x {D}, bf16 -> fp32", None, 2.0 * M * (R + 32) * D,
-                      M * D * 2 + (R + 32) * D * 2 + M * (R + 32) * 4, ms_x),
+        "x_proj": leg(f"{M} x {R + 32} x {D}, bf16 -> fp32 (split-K: partials summed by a second kernel)", None,
+                      2.0 * M * (R + 32) * D, M * D * 2 + (R + 32) * D * 2 + M * (R + 32) * 4, ms_x),
         "dt_proj": leg(f"{M} x {D} x {R}, bf16 -> bf16", None, 2.0 * M * D * R, M * R * 2 + D * R * 2 + M * D * 2,
                        ms_d),
     }
@@ -783,15 +784,17 @@ def run_only(args):
         M, D, R = cfg.batch * cfg.seqlen, cfg.d_inner, 256
         W_x, W_dt, _ = (t.cuda() for t in make_projection_weights(D, R, seed=cfg.seed))
         g = torch.Generator(device="cuda").manual_seed(7)
-        ws = torch.empty(256, dtype=torch.uint8, device="cuda")
         if args.only == "xproj":
-            a = torch.randn((M, D), device="cuda", generator=g).to(torch.bfloat16)
+            lhs = torch.randn((M, D), device="cuda", generator=g).to(torch.bfloat16)
             o = torch.empty((M, R + 32), device="cuda")
-            step = lambda: mm.proj_matmul(a, W_x, out=o, workspace=ws)  # noqa: E731
+            wmat = W_x
         else:
-            a = torch.randn((M, R), device="cuda", generator=g).to(torch.bfloat16)
+            lhs = torch.randn((M, R), device="cuda", generator=g).to(torch.bfloat16)
             o = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
-            step = lambda: mm.proj_matmul(a, W_dt, out=o, workspace=ws)  # noqa: E731
+            wmat = W_dt
+        ws = torch.empty(mm.proj_matmul_workspace_size(M, wmat.shape[0], lhs.shape[1]), dtype=torch.uint8,
+                         device="cuda")
+        step = lambda: mm.proj_matmul(lhs, wmat, out=o, workspace=ws)  # noqa: E731
     elif args.only == "forward":
         cfg = PREFILL
         d = {k: (v.cuda() if v is not None else None)

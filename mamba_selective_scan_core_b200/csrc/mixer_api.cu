@@ -1099,13 +1099,13 @@ bool encode_gemm_2d(CUtensorMap* m, const void* base, int64_t cols, int64_t rows
 // (x_proj's 288 = 2 x 144), else 256-column tiles.
 int gemm_bn(int64_t N) { return N <= 64 ? 64 : N <= 128 ? 128 : (N <= 144 || N == 288) ? 144 : 256; }
 
-template <int BN, int STAGES, bool OUT_BF16>
+template <int BN, int NSUB, int STAGES, bool OUT_BF16>
 cudaError_t launch_gemm_t(const mm::GemmParams& gp, const void* A, const void* W, int ksplit, cudaStream_t s) {
     CUtensorMap ta, tw;
     if (!encode_gemm_2d(&ta, A, gp.K, gp.M, mm::kGemmBM) || !encode_gemm_2d(&tw, W, gp.K, gp.N, BN))
         return cudaErrorInvalidValue;
-    auto kern = mm::proj_gemm_kernel<BN, STAGES, OUT_BF16>;
-    const int smem = mm::GemmLayout<BN>::smem_bytes(STAGES);
+    auto kern = mm::proj_gemm_kernel<BN, NSUB, STAGES, OUT_BF16>;
+    const int smem = mm::GemmLayout<BN, NSUB>::smem_bytes(STAGES);
     static std::atomic<unsigned long long> smem_allowed{0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return cudaGetLastError();
@@ -1116,20 +1116,45 @@ cudaError_t launch_gemm_t(const mm::GemmParams& gp, const void* A, const void* W
         if (bit) smem_allowed.fetch_or(bit);
     }
     const dim3 grid(static_cast<unsigned>((gp.M + mm::kGemmBM - 1) / mm::kGemmBM),
-                    static_cast<unsigned>((gp.N + BN - 1) / BN), static_cast<unsigned>(ksplit));
+                    static_cast<unsigned>((gp.N + BN * NSUB - 1) / (BN * NSUB)), static_cast<unsigned>(ksplit));
     kern<<<grid, mm::kGemmThreads, forced_launch_failure() ? (1 << 20) : smem, s>>>(gp, ta, tw);
     return cudaGetLastError();
 }
 
+// Shapes: up to 128 outputs, one sub-tile; 288 (x_proj), two 144-wide
+// sub-tiles sharing each A tile; otherwise 256-wide tiles.  A product with
+// few K tiles per CTA (dt_proj: 4) takes a 2-deep ring, so two CTAs share an
+// SM and one's epilogue overlaps the other's copies and MMAs.
 template <bool OUT_BF16>
 cudaError_t launch_gemm(mm::GemmParams gp, const void* A, const void* W, int ksplit, cudaStream_t s) {
+    const bool short_k = gp.k_tiles_per_split <= 4;
     switch (gemm_bn(gp.N)) {
-        case 64: return launch_gemm_t<64, 8, OUT_BF16>(gp, A, W, ksplit, s);
-        case 128: return launch_gemm_t<128, 6, OUT_BF16>(gp, A, W, ksplit, s);
-        case 144: return launch_gemm_t<144, 6, OUT_BF16>(gp, A, W, ksplit, s);
-        default: return launch_gemm_t<256, 4, OUT_BF16>(gp, A, W, ksplit, s);
+        case 64: return launch_gemm_t<64, 1, 8, OUT_BF16>(gp, A, W, ksplit, s);
+        case 128: return launch_gemm_t<128, 1, 6, OUT_BF16>(gp, A, W, ksplit, s);
+        case 144: return gp.N > 144 ? launch_gemm_t<144, 2, 4, OUT_BF16>(gp, A, W, ksplit, s)
+                                    : launch_gemm_t<144, 1, 6, OUT_BF16>(gp, A, W, ksplit, s);
+        default: return short_k ? launch_gemm_t<256, 1, 2, OUT_BF16>(gp, A, W, ksplit, s)
+                                : launch_gemm_t<256, 1, 4, OUT_BF16>(gp, A, W, ksplit, s);
     }
 }
+
+// Split of K for a product: until the grid covers the SMs once (its CTAs each
+// fill an SM's shared memory with their ring), at most 16 ways and at least
+// 8 K tiles per CTA.
+int gemm_ksplit(int64_t M, int64_t N, int64_t K, int sms) {
+    const int64_t m_tiles = (M + mm::kGemmBM - 1) / mm::kGemmBM;
+    const int bn = gemm_bn(N);
+    const int64_t n_groups = N == 288 ? 1 : (N + bn - 1) / bn;
+    const int64_t k_tiles = (K + mm::kGemmBK - 1) / mm::kGemmBK;
+    const int64_t split = std::max<int64_t>(1, sms / std::max<int64_t>(1, m_tiles * n_groups));
+    return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({split, k_tiles / 8, 16})));
+}
+
+size_t matmul_ws_bytes(int64_t M, int64_t N, int64_t K, int sms) {
+    const int ks = gemm_ksplit(M, N, K, sms);
+    return kWsHeader + (ks > 1 ? align256(static_cast<size_t>(ks) * M * N * 4) : 0);
+}
+
 
 // Plan of the mixer with its projections: regions of its workspace (each
 // 256-byte aligned; the scan's own workspace first, so mamba_check_status
@@ -1148,12 +1173,7 @@ ProjPlan plan_projected(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t 
     pp.M = batch * seqlen;
     pp.R = static_cast<int>(dt_rank);
     pp.NC = pp.R + 32;
-    const int64_t m_tiles = (pp.M + mm::kGemmBM - 1) / mm::kGemmBM;
-    const int64_t n_tiles = (pp.NC + gemm_bn(pp.NC) - 1) / gemm_bn(pp.NC);
-    const int64_t k_tiles = (d_inner + mm::kGemmBK - 1) / mm::kGemmBK;
-    // split K until the x_proj grid covers the SMs once (one CTA per SM: its ring fills shared memory)
-    int64_t split = std::max<int64_t>(1, sms / std::max<int64_t>(1, m_tiles * n_tiles));
-    pp.ksplit = static_cast<int>(std::min<int64_t>({split, k_tiles, 16}));
+    pp.ksplit = gemm_ksplit(pp.M, pp.NC, d_inner, sms);
     const size_t M = static_cast<size_t>(pp.M), D = static_cast<size_t>(d_inner);
     pp.off_u = align256(pp.scan.ws_bytes);
     pp.off_part = pp.off_u + align256(M * D * 2);
@@ -1180,7 +1200,7 @@ extern "C" {
 size_t mamba_proj_matmul_workspace_size(int64_t M, int64_t N, int64_t K) {
     if (M <= 0 || N <= 0 || K <= 0 || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
         return 0;
-    return kWsHeader;
+    return matmul_ws_bytes(M, N, K, plan_sms());
 }
 
 mm_status mamba_proj_matmul(const void* A, const void* W, void* out, int64_t M, int64_t N, int64_t K,
@@ -1196,9 +1216,11 @@ mm_status mamba_proj_matmul(const void* A, const void* W, void* out, int64_t M, 
     const int64_t es = out_dtype == MM_F32 ? 4 : 2;
     const Span a = span(A, M * K * 2), w = span(W, N * K * 2), o = span(out, M * N * es);
     if (overlaps(o, a) || overlaps(o, w)) return MM_ERR_ALIAS;
-    if (!workspace || workspace_bytes < kWsHeader) return MM_ERR_WORKSPACE;
+    const int sms = plan_sms();
+    const size_t need = matmul_ws_bytes(M, N, K, sms);
+    if (!workspace || workspace_bytes < need) return MM_ERR_WORKSPACE;
     if (!aligned16(workspace)) return MM_ERR_ALIGN;
-    const Span ws = span(workspace, kWsHeader);
+    const Span ws = span(workspace, static_cast<int64_t>(need));
     if (overlaps(ws, a) || overlaps(ws, w) || overlaps(ws, o)) return MM_ERR_ALIAS;
     if (mm_status st = check_device(); st != MM_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -1209,18 +1231,31 @@ mm_status mamba_proj_matmul(const void* A, const void* W, void* out, int64_t M, 
         cudaGetLastError();
         return MM_ERR_CUDA;
     }
+    // a tall, narrow product is split in K: fp32 partials in the workspace,
+    // then summed into `out`
+    const int ks = gemm_ksplit(M, N, K, sms);
+    float* part = ks > 1 ? reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + kWsHeader) : nullptr;
+    const int k_tiles = static_cast<int>((K + mm::kGemmBK - 1) / mm::kGemmBK);
     mm::GemmParams gp{};
-    gp.out = out;
+    gp.out = ks > 1 ? static_cast<void*>(part) : out;
     gp.ldo = N;
-    gp.split_stride = 0;
+    gp.split_stride = M * N;
     gp.M = static_cast<int>(M);
     gp.N = static_cast<int>(N);
     gp.K = static_cast<int>(K);
-    gp.k_tiles_per_split = static_cast<int>((K + mm::kGemmBK - 1) / mm::kGemmBK);
+    gp.k_tiles_per_split = (k_tiles + ks - 1) / ks;
     gp.wait_limit = copy_wait_limit();
     gp.status = hdr;
     gp.status_epoch = epoch;
-    const cudaError_t e = out_dtype == MM_BF16 ? launch_gemm<true>(gp, A, W, 1, s) : launch_gemm<false>(gp, A, W, 1, s);
+    cudaError_t e = (out_dtype == MM_BF16 && ks == 1) ? launch_gemm<true>(gp, A, W, 1, s)
+                                                       : launch_gemm<false>(gp, A, W, ks, s);
+    if (e == cudaSuccess && ks > 1) {
+        const int64_t n = M * N;
+        const unsigned blocks = static_cast<unsigned>((n / 4 + 255) / 256);
+        if (out_dtype == MM_BF16) mm::splitk_reduce_kernel<true><<<blocks, 256, 0, s>>>(part, ks, n, out);
+        else mm::splitk_reduce_kernel<false><<<blocks, 256, 0, s>>>(part, ks, n, out);
+        e = cudaGetLastError();
+    }
     if (e != cudaSuccess) { cudaGetLastError(); return MM_ERR_CUDA; }
     return MM_OK;
 }

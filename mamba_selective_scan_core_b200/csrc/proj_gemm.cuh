@@ -8,8 +8,10 @@
 // with fp32 accumulation: a weight stored one row per output feature, as a
 // projection's weight is.
 //
-// One CTA computes a 128 x BN tile of `out` over a range of K (split-K gives
-// tall, narrow products such as x_proj -- 4096 x 288 x 8192 -- enough CTAs):
+// One CTA computes NSUB adjacent 128 x BN tiles of `out` over a range of K
+// (NSUB = 2 lets x_proj's 288 outputs, 2 x 144, share each tile of A, which
+// is then read once; split-K gives tall, narrow products such as x_proj --
+// 4096 x 288 x 8192 -- enough CTAs):
 //   * warp 0 (one elected lane) streams 128 x 64 tiles of A and BN x 64 tiles
 //     of W into a STAGES-deep shared-memory ring with 2-D tensor copies (TMA,
 //     128-byte swizzle, no multicast);
@@ -126,24 +128,26 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
-template <int BN>
+template <int BN, int NSUB = 1>
 struct GemmLayout {
     static constexpr int a_bytes = kGemmBM * kGemmBK * 2;       // 16 KB, a multiple of 1024
-    static constexpr int b_bytes = BN * kGemmBK * 2;            // BN x 128 B
-    static constexpr int stage_bytes = a_bytes + b_bytes;
-    static constexpr int tmem_cols = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
+    static constexpr int b_bytes = BN * kGemmBK * 2;            // BN x 128 B per sub-tile
+    static constexpr int stage_bytes = a_bytes + NSUB * b_bytes;
+    static constexpr int acc_cols = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;   // per sub-tile
+    static constexpr int tmem_cols = NSUB * acc_cols;
     // ring, then full[STAGES], empty[STAGES], acc barrier and the tensor-memory address
     static constexpr int smem_bytes(int stages) { return 1024 + stages * stage_bytes + (2 * stages + 2) * 8 + 16; }
 };
 
 // OUT_BF16: write bf16 rows (no split-K); else fp32 split-K partials.
-template <int BN, int STAGES, bool OUT_BF16>
+template <int BN, int NSUB, int STAGES, bool OUT_BF16>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 proj_gemm_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w)
 {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 N for M = 128");
     static_assert(GemmLayout<BN>::b_bytes % 1024 == 0, "ring slots stay 1024-byte aligned");
-    using Lay = GemmLayout<BN>;
+    static_assert(NSUB == 1 || NSUB == 2, "one or two sub-tiles");
+    using Lay = GemmLayout<BN, NSUB>;
     extern __shared__ __align__(1024) unsigned char gsm_raw[];
     // the swizzled tiles must start on 1024-byte boundaries
     unsigned char* gsm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~uintptr_t(1023));
@@ -155,7 +159,7 @@ proj_gemm_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tm_a, c
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int m0 = blockIdx.x * kGemmBM;
-    const int n0 = blockIdx.y * BN;
+    const int n0 = blockIdx.y * BN * NSUB;
     const int kt0 = blockIdx.z * p.k_tiles_per_split;
     const int k_tiles_total = (p.K + kGemmBK - 1) / kGemmBK;
     const int nkt = max(0, min(p.k_tiles_per_split, k_tiles_total - kt0));
@@ -195,7 +199,9 @@ proj_gemm_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tm_a, c
                 mbar_arrive_expect_tx(&full[s], tx_bytes);
                 const int kc = (kt0 + k) * kGemmBK;
                 tma_load_2d(st, &tm_a, kc, m0, &full[s]);
-                tma_load_2d(st + Lay::a_bytes, &tm_w, kc, n0, &full[s]);
+#pragma unroll
+                for (int j = 0; j < NSUB; ++j)
+                    tma_load_2d(st + Lay::a_bytes + j * Lay::b_bytes, &tm_w, kc, n0 + j * BN, &full[s]);
                 ++issued;
             }
         }
@@ -212,8 +218,11 @@ proj_gemm_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tm_a, c
                 const uint32_t b_base = a_base + Lay::a_bytes;
 #pragma unroll
                 for (int kk = 0; kk < kGemmBK / 16; ++kk)
-                    umma_bf16(tmem, umma_desc_sw128(a_base + kk * 32), umma_desc_sw128(b_base + kk * 32), idesc,
-                              (k > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int j = 0; j < NSUB; ++j)
+                        umma_bf16(tmem + j * Lay::acc_cols, umma_desc_sw128(a_base + kk * 32),
+                                  umma_desc_sw128(b_base + j * Lay::b_bytes + kk * 32), idesc,
+                                  (k > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(&empty[s]);
             }
             // the accumulator is complete once every MMA issued above has finished
@@ -235,10 +244,16 @@ proj_gemm_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tm_a, c
     if (all_ok && acc_ready) {
         const int row = m0 + warp * 32 + (tid & 31);
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        // sub-tile j's accumulator sits at column j * acc_cols; its BN columns
+        // are read in chunks of 32 (the last one partial when BN is not a
+        // multiple of 32) and written at output column n0 + j * BN + c0
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 32) {
+        for (int jc = 0; jc < NSUB * ((BN + 31) / 32); ++jc) {
+            const int j = jc / ((BN + 31) / 32);
+            const int c0 = (jc - j * ((BN + 31) / 32)) * 32;
+            const int nb = n0 + j * BN;      // first output column of this sub-tile
             float v[32];
-            tmem_ld32(lane_base + c0, v);
+            tmem_ld32(lane_base + j * Lay::acc_cols + c0, v);
             if (nkt == 0) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = 0.0f;
@@ -246,10 +261,10 @@ proj_gemm_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tm_a, c
             if (row < p.M) {
                 // columns of this chunk inside both the tile (BN need not be a
                 // multiple of 32) and the matrix
-                const int ncol = min(min(32, BN - c0), p.N - (n0 + c0));
+                const int ncol = min(min(32, BN - c0), p.N - (nb + c0));
                 if (ncol > 0) {
                     if constexpr (OUT_BF16) {
-                        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row) * p.ldo + n0 + c0;
+                        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row) * p.ldo + nb + c0;
                         if (ncol == 32) {
 #pragma unroll
                             for (int i = 0; i < 32; i += 8) {
@@ -267,7 +282,7 @@ proj_gemm_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tm_a, c
                         }
                     } else {
                         float* o = static_cast<float*>(p.out) + blockIdx.z * p.split_stride +
-                                   static_cast<int64_t>(row) * p.ldo + n0 + c0;
+                                   static_cast<int64_t>(row) * p.ldo + nb + c0;
                         if (ncol == 32) {
 #pragma unroll
                             for (int i = 0; i < 32; i += 4)

@@ -145,4 +145,27 @@ xproj_epilogue_kernel(const float* __restrict__ part, int splits, int64_t split_
     }
 }
 
+// Sum of `splits` fp32 partial products ([splits][n] floats, n a multiple of
+// 4) into fp32 or bf16 output: four elements per thread.
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(256)
+splitk_reduce_kernel(const float* __restrict__ part, int splits, int64_t n, void* __restrict__ out)
+{
+    const int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+    if (i >= n) return;
+    float4 acc = *reinterpret_cast<const float4*>(part + i);
+    for (int s = 1; s < splits; ++s) {
+        const float4 v = *reinterpret_cast<const float4*>(part + s * n + i);
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    if constexpr (OUT_BF16) {
+        uint2 w;
+        w.x = pack_bf16x2(acc.x, acc.y);
+        w.y = pack_bf16x2(acc.z, acc.w);
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out) + i) = w;
+    } else {
+        *reinterpret_cast<float4*>(static_cast<float*>(out) + i) = acc;
+    }
+}
+
 }  // namespace mm

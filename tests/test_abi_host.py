@@ -252,6 +252,50 @@ def test_normed_decode_validation(L):
     assert L.mamba_state_update_normed(*args(upd_args()[12], None)) == EALIAS     # weight under y
 
 
+# ---------------------------------------------------------------- projections
+def test_proj_matmul_validation(L):
+    A, W, O, WS = BASE, BASE + (1 << 33), BASE + (1 << 34), BASE + (1 << 35)
+    need = mm.proj_matmul_workspace_size(4096, 288, 8192)
+    # x_proj's shape splits K four ways on 148 SMs: fp32 partials after the status
+    assert need == 256 + 4 * 4096 * 288 * 4
+    assert mm.proj_matmul_workspace_size(256, 8192, 256) == 256
+    assert L.mamba_proj_matmul(A, W, O, 4096, 288, 8192, 1, WS, need, None) == EDEVICE
+    assert L.mamba_proj_matmul(A, W, O, 4096, 288, 8192, 1, WS, need - 16, None) == EWORKSPACE
+    assert L.mamba_proj_matmul(A, W, O, 64, 64, 64, 3, WS, 256, None) == EDTYPE
+    assert L.mamba_proj_matmul(A, W, O, 64, 64, 60, 0, WS, 256, None) == EUNSUP
+    assert L.mamba_proj_matmul(A, W, O, 64, 60, 64, 0, WS, 256, None) == EUNSUP
+    assert L.mamba_proj_matmul(A, W, O, -1, 64, 64, 0, WS, 256, None) == ESHAPE
+    assert L.mamba_proj_matmul(A, W, O, 0, 64, 64, 0, None, 0, None) == OK
+    assert L.mamba_proj_matmul(None, W, O, 64, 64, 64, 0, WS, 256, None) == ENULL
+    assert L.mamba_proj_matmul(A + 8, W, O, 64, 64, 64, 0, WS, 256, None) == EALIGN
+    assert L.mamba_proj_matmul(A, W, A, 64, 64, 64, 0, WS, 256, None) == EALIAS
+    assert L.mamba_proj_matmul(A, W, O, 64, 64, 64, 0, O, 256, None) == EALIAS
+
+
+def test_projected_validation(L):
+    a = fwd_args(B=1, Lq=64, D=64)
+    xz, conv_w, conv_b, dt_bias, A, Dskip = a[0], a[1], a[2], a[4], a[5], a[8]
+    y, h, cs = a[11], a[12], a[13]
+    WX, WDT, WS, NW = BASE + (1 << 33), BASE + (1 << 34), BASE + (1 << 35), BASE + (1 << 36)
+    need = mm.projected_workspace_size(1, 64, 64, 32)
+    assert need > 256
+
+    def call(act=1, R=32, D=64, eps=1e-6, wd=None, ws=WS, ws_bytes=None, **over):
+        return L.mamba_mixer_fwd_projected(over.get("xz", xz), conv_w, conv_b, WX, WDT, dt_bias, A, Dskip, None, None,
+                                           wd, None, None, eps, y, h, cs, 1, 64, D, 16, R, 4, act, ws,
+                                           need if ws_bytes is None else ws_bytes, None)
+
+    assert call() == EDEVICE
+    assert call(wd=NW) == EDEVICE
+    assert call(act=0) == EUNSUP
+    assert call(R=30) == EUNSUP
+    assert call(D=72) == EUNSUP
+    assert call(wd=NW, eps=0.0) == EARG
+    assert call(ws_bytes=need - 16) == EWORKSPACE
+    assert call(ws=xz) == EALIAS           # the workspace over an input
+    assert call(xz=None) == ENULL
+
+
 # ---------------------------------------------------------------- state_update validation
 def upd_args(NL=2, B=3, D=64, N=16, W=4, act=1, **over):
     es = 4 if act == 0 else 2

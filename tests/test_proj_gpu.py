@@ -10,7 +10,7 @@ import torch
 
 import mamba_selective_scan_core_b200 as mm
 import oracle
-from gpu_util import THREADS, assert_close, np64, to_dev
+from gpu_util import THREADS, _record as gpu_util_record, assert_close, gpu_fwd, np64, to_dev
 from workloads import CONFIGS, make_mixer_inputs, make_mixer_inputs_custom, make_norm_weights, \
     make_projection_weights
 
@@ -89,20 +89,32 @@ def check_projected(inp, R, norms, seed, chans=None):
     ref = oracle.projected_fwd(inp["xz"], inp["conv_w"], inp["conv_b"], W_x, W_dt, inp["dt_bias"], inp["A"],
                                inp["Dskip"], inp.get("h0"), inp.get("conv_state_in"), dt_norm_w=wd, b_norm_w=wb,
                                c_norm_w=wc, norm_eps=1e-6, store="bf16", threads=THREADS)
+    Bsz, L, _ = inp["xz"].shape
+    # 1. each stored intermediate within one bf16 rounding step of the oracle's
+    inter = mm.projected_intermediates(ws, Bsz, L, D, R)
+    for k in ("dt_low", "Bm", "Cm", "dt"):
+        assert_close(np64(inter[k]), ref[k], "bf16", k, stored_bf16=True, rounded_steps=1)
+    # 2. the chain's outputs are exactly the scan of those intermediates (the scan
+    #    itself is checked against the oracle by the parity tests)
+    y2, h2, cs2 = gpu_fwd(dict(dev, dt=inter["dt"].contiguous(), Bm=inter["Bm"].contiguous(),
+                               Cm=inter["Cm"].contiguous()))
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2) and torch.equal(h, h2) and torch.equal(cs, cs2)
+    np.testing.assert_array_equal(np64(cs), ref["conv_state_out"])
+    # 3. end to end against the oracle's chain: the rms bound of the bf16 path.  A
+    #    stored value that rounds one step differently moves y by up to 2^-7
+    #    |C_n h_n| at its token, which exceeds any budget in |y| where the terms
+    #    cancel, so the per-element check is the one of steps 1 and 2.
     got_y, got_h = np64(y), np64(h)
     ref_y, ref_h = ref["y"], ref["h_last"]
     if chans is not None:
         got_y, ref_y = got_y[..., chans], ref_y[..., chans]
         got_h, ref_h = got_h[:, chans], ref_h[:, chans]
-    # four stored intermediates reach y (u, B, C, dt) and three reach h (u, B, dt)
-    assert_close(got_y, ref_y, "bf16", "y", stored_bf16=True, rounded_steps=4)
-    assert_close(got_h, ref_h, "bf16", "h_last", rounded_steps=3)
-    np.testing.assert_array_equal(np64(cs), ref["conv_state_out"])
-    # the intermediates themselves, each within one rounding step of the oracle's
-    Bsz, L, _ = inp["xz"].shape
-    inter = mm.projected_intermediates(ws, Bsz, L, D, R)
-    for k in ("dt_low", "Bm", "Cm", "dt"):
-        assert_close(np64(inter[k]), ref[k], "bf16", k, stored_bf16=True, rounded_steps=1)
+    for got, want, name in ((got_y, ref_y, "y"), (got_h, ref_h, "h_last")):
+        rms = float(np.sqrt(np.mean(want ** 2)))
+        rerr = float(np.sqrt(np.mean((got - want) ** 2)))
+        gpu_util_record(name + " (rms)", got.size, rerr / (2e-2 * rms))
+        assert rerr <= 2e-2 * rms, (name, rerr, rms)
 
 
 @pytest.mark.parametrize("norms", [False, True])
