@@ -80,16 +80,26 @@ def _measured_peaks():
         return None
 
 
-def _kernel_source_sha():
-    """Hash of the CUDA sources (kernels and launch plan) the traffic figures
-    depend on, with comments and blank space stripped so that only code
-    changes invalidate a capture."""
+# The CUDA sources each traffic record depends on (its kernel, the shared
+# helpers and the launch code).
+TRAFFIC_SOURCES = {
+    "mixer_fwd/jamba_prefill": ("mixer_prefill.cuh", "mixer_common.cuh", "mixer_api.cu"),
+    "state_update_kernel/decode_28x128": ("mixer_decode.cuh", "mixer_common.cuh", "mixer_api.cu"),
+    "proj_gemm/x_proj": ("proj_gemm.cuh", "mixer_common.cuh", "mixer_api.cu"),
+    "proj_gemm/dt_proj": ("proj_gemm.cuh", "mixer_common.cuh", "mixer_api.cu"),
+}
+
+
+def _kernel_source_sha(names=None):
+    """Hash of the CUDA sources (kernels and launch plan) a traffic figure
+    depends on (all of csrc/ when `names` is None), with comments and blank
+    space stripped so that only code changes invalidate a capture."""
     import re
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mamba_selective_scan_core_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if not name.endswith((".cuh", ".cu")):
+        if not name.endswith((".cuh", ".cu")) or (names is not None and name not in names):
             continue
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
             src = f.read()
@@ -110,7 +120,7 @@ def _ncu_traffic(kernel_key):
             rec = json.load(f).get(kernel_key)
     except (OSError, ValueError):
         return None
-    if not rec or rec.get("source_sha") != _kernel_source_sha():
+    if not rec or rec.get("source_sha") != _kernel_source_sha(TRAFFIC_SOURCES.get(kernel_key)):
         return None
     return rec.get("bytes_per_launch")
 
@@ -626,20 +636,21 @@ def run_projections(mm, args, world, hbm_peak, hbm_src, peaks):
     ws = torch.empty(max(mm.proj_matmul_workspace_size(M, R + 32, D), mm.proj_matmul_workspace_size(M, D, R)),
                      dtype=torch.uint8, device="cuda")
 
-    def leg(name, fn, flops, nbytes, ms):
+    def leg(name, key, flops, nbytes, ms):
         return {"ms_per_call": round(ms, 5), "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
                 "roofline": {"bound": "tensor", "achieved": round(flops / (ms * 1e-3) / 1e12, 1), "peak": tpeak,
                              "unit": "TFLOP/s", "frac": round(flops / (ms * 1e-3) / 1e12 / tpeak, 4),
-                             "traffic": None, "peak_source": tsrc},
-                "hbm_gbs": round(nbytes / (ms * 1e-3) / 1e9, 1), "shape": name}
+                             "traffic": _ncu_traffic(key), "peak_source": tsrc},
+                "hbm_gbs": round(nbytes / (ms * 1e-3) / 1e9, 1), "algorithmic_bytes": nbytes, "shape": name}
 
     ms_x = _time_loop(lambda: mm.proj_matmul(u, W_x, out=xdbl, workspace=ws), K, world)
     ms_d = _time_loop(lambda: mm.proj_matmul(dtl, W_dt, out=dt, workspace=ws), K, world)
     out = {
-        "x_proj": leg(f"{M} x {R + 32} x {D}, bf16 -> fp32 (split-K: partials summed by a second kernel)", None,
+        "x_proj": leg(f"{M} x {R + 32} x {D}, bf16 -> fp32 (split-K: partials summed by a second kernel)",
+                      "proj_gemm/x_proj",
                       2.0 * M * (R + 32) * D, M * D * 2 + (R + 32) * D * 2 + M * (R + 32) * 4, ms_x),
-        "dt_proj": leg(f"{M} x {D} x {R}, bf16 -> bf16", None, 2.0 * M * D * R, M * R * 2 + D * R * 2 + M * D * 2,
-                       ms_d),
+        "dt_proj": leg(f"{M} x {D} x {R}, bf16 -> bf16", "proj_gemm/dt_proj", 2.0 * M * D * R,
+                       M * R * 2 + D * R * 2 + M * D * 2, ms_d),
     }
     del u, dtl, xdbl, dt
     host = make_mixer_inputs(cfg)
