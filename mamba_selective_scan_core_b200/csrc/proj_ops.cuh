@@ -58,29 +58,39 @@ conv_silu_kernel(const __nv_bfloat16* __restrict__ xz, const float* __restrict__
     }
     const int64_t t_end = min(L, t0 + kConvTokens);
     __nv_bfloat16* urow = u + static_cast<int64_t>(b) * L * D + d0;
-    for (int64_t t = t0; t < t_end; ++t) {
-        const uint4 v = *reinterpret_cast<const uint4*>(xrow + t * 2 * D);
-        const uint32_t wds[4] = {v.x, v.y, v.z, v.w};
-        float o[8];
+    // four tokens per step: their rows of x are requested together, so four
+    // loads are in flight per thread instead of one
+    constexpr int kStep = 4;
+    for (int64_t tb = t0; tb < t_end; tb += kStep) {
+        uint4 xv[kStep];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const float x = __uint_as_float((c & 1) ? (wds[c >> 1] & 0xffff0000u) : (wds[c >> 1] << 16));
-            float pre = cb[c];
-            pre = fmaf(w[c][0], win[c][0], pre);
-            pre = fmaf(w[c][1], win[c][1], pre);
-            pre = fmaf(w[c][2], win[c][2], pre);
-            pre = fmaf(w[c][3], x, pre);
-            o[c] = MathFast::silu(pre);
-            win[c][0] = win[c][1];
-            win[c][1] = win[c][2];
-            win[c][2] = x;
+        for (int j = 0; j < kStep; ++j)
+            xv[j] = tb + j < t_end ? *reinterpret_cast<const uint4*>(xrow + (tb + j) * 2 * D) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int j = 0; j < kStep; ++j) {
+            if (tb + j >= t_end) break;
+            const uint32_t wds[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
+            float o[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float x = __uint_as_float((c & 1) ? (wds[c >> 1] & 0xffff0000u) : (wds[c >> 1] << 16));
+                float pre = cb[c];
+                pre = fmaf(w[c][0], win[c][0], pre);
+                pre = fmaf(w[c][1], win[c][1], pre);
+                pre = fmaf(w[c][2], win[c][2], pre);
+                pre = fmaf(w[c][3], x, pre);
+                o[c] = MathFast::silu(pre);
+                win[c][0] = win[c][1];
+                win[c][1] = win[c][2];
+                win[c][2] = x;
+            }
+            uint4 r;
+            r.x = pack_bf16x2(o[0], o[1]);
+            r.y = pack_bf16x2(o[2], o[3]);
+            r.z = pack_bf16x2(o[4], o[5]);
+            r.w = pack_bf16x2(o[6], o[7]);
+            *reinterpret_cast<uint4*>(urow + (tb + j) * D) = r;
         }
-        uint4 r;
-        r.x = pack_bf16x2(o[0], o[1]);
-        r.y = pack_bf16x2(o[2], o[3]);
-        r.z = pack_bf16x2(o[4], o[5]);
-        r.w = pack_bf16x2(o[6], o[7]);
-        *reinterpret_cast<uint4*>(urow + t * D) = r;
     }
 }
 
