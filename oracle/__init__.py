@@ -58,6 +58,8 @@ def _declare(lib):
     lib.oracle_rmsnorm_rows.argtypes = [P, P, ctypes.c_double, P, I, I]
     lib.oracle_matmul_nt.restype = ctypes.c_int
     lib.oracle_matmul_nt.argtypes = [P, P, P, I, I, I, I, I]
+    lib.oracle_ssd_fwd.restype = ctypes.c_int
+    lib.oracle_ssd_fwd.argtypes = [P] * 11 + [I] * 8
     return lib
 
 
@@ -286,3 +288,34 @@ def projected_fwd(xz, conv_w, conv_b, W_x, W_dt, dt_bias, A, Dskip, h0=None, con
     out.update(u=u, dt_low=dt_low, Bm=Bm, Cm=Cm, dt=dt)
     return out
 
+
+
+def ssd_fwd(x, z, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, headdim: int = 64, threads: int = 1, library=None):
+    """Run the oracle of the Mamba-2 form (scalar-times-identity state matrix
+    per head, oracle_ssd_fwd).  x, z [B,L,H*P] (z None: no gate), dt [B,L,H],
+    dt_bias [H] or None, A [H], Bm, Cm [B,L,G,N], Dskip [H] or None, h0
+    [B,H,P,N] or None, P = headdim.  Returns y [B,L,H*P] and h_last [B,H,P,N]
+    as float64 arrays."""
+    L_ = library or lib()
+    x, z, dt, dt_bias, A, Bm, Cm, Dskip, h0 = map(_f64, (x, z, dt, dt_bias, A, Bm, Cm, Dskip, h0))
+    Bsz, L, C = x.shape
+    H = A.shape[0]
+    P = int(headdim)
+    G, N = Bm.shape[2], Bm.shape[3]
+    assert C == H * P and dt.shape == (Bsz, L, H) and Bm.shape == (Bsz, L, G, N) and Cm.shape == Bm.shape
+    y = np.zeros((Bsz, L, C))
+    h_last = np.zeros((Bsz, H, P, N))
+
+    def run(rng):
+        rc = L_.oracle_ssd_fwd(_p(x), _p(z), _p(dt), _p(dt_bias), _p(A), _p(Bm), _p(Cm), _p(Dskip), _p(h0),
+                               _p(y), _p(h_last), Bsz, L, H, P, N, G, rng[0], rng[1])
+        if rc != 0:
+            raise ValueError(f"oracle_ssd_fwd rejected its arguments (rc={rc})")
+
+    parts = _ranges(C, threads)
+    if len(parts) == 1:
+        run(parts[0])
+    else:
+        with ThreadPoolExecutor(max_workers=len(parts)) as ex:
+            list(ex.map(run, parts))
+    return {"y": y, "h_last": h_last}

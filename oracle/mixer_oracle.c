@@ -38,6 +38,11 @@
  *
  * Inputs are the exact values the GPU receives, widened to double; outputs
  * stay unrounded in double.
+ *
+ * Functions: oracle_mixer_fwd (the forward above), oracle_state_update (its
+ * one-token decode step), oracle_rmsnorm_rows (the RMSNorm of B_t and C_t),
+ * oracle_matmul_nt (the projections either side of the scan) and
+ * oracle_ssd_fwd (the Mamba-2 form: one scalar decay per head, grouped B/C).
  */
 #include <math.h>
 #include <stdint.h>
@@ -241,3 +246,72 @@ int oracle_matmul_nt(const double* A, const double* Bw, double* C, int64_t M, in
     return OR_OK;
 }
 
+
+/*
+ * Mamba-2 form of the selective scan (the variant the lesson's "SSM in one
+ * page" section says simplified the state matrix, and its "Mamba-3" section
+ * says discretised with Euler's rule).  The state matrix of each head is a
+ * scalar times the identity, so one decay per head and token multiplies the
+ * whole state; B_t and C_t are shared by the heads of a group:
+ *
+ *     Delta_t  = softplus(dt_t[h] + dt_bias[h])
+ *     h_t[p,n] = exp(Delta_t A[h]) h_{t-1}[p,n] + Delta_t B_t[g,n] x_t[h,p]
+ *     y_t[h,p] = (sum_n C_t[g,n] h_t[p,n] + D[h] x_t[h,p]) * SiLU(z_t[h,p])
+ *
+ * with g = h / (H / G) (heads split into G equal, consecutive groups) and the
+ * gate left out when z is NULL.  x is the layer's input after its
+ * convolution; channel c = h * P + p.
+ *
+ *   x, z          [B, L, H*P]  (z may be NULL: no gate)
+ *   dt            [B, L, H]    pre-bias step input; dt_bias [H] or NULL (= 0)
+ *   A             [H]          negative
+ *   Bm, Cm        [B, L, G, N]
+ *   Dskip         [H] or NULL (= 0)
+ *   h0            [B, H, P, N] or NULL (= 0)
+ * Outputs (only channels c in [c_begin, c_end) are written):
+ *   y             [B, L, H*P]
+ *   h_last        [B, H, P, N]  state after token L-1
+ */
+int oracle_ssd_fwd(const double* x, const double* z, const double* dt, const double* dt_bias,
+                   const double* A, const double* Bm, const double* Cm, const double* Dskip,
+                   const double* h0, double* y, double* h_last,
+                   int64_t Bsz, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G,
+                   int64_t c_begin, int64_t c_end)
+{
+    if (Bsz < 0 || L < 0 || H < 1 || P < 1 || N < 1 || N > 256 || G < 1 || H % G != 0) return OR_ERR_ARG;
+    const int64_t C = H * P;
+    if (c_begin < 0 || c_end > C || c_begin > c_end) return OR_ERR_ARG;
+    if ((!x || !dt || !Bm || !Cm) && L > 0) return OR_ERR_ARG;
+    if (!A || !y || !h_last) return OR_ERR_ARG;
+
+    double s[256];
+    const int64_t heads_per_group = H / G;
+
+    for (int64_t b = 0; b < Bsz; ++b) {
+        for (int64_t c = c_begin; c < c_end; ++c) {
+            const int64_t h = c / P;
+            const int64_t g = h / heads_per_group;
+            for (int64_t n = 0; n < N; ++n)
+                s[n] = h0 ? h0[(b * C + c) * N + n] : 0.0;
+
+            for (int64_t t = 0; t < L; ++t) {
+                const int64_t row = b * L + t;
+                const double xv = x[row * C + c];
+                const double delta = or_softplus(dt[row * H + h] + (dt_bias ? dt_bias[h] : 0.0));
+                const double decay = exp(delta * A[h]);
+                const double* Bt = Bm + (row * G + g) * N;
+                const double* Ct = Cm + (row * G + g) * N;
+                double acc = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    s[n] = decay * s[n] + delta * Bt[n] * xv;
+                    acc += Ct[n] * s[n];
+                }
+                const double yv = acc + (Dskip ? Dskip[h] : 0.0) * xv;
+                y[row * C + c] = z ? yv * or_silu(z[row * C + c]) : yv;
+            }
+
+            for (int64_t n = 0; n < N; ++n) h_last[(b * C + c) * N + n] = s[n];
+        }
+    }
+    return OR_OK;
+}

@@ -479,7 +479,135 @@ def pin_projected_forward_wiring(lib):
     np.testing.assert_allclose(got_b["y"], want_b["y"], rtol=1e-6, atol=1e-9)
 
 
+# ---------------------------------------------------------------- Mamba-2 form
+def _ssd_case(rng, Bsz, L, H, P, N, G, *, z=True, h0=True, dskip=True, bias=True):
+    return dict(
+        x=rng.standard_normal((Bsz, L, H * P)),
+        z=rng.standard_normal((Bsz, L, H * P)) if z else None,
+        dt=0.4 * rng.standard_normal((Bsz, L, H)),
+        dt_bias=rng.uniform(-3.0, 0.5, H) if bias else None,
+        A=-np.exp(rng.uniform(np.log(0.2), np.log(4.0), H)),
+        Bm=rng.standard_normal((Bsz, L, G, N)),
+        Cm=rng.standard_normal((Bsz, L, G, N)),
+        Dskip=rng.normal(1.0, 0.3, H) if dskip else None,
+        h0=0.5 * rng.standard_normal((Bsz, H, P, N)) if h0 else None,
+    )
+
+
+def _ssd(lib, case, P, **kw):
+    return oracle.ssd_fwd(case["x"], case["z"], case["dt"], case["dt_bias"], case["A"], case["Bm"], case["Cm"],
+                          case["Dskip"], case["h0"], headdim=P, library=lib, **kw)
+
+
+def pin_ssd_quadratic_form(lib):
+    """The Mamba-2 form against its materialised (quadratic, attention-like)
+    form, built here with numpy on tiny inputs: with decays a_t = exp(Delta_t A)
+    of a scalar-times-identity state matrix,
+        y_i = sum_{j<=i} (C_i . B_j) (prod_{k=j+1..i} a_k) Delta_j x_j
+              + (prod_{k<=i} a_k) C_i . h0 + D x_i,   gated by SiLU(z),
+        h_last = sum_j (prod_{k>j} a_k) Delta_j B_j x_j^T + (prod_k a_k) h0,
+    softplus and SiLU through numpy's logaddexp and scipy's logistic."""
+    rng = np.random.default_rng(71)
+    Bsz, L, H, P, N, G = 2, 13, 4, 3, 5, 2
+    for z in (True, False):
+        case = _ssd_case(rng, Bsz, L, H, P, N, G, z=z)
+        got = _ssd(lib, case, P)
+        for b in range(Bsz):
+            for h in range(H):
+                g = h // (H // G)
+                delta = lib_softplus(case["dt"][b, :, h] + case["dt_bias"][h])
+                la = delta * case["A"][h]                     # log of each token's decay
+                cum = np.cumsum(la)
+                Bg, Cg = case["Bm"][b, :, g, :], case["Cm"][b, :, g, :]
+                seg = cum[:, None] - cum[None, :]             # sum_{k=j+1..i} la_k
+                Mq = np.where(np.tril(np.ones((L, L))) > 0, (Cg @ Bg.T) * np.exp(np.minimum(seg, 0.0)), 0.0)
+                xs = case["x"][b, :, h * P:(h + 1) * P]       # [L, P]
+                h0 = case["h0"][b, h]                         # [P, N]
+                y = Mq @ (delta[:, None] * xs) + np.exp(cum)[:, None] * (Cg @ h0.T) + case["Dskip"][h] * xs
+                if z:
+                    y = y * lib_silu(case["z"][b, :, h * P:(h + 1) * P])
+                np.testing.assert_allclose(got["y"][b, :, h * P:(h + 1) * P], y, rtol=1e-10, atol=1e-11)
+                w = np.exp(cum[-1] - cum) * delta             # weight of token j in the final state
+                hl = (w[:, None] * xs).T @ Bg + np.exp(cum[-1]) * h0
+                np.testing.assert_allclose(got["h_last"][b, h], hl, rtol=1e-10, atol=1e-11)
+
+
+def pin_ssd_first_order_iir(lib):
+    """One head, one channel, one state, constant step: the state is the
+    first-order filter h_t = a h_{t-1} + b_t, checked with scipy's lfilter
+    (initial condition from h0), and y_t = C_t h_t + D x_t with no gate."""
+    rng = np.random.default_rng(73)
+    L = 40
+    case = _ssd_case(rng, 1, L, 1, 1, 1, 1, z=False)
+    case["dt"] = np.full((1, L, 1), 0.3)
+    got = _ssd(lib, case, 1)
+    delta = lib_softplus(0.3 + case["dt_bias"][0])
+    a = np.exp(delta * case["A"][0])
+    drive = delta * case["Bm"][0, :, 0, 0] * case["x"][0, :, 0]
+    h0 = case["h0"][0, 0, 0, 0]
+    h, _ = scipy.signal.lfilter([1.0], [1.0, -a], drive, zi=[a * h0])
+    np.testing.assert_allclose(got["h_last"][0, 0, 0, 0], h[-1], rtol=1e-12, atol=1e-13)
+    y = case["Cm"][0, :, 0, 0] * h + case["Dskip"][0] * case["x"][0, :, 0]
+    np.testing.assert_allclose(got["y"][0, :, 0], y, rtol=1e-11, atol=1e-12)
+
+
+def pin_ssd_zero_input(lib):
+    """x = 0 and h0 = 0 give y = 0 and a zero final state, whatever dt, B, C, z."""
+    rng = np.random.default_rng(79)
+    case = _ssd_case(rng, 2, 9, 2, 3, 4, 1, h0=False)
+    case["x"] = np.zeros_like(case["x"])
+    got = _ssd(lib, case, 3)
+    assert np.all(got["y"] == 0.0) and np.all(got["h_last"] == 0.0)
+
+
+def pin_ssd_split_equals_unsplit(lib):
+    """Running a sequence as two calls, the first call's final state carried
+    into the second as h0, equals the single run exactly: the state is all the
+    history the recurrence needs."""
+    rng = np.random.default_rng(83)
+    P = 2
+    case = _ssd_case(rng, 2, 17, 4, P, 3, 2)
+    full = _ssd(lib, case, P)
+    cut = 6
+
+    def part(lo, hi, h0):
+        c = dict(case)
+        for k in ("x", "z", "dt", "Bm", "Cm"):
+            c[k] = case[k][:, lo:hi]
+        c["h0"] = h0
+        return _ssd(lib, c, P)
+
+    first = part(0, cut, case["h0"])
+    second = part(cut, 17, first["h_last"])
+    np.testing.assert_array_equal(np.concatenate([first["y"], second["y"]], axis=1), full["y"])
+    np.testing.assert_array_equal(second["h_last"], full["h_last"])
+
+
+def pin_ssd_group_mapping(lib):
+    """G groups split the H heads into G consecutive blocks: a 2-group run on
+    4 heads equals two 1-group runs, heads 0-1 on group 0's B/C and heads 2-3
+    on group 1's."""
+    rng = np.random.default_rng(89)
+    P = 2
+    case = _ssd_case(rng, 1, 11, 4, P, 3, 2)
+    got = _ssd(lib, case, P)
+    for g in range(2):
+        heads = slice(2 * g, 2 * g + 2)
+        chans = slice(2 * g * P, (2 * g + 2) * P)
+        sub = dict(x=case["x"][..., chans], z=case["z"][..., chans], dt=case["dt"][..., heads],
+                   dt_bias=case["dt_bias"][heads], A=case["A"][heads], Bm=case["Bm"][:, :, g:g + 1],
+                   Cm=case["Cm"][:, :, g:g + 1], Dskip=case["Dskip"][heads], h0=case["h0"][:, heads])
+        one = _ssd(lib, sub, P)
+        np.testing.assert_array_equal(got["y"][..., chans], one["y"])
+        np.testing.assert_array_equal(got["h_last"][:, heads], one["h_last"])
+
+
 ALL_PINS = [
+    pin_ssd_quadratic_form,
+    pin_ssd_first_order_iir,
+    pin_ssd_zero_input,
+    pin_ssd_split_equals_unsplit,
+    pin_ssd_group_mapping,
     pin_matmul_library,
     pin_matmul_selection,
     pin_projected_forward_wiring,

@@ -1,7 +1,8 @@
 """Plants plausible mistakes in copies of the oracle (on the CPU) and checks
 that each one makes at least one pin fail, so the pins really constrain every
 step of the oracle: conv, SiLU, softplus, discretisation, recurrence, readout,
-skip, gate, carried state, the decode step, the RMSNorm of B and C and the projection product."""
+skip, gate, carried state, the decode step, the RMSNorm of B and C, the projection product
+and the Mamba-2 form (scalar decay per head, grouped B/C)."""
 
 import os
 
@@ -61,6 +62,23 @@ MUTANTS = [
      "for (int64_t k = 0; k + 1 < K; ++k) acc += A[m * K + k] * Bw[n * K + k];"),
     ("matmul_no_accumulate", "acc += A[m * K + k] * Bw[n * K + k];", "acc = A[m * K + k] * Bw[n * K + k];"),
     ("matmul_row_of_A", "acc += A[m * K + k] * Bw[n * K + k];", "acc += A[n * K + k] * Bw[n * K + k];"),
+    ("ssd_A_sign", "const double decay = exp(delta * A[h]);", "const double decay = exp(-delta * A[h]);"),
+    ("ssd_decay_not_exp", "const double decay = exp(delta * A[h]);", "const double decay = 1.0 + delta * A[h];"),
+    ("ssd_no_delta_on_B", "s[n] = decay * s[n] + delta * Bt[n] * xv;", "s[n] = decay * s[n] + Bt[n] * xv;"),
+    ("ssd_readout_before_update", "s[n] = decay * s[n] + delta * Bt[n] * xv;\n                    acc += Ct[n] * s[n];",
+     "acc += Ct[n] * s[n];\n                    s[n] = decay * s[n] + delta * Bt[n] * xv;"),
+    ("ssd_C_as_B", "acc += Ct[n] * s[n];", "acc += Bt[n] * s[n];"),
+    ("ssd_group_interleaved", "const int64_t g = h / heads_per_group;", "const int64_t g = h % G;"),
+    ("ssd_skip_dropped", "const double yv = acc + (Dskip ? Dskip[h] : 0.0) * xv;", "const double yv = acc;"),
+    ("ssd_gate_by_z", "y[row * C + c] = z ? yv * or_silu(z[row * C + c]) : yv;",
+     "y[row * C + c] = z ? yv * z[row * C + c] : yv;"),
+    ("ssd_dt_bias_of_head0", "or_softplus(dt[row * H + h] + (dt_bias ? dt_bias[h] : 0.0))",
+     "or_softplus(dt[row * H + h] + (dt_bias ? dt_bias[0] : 0.0))"),
+    ("ssd_dt_of_channel", "or_softplus(dt[row * H + h] +", "or_softplus(dt[row * H + c % H] +"),
+    ("ssd_h0_ignored", "s[n] = h0 ? h0[(b * C + c) * N + n] : 0.0;", "s[n] = 0.0;"),
+    ("ssd_head_of_channel", "const int64_t h = c / P;", "const int64_t h = c % H;"),
+    ("ssd_h_last_not_written", "for (int64_t n = 0; n < N; ++n) h_last[(b * C + c) * N + n] = s[n];",
+     "for (int64_t n = 0; n < N; ++n) h_last[(b * C + c) * N + n] = 0.0;"),
 ]
 
 

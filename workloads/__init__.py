@@ -15,6 +15,10 @@ from .synth import (  # noqa: F401
     make_decode_inputs_custom,
     make_norm_weights,
     make_projection_weights,
+    SsdConfig,
+    SSD_CONFIGS,
+    make_ssd_inputs,
+    make_ssd_inputs_custom,
     sample_channels,
     subset_channels,
 )

@@ -43,6 +43,7 @@ _BLOCK = 1 << 22  # elements per independently seeded block
 # fixed stream ids, one per tensor
 _T_XZ, _T_DT, _T_B, _T_C, _T_CONVW, _T_DTB, _T_D, _T_H0, _T_SSM, _T_CONVS, _T_X, _T_Z, _T_CONVB, _T_A = range(14)
 _T_BNORM, _T_CNORM, _T_WX, _T_WDT, _T_DTNORM = 14, 15, 16, 17, 18
+_T_SSD_X, _T_SSD_Z, _T_SSD_DT, _T_SSD_B, _T_SSD_C, _T_SSD_DTB, _T_SSD_A, _T_SSD_D, _T_SSD_H0 = range(19, 28)
 
 
 def _threads() -> int:
@@ -170,6 +171,73 @@ CONFIGS = {
         "decode_28x128", layers=28, batch=128, d_inner=8192, seed=4,
         desc="one-token state update across 28 stacked Mamba layers, batch 128"),
 }
+
+
+@dataclass(frozen=True)
+class SsdConfig:
+    """A prefill of the Mamba-2 form: H heads of P channels (d_inner = H P),
+    one scalar decay per head and token, B_t/C_t of d_state entries per group."""
+    name: str
+    batch: int
+    seqlen: int
+    heads: int
+    headdim: int = 64
+    d_state: int = 128
+    groups: int = 1
+    seed: int = 0
+    h0_std: float = 0.0
+    gate: bool = True
+    desc: str = ""
+
+    @property
+    def d_inner(self) -> int:
+        return self.heads * self.headdim
+
+    @property
+    def tokens(self) -> int:
+        return self.batch * self.seqlen
+
+
+SSD_CONFIGS = {
+    "mamba2_prefill": SsdConfig(
+        "mamba2_prefill", batch=1, seqlen=4096, heads=128, seed=5,
+        desc="Mamba-2 form at the Jamba width: d_inner 8192 as 128 heads of 64, d_state 128, one B/C group"),
+    "mamba2_batched": SsdConfig(
+        "mamba2_batched", batch=4, seqlen=8192, heads=128, seed=6, h0_std=0.1,
+        desc="Mamba-2 form, 4 x 8192 tokens with an initial state"),
+}
+
+
+def make_ssd_inputs_custom(batch, seqlen, heads, headdim=64, d_state=128, groups=1, seed=0, h0_std=0.0,
+                           gate=True, dt_std=0.1):
+    """Seeded inputs of the Mamba-2 form as CPU torch tensors.
+
+    x, z [B,L,H*P] ~ N(0,1) (bf16; x is the layer's input after its
+    convolution; z None without the gate), dt [B,L,H] ~ dt_std N(0,1) (bf16),
+    Bm/Cm [B,L,G,N] ~ N(0,1) (bf16), per head dt_bias = inverse-softplus of a
+    log-uniform [1e-3, 1e-1] step, A = -exp(U(ln 1, ln 16)), D ~ N(1, 0.1)
+    (fp32), h0 [B,H,P,N] ~ h0_std N(0,1) fp32 or None."""
+    B, L, H, P, N, G = batch, seqlen, heads, headdim, d_state, groups
+    s = seed
+    out = {}
+    out["x"] = _act(_normal((B, L, H * P), s, _T_SSD_X), "bf16")
+    out["z"] = _act(_normal((B, L, H * P), s, _T_SSD_Z), "bf16") if gate else None
+    out["dt"] = _act(_normal((B, L, H), s, _T_SSD_DT, std=dt_std), "bf16")
+    out["Bm"] = _act(_normal((B, L, G, N), s, _T_SSD_B), "bf16")
+    out["Cm"] = _act(_normal((B, L, G, N), s, _T_SSD_C), "bf16")
+    out["dt_bias"] = torch.from_numpy(_dt_bias((H,), s, _T_SSD_DTB))
+    u = _uniform((H,), s, _T_SSD_A, 0.0, math.log(16.0))
+    out["A"] = torch.from_numpy((-np.exp(u.astype(np.float64))).astype(np.float32))
+    out["Dskip"] = torch.from_numpy(_normal((H,), s, _T_SSD_D, std=0.1, mean=1.0))
+    out["h0"] = torch.from_numpy(_normal((B, H, P, N), s, _T_SSD_H0, std=h0_std)) if h0_std > 0 else None
+    return out
+
+
+def make_ssd_inputs(cfg: SsdConfig, **overrides):
+    kw = dict(batch=cfg.batch, seqlen=cfg.seqlen, heads=cfg.heads, headdim=cfg.headdim, d_state=cfg.d_state,
+              groups=cfg.groups, seed=cfg.seed, h0_std=cfg.h0_std, gate=cfg.gate)
+    kw.update(overrides)
+    return make_ssd_inputs_custom(**kw)
 
 
 def make_mixer_inputs_custom(batch, seqlen, d_inner, d_state=16, d_conv=4, act="bf16", seed=0,
