@@ -405,13 +405,60 @@ size_t mamba_mixer_projected_workspace_size(int64_t batch, int64_t seqlen, int64
 mm_status mamba_mixer_projected_layout(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state,
                                        int64_t dt_rank, int64_t d_conv, size_t offsets[5]);
 
+/*
+ * The Mamba-2 form of the selective scan, prefill (bf16 activations, fp32
+ * state; the products run on the tensor cores).  The Jamba lesson's "SSM in
+ * one page" section: Mamba-2 simplified the state matrix -- to a scalar times
+ * the identity per head -- and its "Mamba-3" section: Mamba-2 discretises
+ * with Euler's rule.  For head h of H (P = headdim channels, c = h P + p),
+ * group g = h / (H / groups) and every token t:
+ *
+ *   Delta_t  = softplus(dt_t[h] + dt_bias[h])
+ *   s_t[p,n] = exp(Delta_t A[h]) s_{t-1}[p,n] + Delta_t B_t[g,n] x_t[c]
+ *   y_t[c]   = (sum_n C_t[g,n] s_t[p,n] + D[h] x_t[c]) * SiLU(z_t[c])   (no gate if z is NULL)
+ *
+ * computed chunk by chunk (128 tokens) as dense products -- the same sums,
+ * regrouped.  x is the layer's input after its convolution.
+ *
+ *   x, z           [batch, seqlen, heads*headdim]   bf16  (z may be NULL)
+ *   dt             [batch, seqlen, heads]           bf16  before dt_bias and softplus
+ *   dt_bias        [heads]                          fp32  or NULL (= 0)
+ *   A              [heads]                          fp32  negative
+ *   Bm, Cm         [batch, seqlen, groups, d_state] bf16
+ *   Dskip          [heads]                          fp32  or NULL (= 0)
+ *   h0             [batch, heads, headdim, d_state] fp32  or NULL (= 0)
+ *   y              [batch, seqlen, heads*headdim]   bf16  output
+ *   h_last         [batch, heads, headdim, d_state] fp32  output: the state after the last token
+ *
+ * Supported: headdim == 64, d_state == 128 (MM_ERR_UNSUPPORTED otherwise);
+ * heads a multiple of groups, both positive (MM_ERR_SHAPE).  Every pointer
+ * 16-byte aligned (MM_ERR_ALIGN); y and h_last may not overlap an input or
+ * each other (MM_ERR_ALIAS).  workspace: at least
+ * mamba_ssd_workspace_size(...) bytes, 16-byte aligned, overlapping no other
+ * argument; its first 256 bytes hold the call's status for
+ * mamba_check_status.  seqlen == 0 writes h_last = h0 (or zeros).  Runs on
+ * `stream`; the library allocates nothing.  Errors otherwise as
+ * mamba_mixer_fwd.
+ */
+mm_status mamba_ssd_fwd(const void* x, const void* z, const void* dt, const float* dt_bias, const float* A,
+                        const void* Bm, const void* Cm, const float* Dskip, const float* h0,
+                        void* y, float* h_last,
+                        int64_t batch, int64_t seqlen, int64_t heads, int64_t headdim, int64_t d_state,
+                        int64_t groups, void* workspace, size_t workspace_bytes, void* stream);
+/* Workspace bytes of mamba_ssd_fwd for these sizes (0 if they are not
+ * supported): the status header, the fp32 state each chunk adds from zero,
+ * the state entering each chunk (as two bf16 parts) and each chunk's total
+ * decay. */
+size_t mamba_ssd_workspace_size(int64_t batch, int64_t seqlen, int64_t heads, int64_t headdim, int64_t d_state,
+                                int64_t groups);
+
 /* A static, human-readable name for a status code. */
 const char* mamba_status_string(mm_status status);
 
 /* ABI version of this header (incremented on any signature change). */
 int mamba_mixer_abi_version(void);
 
-#define MAMBA_MIXER_ABI_VERSION 4
+#define MAMBA_MIXER_ABI_VERSION 5
 
 #ifdef __cplusplus
 }

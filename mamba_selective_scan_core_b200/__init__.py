@@ -17,7 +17,7 @@ __all__ = [
     "MM_F32", "MM_BF16", "MixerError", "lib", "library_path", "mixer_fwd", "mixer_fwd_noalloc", "mixer_fwd_host",
     "state_update", "workspace_size", "host_workspace_size", "status_string", "abi_version", "fault_status",
     "check_status", "proj_matmul", "proj_matmul_workspace_size", "mixer_fwd_projected",
-    "projected_workspace_size", "EXPORTED_SYMBOLS",
+    "projected_workspace_size", "ssd_fwd", "ssd_workspace_size", "EXPORTED_SYMBOLS",
 ]
 
 MM_F32 = 0
@@ -45,6 +45,8 @@ EXPORTED_SYMBOLS = (
     "mamba_mixer_fwd_projected",
     "mamba_mixer_projected_workspace_size",
     "mamba_mixer_projected_layout",
+    "mamba_ssd_fwd",
+    "mamba_ssd_workspace_size",
 )
 
 
@@ -99,6 +101,10 @@ def _declare(L):
     L.mamba_mixer_projected_workspace_size.argtypes = [I64] * 6 + [ctypes.c_int]
     L.mamba_mixer_projected_layout.restype = ctypes.c_int
     L.mamba_mixer_projected_layout.argtypes = [I64] * 6 + [P]
+    L.mamba_ssd_fwd.restype = ctypes.c_int
+    L.mamba_ssd_fwd.argtypes = [P] * 11 + [I64] * 6 + [P, ctypes.c_size_t, P]
+    L.mamba_ssd_workspace_size.restype = ctypes.c_size_t
+    L.mamba_ssd_workspace_size.argtypes = [I64] * 6
     return L
 
 
@@ -537,3 +543,57 @@ def mixer_fwd_projected(xz, conv_w, conv_b, W_x, W_dt, dt_bias, A, Dskip, h0=Non
     _keep_alive_on(made, (stream,))
     return y, h_last, conv_state_out
 
+
+
+def ssd_workspace_size(batch, seqlen, heads, headdim=64, d_state=128, groups=1) -> int:
+    return int(lib().mamba_ssd_workspace_size(batch, seqlen, heads, headdim, d_state, groups))
+
+
+def ssd_fwd(x, z, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, *, headdim=64, y=None, h_last=None, workspace=None,
+            stream=None):
+    """The Mamba-2 form of the scan (mamba_ssd_fwd): x, z [B,L,H*P] bf16 (z may
+    be None: no gate), dt [B,L,H] bf16, dt_bias/A/Dskip [H] fp32 (dt_bias and
+    Dskip may be None), Bm/Cm [B,L,G,N] bf16, h0 [B,H,P,N] fp32 or None, P =
+    headdim.  Returns (y [B,L,H*P] bf16, h_last [B,H,P,N] fp32), allocating any
+    output not given."""
+    import torch
+
+    bf, f32 = torch.bfloat16, torch.float32
+    Bsz, L, HP = x.shape
+    H = A.shape[0]
+    P = int(headdim)
+    G, N = Bm.shape[2], Bm.shape[3]
+    if HP != H * P:
+        raise ValueError(f"x has {HP} channels, expected heads x headdim = {H * P}")
+    dev = x.device
+    made = []
+    _check(x, "x", bf, (Bsz, L, H * P), dev)
+    _check(z, "z", bf, (Bsz, L, H * P), dev)
+    _check(dt, "dt", bf, (Bsz, L, H), dev)
+    _check(dt_bias, "dt_bias", f32, (H,), dev)
+    _check(A, "A", f32, (H,), dev)
+    _check(Bm, "Bm", bf, (Bsz, L, G, N), dev)
+    _check(Cm, "Cm", bf, (Bsz, L, G, N), dev)
+    _check(Dskip, "Dskip", f32, (H,), dev)
+    _check(h0, "h0", f32, (Bsz, H, P, N), dev)
+    if y is None:
+        y = torch.empty((Bsz, L, H * P), dtype=bf, device=dev)
+        made.append(y)
+    if h_last is None:
+        h_last = torch.empty((Bsz, H, P, N), dtype=f32, device=dev)
+        made.append(h_last)
+    _check(y, "y", bf, (Bsz, L, H * P), dev)
+    _check(h_last, "h_last", f32, (Bsz, H, P, N), dev)
+    ws_bytes = ssd_workspace_size(Bsz, L, H, P, N, G)
+    if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+        made.append(workspace)
+    with torch.cuda.device(dev):
+        st = lib().mamba_ssd_fwd(_ptr(x), _ptr(z), _ptr(dt), _ptr(dt_bias), _ptr(A), _ptr(Bm), _ptr(Cm),
+                                 _ptr(Dskip), _ptr(h0), _ptr(y), _ptr(h_last), Bsz, L, H, P, N, G,
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                 _stream_handle(stream))
+    if st != 0:
+        raise MixerError(st, "mamba_ssd_fwd")
+    _keep_alive_on(made, (stream,))
+    return y, h_last

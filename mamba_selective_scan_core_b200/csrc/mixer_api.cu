@@ -18,6 +18,7 @@
 #include "mixer_prefill.cuh"
 #include "proj_gemm.cuh"
 #include "proj_ops.cuh"
+#include "ssd.cuh"
 
 namespace {
 
@@ -1389,3 +1390,162 @@ mm_status mamba_mixer_fwd_projected(const void* xz, const float* conv_w, const f
 
 }  // extern "C"
 
+
+// ---------------------------------------------------------------- Mamba-2 form (tcgen05 chunked scan)
+namespace {
+
+// Workspace of mamba_ssd_fwd (every region 256-byte aligned):
+//   header [256 B]                        the call status
+//   S      [B][chunks][H][P][N] f32       chunk states from zero
+//   Hin    [2][B][chunks][H][P][N] bf16   state entering each chunk: hi parts, then lo parts
+//   dec    [B][H][chunks] f32             each chunk's total decay
+struct SsdPlan {
+    int64_t chunks = 0;
+    size_t off_s = 0, off_hin = 0, off_dec = 0, total = 0;
+};
+
+SsdPlan plan_ssd(int64_t batch, int64_t seqlen, int64_t heads) {
+    SsdPlan pl;
+    pl.chunks = (seqlen + mm::kSsdQ - 1) / mm::kSsdQ;
+    const size_t states = static_cast<size_t>(batch) * pl.chunks * heads * mm::kSsdP * mm::kSsdN;
+    pl.off_s = kWsHeader;
+    pl.off_hin = pl.off_s + align256(states * 4);
+    pl.off_dec = pl.off_hin + align256(states * 2 * 2);
+    pl.total = pl.off_dec + align256(static_cast<size_t>(batch) * heads * pl.chunks * 4);
+    return pl;
+}
+
+// Sizes the kernels address: grid y/z limits, 32-bit tensor-copy coordinates
+// (tokens, and rows of the [2 * B * chunks * H * P][N] state copies).
+bool ssd_sizes_ok(int64_t batch, int64_t seqlen, int64_t heads, int64_t groups) {
+    if (batch < 0 || seqlen < 0 || heads <= 0 || groups <= 0 || heads % groups != 0) return false;
+    if (batch > 65535 || heads > 65535 || seqlen >= (int64_t(1) << 31) - mm::kSsdQ) return false;
+    const int64_t chunks = (seqlen + mm::kSsdQ - 1) / mm::kSsdQ;
+    int64_t rows;
+    return mul_ok(batch * chunks, heads * mm::kSsdP, &rows) && 2 * rows < (int64_t(1) << 31) &&
+           seqlen * heads * mm::kSsdP * 2 < (int64_t(1) << 40);
+}
+
+// 3-D map over a bf16 [batch][rows][cols] tensor, [box_rows][64] boxes with
+// the 128-byte swizzle of the products' operand tiles.
+bool encode_sw128_3d(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int64_t batch, int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                                static_cast<cuuint64_t>(batch)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols * 2), static_cast<cuuint64_t>(rows * cols * 2)};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mamba_ssd_workspace_size(int64_t batch, int64_t seqlen, int64_t heads, int64_t headdim, int64_t d_state,
+                                int64_t groups) {
+    if (headdim != mm::kSsdP || d_state != mm::kSsdN || batch <= 0 || !ssd_sizes_ok(batch, seqlen, heads, groups))
+        return 0;
+    return plan_ssd(batch, seqlen, heads).total;
+}
+
+mm_status mamba_ssd_fwd(const void* x, const void* z, const void* dt, const float* dt_bias, const float* A,
+                        const void* Bm, const void* Cm, const float* Dskip, const float* h0,
+                        void* y, float* h_last,
+                        int64_t batch, int64_t seqlen, int64_t heads, int64_t headdim, int64_t d_state,
+                        int64_t groups, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (!ssd_sizes_ok(batch, seqlen, heads, groups)) return MM_ERR_SHAPE;
+    if (headdim != mm::kSsdP || d_state != mm::kSsdN) return MM_ERR_UNSUPPORTED;
+    if (batch == 0) return MM_OK;
+    const bool tokens = seqlen > 0;
+    if (!A || !h_last || (tokens && (!x || !dt || !Bm || !Cm || !y))) return MM_ERR_NULL;
+    for (const void* q : {x, z, dt, static_cast<const void*>(dt_bias), static_cast<const void*>(A), Bm, Cm,
+                          static_cast<const void*>(Dskip), static_cast<const void*>(h0), static_cast<const void*>(y),
+                          static_cast<const void*>(h_last)})
+        if (q && !aligned16(q)) return MM_ERR_ALIGN;
+    const int64_t C = heads * mm::kSsdP, NL = batch * seqlen;
+    const Span sx = span(x, NL * C * 2), sz = span(z, NL * C * 2), sdt = span(dt, NL * heads * 2),
+               sbias = span(dt_bias, heads * 4), sa = span(A, heads * 4), sb = span(Bm, NL * groups * mm::kSsdN * 2),
+               sc = span(Cm, NL * groups * mm::kSsdN * 2), sd = span(Dskip, heads * 4),
+               sh0 = span(h0, batch * C * mm::kSsdN * 4), sy = span(y, NL * C * 2),
+               shl = span(h_last, batch * C * mm::kSsdN * 4);
+    const Span ins[] = {sx, sz, sdt, sbias, sa, sb, sc, sd, sh0};
+    for (const Span& in : ins)
+        if (overlaps(sy, in) || overlaps(shl, in)) return MM_ERR_ALIAS;
+    if (overlaps(sy, shl)) return MM_ERR_ALIAS;
+    const SsdPlan pl = plan_ssd(batch, seqlen, heads);
+    if (!workspace || workspace_bytes < pl.total) return MM_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MM_ERR_ALIGN;
+    const Span sw = span(workspace, static_cast<int64_t>(pl.total));
+    for (const Span& in : ins)
+        if (overlaps(sw, in)) return MM_ERR_ALIAS;
+    if (overlaps(sw, sy) || overlaps(sw, shl)) return MM_ERR_ALIAS;
+    if (mm_status st = check_device(); st != MM_OK) return st;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned char* w = static_cast<unsigned char*>(workspace);
+    unsigned long long* hdr = reinterpret_cast<unsigned long long*>(w);
+    const unsigned long long epoch = next_call_id();
+    if (cudaMemcpyAsync(hdr + 1, &epoch, sizeof(epoch), cudaMemcpyHostToDevice, s) != cudaSuccess) {
+        cudaGetLastError();
+        return MM_ERR_CUDA;
+    }
+    mm::SsdParams p{};
+    p.x = static_cast<const __nv_bfloat16*>(x);
+    p.z = static_cast<const __nv_bfloat16*>(z);
+    p.dt = static_cast<const __nv_bfloat16*>(dt);
+    p.dt_bias = dt_bias;
+    p.A = A;
+    p.Bm = static_cast<const __nv_bfloat16*>(Bm);
+    p.Cm = static_cast<const __nv_bfloat16*>(Cm);
+    p.Dskip = Dskip;
+    p.h0 = h0;
+    p.y = static_cast<__nv_bfloat16*>(y);
+    p.h_last = h_last;
+    p.S = reinterpret_cast<float*>(w + pl.off_s);
+    p.Hin = reinterpret_cast<__nv_bfloat16*>(w + pl.off_hin);
+    p.hin_lo = batch * pl.chunks * heads * mm::kSsdP * mm::kSsdN;
+    p.dec = reinterpret_cast<float*>(w + pl.off_dec);
+    p.L = seqlen;
+    p.H = static_cast<int>(heads);
+    p.G = static_cast<int>(groups);
+    p.chunks = static_cast<int>(pl.chunks);
+    p.batch = static_cast<int>(batch);
+    p.wait_limit = copy_wait_limit();
+    p.status = hdr;
+    p.status_epoch = epoch;
+
+    const dim3 cgrid(static_cast<unsigned>(pl.chunks), static_cast<unsigned>(heads), static_cast<unsigned>(batch));
+    const bool fail = forced_launch_failure();
+    if (pl.chunks > 0) {
+        static std::atomic<unsigned long long> allowed_state{0};
+        if (allow_smem(mm::ssd_chunk_state_kernel, allowed_state) != cudaSuccess) { cudaGetLastError(); return MM_ERR_CUDA; }
+        mm::ssd_chunk_state_kernel<<<cgrid, mm::kSsdThreads,
+                                     fail ? (1 << 20) : mm::SsdStateLayout::smem_bytes, s>>>(p);
+        if (cudaGetLastError() != cudaSuccess) return MM_ERR_CUDA;
+    }
+    const int64_t quads = heads * mm::kSsdP * mm::kSsdN / 4;
+    mm::ssd_state_pass_kernel<<<dim3(static_cast<unsigned>((quads + 255) / 256), static_cast<unsigned>(batch)), 256, 0,
+                                s>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return MM_ERR_CUDA;
+    if (pl.chunks > 0) {
+        CUtensorMap tc, tb, th;
+        const int64_t gn = groups * mm::kSsdN;
+        if (!encode_sw128_3d(&tc, Cm, gn, seqlen, batch, mm::kSsdQ) ||
+            !encode_sw128_3d(&tb, Bm, gn, seqlen, batch, mm::kSsdQ) ||
+            !encode_sw128_3d(&th, p.Hin, mm::kSsdN, 2 * batch * pl.chunks * heads * mm::kSsdP, 1, mm::kSsdP))
+            return MM_ERR_CUDA;
+        static std::atomic<unsigned long long> allowed_scan{0};
+        if (allow_smem(mm::ssd_chunk_scan_kernel, allowed_scan) != cudaSuccess) { cudaGetLastError(); return MM_ERR_CUDA; }
+        mm::ssd_chunk_scan_kernel<<<cgrid, mm::kSsdThreads,
+                                    fail ? (1 << 20) : mm::SsdScanLayout::smem_bytes, s>>>(p, tc, tb, th);
+        if (cudaGetLastError() != cudaSuccess) return MM_ERR_CUDA;
+    }
+    return MM_OK;
+}
+
+}  // extern "C"

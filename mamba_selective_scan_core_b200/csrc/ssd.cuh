@@ -1,0 +1,534 @@
+// The Mamba-2 form of the selective scan on the fifth-generation tensor cores.
+//
+// The lesson's "SSM in one page" section: Mamba-2 simplified the state matrix
+// (to a scalar times the identity, per head), and its "Mamba-3" section:
+// Mamba-2 discretises with Euler's rule.  Per head h (P channels, state N x P),
+// with a_t = Delta_t A[h] and Delta_t = softplus(dt_t[h] + dt_bias[h]):
+//
+//     h_t = exp(a_t) h_{t-1} + Delta_t x_t B_t^T        (x_t: P, B_t: N)
+//     y_t = h_t C_t + D[h] x_t,   gated by SiLU(z_t)
+//
+// A scalar decay makes the recurrence over a chunk of Q tokens a sum of
+// dense products.  With cum_i = a_{t0} + ... + a_i (the chunk's inclusive
+// prefix sum) and H_in the state entering the chunk:
+//
+//     y_i   = sum_{j<=i} (C_i . B_j) exp(cum_i - cum_j) Delta_j x_j   (intra-chunk)
+//           + exp(cum_i) C_i H_in  +  D x_i                            (carried state)
+//     H_out = exp(cum_end) H_in + sum_j exp(cum_end - cum_j) Delta_j x_j B_j^T
+//
+// That is the same recurrence with its sums regrouped (exact up to rounding
+// order).  Three kernels, Q = 128 tokens per chunk:
+//
+//   ssd_chunk_state_kernel (chunk, head, batch): S_c = sum_j w_j B_j x_j^T
+//       with w_j = exp(cum_end - cum_j) Delta_j -- one tcgen05 product
+//       [N x Q] . [Q x P] -- and the chunk's total decay exp(cum_end);
+//   ssd_state_pass_kernel (state entries): H_in[c] = H (as hi and lo bf16
+//       parts), H = dec_c H + S_c over the chunks in order, from h0 (fp32);
+//       the last H is h_last;
+//   ssd_chunk_scan_kernel (chunk, head, batch): G = C B^T (tcgen05), the
+//       masked, decayed M = G o L (+ D on the diagonal) in shared memory,
+//       then Y = M X + exp(cum) (C H_in^T) (tcgen05), gated and stored.
+//
+// Operands of every product sit in shared memory in the K-major, 128-byte
+// swizzled layout; C, B and H_in arrive there by bulk tensor copies, the
+// transposed x and the weighted B^T and M are written by the threads.  fp32
+// accumulation in tensor memory.  x, B and C are bf16 inputs, exact as
+// operands; an operand the kernels compute (w B, M, the carried state) is
+// split into two bf16 parts, hi = bf16(v) and lo = bf16(v - hi), and its
+// product is taken twice and summed: about 16 significant bits over the fp32
+// range, where a single bf16 rounding (8 bits) would put a 2^-9 relative error
+// on every term of the sums.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "mixer_common.cuh"
+#include "proj_gemm.cuh"
+
+namespace mm {
+
+constexpr int kSsdQ = 128;        // tokens per chunk (the products' M)
+constexpr int kSsdP = 64;         // channels per head
+constexpr int kSsdN = 128;        // d_state
+constexpr int kSsdThreads = 128;  // one token (or one state row) per thread
+
+struct SsdParams {
+    const __nv_bfloat16* x;      // [B][L][H*P]
+    const __nv_bfloat16* z;      // [B][L][H*P] or null (no gate)
+    const __nv_bfloat16* dt;     // [B][L][H]
+    const float* dt_bias;        // [H] or null
+    const float* A;              // [H]
+    const __nv_bfloat16* Bm;     // [B][L][G*N]
+    const __nv_bfloat16* Cm;     // [B][L][G*N]
+    const float* Dskip;          // [H] or null
+    const float* h0;             // [B][H][P][N] or null
+    __nv_bfloat16* y;            // [B][L][H*P]
+    float* h_last;               // [B][H][P][N]
+    float* S;                    // [B][chunks][H][P][N]  chunk states from zero (workspace)
+    __nv_bfloat16* Hin;          // [2][B][chunks][H][P][N] state entering each chunk, hi then lo parts (workspace)
+    int64_t hin_lo;              // elements from the hi parts to the lo parts
+    float* dec;                  // [B][H][chunks]        exp(cum_end) of each chunk (workspace)
+    int64_t L;
+    int H, G, chunks, batch;
+    unsigned wait_limit;
+    unsigned long long* status;  // (epoch << 8) | code of the call, or null
+    unsigned long long status_epoch;
+};
+
+// Byte offset of 16-byte piece `piece` (0..7) of row r in one K-block (rows x
+// 64 bf16, 128 bytes a row) of the K-major, 128-byte-swizzled layout: rows
+// 128 bytes apart, 8-row groups 1024 bytes apart, the piece index XORed with
+// the row's index within its group.  The block starts on a 1024-byte boundary.
+__device__ __forceinline__ uint32_t sw128_off(int r, int piece) {
+    return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((piece ^ (r & 7)) << 4));
+}
+// element (r, k), k < 128, of a [rows][128] tile made of two such K-blocks
+__device__ __forceinline__ uint32_t sw128_elem(int rows, int r, int k) {
+    return static_cast<uint32_t>((k >> 6) * rows * 128) + sw128_off(r, (k & 63) >> 3) + (k & 7) * 2;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// v = hi + lo to about 16 significant bits: hi = bf16(v), lo = bf16(v - hi)
+__device__ __forceinline__ void split_bf16(float v, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+    hi = __float2bfloat16_rn(v);
+    lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+}
+// the same for a pair, packed low element first
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+    hi = pack_bf16x2(a, b);
+    lo = pack_bf16x2(a - bf16_lo(hi), b - bf16_hi(hi));
+}
+
+__device__ __forceinline__ void ssd_fail(const SsdParams& p) {
+    atomicOr(&g_mm_fault, 1u);
+    if (p.status) atomicExch(p.status, (p.status_epoch << 8) | 1ull);
+}
+
+// Step size and the inclusive prefix sum of Delta A over the chunk, one token
+// per thread (tokens past the sequence contribute nothing).  Leaves, per token
+// j of the chunk, Delta_j in delta[j] and cum_j * log2(e) in cum2[j]; returns
+// this thread's Delta.  Contains __syncthreads.
+__device__ __forceinline__ void ssd_chunk_prefix(const SsdParams& p, int b, int h, int64_t t0, float* delta,
+                                                 float* cum2, float* warp_sums) {
+    const int j = threadIdx.x, lane = j & 31, warp = j >> 5;
+    const int64_t t = t0 + j;
+    float dl = 0.0f;
+    if (t < p.L) {
+        const float v = __bfloat162float(p.dt[(static_cast<int64_t>(b) * p.L + t) * p.H + h]) +
+                        (p.dt_bias ? p.dt_bias[h] : 0.0f);
+        dl = fmaxf(v, 0.0f) + log1pf(expf(-fabsf(v)));
+    }
+    float v = dl * p.A[h] * kLog2e;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float n = __shfl_up_sync(kFull, v, o);
+        if (lane >= o) v += n;
+    }
+    if (lane == 31) warp_sums[warp] = v;
+    __syncthreads();
+    for (int w = 0; w < warp; ++w) v += warp_sums[w];
+    delta[j] = dl;
+    cum2[j] = v;
+    __syncthreads();
+}
+
+// Thread j's token row of x (P = 64 channels of head h), zeros past the sequence.
+__device__ __forceinline__ void ssd_load_x(const SsdParams& p, int b, int h, int64_t t0, uint4 (&v)[8]) {
+    const int64_t t = t0 + threadIdx.x;
+    if (t < p.L) {
+        const uint4* src = reinterpret_cast<const uint4*>(p.x + (static_cast<int64_t>(b) * p.L + t) *
+                                                                    (static_cast<int64_t>(p.H) * kSsdP) + h * kSsdP);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = src[q];
+    } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = make_uint4(0, 0, 0, 0);
+    }
+}
+
+// ... written as column j of the transposed tile X^T [P rows][Q columns]
+// (K-major over tokens).
+__device__ __forceinline__ void ssd_write_xt(const uint4 (&v)[8], unsigned char* xt) {
+    const int j = threadIdx.x;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const uint32_t w[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const uint16_t bits = static_cast<uint16_t>((e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xffffu));
+            *reinterpret_cast<uint16_t*>(xt + sw128_elem(kSsdP, q * 8 + e, j)) = bits;
+        }
+    }
+}
+
+// ---------------------------------------------------------------- chunk states
+struct SsdStateLayout {
+    static constexpr int bw_bytes = kSsdN * kSsdQ * 2;    // (w B)^T [N rows][Q], hi then lo   2 x 32 KB
+    static constexpr int xt_bytes = kSsdP * kSsdQ * 2;    // X^T     [P rows][Q]               16 KB
+    static constexpr int smem_bytes = 1024 + 2 * bw_bytes + xt_bytes + 2 * kSsdQ * 4 + 64;
+};
+
+__global__ void __launch_bounds__(kSsdThreads, 2)
+ssd_chunk_state_kernel(const SsdParams p)
+{
+    using Lay = SsdStateLayout;
+    extern __shared__ __align__(1024) unsigned char ssm_raw[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(ssm_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char* bw = sm;                               // hi part; the lo part follows
+    unsigned char* xt = sm + 2 * Lay::bw_bytes;
+    float* delta = reinterpret_cast<float*>(xt + Lay::xt_bytes);
+    float* cum2 = delta + kSsdQ;
+    float* warp_sums = cum2 + kSsdQ;                      // 4 floats
+    uint64_t* done = reinterpret_cast<uint64_t*>(warp_sums + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int64_t t0 = static_cast<int64_t>(c) * kSsdQ;
+    const int g = h / (p.H / p.G);
+
+    if (tid == 0) {
+        mbar_init(done, 1);
+        fence_mbar_init();
+    }
+    if (warp == 2) {
+        tmem_alloc(tmem_slot, 64);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    ssd_chunk_prefix(p, b, h, t0, delta, cum2, warp_sums);   // syncs: the barrier and tensor memory are set up
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // column j of (w B)^T: token j's B row scaled by w_j = exp(cum_end - cum_j) Delta_j
+    {
+        const int j = tid;
+        const int64_t t = t0 + j;
+        const float w = t < p.L ? ex2_fast(cum2[kSsdQ - 1] - cum2[j]) * delta[j] : 0.0f;
+        const uint4* src = reinterpret_cast<const uint4*>(
+            p.Bm + ((static_cast<int64_t>(b) * p.L + (t < p.L ? t : 0)) * p.G + g) * kSsdN);
+#pragma unroll 4
+        for (int q = 0; q < kSsdN / 8; ++q) {
+            const uint4 v = t < p.L ? src[q] : make_uint4(0, 0, 0, 0);
+            const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float bv = (e & 1) ? bf16_hi(wd[e >> 1]) : bf16_lo(wd[e >> 1]);
+                __nv_bfloat16 hi, lo;
+                split_bf16(w * bv, hi, lo);
+                const uint32_t off = sw128_elem(kSsdN, q * 8 + e, j);
+                *reinterpret_cast<__nv_bfloat16*>(bw + off) = hi;
+                *reinterpret_cast<__nv_bfloat16*>(bw + Lay::bw_bytes + off) = lo;
+            }
+        }
+    }
+    {
+        uint4 xv[8];
+        ssd_load_x(p, b, h, t0, xv);
+        ssd_write_xt(xv, xt);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // S[n][p] = sum_j (w B)^T[n][j] X^T[p][j] (hi and lo parts): M = N = 128,
+    // N = P = 64, K = Q = 128
+    if (warp == 1 && elect_one_lane()) {
+        constexpr uint32_t idesc = umma_idesc_bf16(kSsdN, kSsdP);
+        const uint32_t a0 = smem_addr(bw), b0 = smem_addr(xt);
+#pragma unroll
+        for (int kk = 0; kk < kSsdQ / 16; ++kk) {
+            const uint32_t koff = (kk & 3) * 32;
+            const uint32_t a = a0 + (kk >> 2) * (kSsdN * 128) + koff;
+            const uint64_t bdesc = umma_desc_sw128(b0 + (kk >> 2) * (kSsdP * 128) + koff);
+            umma_bf16(tmem, umma_desc_sw128(a), bdesc, idesc, kk > 0 ? 1u : 0u);
+            umma_bf16(tmem, umma_desc_sw128(a + Lay::bw_bytes), bdesc, idesc, 1u);
+        }
+        umma_commit(done);
+    }
+    const bool ok = mbar_wait_bounded(done, 0, p.wait_limit);
+    tc_fence_after();
+    if (__syncthreads_and(ok)) {
+        // thread n owns state row n: S[b][c][h][p][n] for p = 0..63 (a warp stores 32 consecutive n)
+        const int n = tid;
+        float* dst = p.S + ((static_cast<int64_t>(b) * p.chunks + c) * p.H + h) * (kSsdP * kSsdN) + n;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+            float v[32];
+            tmem_ld32(lane_base + half * 32, v);
+#pragma unroll
+            for (int q = 0; q < 32; ++q) dst[(half * 32 + q) * kSsdN] = v[q];
+        }
+        if (tid == 0) p.dec[(static_cast<int64_t>(b) * p.H + h) * p.chunks + c] = ex2_fast(cum2[kSsdQ - 1]);
+    } else {
+        if (tid == 0) ssd_fail(p);
+        mbar_wait_bounded(done, 0, 1u << 20);   // the MMAs finish before tensor memory is freed
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 64);
+    }
+}
+
+// ---------------------------------------------------------------- state passing
+// One thread: 4 consecutive state entries (same head, channel; n..n+3) of one
+// sequence, walked through every chunk in order.
+__global__ void __launch_bounds__(256)
+ssd_state_pass_kernel(const SsdParams p)
+{
+    constexpr int64_t kHead = int64_t(kSsdP) * kSsdN;
+    const int64_t per_seq = int64_t(p.H) * kHead;
+    const int64_t f = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+    if (f >= per_seq) return;
+    const int b = blockIdx.y;
+    const int h = static_cast<int>(f / kHead);
+    float4 s = p.h0 ? *reinterpret_cast<const float4*>(p.h0 + b * per_seq + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float* dec = p.dec + (static_cast<int64_t>(b) * p.H + h) * p.chunks;
+    for (int c = 0; c < p.chunks; ++c) {
+        const int64_t off = (static_cast<int64_t>(b) * p.chunks + c) * per_seq + f;
+        uint2 hi, lo;
+        split_bf16x2(s.x, s.y, hi.x, lo.x);
+        split_bf16x2(s.z, s.w, hi.y, lo.y);
+        *reinterpret_cast<uint2*>(p.Hin + off) = hi;
+        *reinterpret_cast<uint2*>(p.Hin + p.hin_lo + off) = lo;
+        const float d = dec[c];
+        const float4 add = *reinterpret_cast<const float4*>(p.S + off);
+        s.x = fmaf(d, s.x, add.x);
+        s.y = fmaf(d, s.y, add.y);
+        s.z = fmaf(d, s.z, add.z);
+        s.w = fmaf(d, s.w, add.w);
+    }
+    *reinterpret_cast<float4*>(p.h_last + b * per_seq + f) = s;
+}
+
+// ---------------------------------------------------------------- chunk scan
+// Shared memory of the chunk scan.  The first products read C, B and H_in;
+// once they complete, the same space holds M (hi over B, lo over H_in) and
+// X^T (over C) for the second.
+struct SsdScanLayout {
+    static constexpr int c_off = 0;                                 // C [Q rows][N] 32 KB, then X^T [P rows][Q]
+    static constexpr int b_off = c_off + kSsdQ * kSsdN * 2;         // B [Q rows][N] 32 KB, then M hi [Q rows][Q]
+    static constexpr int h_off = b_off + kSsdQ * kSsdN * 2;         // H_in hi, lo [P rows][N] 2 x 16 KB, then M lo
+    static constexpr int hin_bytes = kSsdP * kSsdN * 2;
+    static constexpr int f_off = h_off + 2 * hin_bytes;             // delta, cum2, warp sums
+    static constexpr int bar_off = f_off + 2 * kSsdQ * 4 + 16;
+    static constexpr int smem_bytes = 1024 + bar_off + 4 * 8 + 16;
+    static constexpr uint32_t tx_bytes = 2 * kSsdQ * kSsdN * 2 + 2 * hin_bytes;
+};
+static_assert(SsdScanLayout::b_off % 1024 == 0 && SsdScanLayout::h_off % 1024 == 0 &&
+              SsdScanLayout::hin_bytes % 1024 == 0, "operand tiles start on 1024-byte boundaries");
+
+// Tensor memory columns of the chunk scan: G [Q x Q], C H_in^T [Q x P], M X [Q x P].
+constexpr uint32_t kSsdColG = 0, kSsdColOff = 128, kSsdColDiag = 192, kSsdCols = 256;
+
+__global__ void __launch_bounds__(kSsdThreads, 2)
+ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_c,
+                      const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_h)
+{
+    using Lay = SsdScanLayout;
+    extern __shared__ __align__(1024) unsigned char ssc_raw[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(ssc_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char* ct = sm + Lay::c_off;      // C, then X^T
+    unsigned char* bt = sm + Lay::b_off;      // B, then M hi
+    unsigned char* ht = sm + Lay::h_off;      // H_in hi and lo, then M lo
+    float* delta = reinterpret_cast<float*>(sm + Lay::f_off);
+    float* cum2 = delta + kSsdQ;
+    float* warp_sums = cum2 + kSsdQ;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::bar_off);   // loaded, products 1, product 2
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int64_t t0 = static_cast<int64_t>(c) * kSsdQ;
+    const int g = h / (p.H / p.G);
+
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        mbar_init(&bars[2], 1);
+        fence_mbar_init();
+        // C and B rows of the chunk (rows past the sequence read as zeros), and
+        // the state entering it (hi and lo parts): two 64-wide K-blocks each
+        mbar_arrive_expect_tx(&bars[0], Lay::tx_bytes);
+        const int tok = static_cast<int>(t0);
+        const int hrow = static_cast<int>(((static_cast<int64_t>(b) * p.chunks + c) * p.H + h) * kSsdP);
+        const int lo_rows = static_cast<int>(p.hin_lo / kSsdN);
+        for (int kb = 0; kb < 2; ++kb) {
+            tma_load_3d(ct + kb * (kSsdQ * 128), &tm_c, g * kSsdN + kb * 64, tok, b, &bars[0]);
+            tma_load_3d(bt + kb * (kSsdQ * 128), &tm_b, g * kSsdN + kb * 64, tok, b, &bars[0]);
+            tma_load_3d(ht + kb * (kSsdP * 128), &tm_h, kb * 64, hrow, 0, &bars[0]);
+            tma_load_3d(ht + Lay::hin_bytes + kb * (kSsdP * 128), &tm_h, kb * 64, lo_rows + hrow, 0, &bars[0]);
+        }
+    }
+    if (warp == 2) {
+        tmem_alloc(tmem_slot, kSsdCols);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    ssd_chunk_prefix(p, b, h, t0, delta, cum2, warp_sums);   // syncs
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    uint4 xv[8];
+    ssd_load_x(p, b, h, t0, xv);             // lands while the first products run
+
+    // products 1: G = C B^T (N = Q) and C H_in^T (N = P, hi and lo), K = N = 128
+    bool loaded = true, ok = true;
+    if (warp == 1 && elect_one_lane()) {
+        loaded = mbar_wait_bounded(&bars[0], 0, p.wait_limit);
+        if (loaded) {
+            tc_fence_after();
+            constexpr uint32_t id_g = umma_idesc_bf16(kSsdQ, kSsdQ);
+            constexpr uint32_t id_o = umma_idesc_bf16(kSsdQ, kSsdP);
+            const uint32_t ca = smem_addr(ct), ba = smem_addr(bt), ha = smem_addr(ht);
+#pragma unroll
+            for (int kk = 0; kk < kSsdN / 16; ++kk) {
+                const uint32_t koff = (kk & 3) * 32;
+                const uint64_t adesc = umma_desc_sw128(ca + (kk >> 2) * (kSsdQ * 128) + koff);
+                umma_bf16(tmem + kSsdColG, adesc, umma_desc_sw128(ba + (kk >> 2) * (kSsdQ * 128) + koff), id_g,
+                          kk > 0 ? 1u : 0u);
+                const uint32_t hk = ha + (kk >> 2) * (kSsdP * 128) + koff;
+                umma_bf16(tmem + kSsdColOff, adesc, umma_desc_sw128(hk), id_o, kk > 0 ? 1u : 0u);
+                umma_bf16(tmem + kSsdColOff, adesc, umma_desc_sw128(hk + Lay::hin_bytes), id_o, 1u);
+            }
+            umma_commit(&bars[1]);
+        }
+    }
+    const bool issued1 = __syncthreads_and(loaded);
+    if (issued1) ok = mbar_wait_bounded(&bars[1], 0, p.wait_limit);
+    tc_fence_after();
+    const bool g_ready = __syncthreads_and(issued1 && ok);
+
+    // M[i][j] = G[i][j] exp(cum_i - cum_j) Delta_j for j <= i, 0 above the
+    // diagonal, plus D on it; row i (this thread) as hi and lo parts over the
+    // B and H_in tiles, and X^T over the C tile (all three free now)
+    const int i = tid;
+    if (g_ready) {
+        ssd_write_xt(xv, ct);
+        const float ci = cum2[i];
+        const float dsk = p.Dskip ? p.Dskip[h] : 0.0f;
+#pragma unroll 1
+        for (int jb = 0; jb < kSsdQ / 32; ++jb) {
+            float m[32];
+            if (jb <= warp) {     // warp-uniform: blocks above the diagonal block are zero
+                tmem_ld32(lane_base + kSsdColG + jb * 32, m);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const int j = jb * 32 + q;
+                    m[q] = j <= i ? m[q] * ex2_fast(ci - cum2[j]) * delta[j] : 0.0f;
+                    if (j == i) m[q] += dsk;
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 32; ++q) m[q] = 0.0f;
+            }
+            const uint32_t blk = (jb >> 1) * (kSsdQ * 128);
+#pragma unroll
+            for (int pp = 0; pp < 4; ++pp) {
+                uint4 hi, lo;
+                split_bf16x2(m[pp * 8 + 0], m[pp * 8 + 1], hi.x, lo.x);
+                split_bf16x2(m[pp * 8 + 2], m[pp * 8 + 3], hi.y, lo.y);
+                split_bf16x2(m[pp * 8 + 4], m[pp * 8 + 5], hi.z, lo.z);
+                split_bf16x2(m[pp * 8 + 6], m[pp * 8 + 7], hi.w, lo.w);
+                const uint32_t off = blk + sw128_off(i, (jb & 1) * 4 + pp);
+                *reinterpret_cast<uint4*>(bt + off) = hi;
+                *reinterpret_cast<uint4*>(ht + off) = lo;
+            }
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // product 2: M X (hi and lo), K = Q = 128, N = P
+    if (g_ready && warp == 1 && elect_one_lane()) {
+        constexpr uint32_t id_y = umma_idesc_bf16(kSsdQ, kSsdP);
+        const uint32_t mh = smem_addr(bt), ml = smem_addr(ht), xa = smem_addr(ct);
+#pragma unroll
+        for (int kk = 0; kk < kSsdQ / 16; ++kk) {
+            const uint32_t koff = (kk & 3) * 32;
+            const uint32_t mk = (kk >> 2) * (kSsdQ * 128) + koff;
+            const uint64_t xdesc = umma_desc_sw128(xa + (kk >> 2) * (kSsdP * 128) + koff);
+            umma_bf16(tmem + kSsdColDiag, umma_desc_sw128(mh + mk), xdesc, id_y, kk > 0 ? 1u : 0u);
+            umma_bf16(tmem + kSsdColDiag, umma_desc_sw128(ml + mk), xdesc, id_y, 1u);
+        }
+        umma_commit(&bars[2]);
+    }
+    bool y_ok = false;
+    if (g_ready) y_ok = mbar_wait_bounded(&bars[2], 0, p.wait_limit);
+    tc_fence_after();
+    const bool y_ready = __syncthreads_and(y_ok);
+
+    // y_i = (M X)_i + exp(cum_i) (C H_in^T)_i, gated; the tensor-memory loads
+    // are warp-wide, so every lane takes part and only in-sequence rows store
+    const int64_t t = t0 + i;
+    if (y_ready) {
+        const float e = ex2_fast(cum2[i]);
+        const int64_t row = (static_cast<int64_t>(b) * p.L + (t < p.L ? t : 0)) * (static_cast<int64_t>(p.H) * kSsdP) +
+                            h * kSsdP;
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+            float yo[32], yd[32];
+            tmem_ld32(lane_base + kSsdColOff + half * 32, yo);
+            tmem_ld32(lane_base + kSsdColDiag + half * 32, yd);
+            if (t < p.L) {
+                float gz[32];
+                if (p.z) {
+                    const uint4* zs = reinterpret_cast<const uint4*>(p.z + row + half * 32);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 v = zs[q];
+                        const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int e2 = 0; e2 < 8; ++e2) {
+                            const float zv = (e2 & 1) ? bf16_hi(wd[e2 >> 1]) : bf16_lo(wd[e2 >> 1]);
+                            gz[q * 8 + e2] = zv / (1.0f + expf(-zv));
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) gz[q] = 1.0f;
+                }
+                uint4* dst = reinterpret_cast<uint4*>(p.y + row + half * 32);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float o[8];
+#pragma unroll
+                    for (int e2 = 0; e2 < 8; ++e2) o[e2] = fmaf(e, yo[q * 8 + e2], yd[q * 8 + e2]) * gz[q * 8 + e2];
+                    uint4 w;
+                    w.x = pack_bf16x2(o[0], o[1]);
+                    w.y = pack_bf16x2(o[2], o[3]);
+                    w.z = pack_bf16x2(o[4], o[5]);
+                    w.w = pack_bf16x2(o[6], o[7]);
+                    dst[q] = w;
+                }
+            }
+        }
+    }
+
+    if (!y_ready) {
+        if (tid == 0) ssd_fail(p);
+        // copies and products of this CTA finish before shared and tensor memory go away
+        if (warp == 1 && elect_one_lane()) {
+            if (!loaded) mbar_wait_bounded(&bars[0], 0, 1u << 20);
+            if (issued1) mbar_wait_bounded(&bars[1], 0, 1u << 20);
+            if (g_ready) mbar_wait_bounded(&bars[2], 0, 1u << 20);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kSsdCols);
+    }
+}
+
+}  // namespace mm

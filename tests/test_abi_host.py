@@ -59,7 +59,7 @@ def test_exported_symbols_are_c_linkage():
 
 def test_version_and_strings():
     mmbuild.build()
-    assert mm.abi_version() == 4
+    assert mm.abi_version() == 5
     for code in range(13):
         s = mm.status_string(code)
         assert s and s != "unknown status"
@@ -294,6 +294,54 @@ def test_projected_validation(L):
     assert call(ws_bytes=need - 16) == EWORKSPACE
     assert call(ws=xz) == EALIAS           # the workspace over an input
     assert call(xz=None) == ENULL
+
+
+# ---------------------------------------------------------------- Mamba-2 form
+def ssd_args(B=2, Lq=300, H=4, P=64, N=128, G=2, ws_bytes=None, **over):
+    """mamba_ssd_fwd arguments on fake addresses, each buffer 2^32 apart."""
+    names = ["x", "z", "dt", "dt_bias", "A", "Bm", "Cm", "Dskip", "h0", "y", "h_last"]
+    addr = {n: BASE + (i << 32) for i, n in enumerate(names)}
+    addr.update(over)
+    ws = over.get("ws", WS_ADDR)
+    need = mm.ssd_workspace_size(max(B, 1), Lq, H, P, N, G) if ws_bytes is None else ws_bytes
+    return [addr[n] for n in names] + [B, Lq, H, P, N, G, ws, need, None]
+
+
+def test_ssd_workspace_size_rules():
+    # header, fp32 chunk states, entering states as two bf16 parts, fp32 chunk
+    # decays: 4096 tokens are 32 chunks of 128; 128 heads of 64 x 128 states
+    states = 32 * 128 * 64 * 128
+    assert mm.ssd_workspace_size(1, 4096, 128) == 256 + states * 4 + states * 4 + 128 * 32 * 4
+    assert mm.ssd_workspace_size(1, 0, 128) == 256
+    assert mm.ssd_workspace_size(1, 4096, 128, headdim=32) == 0
+    assert mm.ssd_workspace_size(1, 4096, 128, d_state=64) == 0
+    assert mm.ssd_workspace_size(1, 4096, 6, groups=4) == 0
+    assert mm.ssd_workspace_size(0, 4096, 128) == 0
+
+
+def test_ssd_validation(L):
+    assert L.mamba_ssd_fwd(*ssd_args()) == EDEVICE
+    assert L.mamba_ssd_fwd(*ssd_args(z=None, dt_bias=None, Dskip=None, h0=None)) == EDEVICE
+    assert L.mamba_ssd_fwd(*ssd_args(P=32)) == EUNSUP
+    assert L.mamba_ssd_fwd(*ssd_args(N=64)) == EUNSUP
+    assert L.mamba_ssd_fwd(*ssd_args(H=6, G=4)) == ESHAPE
+    assert L.mamba_ssd_fwd(*ssd_args(G=0)) == ESHAPE
+    assert L.mamba_ssd_fwd(*ssd_args(Lq=-1, ws_bytes=0)) == ESHAPE
+    assert L.mamba_ssd_fwd(*ssd_args(B=0, ws_bytes=0)) == OK
+    for name in ("x", "dt", "A", "Bm", "Cm", "y", "h_last"):
+        assert L.mamba_ssd_fwd(*ssd_args(**{name: None})) == ENULL, name
+    # no token: only A and h_last are needed
+    assert L.mamba_ssd_fwd(*ssd_args(Lq=0, x=None, dt=None, Bm=None, Cm=None, y=None)) == EDEVICE
+    for name in ("x", "Bm", "h0", "y", "dt_bias"):
+        assert L.mamba_ssd_fwd(*ssd_args(**{name: BASE + (1 << 40) + 8})) == EALIGN, name
+    assert L.mamba_ssd_fwd(*ssd_args(y=BASE)) == EALIAS                      # y over x
+    assert L.mamba_ssd_fwd(*ssd_args(h_last=BASE + (8 << 32))) == EALIAS     # h_last over h0
+    assert L.mamba_ssd_fwd(*ssd_args(h_last=BASE + (9 << 32) + 64)) == EALIAS   # h_last over y
+    assert L.mamba_ssd_fwd(*ssd_args(ws=BASE + (5 << 32))) == EALIAS         # workspace over B
+    need = mm.ssd_workspace_size(2, 300, 4, 64, 128, 2)
+    assert L.mamba_ssd_fwd(*ssd_args(ws_bytes=need - 16)) == EWORKSPACE
+    assert L.mamba_ssd_fwd(*ssd_args(ws=None)) == EWORKSPACE
+    assert L.mamba_ssd_fwd(*ssd_args(ws=WS_ADDR + 8)) == EALIGN
 
 
 # ---------------------------------------------------------------- state_update validation
