@@ -135,55 +135,55 @@ __device__ __forceinline__ void ssd_chunk_prefix(const SsdParams& p, int b, int 
     __syncthreads();
 }
 
-// Thread j's token row of x (P = 64 channels of head h), zeros past the sequence.
-__device__ __forceinline__ void ssd_load_x(const SsdParams& p, int b, int h, int64_t t0, uint4 (&v)[8]) {
-    const int64_t t = t0 + threadIdx.x;
-    if (t < p.L) {
-        const uint4* src = reinterpret_cast<const uint4*>(p.x + (static_cast<int64_t>(b) * p.L + t) *
-                                                                    (static_cast<int64_t>(p.H) * kSsdP) + h * kSsdP);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) v[q] = src[q];
-    } else {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) v[q] = make_uint4(0, 0, 0, 0);
-    }
+// ---------------------------------------------------------------- MN-major operands
+// Shared-memory descriptor of an MN-major operand tile as a 128-byte swizzled
+// tensor copy writes it: along M (or N) 64 bf16 per 128-byte row, one row per
+// k, 8-row groups 1024 bytes apart (stride byte offset), 64-wide M/N blocks
+// `lbo` bytes apart (leading byte offset; 0 for a single block).  Version 1,
+// 128-byte swizzle; the tile starts on a 1024-byte boundary, and a K step of
+// 16 advances the start by two groups (2048 bytes).
+__device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t smem_byte_addr, uint32_t lbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((smem_byte_addr >> 4) & 0x3FFF);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFF) << 16;
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
 }
-
-// ... written as column j of the transposed tile X^T [P rows][Q columns]
-// (K-major over tokens).
-__device__ __forceinline__ void ssd_write_xt(const uint4 (&v)[8], unsigned char* xt) {
-    const int j = threadIdx.x;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        const uint32_t w[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const uint16_t bits = static_cast<uint16_t>((e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xffffu));
-            *reinterpret_cast<uint16_t*>(xt + sw128_elem(kSsdP, q * 8 + e, j)) = bits;
-        }
-    }
+// instruction descriptor of kind::f16 (bf16 operands, fp32 accumulator) with
+// A and/or B MN-major (bits 15 and 16)
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_mn(int m, int n, bool a_mn, bool b_mn) {
+    return umma_idesc_bf16(m, n) | (a_mn ? 1u << 15 : 0u) | (b_mn ? 1u << 16 : 0u);
 }
 
 // ---------------------------------------------------------------- chunk states
+// S[n][p] = sum_j B_j[n] (w_j x_j[p]): A = B as copied ([token][n], MN-major,
+// two 64-wide blocks of n), B = the x tile as copied ([token][p], MN-major),
+// each row scaled in place by its w_j and split into hi and lo parts.
 struct SsdStateLayout {
-    static constexpr int bw_bytes = kSsdN * kSsdQ * 2;    // (w B)^T [N rows][Q], hi then lo   2 x 32 KB
-    static constexpr int xt_bytes = kSsdP * kSsdQ * 2;    // X^T     [P rows][Q]               16 KB
-    static constexpr int smem_bytes = 1024 + 2 * bw_bytes + xt_bytes + 2 * kSsdQ * 4 + 64;
+    static constexpr int b_bytes = kSsdQ * kSsdN * 2;     // B [Q rows][N]: two [Q][64] blocks   32 KB
+    static constexpr int x_bytes = kSsdQ * kSsdP * 2;     // x [Q rows][P], then hi of w x      16 KB; lo 16 KB
+    static constexpr int f_off = b_bytes + 2 * x_bytes;
+    static constexpr int smem_bytes = 1024 + f_off + 2 * kSsdQ * 4 + 16 + 2 * 8 + 16;
+    static constexpr uint32_t tx_bytes = b_bytes + x_bytes;
 };
 
-__global__ void __launch_bounds__(kSsdThreads, 2)
-ssd_chunk_state_kernel(const SsdParams p)
+__global__ void __launch_bounds__(kSsdThreads, 3)
+ssd_chunk_state_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_b,
+                       const __grid_constant__ CUtensorMap tm_x)
 {
     using Lay = SsdStateLayout;
     extern __shared__ __align__(1024) unsigned char ssm_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(ssm_raw) + 1023) & ~uintptr_t(1023));
-    unsigned char* bw = sm;                               // hi part; the lo part follows
-    unsigned char* xt = sm + 2 * Lay::bw_bytes;
-    float* delta = reinterpret_cast<float*>(xt + Lay::xt_bytes);
+    unsigned char* bt = sm;
+    unsigned char* xh = sm + Lay::b_bytes;
+    unsigned char* xl = xh + Lay::x_bytes;
+    float* delta = reinterpret_cast<float*>(sm + Lay::f_off);
     float* cum2 = delta + kSsdQ;
     float* warp_sums = cum2 + kSsdQ;                      // 4 floats
-    uint64_t* done = reinterpret_cast<uint64_t*>(warp_sums + 4);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(warp_sums + 4);   // loaded, products done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
 
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -191,66 +191,66 @@ ssd_chunk_state_kernel(const SsdParams p)
     const int g = h / (p.H / p.G);
 
     if (tid == 0) {
-        mbar_init(done, 1);
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
         fence_mbar_init();
+        // B and x rows of the chunk (rows past the sequence read as zeros)
+        mbar_arrive_expect_tx(&bars[0], Lay::tx_bytes);
+        const int tok = static_cast<int>(t0);
+        tma_load_3d(bt, &tm_b, g * kSsdN, tok, b, &bars[0]);
+        tma_load_3d(bt + kSsdQ * 128, &tm_b, g * kSsdN + 64, tok, b, &bars[0]);
+        tma_load_3d(xh, &tm_x, h * kSsdP, tok, b, &bars[0]);
     }
     if (warp == 2) {
         tmem_alloc(tmem_slot, 64);
         tmem_relinquish();
         tc_fence_before();
     }
-    ssd_chunk_prefix(p, b, h, t0, delta, cum2, warp_sums);   // syncs: the barrier and tensor memory are set up
+    ssd_chunk_prefix(p, b, h, t0, delta, cum2, warp_sums);   // syncs: the barriers and tensor memory are set up
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // column j of (w B)^T: token j's B row scaled by w_j = exp(cum_end - cum_j) Delta_j
-    {
+    const bool loaded = __syncthreads_and(mbar_wait_bounded(&bars[0], 0, p.wait_limit));
+    if (loaded) {
+        // row j of the x tile (its 16-byte pieces in swizzled order, which a
+        // scale of the whole row does not see) times w_j = exp(cum_end - cum_j)
+        // Delta_j, as hi and lo parts
         const int j = tid;
-        const int64_t t = t0 + j;
-        const float w = t < p.L ? ex2_fast(cum2[kSsdQ - 1] - cum2[j]) * delta[j] : 0.0f;
-        const uint4* src = reinterpret_cast<const uint4*>(
-            p.Bm + ((static_cast<int64_t>(b) * p.L + (t < p.L ? t : 0)) * p.G + g) * kSsdN);
-#pragma unroll 4
-        for (int q = 0; q < kSsdN / 8; ++q) {
-            const uint4 v = t < p.L ? src[q] : make_uint4(0, 0, 0, 0);
-            const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+        const float w = t0 + j < p.L ? ex2_fast(cum2[kSsdQ - 1] - cum2[j]) * delta[j] : 0.0f;
+        uint4* rh = reinterpret_cast<uint4*>(xh + j * 128);
+        uint4* rl = reinterpret_cast<uint4*>(xl + j * 128);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float bv = (e & 1) ? bf16_hi(wd[e >> 1]) : bf16_lo(wd[e >> 1]);
-                __nv_bfloat16 hi, lo;
-                split_bf16(w * bv, hi, lo);
-                const uint32_t off = sw128_elem(kSsdN, q * 8 + e, j);
-                *reinterpret_cast<__nv_bfloat16*>(bw + off) = hi;
-                *reinterpret_cast<__nv_bfloat16*>(bw + Lay::bw_bytes + off) = lo;
-            }
+        for (int q = 0; q < 8; ++q) {
+            const uint4 v = rh[q];
+            uint4 hi, lo;
+            split_bf16x2(w * bf16_lo(v.x), w * bf16_hi(v.x), hi.x, lo.x);
+            split_bf16x2(w * bf16_lo(v.y), w * bf16_hi(v.y), hi.y, lo.y);
+            split_bf16x2(w * bf16_lo(v.z), w * bf16_hi(v.z), hi.z, lo.z);
+            split_bf16x2(w * bf16_lo(v.w), w * bf16_hi(v.w), hi.w, lo.w);
+            rh[q] = hi;
+            rl[q] = lo;
         }
-    }
-    {
-        uint4 xv[8];
-        ssd_load_x(p, b, h, t0, xv);
-        ssd_write_xt(xv, xt);
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
 
-    // S[n][p] = sum_j (w B)^T[n][j] X^T[p][j] (hi and lo parts): M = N = 128,
-    // N = P = 64, K = Q = 128
-    if (warp == 1 && elect_one_lane()) {
-        constexpr uint32_t idesc = umma_idesc_bf16(kSsdN, kSsdP);
-        const uint32_t a0 = smem_addr(bw), b0 = smem_addr(xt);
+    // M = N = 128, N = P = 64, K = Q = 128; both operands MN-major
+    if (loaded && warp == 1 && elect_one_lane()) {
+        constexpr uint32_t idesc = umma_idesc_bf16_mn(kSsdN, kSsdP, true, true);
+        const uint32_t a0 = smem_addr(bt), h0 = smem_addr(xh), l0 = smem_addr(xl);
 #pragma unroll
         for (int kk = 0; kk < kSsdQ / 16; ++kk) {
-            const uint32_t koff = (kk & 3) * 32;
-            const uint32_t a = a0 + (kk >> 2) * (kSsdN * 128) + koff;
-            const uint64_t bdesc = umma_desc_sw128(b0 + (kk >> 2) * (kSsdP * 128) + koff);
-            umma_bf16(tmem, umma_desc_sw128(a), bdesc, idesc, kk > 0 ? 1u : 0u);
-            umma_bf16(tmem, umma_desc_sw128(a + Lay::bw_bytes), bdesc, idesc, 1u);
+            const uint32_t koff = kk * 2048;
+            const uint64_t adesc = umma_desc_sw128_mn(a0 + koff, kSsdQ * 128);
+            umma_bf16(tmem, adesc, umma_desc_sw128_mn(h0 + koff, 0), idesc, kk > 0 ? 1u : 0u);
+            umma_bf16(tmem, adesc, umma_desc_sw128_mn(l0 + koff, 0), idesc, 1u);
         }
-        umma_commit(done);
+        umma_commit(&bars[1]);
     }
-    const bool ok = mbar_wait_bounded(done, 0, p.wait_limit);
+    bool ok = false;
+    if (loaded) ok = mbar_wait_bounded(&bars[1], 0, p.wait_limit);
     tc_fence_after();
     if (__syncthreads_and(ok)) {
         // thread n owns state row n: S[b][c][h][p][n] for p = 0..63 (a warp stores 32 consecutive n)
@@ -267,7 +267,11 @@ ssd_chunk_state_kernel(const SsdParams p)
         if (tid == 0) p.dec[(static_cast<int64_t>(b) * p.H + h) * p.chunks + c] = ex2_fast(cum2[kSsdQ - 1]);
     } else {
         if (tid == 0) ssd_fail(p);
-        mbar_wait_bounded(done, 0, 1u << 20);   // the MMAs finish before tensor memory is freed
+        // the copies and products finish before shared and tensor memory go away
+        if (warp == 1 && elect_one_lane()) {
+            if (!loaded) mbar_wait_bounded(&bars[0], 0, 1u << 20);
+            else mbar_wait_bounded(&bars[1], 0, 1u << 20);
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -311,9 +315,9 @@ ssd_state_pass_kernel(const SsdParams p)
 // ---------------------------------------------------------------- chunk scan
 // Shared memory of the chunk scan.  The first products read C, B and H_in;
 // once they complete, the same space holds M (hi over B, lo over H_in) and
-// X^T (over C) for the second.
+// the x tile (over C, MN-major: [token][p]) for the second.
 struct SsdScanLayout {
-    static constexpr int c_off = 0;                                 // C [Q rows][N] 32 KB, then X^T [P rows][Q]
+    static constexpr int c_off = 0;                                 // C [Q rows][N] 32 KB, then x [Q rows][P]
     static constexpr int b_off = c_off + kSsdQ * kSsdN * 2;         // B [Q rows][N] 32 KB, then M hi [Q rows][Q]
     static constexpr int h_off = b_off + kSsdQ * kSsdN * 2;         // H_in hi, lo [P rows][N] 2 x 16 KB, then M lo
     static constexpr int hin_bytes = kSsdP * kSsdN * 2;
@@ -330,18 +334,19 @@ constexpr uint32_t kSsdColG = 0, kSsdColOff = 128, kSsdColDiag = 192, kSsdCols =
 
 __global__ void __launch_bounds__(kSsdThreads, 2)
 ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_c,
-                      const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_h)
+                      const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_h,
+                      const __grid_constant__ CUtensorMap tm_x)
 {
     using Lay = SsdScanLayout;
     extern __shared__ __align__(1024) unsigned char ssc_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(ssc_raw) + 1023) & ~uintptr_t(1023));
-    unsigned char* ct = sm + Lay::c_off;      // C, then X^T
+    unsigned char* ct = sm + Lay::c_off;      // C, then x
     unsigned char* bt = sm + Lay::b_off;      // B, then M hi
     unsigned char* ht = sm + Lay::h_off;      // H_in hi and lo, then M lo
     float* delta = reinterpret_cast<float*>(sm + Lay::f_off);
     float* cum2 = delta + kSsdQ;
     float* warp_sums = cum2 + kSsdQ;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::bar_off);   // loaded, products 1, product 2
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::bar_off);   // loaded, products 1, product 2, x loaded
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
 
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -353,6 +358,7 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
         mbar_init(&bars[0], 1);
         mbar_init(&bars[1], 1);
         mbar_init(&bars[2], 1);
+        mbar_init(&bars[3], 1);
         fence_mbar_init();
         // C and B rows of the chunk (rows past the sequence read as zeros), and
         // the state entering it (hi and lo parts): two 64-wide K-blocks each
@@ -376,11 +382,10 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    uint4 xv[8];
-    ssd_load_x(p, b, h, t0, xv);             // lands while the first products run
 
     // products 1: G = C B^T (N = Q) and C H_in^T (N = P, hi and lo), K = N = 128
     bool loaded = true, ok = true;
+    bool x_issued = false, x_done = false;    // the x tile's copy (warp 1's elected lane)
     if (warp == 1 && elect_one_lane()) {
         loaded = mbar_wait_bounded(&bars[0], 0, p.wait_limit);
         if (loaded) {
@@ -399,6 +404,13 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
                 umma_bf16(tmem + kSsdColOff, adesc, umma_desc_sw128(hk + Lay::hin_bytes), id_o, 1u);
             }
             umma_commit(&bars[1]);
+            // C is free once these products complete: the x tile goes there,
+            // copied while M is built
+            if (mbar_wait_bounded(&bars[1], 0, p.wait_limit)) {
+                mbar_arrive_expect_tx(&bars[3], kSsdQ * kSsdP * 2);
+                tma_load_3d(ct, &tm_x, h * kSsdP, static_cast<int>(t0), b, &bars[3]);
+                x_issued = true;
+            }
         }
     }
     const bool issued1 = __syncthreads_and(loaded);
@@ -408,10 +420,9 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
 
     // M[i][j] = G[i][j] exp(cum_i - cum_j) Delta_j for j <= i, 0 above the
     // diagonal, plus D on it; row i (this thread) as hi and lo parts over the
-    // B and H_in tiles, and X^T over the C tile (all three free now)
+    // B and H_in tiles (both free now)
     const int i = tid;
     if (g_ready) {
-        ssd_write_xt(xv, ct);
         const float ci = cum2[i];
         const float dsk = p.Dskip ? p.Dskip[h] : 0.0f;
 #pragma unroll 1
@@ -448,61 +459,65 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
     __syncthreads();
     tc_fence_after();
 
-    // product 2: M X (hi and lo), K = Q = 128, N = P
+    // product 2: M X (hi and lo), K = Q = 128, N = P; x MN-major as copied
+    bool x_loaded = true;
     if (g_ready && warp == 1 && elect_one_lane()) {
-        constexpr uint32_t id_y = umma_idesc_bf16(kSsdQ, kSsdP);
-        const uint32_t mh = smem_addr(bt), ml = smem_addr(ht), xa = smem_addr(ct);
+        x_done = x_issued && mbar_wait_bounded(&bars[3], 0, p.wait_limit);
+        x_loaded = x_done;
+        if (x_loaded) {
+            constexpr uint32_t id_y = umma_idesc_bf16_mn(kSsdQ, kSsdP, false, true);
+            const uint32_t mh = smem_addr(bt), ml = smem_addr(ht), xa = smem_addr(ct);
 #pragma unroll
-        for (int kk = 0; kk < kSsdQ / 16; ++kk) {
-            const uint32_t koff = (kk & 3) * 32;
-            const uint32_t mk = (kk >> 2) * (kSsdQ * 128) + koff;
-            const uint64_t xdesc = umma_desc_sw128(xa + (kk >> 2) * (kSsdP * 128) + koff);
-            umma_bf16(tmem + kSsdColDiag, umma_desc_sw128(mh + mk), xdesc, id_y, kk > 0 ? 1u : 0u);
-            umma_bf16(tmem + kSsdColDiag, umma_desc_sw128(ml + mk), xdesc, id_y, 1u);
+            for (int kk = 0; kk < kSsdQ / 16; ++kk) {
+                const uint32_t mk = (kk >> 2) * (kSsdQ * 128) + (kk & 3) * 32;
+                const uint64_t xdesc = umma_desc_sw128_mn(xa + kk * 2048, 0);
+                umma_bf16(tmem + kSsdColDiag, umma_desc_sw128(mh + mk), xdesc, id_y, kk > 0 ? 1u : 0u);
+                umma_bf16(tmem + kSsdColDiag, umma_desc_sw128(ml + mk), xdesc, id_y, 1u);
+            }
+            umma_commit(&bars[2]);
         }
-        umma_commit(&bars[2]);
+    }
+    const bool issued2 = __syncthreads_and(x_loaded) && g_ready;
+    // the gate's z row, requested while the product runs
+    const int64_t t = t0 + i;
+    const int64_t row = (static_cast<int64_t>(b) * p.L + (t < p.L ? t : 0)) * (static_cast<int64_t>(p.H) * kSsdP) +
+                        h * kSsdP;
+    uint4 zr[8];
+    if (p.z && t < p.L) {
+        const uint4* zs = reinterpret_cast<const uint4*>(p.z + row);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) zr[q] = zs[q];
     }
     bool y_ok = false;
-    if (g_ready) y_ok = mbar_wait_bounded(&bars[2], 0, p.wait_limit);
+    if (issued2) y_ok = mbar_wait_bounded(&bars[2], 0, p.wait_limit);
     tc_fence_after();
     const bool y_ready = __syncthreads_and(y_ok);
 
     // y_i = (M X)_i + exp(cum_i) (C H_in^T)_i, gated; the tensor-memory loads
     // are warp-wide, so every lane takes part and only in-sequence rows store
-    const int64_t t = t0 + i;
     if (y_ready) {
         const float e = ex2_fast(cum2[i]);
-        const int64_t row = (static_cast<int64_t>(b) * p.L + (t < p.L ? t : 0)) * (static_cast<int64_t>(p.H) * kSsdP) +
-                            h * kSsdP;
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {     // unrolled: zr is indexed by it
             float yo[32], yd[32];
             tmem_ld32(lane_base + kSsdColOff + half * 32, yo);
             tmem_ld32(lane_base + kSsdColDiag + half * 32, yd);
             if (t < p.L) {
-                float gz[32];
-                if (p.z) {
-                    const uint4* zs = reinterpret_cast<const uint4*>(p.z + row + half * 32);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint4 v = zs[q];
-                        const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                        for (int e2 = 0; e2 < 8; ++e2) {
-                            const float zv = (e2 & 1) ? bf16_hi(wd[e2 >> 1]) : bf16_lo(wd[e2 >> 1]);
-                            gz[q * 8 + e2] = zv / (1.0f + expf(-zv));
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) gz[q] = 1.0f;
-                }
                 uint4* dst = reinterpret_cast<uint4*>(p.y + row + half * 32);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     float o[8];
 #pragma unroll
-                    for (int e2 = 0; e2 < 8; ++e2) o[e2] = fmaf(e, yo[q * 8 + e2], yd[q * 8 + e2]) * gz[q * 8 + e2];
+                    for (int e2 = 0; e2 < 8; ++e2) o[e2] = fmaf(e, yo[q * 8 + e2], yd[q * 8 + e2]);
+                    if (p.z) {
+                        // SiLU(z) = z / (1 + 2^(-z log2 e))
+                        const uint4 zv = zr[half * 4 + q];
+                        const float zf[8] = {bf16_lo(zv.x), bf16_hi(zv.x), bf16_lo(zv.y), bf16_hi(zv.y),
+                                             bf16_lo(zv.z), bf16_hi(zv.z), bf16_lo(zv.w), bf16_hi(zv.w)};
+#pragma unroll
+                        for (int e2 = 0; e2 < 8; ++e2)
+                            o[e2] *= __fdividef(zf[e2], 1.0f + ex2_fast(-zf[e2] * kLog2e));
+                    }
                     uint4 w;
                     w.x = pack_bf16x2(o[0], o[1]);
                     w.y = pack_bf16x2(o[2], o[3]);
@@ -520,7 +535,8 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
         if (warp == 1 && elect_one_lane()) {
             if (!loaded) mbar_wait_bounded(&bars[0], 0, 1u << 20);
             if (issued1) mbar_wait_bounded(&bars[1], 0, 1u << 20);
-            if (g_ready) mbar_wait_bounded(&bars[2], 0, 1u << 20);
+            if (x_issued && !x_done) mbar_wait_bounded(&bars[3], 0, 1u << 20);
+            if (issued2) mbar_wait_bounded(&bars[2], 0, 1u << 20);
         }
     }
     tc_fence_before();
