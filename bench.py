@@ -34,11 +34,12 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from workloads import CONFIGS, make_decode_inputs, make_mixer_inputs  # noqa: E402
+from workloads import CONFIGS, SSD_CONFIGS, make_decode_inputs, make_mixer_inputs, make_ssd_inputs  # noqa: E402
 
 METRIC = "Mamba mixer tokens/s per layer (d_inner 8192) and % of B200 HBM roofline"
 PREFILL = CONFIGS["jamba_prefill"]
 DECODE = CONFIGS["decode_28x128"]
+SSD = SSD_CONFIGS["mamba2_prefill"]
 
 SMS = 148
 FP32_LANES_PER_SM = 128
@@ -87,6 +88,7 @@ TRAFFIC_SOURCES = {
     "state_update_kernel/decode_28x128": ("mixer_decode.cuh", "mixer_common.cuh", "mixer_api.cu"),
     "proj_gemm/x_proj": ("proj_gemm.cuh", "mixer_common.cuh", "mixer_api.cu"),
     "proj_gemm/dt_proj": ("proj_gemm.cuh", "mixer_common.cuh", "mixer_api.cu"),
+    "ssd/mamba2_prefill": ("ssd.cuh", "proj_gemm.cuh", "mixer_common.cuh", "mixer_api.cu"),
 }
 
 
@@ -323,6 +325,9 @@ def run_gpu(args):
     # mixer with its producers (conv -> x_proj -> norms -> dt_proj -> scan)
     proj = run_projections(mm, args, world, hbm_peak, hbm_src, peaks)
 
+    # ---- the Mamba-2 form (scalar decay per head, chunked products on the tensor cores)
+    ssd = run_ssd(mm, args, world, hbm_peak, hbm_src, peaks)
+
     result = None
     if rank == 0:
         cpu = cpu_baseline(host, cfg) if world == 1 and not args.no_cpu_baseline else None
@@ -359,6 +364,7 @@ def run_gpu(args):
             "general_a": gen,
             "bc_rmsnorm": normed,
             "projections": proj,
+            "mamba2_ssd": ssd,
             **legs,
             "launch_ms": {"mean": round(statistics.mean(launch_ms), 5), "min": round(min(launch_ms), 5),
                           "max": round(max(launch_ms), 5)},
@@ -678,6 +684,79 @@ def run_projections(mm, args, world, hbm_peak, hbm_src, peaks):
     return out
 
 
+def ssd_bytes(cfg):
+    """Algorithmic HBM bytes of one Mamba-2 forward call: x, z and y (bf16),
+    dt, B and C (bf16), h_last (fp32) and h0 when given, and the per-head
+    parameters, each moved once."""
+    B, L, H, P, N, G = cfg.batch, cfg.seqlen, cfg.heads, cfg.headdim, cfg.d_state, cfg.groups
+    act = B * L * H * P * 2
+    return (3 if cfg.gate else 2) * act + B * L * H * 2 + 2 * B * L * G * N * 2 + \
+        B * H * P * N * 4 * (2 if cfg.h0_std > 0 else 1) + 3 * H * 4
+
+
+def ssd_flops(cfg):
+    """The dense products of the chunked form, each counted once per
+    (chunk, head) over full 128-token chunks: G = C B^T (2 Q^2 N), M X
+    (2 Q^2 P), C H_in^T (2 Q N P) and the chunk state B^T (w x) (2 Q N P).
+    The kernels run the last three twice (hi and lo parts of their computed
+    operand); that doubling is not counted."""
+    Q = 128
+    chunks = -(-cfg.seqlen // Q)
+    per = 2 * Q * Q * cfg.d_state + 2 * Q * Q * cfg.headdim + 4 * Q * cfg.d_state * cfg.headdim
+    return float(cfg.batch * chunks * cfg.heads * per)
+
+
+def _ssd_call(mm, d, out, ws):
+    mm.ssd_fwd(d["x"], d["z"], d["dt"], d["dt_bias"], d["A"], d["Bm"], d["Cm"], d["Dskip"], d["h0"],
+               y=out[0], h_last=out[1], workspace=ws)
+
+
+def run_ssd(mm, args, world, hbm_peak, hbm_src, peaks):
+    """The Mamba-2 form (scalar decay per head, d_state 128, head dim 64, 128
+    heads: d_inner 8192) on 4096 tokens: three launches per call (chunk states,
+    state passing, chunk scan), inputs rotated over two sets larger than L2.
+    Roofline: algorithmic HBM bytes against the copy bandwidth, and the chunked
+    form's products against the dense bf16 rate."""
+    cfg = SSD
+    B, L, H = cfg.batch, cfg.seqlen, cfg.heads
+    if peaks and "bf16_tflops" in peaks:
+        tpeak, tsrc = float(peaks["bf16_tflops"]), "measured"
+    else:
+        tpeak, tsrc = BF16_FALLBACK_TFLOPS, "fallback"
+    host = make_ssd_inputs(cfg)
+    sets = [{k: (v.cuda() if v is not None else None) for k, v in host.items()} for _ in range(2)]
+    outs = [(torch.empty((B, L, H * cfg.headdim), dtype=torch.bfloat16, device="cuda"),
+             torch.empty((B, H, cfg.headdim, cfg.d_state), device="cuda")) for _ in range(2)]
+    ws = torch.empty(mm.ssd_workspace_size(B, L, H), dtype=torch.uint8, device="cuda")
+    it = [0]
+
+    def step():
+        i = it[0]
+        it[0] += 1
+        _ssd_call(mm, sets[i % 2], outs[i % 2], ws)
+
+    K = max(3, min(args.steps, 200))
+    ms = _time_loop(step, K, world)
+    nbytes = ssd_bytes(cfg)
+    flops = ssd_flops(cfg)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    tf = flops / (ms * 1e-3) / 1e12
+    status = mm.check_status(ws)
+    del sets, outs, ws
+    torch.cuda.empty_cache()
+    return {
+        "workload": cfg.name, "batch": B, "seq_len": L, "heads": H, "headdim": cfg.headdim,
+        "d_state": cfg.d_state, "groups": cfg.groups, "steps": K, "ms_per_step": round(ms, 5),
+        "value": round(_job_rate(world, B * L, ms), 1), "unit": "tokens/s", "launches_per_call": 3,
+        "status": status,
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(gbs / hbm_peak, 4), "traffic": _ncu_traffic("ssd/mamba2_prefill"),
+                     "algorithmic_bytes": nbytes, "peak_source": hbm_src},
+        "roofline_tensor": {"bound": "tensor", "achieved": round(tf, 1), "peak": tpeak, "unit": "TFLOP/s",
+                            "frac": round(tf / tpeak, 4), "algorithmic_flops": flops, "peak_source": tsrc},
+    }
+
+
 # ---------------------------------------------------------------- CPU oracle
 def cpu_baseline(host, cfg, target_s=12.0, sample_override=None, threads=None):
     """The fp64 oracle as it stands, on all host cores (or `threads` of
@@ -806,6 +885,13 @@ def run_only(args):
         ws = torch.empty(mm.proj_matmul_workspace_size(M, wmat.shape[0], lhs.shape[1]), dtype=torch.uint8,
                          device="cuda")
         step = lambda: mm.proj_matmul(lhs, wmat, out=o, workspace=ws)  # noqa: E731
+    elif args.only == "ssd":
+        cfg = SSD
+        d = {k: (v.cuda() if v is not None else None) for k, v in make_ssd_inputs(cfg).items()}
+        out = (torch.empty((cfg.batch, cfg.seqlen, cfg.heads * cfg.headdim), dtype=torch.bfloat16, device="cuda"),
+               torch.empty((cfg.batch, cfg.heads, cfg.headdim, cfg.d_state), device="cuda"))
+        ws = torch.empty(mm.ssd_workspace_size(cfg.batch, cfg.seqlen, cfg.heads), dtype=torch.uint8, device="cuda")
+        step = lambda: _ssd_call(mm, d, out, ws)  # noqa: E731
     elif args.only == "forward":
         cfg = PREFILL
         d = {k: (v.cuda() if v is not None else None)
@@ -845,7 +931,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra-prefill", action="store_true",
                     help="skip the 4 x 32768 and 262,144-token prefill legs")
-    ap.add_argument("--only", choices=["forward", "decode", "xproj", "dtproj"], default=None,
+    ap.add_argument("--only", choices=["forward", "decode", "xproj", "dtproj", "ssd"], default=None,
                     help="run one kernel's timed loop only (for profiler captures); prints no JSON line")
     ap.add_argument("--decode-layers", type=int, default=None,
                     help="with --only decode: stacked layers (default: the workload's 28)")

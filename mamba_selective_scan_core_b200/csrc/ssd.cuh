@@ -220,7 +220,8 @@ ssd_chunk_state_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm
         uint4* rh = reinterpret_cast<uint4*>(xh + j * 128);
         uint4* rl = reinterpret_cast<uint4*>(xl + j * 128);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int q0 = 0; q0 < 8; ++q0) {
+            const int q = q0 ^ (j & 7);     // lanes j..j+7 start on different banks
             const uint4 v = rh[q];
             uint4 hi, lo;
             split_bf16x2(w * bf16_lo(v.x), w * bf16_hi(v.x), hi.x, lo.x);
@@ -253,17 +254,24 @@ ssd_chunk_state_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm
     if (loaded) ok = mbar_wait_bounded(&bars[1], 0, p.wait_limit);
     tc_fence_after();
     if (__syncthreads_and(ok)) {
-        // thread n owns state row n: S[b][c][h][p][n] for p = 0..63 (a warp stores 32 consecutive n)
+        // thread n owns state row n; the [P][N] block S[b][c][h] is staged in
+        // B's tile (free now) and written out with coalesced 16-byte stores
         const int n = tid;
-        float* dst = p.S + ((static_cast<int64_t>(b) * p.chunks + c) * p.H + h) * (kSsdP * kSsdN) + n;
+        float* stage = reinterpret_cast<float*>(bt);
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
             float v[32];
             tmem_ld32(lane_base + half * 32, v);
 #pragma unroll
-            for (int q = 0; q < 32; ++q) dst[(half * 32 + q) * kSsdN] = v[q];
+            for (int q = 0; q < 32; ++q) stage[(half * 32 + q) * kSsdN + n] = v[q];
         }
+        __syncthreads();
+        float4* dst = reinterpret_cast<float4*>(p.S + ((static_cast<int64_t>(b) * p.chunks + c) * p.H + h) *
+                                                          (kSsdP * kSsdN));
+        const float4* src = reinterpret_cast<const float4*>(stage);
+#pragma unroll 4
+        for (int r = 0; r < kSsdP * kSsdN / 4 / kSsdThreads; ++r) dst[r * kSsdThreads + tid] = src[r * kSsdThreads + tid];
         if (tid == 0) p.dec[(static_cast<int64_t>(b) * p.H + h) * p.chunks + c] = ex2_fast(cum2[kSsdQ - 1]);
     } else {
         if (tid == 0) ssd_fail(p);
@@ -335,7 +343,7 @@ constexpr uint32_t kSsdColG = 0, kSsdColOff = 128, kSsdColDiag = 192, kSsdCols =
 __global__ void __launch_bounds__(kSsdThreads, 2)
 ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_c,
                       const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_h,
-                      const __grid_constant__ CUtensorMap tm_x)
+                      const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z)
 {
     using Lay = SsdScanLayout;
     extern __shared__ __align__(1024) unsigned char ssc_raw[];
@@ -404,11 +412,12 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
                 umma_bf16(tmem + kSsdColOff, adesc, umma_desc_sw128(hk + Lay::hin_bytes), id_o, 1u);
             }
             umma_commit(&bars[1]);
-            // C is free once these products complete: the x tile goes there,
-            // copied while M is built
+            // C is free once these products complete: the x tile (and the
+            // gate's z tile after it) go there, copied while M is built
             if (mbar_wait_bounded(&bars[1], 0, p.wait_limit)) {
-                mbar_arrive_expect_tx(&bars[3], kSsdQ * kSsdP * 2);
+                mbar_arrive_expect_tx(&bars[3], (p.z ? 2 : 1) * kSsdQ * kSsdP * 2);
                 tma_load_3d(ct, &tm_x, h * kSsdP, static_cast<int>(t0), b, &bars[3]);
+                if (p.z) tma_load_3d(ct + kSsdQ * kSsdP * 2, &tm_z, h * kSsdP, static_cast<int>(t0), b, &bars[3]);
                 x_issued = true;
             }
         }
@@ -478,53 +487,56 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
         }
     }
     const bool issued2 = __syncthreads_and(x_loaded) && g_ready;
-    // the gate's z row, requested while the product runs
-    const int64_t t = t0 + i;
-    const int64_t row = (static_cast<int64_t>(b) * p.L + (t < p.L ? t : 0)) * (static_cast<int64_t>(p.H) * kSsdP) +
-                        h * kSsdP;
-    uint4 zr[8];
-    if (p.z && t < p.L) {
-        const uint4* zs = reinterpret_cast<const uint4*>(p.z + row);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) zr[q] = zs[q];
-    }
     bool y_ok = false;
     if (issued2) y_ok = mbar_wait_bounded(&bars[2], 0, p.wait_limit);
     tc_fence_after();
     const bool y_ready = __syncthreads_and(y_ok);
 
-    // y_i = (M X)_i + exp(cum_i) (C H_in^T)_i, gated; the tensor-memory loads
-    // are warp-wide, so every lane takes part and only in-sequence rows store
+    // y_i = (M X)_i + exp(cum_i) (C H_in^T)_i, gated by SiLU of the copied z
+    // row; row i is staged over the x tile (free now) and the tile then goes
+    // out with coalesced 16-byte stores.  Rows are 128 bytes, their 16-byte
+    // pieces in the copies' swizzled order (piece q of row r at q ^ (r % 8)).
     if (y_ready) {
         const float e = ex2_fast(cum2[i]);
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {     // unrolled: zr is indexed by it
+        const unsigned char* zrow = ct + kSsdQ * kSsdP * 2 + i * 128;
+        unsigned char* yrow = ct + i * 128;
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
             float yo[32], yd[32];
             tmem_ld32(lane_base + kSsdColOff + half * 32, yo);
             tmem_ld32(lane_base + kSsdColDiag + half * 32, yd);
-            if (t < p.L) {
-                uint4* dst = reinterpret_cast<uint4*>(p.y + row + half * 32);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float o[8];
+            for (int q = 0; q < 4; ++q) {
+                const int piece = (half * 4 + q) ^ (i & 7);
+                float o[8];
 #pragma unroll
-                    for (int e2 = 0; e2 < 8; ++e2) o[e2] = fmaf(e, yo[q * 8 + e2], yd[q * 8 + e2]);
-                    if (p.z) {
-                        // SiLU(z) = z / (1 + 2^(-z log2 e))
-                        const uint4 zv = zr[half * 4 + q];
-                        const float zf[8] = {bf16_lo(zv.x), bf16_hi(zv.x), bf16_lo(zv.y), bf16_hi(zv.y),
-                                             bf16_lo(zv.z), bf16_hi(zv.z), bf16_lo(zv.w), bf16_hi(zv.w)};
+                for (int e2 = 0; e2 < 8; ++e2) o[e2] = fmaf(e, yo[q * 8 + e2], yd[q * 8 + e2]);
+                if (p.z) {
+                    // SiLU(z) = z / (1 + 2^(-z log2 e))
+                    const uint4 zv = *reinterpret_cast<const uint4*>(zrow + piece * 16);
+                    const float zf[8] = {bf16_lo(zv.x), bf16_hi(zv.x), bf16_lo(zv.y), bf16_hi(zv.y),
+                                         bf16_lo(zv.z), bf16_hi(zv.z), bf16_lo(zv.w), bf16_hi(zv.w)};
 #pragma unroll
-                        for (int e2 = 0; e2 < 8; ++e2)
-                            o[e2] *= __fdividef(zf[e2], 1.0f + ex2_fast(-zf[e2] * kLog2e));
-                    }
-                    uint4 w;
-                    w.x = pack_bf16x2(o[0], o[1]);
-                    w.y = pack_bf16x2(o[2], o[3]);
-                    w.z = pack_bf16x2(o[4], o[5]);
-                    w.w = pack_bf16x2(o[6], o[7]);
-                    dst[q] = w;
+                    for (int e2 = 0; e2 < 8; ++e2) o[e2] *= __fdividef(zf[e2], 1.0f + ex2_fast(-zf[e2] * kLog2e));
                 }
+                uint4 w;
+                w.x = pack_bf16x2(o[0], o[1]);
+                w.y = pack_bf16x2(o[2], o[3]);
+                w.z = pack_bf16x2(o[4], o[5]);
+                w.w = pack_bf16x2(o[6], o[7]);
+                *reinterpret_cast<uint4*>(yrow + piece * 16) = w;
+            }
+        }
+        __syncthreads();
+        // thread k: piece k % 8 of rows k / 8 + 16 m; only rows in the sequence
+        const int q = tid & 7;
+        const int64_t ld = static_cast<int64_t>(p.H) * kSsdP;
+#pragma unroll 4
+        for (int m = 0; m < kSsdQ / 16; ++m) {
+            const int r = (tid >> 3) + 16 * m;
+            if (t0 + r < p.L) {
+                const uint4 v = *reinterpret_cast<const uint4*>(ct + r * 128 + ((q ^ (r & 7)) << 4));
+                *reinterpret_cast<uint4*>(p.y + (static_cast<int64_t>(b) * p.L + t0 + r) * ld + h * kSsdP + q * 8) = v;
             }
         }
     }
