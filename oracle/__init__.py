@@ -60,6 +60,8 @@ def _declare(lib):
     lib.oracle_matmul_nt.argtypes = [P, P, P, I, I, I, I, I]
     lib.oracle_ssd_fwd.restype = ctypes.c_int
     lib.oracle_ssd_fwd.argtypes = [P] * 11 + [I] * 8
+    lib.oracle_m3_fwd.restype = ctypes.c_int
+    lib.oracle_m3_fwd.argtypes = [P] * 15 + [I] * 9
     return lib
 
 
@@ -311,6 +313,42 @@ def ssd_fwd(x, z, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, headdim: int = 64, thr
                                _p(y), _p(h_last), Bsz, L, H, P, N, G, rng[0], rng[1])
         if rc != 0:
             raise ValueError(f"oracle_ssd_fwd rejected its arguments (rc={rc})")
+
+    parts = _ranges(C, threads)
+    if len(parts) == 1:
+        run(parts[0])
+    else:
+        with ThreadPoolExecutor(max_workers=len(parts)) as ex:
+            list(ex.map(run, parts))
+    return {"y": y, "h_last": h_last}
+
+
+def m3_fwd(x, z, dt, trap, dt_bias, A, theta, Bm, Cm, Dskip, h0=None, x_prev=None, B_prev=None,
+           headdim: int = 64, threads: int = 1, library=None):
+    """Run the oracle of the Mamba-3 form (oracle_m3_fwd): x, z [B,L,R,H*P]
+    (z None: no gate), dt and trap [B,L,H] (trap None: 1/2), dt_bias [H] or
+    None, A [H], theta [H,N/2], Bm, Cm [B,L,R,G,N], Dskip [H] or None, h0
+    [B,H,P,N] or None, x_prev [B,R,H*P] and B_prev [B,R,G,N] (the token before
+    the call) or None, P = headdim.  Returns y [B,L,R,H*P] and h_last
+    [B,H,P,N] as float64 arrays."""
+    L_ = library or lib()
+    x, z, dt, trap, dt_bias, A, theta, Bm, Cm, Dskip, h0, x_prev, B_prev = map(
+        _f64, (x, z, dt, trap, dt_bias, A, theta, Bm, Cm, Dskip, h0, x_prev, B_prev))
+    Bsz, L, R, C = x.shape
+    H = A.shape[0]
+    P = int(headdim)
+    G, N = Bm.shape[3], Bm.shape[4]
+    assert C == H * P and dt.shape == (Bsz, L, H) and Bm.shape == (Bsz, L, R, G, N) and Cm.shape == Bm.shape
+    assert theta.shape == (H, N // 2)
+    y = np.zeros((Bsz, L, R, C))
+    h_last = np.zeros((Bsz, H, P, N))
+
+    def run(rng):
+        rc = L_.oracle_m3_fwd(_p(x), _p(z), _p(dt), _p(trap), _p(dt_bias), _p(A), _p(theta), _p(Bm), _p(Cm),
+                              _p(Dskip), _p(h0), _p(x_prev), _p(B_prev), _p(y), _p(h_last),
+                              Bsz, L, R, H, P, N, G, rng[0], rng[1])
+        if rc != 0:
+            raise ValueError(f"oracle_m3_fwd rejected its arguments (rc={rc})")
 
     parts = _ranges(C, threads)
     if len(parts) == 1:

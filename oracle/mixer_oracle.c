@@ -41,8 +41,10 @@
  *
  * Functions: oracle_mixer_fwd (the forward above), oracle_state_update (its
  * one-token decode step), oracle_rmsnorm_rows (the RMSNorm of B_t and C_t),
- * oracle_matmul_nt (the projections either side of the scan) and
- * oracle_ssd_fwd (the Mamba-2 form: one scalar decay per head, grouped B/C).
+ * oracle_matmul_nt (the projections either side of the scan),
+ * oracle_ssd_fwd (the Mamba-2 form: one scalar decay per head, grouped B/C)
+ * and oracle_m3_fwd (the Mamba-3 form: trapezoidal rule, rotating complex
+ * state, several inputs and outputs per state).
  */
 #include <math.h>
 #include <stdint.h>
@@ -311,6 +313,115 @@ int oracle_ssd_fwd(const double* x, const double* z, const double* dt, const dou
             }
 
             for (int64_t n = 0; n < N; ++n) h_last[(b * C + c) * N + n] = s[n];
+        }
+    }
+    return OR_OK;
+}
+
+/*
+ * Mamba-3 form (the lesson's "Mamba-3" section: exponential-trapezoidal
+ * discretisation, a complex-valued state equivalent to a data-dependent
+ * rotary embedding, and multi-input multi-output projections), on the
+ * Mamba-2 layout of heads, groups and channels.  Readings (the section gives
+ * no formula): the d_state entries of a channel form N/2 complex numbers
+ * (entries 2k, 2k+1 = real, imaginary part of pair k); per head h and token t
+ *
+ *     Delta_t  = softplus(dt_t[h] + dt_bias[h]),  lambda_t = trap_t[h] (0.5 when trap is NULL)
+ *     a_t[k]   = exp(Delta_t A[h]) * (cos(Delta_t theta[h,k]) + i sin(Delta_t theta[h,k]))
+ *     u_t[k]   = sum_r (B_t[r,g,2k] + i B_t[r,g,2k+1]) x_t[r,c]        (R inputs share the state)
+ *     s_t[k]   = a_t[k] (s_{t-1}[k] + (1 - lambda_t) Delta_t u_{t-1}[k]) + lambda_t Delta_t u_t[k]
+ *     y_t[r,c] = (sum_k Re(conj(C_t[r,g,k]) s_t[k]) + D[h] x_t[r,c]) * SiLU(z_t[r,c])   (no gate if z is NULL)
+ *
+ * The state input u enters through a two-tap (trapezoidal) rule inside the
+ * recurrence -- at lambda = 1 it is Mamba-2's Euler step, at 1/2 the
+ * trapezoid -- and u_{-1} comes from x_prev / B_prev (the token before the
+ * call; zero when NULL), so a sequence split into calls continues exactly.
+ *
+ *   x, z          [B, L, R, H*P]   (z may be NULL)
+ *   dt, trap      [B, L, H]        (trap may be NULL)
+ *   dt_bias       [H] or NULL;  A [H] (negative);  theta [H, N/2];  Dskip [H] or NULL
+ *   Bm, Cm        [B, L, R, G, N]
+ *   h0            [B, H, P, N] or NULL
+ *   x_prev        [B, R, H*P] or NULL;  B_prev [B, R, G, N] or NULL
+ * Outputs (only channels c in [c_begin, c_end) are written):
+ *   y             [B, L, R, H*P]
+ *   h_last        [B, H, P, N]
+ */
+int oracle_m3_fwd(const double* x, const double* z, const double* dt, const double* trap, const double* dt_bias,
+                  const double* A, const double* theta, const double* Bm, const double* Cm, const double* Dskip,
+                  const double* h0, const double* x_prev, const double* B_prev, double* y, double* h_last,
+                  int64_t Bsz, int64_t L, int64_t R, int64_t H, int64_t P, int64_t N, int64_t G,
+                  int64_t c_begin, int64_t c_end)
+{
+    if (Bsz < 0 || L < 0 || R < 1 || R > 16 || H < 1 || P < 1 || N < 2 || N > 256 || N % 2 != 0 || G < 1 ||
+        H % G != 0)
+        return OR_ERR_ARG;
+    const int64_t C = H * P, K = N / 2;
+    if (c_begin < 0 || c_end > C || c_begin > c_end) return OR_ERR_ARG;
+    if ((!x || !dt || !Bm || !Cm) && L > 0) return OR_ERR_ARG;
+    if (!A || !theta || !y || !h_last) return OR_ERR_ARG;
+
+    double sr[128], si[128];     /* state, pair k = sr[k] + i si[k] */
+    double ur[128], ui[128];     /* u of the previous token */
+
+    for (int64_t b = 0; b < Bsz; ++b) {
+        for (int64_t c = c_begin; c < c_end; ++c) {
+            const int64_t h = c / P;
+            const int64_t g = h * G / H;   /* the head's B/C group: H / G consecutive heads each */
+            for (int64_t k = 0; k < K; ++k) {
+                sr[k] = h0 ? h0[(b * C + c) * N + 2 * k] : 0.0;
+                si[k] = h0 ? h0[(b * C + c) * N + 2 * k + 1] : 0.0;
+                ur[k] = 0.0;
+                ui[k] = 0.0;
+                if (x_prev && B_prev) {
+                    for (int64_t r = 0; r < R; ++r) {
+                        const double xv = x_prev[(b * R + r) * C + c];
+                        const double* Bp = B_prev + ((b * R + r) * G + g) * N;
+                        ur[k] += Bp[2 * k] * xv;
+                        ui[k] += Bp[2 * k + 1] * xv;
+                    }
+                }
+            }
+
+            for (int64_t t = 0; t < L; ++t) {
+                const int64_t row = b * L + t;
+                const double delta = or_softplus(dt[row * H + h] + (dt_bias ? dt_bias[h] : 0.0));
+                const double lam = trap ? trap[row * H + h] : 0.5;
+                const double mag = exp(delta * A[h]);
+                for (int64_t k = 0; k < K; ++k) {
+                    /* u_t[k] = sum_r B_t[r] pair k * x_t[r] */
+                    double vr = 0.0, vi = 0.0;
+                    for (int64_t r = 0; r < R; ++r) {
+                        const double xv = x[(row * R + r) * C + c];
+                        const double* Bt = Bm + ((row * R + r) * G + g) * N;
+                        vr += Bt[2 * k] * xv;
+                        vi += Bt[2 * k + 1] * xv;
+                    }
+                    /* s = a (s + (1 - lambda) Delta u_prev) + lambda Delta u */
+                    const double pr = sr[k] + (1.0 - lam) * delta * ur[k];
+                    const double pi = si[k] + (1.0 - lam) * delta * ui[k];
+                    const double ang = delta * theta[h * K + k];
+                    const double ar = mag * cos(ang), ai = mag * sin(ang);
+                    sr[k] = ar * pr - ai * pi + lam * delta * vr;
+                    si[k] = ar * pi + ai * pr + lam * delta * vi;
+                    ur[k] = vr;
+                    ui[k] = vi;
+                }
+                for (int64_t r = 0; r < R; ++r) {
+                    const double* Ct = Cm + ((row * R + r) * G + g) * N;
+                    double acc = 0.0;
+                    for (int64_t k = 0; k < K; ++k) acc += Ct[2 * k] * sr[k] + Ct[2 * k + 1] * si[k];
+                    const double xv = x[(row * R + r) * C + c];
+                    const double yv = acc + (Dskip ? Dskip[h] : 0.0) * xv;
+                    const int64_t o = (row * R + r) * C + c;
+                    y[o] = z ? yv * or_silu(z[o]) : yv;
+                }
+            }
+
+            for (int64_t k = 0; k < K; ++k) {
+                h_last[(b * C + c) * N + 2 * k] = sr[k];
+                h_last[(b * C + c) * N + 2 * k + 1] = si[k];
+            }
         }
     }
     return OR_OK;

@@ -602,7 +602,193 @@ def pin_ssd_group_mapping(lib):
         np.testing.assert_array_equal(got["h_last"][:, heads], one["h_last"])
 
 
+# ---------------------------------------------------------------- Mamba-3 form
+def _m3_case(rng, Bsz, L, R, H, P, N, G, *, z=True, h0=True, prev=True, trap=True, dskip=True):
+    return dict(
+        x=rng.standard_normal((Bsz, L, R, H * P)),
+        z=rng.standard_normal((Bsz, L, R, H * P)) if z else None,
+        dt=0.4 * rng.standard_normal((Bsz, L, H)),
+        trap=rng.uniform(0.0, 1.0, (Bsz, L, H)) if trap else None,
+        dt_bias=rng.uniform(-3.0, 0.5, H),
+        A=-np.exp(rng.uniform(np.log(0.2), np.log(4.0), H)),
+        theta=rng.uniform(-3.0, 3.0, (H, N // 2)),
+        Bm=rng.standard_normal((Bsz, L, R, G, N)),
+        Cm=rng.standard_normal((Bsz, L, R, G, N)),
+        Dskip=rng.normal(1.0, 0.3, H) if dskip else None,
+        h0=0.5 * rng.standard_normal((Bsz, H, P, N)) if h0 else None,
+        x_prev=rng.standard_normal((Bsz, R, H * P)) if prev else None,
+        B_prev=rng.standard_normal((Bsz, R, G, N)) if prev else None,
+    )
+
+
+def _m3(lib, case, P, **kw):
+    return oracle.m3_fwd(case["x"], case["z"], case["dt"], case["trap"], case["dt_bias"], case["A"], case["theta"],
+                         case["Bm"], case["Cm"], case["Dskip"], case["h0"], case["x_prev"], case["B_prev"],
+                         headdim=P, library=lib, **kw)
+
+
+def _cplx(v):
+    """[..., N] real pairs (2k, 2k+1) as [..., N/2] complex numbers."""
+    return v[..., 0::2] + 1j * v[..., 1::2]
+
+
+def pin_m3_quadratic_form(lib):
+    """The Mamba-3 form against its materialised form, built with numpy's
+    complex arithmetic on tiny inputs.  With a_q = exp(Delta_q (A + i theta))
+    per state pair, token s's input u_s = sum_r b_s[r] x_s[r] reaches the
+    state after token t >= s with weight prod_{q=s+1..t} a_q times
+    lambda_s Delta_s (its own step) plus, when s < t, (1 - lambda_{s+1})
+    Delta_{s+1} (the next step's trapezoid tap); h0 and the previous call's
+    input u_{-1} (weight (1 - lambda_0) Delta_0) reach it through
+    prod_{q=0..t} a_q.  y reads Re(conj(c) s)."""
+    rng = np.random.default_rng(97)
+    Bsz, L, R, H, P, N, G = 2, 9, 2, 4, 2, 6, 2
+    for trap in (True, False):          # no trap input: the plain trapezoid, lambda = 1/2
+        _m3_quadratic_case(lib, _m3_case(rng, Bsz, L, R, H, P, N, G, trap=trap), P, G)
+
+
+def _m3_quadratic_case(lib, case, P, G):
+    got = _m3(lib, case, P)
+    Bsz, L, R, C = case["x"].shape
+    H = case["A"].shape[0]
+    for b in range(Bsz):
+        for h in range(H):
+            g = h // (H // G)
+            delta = lib_softplus(case["dt"][b, :, h] + case["dt_bias"][h])
+            lam = case["trap"][b, :, h] if case["trap"] is not None else np.full(L, 0.5)
+            la = delta[:, None] * (case["A"][h] + 1j * case["theta"][h][None, :])     # [L, K] log of a_q
+            cum = np.cumsum(la, axis=0)
+            bb = _cplx(case["Bm"][b, :, :, g, :])          # [L, R, K]
+            cc = _cplx(case["Cm"][b, :, :, g, :])
+            bp = _cplx(case["B_prev"][b, :, g, :])           # [R, K]
+            for p in range(P):
+                c = h * P + p
+                xs = case["x"][b, :, :, c]                   # [L, R]
+                u = np.einsum("lrk,lr->lk", bb, xs)          # [L, K]
+                u_prev = np.einsum("rk,r->k", bp, case["x_prev"][b, :, c])
+                s0 = _cplx(case["h0"][b, h, p])
+                states = []
+                for t in range(L):
+                    st = np.exp(cum[t]) * (s0 + (1 - lam[0]) * delta[0] * u_prev)
+                    for s_ in range(t + 1):
+                        w = lam[s_] * delta[s_] + ((1 - lam[s_ + 1]) * delta[s_ + 1] if s_ < t else 0.0)
+                        st = st + np.exp(cum[t] - cum[s_]) * w * u[s_]
+                    states.append(st)
+                    for r in range(R):
+                        yv = np.real(np.sum(np.conj(cc[t, r]) * st)) + case["Dskip"][h] * xs[t, r]
+                        yv = yv * lib_silu(case["z"][b, t, r, c])
+                        np.testing.assert_allclose(got["y"][b, t, r, c], yv, rtol=1e-9, atol=1e-10)
+                hl = got["h_last"][b, h, p]
+                np.testing.assert_allclose(hl[0::2] + 1j * hl[1::2], states[-1], rtol=1e-9, atol=1e-10)
+
+
+def pin_m3_rotary_equivalence(lib):
+    """The complex state is a data-dependent rotary embedding: with the
+    rotation frequencies theta, the run equals the theta = 0 run on B and C
+    rotated by the cumulative phase Phi_t = theta * sum_{q<=t} Delta_q
+    (numpy's complex exp), its final state rotated back by Phi_{L-1}.  One
+    head per group, since the phase belongs to the head."""
+    rng = np.random.default_rng(101)
+    Bsz, L, R, H, P, N, G = 1, 14, 2, 2, 3, 8, 2
+    case = _m3_case(rng, Bsz, L, R, H, P, N, G)
+    got = _m3(lib, case, P)
+    rot = dict(case, theta=np.zeros_like(case["theta"]), Bm=case["Bm"].copy(), Cm=case["Cm"].copy())
+    phases = []
+    for h in range(H):
+        delta = lib_softplus(case["dt"][0, :, h] + case["dt_bias"][h])
+        phi = np.cumsum(delta)[:, None] * case["theta"][h][None, :]        # [L, K]
+        phases.append(phi)
+        e = np.exp(-1j * phi)                                                # [L, K]
+        for M_ in ("Bm", "Cm"):
+            v = _cplx(case[M_][0, :, :, h, :]) * e[:, None, :]
+            rot[M_][0, :, :, h, 0::2] = v.real
+            rot[M_][0, :, :, h, 1::2] = v.imag
+    plain = _m3(lib, rot, P)
+    np.testing.assert_allclose(got["y"], plain["y"], rtol=1e-9, atol=1e-10)
+    for h in range(H):
+        back = _cplx(plain["h_last"][0, h]) * np.exp(1j * phases[h][-1])[None, :]
+        np.testing.assert_allclose(_cplx(got["h_last"][0, h]), back, rtol=1e-9, atol=1e-10)
+
+
+def pin_m3_euler_is_mamba2(lib):
+    """With lambda = 1, theta = 0 and one input (R = 1) the form is the
+    Mamba-2 recurrence (oracle_ssd_fwd, pinned on its own)."""
+    rng = np.random.default_rng(103)
+    Bsz, L, H, P, N, G = 2, 11, 4, 3, 6, 2
+    case = _m3_case(rng, Bsz, L, 1, H, P, N, G)
+    case.update(trap=np.ones((Bsz, L, H)), theta=np.zeros((H, N // 2)))
+    got = _m3(lib, case, P)
+    ref = oracle.ssd_fwd(case["x"][:, :, 0], case["z"][:, :, 0], case["dt"], case["dt_bias"], case["A"],
+                         case["Bm"][:, :, 0], case["Cm"][:, :, 0], case["Dskip"], case["h0"], headdim=P,
+                         library=lib)
+    np.testing.assert_allclose(got["y"][:, :, 0], ref["y"], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(got["h_last"], ref["h_last"], rtol=1e-12, atol=1e-13)
+
+
+def pin_m3_mimo_superposition(lib):
+    """The R inputs share one state, which is linear in them: with no gate,
+    the rank-2 run's output r equals the sum of two single-input runs (input
+    0 with h0 and its previous token, input 1 with neither), both read out
+    with output r's C and no skip, plus D x_r; its final state is the sum of
+    theirs."""
+    rng = np.random.default_rng(107)
+    Bsz, L, H, P, N, G = 1, 10, 2, 2, 4, 1
+    case = _m3_case(rng, Bsz, L, 2, H, P, N, G, z=False)
+    got = _m3(lib, case, P)
+    for r_out in range(2):
+        total_y = np.zeros((Bsz, L, H * P))
+        total_h = np.zeros((Bsz, H, P, N))
+        for r_in in range(2):
+            one = dict(case, x=case["x"][:, :, r_in:r_in + 1], Bm=case["Bm"][:, :, r_in:r_in + 1],
+                       Cm=case["Cm"][:, :, r_out:r_out + 1], Dskip=None,
+                       h0=case["h0"] if r_in == 0 else None,
+                       x_prev=case["x_prev"][:, r_in:r_in + 1], B_prev=case["B_prev"][:, r_in:r_in + 1])
+            o = _m3(lib, one, P)
+            total_y += o["y"][:, :, 0]
+            total_h += o["h_last"]
+        want = total_y + case["Dskip"].repeat(P)[None, None, :] * case["x"][:, :, r_out]
+        np.testing.assert_allclose(got["y"][:, :, r_out], want, rtol=1e-10, atol=1e-11)
+        np.testing.assert_allclose(got["h_last"], total_h, rtol=1e-10, atol=1e-11)
+
+
+def pin_m3_split_equals_unsplit(lib):
+    """Two calls, the first one's final state carried as h0 and its last
+    token's x and B passed as x_prev / B_prev, equal the single run exactly."""
+    rng = np.random.default_rng(109)
+    P = 2
+    case = _m3_case(rng, 2, 15, 2, 4, P, 6, 2)
+    full = _m3(lib, case, P)
+    cut = 6
+
+    def part(lo, hi, h0, xp, bp):
+        c = dict(case)
+        for k in ("x", "z", "dt", "trap", "Bm", "Cm"):
+            c[k] = case[k][:, lo:hi]
+        c.update(h0=h0, x_prev=xp, B_prev=bp)
+        return _m3(lib, c, P)
+
+    first = part(0, cut, case["h0"], case["x_prev"], case["B_prev"])
+    second = part(cut, 15, first["h_last"], case["x"][:, cut - 1], case["Bm"][:, cut - 1])
+    np.testing.assert_array_equal(np.concatenate([first["y"], second["y"]], axis=1), full["y"])
+    np.testing.assert_array_equal(second["h_last"], full["h_last"])
+
+
+def pin_m3_zero_input(lib):
+    """x = 0, no h0 and no previous token give y = 0 and a zero state."""
+    rng = np.random.default_rng(113)
+    case = _m3_case(rng, 1, 7, 2, 2, 2, 4, 1, h0=False, prev=False)
+    case["x"] = np.zeros_like(case["x"])
+    got = _m3(lib, case, 2)
+    assert np.all(got["y"] == 0.0) and np.all(got["h_last"] == 0.0)
+
+
 ALL_PINS = [
+    pin_m3_quadratic_form,
+    pin_m3_rotary_equivalence,
+    pin_m3_euler_is_mamba2,
+    pin_m3_mimo_superposition,
+    pin_m3_split_equals_unsplit,
+    pin_m3_zero_input,
     pin_ssd_quadratic_form,
     pin_ssd_first_order_iir,
     pin_ssd_zero_input,

@@ -2,7 +2,8 @@
 that each one makes at least one pin fail, so the pins really constrain every
 step of the oracle: conv, SiLU, softplus, discretisation, recurrence, readout,
 skip, gate, carried state, the decode step, the RMSNorm of B and C, the projection product
-and the Mamba-2 form (scalar decay per head, grouped B/C)."""
+the Mamba-2 form (scalar decay per head, grouped B/C) and the Mamba-3 form
+(trapezoidal rule, rotating complex state, several inputs and outputs)."""
 
 import os
 
@@ -69,16 +70,44 @@ MUTANTS = [
      "acc += Ct[n] * s[n];\n                    s[n] = decay * s[n] + delta * Bt[n] * xv;"),
     ("ssd_C_as_B", "acc += Ct[n] * s[n];", "acc += Bt[n] * s[n];"),
     ("ssd_group_interleaved", "const int64_t g = h / heads_per_group;", "const int64_t g = h % G;"),
-    ("ssd_skip_dropped", "const double yv = acc + (Dskip ? Dskip[h] : 0.0) * xv;", "const double yv = acc;"),
+    ("ssd_skip_dropped", "const double yv = acc + (Dskip ? Dskip[h] : 0.0) * xv;\n                y[row * C + c]",
+     "const double yv = acc;\n                y[row * C + c]"),
     ("ssd_gate_by_z", "y[row * C + c] = z ? yv * or_silu(z[row * C + c]) : yv;",
      "y[row * C + c] = z ? yv * z[row * C + c] : yv;"),
-    ("ssd_dt_bias_of_head0", "or_softplus(dt[row * H + h] + (dt_bias ? dt_bias[h] : 0.0))",
-     "or_softplus(dt[row * H + h] + (dt_bias ? dt_bias[0] : 0.0))"),
-    ("ssd_dt_of_channel", "or_softplus(dt[row * H + h] +", "or_softplus(dt[row * H + c % H] +"),
+    ("ssd_dt_bias_of_head0", "or_softplus(dt[row * H + h] + (dt_bias ? dt_bias[h] : 0.0));\n                const double decay",
+     "or_softplus(dt[row * H + h] + (dt_bias ? dt_bias[0] : 0.0));\n                const double decay"),
+    ("ssd_dt_of_channel", "or_softplus(dt[row * H + h] + (dt_bias ? dt_bias[h] : 0.0));\n                const double decay",
+     "or_softplus(dt[row * H + c % H] + (dt_bias ? dt_bias[h] : 0.0));\n                const double decay"),
     ("ssd_h0_ignored", "s[n] = h0 ? h0[(b * C + c) * N + n] : 0.0;", "s[n] = 0.0;"),
-    ("ssd_head_of_channel", "const int64_t h = c / P;", "const int64_t h = c % H;"),
+    ("ssd_head_of_channel", "const int64_t h = c / P;\n            const int64_t g = h / heads_per_group;",
+     "const int64_t h = c % H;\n            const int64_t g = h / heads_per_group;"),
     ("ssd_h_last_not_written", "for (int64_t n = 0; n < N; ++n) h_last[(b * C + c) * N + n] = s[n];",
      "for (int64_t n = 0; n < N; ++n) h_last[(b * C + c) * N + n] = 0.0;"),
+    ("m3_lambda_swapped", "const double pr = sr[k] + (1.0 - lam) * delta * ur[k];",
+     "const double pr = sr[k] + lam * delta * ur[k];"),
+    ("m3_trapezoid_tap_undecayed",
+     "sr[k] = ar * pr - ai * pi + lam * delta * vr;",
+     "sr[k] = ar * sr[k] - ai * si[k] + (1.0 - lam) * delta * ur[k] + lam * delta * vr;"),
+    ("m3_rotation_sign", "const double ar = mag * cos(ang), ai = mag * sin(ang);",
+     "const double ar = mag * cos(ang), ai = -mag * sin(ang);"),
+    ("m3_rotation_dropped", "const double ar = mag * cos(ang), ai = mag * sin(ang);",
+     "const double ar = mag, ai = 0.0 * ang;"),
+    ("m3_readout_imag_dropped", "acc += Ct[2 * k] * sr[k] + Ct[2 * k + 1] * si[k];", "acc += Ct[2 * k] * sr[k];"),
+    ("m3_pairs_as_halves", "vr += Bt[2 * k] * xv;\n                        vi += Bt[2 * k + 1] * xv;",
+     "vr += Bt[k] * xv;\n                        vi += Bt[k + K] * xv;"),
+    ("m3_prev_input_not_kept", "                    ur[k] = vr;\n                    ui[k] = vi;\n", ""),
+    ("m3_x_prev_ignored", "if (x_prev && B_prev) {", "if (0) {"),
+    ("m3_mimo_first_input_only", "for (int64_t r = 0; r < R; ++r) {\n                        const double xv = x[(row * R + r) * C + c];\n                        const double* Bt",
+     "for (int64_t r = 0; r < 1; ++r) {\n                        const double xv = x[(row * R + r) * C + c];\n                        const double* Bt"),
+    ("m3_readout_with_first_C", "const double* Ct = Cm + ((row * R + r) * G + g) * N;",
+     "const double* Ct = Cm + ((row * R + 0) * G + g) * N;"),
+    ("m3_trap_default", "const double lam = trap ? trap[row * H + h] : 0.5;", "const double lam = trap ? trap[row * H + h] : 1.0;"),
+    ("m3_theta_of_head0", "const double ang = delta * theta[h * K + k];", "const double ang = delta * theta[k];"),
+    ("m3_h_last_imag_part", "h_last[(b * C + c) * N + 2 * k + 1] = si[k];", "h_last[(b * C + c) * N + 2 * k + 1] = sr[k];"),
+    ("m3_group_interleaved", "const int64_t g = h * G / H;",
+     "const int64_t g = h % G;"),
+    ("m3_skip_dropped", "const double yv = acc + (Dskip ? Dskip[h] : 0.0) * xv;\n                    const int64_t o",
+     "const double yv = acc;\n                    const int64_t o"),
 ]
 
 

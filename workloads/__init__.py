@@ -19,6 +19,10 @@ from .synth import (  # noqa: F401
     SSD_CONFIGS,
     make_ssd_inputs,
     make_ssd_inputs_custom,
+    M3Config,
+    M3_CONFIGS,
+    make_m3_inputs,
+    make_m3_inputs_custom,
     sample_channels,
     subset_channels,
 )

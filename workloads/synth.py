@@ -44,6 +44,7 @@ _BLOCK = 1 << 22  # elements per independently seeded block
 _T_XZ, _T_DT, _T_B, _T_C, _T_CONVW, _T_DTB, _T_D, _T_H0, _T_SSM, _T_CONVS, _T_X, _T_Z, _T_CONVB, _T_A = range(14)
 _T_BNORM, _T_CNORM, _T_WX, _T_WDT, _T_DTNORM = 14, 15, 16, 17, 18
 _T_SSD_X, _T_SSD_Z, _T_SSD_DT, _T_SSD_B, _T_SSD_C, _T_SSD_DTB, _T_SSD_A, _T_SSD_D, _T_SSD_H0 = range(19, 28)
+_T_M3_TRAP, _T_M3_THETA, _T_M3_XP, _T_M3_BP = range(28, 32)
 
 
 def _threads() -> int:
@@ -378,3 +379,79 @@ def make_projection_weights(d_inner: int, dt_rank: int = 256, d_state: int = 16,
     wn = _uniform((dt_rank,), seed, _T_DTNORM, 0.5, 1.5)
     return _act(wx, "bf16"), _act(wdt, "bf16"), torch.from_numpy(wn)
 
+
+
+@dataclass(frozen=True)
+class M3Config:
+    """A prefill of the Mamba-3 form: H heads of P channels, each channel's
+    d_state entries as d_state/2 complex numbers, R inputs and outputs
+    sharing a state (R = 1: single input)."""
+    name: str
+    batch: int
+    seqlen: int
+    heads: int
+    headdim: int = 64
+    d_state: int = 16
+    groups: int = 1
+    rank: int = 1
+    seed: int = 0
+    h0_std: float = 0.0
+    prev: bool = False
+    gate: bool = True
+    desc: str = ""
+
+    @property
+    def d_inner(self) -> int:
+        return self.heads * self.headdim
+
+    @property
+    def tokens(self) -> int:
+        return self.batch * self.seqlen
+
+
+M3_CONFIGS = {
+    "mamba3_prefill": M3Config(
+        "mamba3_prefill", batch=1, seqlen=4096, heads=128, seed=7,
+        desc="Mamba-3 form at the Jamba width: 128 heads of 64, d_state 16 (8 complex pairs), one input"),
+    "mamba3_mimo": M3Config(
+        "mamba3_mimo", batch=1, seqlen=4096, heads=128, rank=4, seed=8, h0_std=0.1, prev=True,
+        desc="Mamba-3 form with 4 inputs and outputs per state, an initial state and a previous token"),
+}
+
+
+def make_m3_inputs_custom(batch, seqlen, heads, headdim=64, d_state=16, groups=1, rank=1, seed=0, h0_std=0.0,
+                          prev=False, gate=True, trap=True, dt_std=0.1):
+    """Seeded inputs of the Mamba-3 form as CPU torch tensors.
+
+    x, z [B,L,R,H*P] ~ N(0,1) (bf16; z None without the gate), dt [B,L,H] ~
+    dt_std N(0,1) (bf16), trap [B,L,H] ~ U(0,1) (bf16; None: 1/2),
+    Bm/Cm [B,L,R,G,N] ~ N(0,1) (bf16); per head dt_bias = inverse-softplus of
+    a log-uniform [1e-3, 1e-1] step, A = -exp(U(ln 1, ln 16)), D ~ N(1, 0.1),
+    rotation frequencies theta [H, N/2] ~ U(-2, 2) (fp32); h0 [B,H,P,N] ~
+    h0_std N(0,1) fp32 or None; x_prev [B,R,H*P] and B_prev [B,R,G,N] ~ N(0,1)
+    (bf16) when prev."""
+    B, L, H, P, N, G, R = batch, seqlen, heads, headdim, d_state, groups, rank
+    s = seed
+    out = {}
+    out["x"] = _act(_normal((B, L, R, H * P), s, _T_SSD_X), "bf16")
+    out["z"] = _act(_normal((B, L, R, H * P), s, _T_SSD_Z), "bf16") if gate else None
+    out["dt"] = _act(_normal((B, L, H), s, _T_SSD_DT, std=dt_std), "bf16")
+    out["trap"] = _act(_uniform((B, L, H), s, _T_M3_TRAP, 0.0, 1.0), "bf16") if trap else None
+    out["Bm"] = _act(_normal((B, L, R, G, N), s, _T_SSD_B), "bf16")
+    out["Cm"] = _act(_normal((B, L, R, G, N), s, _T_SSD_C), "bf16")
+    out["dt_bias"] = torch.from_numpy(_dt_bias((H,), s, _T_SSD_DTB))
+    u = _uniform((H,), s, _T_SSD_A, 0.0, math.log(16.0))
+    out["A"] = torch.from_numpy((-np.exp(u.astype(np.float64))).astype(np.float32))
+    out["theta"] = torch.from_numpy(_uniform((H, N // 2), s, _T_M3_THETA, -2.0, 2.0))
+    out["Dskip"] = torch.from_numpy(_normal((H,), s, _T_SSD_D, std=0.1, mean=1.0))
+    out["h0"] = torch.from_numpy(_normal((B, H, P, N), s, _T_SSD_H0, std=h0_std)) if h0_std > 0 else None
+    out["x_prev"] = _act(_normal((B, R, H * P), s, _T_M3_XP), "bf16") if prev else None
+    out["B_prev"] = _act(_normal((B, R, G, N), s, _T_M3_BP), "bf16") if prev else None
+    return out
+
+
+def make_m3_inputs(cfg: M3Config, **overrides):
+    kw = dict(batch=cfg.batch, seqlen=cfg.seqlen, heads=cfg.heads, headdim=cfg.headdim, d_state=cfg.d_state,
+              groups=cfg.groups, rank=cfg.rank, seed=cfg.seed, h0_std=cfg.h0_std, prev=cfg.prev, gate=cfg.gate)
+    kw.update(overrides)
+    return make_m3_inputs_custom(**kw)
