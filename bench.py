@@ -34,12 +34,15 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from workloads import CONFIGS, SSD_CONFIGS, make_decode_inputs, make_mixer_inputs, make_ssd_inputs  # noqa: E402
+from workloads import (CONFIGS, M3_CONFIGS, SSD_CONFIGS, make_decode_inputs, make_m3_inputs,  # noqa: E402
+                       make_mixer_inputs, make_ssd_inputs)
 
 METRIC = "Mamba mixer tokens/s per layer (d_inner 8192) and % of B200 HBM roofline"
 PREFILL = CONFIGS["jamba_prefill"]
 DECODE = CONFIGS["decode_28x128"]
 SSD = SSD_CONFIGS["mamba2_prefill"]
+M3 = M3_CONFIGS["mamba3_prefill"]
+M3_MIMO = M3_CONFIGS["mamba3_mimo"]
 
 SMS = 148
 FP32_LANES_PER_SM = 128
@@ -328,6 +331,9 @@ def run_gpu(args):
     # ---- the Mamba-2 form (scalar decay per head, chunked products on the tensor cores)
     ssd = run_ssd(mm, args, world, hbm_peak, hbm_src, peaks)
 
+    # ---- the Mamba-3 form (trapezoidal rule, rotating complex state), single input and rank 4
+    m3 = {cfg.name: run_m3(mm, args, world, hbm_peak, hbm_src, alu_peak, cfg) for cfg in (M3, M3_MIMO)}
+
     result = None
     if rank == 0:
         cpu = cpu_baseline(host, cfg) if world == 1 and not args.no_cpu_baseline else None
@@ -365,6 +371,7 @@ def run_gpu(args):
             "bc_rmsnorm": normed,
             "projections": proj,
             "mamba2_ssd": ssd,
+            "mamba3": m3,
             **legs,
             "launch_ms": {"mean": round(statistics.mean(launch_ms), 5), "min": round(min(launch_ms), 5),
                           "max": round(max(launch_ms), 5)},
@@ -757,6 +764,71 @@ def run_ssd(mm, args, world, hbm_peak, hbm_src, peaks):
     }
 
 
+M3_KEYS = ("x", "z", "dt", "trap", "dt_bias", "A", "theta", "Bm", "Cm", "Dskip", "h0", "x_prev", "B_prev")
+
+
+def m3_bytes(cfg):
+    """Algorithmic HBM bytes of one Mamba-3 forward call: x, z and y
+    (R x tokens x d_inner bf16), dt and the trapezoid weight (per token and
+    head, bf16), B and C (R x tokens x groups x d_state bf16), h_last (fp32),
+    h0 and the previous token's x and B when given, and the parameters."""
+    B, L, H, P, N, G, R = cfg.batch, cfg.seqlen, cfg.heads, cfg.headdim, cfg.d_state, cfg.groups, cfg.rank
+    act = B * L * R * H * P * 2
+    return (3 if cfg.gate else 2) * act + 2 * B * L * H * 2 + 2 * B * L * R * G * N * 2 + \
+        B * H * P * N * 4 * (2 if cfg.h0_std > 0 else 1) + \
+        (B * R * (H * P + G * N) * 2 if cfg.prev else 0) + (3 * H + H * N // 2) * 4
+
+
+def m3_fp32_ops(cfg):
+    """FP32-pipe work per token and channel of the recurrence: per complex
+    pair the trapezoid tap (2), the rotation-decay product (4), the new
+    input (2) and, per input, its state input (2) and, per output, the
+    readout (2); plus per input/output the skip and gate (2)."""
+    pairs = cfg.d_state // 2
+    return pairs * (8 + 4 * cfg.rank) + 2 * cfg.rank
+
+
+def run_m3(mm, args, world, hbm_peak, hbm_src, alu_peak, cfg):
+    """The Mamba-3 form on 4096 tokens of 128 heads (d_state 16): a summary
+    pass and a full pass per call (fp32 recurrence on the CUDA cores), inputs
+    rotated over two sets.  Roofline: algorithmic HBM bytes against the copy
+    bandwidth, and the recurrence's FP32 work against the derived FP32 peak."""
+    B, L, H = cfg.batch, cfg.seqlen, cfg.heads
+    host = make_m3_inputs(cfg)
+    sets = [{k: (v.cuda() if v is not None else None) for k, v in host.items()} for _ in range(2)]
+    outs = [(torch.empty((B, L, cfg.rank, H * cfg.headdim), dtype=torch.bfloat16, device="cuda"),
+             torch.empty((B, H, cfg.headdim, cfg.d_state), device="cuda")) for _ in range(2)]
+    ws = torch.empty(mm.m3_workspace_size(B, L, H, cfg.rank), dtype=torch.uint8, device="cuda")
+    it = [0]
+
+    def step():
+        i = it[0]
+        it[0] += 1
+        d, o = sets[i % 2], outs[i % 2]
+        mm.m3_fwd(*(d.get(k) for k in M3_KEYS), y=o[0], h_last=o[1], workspace=ws)
+
+    K = max(3, min(args.steps, 200))
+    ms = _time_loop(step, K, world)
+    nbytes = m3_bytes(cfg)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    ops = m3_fp32_ops(cfg) * B * L * H * cfg.headdim
+    alu = ops / (ms * 1e-3) / 1e12
+    del sets, outs, ws
+    torch.cuda.empty_cache()
+    return {
+        "workload": cfg.name, "batch": B, "seq_len": L, "heads": H, "headdim": cfg.headdim,
+        "d_state": cfg.d_state, "rank": cfg.rank, "steps": K, "ms_per_step": round(ms, 5),
+        "value": round(_job_rate(world, B * L, ms), 1), "unit": "tokens/s", "launches_per_call": 2,
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(gbs / hbm_peak, 4), "traffic": None, "algorithmic_bytes": nbytes,
+                     "peak_source": hbm_src},
+        "roofline_alu": {"bound": "alu", "achieved": round(alu, 3), "peak": round(alu_peak, 3),
+                         "unit": "T fp32-pipe ops/s", "frac": round(alu / alu_peak, 4),
+                         "ops_per_token_channel": m3_fp32_ops(cfg),
+                         "peak_source": "derived, nominal: 148 SMs x 128 fp32 lanes x max SM clock (not measured)"},
+    }
+
+
 # ---------------------------------------------------------------- CPU oracle
 def cpu_baseline(host, cfg, target_s=12.0, sample_override=None, threads=None):
     """The fp64 oracle as it stands, on all host cores (or `threads` of
@@ -892,6 +964,15 @@ def run_only(args):
                torch.empty((cfg.batch, cfg.heads, cfg.headdim, cfg.d_state), device="cuda"))
         ws = torch.empty(mm.ssd_workspace_size(cfg.batch, cfg.seqlen, cfg.heads), dtype=torch.uint8, device="cuda")
         step = lambda: _ssd_call(mm, d, out, ws)  # noqa: E731
+    elif args.only in ("m3", "m3mimo"):
+        cfg = M3 if args.only == "m3" else M3_MIMO
+        d = {k: (v.cuda() if v is not None else None) for k, v in make_m3_inputs(cfg).items()}
+        out = (torch.empty((cfg.batch, cfg.seqlen, cfg.rank, cfg.heads * cfg.headdim), dtype=torch.bfloat16,
+                           device="cuda"),
+               torch.empty((cfg.batch, cfg.heads, cfg.headdim, cfg.d_state), device="cuda"))
+        ws = torch.empty(mm.m3_workspace_size(cfg.batch, cfg.seqlen, cfg.heads, cfg.rank), dtype=torch.uint8,
+                         device="cuda")
+        step = lambda: mm.m3_fwd(*(d.get(k) for k in M3_KEYS), y=out[0], h_last=out[1], workspace=ws)  # noqa: E731
     elif args.only == "forward":
         cfg = PREFILL
         d = {k: (v.cuda() if v is not None else None)
@@ -931,7 +1012,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra-prefill", action="store_true",
                     help="skip the 4 x 32768 and 262,144-token prefill legs")
-    ap.add_argument("--only", choices=["forward", "decode", "xproj", "dtproj", "ssd"], default=None,
+    ap.add_argument("--only", choices=["forward", "decode", "xproj", "dtproj", "ssd", "m3", "m3mimo"], default=None,
                     help="run one kernel's timed loop only (for profiler captures); prints no JSON line")
     ap.add_argument("--decode-layers", type=int, default=None,
                     help="with --only decode: stacked layers (default: the workload's 28)")

@@ -452,13 +452,66 @@ mm_status mamba_ssd_fwd(const void* x, const void* z, const void* dt, const floa
 size_t mamba_ssd_workspace_size(int64_t batch, int64_t seqlen, int64_t heads, int64_t headdim, int64_t d_state,
                                 int64_t groups);
 
+/*
+ * The Mamba-3 form of the selective scan, prefill (bf16 activations, fp32
+ * state and arithmetic).  The Jamba lesson's "Mamba-3" section names three
+ * changes over Mamba-2: an exponential-trapezoidal discretisation, whose
+ * conv-like rule acts on the state input inside the recurrence; a complex
+ * state, equivalent to a data-dependent rotary embedding; and multi-input
+ * multi-output (MIMO) projections.  The section gives no formula; the
+ * readings: per head h, group g = h / (H / groups), channel c = h P + p and
+ * state pair k (d_state entries 2k, 2k+1 = real and imaginary part),
+ *
+ *   Delta_t  = softplus(dt_t[h] + dt_bias[h]);   lambda_t = trap_t[h] (1/2 when trap is NULL)
+ *   a_t[k]   = exp(Delta_t A[h]) (cos(Delta_t theta[h,k]) + i sin(Delta_t theta[h,k]))
+ *   u_t[k]   = sum_r (B_t[r,g,2k] + i B_t[r,g,2k+1]) x_t[r,c]     (rank inputs r share the state)
+ *   s_t[k]   = a_t[k] (s_{t-1}[k] + (1 - lambda_t) Delta_t u_{t-1}[k]) + lambda_t Delta_t u_t[k]
+ *   y_t[r,c] = (sum_k Re(conj(C_t[r,g,k]) s_t[k]) + D[h] x_t[r,c]) * SiLU(z_t[r,c])   (no gate if z is NULL)
+ *
+ * lambda = 1 gives Euler's rule (the Mamba-2 step), 1/2 the trapezoid.
+ * u_{-1} is the input of the token before the call, from x_prev and B_prev
+ * (zero when both are NULL): a sequence split into calls continues exactly
+ * when each call passes the previous call's h_last as h0 and its last token's
+ * x and B rows as x_prev and B_prev.
+ *
+ *   x, z           [batch, seqlen, rank, heads*headdim]          bf16  (z may be NULL)
+ *   dt, trap       [batch, seqlen, heads]                        bf16  (trap may be NULL)
+ *   dt_bias        [heads] fp32 or NULL;  A [heads] fp32 (negative)
+ *   theta          [heads, d_state/2]                            fp32  rotation frequencies
+ *   Bm, Cm         [batch, seqlen, rank, groups, d_state]        bf16
+ *   Dskip          [heads] fp32 or NULL
+ *   h0             [batch, heads, headdim, d_state]              fp32  or NULL (= 0)
+ *   x_prev         [batch, rank, heads*headdim]                  bf16  or NULL (together with B_prev)
+ *   B_prev         [batch, rank, groups, d_state]                bf16  or NULL
+ *   y              [batch, seqlen, rank, heads*headdim]          bf16  output
+ *   h_last         [batch, heads, headdim, d_state]              fp32  output
+ *
+ * Supported: headdim == 64, d_state == 16, rank 1, 2 or 4, an even number
+ * of heads (MM_ERR_UNSUPPORTED otherwise); heads a multiple of groups
+ * (MM_ERR_SHAPE).  x_prev and B_prev are given together or not at all
+ * (MM_ERR_NULL).  Every pointer 16-byte aligned (MM_ERR_ALIGN); y and h_last
+ * may not overlap an input or each other (MM_ERR_ALIAS).  workspace: at least
+ * mamba_m3_workspace_size(...) bytes (the chunk end states of a sequence cut
+ * in time), 16-byte aligned, overlapping no other argument; its first 256
+ * bytes hold the call's status for mamba_check_status.  seqlen == 0 writes
+ * h_last = h0 (or zeros).  Runs on `stream`; the library allocates nothing.
+ */
+mm_status mamba_m3_fwd(const void* x, const void* z, const void* dt, const void* trap, const float* dt_bias,
+                       const float* A, const float* theta, const void* Bm, const void* Cm, const float* Dskip,
+                       const float* h0, const void* x_prev, const void* B_prev, void* y, float* h_last,
+                       int64_t batch, int64_t seqlen, int64_t rank, int64_t heads, int64_t headdim,
+                       int64_t d_state, int64_t groups, void* workspace, size_t workspace_bytes, void* stream);
+/* Workspace bytes of mamba_m3_fwd for these sizes (0 if not supported). */
+size_t mamba_m3_workspace_size(int64_t batch, int64_t seqlen, int64_t rank, int64_t heads, int64_t headdim,
+                               int64_t d_state, int64_t groups);
+
 /* A static, human-readable name for a status code. */
 const char* mamba_status_string(mm_status status);
 
 /* ABI version of this header (incremented on any signature change). */
 int mamba_mixer_abi_version(void);
 
-#define MAMBA_MIXER_ABI_VERSION 5
+#define MAMBA_MIXER_ABI_VERSION 6
 
 #ifdef __cplusplus
 }

@@ -17,7 +17,7 @@ __all__ = [
     "MM_F32", "MM_BF16", "MixerError", "lib", "library_path", "mixer_fwd", "mixer_fwd_noalloc", "mixer_fwd_host",
     "state_update", "workspace_size", "host_workspace_size", "status_string", "abi_version", "fault_status",
     "check_status", "proj_matmul", "proj_matmul_workspace_size", "mixer_fwd_projected",
-    "projected_workspace_size", "ssd_fwd", "ssd_workspace_size", "EXPORTED_SYMBOLS",
+    "projected_workspace_size", "ssd_fwd", "ssd_workspace_size", "m3_fwd", "m3_workspace_size", "EXPORTED_SYMBOLS",
 ]
 
 MM_F32 = 0
@@ -47,6 +47,8 @@ EXPORTED_SYMBOLS = (
     "mamba_mixer_projected_layout",
     "mamba_ssd_fwd",
     "mamba_ssd_workspace_size",
+    "mamba_m3_fwd",
+    "mamba_m3_workspace_size",
 )
 
 
@@ -105,6 +107,10 @@ def _declare(L):
     L.mamba_ssd_fwd.argtypes = [P] * 11 + [I64] * 6 + [P, ctypes.c_size_t, P]
     L.mamba_ssd_workspace_size.restype = ctypes.c_size_t
     L.mamba_ssd_workspace_size.argtypes = [I64] * 6
+    L.mamba_m3_fwd.restype = ctypes.c_int
+    L.mamba_m3_fwd.argtypes = [P] * 15 + [I64] * 7 + [P, ctypes.c_size_t, P]
+    L.mamba_m3_workspace_size.restype = ctypes.c_size_t
+    L.mamba_m3_workspace_size.argtypes = [I64] * 7
     return L
 
 
@@ -595,5 +601,64 @@ def ssd_fwd(x, z, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, *, headdim=64, y=None,
                                  _stream_handle(stream))
     if st != 0:
         raise MixerError(st, "mamba_ssd_fwd")
+    _keep_alive_on(made, (stream,))
+    return y, h_last
+
+
+def m3_workspace_size(batch, seqlen, heads, rank=1, headdim=64, d_state=16, groups=1) -> int:
+    return int(lib().mamba_m3_workspace_size(batch, seqlen, rank, heads, headdim, d_state, groups))
+
+
+def m3_fwd(x, z, dt, trap, dt_bias, A, theta, Bm, Cm, Dskip, h0=None, x_prev=None, B_prev=None, *,
+           headdim=64, y=None, h_last=None, workspace=None, stream=None):
+    """The Mamba-3 form of the scan (mamba_m3_fwd): x, z [B,L,R,H*P] bf16
+    (z may be None: no gate), dt and trap [B,L,H] bf16 (trap None: 1/2),
+    dt_bias/A/Dskip [H] fp32 (dt_bias and Dskip may be None), theta [H,N/2]
+    fp32, Bm/Cm [B,L,R,G,N] bf16, h0 [B,H,P,N] fp32 or None, x_prev [B,R,H*P]
+    and B_prev [B,R,G,N] bf16 or None, P = headdim.  Returns (y [B,L,R,H*P]
+    bf16, h_last [B,H,P,N] fp32), allocating any output not given."""
+    import torch
+
+    bf, f32 = torch.bfloat16, torch.float32
+    Bsz, L, R, HP = x.shape
+    H = A.shape[0]
+    P = int(headdim)
+    G, N = Bm.shape[3], Bm.shape[4]
+    if HP != H * P:
+        raise ValueError(f"x has {HP} channels, expected heads x headdim = {H * P}")
+    dev = x.device
+    made = []
+    _check(x, "x", bf, (Bsz, L, R, H * P), dev)
+    _check(z, "z", bf, (Bsz, L, R, H * P), dev)
+    _check(dt, "dt", bf, (Bsz, L, H), dev)
+    _check(trap, "trap", bf, (Bsz, L, H), dev)
+    _check(dt_bias, "dt_bias", f32, (H,), dev)
+    _check(A, "A", f32, (H,), dev)
+    _check(theta, "theta", f32, (H, N // 2), dev)
+    _check(Bm, "Bm", bf, (Bsz, L, R, G, N), dev)
+    _check(Cm, "Cm", bf, (Bsz, L, R, G, N), dev)
+    _check(Dskip, "Dskip", f32, (H,), dev)
+    _check(h0, "h0", f32, (Bsz, H, P, N), dev)
+    _check(x_prev, "x_prev", bf, (Bsz, R, H * P), dev)
+    _check(B_prev, "B_prev", bf, (Bsz, R, G, N), dev)
+    if y is None:
+        y = torch.empty((Bsz, L, R, H * P), dtype=bf, device=dev)
+        made.append(y)
+    if h_last is None:
+        h_last = torch.empty((Bsz, H, P, N), dtype=f32, device=dev)
+        made.append(h_last)
+    _check(y, "y", bf, (Bsz, L, R, H * P), dev)
+    _check(h_last, "h_last", f32, (Bsz, H, P, N), dev)
+    ws_bytes = m3_workspace_size(Bsz, L, H, R, P, N, G)
+    if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+        made.append(workspace)
+    with torch.cuda.device(dev):
+        st = lib().mamba_m3_fwd(_ptr(x), _ptr(z), _ptr(dt), _ptr(trap), _ptr(dt_bias), _ptr(A), _ptr(theta),
+                                _ptr(Bm), _ptr(Cm), _ptr(Dskip), _ptr(h0), _ptr(x_prev), _ptr(B_prev), _ptr(y),
+                                _ptr(h_last), Bsz, L, R, H, P, N, G, _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    if st != 0:
+        raise MixerError(st, "mamba_m3_fwd")
     _keep_alive_on(made, (stream,))
     return y, h_last

@@ -19,6 +19,7 @@
 #include "proj_gemm.cuh"
 #include "proj_ops.cuh"
 #include "ssd.cuh"
+#include "m3.cuh"
 
 namespace {
 
@@ -1547,6 +1548,142 @@ mm_status mamba_ssd_fwd(const void* x, const void* z, const void* dt, const floa
                                     fail ? (1 << 20) : mm::SsdScanLayout::smem_bytes, s>>>(p, tc, tb, th, tx, tz);
         if (cudaGetLastError() != cudaSuccess) return MM_ERR_CUDA;
     }
+    return MM_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- Mamba-3 form (chunked fp32 recurrence)
+namespace {
+
+// Time chunks of mamba_m3_fwd: enough that the grid holds about 8 CTAs of
+// 128 channels per SM, in whole 32-token tiles.  Workspace (256-byte
+// aligned regions): header [256 B]; end states [K-1][B][H*P][16] fp32;
+// chunk products [K-1][B][H][16] fp32.
+struct M3Plan {
+    int chunks = 1;
+    int64_t chunk_len = 0;
+    size_t off_state = 0, off_prod = 0, total = 0;
+};
+
+M3Plan plan_m3(int64_t batch, int64_t seqlen, int64_t heads, int sms) {
+    M3Plan pl;
+    const int64_t ctas = std::max<int64_t>(1, batch * heads * mm::kM3P / mm::kM3Threads);
+    const int64_t want = std::min<int64_t>(64, std::max<int64_t>(1, (int64_t(sms) * 8 + ctas - 1) / ctas));
+    const int64_t tiles = std::max<int64_t>(1, (seqlen + mm::kM3Tile - 1) / mm::kM3Tile);
+    pl.chunk_len = ((tiles + want - 1) / want) * mm::kM3Tile;
+    pl.chunks = static_cast<int>(seqlen > 0 ? (seqlen + pl.chunk_len - 1) / pl.chunk_len : 1);
+    const size_t k1 = static_cast<size_t>(pl.chunks - 1), B = static_cast<size_t>(batch);
+    pl.off_state = kWsHeader;
+    pl.off_prod = pl.off_state + align256(k1 * B * heads * mm::kM3P * mm::kM3N * 4);
+    pl.total = pl.off_prod + align256(k1 * B * heads * mm::kM3N * 4);
+    return pl;
+}
+
+bool m3_sizes_ok(int64_t batch, int64_t seqlen, int64_t rank, int64_t heads, int64_t groups) {
+    if (batch < 0 || seqlen < 0 || heads <= 0 || groups <= 0 || heads % groups != 0) return false;
+    if (rank != 1 && rank != 2 && rank != 4) return false;
+    if (heads % mm::kM3Heads != 0 || batch > 65535 || heads > (1 << 20)) return false;
+    int64_t tokens;
+    return mul_ok(batch, seqlen, &tokens) && tokens < (int64_t(1) << 40) / (rank * heads * mm::kM3P * 2);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mamba_m3_workspace_size(int64_t batch, int64_t seqlen, int64_t rank, int64_t heads, int64_t headdim,
+                               int64_t d_state, int64_t groups) {
+    if (headdim != mm::kM3P || d_state != mm::kM3N || batch <= 0 || !m3_sizes_ok(batch, seqlen, rank, heads, groups))
+        return 0;
+    return plan_m3(batch, seqlen, heads, plan_sms()).total;
+}
+
+mm_status mamba_m3_fwd(const void* x, const void* z, const void* dt, const void* trap, const float* dt_bias,
+                       const float* A, const float* theta, const void* Bm, const void* Cm, const float* Dskip,
+                       const float* h0, const void* x_prev, const void* B_prev, void* y, float* h_last,
+                       int64_t batch, int64_t seqlen, int64_t rank, int64_t heads, int64_t headdim,
+                       int64_t d_state, int64_t groups, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (headdim != mm::kM3P || d_state != mm::kM3N) return MM_ERR_UNSUPPORTED;
+    if (rank != 1 && rank != 2 && rank != 4) return MM_ERR_UNSUPPORTED;
+    if (heads > 0 && heads % mm::kM3Heads != 0) return MM_ERR_UNSUPPORTED;
+    if (!m3_sizes_ok(batch, seqlen, rank, heads, groups)) return MM_ERR_SHAPE;
+    if (batch == 0) return MM_OK;
+    const bool tokens = seqlen > 0;
+    if (!A || !theta || !h_last || (tokens && (!x || !dt || !Bm || !Cm || !y))) return MM_ERR_NULL;
+    if ((x_prev == nullptr) != (B_prev == nullptr)) return MM_ERR_NULL;
+    for (const void* q : {x, z, dt, trap, static_cast<const void*>(dt_bias), static_cast<const void*>(A),
+                          static_cast<const void*>(theta), Bm, Cm, static_cast<const void*>(Dskip),
+                          static_cast<const void*>(h0), x_prev, B_prev, static_cast<const void*>(y),
+                          static_cast<const void*>(h_last)})
+        if (q && !aligned16(q)) return MM_ERR_ALIGN;
+    const int64_t C = heads * mm::kM3P, NL = batch * seqlen;
+    const int64_t bc = groups * mm::kM3N;
+    const Span sx = span(x, NL * rank * C * 2), sz = span(z, NL * rank * C * 2), sdt = span(dt, NL * heads * 2),
+               str = span(trap, NL * heads * 2), sbias = span(dt_bias, heads * 4), sa = span(A, heads * 4),
+               sth = span(theta, heads * mm::kM3Pairs * 4), sb = span(Bm, NL * rank * bc * 2),
+               sc = span(Cm, NL * rank * bc * 2), sd = span(Dskip, heads * 4),
+               sh0 = span(h0, batch * C * mm::kM3N * 4), sxp = span(x_prev, batch * rank * C * 2),
+               sbp = span(B_prev, batch * rank * bc * 2), sy = span(y, NL * rank * C * 2),
+               shl = span(h_last, batch * C * mm::kM3N * 4);
+    const Span ins[] = {sx, sz, sdt, str, sbias, sa, sth, sb, sc, sd, sh0, sxp, sbp};
+    for (const Span& in : ins)
+        if (overlaps(sy, in) || overlaps(shl, in)) return MM_ERR_ALIAS;
+    if (overlaps(sy, shl)) return MM_ERR_ALIAS;
+    const int sms = plan_sms();
+    const M3Plan pl = plan_m3(batch, seqlen, heads, sms);
+    if (!workspace || workspace_bytes < pl.total) return MM_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MM_ERR_ALIGN;
+    const Span sw = span(workspace, static_cast<int64_t>(pl.total));
+    for (const Span& in : ins)
+        if (overlaps(sw, in)) return MM_ERR_ALIAS;
+    if (overlaps(sw, sy) || overlaps(sw, shl)) return MM_ERR_ALIAS;
+    if (mm_status st = check_device(); st != MM_OK) return st;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned char* w = static_cast<unsigned char*>(workspace);
+    // the call's status word: the epoch in the header's second word (these
+    // kernels have no wait that can give up, so it always reads complete)
+    const unsigned long long epoch = next_call_id();
+    if (cudaMemcpyAsync(w + 8, &epoch, sizeof(epoch), cudaMemcpyHostToDevice, s) != cudaSuccess) {
+        cudaGetLastError();
+        return MM_ERR_CUDA;
+    }
+    mm::M3Params p{};
+    p.x = static_cast<const __nv_bfloat16*>(x);
+    p.z = static_cast<const __nv_bfloat16*>(z);
+    p.dt = static_cast<const __nv_bfloat16*>(dt);
+    p.trap = static_cast<const __nv_bfloat16*>(trap);
+    p.dt_bias = dt_bias;
+    p.A = A;
+    p.theta = theta;
+    p.Bm = static_cast<const __nv_bfloat16*>(Bm);
+    p.Cm = static_cast<const __nv_bfloat16*>(Cm);
+    p.Dskip = Dskip;
+    p.h0 = h0;
+    p.x_prev = static_cast<const __nv_bfloat16*>(x_prev);
+    p.B_prev = static_cast<const __nv_bfloat16*>(B_prev);
+    p.y = static_cast<__nv_bfloat16*>(y);
+    p.h_last = h_last;
+    p.ws_state = reinterpret_cast<float*>(w + pl.off_state);
+    p.ws_prod = reinterpret_cast<float*>(w + pl.off_prod);
+    p.L = seqlen;
+    p.chunk_len = pl.chunk_len;
+    p.R = static_cast<int>(rank);
+    p.H = static_cast<int>(heads);
+    p.G = static_cast<int>(groups);
+    p.chunks = pl.chunks;
+    const unsigned cx = static_cast<unsigned>(C / mm::kM3Threads);
+    const bool fail = forced_launch_failure();
+    if (pl.chunks > 1) {
+        mm::m3_chunk_kernel<false><<<dim3(cx, static_cast<unsigned>(pl.chunks - 1), static_cast<unsigned>(batch)),
+                                     fail ? 2048 : mm::kM3Threads, 0, s>>>(p);
+        if (cudaGetLastError() != cudaSuccess) return MM_ERR_CUDA;
+    }
+    mm::m3_chunk_kernel<true><<<dim3(cx, static_cast<unsigned>(pl.chunks), static_cast<unsigned>(batch)),
+                                fail ? 2048 : mm::kM3Threads, 0, s>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return MM_ERR_CUDA;
     return MM_OK;
 }
 

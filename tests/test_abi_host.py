@@ -59,7 +59,7 @@ def test_exported_symbols_are_c_linkage():
 
 def test_version_and_strings():
     mmbuild.build()
-    assert mm.abi_version() == 5
+    assert mm.abi_version() == 6
     for code in range(13):
         s = mm.status_string(code)
         assert s and s != "unknown status"
@@ -342,6 +342,54 @@ def test_ssd_validation(L):
     assert L.mamba_ssd_fwd(*ssd_args(ws_bytes=need - 16)) == EWORKSPACE
     assert L.mamba_ssd_fwd(*ssd_args(ws=None)) == EWORKSPACE
     assert L.mamba_ssd_fwd(*ssd_args(ws=WS_ADDR + 8)) == EALIGN
+
+
+# ---------------------------------------------------------------- Mamba-3 form
+def m3_args(B=2, Lq=300, R=2, H=4, P=64, N=16, G=2, ws_bytes=None, **over):
+    """mamba_m3_fwd arguments on fake addresses, each buffer 2^32 apart."""
+    names = ["x", "z", "dt", "trap", "dt_bias", "A", "theta", "Bm", "Cm", "Dskip", "h0", "x_prev", "B_prev",
+             "y", "h_last"]
+    addr = {n: BASE + (i << 32) for i, n in enumerate(names)}
+    addr.update(over)
+    ws = over.get("ws", WS_ADDR)
+    need = mm.m3_workspace_size(max(B, 1), Lq, H, R, P, N, G) if ws_bytes is None else ws_bytes
+    return [addr[n] for n in names] + [B, Lq, R, H, P, N, G, ws, need, None]
+
+
+def test_m3_workspace_size_rules():
+    # 4096 tokens of one sequence with 128 heads: 64 CTAs of 128 channels a
+    # chunk; 8 CTAs on each of 148 SMs want 19 chunks, of 7 tiles (224
+    # tokens), so 19 chunks and 18 chunk end states (fp32, 16 per channel) and
+    # 18 products per head
+    assert mm.m3_workspace_size(1, 4096, 128) == 256 + 18 * 8192 * 16 * 4 + 18 * 128 * 16 * 4
+    assert mm.m3_workspace_size(1, 0, 128) == 256
+    assert mm.m3_workspace_size(1, 4096, 128, rank=3) == 0
+    assert mm.m3_workspace_size(1, 4096, 128, d_state=32) == 0
+    assert mm.m3_workspace_size(1, 4096, 3) == 0
+
+
+def test_m3_validation(L):
+    assert L.mamba_m3_fwd(*m3_args()) == EDEVICE
+    assert L.mamba_m3_fwd(*m3_args(z=None, trap=None, dt_bias=None, Dskip=None, h0=None, x_prev=None,
+                                   B_prev=None)) == EDEVICE
+    assert L.mamba_m3_fwd(*m3_args(P=32)) == EUNSUP
+    assert L.mamba_m3_fwd(*m3_args(N=32)) == EUNSUP
+    assert L.mamba_m3_fwd(*m3_args(R=3)) == EUNSUP
+    assert L.mamba_m3_fwd(*m3_args(H=3, G=1)) == EUNSUP
+    assert L.mamba_m3_fwd(*m3_args(H=6, G=4)) == ESHAPE
+    assert L.mamba_m3_fwd(*m3_args(Lq=-1, ws_bytes=0)) == ESHAPE
+    assert L.mamba_m3_fwd(*m3_args(B=0, ws_bytes=0)) == OK
+    for name in ("x", "dt", "A", "theta", "Bm", "Cm", "y", "h_last"):
+        assert L.mamba_m3_fwd(*m3_args(**{name: None})) == ENULL, name
+    assert L.mamba_m3_fwd(*m3_args(x_prev=None)) == ENULL       # x_prev and B_prev together
+    assert L.mamba_m3_fwd(*m3_args(Lq=0, x=None, dt=None, Bm=None, Cm=None, y=None)) == EDEVICE
+    for name in ("x", "trap", "theta", "B_prev", "y"):
+        assert L.mamba_m3_fwd(*m3_args(**{name: BASE + (1 << 40) + 8})) == EALIGN, name
+    assert L.mamba_m3_fwd(*m3_args(y=BASE)) == EALIAS                        # y over x
+    assert L.mamba_m3_fwd(*m3_args(h_last=BASE + (10 << 32))) == EALIAS      # h_last over h0
+    assert L.mamba_m3_fwd(*m3_args(ws=BASE + (7 << 32))) == EALIAS           # workspace over B
+    need = mm.m3_workspace_size(2, 300, 4, 2, 64, 16, 2)
+    assert L.mamba_m3_fwd(*m3_args(ws_bytes=need - 16)) == EWORKSPACE
 
 
 # ---------------------------------------------------------------- state_update validation
