@@ -15,16 +15,17 @@
 // registers, in fp32.  The recurrence is linear in the state, so a sequence
 // is cut into time chunks for parallelism, an exact regrouping:
 //   m3_chunk_kernel<false> (summary pass, chunks 0..K-2): each chunk's end
-//       state from a zero start (the first token's trapezoid tap on the
-//       previous token's input included), per channel, and the chunk's
+//       pre-state (below) from a zero start, per channel, and the chunk's
 //       product of a_t, per head;
-//   m3_chunk_kernel<true> (full pass, every chunk): the entering state as
-//       h0 carried through the earlier chunks' (product, end state) pairs,
-//       then the recurrence with readout, skip and gate; the last chunk
-//       writes h_last.
+//   m3_chunk_kernel<true> (full pass, every chunk): the entering pre-state
+//       from h0 and the previous call's last input, carried through the
+//       earlier chunks' (product, end pre-state) pairs, then the recurrence
+//       with readout, skip and gate; the last chunk writes h_last.
+// A CTA's tiles of x, z, B, C, dt and the trapezoid weight arrive by
+// asynchronous 16-byte copies one tile ahead of the compute (two buffers).
 // Per-(token, head) factors -- a_t (one exp and one sincos per pair) and the
-// two tap weights -- are computed once per CTA tile into shared memory, as
-// are the tile's B and C rows; x, z and y move per thread, 2 bytes each, a
+// two tap weights -- are computed once per tile into shared memory, with the
+// tile's B and C rows widened to fp32; y goes out per thread, 2 bytes each, a
 // warp's 32 channels contiguous.
 #pragma once
 
@@ -40,8 +41,7 @@ constexpr int kM3N = 2 * kM3Pairs;
 constexpr int kM3P = 64;           // channels per head
 constexpr int kM3Threads = 128;    // channels per CTA: two heads
 constexpr int kM3Heads = kM3Threads / kM3P;
-constexpr int kM3Tile = 32;        // tokens per staged tile
-constexpr int kM3MaxRank = 4;
+constexpr int kM3Tile = 32;        // chunk lengths are whole multiples of this
 
 struct M3Params {
     const __nv_bfloat16* x;        // [B][L][R][H*P]
@@ -65,38 +65,120 @@ struct M3Params {
     int R, H, G, chunks;
 };
 
-struct M3Smem {
-    float2 a[kM3Tile][kM3Heads][kM3Pairs];             // a_t per head and pair
-    float2 w[kM3Tile][kM3Heads];                        // ((1 - lambda) Delta, lambda Delta)
-    float4 b[kM3Tile][kM3MaxRank][kM3Heads][kM3N / 4];   // B rows of each head's group
-    float4 c[kM3Tile][kM3MaxRank][kM3Heads][kM3N / 4];   // C rows
+// Shared memory of a CTA: two buffers of raw tile inputs, filled by
+// asynchronous copies one tile ahead of the compute, and the tile's
+// per-(token, head) factors and widened B / C rows.  A tile is 32 / R tokens
+// (R = 1, 2, 4), so its x and z rows are 8 KB each whatever R is.
+struct M3Layout {
+    int T, R;
+    __host__ __device__ int xs() const { return T * R * kM3Threads * 2; }          // x or z rows, bf16
+    __host__ __device__ int bs() const { return T * R * kM3Heads * kM3N * 2; }     // B or C rows, bf16
+    __host__ __device__ int ds() const { return (T + 1) * kM3Heads * 2; }          // dt or trap (one token more), bf16
+    __host__ __device__ int buf() const { return (2 * xs() + 2 * bs() + 2 * ds() + 15) & ~15; }
+    __host__ __device__ int off_x(int i) const { return i * buf(); }
+    __host__ __device__ int off_z(int i) const { return i * buf() + xs(); }
+    __host__ __device__ int off_b(int i) const { return i * buf() + 2 * xs(); }
+    __host__ __device__ int off_c(int i) const { return i * buf() + 2 * xs() + bs(); }
+    __host__ __device__ int off_dt(int i) const { return i * buf() + 2 * xs() + 2 * bs(); }
+    __host__ __device__ int off_tr(int i) const { return i * buf() + 2 * xs() + 2 * bs() + ds(); }
+    __host__ __device__ int off_a() const { return 2 * buf(); }                      // float2 [T][heads][pairs]
+    __host__ __device__ int off_w() const { return off_a() + T * kM3Heads * kM3Pairs * 8; }   // float2 [T+1][heads]
+    __host__ __device__ int off_bf() const { return off_w() + (T + 1) * kM3Heads * 8; }       // float4 [T][R][heads][N/4]
+    __host__ __device__ int off_cf() const { return off_bf() + T * R * kM3Heads * kM3N * 4; }
+    __host__ __device__ int off_k() const { return off_cf() + T * R * kM3Heads * kM3N * 4; }  // float [T][heads][R][R]
+    __host__ __device__ int bytes() const { return off_k() + T * kM3Heads * R * R * 4; }
 };
+__host__ __device__ inline M3Layout m3_layout(int R) { return M3Layout{32 / R, R}; }
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" :: "r"(smem_addr(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" :: "r"(smem_addr(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+// wait until at most `pending` of this thread's committed groups are in flight
+template <int pending>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" :: "n"(pending) : "memory"); }
 
 __device__ __forceinline__ float m3_bf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
-// Thread j's channel input u of token t (or of the token before the call):
-// sum_r (B[r, 2k] + i B[r, 2k+1]) x[r], from global rows.
+// a * s + e for complex numbers held as (re, im) float2, on packed f32x2 operations:
+// (a.re s.re - a.im s.im, a.re s.im + a.im s.re) + e
+__device__ __forceinline__ float2 cmul_add(float2 a, float2 s, float2 e) {
+    const float2 t = fma2(make_float2(-a.y, a.y), make_float2(s.y, s.x), e);
+    return fma2(make_float2(a.x, a.x), s, t);
+}
+__device__ __forceinline__ float4 m3_widen4(uint2 v) {
+    return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                       __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+}
+
+// Thread j's channel input u of one token (or of the token before the call):
+// sum_r (B[r, 2k] + i B[r, 2k+1]) x[r], from global rows, as (re, im) pairs.
+template <int R>
 __device__ __forceinline__ void m3_input_global(const M3Params& p, const __nv_bfloat16* xrow,
                                                 const __nv_bfloat16* brow, int64_t x_rstride,
-                                                int64_t b_rstride, float (&ur)[kM3Pairs], float (&ui)[kM3Pairs]) {
+                                                int64_t b_rstride, float2 (&u)[kM3Pairs]) {
 #pragma unroll
-    for (int k = 0; k < kM3Pairs; ++k) ur[k] = ui[k] = 0.0f;
-    for (int r = 0; r < p.R; ++r) {
+    for (int k = 0; k < kM3Pairs; ++k) u[k] = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
         const float xv = m3_bf(xrow + r * x_rstride);
         const __nv_bfloat16* br = brow + r * b_rstride;
 #pragma unroll
         for (int k = 0; k < kM3Pairs; ++k) {
-            ur[k] = fmaf(m3_bf(br + 2 * k), xv, ur[k]);
-            ui[k] = fmaf(m3_bf(br + 2 * k + 1), xv, ui[k]);
+            u[k].x = fmaf(m3_bf(br + 2 * k), xv, u[k].x);
+            u[k].y = fmaf(m3_bf(br + 2 * k + 1), xv, u[k].y);
         }
     }
 }
 
-template <bool FULL>
+// Issue the asynchronous copies of one tile's raw inputs (tokens ts ..
+// ts + n - 1 of sequence b) into buffer `buf`.
+template <bool FULL, int R>
+__device__ __forceinline__ void m3_issue_tile(const M3Params& p, const M3Layout& lay, unsigned char* sm, int buf,
+                                              int b, int64_t ts, int n) {
+    const int tid = threadIdx.x;
+    const int64_t C = static_cast<int64_t>(p.H) * kM3P;
+    const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kM3Threads;
+    const int h0_ = blockIdx.x * kM3Heads;
+    // x (and z): 16 pieces of 16 bytes per (token, input) row of the CTA's 128 channels
+    for (int e = tid; e < n * R * 16; e += kM3Threads) {
+        const int q = e & 15, tr = e >> 4;                 // tr = token * R + r
+        const int64_t g = (static_cast<int64_t>(b) * p.L + ts) * R * C + static_cast<int64_t>(tr) * C + c0 + 8 * q;
+        cp_async16(sm + lay.off_x(buf) + tr * (kM3Threads * 2) + 16 * q, p.x + g);
+        if (FULL && p.z) cp_async16(sm + lay.off_z(buf) + tr * (kM3Threads * 2) + 16 * q, p.z + g);
+    }
+    // B (and C) rows of each head's group: two 16-byte pieces per (token, input, head)
+    const int64_t br = static_cast<int64_t>(p.G) * kM3N;
+    for (int e = tid; e < n * R * kM3Heads * 2; e += kM3Threads) {
+        const int q = e & 1, hh = (e >> 1) % kM3Heads, tr = e / (2 * kM3Heads);
+        const int gh = (h0_ + hh) * p.G / p.H;
+        const int64_t g = ((static_cast<int64_t>(b) * p.L + ts) * R + tr) * br + gh * kM3N + 8 * q;
+        const int so = (tr * kM3Heads + hh) * (kM3N * 2) + 16 * q;
+        cp_async16(sm + lay.off_b(buf) + so, p.Bm + g);
+        if (FULL) cp_async16(sm + lay.off_c(buf) + so, p.Cm + g);
+    }
+    // dt (and trap) of the CTA's two heads: 4 bytes per token, and of the
+    // token after the tile when there is one (its trapezoid tap weight)
+    const int nd = ts + n < p.L ? n + 1 : n;
+    for (int e = tid; e < nd; e += kM3Threads) {
+        const int64_t g = (static_cast<int64_t>(b) * p.L + ts + e) * p.H + h0_;
+        cp_async4(sm + lay.off_dt(buf) + 4 * e, p.dt + g);
+        if (p.trap) cp_async4(sm + lay.off_tr(buf) + 4 * e, p.trap + g);
+    }
+}
+
+// R: inputs per state (1, 2 or 4), a compile-time constant so that the
+// per-token loops over inputs and outputs unroll.
+template <bool FULL, int R>
 __global__ void __launch_bounds__(kM3Threads)
 m3_chunk_kernel(const M3Params p)
 {
-    __shared__ __align__(16) M3Smem sm;
+    extern __shared__ __align__(16) unsigned char m3_sm[];
+    constexpr int T = 32 / R;
+    const M3Layout lay = m3_layout(R);
     const int tid = threadIdx.x;
     const int64_t C = static_cast<int64_t>(p.H) * kM3P;
     const int64_t c = static_cast<int64_t>(blockIdx.x) * kM3Threads + tid;   // channel
@@ -107,27 +189,49 @@ m3_chunk_kernel(const M3Params p)
     const int b = blockIdx.z;
     const int64_t t0 = static_cast<int64_t>(chunk) * p.chunk_len;
     const int64_t t1 = min(p.L, t0 + p.chunk_len);
-    const int R = p.R;
     const int64_t xr = C;                              // elements between the R inputs of a token
     const int64_t xt = static_cast<int64_t>(R) * C;    // ... between tokens
     const int64_t br = static_cast<int64_t>(p.G) * kM3N;
-    const int64_t bt = static_cast<int64_t>(R) * br;
     const int g = h * p.G / p.H;
 
-    // the state entering the chunk
-    float sr[kM3Pairs], si[kM3Pairs];
+    // the first tile's copies are in flight during the setup
+    if (t0 < t1) m3_issue_tile<FULL, R>(p, lay, m3_sm, 0, b, t0, static_cast<int>(min(static_cast<int64_t>(T), t1 - t0)));
+    cp_async_commit();
+
+    // The kernel carries the pre-state  q_t = s_t + (1 - lambda_{t+1}) Delta_{t+1} u_t,
+    // which obeys one multiply-add per pair and token,
+    //     q_t = a_t q_{t-1} + omega_t u_t,   omega_t = lambda_t Delta_t + (1 - lambda_{t+1}) Delta_{t+1},
+    // and reads out s_t = q_t - (1 - lambda_{t+1}) Delta_{t+1} u_t: the second
+    // term is, per output r, sum_r' x_t[r'] (C_t[r] . B_t[r']) times that
+    // weight, a per-(token, head) matrix kappa that also holds the skip D.
+    // Past the last token the weight is 0, so q is s there.
+    float2 st[kM3Pairs];
 #pragma unroll
-    for (int k = 0; k < kM3Pairs; ++k) sr[k] = si[k] = 0.0f;
+    for (int k = 0; k < kM3Pairs; ++k) st[k] = make_float2(0.0f, 0.0f);
     if (FULL) {
+        // q_{-1} = h0 + (1 - lambda_0) Delta_0 u_{-1}
         if (p.h0) {
             const float4* hp = reinterpret_cast<const float4*>(p.h0 + (static_cast<int64_t>(b) * C + c) * kM3N);
 #pragma unroll
             for (int q = 0; q < kM3N / 4; ++q) {
                 const float4 v = hp[q];
-                sr[2 * q] = v.x; si[2 * q] = v.y; sr[2 * q + 1] = v.z; si[2 * q + 1] = v.w;
+                st[2 * q] = make_float2(v.x, v.y);
+                st[2 * q + 1] = make_float2(v.z, v.w);
             }
         }
-        // carried through the earlier chunks: s = prod_c' s + e_c'
+        if (p.x_prev && p.B_prev && p.L > 0) {
+            const int64_t row = static_cast<int64_t>(b) * p.L;
+            const float v = __bfloat162float(p.dt[row * p.H + h]) + (p.dt_bias ? p.dt_bias[h] : 0.0f);
+            const float dl = fmaxf(v, 0.0f) + log1pf(expf(-fabsf(v)));
+            const float lam = p.trap ? __bfloat162float(p.trap[row * p.H + h]) : 0.5f;
+            float2 up[kM3Pairs];
+            m3_input_global<R>(p, p.x_prev + static_cast<int64_t>(b) * R * C + c,
+                            p.B_prev + static_cast<int64_t>(b) * R * br + g * kM3N, xr, br, up);
+            const float2 w0 = make_float2((1.0f - lam) * dl, (1.0f - lam) * dl);
+#pragma unroll
+            for (int k = 0; k < kM3Pairs; ++k) st[k] = fma2(w0, up[k], st[k]);
+        }
+        // carried through the earlier chunks: q = prod_c' q + e_c'
         for (int cc = 0; cc < chunk; ++cc) {
             const float4* pp = reinterpret_cast<const float4*>(
                 p.ws_prod + ((static_cast<int64_t>(cc) * gridDim.z + b) * p.H + h) * kM3N);
@@ -136,153 +240,160 @@ m3_chunk_kernel(const M3Params p)
 #pragma unroll
             for (int q = 0; q < kM3N / 4; ++q) {
                 const float4 a = pp[q], e = ep[q];
-                const int k0 = 2 * q, k1 = 2 * q + 1;
-                float r0 = fmaf(a.x, sr[k0], fmaf(-a.y, si[k0], e.x));
-                float i0 = fmaf(a.x, si[k0], fmaf(a.y, sr[k0], e.y));
-                float r1 = fmaf(a.z, sr[k1], fmaf(-a.w, si[k1], e.z));
-                float i1 = fmaf(a.z, si[k1], fmaf(a.w, sr[k1], e.w));
-                sr[k0] = r0; si[k0] = i0; sr[k1] = r1; si[k1] = i1;
+                st[2 * q] = cmul_add(make_float2(a.x, a.y), st[2 * q], make_float2(e.x, e.y));
+                st[2 * q + 1] = cmul_add(make_float2(a.z, a.w), st[2 * q + 1], make_float2(e.z, e.w));
             }
         }
     }
-    // the previous token's input u (the trapezoid's first tap)
-    float ur[kM3Pairs], ui[kM3Pairs];
-    if (t0 > 0) {
-        const int64_t row = static_cast<int64_t>(b) * p.L + (t0 - 1);
-        m3_input_global(p, p.x + row * xt + c, p.Bm + row * bt + g * kM3N, xr, br, ur, ui);
-    } else if (p.x_prev && p.B_prev) {
-        m3_input_global(p, p.x_prev + static_cast<int64_t>(b) * R * C + c,
-                        p.B_prev + static_cast<int64_t>(b) * R * br + g * kM3N, xr, br, ur, ui);
-    } else {
-#pragma unroll
-        for (int k = 0; k < kM3Pairs; ++k) ur[k] = ui[k] = 0.0f;
-    }
-    // the chunk's product of a_t (summary pass; the head's first thread keeps it)
-    float pr[kM3Pairs], pi[kM3Pairs];
-#pragma unroll
-    for (int k = 0; k < kM3Pairs; ++k) { pr[k] = 1.0f; pi[k] = 0.0f; }
+    // summary pass: the chunk's product of a_t for (head, pair) tid, tid < 16
+    float2 prod = make_float2(1.0f, 0.0f);
 
-    const float dsk = p.Dskip ? p.Dskip[h] : 0.0f;
-    for (int64_t ts = t0; ts < t1; ts += kM3Tile) {
-        const int T = static_cast<int>(min(static_cast<int64_t>(kM3Tile), t1 - ts));
-        __syncthreads();   // the previous tile's factors are consumed
-        // factors of each (token, head): a_t per pair, then the tap weights
-        for (int e = tid; e < kM3Tile * kM3Heads * kM3Pairs; e += kM3Threads) {
-            const int k = e % kM3Pairs, hh = (e / kM3Pairs) % kM3Heads, tt = e / (kM3Pairs * kM3Heads);
-            if (tt < T) {
-                const int hd = h0_ + hh;
-                const int64_t row = static_cast<int64_t>(b) * p.L + ts + tt;
-                const float v = __bfloat162float(p.dt[row * p.H + hd]) + (p.dt_bias ? p.dt_bias[hd] : 0.0f);
+    float2* fa = reinterpret_cast<float2*>(m3_sm + lay.off_a());
+    float2* fw = reinterpret_cast<float2*>(m3_sm + lay.off_w());
+    float4* fb = reinterpret_cast<float4*>(m3_sm + lay.off_bf());
+    float4* fc = reinterpret_cast<float4*>(m3_sm + lay.off_cf());
+    float* fk = reinterpret_cast<float*>(m3_sm + lay.off_k());
+    int buf = 0;
+    for (int64_t ts = t0; ts < t1; ts += T, buf ^= 1) {
+        const int n = static_cast<int>(min(static_cast<int64_t>(T), t1 - ts));
+        const int nd = ts + n < p.L ? n + 1 : n;
+        // the next tile's copies go into the other buffer while this one is used
+        const int64_t tn = ts + T;
+        if (tn < t1) m3_issue_tile<FULL, R>(p, lay, m3_sm, buf ^ 1, b, tn, static_cast<int>(min(static_cast<int64_t>(T), t1 - tn)));
+        cp_async_commit();
+        cp_async_wait<1>();           // this tile's copies have landed (this thread's)
+        __syncthreads();              // ... and every thread's
+        const __nv_bfloat16* xs = reinterpret_cast<const __nv_bfloat16*>(m3_sm + lay.off_x(buf));
+        const __nv_bfloat16* zs = reinterpret_cast<const __nv_bfloat16*>(m3_sm + lay.off_z(buf));
+        const __nv_bfloat16* dts = reinterpret_cast<const __nv_bfloat16*>(m3_sm + lay.off_dt(buf));
+        const __nv_bfloat16* trs = reinterpret_cast<const __nv_bfloat16*>(m3_sm + lay.off_tr(buf));
+        // tap weights ((1 - lambda) Delta, lambda Delta) per (token, head), the
+        // token after the tile included (zero past the sequence)
+        for (int e = tid; e < (T + 1) * kM3Heads; e += kM3Threads) {
+            const int tt = e / kM3Heads, hh = e % kM3Heads, hd = h0_ + hh;
+            float2 w = make_float2(0.0f, 0.0f);
+            if (tt < nd) {
+                const float v = __bfloat162float(dts[e]) + (p.dt_bias ? p.dt_bias[hd] : 0.0f);
                 const float dl = fmaxf(v, 0.0f) + log1pf(expf(-fabsf(v)));
-                const float mag = expf(dl * p.A[hd]);
-                float sn, cs;
-                sincosf(dl * p.theta[hd * kM3Pairs + k], &sn, &cs);
-                sm.a[tt][hh][k] = make_float2(mag * cs, mag * sn);
-                if (k == 0) {
-                    const float lam = p.trap ? __bfloat162float(p.trap[row * p.H + hd]) : 0.5f;
-                    sm.w[tt][hh] = make_float2((1.0f - lam) * dl, lam * dl);
-                }
+                const float lam = p.trap ? __bfloat162float(trs[e]) : 0.5f;
+                w = make_float2((1.0f - lam) * dl, lam * dl);
             }
+            fw[e] = w;
         }
-        // B and C rows of each head's group, widened to fp32
-        for (int e = tid; e < kM3Tile * R * kM3Heads * (kM3N / 4); e += kM3Threads) {
-            const int q = e % (kM3N / 4), hh = (e / (kM3N / 4)) % kM3Heads, r = (e / (kM3N / 4 * kM3Heads)) % R;
-            const int tt = e / (kM3N / 4 * kM3Heads * R);
-            if (tt < T) {
-                const int gh = (h0_ + hh) * p.G / p.H;
-                const int64_t off = (static_cast<int64_t>(b) * p.L + ts + tt) * bt + r * br + gh * kM3N + 4 * q;
-                const uint2 bv = *reinterpret_cast<const uint2*>(p.Bm + off);
-                const uint2 cv = *reinterpret_cast<const uint2*>(p.Cm + off);
-                sm.b[tt][r][hh][q] = make_float4(__uint_as_float(bv.x << 16), __uint_as_float(bv.x & 0xffff0000u),
-                                                 __uint_as_float(bv.y << 16), __uint_as_float(bv.y & 0xffff0000u));
-                sm.c[tt][r][hh][q] = make_float4(__uint_as_float(cv.x << 16), __uint_as_float(cv.x & 0xffff0000u),
-                                                 __uint_as_float(cv.y << 16), __uint_as_float(cv.y & 0xffff0000u));
+        __syncthreads();
+        // a_t per pair
+        for (int e = tid; e < n * kM3Heads * kM3Pairs; e += kM3Threads) {
+            const int k = e % kM3Pairs, th = e / kM3Pairs, hd = h0_ + th % kM3Heads;
+            const float2 w = fw[th];
+            const float dl = w.x + w.y;
+            float sn, cs;
+            sincosf(dl * p.theta[hd * kM3Pairs + k], &sn, &cs);
+            const float mag = expf(dl * p.A[hd]);
+            fa[e] = make_float2(mag * cs, mag * sn);
+        }
+        // omega_t B_t and C_t, widened to fp32
+        const uint2* braw = reinterpret_cast<const uint2*>(m3_sm + lay.off_b(buf));
+        const uint2* craw = reinterpret_cast<const uint2*>(m3_sm + lay.off_c(buf));
+        for (int e = tid; e < n * R * kM3Heads * (kM3N / 4); e += kM3Threads) {
+            const int hh = (e / (kM3N / 4)) % kM3Heads, tt = e / (kM3N / 4 * kM3Heads * R);
+            const float om = fw[tt * kM3Heads + hh].y + fw[(tt + 1) * kM3Heads + hh].x;
+            const float4 bv = m3_widen4(braw[e]);
+            fb[e] = make_float4(om * bv.x, om * bv.y, om * bv.z, om * bv.w);
+            if (FULL) fc[e] = m3_widen4(craw[e]);
+        }
+        // kappa[t][head][r][r'] = D [r == r'] - (1 - lambda_{t+1}) Delta_{t+1} (C_t[r] . B_t[r'])
+        if (FULL) {
+            for (int e = tid; e < n * kM3Heads * R * R; e += kM3Threads) {
+                const int rp = e % R, r = (e / R) % R, hh = (e / (R * R)) % kM3Heads, tt = e / (R * R * kM3Heads);
+                const uint2* bq = braw + ((tt * R + rp) * kM3Heads + hh) * (kM3N / 4);
+                const uint2* cq = craw + ((tt * R + r) * kM3Heads + hh) * (kM3N / 4);
+                float dot = 0.0f;
+#pragma unroll
+                for (int q = 0; q < kM3N / 4; ++q) {
+                    const float4 bv = m3_widen4(bq[q]), cv = m3_widen4(cq[q]);
+                    dot = fmaf(cv.x, bv.x, fmaf(cv.y, bv.y, fmaf(cv.z, bv.z, fmaf(cv.w, bv.w, dot))));
+                }
+                const float dh = p.Dskip ? p.Dskip[h0_ + hh] : 0.0f;
+                fk[e] = (r == rp ? dh : 0.0f) - fw[(tt + 1) * kM3Heads + hh].x * dot;
             }
         }
         __syncthreads();
+        if (!FULL && tid < kM3Heads * kM3Pairs) {
+            for (int tt = 0; tt < n; ++tt) prod = cmul_add(fa[tt * kM3Heads * kM3Pairs + tid], prod, make_float2(0.0f, 0.0f));
+        }
 
-        for (int tt = 0; tt < T; ++tt) {
-            const int64_t row = static_cast<int64_t>(b) * p.L + ts + tt;
-            const __nv_bfloat16* xrow = p.x + row * xt + c;
-            float xv[kM3MaxRank];
+        for (int tt = 0; tt < n; ++tt) {
+            float xv[R];
 #pragma unroll
-            for (int r = 0; r < kM3MaxRank; ++r) xv[r] = r < R ? m3_bf(xrow + r * xr) : 0.0f;
-            // u_t
-            float vr[kM3Pairs], vi[kM3Pairs];
+            for (int r = 0; r < R; ++r) xv[r] = __bfloat162float(xs[(tt * R + r) * kM3Threads + tid]);
+            // q = a q + sum_r (omega b_r) x_r
+            float2 v[kM3Pairs];
 #pragma unroll
-            for (int k = 0; k < kM3Pairs; ++k) vr[k] = vi[k] = 0.0f;
+            for (int k = 0; k < kM3Pairs; ++k) v[k] = make_float2(0.0f, 0.0f);
 #pragma unroll
-            for (int r = 0; r < kM3MaxRank; ++r) {
-                if (r < R) {
+            for (int r = 0; r < R; ++r) {
+                const float2 x2 = make_float2(xv[r], xv[r]);
 #pragma unroll
-                    for (int q = 0; q < kM3N / 4; ++q) {
-                        const float4 bb = sm.b[tt][r][hl][q];
-                        vr[2 * q] = fmaf(bb.x, xv[r], vr[2 * q]);
-                        vi[2 * q] = fmaf(bb.y, xv[r], vi[2 * q]);
-                        vr[2 * q + 1] = fmaf(bb.z, xv[r], vr[2 * q + 1]);
-                        vi[2 * q + 1] = fmaf(bb.w, xv[r], vi[2 * q + 1]);
-                    }
+                for (int q = 0; q < kM3N / 4; ++q) {
+                    const float4 bb = fb[((tt * R + r) * kM3Heads + hl) * (kM3N / 4) + q];
+                    v[2 * q] = fma2(make_float2(bb.x, bb.y), x2, v[2 * q]);
+                    v[2 * q + 1] = fma2(make_float2(bb.z, bb.w), x2, v[2 * q + 1]);
                 }
             }
-            // s = a (s + (1 - lambda) Delta u_prev) + lambda Delta u
-            const float2 w = sm.w[tt][hl];
+            const float4* fa4 = reinterpret_cast<const float4*>(fa + (tt * kM3Heads + hl) * kM3Pairs);
 #pragma unroll
-            for (int k = 0; k < kM3Pairs; ++k) {
-                const float2 a = sm.a[tt][hl][k];
-                const float qr = fmaf(w.x, ur[k], sr[k]);
-                const float qi = fmaf(w.x, ui[k], si[k]);
-                sr[k] = fmaf(a.x, qr, fmaf(-a.y, qi, w.y * vr[k]));
-                si[k] = fmaf(a.x, qi, fmaf(a.y, qr, w.y * vi[k]));
-                ur[k] = vr[k];
-                ui[k] = vi[k];
-                if (!FULL) {
-                    const float nr = a.x * pr[k] - a.y * pi[k];
-                    pi[k] = a.x * pi[k] + a.y * pr[k];
-                    pr[k] = nr;
-                }
+            for (int q = 0; q < kM3Pairs / 2; ++q) {
+                const float4 a = fa4[q];
+                st[2 * q] = cmul_add(make_float2(a.x, a.y), st[2 * q], v[2 * q]);
+                st[2 * q + 1] = cmul_add(make_float2(a.z, a.w), st[2 * q + 1], v[2 * q + 1]);
             }
             if (FULL) {
+                const int64_t row = static_cast<int64_t>(b) * p.L + ts + tt;
+                const float* kap = fk + (tt * kM3Heads + hl) * R * R;
 #pragma unroll
-                for (int r = 0; r < kM3MaxRank; ++r) {
-                    if (r < R) {
-                        float acc = 0.0f;
+                for (int r = 0; r < R; ++r) {
+                    // sum_k Re(conj(c_k) q_k) = sum_k (c_re q_re + c_im q_im), then kappa
+                    float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
-                        for (int q = 0; q < kM3N / 4; ++q) {
-                            const float4 cc = sm.c[tt][r][hl][q];
-                            acc = fmaf(cc.x, sr[2 * q], acc);
-                            acc = fmaf(cc.y, si[2 * q], acc);
-                            acc = fmaf(cc.z, sr[2 * q + 1], acc);
-                            acc = fmaf(cc.w, si[2 * q + 1], acc);
-                        }
-                        float yv = fmaf(dsk, xv[r], acc);
-                        if (p.z) {
-                            const float zv = m3_bf(p.z + row * xt + r * xr + c);
-                            yv *= zv / (1.0f + expf(-zv));
-                        }
-                        p.y[row * xt + r * xr + c] = __float2bfloat16_rn(yv);
+                    for (int q = 0; q < kM3N / 4; ++q) {
+                        const float4 cc = fc[((tt * R + r) * kM3Heads + hl) * (kM3N / 4) + q];
+                        acc = fma2(make_float2(cc.x, cc.y), st[2 * q], acc);
+                        acc = fma2(make_float2(cc.z, cc.w), st[2 * q + 1], acc);
                     }
+                    float yv = acc.x + acc.y;
+#pragma unroll
+                    for (int rp = 0; rp < R; ++rp) yv = fmaf(kap[r * R + rp], xv[rp], yv);
+                    if (p.z) {
+                        // SiLU(z) = z / (1 + 2^(-z log2 e))
+                        const float zv = __bfloat162float(zs[(tt * R + r) * kM3Threads + tid]);
+                        yv *= __fdividef(zv, 1.0f + ex2_fast(-zv * kLog2e));
+                    }
+                    p.y[row * xt + r * xr + c] = __float2bfloat16_rn(yv);
                 }
             }
         }
+        __syncthreads();              // the buffer and the factors are free for the next tile
     }
+    cp_async_wait<0>();
 
     if (FULL) {
         if (chunk == p.chunks - 1) {
+            // past the last token the tap weight is 0: q is the state s
             float4* hp = reinterpret_cast<float4*>(p.h_last + (static_cast<int64_t>(b) * C + c) * kM3N);
 #pragma unroll
-            for (int q = 0; q < kM3N / 4; ++q)
-                hp[q] = make_float4(sr[2 * q], si[2 * q], sr[2 * q + 1], si[2 * q + 1]);
+            for (int q = 0; q < kM3N / 4; ++q) hp[q] = make_float4(st[2 * q].x, st[2 * q].y, st[2 * q + 1].x, st[2 * q + 1].y);
         }
     } else {
         float4* ep = reinterpret_cast<float4*>(
             p.ws_state + ((static_cast<int64_t>(chunk) * gridDim.z + b) * C + c) * kM3N);
 #pragma unroll
-        for (int q = 0; q < kM3N / 4; ++q) ep[q] = make_float4(sr[2 * q], si[2 * q], sr[2 * q + 1], si[2 * q + 1]);
-        if (tid % kM3P == 0) {
-            float4* pp = reinterpret_cast<float4*>(
-                p.ws_prod + ((static_cast<int64_t>(chunk) * gridDim.z + b) * p.H + h) * kM3N);
-#pragma unroll
-            for (int q = 0; q < kM3N / 4; ++q) pp[q] = make_float4(pr[2 * q], pi[2 * q], pr[2 * q + 1], pi[2 * q + 1]);
+        for (int q = 0; q < kM3N / 4; ++q) ep[q] = make_float4(st[2 * q].x, st[2 * q].y, st[2 * q + 1].x, st[2 * q + 1].y);
+        if (tid < kM3Heads * kM3Pairs) {
+            // (head h0_ + tid / pairs, pair tid % pairs)
+            float* pp = p.ws_prod + ((static_cast<int64_t>(chunk) * gridDim.z + b) * p.H + h0_ + tid / kM3Pairs) * kM3N +
+                        2 * (tid % kM3Pairs);
+            pp[0] = prod.x;
+            pp[1] = prod.y;
         }
     }
 }

@@ -1580,6 +1580,25 @@ M3Plan plan_m3(int64_t batch, int64_t seqlen, int64_t heads, int sms) {
     return pl;
 }
 
+// The summary pass (when the sequence is cut in time) and the full pass, for
+// R inputs per state.
+template <int R>
+cudaError_t launch_m3(const mm::M3Params& p, unsigned cx, int64_t batch, cudaStream_t s) {
+    const int smem = forced_launch_failure() ? (1 << 20) : mm::m3_layout(R).bytes();
+    static std::atomic<unsigned long long> allowed_sum{0}, allowed_full{0};
+    cudaError_t e = allow_smem(mm::m3_chunk_kernel<false, R>, allowed_sum);
+    if (e == cudaSuccess) e = allow_smem(mm::m3_chunk_kernel<true, R>, allowed_full);
+    if (e != cudaSuccess) return e;
+    if (p.chunks > 1) {
+        mm::m3_chunk_kernel<false, R><<<dim3(cx, static_cast<unsigned>(p.chunks - 1), static_cast<unsigned>(batch)),
+                                        mm::kM3Threads, smem, s>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    mm::m3_chunk_kernel<true, R><<<dim3(cx, static_cast<unsigned>(p.chunks), static_cast<unsigned>(batch)),
+                                   mm::kM3Threads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
 bool m3_sizes_ok(int64_t batch, int64_t seqlen, int64_t rank, int64_t heads, int64_t groups) {
     if (batch < 0 || seqlen < 0 || heads <= 0 || groups <= 0 || heads % groups != 0) return false;
     if (rank != 1 && rank != 2 && rank != 4) return false;
@@ -1675,15 +1694,9 @@ mm_status mamba_m3_fwd(const void* x, const void* z, const void* dt, const void*
     p.G = static_cast<int>(groups);
     p.chunks = pl.chunks;
     const unsigned cx = static_cast<unsigned>(C / mm::kM3Threads);
-    const bool fail = forced_launch_failure();
-    if (pl.chunks > 1) {
-        mm::m3_chunk_kernel<false><<<dim3(cx, static_cast<unsigned>(pl.chunks - 1), static_cast<unsigned>(batch)),
-                                     fail ? 2048 : mm::kM3Threads, 0, s>>>(p);
-        if (cudaGetLastError() != cudaSuccess) return MM_ERR_CUDA;
-    }
-    mm::m3_chunk_kernel<true><<<dim3(cx, static_cast<unsigned>(pl.chunks), static_cast<unsigned>(batch)),
-                                fail ? 2048 : mm::kM3Threads, 0, s>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return MM_ERR_CUDA;
+    cudaError_t e = rank == 1 ? launch_m3<1>(p, cx, batch, s) : rank == 2 ? launch_m3<2>(p, cx, batch, s)
+                                                                          : launch_m3<4>(p, cx, batch, s);
+    if (e != cudaSuccess) { cudaGetLastError(); return MM_ERR_CUDA; }
     return MM_OK;
 }
 
