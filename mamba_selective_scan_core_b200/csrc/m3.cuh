@@ -205,9 +205,13 @@ m3_chunk_kernel(const M3Params p)
     // term is, per output r, sum_r' x_t[r'] (C_t[r] . B_t[r']) times that
     // weight, a per-(token, head) matrix kappa that also holds the skip D.
     // Past the last token the weight is 0, so q is s there.
-    float2 st[kM3Pairs];
+    // The state of pairs 2q and 2q+1 as two packed registers: sre[q] their
+    // real parts, sim[q] their imaginary parts, so that a complex
+    // multiply-add of both pairs is four packed f32x2 FMAs with no operand
+    // swaps.  Memory keeps (re, im) per pair.
+    float2 sre[kM3Pairs / 2], sim[kM3Pairs / 2];
 #pragma unroll
-    for (int k = 0; k < kM3Pairs; ++k) st[k] = make_float2(0.0f, 0.0f);
+    for (int q = 0; q < kM3Pairs / 2; ++q) sre[q] = sim[q] = make_float2(0.0f, 0.0f);
     if (FULL) {
         // q_{-1} = h0 + (1 - lambda_0) Delta_0 u_{-1}
         if (p.h0) {
@@ -215,8 +219,8 @@ m3_chunk_kernel(const M3Params p)
 #pragma unroll
             for (int q = 0; q < kM3N / 4; ++q) {
                 const float4 v = hp[q];
-                st[2 * q] = make_float2(v.x, v.y);
-                st[2 * q + 1] = make_float2(v.z, v.w);
+                sre[q] = make_float2(v.x, v.z);
+                sim[q] = make_float2(v.y, v.w);
             }
         }
         if (p.x_prev && p.B_prev && p.L > 0) {
@@ -229,7 +233,10 @@ m3_chunk_kernel(const M3Params p)
                             p.B_prev + static_cast<int64_t>(b) * R * br + g * kM3N, xr, br, up);
             const float2 w0 = make_float2((1.0f - lam) * dl, (1.0f - lam) * dl);
 #pragma unroll
-            for (int k = 0; k < kM3Pairs; ++k) st[k] = fma2(w0, up[k], st[k]);
+            for (int q = 0; q < kM3Pairs / 2; ++q) {
+                sre[q] = fma2(w0, make_float2(up[2 * q].x, up[2 * q + 1].x), sre[q]);
+                sim[q] = fma2(w0, make_float2(up[2 * q].y, up[2 * q + 1].y), sim[q]);
+            }
         }
         // carried through the earlier chunks: q = prod_c' q + e_c'
         for (int cc = 0; cc < chunk; ++cc) {
@@ -239,9 +246,12 @@ m3_chunk_kernel(const M3Params p)
                 p.ws_state + ((static_cast<int64_t>(cc) * gridDim.z + b) * C + c) * kM3N);
 #pragma unroll
             for (int q = 0; q < kM3N / 4; ++q) {
-                const float4 a = pp[q], e = ep[q];
-                st[2 * q] = cmul_add(make_float2(a.x, a.y), st[2 * q], make_float2(e.x, e.y));
-                st[2 * q + 1] = cmul_add(make_float2(a.z, a.w), st[2 * q + 1], make_float2(e.z, e.w));
+                const float4 a = pp[q], e = ep[q];     // (re, im) of pairs 2q, 2q+1
+                const float2 ar = make_float2(a.x, a.z), ai = make_float2(a.y, a.w);
+                const float2 nr = fma2(ar, sre[q], fma2(make_float2(-ai.x, -ai.y), sim[q], make_float2(e.x, e.z)));
+                const float2 ni = fma2(ar, sim[q], fma2(ai, sre[q], make_float2(e.y, e.w)));
+                sre[q] = nr;
+                sim[q] = ni;
             }
         }
     }
@@ -289,7 +299,10 @@ m3_chunk_kernel(const M3Params p)
             float sn, cs;
             sincosf(dl * p.theta[hd * kM3Pairs + k], &sn, &cs);
             const float mag = expf(dl * p.A[hd]);
-            fa[e] = make_float2(mag * cs, mag * sn);
+            // per (token, head) and pair block q: (re 2q, re 2q+1, im 2q, im 2q+1)
+            float* fq = reinterpret_cast<float*>(fa) + th * kM3N + (k >> 1) * 4 + (k & 1);
+            fq[0] = mag * cs;
+            fq[2] = mag * sn;
         }
         // omega_t B_t and C_t, widened to fp32
         const uint2* braw = reinterpret_cast<const uint2*>(m3_sm + lay.off_b(buf));
@@ -297,9 +310,12 @@ m3_chunk_kernel(const M3Params p)
         for (int e = tid; e < n * R * kM3Heads * (kM3N / 4); e += kM3Threads) {
             const int hh = (e / (kM3N / 4)) % kM3Heads, tt = e / (kM3N / 4 * kM3Heads * R);
             const float om = fw[tt * kM3Heads + hh].y + fw[(tt + 1) * kM3Heads + hh].x;
-            const float4 bv = m3_widen4(braw[e]);
-            fb[e] = make_float4(om * bv.x, om * bv.y, om * bv.z, om * bv.w);
-            if (FULL) fc[e] = m3_widen4(craw[e]);
+            const float4 bv = m3_widen4(braw[e]);      // (re, im, re, im) of pairs 2q, 2q+1
+            fb[e] = make_float4(om * bv.x, om * bv.z, om * bv.y, om * bv.w);
+            if (FULL) {
+                const float4 cv = m3_widen4(craw[e]);
+                fc[e] = make_float4(cv.x, cv.z, cv.y, cv.w);
+            }
         }
         // kappa[t][head][r][r'] = D [r == r'] - (1 - lambda_{t+1}) Delta_{t+1} (C_t[r] . B_t[r'])
         if (FULL) {
@@ -319,33 +335,40 @@ m3_chunk_kernel(const M3Params p)
         }
         __syncthreads();
         if (!FULL && tid < kM3Heads * kM3Pairs) {
-            for (int tt = 0; tt < n; ++tt) prod = cmul_add(fa[tt * kM3Heads * kM3Pairs + tid], prod, make_float2(0.0f, 0.0f));
+            const float* fq = reinterpret_cast<const float*>(fa) + (tid / kM3Pairs) * kM3N +
+                              ((tid % kM3Pairs) >> 1) * 4 + (tid & 1);
+            for (int tt = 0; tt < n; ++tt)
+                prod = cmul_add(make_float2(fq[tt * kM3Heads * kM3N], fq[tt * kM3Heads * kM3N + 2]), prod,
+                                make_float2(0.0f, 0.0f));
         }
 
         for (int tt = 0; tt < n; ++tt) {
             float xv[R];
 #pragma unroll
             for (int r = 0; r < R; ++r) xv[r] = __bfloat162float(xs[(tt * R + r) * kM3Threads + tid]);
-            // q = a q + sum_r (omega b_r) x_r
-            float2 v[kM3Pairs];
+            // q = a q + sum_r (omega b_r) x_r, two pairs per packed register
+            float2 vre[kM3Pairs / 2], vim[kM3Pairs / 2];
 #pragma unroll
-            for (int k = 0; k < kM3Pairs; ++k) v[k] = make_float2(0.0f, 0.0f);
+            for (int q = 0; q < kM3Pairs / 2; ++q) vre[q] = vim[q] = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int r = 0; r < R; ++r) {
                 const float2 x2 = make_float2(xv[r], xv[r]);
 #pragma unroll
                 for (int q = 0; q < kM3N / 4; ++q) {
                     const float4 bb = fb[((tt * R + r) * kM3Heads + hl) * (kM3N / 4) + q];
-                    v[2 * q] = fma2(make_float2(bb.x, bb.y), x2, v[2 * q]);
-                    v[2 * q + 1] = fma2(make_float2(bb.z, bb.w), x2, v[2 * q + 1]);
+                    vre[q] = fma2(make_float2(bb.x, bb.y), x2, vre[q]);
+                    vim[q] = fma2(make_float2(bb.z, bb.w), x2, vim[q]);
                 }
             }
-            const float4* fa4 = reinterpret_cast<const float4*>(fa + (tt * kM3Heads + hl) * kM3Pairs);
+            const float4* fa4 = reinterpret_cast<const float4*>(fa) + (tt * kM3Heads + hl) * (kM3N / 4);
 #pragma unroll
             for (int q = 0; q < kM3Pairs / 2; ++q) {
-                const float4 a = fa4[q];
-                st[2 * q] = cmul_add(make_float2(a.x, a.y), st[2 * q], v[2 * q]);
-                st[2 * q + 1] = cmul_add(make_float2(a.z, a.w), st[2 * q + 1], v[2 * q + 1]);
+                const float4 a = fa4[q];              // (re, re, im, im) of pairs 2q, 2q+1
+                const float2 ar = make_float2(a.x, a.y), ai = make_float2(a.z, a.w);
+                const float2 nr = fma2(ar, sre[q], fma2(make_float2(-a.z, -a.w), sim[q], vre[q]));
+                const float2 ni = fma2(ar, sim[q], fma2(ai, sre[q], vim[q]));
+                sre[q] = nr;
+                sim[q] = ni;
             }
             if (FULL) {
                 const int64_t row = static_cast<int64_t>(b) * p.L + ts + tt;
@@ -357,8 +380,8 @@ m3_chunk_kernel(const M3Params p)
 #pragma unroll
                     for (int q = 0; q < kM3N / 4; ++q) {
                         const float4 cc = fc[((tt * R + r) * kM3Heads + hl) * (kM3N / 4) + q];
-                        acc = fma2(make_float2(cc.x, cc.y), st[2 * q], acc);
-                        acc = fma2(make_float2(cc.z, cc.w), st[2 * q + 1], acc);
+                        acc = fma2(make_float2(cc.x, cc.y), sre[q], acc);
+                        acc = fma2(make_float2(cc.z, cc.w), sim[q], acc);
                     }
                     float yv = acc.x + acc.y;
 #pragma unroll
@@ -381,13 +404,13 @@ m3_chunk_kernel(const M3Params p)
             // past the last token the tap weight is 0: q is the state s
             float4* hp = reinterpret_cast<float4*>(p.h_last + (static_cast<int64_t>(b) * C + c) * kM3N);
 #pragma unroll
-            for (int q = 0; q < kM3N / 4; ++q) hp[q] = make_float4(st[2 * q].x, st[2 * q].y, st[2 * q + 1].x, st[2 * q + 1].y);
+            for (int q = 0; q < kM3N / 4; ++q) hp[q] = make_float4(sre[q].x, sim[q].x, sre[q].y, sim[q].y);
         }
     } else {
         float4* ep = reinterpret_cast<float4*>(
             p.ws_state + ((static_cast<int64_t>(chunk) * gridDim.z + b) * C + c) * kM3N);
 #pragma unroll
-        for (int q = 0; q < kM3N / 4; ++q) ep[q] = make_float4(st[2 * q].x, st[2 * q].y, st[2 * q + 1].x, st[2 * q + 1].y);
+        for (int q = 0; q < kM3N / 4; ++q) ep[q] = make_float4(sre[q].x, sim[q].x, sre[q].y, sim[q].y);
         if (tid < kM3Heads * kM3Pairs) {
             // (head h0_ + tid / pairs, pair tid % pairs)
             float* pp = p.ws_prod + ((static_cast<int64_t>(chunk) * gridDim.z + b) * p.H + h0_ + tid / kM3Pairs) * kM3N +
