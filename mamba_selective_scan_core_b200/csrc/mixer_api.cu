@@ -1544,7 +1544,7 @@ mm_status mamba_ssd_fwd(const void* x, const void* z, const void* dt, const floa
     if (pl.chunks > 0) {
         static std::atomic<unsigned long long> allowed_scan{0};
         if (allow_smem(mm::ssd_chunk_scan_kernel, allowed_scan) != cudaSuccess) { cudaGetLastError(); return MM_ERR_CUDA; }
-        mm::ssd_chunk_scan_kernel<<<cgrid, mm::kSsdThreads,
+        mm::ssd_chunk_scan_kernel<<<cgrid, mm::kSsdScanThreads,
                                     fail ? (1 << 20) : mm::SsdScanLayout::smem_bytes, s>>>(p, tc, tb, th, tx, tz);
         if (cudaGetLastError() != cudaSuccess) return MM_ERR_CUDA;
     }

@@ -52,6 +52,7 @@ constexpr int kSsdQ = 128;        // tokens per chunk (the products' M)
 constexpr int kSsdP = 64;         // channels per head
 constexpr int kSsdN = 128;        // d_state
 constexpr int kSsdThreads = 128;  // one token (or one state row) per thread
+constexpr int kSsdScanThreads = 256;   // the chunk scan: two warpgroups share each row
 
 struct SsdParams {
     const __nv_bfloat16* x;      // [B][L][H*P]
@@ -113,10 +114,10 @@ __device__ __forceinline__ void ssd_fail(const SsdParams& p) {
 // this thread's Delta.  Contains __syncthreads.
 __device__ __forceinline__ void ssd_chunk_prefix(const SsdParams& p, int b, int h, int64_t t0, float* delta,
                                                  float* cum2, float* warp_sums) {
-    const int j = threadIdx.x, lane = j & 31, warp = j >> 5;
+    const int j = threadIdx.x, lane = j & 31, warp = j >> 5;   // token j of the chunk (threads past Q idle)
     const int64_t t = t0 + j;
     float dl = 0.0f;
-    if (t < p.L) {
+    if (j < kSsdQ && t < p.L) {
         const float v = __bfloat162float(p.dt[(static_cast<int64_t>(b) * p.L + t) * p.H + h]) +
                         (p.dt_bias ? p.dt_bias[h] : 0.0f);
         dl = fmaxf(v, 0.0f) + log1pf(expf(-fabsf(v)));
@@ -127,11 +128,13 @@ __device__ __forceinline__ void ssd_chunk_prefix(const SsdParams& p, int b, int 
         const float n = __shfl_up_sync(kFull, v, o);
         if (lane >= o) v += n;
     }
-    if (lane == 31) warp_sums[warp] = v;
+    if (lane == 31 && j < kSsdQ) warp_sums[warp] = v;
     __syncthreads();
-    for (int w = 0; w < warp; ++w) v += warp_sums[w];
-    delta[j] = dl;
-    cum2[j] = v;
+    if (j < kSsdQ) {
+        for (int w = 0; w < warp; ++w) v += warp_sums[w];
+        delta[j] = dl;
+        cum2[j] = v;
+    }
     __syncthreads();
 }
 
@@ -296,6 +299,7 @@ __global__ void __launch_bounds__(256)
 ssd_state_pass_kernel(const SsdParams p)
 {
     constexpr int64_t kHead = int64_t(kSsdP) * kSsdN;
+    constexpr int kAhead = 4;     // chunks whose S is requested before their H_in stores
     const int64_t per_seq = int64_t(p.H) * kHead;
     const int64_t f = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
     if (f >= per_seq) return;
@@ -303,19 +307,32 @@ ssd_state_pass_kernel(const SsdParams p)
     const int h = static_cast<int>(f / kHead);
     float4 s = p.h0 ? *reinterpret_cast<const float4*>(p.h0 + b * per_seq + f) : make_float4(0.f, 0.f, 0.f, 0.f);
     const float* dec = p.dec + (static_cast<int64_t>(b) * p.H + h) * p.chunks;
-    for (int c = 0; c < p.chunks; ++c) {
-        const int64_t off = (static_cast<int64_t>(b) * p.chunks + c) * per_seq + f;
-        uint2 hi, lo;
-        split_bf16x2(s.x, s.y, hi.x, lo.x);
-        split_bf16x2(s.z, s.w, hi.y, lo.y);
-        *reinterpret_cast<uint2*>(p.Hin + off) = hi;
-        *reinterpret_cast<uint2*>(p.Hin + p.hin_lo + off) = lo;
-        const float d = dec[c];
-        const float4 add = *reinterpret_cast<const float4*>(p.S + off);
-        s.x = fmaf(d, s.x, add.x);
-        s.y = fmaf(d, s.y, add.y);
-        s.z = fmaf(d, s.z, add.z);
-        s.w = fmaf(d, s.w, add.w);
+    const float* __restrict__ S = p.S;
+    for (int c0 = 0; c0 < p.chunks; c0 += kAhead) {
+        float4 add[kAhead];
+        float d[kAhead];
+#pragma unroll
+        for (int j = 0; j < kAhead; ++j) {
+            if (c0 + j < p.chunks) {
+                add[j] = __ldcs(reinterpret_cast<const float4*>(S + (static_cast<int64_t>(b) * p.chunks + c0 + j) * per_seq + f));
+                d[j] = dec[c0 + j];
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kAhead; ++j) {
+            if (c0 + j < p.chunks) {
+                const int64_t off = (static_cast<int64_t>(b) * p.chunks + c0 + j) * per_seq + f;
+                uint2 hi, lo;
+                split_bf16x2(s.x, s.y, hi.x, lo.x);
+                split_bf16x2(s.z, s.w, hi.y, lo.y);
+                *reinterpret_cast<uint2*>(p.Hin + off) = hi;
+                *reinterpret_cast<uint2*>(p.Hin + p.hin_lo + off) = lo;
+                s.x = fmaf(d[j], s.x, add[j].x);
+                s.y = fmaf(d[j], s.y, add[j].y);
+                s.z = fmaf(d[j], s.z, add[j].z);
+                s.w = fmaf(d[j], s.w, add[j].w);
+            }
+        }
     }
     *reinterpret_cast<float4*>(p.h_last + b * per_seq + f) = s;
 }
@@ -340,7 +357,7 @@ static_assert(SsdScanLayout::b_off % 1024 == 0 && SsdScanLayout::h_off % 1024 ==
 // Tensor memory columns of the chunk scan: G [Q x Q], C H_in^T [Q x P], M X [Q x P].
 constexpr uint32_t kSsdColG = 0, kSsdColOff = 128, kSsdColDiag = 192, kSsdCols = 256;
 
-__global__ void __launch_bounds__(kSsdThreads, 2)
+__global__ void __launch_bounds__(kSsdScanThreads, 2)
 ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_c,
                       const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_h,
                       const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z)
@@ -358,7 +375,8 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
 
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, wg = warp >> 2;   // tensor-memory lane quarter; warpgroup
     const int64_t t0 = static_cast<int64_t>(c) * kSsdQ;
     const int g = h / (p.H / p.G);
 
@@ -389,7 +407,7 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
     ssd_chunk_prefix(p, b, h, t0, delta, cum2, warp_sums);   // syncs
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
 
     // products 1: G = C B^T (N = Q) and C H_in^T (N = P, hi and lo), K = N = 128
     bool loaded = true, ok = true;
@@ -428,16 +446,17 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
     const bool g_ready = __syncthreads_and(issued1 && ok);
 
     // M[i][j] = G[i][j] exp(cum_i - cum_j) Delta_j for j <= i, 0 above the
-    // diagonal, plus D on it; row i (this thread) as hi and lo parts over the
-    // B and H_in tiles (both free now)
-    const int i = tid;
+    // diagonal, plus D on it; row i as hi and lo parts over the B and H_in
+    // tiles (both free now).  Row i belongs to lane quarter i / 32; the two
+    // warpgroups take its even and odd 32-column blocks.
+    const int i = quarter * 32 + lane;
     if (g_ready) {
         const float ci = cum2[i];
         const float dsk = p.Dskip ? p.Dskip[h] : 0.0f;
 #pragma unroll 1
-        for (int jb = 0; jb < kSsdQ / 32; ++jb) {
+        for (int jb = wg; jb < kSsdQ / 32; jb += 2) {
             float m[32];
-            if (jb <= warp) {     // warp-uniform: blocks above the diagonal block are zero
+            if (jb <= quarter) {     // warp-uniform: blocks above the diagonal block are zero
                 tmem_ld32(lane_base + kSsdColG + jb * 32, m);
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
@@ -500,14 +519,14 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
         const float e = ex2_fast(cum2[i]);
         const unsigned char* zrow = ct + kSsdQ * kSsdP * 2 + i * 128;
         unsigned char* yrow = ct + i * 128;
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
+        {
+            // this warpgroup's 32 output columns of row i
             float yo[32], yd[32];
-            tmem_ld32(lane_base + kSsdColOff + half * 32, yo);
-            tmem_ld32(lane_base + kSsdColDiag + half * 32, yd);
+            tmem_ld32(lane_base + kSsdColOff + wg * 32, yo);
+            tmem_ld32(lane_base + kSsdColDiag + wg * 32, yd);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const int piece = (half * 4 + q) ^ (i & 7);
+                const int piece = (wg * 4 + q) ^ (i & 7);
                 float o[8];
 #pragma unroll
                 for (int e2 = 0; e2 < 8; ++e2) o[e2] = fmaf(e, yo[q * 8 + e2], yd[q * 8 + e2]);
@@ -528,12 +547,12 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
             }
         }
         __syncthreads();
-        // thread k: piece k % 8 of rows k / 8 + 16 m; only rows in the sequence
+        // thread k: piece k % 8 of rows k / 8 + 32 m; only rows in the sequence
         const int q = tid & 7;
         const int64_t ld = static_cast<int64_t>(p.H) * kSsdP;
-#pragma unroll 4
-        for (int m = 0; m < kSsdQ / 16; ++m) {
-            const int r = (tid >> 3) + 16 * m;
+#pragma unroll
+        for (int m = 0; m < kSsdQ * 8 / kSsdScanThreads; ++m) {
+            const int r = (tid >> 3) + (kSsdScanThreads / 8) * m;
             if (t0 + r < p.L) {
                 const uint4 v = *reinterpret_cast<const uint4*>(ct + r * 128 + ((q ^ (r & 7)) << 4));
                 *reinterpret_cast<uint4*>(p.y + (static_cast<int64_t>(b) * p.L + t0 + r) * ld + h * kSsdP + q * 8) = v;
