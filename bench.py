@@ -85,13 +85,19 @@ def _measured_peaks():
 
 
 # The CUDA sources each traffic record depends on (its kernel, the shared
-# helpers and the launch code).
+# helpers and the launch code).  "mixer_api.cu#head" is the host file up to
+# its Mamba-2 section: the launch code of the Mamba form, its decode step and
+# the projections, which the Mamba-2 and Mamba-3 host code after it does not
+# touch.
+API_HEAD = "mixer_api.cu#head"
+API_HEAD_END = "// ---------------------------------------------------------------- Mamba-2 form"
 TRAFFIC_SOURCES = {
-    "mixer_fwd/jamba_prefill": ("mixer_prefill.cuh", "mixer_common.cuh", "mixer_api.cu"),
-    "state_update_kernel/decode_28x128": ("mixer_decode.cuh", "mixer_common.cuh", "mixer_api.cu"),
-    "proj_gemm/x_proj": ("proj_gemm.cuh", "mixer_common.cuh", "mixer_api.cu"),
-    "proj_gemm/dt_proj": ("proj_gemm.cuh", "mixer_common.cuh", "mixer_api.cu"),
+    "mixer_fwd/jamba_prefill": ("mixer_prefill.cuh", "mixer_common.cuh", API_HEAD),
+    "state_update_kernel/decode_28x128": ("mixer_decode.cuh", "mixer_common.cuh", API_HEAD),
+    "proj_gemm/x_proj": ("proj_gemm.cuh", "mixer_common.cuh", API_HEAD),
+    "proj_gemm/dt_proj": ("proj_gemm.cuh", "mixer_common.cuh", API_HEAD),
     "ssd/mamba2_prefill": ("ssd.cuh", "proj_gemm.cuh", "mixer_common.cuh", "mixer_api.cu"),
+    "m3/mamba3_prefill": ("m3.cuh", "mixer_common.cuh", "mixer_api.cu"),
 }
 
 
@@ -104,10 +110,13 @@ def _kernel_source_sha(names=None):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mamba_selective_scan_core_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if not name.endswith((".cuh", ".cu")) or (names is not None and name not in names):
+        head_only = names is not None and name + "#head" in names
+        if not name.endswith((".cuh", ".cu")) or (names is not None and name not in names and not head_only):
             continue
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
             src = f.read()
+        if head_only and API_HEAD_END in src:
+            src = src[:src.index(API_HEAD_END)]
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
         src = re.sub(r"//[^\n]*", "", src)
         src = "\n".join(line.strip() for line in src.splitlines() if line.strip())
@@ -820,8 +829,9 @@ def run_m3(mm, args, world, hbm_peak, hbm_src, alu_peak, cfg):
         "d_state": cfg.d_state, "rank": cfg.rank, "steps": K, "ms_per_step": round(ms, 5),
         "value": round(_job_rate(world, B * L, ms), 1), "unit": "tokens/s", "launches_per_call": 2,
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
-                     "frac": round(gbs / hbm_peak, 4), "traffic": None, "algorithmic_bytes": nbytes,
-                     "peak_source": hbm_src},
+                     "frac": round(gbs / hbm_peak, 4),
+                     "traffic": _ncu_traffic("m3/" + cfg.name) if cfg.name in ("mamba3_prefill",) else None,
+                     "algorithmic_bytes": nbytes, "peak_source": hbm_src},
         "roofline_alu": {"bound": "alu", "achieved": round(alu, 3), "peak": round(alu_peak, 3),
                          "unit": "T fp32-pipe ops/s", "frac": round(alu / alu_peak, 4),
                          "ops_per_token_channel": m3_fp32_ops(cfg),
