@@ -346,8 +346,8 @@ struct SsdScanLayout {
     static constexpr int b_off = c_off + kSsdQ * kSsdN * 2;         // B [Q rows][N] 32 KB, then M hi [Q rows][Q]
     static constexpr int h_off = b_off + kSsdQ * kSsdN * 2;         // H_in hi, lo [P rows][N] 2 x 16 KB, then M lo
     static constexpr int hin_bytes = kSsdP * kSsdN * 2;
-    static constexpr int f_off = h_off + 2 * hin_bytes;             // delta, cum2, warp sums
-    static constexpr int bar_off = f_off + 2 * kSsdQ * 4 + 16;
+    static constexpr int f_off = h_off + 2 * hin_bytes;             // delta, cum2, warp sums, column factors
+    static constexpr int bar_off = f_off + 3 * kSsdQ * 4 + 16;
     static constexpr int smem_bytes = 1024 + bar_off + 4 * 8 + 16;
     static constexpr uint32_t tx_bytes = 2 * kSsdQ * kSsdN * 2 + 2 * hin_bytes;
 };
@@ -371,6 +371,7 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
     float* delta = reinterpret_cast<float*>(sm + Lay::f_off);
     float* cum2 = delta + kSsdQ;
     float* warp_sums = cum2 + kSsdQ;
+    float* colf = warp_sums + 4;          // exp(cum_j0 - cum_j) Delta_j, j0 the first column of j's 32-column block
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::bar_off);   // loaded, products 1, product 2, x loaded
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
 
@@ -405,6 +406,12 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
         tc_fence_before();
     }
     ssd_chunk_prefix(p, b, h, t0, delta, cum2, warp_sums);   // syncs
+    // The decay of M's element (i, j) factors within j's 32-column block:
+    // exp(cum_i - cum_j) = exp(cum_i - cum_j0) exp(cum_j0 - cum_j), the second
+    // factor (with Delta_j) once per column here, the first once per row and
+    // block below.  A block whose own decay range exceeds 2^60 keeps one
+    // exponential per element instead (no overflow, no lost small terms).
+    if (tid < kSsdQ) colf[tid] = ex2_fast(cum2[tid & ~31] - cum2[tid]) * delta[tid];
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -458,11 +465,22 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
             float m[32];
             if (jb <= quarter) {     // warp-uniform: blocks above the diagonal block are zero
                 tmem_ld32(lane_base + kSsdColG + jb * 32, m);
+                const float c0 = cum2[jb * 32];
+                if (c0 - cum2[jb * 32 + 31] <= 60.0f) {     // the same for every thread of the CTA
+                    const float ei = ex2_fast(ci - c0);
 #pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    const int j = jb * 32 + q;
-                    m[q] = j <= i ? m[q] * ex2_fast(ci - cum2[j]) * delta[j] : 0.0f;
-                    if (j == i) m[q] += dsk;
+                    for (int q = 0; q < 32; ++q) {
+                        const int j = jb * 32 + q;
+                        m[q] = j <= i ? m[q] * ei * colf[j] : 0.0f;
+                        if (j == i) m[q] += dsk;
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) {
+                        const int j = jb * 32 + q;
+                        m[q] = j <= i ? m[q] * ex2_fast(ci - cum2[j]) * delta[j] : 0.0f;
+                        if (j == i) m[q] += dsk;
+                    }
                 }
             } else {
 #pragma unroll
