@@ -160,3 +160,27 @@ def test_m3_mimo_full_size_sampled_heads():
     y, h = gpu_m3(to_dev(inp))
     torch.cuda.synchronize()
     check(inp, y, h, heads=[0, 1, 13, 29, 41, 57, 64, 77, 90, 103, 126, 127])
+
+
+def test_m3_token_by_token_continues_prefill():
+    """Decode use: a prefill of 45 tokens, then three one-token calls, each
+    taking the previous call's h_last as h0 and its last x and B rows as
+    x_prev / B_prev, matches the oracle's single run of all 48 tokens."""
+    inp = make_m3_inputs_custom(2, 48, 4, rank=2, groups=2, seed=47, h0_std=0.2, prev=True)
+    d = to_dev(inp)
+
+    def part(lo, hi, h0, xp, bp):
+        c = dict(d)
+        for k in ("x", "z", "dt", "trap", "Bm", "Cm"):
+            c[k] = d[k][:, lo:hi].contiguous()
+        c.update(h0=h0, x_prev=xp, B_prev=bp)
+        return gpu_m3(c)
+
+    ys = []
+    y, h = part(0, 45, d["h0"], d["x_prev"], d["B_prev"])
+    ys.append(y)
+    for t in range(45, 48):
+        y, h = part(t, t + 1, h, d["x"][:, t - 1].contiguous(), d["Bm"][:, t - 1].contiguous())
+        ys.append(y)
+    torch.cuda.synchronize()
+    check(inp, torch.cat(ys, dim=1), h)
