@@ -63,6 +63,8 @@ struct M3Params {
     float* ws_prod;                // [K-1][B][H][N]     chunk products of a_t (pairs)
     int64_t L, chunk_len;
     int R, H, G, chunks;
+    unsigned long long* status;    // [1] <- the call's epoch (these kernels have no wait that can give up)
+    unsigned long long status_epoch;
 };
 
 // Shared memory of a CTA: two buffers of raw tile inputs, filled by
@@ -178,6 +180,8 @@ m3_chunk_kernel(const M3Params p)
 {
     extern __shared__ __align__(16) unsigned char m3_sm[];
     constexpr int T = 32 / R;
+    if (FULL && p.status && threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+        p.status[1] = p.status_epoch;
     const M3Layout lay = m3_layout(R);
     const int tid = threadIdx.x;
     const int64_t C = static_cast<int64_t>(p.H) * kM3P;

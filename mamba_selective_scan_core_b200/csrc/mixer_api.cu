@@ -1226,13 +1226,9 @@ mm_status mamba_proj_matmul(const void* A, const void* W, void* out, int64_t M, 
     if (overlaps(ws, a) || overlaps(ws, w) || overlaps(ws, o)) return MM_ERR_ALIAS;
     if (mm_status st = check_device(); st != MM_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // the call's status: hdr[1] = epoch, written before the GEMM in stream order
+    // the call's status: the GEMM writes the epoch into hdr[1]
     const unsigned long long epoch = next_call_id();
     unsigned long long* hdr = static_cast<unsigned long long*>(workspace);
-    if (cudaMemcpyAsync(hdr + 1, &epoch, sizeof(epoch), cudaMemcpyHostToDevice, s) != cudaSuccess) {
-        cudaGetLastError();
-        return MM_ERR_CUDA;
-    }
     // a tall, narrow product is split in K: fp32 partials in the workspace,
     // then summed into `out`
     const int ks = gemm_ksplit(M, N, K, sms);
@@ -1490,11 +1486,7 @@ mm_status mamba_ssd_fwd(const void* x, const void* z, const void* dt, const floa
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     unsigned char* w = static_cast<unsigned char*>(workspace);
     unsigned long long* hdr = reinterpret_cast<unsigned long long*>(w);
-    const unsigned long long epoch = next_call_id();
-    if (cudaMemcpyAsync(hdr + 1, &epoch, sizeof(epoch), cudaMemcpyHostToDevice, s) != cudaSuccess) {
-        cudaGetLastError();
-        return MM_ERR_CUDA;
-    }
+    const unsigned long long epoch = next_call_id();   // written into hdr[1] by the state-passing launch
     mm::SsdParams p{};
     p.x = static_cast<const __nv_bfloat16*>(x);
     p.z = static_cast<const __nv_bfloat16*>(z);
@@ -1662,14 +1654,12 @@ mm_status mamba_m3_fwd(const void* x, const void* z, const void* dt, const void*
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     unsigned char* w = static_cast<unsigned char*>(workspace);
-    // the call's status word: the epoch in the header's second word (these
-    // kernels have no wait that can give up, so it always reads complete)
-    const unsigned long long epoch = next_call_id();
-    if (cudaMemcpyAsync(w + 8, &epoch, sizeof(epoch), cudaMemcpyHostToDevice, s) != cudaSuccess) {
-        cudaGetLastError();
-        return MM_ERR_CUDA;
-    }
     mm::M3Params p{};
+    // the call's status word: the full pass writes the epoch into the
+    // header's second word (these kernels have no wait that can give up, so
+    // the status always reads complete)
+    p.status = reinterpret_cast<unsigned long long*>(w);
+    p.status_epoch = next_call_id();
     p.x = static_cast<const __nv_bfloat16*>(x);
     p.z = static_cast<const __nv_bfloat16*>(z);
     p.dt = static_cast<const __nv_bfloat16*>(dt);

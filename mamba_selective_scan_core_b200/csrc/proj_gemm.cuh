@@ -44,7 +44,7 @@ struct GemmParams {
     int M, N, K;
     int k_tiles_per_split;  // 64-wide K tiles per CTA (blockIdx.z covers its own range)
     unsigned wait_limit;    // tries per mbarrier wait before giving up
-    unsigned long long* status;   // optional (epoch << 8) | code word of the call, or NULL
+    unsigned long long* status;   // optional: [0] (epoch << 8) | code of a failure, [1] the call's epoch; or NULL
     unsigned long long status_epoch;
 };
 
@@ -158,6 +158,9 @@ proj_gemm_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tm_a, c
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
+    // the call's epoch, in the status word's second half (written from the
+    // device, so that a captured call records no host copy)
+    if (p.status && tid == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) p.status[1] = p.status_epoch;
     const int m0 = blockIdx.x * kGemmBM;
     const int n0 = blockIdx.y * BN * NSUB;
     const int kt0 = blockIdx.z * p.k_tiles_per_split;

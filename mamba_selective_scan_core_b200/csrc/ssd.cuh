@@ -73,7 +73,7 @@ struct SsdParams {
     int64_t L;
     int H, G, chunks, batch;
     unsigned wait_limit;
-    unsigned long long* status;  // (epoch << 8) | code of the call, or null
+    unsigned long long* status;  // [0] (epoch << 8) | code of a failure, [1] the call's epoch; or null
     unsigned long long status_epoch;
 };
 
@@ -302,6 +302,8 @@ ssd_state_pass_kernel(const SsdParams p)
     constexpr int kAhead = 4;     // chunks whose S is requested before their H_in stores
     const int64_t per_seq = int64_t(p.H) * kHead;
     const int64_t f = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+    // the call's epoch for its status word (this launch always runs)
+    if (p.status && f == 0 && blockIdx.y == 0) p.status[1] = p.status_epoch;
     if (f >= per_seq) return;
     const int b = blockIdx.y;
     const int h = static_cast<int>(f / kHead);

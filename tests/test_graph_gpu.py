@@ -81,3 +81,69 @@ def test_decode_graph_replay_advances_state_like_eager():
     assert torch.equal(st, st_e)
     assert torch.equal(cs, cs_e)
     assert torch.equal(y, y_e)
+
+
+def _replay_matches(call, outs_eager, outs):
+    """Capture call() (writing `outs`) in a graph and check that each replay
+    gives the same bits as the eager outputs."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):                       # warm up outside capture on the capture stream
+        call()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    for _ in range(2):
+        for o in outs:
+            o.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        for o, e in zip(outs, outs_eager):
+            assert torch.equal(o, e)
+
+
+def test_ssd_graph_replay_matches_eager():
+    """The Mamba-2 call (three launches; the call's epoch written by a kernel,
+    not by a host copy) captured and replayed."""
+    from workloads import make_ssd_inputs_custom
+
+    d = to_dev(make_ssd_inputs_custom(2, 600, 4, groups=2, seed=93, h0_std=0.3))
+    args = (d["x"], d["z"], d["dt"], d["dt_bias"], d["A"], d["Bm"], d["Cm"], d["Dskip"], d["h0"])
+    y_e, h_e = mm.ssd_fwd(*args)
+    torch.cuda.synchronize()
+    ws = torch.empty(mm.ssd_workspace_size(2, 600, 4, groups=2), dtype=torch.uint8, device="cuda")
+    y, h = torch.empty_like(y_e), torch.empty_like(h_e)
+    _replay_matches(lambda: mm.ssd_fwd(*args, y=y, h_last=h, workspace=ws), (y_e, h_e), (y, h))
+    assert mm.check_status(ws) == 0
+
+
+def test_m3_graph_replay_matches_eager():
+    """The Mamba-3 call (summary and full pass) captured and replayed."""
+    from workloads import make_m3_inputs_custom
+
+    d = to_dev(make_m3_inputs_custom(2, 700, 4, rank=2, groups=2, seed=94, h0_std=0.3, prev=True))
+    keys = ("x", "z", "dt", "trap", "dt_bias", "A", "theta", "Bm", "Cm", "Dskip", "h0", "x_prev", "B_prev")
+    args = tuple(d[k] for k in keys)
+    y_e, h_e = mm.m3_fwd(*args)
+    torch.cuda.synchronize()
+    ws = torch.empty(mm.m3_workspace_size(2, 700, 4, 2, groups=2), dtype=torch.uint8, device="cuda")
+    y, h = torch.empty_like(y_e), torch.empty_like(h_e)
+    _replay_matches(lambda: mm.m3_fwd(*args, y=y, h_last=h, workspace=ws), (y_e, h_e), (y, h))
+    assert mm.check_status(ws) == 0
+
+
+def test_proj_matmul_graph_replay_matches_eager():
+    """A projection product split in K (GEMM, then the sum of the partials)
+    captured and replayed."""
+    g = torch.Generator(device="cuda").manual_seed(95)
+    A = torch.randn((256, 4096), device="cuda", generator=g).to(torch.bfloat16)
+    W = (torch.randn((288, 4096), device="cuda", generator=g) / 64).to(torch.bfloat16)
+    assert mm.proj_matmul_workspace_size(256, 288, 4096) > 256, "expected a split-K plan"
+    o_e = mm.proj_matmul(A, W)
+    torch.cuda.synchronize()
+    ws = torch.empty(mm.proj_matmul_workspace_size(256, 288, 4096), dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(o_e)
+    _replay_matches(lambda: mm.proj_matmul(A, W, out=o, workspace=ws), (o_e,), (o,))
+    assert mm.check_status(ws) == 0
