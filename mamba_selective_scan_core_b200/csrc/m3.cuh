@@ -338,15 +338,66 @@ m3_chunk_kernel(const M3Params p)
             }
         }
         __syncthreads();
-        if (!FULL && tid < kM3Heads * kM3Pairs) {
-            const float* fq = reinterpret_cast<const float*>(fa) + (tid / kM3Pairs) * kM3N +
-                              ((tid % kM3Pairs) >> 1) * 4 + (tid & 1);
-            for (int tt = 0; tt < n; ++tt)
-                prod = cmul_add(make_float2(fq[tt * kM3Heads * kM3N], fq[tt * kM3Heads * kM3N + 2]), prod,
-                                make_float2(0.0f, 0.0f));
+        if (!FULL) {
+            // The summary pass needs only the chunk's end pre-state,
+            //     F = sum_t (prod_{s>t} a_s) omega_t sum_r b_{t,r} x_{t,r},
+            // whose factor V_{t,r} = (prod_{s>t} a_s) omega_t b_{t,r} is the
+            // same for all channels of a head.  Within the tile: W_t = the
+            // product of a_s over the tile's later tokens (16 threads, one per
+            // (head, pair), walking back), P = the tile's whole product; then
+            // V = W omega b in place of omega b.  Each channel then carries
+            // F <- P F + sum_t x_t V_t.
+            float* fW = reinterpret_cast<float*>(fc);           // [T][heads][N], split layout as fa
+            float* fP = fk;                                       // [heads][N]
+            if (tid < kM3Heads * kM3Pairs) {
+                const int off = (tid / kM3Pairs) * kM3N + ((tid % kM3Pairs) >> 1) * 4 + (tid & 1);
+                const float* faf = reinterpret_cast<const float*>(fa);
+                float2 w = make_float2(1.0f, 0.0f);
+                for (int tt = n - 1; tt >= 0; --tt) {
+                    fW[tt * kM3Heads * kM3N + off] = w.x;
+                    fW[tt * kM3Heads * kM3N + off + 2] = w.y;
+                    w = cmul_add(make_float2(faf[tt * kM3Heads * kM3N + off], faf[tt * kM3Heads * kM3N + off + 2]), w,
+                                 make_float2(0.0f, 0.0f));
+                }
+                fP[off] = w.x;
+                fP[off + 2] = w.y;
+                prod = cmul_add(w, prod, make_float2(0.0f, 0.0f));
+            }
+            __syncthreads();
+            for (int e = tid; e < n * R * kM3Heads * (kM3N / 4); e += kM3Threads) {
+                const int q = e % (kM3N / 4), hh = (e / (kM3N / 4)) % kM3Heads, tt = e / (kM3N / 4 * kM3Heads * R);
+                const float4 w = reinterpret_cast<const float4*>(fW)[(tt * kM3Heads + hh) * (kM3N / 4) + q];
+                const float4 v = fb[e];     // (re, re, im, im) of pairs 2q, 2q+1
+                fb[e] = make_float4(w.x * v.x - w.z * v.z, w.y * v.y - w.w * v.w,
+                                    w.x * v.z + w.z * v.x, w.y * v.w + w.w * v.y);
+            }
+            __syncthreads();
+            const float4* p4 = reinterpret_cast<const float4*>(fP) + hl * (kM3N / 4);
+#pragma unroll
+            for (int q = 0; q < kM3Pairs / 2; ++q) {
+                const float4 a = p4[q];
+                const float2 ar = make_float2(a.x, a.y), ai = make_float2(a.z, a.w);
+                const float2 nr = fma2(ar, sre[q], mul2(make_float2(-a.z, -a.w), sim[q]));
+                const float2 ni = fma2(ar, sim[q], mul2(ai, sre[q]));
+                sre[q] = nr;
+                sim[q] = ni;
+            }
+            for (int tt = 0; tt < n; ++tt) {
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const float xr_ = __bfloat162float(xs[(tt * R + r) * kM3Threads + tid]);
+                    const float2 x2 = make_float2(xr_, xr_);
+#pragma unroll
+                    for (int q = 0; q < kM3N / 4; ++q) {
+                        const float4 vv = fb[((tt * R + r) * kM3Heads + hl) * (kM3N / 4) + q];
+                        sre[q] = fma2(make_float2(vv.x, vv.y), x2, sre[q]);
+                        sim[q] = fma2(make_float2(vv.z, vv.w), x2, sim[q]);
+                    }
+                }
+            }
         }
 
-        for (int tt = 0; tt < n; ++tt) {
+        for (int tt = 0; FULL && tt < n; ++tt) {
             float xv[R];
 #pragma unroll
             for (int r = 0; r < R; ++r) xv[r] = __bfloat162float(xs[(tt * R + r) * kM3Threads + tid]);
