@@ -325,10 +325,10 @@ bool forced_launch_failure() { return env_int("MAMBA_MIXER_TEST_LAUNCH_FAIL", 1,
 
 // `dependent`: launch as a programmatic dependent of the kernel before it in
 // the stream (the summary pass of the same call), see mixer_fwd_kernel.
-template <typename T, typename M, int STAGES, bool SUMMARY>
+template <typename T, typename M, int STAGES, bool SUMMARY, int OCT = 0>
 cudaError_t launch_prefill(const PrefillParams& p, int64_t batch, int chunks, int threads, bool dependent,
                            cudaStream_t s) {
-    auto kern = mm::mixer_fwd_kernel<T, M, kTile, STAGES, SUMMARY>;
+    auto kern = mm::mixer_fwd_kernel<T, M, kTile, STAGES, SUMMARY, OCT>;
     TensorMaps maps;
     if (!make_maps<T>(p, batch, &maps)) return cudaErrorInvalidValue;
     const int smem = PrefillLayout<T>::smem_bytes(kTile, STAGES, p.octets);
@@ -404,6 +404,12 @@ cudaError_t launch_pass(PrefillParams p, const CtaShape& sh, int64_t batch, int 
                         cudaStream_t s) {
     p.octets = sh.octets;
     p.ctas_per_seq = sh.ctas_per_seq;
+    // the widest CTA (256 channels) of the bf16 path, the shape of wide layers,
+    // with its row width as a compile-time constant
+    if constexpr (std::is_same<T, __nv_bfloat16>::value && std::is_same<M, mm::MathFast>::value) {
+        if (sh.octets == 32 && sh.stages == 2 && env_int("MAMBA_MIXER_GENERIC_WIDTH", 1, 1) == 0)
+            return launch_prefill<T, M, 2, SUMMARY, 32>(p, batch, chunks, sh.threads, dependent, s);
+    }
     if (sh.stages >= 4) return launch_prefill<T, M, 4, SUMMARY>(p, batch, chunks, sh.threads, dependent, s);
     if (sh.stages == 3) return launch_prefill<T, M, 3, SUMMARY>(p, batch, chunks, sh.threads, dependent, s);
     return launch_prefill<T, M, 2, SUMMARY>(p, batch, chunks, sh.threads, dependent, s);

@@ -145,7 +145,7 @@ struct PrefillLayout {
     __host__ __device__ static constexpr int x_bytes(int tile, int octets) { return a128((tile + kHalo) * row_bytes(octets)); }
     __host__ __device__ static constexpr int zdt_bytes(int tile, int octets) { return a128(tile * row_bytes(octets)); }
     __host__ __device__ static constexpr int bc_bytes(int tile) { return a128(tile * 16 * static_cast<int>(sizeof(T))); }
-    __host__ __device__ static int stage_bytes(int tile, int octets) {
+    __host__ __device__ static constexpr int stage_bytes(int tile, int octets) {
         return x_bytes(tile, octets) + 2 * zdt_bytes(tile, octets) + 2 * bc_bytes(tile);
     }
     // plus the tile's B/C in fp32, each value duplicated ([token][B0 B0 .. C15
@@ -202,7 +202,10 @@ __device__ __forceinline__ float2 decay2(float2 l, float2 a) {
 
 // SUMMARY = true: the summary pass (chunk end state from zero + sum of l).
 // SUMMARY = false: the full fused forward over one chunk.
-template <typename T, typename M, int TILE, int STAGES, bool SUMMARY>
+// OCT > 0: the CTA width in channel octets is the compile-time constant OCT
+// (p.octets == OCT), so staged-row offsets fold into the loads' immediates;
+// OCT = 0: any width.
+template <typename T, typename M, int TILE, int STAGES, bool SUMMARY, int OCT = 0>
 __global__ void __launch_bounds__(128, MM_FWD_MIN_BLOCKS)
 mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x,
                  const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_dt,
@@ -220,24 +223,25 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
     const int seq = blockIdx.x / p.ctas_per_seq;
     const int blk = blockIdx.x - seq * p.ctas_per_seq;
     const int chunk = blockIdx.y;
-    const int d0 = blk * p.octets * 8;
-    const int nch = min(p.octets * 8, p.D - d0);
+    const int octs = OCT > 0 ? OCT : p.octets;
+    const int d0 = blk * octs * 8;
+    const int nch = min(octs * 8, p.D - d0);
     const int cl = 2 * tid;                      // first of my two channels, within the CTA
     const bool active = cl < nch;
     const int d = d0 + (active ? cl : 0);
-    const int cls = min(cl, p.octets * 8 - 2);   // staged column (padding threads read a real one)
+    const int cls = min(cl, octs * 8 - 2);   // staged column (padding threads read a real one)
     const int64_t L = p.L;
     const int D = p.D;
-    const int nthreads = blockDim.x;
+    const int nthreads = OCT > 0 ? (OCT * 4 + 31) / 32 * 32 : static_cast<int>(blockDim.x);
     const int64_t t_begin = chunk == 0 ? 0 : p.chunk0_len + static_cast<int64_t>(chunk - 1) * p.chunk_len;
     const int64_t t_end = min(L, chunk == 0 ? p.chunk0_len : t_begin + p.chunk_len);
 
     using Lay = PrefillLayout<T>;
-    const int rs = p.octets * 8;                 // elements per staged row (the copy box width)
-    const int stageB = Lay::stage_bytes(TILE, p.octets);
-    const int offZ = Lay::x_bytes(TILE, p.octets);
-    const int offDT = offZ + Lay::zdt_bytes(TILE, p.octets);
-    const int offBC = offDT + Lay::zdt_bytes(TILE, p.octets);
+    const int rs = octs * 8;                     // elements per staged row (the copy box width)
+    const int stageB = Lay::stage_bytes(TILE, octs);
+    const int offZ = Lay::x_bytes(TILE, octs);
+    const int offDT = offZ + Lay::zdt_bytes(TILE, octs);
+    const int offBC = offDT + Lay::zdt_bytes(TILE, octs);
     float* bcf = reinterpret_cast<float*>(smem + STAGES * stageB);   // [TILE][64]
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * stageB + TILE * 64 * 4);
 
@@ -555,7 +559,7 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
                 return false;
             }
             unsigned char* st = smem + slot * stageB;
-            if (t_begin == 0 && tile_of(k) == 0 && cl < p.octets * 8) {
+            if (t_begin == 0 && tile_of(k) == 0 && cl < octs * 8) {
                 // left context of token 0: the carried conv window (zeros if none)
                 T* xs = reinterpret_cast<T*>(st);
 #pragma unroll
