@@ -420,6 +420,11 @@ cudaError_t dispatch_prefill(PrefillParams p, int64_t batch, const FwdPlan& pl, 
     p.chunk_len = pl.chunk_len;
     p.chunk0_len = pl.chunk0_len;
     p.n_chunks = pl.chunks;
+    // the summary pass takes every token of its chunks as valid: they must be
+    // whole tiles that end inside the sequence
+    if (pl.chunks > 1 && (pl.chunk0_len % kTile != 0 || pl.chunk_len % kTile != 0 ||
+                          pl.chunk0_len + static_cast<int64_t>(pl.chunks - 2) * pl.chunk_len > p.L))
+        return cudaErrorInvalidValue;
     const CtaShape full = shape_ctas<T>(p.D, batch, pl.chunks, sm_count);
     // The summary pass is launched normally: it starts after everything
     // before it in the stream, the producers of the inputs included.  The

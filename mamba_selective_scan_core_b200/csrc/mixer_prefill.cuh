@@ -424,7 +424,9 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
         const T* xs = reinterpret_cast<const T*>(st);          // row rho = token - 3 (tile-relative)
         [[maybe_unused]] const T* zs = reinterpret_cast<const T*>(st + offZ);   // full pass only
         const T* ds = reinterpret_cast<const T*>(st + offDT);
-        const int nvalid = static_cast<int>(min(static_cast<int64_t>(SUB), t_end - t0));   // tokens of the chunk here
+        // tokens of the chunk here; the summary pass covers whole tiles inside
+        // the sequence (the launch plan guarantees it), so all of them
+        const int nvalid = SUMMARY ? SUB : static_cast<int>(min(static_cast<int64_t>(SUB), t_end - t0));
 
         // ---- A: per-token work (conv, SiLU, step, Delta*u), both channels packed
         float2 xw[SUB + 3];
