@@ -424,9 +424,6 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
         const T* xs = reinterpret_cast<const T*>(st);          // row rho = token - 3 (tile-relative)
         [[maybe_unused]] const T* zs = reinterpret_cast<const T*>(st + offZ);   // full pass only
         const T* ds = reinterpret_cast<const T*>(st + offDT);
-        // tokens of the chunk here; the summary pass covers whole tiles inside
-        // the sequence (the launch plan guarantees it), so all of them
-        const int nvalid = SUMMARY ? SUB : static_cast<int>(min(static_cast<int64_t>(SUB), t_end - t0));
 
         // ---- A: per-token work (conv, SiLU, step, Delta*u), both channels packed
         float2 xw[SUB + 3];
@@ -441,8 +438,8 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
             float2 u;
             if constexpr (kFast) u = fma2(pre, f2(tanh_fast(pre.x), tanh_fast(pre.y)), pre);   // pre = v/2
             else u = silu2<M>(pre);
-            float2 l = step_pair<M>(P_::load(ds + (r0 + m) * rs + cls), bias2);
-            if (m >= nvalid) l = f2(0.f, 0.f);                  // past the chunk: no step
+            // past the sequence end the staged dt is -inf: l = 0, so s = 0 and the decay is 1
+            const float2 l = step_pair<M>(P_::load(ds + (r0 + m) * rs + cls), bias2);
             const float2 s = mul2(l, u);                         // Delta*u in B' units (B' = B * step_scale)
             if constexpr (!SUMMARY && kStruct) {
                 const float2 la = mul2(l, A02);
@@ -536,13 +533,24 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
                 yacc[m] = __fadd2_rn(acc0, acc1);
             }
 
-            // ---- C: skip, gate, store
-            T* yrow = yg + (seq_row0 + t0) * D + d;
+            // ---- C: skip, gate, store (the tokens of the chunk here; every one but
+            // in the sequence's last sub-tile)
 #pragma unroll
             for (int m = 0; m < SUB; ++m) {
                 const float2 g = silu2<M>(P_::load(zs + (r0 + m) * rs + cls));
-                const float2 yv = mul2(fma2(dsk2, ua[m], yacc[m]), g);
-                if (m < nvalid && active) P_::store(yrow + m * D, yv);
+                yacc[m] = mul2(fma2(dsk2, ua[m], yacc[m]), g);
+            }
+            T* yrow = yg + (seq_row0 + t0) * D + d;
+            if (t0 + SUB <= t_end) {
+                if (active) {
+#pragma unroll
+                    for (int m = 0; m < SUB; ++m) P_::store(yrow + m * D, yacc[m]);
+                }
+            } else {
+                const int nvalid = static_cast<int>(t_end - t0);
+#pragma unroll
+                for (int m = 0; m < SUB; ++m)
+                    if (m < nvalid && active) P_::store(yrow + m * D, yacc[m]);
             }
         }
     };
@@ -561,6 +569,17 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
                 return false;
             }
             unsigned char* st = smem + slot * stageB;
+            const int64_t tile_t0 = t_begin + tile_of(k) * TILE;
+            if (!SUMMARY && tile_t0 + TILE > L && cl < octs * 8) {
+                // the sequence's last tile: dt = -inf past its end makes the step
+                // l = softplus(-inf) = 0 there (no input, decay 1), so the sub-tile
+                // code needs no per-token mask
+                T* dsw = reinterpret_cast<T*>(st + offDT);
+                for (int r = static_cast<int>(L - tile_t0); r < TILE; ++r) {
+                    dsw[r * rs + cl] = A_::from_f32(-INFINITY);
+                    dsw[r * rs + cl + 1] = A_::from_f32(-INFINITY);
+                }
+            }
             if (t_begin == 0 && tile_of(k) == 0 && cl < octs * 8) {
                 // left context of token 0: the carried conv window (zeros if none)
                 T* xs = reinterpret_cast<T*>(st);
@@ -599,7 +618,6 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
                 issue_tile(k + STAGES - 1);
             }
             __syncthreads();
-            const int64_t tile_t0 = t_begin + tile_of(k) * TILE;
 #pragma unroll 1
             for (int j = 0; j < TILE / SUB; ++j) {
                 const int r0 = (SUMMARY ? TILE / SUB - 1 - j : j) * SUB;
