@@ -85,6 +85,18 @@ def test_time_chunked(act, chunks, A_mode):
     check_fwd(inp, act)
 
 
+@pytest.mark.parametrize("A_mode", ["structured", "general"])
+def test_wide_ctas_partial_last_block(A_mode):
+    """d_inner 504 (63 channel octets) in 256-channel CTAs, the second of each
+    pair 248 channels wide; 8 sequences x 12 time chunks need more than one
+    CTA per SM, so the two-stage ring compiled for the 256-channel width runs
+    (summary and full pass), with inactive threads in every second CTA."""
+    os.environ["MAMBA_MIXER_CHUNKS"] = "12"
+    inp = make_mixer_inputs_custom(8, 1100, 504, act="bf16", seed=4242, h0_std=0.5, conv_state_std=1.0,
+                                   conv_b_std=0.2, A_mode=A_mode, dt_std=0.5)
+    check_fwd(inp, "bf16")
+
+
 @pytest.mark.parametrize("act", ["bf16", "f32"])
 def test_optional_inputs_absent(act):
     inp = make_mixer_inputs_custom(2, 70, 32, act=act, seed=77)
