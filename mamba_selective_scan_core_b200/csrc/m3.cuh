@@ -105,6 +105,19 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 
 __device__ __forceinline__ float m3_bf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
+// sin and cos of an angle of any size: Cody and Waite's additive range
+// reduction by 2 pi (a two-part constant: the float nearest 2 pi and the
+// float nearest the rest), then the hardware approximations on [-pi, pi],
+// whose absolute error there is about 2^-21.
+__device__ __forceinline__ void m3_sincos(float x, float* sn, float* cs) {
+    constexpr float kTwoPiHi = 6.28318548202514648f;       // float(2 pi)
+    constexpr float kTwoPiLo = -1.7484555314695172e-07f;   // float(2 pi - kTwoPiHi)
+    constexpr float kInvTwoPi = 0.15915494309189535f;
+    const float k = rintf(x * kInvTwoPi);
+    const float r = fmaf(-k, kTwoPiLo, fmaf(-k, kTwoPiHi, x));
+    __sincosf(r, sn, cs);
+}
+
 // a * s + e for complex numbers held as (re, im) float2, on packed f32x2 operations:
 // (a.re s.re - a.im s.im, a.re s.im + a.im s.re) + e
 __device__ __forceinline__ float2 cmul_add(float2 a, float2 s, float2 e) {
@@ -301,8 +314,8 @@ m3_chunk_kernel(const M3Params p)
             const float2 w = fw[th];
             const float dl = w.x + w.y;
             float sn, cs;
-            sincosf(dl * p.theta[hd * kM3Pairs + k], &sn, &cs);
-            const float mag = expf(dl * p.A[hd]);
+            m3_sincos(dl * p.theta[hd * kM3Pairs + k], &sn, &cs);
+            const float mag = ex2_fast(dl * p.A[hd] * kLog2e);
             // per (token, head) and pair block q: (re 2q, re 2q+1, im 2q, im 2q+1)
             float* fq = reinterpret_cast<float*>(fa) + th * kM3N + (k >> 1) * 4 + (k & 1);
             fq[0] = mag * cs;
@@ -397,7 +410,9 @@ m3_chunk_kernel(const M3Params p)
             }
         }
 
-        for (int tt = 0; FULL && tt < n; ++tt) {
+        // y of this tile's first token for this thread's channel (output r at + r xr)
+        __nv_bfloat16* yp = p.y + (static_cast<int64_t>(b) * p.L + ts) * xt + c;
+        for (int tt = 0; FULL && tt < n; ++tt, yp += xt) {
             float xv[R];
 #pragma unroll
             for (int r = 0; r < R; ++r) xv[r] = __bfloat162float(xs[(tt * R + r) * kM3Threads + tid]);
@@ -426,7 +441,6 @@ m3_chunk_kernel(const M3Params p)
                 sim[q] = ni;
             }
             if (FULL) {
-                const int64_t row = static_cast<int64_t>(b) * p.L + ts + tt;
                 const float* kap = fk + (tt * kM3Heads + hl) * R * R;
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
@@ -442,11 +456,11 @@ m3_chunk_kernel(const M3Params p)
 #pragma unroll
                     for (int rp = 0; rp < R; ++rp) yv = fmaf(kap[r * R + rp], xv[rp], yv);
                     if (p.z) {
-                        // SiLU(z) = z / (1 + 2^(-z log2 e))
-                        const float zv = __bfloat162float(zs[(tt * R + r) * kM3Threads + tid]);
-                        yv *= __fdividef(zv, 1.0f + ex2_fast(-zv * kLog2e));
+                        // SiLU(z) = hz + hz tanh(hz), hz = z / 2
+                        const float hz = 0.5f * __bfloat162float(zs[(tt * R + r) * kM3Threads + tid]);
+                        yv *= fmaf(hz, tanh_fast(hz), hz);
                     }
-                    p.y[row * xt + r * xr + c] = __float2bfloat16_rn(yv);
+                    yp[r * xr] = __float2bfloat16_rn(yv);
                 }
             }
         }
