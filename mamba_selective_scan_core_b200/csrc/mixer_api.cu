@@ -1112,11 +1112,34 @@ bool encode_gemm_2d(CUtensorMap* m, const void* base, int64_t cols, int64_t rows
 // (x_proj's 288 = 2 x 144), else 256-column tiles.
 int gemm_bn(int64_t N) { return N <= 64 ? 64 : N <= 128 ? 128 : (N <= 144 || N == 288) ? 144 : 256; }
 
+// Map of a bf16 output [M][N] (rows ldo elements apart) in 64-column x
+// 32-row boxes with the 128-byte swizzle: the GEMM's staged epilogue.
+bool encode_gemm_out(CUtensorMap* m, void* base, int64_t cols, int64_t rows, int64_t ldo) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldo * 2)};
+    const cuuint32_t box[2] = {64, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int BN, int NSUB, int STAGES, bool OUT_BF16>
-cudaError_t launch_gemm_t(const mm::GemmParams& gp, const void* A, const void* W, int ksplit, cudaStream_t s) {
-    CUtensorMap ta, tw;
+cudaError_t launch_gemm_t(mm::GemmParams gp, const void* A, const void* W, int ksplit, cudaStream_t s) {
+    CUtensorMap ta, tw, to;
     if (!encode_gemm_2d(&ta, A, gp.K, gp.M, mm::kGemmBM) || !encode_gemm_2d(&tw, W, gp.K, gp.N, BN))
         return cudaErrorInvalidValue;
+    // bf16 tiles of whole 64-column boxes go out by bulk tensor stores when the
+    // rows are 16-byte multiples (MAMBA_MIXER_GEMM_ROW_STORES=1 keeps the
+    // per-thread row stores, for comparison)
+    std::memset(&to, 0, sizeof(to));
+    gp.tma_out = 0;
+    if (OUT_BF16 && NSUB == 1 && BN % 64 == 0 && gp.ldo % 8 == 0 && gp.M > 0 &&
+        env_int("MAMBA_MIXER_GEMM_ROW_STORES", 1, 1) == 0) {
+        gp.tma_out = encode_gemm_out(&to, gp.out, gp.N, gp.M, gp.ldo) ? 1 : 0;   // else the row stores
+    }
     auto kern = mm::proj_gemm_kernel<BN, NSUB, STAGES, OUT_BF16>;
     const int smem = mm::GemmLayout<BN, NSUB>::smem_bytes(STAGES);
     static std::atomic<unsigned long long> smem_allowed{0};
@@ -1130,7 +1153,7 @@ cudaError_t launch_gemm_t(const mm::GemmParams& gp, const void* A, const void* W
     }
     const dim3 grid(static_cast<unsigned>((gp.M + mm::kGemmBM - 1) / mm::kGemmBM),
                     static_cast<unsigned>((gp.N + BN * NSUB - 1) / (BN * NSUB)), static_cast<unsigned>(ksplit));
-    kern<<<grid, mm::kGemmThreads, forced_launch_failure() ? (1 << 20) : smem, s>>>(gp, ta, tw);
+    kern<<<grid, mm::kGemmThreads, forced_launch_failure() ? (1 << 20) : smem, s>>>(gp, ta, tw, to);
     return cudaGetLastError();
 }
 

@@ -20,7 +20,12 @@
 //     and releases each ring slot with tcgen05.commit once its MMAs are done;
 //   * after the last MMA commits, all four warps read the accumulator with
 //     tcgen05.ld (warp w owns rows 32w .. 32w+31, one row per thread) and
-//     write it out: fp32 (a split-K partial) or bf16.
+//     write it out: fp32 (a split-K partial) or bf16.  A bf16 output whose
+//     tiles are whole 64-column boxes (and whose rows are 16-byte multiples)
+//     is staged per warp in the ring's shared memory, free once the
+//     accumulator is complete, as 32 x 64 boxes in the 128-byte swizzle, and
+//     written by bulk tensor stores: whole lines, instead of one 16-byte piece
+//     of 32 different rows per store instruction.
 // Every wait on an mbarrier is bounded; a CTA that gives up sets the fault
 // word, waits (bounded) for its own MMAs and copies, frees its tensor memory
 // and exits.
@@ -43,6 +48,7 @@ struct GemmParams {
     int64_t split_stride;   // elements between split-K partials (fp32 output)
     int M, N, K;
     int k_tiles_per_split;  // 64-wide K tiles per CTA (blockIdx.z covers its own range)
+    int tma_out;            // bf16 output written by bulk tensor stores through the output map
     unsigned wait_limit;    // tries per mbarrier wait before giving up
     unsigned long long* status;   // optional: [0] (epoch << 8) | code of a failure, [1] the call's epoch; or NULL
     unsigned long long status_epoch;
@@ -120,6 +126,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 2-D tiled bulk tensor copy shared -> global (a store), in this thread's
+// bulk group; rows and columns outside the tensor are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];\n"
+                 :: "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(src)) : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+// every bulk store this thread committed has completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+
 // 2-D tiled bulk tensor copy global -> shared, completion on `bar`.  No multicast.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
     asm volatile(
@@ -142,7 +158,8 @@ struct GemmLayout {
 // OUT_BF16: write bf16 rows (no split-K); else fp32 split-K partials.
 template <int BN, int NSUB, int STAGES, bool OUT_BF16>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-proj_gemm_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w)
+proj_gemm_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
+                 const __grid_constant__ CUtensorMap tm_out)
 {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 N for M = 128");
     static_assert(GemmLayout<BN>::b_bytes % 1024 == 0, "ring slots stay 1024-byte aligned");
@@ -244,7 +261,47 @@ proj_gemm_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tm_a, c
     const bool acc_ready = mbar_wait_bounded(accb, 0, all_ok ? p.wait_limit : (1u << 20));
     tc_fence_after();
 
-    if (all_ok && acc_ready) {
+    // staged bf16 output: 128 rows x BN columns in the ring (free: every MMA
+    // that read it has completed); warp w's 32 rows of 64-column box bx at
+    // (bx * 4 + w) * 4 KB, 16-byte pieces swizzled by row as the map expects
+    constexpr bool kStaged = OUT_BF16 && NSUB == 1 && BN % 64 == 0 &&
+                             STAGES * Lay::stage_bytes >= kGemmBM * BN * 2;
+    if (kStaged && p.tma_out && all_ok && acc_ready) {
+        const int r = tid & 31;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+#pragma unroll 1
+        for (int cb = 0; cb < BN / 32; ++cb) {
+            float v[32];
+            tmem_ld32(lane_base + cb * 32, v);
+            if (nkt == 0) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+            }
+            unsigned char* slab = gsm + ((cb >> 1) * 4 + warp) * 4096;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int piece = (cb & 1) * 4 + i;       // 16-byte piece of the 128-byte box row
+                uint4 w;
+                w.x = pack_bf16x2(v[8 * i], v[8 * i + 1]);
+                w.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
+                w.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
+                w.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
+                *reinterpret_cast<uint4*>(slab + (r >> 3) * 1024 + (r & 7) * 128 + ((piece ^ (r & 7)) << 4)) = w;
+            }
+        }
+        // the generic-proxy writes above, before the bulk stores read them
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (elect_one_lane()) {
+#pragma unroll 1
+            for (int bx = 0; bx < BN / 64; ++bx)
+                tma_store_2d(&tm_out, gsm + (bx * 4 + warp) * 4096, n0 + bx * 64, m0 + warp * 32);
+            bulk_commit_group();
+            // the stores have read shared memory and written the output before the CTA ends
+            bulk_wait_all();
+        }
+        __syncwarp();
+    } else if (all_ok && acc_ready) {
         const int row = m0 + warp * 32 + (tid & 31);
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
         // sub-tile j's accumulator sits at column j * acc_cols; its BN columns
