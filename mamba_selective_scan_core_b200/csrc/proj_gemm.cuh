@@ -126,6 +126,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 fp32 columns of this thread's row of tensor memory, without waiting:
+// the registers are valid after tmem_wait_ld
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+
 // 2-D tiled bulk tensor copy shared -> global (a store), in this thread's
 // bulk group; rows and columns outside the tensor are not written.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
@@ -133,8 +148,9 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
                  :: "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(src)) : "memory");
 }
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
-// every bulk store this thread committed has completed
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+// every bulk store this thread committed has read its shared-memory source
+// (the writes themselves complete before the grid does)
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
 
 // 2-D tiled bulk tensor copy global -> shared, completion on `bar`.  No multicast.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
@@ -269,23 +285,25 @@ proj_gemm_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tm_a, c
     if (kStaged && p.tma_out && all_ok && acc_ready) {
         const int r = tid & 31;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        // a box's 64 columns per round: two tensor-memory loads, one wait
 #pragma unroll 1
-        for (int cb = 0; cb < BN / 32; ++cb) {
-            float v[32];
-            tmem_ld32(lane_base + cb * 32, v);
-            if (nkt == 0) {
+        for (int bx = 0; bx < BN / 64; ++bx) {
+            uint32_t u[2][32];
+            tmem_ld32_async(lane_base + bx * 64, u[0]);
+            tmem_ld32_async(lane_base + bx * 64 + 32, u[1]);
+            tmem_wait_ld();
+            unsigned char* slab = gsm + (bx * 4 + warp) * 4096;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = 0.0f;
-            }
-            unsigned char* slab = gsm + ((cb >> 1) * 4 + warp) * 4096;
+            for (int piece = 0; piece < 8; ++piece) {     // 16-byte piece of the 128-byte box row
+                const uint32_t* q = u[piece >> 2] + 8 * (piece & 3);
+                float v[8];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int piece = (cb & 1) * 4 + i;       // 16-byte piece of the 128-byte box row
+                for (int i = 0; i < 8; ++i) v[i] = nkt == 0 ? 0.0f : __uint_as_float(q[i]);
                 uint4 w;
-                w.x = pack_bf16x2(v[8 * i], v[8 * i + 1]);
-                w.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
-                w.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
-                w.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
+                w.x = pack_bf16x2(v[0], v[1]);
+                w.y = pack_bf16x2(v[2], v[3]);
+                w.z = pack_bf16x2(v[4], v[5]);
+                w.w = pack_bf16x2(v[6], v[7]);
                 *reinterpret_cast<uint4*>(slab + (r >> 3) * 1024 + (r & 7) * 128 + ((piece ^ (r & 7)) << 4)) = w;
             }
         }
@@ -297,8 +315,8 @@ proj_gemm_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tm_a, c
             for (int bx = 0; bx < BN / 64; ++bx)
                 tma_store_2d(&tm_out, gsm + (bx * 4 + warp) * 4096, n0 + bx * 64, m0 + warp * 32);
             bulk_commit_group();
-            // the stores have read shared memory and written the output before the CTA ends
-            bulk_wait_all();
+            // the stores have read shared memory before the CTA ends
+            bulk_wait_read_all();
         }
         __syncwarp();
     } else if (all_ok && acc_ready) {
