@@ -470,11 +470,29 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
                 const float c0 = cum2[jb * 32];
                 if (c0 - cum2[jb * 32 + 31] <= 60.0f) {     // the same for every thread of the CTA
                     const float ei = ex2_fast(ci - c0);
+                    const float4* cf4 = reinterpret_cast<const float4*>(colf + jb * 32);
+                    if (jb < quarter) {
+                        // a block below the diagonal block: every j < i
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) {
-                        const int j = jb * 32 + q;
-                        m[q] = j <= i ? m[q] * ei * colf[j] : 0.0f;
-                        if (j == i) m[q] += dsk;
+                        for (int q4 = 0; q4 < 8; ++q4) {
+                            const float4 cf = cf4[q4];
+                            m[4 * q4] = m[4 * q4] * ei * cf.x;
+                            m[4 * q4 + 1] = m[4 * q4 + 1] * ei * cf.y;
+                            m[4 * q4 + 2] = m[4 * q4 + 2] * ei * cf.z;
+                            m[4 * q4 + 3] = m[4 * q4 + 3] * ei * cf.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4) {
+                            const float4 cf = cf4[q4];
+                            const float cv[4] = {cf.x, cf.y, cf.z, cf.w};
+#pragma unroll
+                            for (int e4 = 0; e4 < 4; ++e4) {
+                                const int q = 4 * q4 + e4, j = jb * 32 + q;
+                                m[q] = j <= i ? m[q] * ei * cv[e4] : 0.0f;
+                                if (j == i) m[q] += dsk;
+                            }
+                        }
                     }
                 } else {
 #pragma unroll
@@ -551,12 +569,15 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
 #pragma unroll
                 for (int e2 = 0; e2 < 8; ++e2) o[e2] = fmaf(e, yo[q * 8 + e2], yd[q * 8 + e2]);
                 if (p.z) {
-                    // SiLU(z) = z / (1 + 2^(-z log2 e))
+                    // SiLU(z) = hz + hz tanh(hz), hz = z / 2: one MUFU op
                     const uint4 zv = *reinterpret_cast<const uint4*>(zrow + piece * 16);
                     const float zf[8] = {bf16_lo(zv.x), bf16_hi(zv.x), bf16_lo(zv.y), bf16_hi(zv.y),
                                          bf16_lo(zv.z), bf16_hi(zv.z), bf16_lo(zv.w), bf16_hi(zv.w)};
 #pragma unroll
-                    for (int e2 = 0; e2 < 8; ++e2) o[e2] *= __fdividef(zf[e2], 1.0f + ex2_fast(-zf[e2] * kLog2e));
+                    for (int e2 = 0; e2 < 8; ++e2) {
+                        const float hz = 0.5f * zf[e2];
+                        o[e2] *= fmaf(hz, tanh_fast(hz), hz);
+                    }
                 }
                 uint4 w;
                 w.x = pack_bf16x2(o[0], o[1]);
