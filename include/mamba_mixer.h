@@ -216,7 +216,13 @@ mm_status mamba_mixer_fwd_noalloc(const void* xz, const float* conv_w, const flo
  * these may change between this call and the forward that uses the result.
  * MAMBA_MIXER_CHUNKS=K (a positive integer) forces K time chunks per sequence
  * instead of the launch plan's choice, capped at one chunk per 32-token tile;
- * the result is the same up to fp32 rounding.  It is a tuning and test knob. */
+ * the result is the same up to fp32 rounding.  It is a tuning and test knob.
+ * Two more such knobs select slower code paths, for comparison only, and
+ * leave the results the same up to fp32 rounding:
+ * MAMBA_MIXER_GENERIC_WIDTH=1 runs the forward's any-width kernels where the
+ * 256-channel CTA would run one compiled for that width, and
+ * MAMBA_MIXER_GEMM_ROW_STORES=1 makes the projection GEMM write bf16 outputs
+ * with per-thread row stores instead of staged bulk tensor stores. */
 size_t mamba_mixer_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner,
                                   int64_t d_state, int64_t d_conv, mm_dtype act);
 
