@@ -967,6 +967,22 @@ def run_only(args):
         ws = torch.empty(mm.proj_matmul_workspace_size(M, wmat.shape[0], lhs.shape[1]), dtype=torch.uint8,
                          device="cuda")
         step = lambda: mm.proj_matmul(lhs, wmat, out=o, workspace=ws)  # noqa: E731
+    elif args.only == "projected":
+        from workloads import make_norm_weights, make_projection_weights
+
+        cfg = PREFILL
+        B, L, D, R = cfg.batch, cfg.seqlen, cfg.d_inner, 256
+        W_x, W_dt, wd = (t.cuda() for t in make_projection_weights(D, R, seed=cfg.seed))
+        wb, wc = (w.cuda() for w in make_norm_weights(seed=cfg.seed))
+        d = {k: (v.cuda() if v is not None else None) for k, v in make_mixer_inputs(cfg).items()}
+        y = torch.empty((B, L, D), dtype=torch.bfloat16, device="cuda")
+        h = torch.empty((B, D, 16), device="cuda")
+        cs = torch.empty((B, D, 3), dtype=torch.bfloat16, device="cuda")
+        pws = torch.empty(mm.projected_workspace_size(B, L, D, R), dtype=torch.uint8, device="cuda")
+        step = lambda: mm.mixer_fwd_projected(  # noqa: E731
+            d["xz"], d["conv_w"], d["conv_b"], W_x, W_dt, d["dt_bias"], d["A"], d["Dskip"], d["h0"],
+            d["conv_state_in"], dt_norm_w=wd, b_norm_w=wb, c_norm_w=wc, y=y, h_last=h, conv_state_out=cs,
+            workspace=pws)
     elif args.only == "ssd":
         cfg = SSD
         d = {k: (v.cuda() if v is not None else None) for k, v in make_ssd_inputs(cfg).items()}
@@ -1022,7 +1038,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra-prefill", action="store_true",
                     help="skip the 4 x 32768 and 262,144-token prefill legs")
-    ap.add_argument("--only", choices=["forward", "decode", "xproj", "dtproj", "ssd", "m3", "m3mimo"], default=None,
+    ap.add_argument("--only", choices=["forward", "decode", "xproj", "dtproj", "projected", "ssd", "m3", "m3mimo"],
+                    default=None,
                     help="run one kernel's timed loop only (for profiler captures); prints no JSON line")
     ap.add_argument("--decode-layers", type=int, default=None,
                     help="with --only decode: stacked layers (default: the workload's 28)")

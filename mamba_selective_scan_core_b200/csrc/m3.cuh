@@ -42,6 +42,11 @@ constexpr int kM3P = 64;           // channels per head
 constexpr int kM3Threads = 128;    // channels per CTA: two heads
 constexpr int kM3Heads = kM3Threads / kM3P;
 constexpr int kM3Tile = 32;        // chunk lengths are whole multiples of this
+#ifndef MM_M3_TILE_ROWS
+#define MM_M3_TILE_ROWS 32         // (token, input) rows per shared-memory tile: T = rows / R tokens (16 measured slower)
+#endif
+constexpr int kM3TileRows = MM_M3_TILE_ROWS;
+static_assert(kM3Tile % kM3TileRows == 0, "tiles divide the chunks");
 
 struct M3Params {
     const __nv_bfloat16* x;        // [B][L][R][H*P]
@@ -69,8 +74,9 @@ struct M3Params {
 
 // Shared memory of a CTA: two buffers of raw tile inputs, filled by
 // asynchronous copies one tile ahead of the compute, and the tile's
-// per-(token, head) factors and widened B / C rows.  A tile is 32 / R tokens
-// (R = 1, 2, 4), so its x and z rows are 8 KB each whatever R is.
+// per-(token, head) factors and widened B / C rows.  A tile is
+// kM3TileRows / R tokens (R = 1, 2, 4), so its x and z rows are 8 KB each
+// whatever R is.
 struct M3Layout {
     int T, R;
     __host__ __device__ int xs() const { return T * R * kM3Threads * 2; }          // x or z rows, bf16
@@ -90,7 +96,7 @@ struct M3Layout {
     __host__ __device__ int off_k() const { return off_cf() + T * R * kM3Heads * kM3N * 4; }  // float [T][heads][R][R]
     __host__ __device__ int bytes() const { return off_k() + T * kM3Heads * R * R * 4; }
 };
-__host__ __device__ inline M3Layout m3_layout(int R) { return M3Layout{32 / R, R}; }
+__host__ __device__ inline M3Layout m3_layout(int R) { return M3Layout{kM3TileRows / R, R}; }
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" :: "r"(smem_addr(smem)), "l"(gmem) : "memory");
@@ -192,7 +198,7 @@ __global__ void __launch_bounds__(kM3Threads)
 m3_chunk_kernel(const M3Params p)
 {
     extern __shared__ __align__(16) unsigned char m3_sm[];
-    constexpr int T = 32 / R;
+    constexpr int T = kM3TileRows / R;
     if (FULL && p.status && threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
         p.status[1] = p.status_epoch;
     const M3Layout lay = m3_layout(R);

@@ -19,6 +19,9 @@
 namespace mm {
 
 constexpr int kConvTokens = 32;   // tokens one thread walks with its window in registers
+#ifndef MM_CONV_STEP
+#define MM_CONV_STEP 4             // tokens whose x rows one thread requests at once (8 and 16 measured slower)
+#endif
 
 // One thread: 8 consecutive channels of one sequence over kConvTokens tokens.
 __global__ void __launch_bounds__(128)
@@ -58,9 +61,9 @@ conv_silu_kernel(const __nv_bfloat16* __restrict__ xz, const float* __restrict__
     }
     const int64_t t_end = min(L, t0 + kConvTokens);
     __nv_bfloat16* urow = u + static_cast<int64_t>(b) * L * D + d0;
-    // four tokens per step: their rows of x are requested together, so four
-    // loads are in flight per thread instead of one
-    constexpr int kStep = 4;
+    // kStep tokens per step: their rows of x are requested together, so that
+    // many loads are in flight per thread instead of one
+    constexpr int kStep = MM_CONV_STEP;
     for (int64_t tb = t0; tb < t_end; tb += kStep) {
         uint4 xv[kStep];
 #pragma unroll
