@@ -1548,13 +1548,14 @@ mm_status mamba_ssd_fwd(const void* x, const void* z, const void* dt, const floa
 
     const dim3 cgrid(static_cast<unsigned>(pl.chunks), static_cast<unsigned>(heads), static_cast<unsigned>(batch));
     const bool fail = forced_launch_failure();
-    CUtensorMap tc, tb, th, tx, tz;
+    CUtensorMap tc, tb, th, tx, tz, ty;
     if (pl.chunks > 0) {
         const int64_t gn = groups * mm::kSsdN;
         if (!encode_sw128_3d(&tc, Cm, gn, seqlen, batch, mm::kSsdQ) ||
             !encode_sw128_3d(&tb, Bm, gn, seqlen, batch, mm::kSsdQ) ||
             !encode_sw128_3d(&tx, x, C, seqlen, batch, mm::kSsdQ) ||
             !encode_sw128_3d(&tz, z ? z : x, C, seqlen, batch, mm::kSsdQ) ||
+            !encode_sw128_3d(&ty, y, C, seqlen, batch, mm::kSsdQ) ||
             !encode_sw128_3d(&th, p.Hin, mm::kSsdN, 2 * batch * pl.chunks * heads * mm::kSsdP, 1, mm::kSsdP))
             return MM_ERR_CUDA;
         static std::atomic<unsigned long long> allowed_state{0};
@@ -1571,7 +1572,7 @@ mm_status mamba_ssd_fwd(const void* x, const void* z, const void* dt, const floa
         static std::atomic<unsigned long long> allowed_scan{0};
         if (allow_smem(mm::ssd_chunk_scan_kernel, allowed_scan) != cudaSuccess) { cudaGetLastError(); return MM_ERR_CUDA; }
         mm::ssd_chunk_scan_kernel<<<cgrid, mm::kSsdScanThreads,
-                                    fail ? (1 << 20) : mm::SsdScanLayout::smem_bytes, s>>>(p, tc, tb, th, tx, tz);
+                                    fail ? (1 << 20) : mm::SsdScanLayout::smem_bytes, s>>>(p, tc, tb, th, tx, tz, ty);
         if (cudaGetLastError() != cudaSuccess) return MM_ERR_CUDA;
     }
     return MM_OK;

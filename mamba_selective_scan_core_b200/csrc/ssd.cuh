@@ -103,6 +103,19 @@ __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uin
     lo = pack_bf16x2(a - bf16_lo(hi), b - bf16_hi(hi));
 }
 
+// One contiguous bulk copy shared -> global (16-byte aligned, a multiple of
+// 16 bytes), in this thread's bulk group.
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n"
+                 :: "l"(reinterpret_cast<uint64_t>(gdst)), "r"(smem_addr(ssrc)), "r"(bytes) : "memory");
+}
+// 3-D tiled bulk tensor copy shared -> global (a store; rows and columns
+// outside the tensor are not written), in this thread's bulk group.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];\n"
+                 :: "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(src)) : "memory");
+}
+
 __device__ __forceinline__ void ssd_fail(const SsdParams& p) {
     atomicOr(&g_mm_fault, 1u);
     if (p.status) atomicExch(p.status, (p.status_epoch << 8) | 1ull);
@@ -257,8 +270,9 @@ ssd_chunk_state_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm
     if (loaded) ok = mbar_wait_bounded(&bars[1], 0, p.wait_limit);
     tc_fence_after();
     if (__syncthreads_and(ok)) {
-        // thread n owns state row n; the [P][N] block S[b][c][h] is staged in
-        // B's tile (free now) and written out with coalesced 16-byte stores
+        // thread n owns state row n; the [P][N] block S[b][c][h], contiguous
+        // in the workspace, is staged in B's tile (free now) and written out
+        // by one bulk copy
         const int n = tid;
         float* stage = reinterpret_cast<float*>(bt);
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
@@ -269,13 +283,17 @@ ssd_chunk_state_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm
 #pragma unroll
             for (int q = 0; q < 32; ++q) stage[(half * 32 + q) * kSsdN + n] = v[q];
         }
+        // the staging writes, before the bulk copy reads them
+        fence_proxy_async_smem();
         __syncthreads();
-        float4* dst = reinterpret_cast<float4*>(p.S + ((static_cast<int64_t>(b) * p.chunks + c) * p.H + h) *
-                                                          (kSsdP * kSsdN));
-        const float4* src = reinterpret_cast<const float4*>(stage);
-#pragma unroll 4
-        for (int r = 0; r < kSsdP * kSsdN / 4 / kSsdThreads; ++r) dst[r * kSsdThreads + tid] = src[r * kSsdThreads + tid];
-        if (tid == 0) p.dec[(static_cast<int64_t>(b) * p.H + h) * p.chunks + c] = ex2_fast(cum2[kSsdQ - 1]);
+        if (tid == 0) {
+            bulk_store(p.S + ((static_cast<int64_t>(b) * p.chunks + c) * p.H + h) * (kSsdP * kSsdN), stage,
+                       kSsdP * kSsdN * 4);
+            bulk_commit_group();
+            p.dec[(static_cast<int64_t>(b) * p.H + h) * p.chunks + c] = ex2_fast(cum2[kSsdQ - 1]);
+            // the copy has read shared memory before the CTA ends
+            bulk_wait_read_all();
+        }
     } else {
         if (tid == 0) ssd_fail(p);
         // the copies and products finish before shared and tensor memory go away
@@ -310,9 +328,12 @@ ssd_state_pass_kernel(const SsdParams p)
     float4 s = p.h0 ? *reinterpret_cast<const float4*>(p.h0 + b * per_seq + f) : make_float4(0.f, 0.f, 0.f, 0.f);
     const float* dec = p.dec + (static_cast<int64_t>(b) * p.H + h) * p.chunks;
     const float* __restrict__ S = p.S;
-    for (int c0 = 0; c0 < p.chunks; c0 += kAhead) {
-        float4 add[kAhead];
-        float d[kAhead];
+    // Two groups of kAhead chunks' S in registers: the next group's loads are
+    // issued before the current group is passed on, so the stream of loads
+    // does not stop at each group's end.
+    float4 addA[kAhead], addB[kAhead];
+    float dA[kAhead], dB[kAhead];
+    auto load = [&](float4 (&add)[kAhead], float (&d)[kAhead], int c0) {
 #pragma unroll
         for (int j = 0; j < kAhead; ++j) {
             if (c0 + j < p.chunks) {
@@ -320,6 +341,8 @@ ssd_state_pass_kernel(const SsdParams p)
                 d[j] = dec[c0 + j];
             }
         }
+    };
+    auto pass = [&](const float4 (&add)[kAhead], const float (&d)[kAhead], int c0) {
 #pragma unroll
         for (int j = 0; j < kAhead; ++j) {
             if (c0 + j < p.chunks) {
@@ -335,6 +358,13 @@ ssd_state_pass_kernel(const SsdParams p)
                 s.w = fmaf(d[j], s.w, add[j].w);
             }
         }
+    };
+    load(addA, dA, 0);
+    for (int c0 = 0; c0 < p.chunks; c0 += 2 * kAhead) {
+        load(addB, dB, c0 + kAhead);
+        pass(addA, dA, c0);
+        load(addA, dA, c0 + 2 * kAhead);
+        pass(addB, dB, c0 + kAhead);
     }
     *reinterpret_cast<float4*>(p.h_last + b * per_seq + f) = s;
 }
@@ -362,7 +392,8 @@ constexpr uint32_t kSsdColG = 0, kSsdColOff = 128, kSsdColDiag = 192, kSsdCols =
 __global__ void __launch_bounds__(kSsdScanThreads, 2)
 ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_c,
                       const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_h,
-                      const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z)
+                      const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
+                      const __grid_constant__ CUtensorMap tm_y)
 {
     using Lay = SsdScanLayout;
     extern __shared__ __align__(1024) unsigned char ssc_raw[];
@@ -550,9 +581,10 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
     const bool y_ready = __syncthreads_and(y_ok);
 
     // y_i = (M X)_i + exp(cum_i) (C H_in^T)_i, gated by SiLU of the copied z
-    // row; row i is staged over the x tile (free now) and the tile then goes
-    // out with coalesced 16-byte stores.  Rows are 128 bytes, their 16-byte
-    // pieces in the copies' swizzled order (piece q of row r at q ^ (r % 8)).
+    // row; row i is staged over the x tile (free now), rows of 128 bytes with
+    // their 16-byte pieces in the copies' swizzled order (piece q of row r at
+    // q ^ (r % 8)), and the tile goes out by one bulk tensor store, which
+    // writes no row past the sequence.
     if (y_ready) {
         const float e = ex2_fast(cum2[i]);
         const unsigned char* zrow = ct + kSsdQ * kSsdP * 2 + i * 128;
@@ -587,17 +619,13 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
                 *reinterpret_cast<uint4*>(yrow + piece * 16) = w;
             }
         }
+        // the staging writes, before the bulk store reads them
+        fence_proxy_async_smem();
         __syncthreads();
-        // thread k: piece k % 8 of rows k / 8 + 32 m; only rows in the sequence
-        const int q = tid & 7;
-        const int64_t ld = static_cast<int64_t>(p.H) * kSsdP;
-#pragma unroll
-        for (int m = 0; m < kSsdQ * 8 / kSsdScanThreads; ++m) {
-            const int r = (tid >> 3) + (kSsdScanThreads / 8) * m;
-            if (t0 + r < p.L) {
-                const uint4 v = *reinterpret_cast<const uint4*>(ct + r * 128 + ((q ^ (r & 7)) << 4));
-                *reinterpret_cast<uint4*>(p.y + (static_cast<int64_t>(b) * p.L + t0 + r) * ld + h * kSsdP + q * 8) = v;
-            }
+        if (tid == 0) {
+            tma_store_3d(&tm_y, ct, h * kSsdP, static_cast<int>(t0), b);
+            bulk_commit_group();
+            bulk_wait_read_all();     // the store has read shared memory before the CTA ends
         }
     }
 
