@@ -82,7 +82,8 @@ typedef enum mm_status {
     MM_ERR_SCRATCH_LIMIT = 10, /* mamba_mixer_fwd_noalloc: sizes need more than its built-in scratch */
     MM_ERR_TIMEOUT = 11,    /* mamba_check_status / mamba_mixer_fault_status: a kernel gave up a
                                bounded wait (its bulk copies, or a chunk summary never written) */
-    MM_ERR_ARG = 12         /* an argument value out of range (norm_eps not positive and finite) */
+    MM_ERR_ARG = 12,        /* an argument value out of range (norm_eps not positive and finite) */
+    MM_ERR_BOUNDS = 13      /* debug build only: a kernel skipped an access outside its buffer */
 } mm_status;
 
 typedef enum mm_dtype {
@@ -517,7 +518,7 @@ const char* mamba_status_string(mm_status status);
 /* ABI version of this header (incremented on any signature change). */
 int mamba_mixer_abi_version(void);
 
-#define MAMBA_MIXER_ABI_VERSION 6
+#define MAMBA_MIXER_ABI_VERSION 7
 
 #ifdef __cplusplus
 }

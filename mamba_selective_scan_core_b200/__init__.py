@@ -61,6 +61,12 @@ class MixerError(RuntimeError):
 
 
 def library_path() -> str:
+    """The library this process loads: libmamba_mixer.so, or its checked build
+    libmamba_mixer_checked.so when MAMBA_MIXER_CHECKED=1 is set before the
+    first call (index checks in the forward and decode kernels; an access
+    outside its buffer is skipped and reported as MM_ERR_BOUNDS)."""
+    if os.environ.get("MAMBA_MIXER_CHECKED") == "1":
+        return os.path.join(_HERE, "libmamba_mixer_checked.so")
     return os.path.join(_HERE, _LIB_NAME)
 
 
@@ -137,7 +143,9 @@ def abi_version() -> int:
 
 def fault_status(reset: bool = False) -> int:
     """0 if no kernel gave up waiting for its bulk copies on the current
-    device, else MM_ERR_TIMEOUT (11); clears the flag when reset is set."""
+    device, else MM_ERR_TIMEOUT (11) -- or MM_ERR_BOUNDS (13) when a kernel of
+    the checked build skipped an access outside its buffer; clears the word
+    when reset is set."""
     return int(lib().mamba_mixer_fault_status(1 if reset else 0))
 
 
@@ -145,7 +153,8 @@ def check_status(workspace=None, stream=None) -> int:
     """Status of the last forward that ran on `workspace` (a CUDA uint8
     tensor given to mixer_fwd or mixer_fwd_host; None = the fixed scratch of
     mixer_fwd_noalloc): 0 if it completed, MM_ERR_TIMEOUT (11) if one of its
-    kernels gave up a bounded wait.  Waits for `stream` (default: current)."""
+    kernels gave up a bounded wait, MM_ERR_BOUNDS (13) if the checked build
+    skipped an access outside its buffer.  Waits for `stream` (default: current)."""
     import torch
 
     dev = workspace.device if workspace is not None else torch.device("cuda", torch.cuda.current_device())

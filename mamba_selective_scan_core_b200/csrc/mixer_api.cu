@@ -420,6 +420,10 @@ cudaError_t dispatch_prefill(PrefillParams p, int64_t batch, const FwdPlan& pl, 
     p.chunk_len = pl.chunk_len;
     p.chunk0_len = pl.chunk0_len;
     p.n_chunks = pl.chunks;
+    // checked build's test hook: MAMBA_MIXER_TEST_BOUNDS_SHRINK=k takes k
+    // elements off the extent the kernels check y's stores against (the buffer
+    // itself is whole): the last k elements' stores are skipped and reported
+    p.check_shrink = mm::kCheckBounds ? env_int("MAMBA_MIXER_TEST_BOUNDS_SHRINK", 1, 1 << 30) : 0;
     // the summary pass takes every token of its chunks as valid: they must be
     // whole tiles that end inside the sequence
     if (pl.chunks > 1 && (pl.chunk0_len % kTile != 0 || pl.chunk_len % kTile != 0 ||
@@ -712,6 +716,7 @@ const char* mamba_status_string(mm_status status) {
             return "a kernel of the call gave up waiting (for its bulk copies, or for a chunk summary that was "
                    "never written); its outputs are not valid";
         case MM_ERR_ARG: return "an argument value is out of range (norm_eps must be positive and finite)";
+        case MM_ERR_BOUNDS: return "a kernel of the checked build skipped an access outside its buffer";
         case MM_ERR_SCRATCH_LIMIT:
             return "sizes need more scratch than mamba_mixer_fwd_noalloc's built-in 8 MiB; pass a workspace to "
                    "mamba_mixer_fwd instead";
@@ -726,6 +731,7 @@ mm_status mamba_mixer_fault_status(int reset) {
         const unsigned zero = 0;
         if (cudaMemcpyToSymbol(mm::g_mm_fault, &zero, sizeof(zero)) != cudaSuccess) { cudaGetLastError(); return MM_ERR_CUDA; }
     }
+    if (v & mm::kFaultBounds) return MM_ERR_BOUNDS;
     return v ? MM_ERR_TIMEOUT : MM_OK;
 }
 
@@ -744,7 +750,8 @@ mm_status mamba_check_status(const void* workspace, void* stream) {
         cudaGetLastError();
         return MM_ERR_CUDA;
     }
-    return (hdr[0] & 0xff) != 0 && (hdr[0] >> 8) == hdr[1] ? MM_ERR_TIMEOUT : MM_OK;
+    if ((hdr[0] & 0xff) == 0 || (hdr[0] >> 8) != hdr[1]) return MM_OK;
+    return (hdr[0] & 0xff) == mm::kStatusBounds ? MM_ERR_BOUNDS : MM_ERR_TIMEOUT;
 }
 
 size_t mamba_mixer_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state,

@@ -120,6 +120,31 @@ namespace mm {
 // the wait limits only guard against a hung copy turning into a hung GPU).
 __device__ unsigned int g_mm_fault;
 
+// Index checks of the debug build (compiled with MM_CHECK_BOUNDS; the library
+// file libmamba_mixer_checked.so): an access of `count` elements from index
+// `first` of a buffer of `extent` elements is made only when it lies inside
+// the buffer; otherwise it is skipped and recorded -- bit 1 of the device
+// fault word and code kStatusBounds in the call's status -- instead of
+// faulting.  The release build compiles every check to `true`.
+#ifdef MM_CHECK_BOUNDS
+constexpr bool kCheckBounds = true;
+#else
+constexpr bool kCheckBounds = false;
+#endif
+constexpr unsigned long long kStatusBounds = 3;    // call status code of a skipped access
+constexpr unsigned kFaultBounds = 2;               // its bit in the device fault word
+__device__ __forceinline__ bool mm_in_bounds(int64_t first, int64_t count, int64_t extent,
+                                             unsigned long long* status, unsigned long long epoch) {
+    if constexpr (!kCheckBounds) {
+        return true;
+    } else {
+        if (first >= 0 && count >= 0 && first + count <= extent) return true;
+        atomicOr(&g_mm_fault, kFaultBounds);
+        if (status) atomicExch(status, (epoch << 8) | kStatusBounds);
+        return false;
+    }
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" :: "r"(smem_addr(bar)), "r"(count) : "memory");
 }

@@ -92,6 +92,13 @@ state_update_kernel(const T* __restrict__ x, const T* __restrict__ z, const T* _
     const int d0 = cb * 32;
     const int b_begin = bc * kDecodeBatchChunk;
     const int b_end = min(batch, b_begin + kDecodeBatchChunk);
+    // index checks of the checked build (all `true` in the release build); the
+    // decode has no status word, so a skipped access shows in the fault word
+    const int64_t nLD = static_cast<int64_t>(n_layers) * D, nLB = static_cast<int64_t>(n_layers) * batch;
+    const int64_t nLBD = nLB * D;
+    auto inb = [&](int64_t first, int64_t count, int64_t extent) {
+        return mm_in_bounds(first, count, extent, nullptr, 0ull);
+    };
 
     // ---- per-(layer, channel) values shared by every batch row
     const float* Aw = A + (static_cast<int64_t>(layer) * D + d0 + rr) * 16 + q * 4;  // pass 0's slice
@@ -99,7 +106,8 @@ state_update_kernel(const T* __restrict__ x, const T* __restrict__ z, const T* _
     const bool lok = dl < D;
     float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
     float cbias = 0.f, bias2 = 0.f, dsk = 0.f;
-    if (lok) {
+    if (lok && inb((static_cast<int64_t>(layer) * D + dl) * 4, 4, nLD * 4) &&
+        inb(static_cast<int64_t>(layer) * D + dl, 1, nLD)) {
         const int64_t ld = static_cast<int64_t>(layer) * D + dl;
         w = *reinterpret_cast<const float4*>(conv_w + ld * 4);
         cbias = conv_b ? conv_b[ld] : 0.0f;
@@ -116,11 +124,12 @@ state_update_kernel(const T* __restrict__ x, const T* __restrict__ z, const T* _
         float4 hv[4];
 #pragma unroll
         for (int pass = 0; pass < 4; ++pass)
-            hv[pass] = d0 + pass * 8 + rr < D
+            hv[pass] = d0 + pass * 8 + rr < D && inb((rowbase + pass * 8 + rr) * 16 + q * 4, 4, nLBD * 16)
                            ? __ldcs(reinterpret_cast<const float4*>(ssm_state + (rowbase + pass * 8 + rr) * 16 + q * 4))
                            : make_float4(0.f, 0.f, 0.f, 0.f);
-        float4 bq = Vec4Act<T>::load(Bm + lb * 16 + q * 4);
-        float4 cq = Vec4Act<T>::load(Cm + lb * 16 + q * 4);
+        const bool bcok = inb(lb * 16 + q * 4, 4, nLB * 16);
+        float4 bq = bcok ? Vec4Act<T>::load(Bm + lb * 16 + q * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 cq = bcok ? Vec4Act<T>::load(Cm + lb * 16 + q * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
         // optional RMSNorm of the row's B and C over their 16 entries (4 lanes x 4)
         if constexpr (NORM) {
             if (b_norm_w) bq = rms_scale4(bq, b_norm_w + static_cast<int64_t>(layer) * 16 + q * 4, norm_eps);
@@ -129,7 +138,8 @@ state_update_kernel(const T* __restrict__ x, const T* __restrict__ z, const T* _
 
         // ---- row phase: lane i does the per-row work of channel d0 + i
         float l = 0.f, s = 0.f, u = 0.f, gz = 0.f;
-        if (lok) {
+        const bool rok = lok && inb((rowbase + lane) * 3, 3, nLBD * 3) && inb(rowbase + lane, 1, nLBD);
+        if (rok) {
             const int64_t r = rowbase + lane;
             T* cs = conv_state + r * 3;
             const T w0 = cs[0], w1 = cs[1], w2 = cs[2];
@@ -159,7 +169,8 @@ state_update_kernel(const T* __restrict__ x, const T* __restrict__ z, const T* _
             const float lr = __shfl_sync(kFull, l, src);
             const float sr = __shfl_sync(kFull, s, src);
             float part = 0.f;
-            if (d0 + src < D) {
+            if (d0 + src < D && inb((static_cast<int64_t>(layer) * D + d0 + src) * 16 + q * 4, 4, nLD * 16) &&
+                inb((rowbase + src) * 16 + q * 4, 4, nLBD * 16)) {
                 float4 h = hv[pass];
                 const float4 a = __ldg(reinterpret_cast<const float4*>(Aw + pass * 8 * 16));  // L1 after row 0
                 h.x = fmaf(M::decay(lr, a.x), h.x, sr * bq.x);
@@ -175,7 +186,7 @@ state_update_kernel(const T* __restrict__ x, const T* __restrict__ z, const T* _
             const float got = __shfl_sync(kFull, part, ((lane - pass * 8) & 7) * 4);
             if ((lane >> 3) == pass) ysum = got;
         }
-        if (lok) y[rowbase + lane] = Act<T>::from_f32(fmaf(dsk, u, ysum) * gz);
+        if (rok) y[rowbase + lane] = Act<T>::from_f32(fmaf(dsk, u, ysum) * gz);
     }
 }
 

@@ -128,6 +128,7 @@ struct PrefillParams {
     float norm_eps;
     int batch;
     unsigned wait_limit;  // tries per wait on a bulk copy before giving up (fault)
+    int64_t check_shrink; // checked build's test hook: elements taken off y's extent (0 otherwise)
 };
 
 constexpr unsigned long long kStatusCopyTimeout = 1;  // a wait on the CTA's own bulk copies gave up
@@ -249,6 +250,14 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
     const int64_t seq_row0 = static_cast<int64_t>(seq) * L;
     const int64_t chan = static_cast<int64_t>(seq) * D + d;           // (sequence, first channel) row
 
+    // Index checks of the checked build (every one is `true` in the release
+    // build): the extents, in elements, of the buffers threads address directly.
+    const int64_t nBD = static_cast<int64_t>(p.batch) * D;
+    const int64_t nSum = static_cast<int64_t>(p.n_chunks - 1) * nBD;  // chunk summaries per state
+    auto inb = [&](int64_t first, int64_t count, int64_t extent) {
+        return mm_in_bounds(first, count, extent, p.ws_hdr, p.status_epoch);
+    };
+
     // ---------------------------------------------------------- tile loader
     const int64_t ntiles = t_end > t_begin ? (t_end - t_begin + TILE - 1) / TILE : 0;
     constexpr int kBC = SUMMARY ? 1 : 2;              // the summary pass needs B but not C (nor z)
@@ -315,7 +324,7 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
 #pragma unroll
     for (int k = 0; k < 4; ++k) w2[k] = f2(0.f, 0.f);
     float2 cb2 = f2(0.f, 0.f), bias2 = f2(0.f, 0.f), dsk2 = f2(0.f, 0.f), A02 = f2(0.f, 0.f);
-    if (active) {
+    if (active && inb(static_cast<int64_t>(d) * 4, 8, static_cast<int64_t>(D) * 4) && inb(d, 2, D)) {
         const float4 wa = *reinterpret_cast<const float4*>(p.conv_w + static_cast<int64_t>(d) * 4);
         const float4 wb = *reinterpret_cast<const float4*>(p.conv_w + static_cast<int64_t>(d + 1) * 4);
         w2[0] = f2(wa.x, wb.x); w2[1] = f2(wa.y, wb.y); w2[2] = f2(wa.z, wb.z); w2[3] = f2(wa.w, wb.w);
@@ -336,10 +345,11 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
     float2 a2[16];
     {
         float av[32];
+        const bool aok = active && inb(static_cast<int64_t>(d) * 16, 32, static_cast<int64_t>(D) * 16);
 #pragma unroll
         for (int q = 0; q < 8; ++q)
             *reinterpret_cast<float4*>(av + 4 * q) =
-                active ? __ldg(reinterpret_cast<const float4*>(p.A + static_cast<int64_t>(d) * 16) + q)
+                aok ? __ldg(reinterpret_cast<const float4*>(p.A + static_cast<int64_t>(d) * 16) + q)
                        : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int n = 0; n < 16; ++n) a2[n] = f2(av[n], av[16 + n]);
@@ -352,7 +362,7 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
 #pragma unroll
         for (int n = 0; n < 16; ++n) h[n] = f2(0.f, 0.f);
     } else {
-        if (p.h0 && active) {
+        if (p.h0 && active && inb(chan * 16, 32, nBD * 16)) {
             float hv[32];   // my two channels' rows of h0: 128 contiguous bytes
 #pragma unroll
             for (int q = 0; q < 8; ++q)
@@ -376,9 +386,12 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
                 const int span = 8 * p.sum_octets;
                 const int64_t octs = D / 8;
                 for (int c = 0; c < chunk; ++c)
-                    for (int sb = d0 / span; sb <= (d0 + nch - 1) / span; ++sb)
-                        ok &= p.ws_tags[(static_cast<int64_t>(c) * p.batch + seq) * octs +
-                                        static_cast<int64_t>(sb) * p.sum_octets] == p.call_id;
+                    for (int sb = d0 / span; sb <= (d0 + nch - 1) / span; ++sb) {
+                        const int64_t ti = (static_cast<int64_t>(c) * p.batch + seq) * octs +
+                                           static_cast<int64_t>(sb) * p.sum_octets;
+                        ok &= inb(ti, 1, static_cast<int64_t>(p.n_chunks - 1) * p.batch * octs) &&
+                              p.ws_tags[ti] == p.call_id;
+                    }
             }
             if (__syncthreads_or(!ok)) {
                 fail(kStatusNoSummary);
@@ -390,6 +403,9 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
             const int64_t stride = static_cast<int64_t>(p.batch) * D;
 #pragma unroll 1
             for (int c = 0; c < chunk; ++c) {
+                if (!inb(c * stride + chan, 2, nSum) ||
+                    !inb((c * stride + static_cast<int64_t>(seq) * D) * 16 + d, 15 * static_cast<int64_t>(D) + 2, nSum * 16))
+                    continue;
                 const float2 ls = *reinterpret_cast<const float2*>(p.ws_lsum + c * stride + chan);
                 const float* e = p.ws_state + (c * stride + static_cast<int64_t>(seq) * D) * 16 + d;
                 float2 ev[16];
@@ -541,22 +557,26 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
                 yacc[m] = mul2(fma2(dsk2, ua[m], yacc[m]), g);
             }
             T* yrow = yg + (seq_row0 + t0) * D + d;
+            const int64_t yi = (seq_row0 + t0) * D + d;     // y's index of yrow
             if (t0 + SUB <= t_end) {
                 if (active) {
 #pragma unroll
-                    for (int m = 0; m < SUB; ++m) P_::store(yrow + m * D, yacc[m]);
+                    for (int m = 0; m < SUB; ++m)
+                        if (inb(yi + static_cast<int64_t>(m) * D, 2, nBD * L - p.check_shrink))
+                            P_::store(yrow + m * D, yacc[m]);
                 }
             } else {
                 const int nvalid = static_cast<int>(t_end - t0);
 #pragma unroll
                 for (int m = 0; m < SUB; ++m)
-                    if (m < nvalid && active) P_::store(yrow + m * D, yacc[m]);
+                    if (m < nvalid && active && inb(yi + static_cast<int64_t>(m) * D, 2, nBD * L - p.check_shrink))
+                        P_::store(yrow + m * D, yacc[m]);
             }
         }
     };
 
     // ---------------------------------------------------------- main loop
-    const T* csi = (p.cs_in && active) ? static_cast<const T*>(p.cs_in) + chan * 3 : nullptr;
+    const T* csi = (p.cs_in && active && inb(chan * 3, 6, nBD * 3)) ? static_cast<const T*>(p.cs_in) + chan * 3 : nullptr;
     // returns false when a copy did not land (fault set; the caller exits)
     auto main_loop = [&](auto structured_tag, const float2* a2) -> bool {
 #pragma unroll 1
@@ -636,8 +656,9 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
 
     // ---------------------------------------------------------- carried state out
     if constexpr (SUMMARY) {
-        if (active) {
-            const int64_t stride = static_cast<int64_t>(p.batch) * D;
+        const int64_t stride = static_cast<int64_t>(p.batch) * D;
+        if (active && inb(chunk * stride + chan, 2, nSum) &&
+            inb((chunk * stride + static_cast<int64_t>(seq) * D) * 16 + d, 15 * static_cast<int64_t>(D) + 2, nSum * 16)) {
             float* e = p.ws_state + (chunk * stride + static_cast<int64_t>(seq) * D) * 16 + d;
 #pragma unroll
             for (int n = 0; n < 16; ++n) *reinterpret_cast<float2*>(e + static_cast<int64_t>(n) * D) = h[n];
@@ -646,9 +667,9 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
         // this CTA's summaries are stored (the full pass reads them only after
         // this grid has completed, so no fence is needed)
         __syncthreads();
-        if (tid == 0)
-            p.ws_tags[(static_cast<int64_t>(chunk) * p.batch + seq) * (D / 8) + d0 / 8] = p.call_id;
-    } else if (active && chunk == p.n_chunks - 1) {
+        const int64_t ti = (static_cast<int64_t>(chunk) * p.batch + seq) * (D / 8) + d0 / 8;
+        if (tid == 0 && inb(ti, 1, static_cast<int64_t>(p.n_chunks - 1) * p.batch * (D / 8))) p.ws_tags[ti] = p.call_id;
+    } else if (active && chunk == p.n_chunks - 1 && inb(chan * 16, 32, nBD * 16) && inb(chan * 3, 6, nBD * 3)) {
         // my two channels' rows of h_last: 128 contiguous bytes, in 16-byte stores
         float4* hl = reinterpret_cast<float4*>(p.h_last + chan * 16);
 #pragma unroll
@@ -664,7 +685,8 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
             for (int q = 0; q < 3; ++q) {
                 const int64_t tpos = L - 3 + q;
                 T v;
-                if (tpos >= 0) v = xz[(seq_row0 + tpos) * 2 * D + d + c];
+                if (tpos >= 0) v = inb((seq_row0 + tpos) * 2 * D + d + c, 1, nBD * L * 2) ? xz[(seq_row0 + tpos) * 2 * D + d + c]
+                                                                                         : A_::from_f32(0.f);
                 else v = csi ? csi[3 * c + tpos + 3] : A_::from_f32(0.f);
                 cso[3 * c + q] = v;
             }

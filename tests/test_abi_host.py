@@ -50,6 +50,16 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(lib, name), f"{name} missing from {mm.library_path()}"
 
 
+def test_checked_build_exports_the_same_symbols():
+    """The checked build (index checks in the forward and decode kernels)
+    is the same C ABI: every declared function, C linkage."""
+    path = mmbuild.build_checked()
+    out = os.popen(f"nm -D --defined-only {path}").read()
+    names = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_functions():
+        assert name in names, f"{name} missing from {path}"
+
+
 def test_exported_symbols_are_c_linkage():
     out = os.popen(f"nm -D --defined-only {mm.library_path()}").read()
     names = {line.split()[-1] for line in out.splitlines() if line.strip()}
@@ -59,8 +69,8 @@ def test_exported_symbols_are_c_linkage():
 
 def test_version_and_strings():
     mmbuild.build()
-    assert mm.abi_version() == 6
-    for code in range(13):
+    assert mm.abi_version() == 7
+    for code in range(14):
         s = mm.status_string(code)
         assert s and s != "unknown status"
     assert mm.status_string(99) == "unknown status"
