@@ -614,22 +614,32 @@ mixer_fwd_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_x
                 const T* bs = reinterpret_cast<const T*>(st + offBC);
                 constexpr int cstride = Lay::bc_bytes(TILE) / static_cast<int>(sizeof(T));   // elements from B to C
                 const bool normed = p.b_norm_w != nullptr || p.c_norm_w != nullptr;
-                // The loop's trip count and thread count are multiples of 32, so each
-                // half-warp holds one 16-entry row (one token's B or C) in every pass:
-                // the RMSNorm's sum of squares is four shuffles within it.
-                for (int i = tid; i < TILE * 16 * kBC; i += nthreads) {
-                    const int r = i / (16 * kBC);
-                    const int e = i - r * 16 * kBC;               // 0..15 B, 16..31 C
-                    float v = A_::to_f32(bs[(e >> 4) * cstride + r * 16 + (e & 15)]);
+                // A thread converts a pair of adjacent entries per pass (both of B or
+                // both of C).  The loop's trip count and thread count are multiples of
+                // 32, so each group of 8 lanes holds one 16-entry row (one token's B or
+                // C) in every pass: the RMSNorm's sum of squares is three shuffles
+                // within it.
+                for (int i = tid; i < TILE * 8 * kBC; i += nthreads) {
+                    const int r = i / (8 * kBC);
+                    const int e = 2 * (i - r * 8 * kBC);          // 0..15 B, 16..31 C; even
+                    const float2 v2 = P_::load(bs + (e >> 4) * cstride + r * 16 + (e & 15));
+                    float va = v2.x, vb = v2.y;
                     if (normed) {
-                        float ss = v * v;
+                        float ss = fmaf(va, va, vb * vb);
 #pragma unroll
-                        for (int o = 1; o < 16; o <<= 1) ss += __shfl_xor_sync(kFull, ss, o);
+                        for (int o = 1; o < 8; o <<= 1) ss += __shfl_xor_sync(kFull, ss, o);
                         const float* w = (e >> 4) ? p.c_norm_w : p.b_norm_w;
-                        if (w) v *= rsqrtf(fmaf(ss, 1.0f / 16.0f, p.norm_eps)) * __ldg(w + (e & 15));
+                        if (w) {
+                            const float sc = rsqrtf(fmaf(ss, 1.0f / 16.0f, p.norm_eps));
+                            va *= sc * __ldg(w + (e & 15));
+                            vb *= sc * __ldg(w + (e & 15) + 1);
+                        }
                     }
-                    if (e < 16) v *= M::step_scale;
-                    *reinterpret_cast<float2*>(bcf + r * 64 + 2 * e) = f2(v, v);
+                    if (e < 16) {
+                        va *= M::step_scale;
+                        vb *= M::step_scale;
+                    }
+                    *reinterpret_cast<float4*>(bcf + r * 64 + 2 * e) = make_float4(va, va, vb, vb);
                 }
             }
             if (tid == 0) {
