@@ -47,6 +47,7 @@ constexpr int kM3Tile = 32;        // chunk lengths are whole multiples of this
 #endif
 constexpr int kM3TileRows = MM_M3_TILE_ROWS;
 
+
 static_assert(kM3Tile % kM3TileRows == 0, "tiles divide the chunks");
 
 struct M3Params {
@@ -202,7 +203,7 @@ m3_chunk_kernel(const M3Params p)
     constexpr int T = kM3TileRows / R;
     // tokens of the per-token loops unrolled together, so that one token's
     // shared-memory loads overlap another's arithmetic (B200: 244 -> 228 us
-    // at R = 1 with 4; at R = 4, 2 is best, 4 slower)
+    // at R = 1 with 4, 8 no better; at R = 4, 2 is best, 4 slower)
     constexpr int kUnroll = R == 1 ? 4 : 2;
     if (FULL && p.status && threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
         p.status[1] = p.status_epoch;
