@@ -198,6 +198,11 @@ __device__ __forceinline__ float2 step_pair(float2 dt, float2 bias) {
 
 template <typename M>
 __device__ __forceinline__ float2 decay2(float2 l, float2 a) {
+    if constexpr (M::step_scale != 1.0f) {
+        // MathFast::decay on both channels with the product packed: 2^(l a)
+        const float2 la = mul2(l, a);
+        return f2(ex2_fast(la.x), ex2_fast(la.y));
+    }
     return f2(M::decay(l.x, a.x), M::decay(l.y, a.y));
 }
 
