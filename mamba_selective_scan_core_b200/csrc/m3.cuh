@@ -25,8 +25,9 @@
 // asynchronous 16-byte copies one tile ahead of the compute (two buffers).
 // Per-(token, head) factors -- a_t (one exp and one sincos per pair) and the
 // two tap weights -- are computed once per tile into shared memory, with the
-// tile's B and C rows widened to fp32; y goes out per thread, 2 bytes each, a
-// warp's 32 channels contiguous.
+// tile's B and C rows widened to fp32.  A thread holds two adjacent channels
+// of one head (a warp per head), so every factor it reads serves both; y goes
+// out as 4 bytes per thread, a warp's 64 channels contiguous.
 #pragma once
 
 #include <cstdint>
@@ -41,9 +42,11 @@ constexpr int kM3N = 2 * kM3Pairs;
 constexpr int kM3P = 64;           // channels per head
 constexpr int kM3Threads = 128;    // channels per CTA: two heads
 constexpr int kM3Heads = kM3Threads / kM3P;
+constexpr int kM3Cpt = 2;          // channels per thread (adjacent, of one head)
+constexpr int kM3Block = kM3Threads / kM3Cpt;   // threads per CTA: a warp per head
 constexpr int kM3Tile = 32;        // chunk lengths are whole multiples of this
 #ifndef MM_M3_TILE_ROWS
-#define MM_M3_TILE_ROWS 32         // (token, input) rows per shared-memory tile: T = rows / R tokens (16 measured slower)
+#define MM_M3_TILE_ROWS 16         // (token, input) rows per shared-memory tile: T = rows / R tokens
 #endif
 constexpr int kM3TileRows = MM_M3_TILE_ROWS;
 
@@ -77,7 +80,7 @@ struct M3Params {
 // Shared memory of a CTA: two buffers of raw tile inputs, filled by
 // asynchronous copies one tile ahead of the compute, and the tile's
 // per-(token, head) factors and widened B / C rows.  A tile is
-// kM3TileRows / R tokens (R = 1, 2, 4), so its x and z rows are 8 KB each
+// kM3TileRows / R tokens (R = 1, 2, 4), so its x and z rows are 4 KB each
 // whatever R is.
 struct M3Layout {
     int T, R;
@@ -167,7 +170,7 @@ __device__ __forceinline__ void m3_issue_tile(const M3Params& p, const M3Layout&
     const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kM3Threads;
     const int h0_ = blockIdx.x * kM3Heads;
     // x (and z): 16 pieces of 16 bytes per (token, input) row of the CTA's 128 channels
-    for (int e = tid; e < n * R * 16; e += kM3Threads) {
+    for (int e = tid; e < n * R * 16; e += kM3Block) {
         const int q = e & 15, tr = e >> 4;                 // tr = token * R + r
         const int64_t g = (static_cast<int64_t>(b) * p.L + ts) * R * C + static_cast<int64_t>(tr) * C + c0 + 8 * q;
         cp_async16(sm + lay.off_x(buf) + tr * (kM3Threads * 2) + 16 * q, p.x + g);
@@ -175,7 +178,7 @@ __device__ __forceinline__ void m3_issue_tile(const M3Params& p, const M3Layout&
     }
     // B (and C) rows of each head's group: two 16-byte pieces per (token, input, head)
     const int64_t br = static_cast<int64_t>(p.G) * kM3N;
-    for (int e = tid; e < n * R * kM3Heads * 2; e += kM3Threads) {
+    for (int e = tid; e < n * R * kM3Heads * 2; e += kM3Block) {
         const int q = e & 1, hh = (e >> 1) % kM3Heads, tr = e / (2 * kM3Heads);
         const int gh = (h0_ + hh) * p.G / p.H;
         const int64_t g = ((static_cast<int64_t>(b) * p.L + ts) * R + tr) * br + gh * kM3N + 8 * q;
@@ -186,7 +189,7 @@ __device__ __forceinline__ void m3_issue_tile(const M3Params& p, const M3Layout&
     // dt (and trap) of the CTA's two heads: 4 bytes per token, and of the
     // token after the tile when there is one (its trapezoid tap weight)
     const int nd = ts + n < p.L ? n + 1 : n;
-    for (int e = tid; e < nd; e += kM3Threads) {
+    for (int e = tid; e < nd; e += kM3Block) {
         const int64_t g = (static_cast<int64_t>(b) * p.L + ts + e) * p.H + h0_;
         cp_async4(sm + lay.off_dt(buf) + 4 * e, p.dt + g);
         if (p.trap) cp_async4(sm + lay.off_tr(buf) + 4 * e, p.trap + g);
@@ -196,23 +199,23 @@ __device__ __forceinline__ void m3_issue_tile(const M3Params& p, const M3Layout&
 // R: inputs per state (1, 2 or 4), a compile-time constant so that the
 // per-token loops over inputs and outputs unroll.
 template <bool FULL, int R>
-__global__ void __launch_bounds__(kM3Threads)
+__global__ void __launch_bounds__(kM3Block)
 m3_chunk_kernel(const M3Params p)
 {
     extern __shared__ __align__(16) unsigned char m3_sm[];
     constexpr int T = kM3TileRows / R;
     // tokens of the per-token loops unrolled together, so that one token's
-    // shared-memory loads overlap another's arithmetic (B200: 244 -> 228 us
-    // at R = 1 with 4, 8 no better; at R = 4, 2 is best, 4 slower)
+    // shared-memory loads overlap another's arithmetic
     constexpr int kUnroll = R == 1 ? 4 : 2;
     if (FULL && p.status && threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
         p.status[1] = p.status_epoch;
     const M3Layout lay = m3_layout(R);
     const int tid = threadIdx.x;
+    const int cl = kM3Cpt * tid;                                              // first channel, CTA-local
     const int64_t C = static_cast<int64_t>(p.H) * kM3P;
-    const int64_t c = static_cast<int64_t>(blockIdx.x) * kM3Threads + tid;   // channel
+    const int64_t c = static_cast<int64_t>(blockIdx.x) * kM3Threads + cl;    // first channel
     const int h0_ = blockIdx.x * kM3Heads;                                    // first head of the CTA
-    const int hl = tid / kM3P;                                                // this thread's head, local
+    const int hl = cl / kM3P;                                                 // this thread's head, local
     const int h = h0_ + hl;
     const int chunk = blockIdx.y;
     const int b = blockIdx.z;
@@ -234,22 +237,29 @@ m3_chunk_kernel(const M3Params p)
     // term is, per output r, sum_r' x_t[r'] (C_t[r] . B_t[r']) times that
     // weight, a per-(token, head) matrix kappa that also holds the skip D.
     // Past the last token the weight is 0, so q is s there.
-    // The state of pairs 2q and 2q+1 as two packed registers: sre[q] their
-    // real parts, sim[q] their imaginary parts, so that a complex
-    // multiply-add of both pairs is four packed f32x2 FMAs with no operand
-    // swaps.  Memory keeps (re, im) per pair.
-    float2 sre[kM3Pairs / 2], sim[kM3Pairs / 2];
+    // A thread holds two adjacent channels of one head, so each per-token
+    // factor it reads from shared memory serves both.  The state of pairs 2q
+    // and 2q+1 of channel j as two packed registers: sre[j][q] their real
+    // parts, sim[j][q] their imaginary parts, so that a complex multiply-add
+    // of both pairs is four packed f32x2 FMAs with no operand swaps.  Memory
+    // keeps (re, im) per pair.
+    float2 sre[kM3Cpt][kM3Pairs / 2], sim[kM3Cpt][kM3Pairs / 2];
 #pragma unroll
-    for (int q = 0; q < kM3Pairs / 2; ++q) sre[q] = sim[q] = make_float2(0.0f, 0.0f);
+    for (int j = 0; j < kM3Cpt; ++j)
+#pragma unroll
+        for (int q = 0; q < kM3Pairs / 2; ++q) sre[j][q] = sim[j][q] = make_float2(0.0f, 0.0f);
     if (FULL) {
         // q_{-1} = h0 + (1 - lambda_0) Delta_0 u_{-1}
         if (p.h0) {
-            const float4* hp = reinterpret_cast<const float4*>(p.h0 + (static_cast<int64_t>(b) * C + c) * kM3N);
 #pragma unroll
-            for (int q = 0; q < kM3N / 4; ++q) {
-                const float4 v = hp[q];
-                sre[q] = make_float2(v.x, v.z);
-                sim[q] = make_float2(v.y, v.w);
+            for (int j = 0; j < kM3Cpt; ++j) {
+                const float4* hp = reinterpret_cast<const float4*>(p.h0 + (static_cast<int64_t>(b) * C + c + j) * kM3N);
+#pragma unroll
+                for (int q = 0; q < kM3N / 4; ++q) {
+                    const float4 v = hp[q];
+                    sre[j][q] = make_float2(v.x, v.z);
+                    sim[j][q] = make_float2(v.y, v.w);
+                }
             }
         }
         if (p.x_prev && p.B_prev && p.L > 0) {
@@ -257,14 +267,17 @@ m3_chunk_kernel(const M3Params p)
             const float v = __bfloat162float(p.dt[row * p.H + h]) + (p.dt_bias ? p.dt_bias[h] : 0.0f);
             const float dl = fmaxf(v, 0.0f) + log1pf(expf(-fabsf(v)));
             const float lam = p.trap ? __bfloat162float(p.trap[row * p.H + h]) : 0.5f;
-            float2 up[kM3Pairs];
-            m3_input_global<R>(p, p.x_prev + static_cast<int64_t>(b) * R * C + c,
-                            p.B_prev + static_cast<int64_t>(b) * R * br + g * kM3N, xr, br, up);
             const float2 w0 = make_float2((1.0f - lam) * dl, (1.0f - lam) * dl);
 #pragma unroll
-            for (int q = 0; q < kM3Pairs / 2; ++q) {
-                sre[q] = fma2(w0, make_float2(up[2 * q].x, up[2 * q + 1].x), sre[q]);
-                sim[q] = fma2(w0, make_float2(up[2 * q].y, up[2 * q + 1].y), sim[q]);
+            for (int j = 0; j < kM3Cpt; ++j) {
+                float2 up[kM3Pairs];
+                m3_input_global<R>(p, p.x_prev + static_cast<int64_t>(b) * R * C + c + j,
+                                p.B_prev + static_cast<int64_t>(b) * R * br + g * kM3N, xr, br, up);
+#pragma unroll
+                for (int q = 0; q < kM3Pairs / 2; ++q) {
+                    sre[j][q] = fma2(w0, make_float2(up[2 * q].x, up[2 * q + 1].x), sre[j][q]);
+                    sim[j][q] = fma2(w0, make_float2(up[2 * q].y, up[2 * q + 1].y), sim[j][q]);
+                }
             }
         }
         // carried through the earlier chunks: q = prod_c' q + e_c'
@@ -275,12 +288,16 @@ m3_chunk_kernel(const M3Params p)
                 p.ws_state + ((static_cast<int64_t>(cc) * gridDim.z + b) * C + c) * kM3N);
 #pragma unroll
             for (int q = 0; q < kM3N / 4; ++q) {
-                const float4 a = pp[q], e = ep[q];     // (re, im) of pairs 2q, 2q+1
+                const float4 a = pp[q];                // (re, im) of pairs 2q, 2q+1
                 const float2 ar = make_float2(a.x, a.z), ai = make_float2(a.y, a.w);
-                const float2 nr = fma2(ar, sre[q], fma2(make_float2(-ai.x, -ai.y), sim[q], make_float2(e.x, e.z)));
-                const float2 ni = fma2(ar, sim[q], fma2(ai, sre[q], make_float2(e.y, e.w)));
-                sre[q] = nr;
-                sim[q] = ni;
+#pragma unroll
+                for (int j = 0; j < kM3Cpt; ++j) {
+                    const float4 e = ep[j * (kM3N / 4) + q];
+                    const float2 nr = fma2(ar, sre[j][q], fma2(make_float2(-ai.x, -ai.y), sim[j][q], make_float2(e.x, e.z)));
+                    const float2 ni = fma2(ar, sim[j][q], fma2(ai, sre[j][q], make_float2(e.y, e.w)));
+                    sre[j][q] = nr;
+                    sim[j][q] = ni;
+                }
             }
         }
     }
@@ -308,7 +325,7 @@ m3_chunk_kernel(const M3Params p)
         const __nv_bfloat16* trs = reinterpret_cast<const __nv_bfloat16*>(m3_sm + lay.off_tr(buf));
         // tap weights ((1 - lambda) Delta, lambda Delta) per (token, head), the
         // token after the tile included (zero past the sequence)
-        for (int e = tid; e < (T + 1) * kM3Heads; e += kM3Threads) {
+        for (int e = tid; e < (T + 1) * kM3Heads; e += kM3Block) {
             const int tt = e / kM3Heads, hh = e % kM3Heads, hd = h0_ + hh;
             float2 w = make_float2(0.0f, 0.0f);
             if (tt < nd) {
@@ -321,7 +338,7 @@ m3_chunk_kernel(const M3Params p)
         }
         __syncthreads();
         // a_t per pair
-        for (int e = tid; e < n * kM3Heads * kM3Pairs; e += kM3Threads) {
+        for (int e = tid; e < n * kM3Heads * kM3Pairs; e += kM3Block) {
             const int k = e % kM3Pairs, th = e / kM3Pairs, hd = h0_ + th % kM3Heads;
             const float2 w = fw[th];
             const float dl = w.x + w.y;
@@ -336,7 +353,7 @@ m3_chunk_kernel(const M3Params p)
         // omega_t B_t and C_t, widened to fp32
         const uint2* braw = reinterpret_cast<const uint2*>(m3_sm + lay.off_b(buf));
         const uint2* craw = reinterpret_cast<const uint2*>(m3_sm + lay.off_c(buf));
-        for (int e = tid; e < n * R * kM3Heads * (kM3N / 4); e += kM3Threads) {
+        for (int e = tid; e < n * R * kM3Heads * (kM3N / 4); e += kM3Block) {
             const int hh = (e / (kM3N / 4)) % kM3Heads, tt = e / (kM3N / 4 * kM3Heads * R);
             const float om = fw[tt * kM3Heads + hh].y + fw[(tt + 1) * kM3Heads + hh].x;
             const float4 bv = m3_widen4(braw[e]);      // (re, im, re, im) of pairs 2q, 2q+1
@@ -348,7 +365,7 @@ m3_chunk_kernel(const M3Params p)
         }
         // kappa[t][head][r][r'] = D [r == r'] - (1 - lambda_{t+1}) Delta_{t+1} (C_t[r] . B_t[r'])
         if (FULL) {
-            for (int e = tid; e < n * kM3Heads * R * R; e += kM3Threads) {
+            for (int e = tid; e < n * kM3Heads * R * R; e += kM3Block) {
                 const int rp = e % R, r = (e / R) % R, hh = (e / (R * R)) % kM3Heads, tt = e / (R * R * kM3Heads);
                 const uint2* bq = braw + ((tt * R + rp) * kM3Heads + hh) * (kM3N / 4);
                 const uint2* cq = craw + ((tt * R + r) * kM3Heads + hh) * (kM3N / 4);
@@ -389,7 +406,7 @@ m3_chunk_kernel(const M3Params p)
                 prod = cmul_add(w, prod, make_float2(0.0f, 0.0f));
             }
             __syncthreads();
-            for (int e = tid; e < n * R * kM3Heads * (kM3N / 4); e += kM3Threads) {
+            for (int e = tid; e < n * R * kM3Heads * (kM3N / 4); e += kM3Block) {
                 const int q = e % (kM3N / 4), hh = (e / (kM3N / 4)) % kM3Heads, tt = e / (kM3N / 4 * kM3Heads * R);
                 const float4 w = reinterpret_cast<const float4*>(fW)[(tt * kM3Heads + hh) * (kM3N / 4) + q];
                 const float4 v = fb[e];     // (re, re, im, im) of pairs 2q, 2q+1
@@ -401,80 +418,103 @@ m3_chunk_kernel(const M3Params p)
 #pragma unroll
             for (int q = 0; q < kM3Pairs / 2; ++q) {
                 const float4 a = p4[q];
-                const float2 ar = make_float2(a.x, a.y), ai = make_float2(a.z, a.w);
-                const float2 nr = fma2(ar, sre[q], mul2(make_float2(-a.z, -a.w), sim[q]));
-                const float2 ni = fma2(ar, sim[q], mul2(ai, sre[q]));
-                sre[q] = nr;
-                sim[q] = ni;
+                const float2 ar = make_float2(a.x, a.y), nai = make_float2(-a.z, -a.w), ai = make_float2(a.z, a.w);
+#pragma unroll
+                for (int j = 0; j < kM3Cpt; ++j) {
+                    const float2 nr = fma2(ar, sre[j][q], mul2(nai, sim[j][q]));
+                    const float2 ni = fma2(ar, sim[j][q], mul2(ai, sre[j][q]));
+                    sre[j][q] = nr;
+                    sim[j][q] = ni;
+                }
             }
 #pragma unroll kUnroll
             for (int tt = 0; tt < n; ++tt) {
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    const float xr_ = __bfloat162float(xs[(tt * R + r) * kM3Threads + tid]);
-                    const float2 x2 = make_float2(xr_, xr_);
+                    const float2 xv = __bfloat1622float2(
+                        *reinterpret_cast<const __nv_bfloat162*>(xs + (tt * R + r) * kM3Threads + cl));
+                    const float2 x2[kM3Cpt] = {make_float2(xv.x, xv.x), make_float2(xv.y, xv.y)};
 #pragma unroll
                     for (int q = 0; q < kM3N / 4; ++q) {
                         const float4 vv = fb[((tt * R + r) * kM3Heads + hl) * (kM3N / 4) + q];
-                        sre[q] = fma2(make_float2(vv.x, vv.y), x2, sre[q]);
-                        sim[q] = fma2(make_float2(vv.z, vv.w), x2, sim[q]);
+#pragma unroll
+                        for (int j = 0; j < kM3Cpt; ++j) {
+                            sre[j][q] = fma2(make_float2(vv.x, vv.y), x2[j], sre[j][q]);
+                            sim[j][q] = fma2(make_float2(vv.z, vv.w), x2[j], sim[j][q]);
+                        }
                     }
                 }
             }
         }
 
-        // y of this tile's first token for this thread's channel (output r at + r xr)
+        // y of this tile's first token for this thread's channels (output r at + r xr)
         __nv_bfloat16* yp = p.y + (static_cast<int64_t>(b) * p.L + ts) * xt + c;
 #pragma unroll kUnroll
         for (int tt = 0; FULL && tt < n; ++tt, yp += xt) {
-            float xv[R];
+            float2 xv[R];
 #pragma unroll
-            for (int r = 0; r < R; ++r) xv[r] = __bfloat162float(xs[(tt * R + r) * kM3Threads + tid]);
+            for (int r = 0; r < R; ++r)
+                xv[r] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(xs + (tt * R + r) * kM3Threads + cl));
             // q = a q + sum_r (omega b_r) x_r, two pairs per packed register
-            float2 vre[kM3Pairs / 2], vim[kM3Pairs / 2];
+            float2 vre[kM3Cpt][kM3Pairs / 2], vim[kM3Cpt][kM3Pairs / 2];
 #pragma unroll
-            for (int q = 0; q < kM3Pairs / 2; ++q) vre[q] = vim[q] = make_float2(0.0f, 0.0f);
+            for (int j = 0; j < kM3Cpt; ++j)
+#pragma unroll
+                for (int q = 0; q < kM3Pairs / 2; ++q) vre[j][q] = vim[j][q] = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                const float2 x2 = make_float2(xv[r], xv[r]);
+                const float2 x2[kM3Cpt] = {make_float2(xv[r].x, xv[r].x), make_float2(xv[r].y, xv[r].y)};
 #pragma unroll
                 for (int q = 0; q < kM3N / 4; ++q) {
                     const float4 bb = fb[((tt * R + r) * kM3Heads + hl) * (kM3N / 4) + q];
-                    vre[q] = fma2(make_float2(bb.x, bb.y), x2, vre[q]);
-                    vim[q] = fma2(make_float2(bb.z, bb.w), x2, vim[q]);
+#pragma unroll
+                    for (int j = 0; j < kM3Cpt; ++j) {
+                        vre[j][q] = fma2(make_float2(bb.x, bb.y), x2[j], vre[j][q]);
+                        vim[j][q] = fma2(make_float2(bb.z, bb.w), x2[j], vim[j][q]);
+                    }
                 }
             }
             const float4* fa4 = reinterpret_cast<const float4*>(fa) + (tt * kM3Heads + hl) * (kM3N / 4);
 #pragma unroll
             for (int q = 0; q < kM3Pairs / 2; ++q) {
                 const float4 a = fa4[q];              // (re, re, im, im) of pairs 2q, 2q+1
-                const float2 ar = make_float2(a.x, a.y), ai = make_float2(a.z, a.w);
-                const float2 nr = fma2(ar, sre[q], fma2(make_float2(-a.z, -a.w), sim[q], vre[q]));
-                const float2 ni = fma2(ar, sim[q], fma2(ai, sre[q], vim[q]));
-                sre[q] = nr;
-                sim[q] = ni;
+                const float2 ar = make_float2(a.x, a.y), ai = make_float2(a.z, a.w), nai = make_float2(-a.z, -a.w);
+#pragma unroll
+                for (int j = 0; j < kM3Cpt; ++j) {
+                    const float2 nr = fma2(ar, sre[j][q], fma2(nai, sim[j][q], vre[j][q]));
+                    const float2 ni = fma2(ar, sim[j][q], fma2(ai, sre[j][q], vim[j][q]));
+                    sre[j][q] = nr;
+                    sim[j][q] = ni;
+                }
             }
             if (FULL) {
                 const float* kap = fk + (tt * kM3Heads + hl) * R * R;
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
                     // sum_k Re(conj(c_k) q_k) = sum_k (c_re q_re + c_im q_im), then kappa
-                    float2 acc = make_float2(0.0f, 0.0f);
+                    float2 acc[kM3Cpt];
+#pragma unroll
+                    for (int j = 0; j < kM3Cpt; ++j) acc[j] = make_float2(0.0f, 0.0f);
 #pragma unroll
                     for (int q = 0; q < kM3N / 4; ++q) {
                         const float4 cc = fc[((tt * R + r) * kM3Heads + hl) * (kM3N / 4) + q];
-                        acc = fma2(make_float2(cc.x, cc.y), sre[q], acc);
-                        acc = fma2(make_float2(cc.z, cc.w), sim[q], acc);
-                    }
-                    float yv = acc.x + acc.y;
 #pragma unroll
-                    for (int rp = 0; rp < R; ++rp) yv = fmaf(kap[r * R + rp], xv[rp], yv);
+                        for (int j = 0; j < kM3Cpt; ++j) {
+                            acc[j] = fma2(make_float2(cc.x, cc.y), sre[j][q], acc[j]);
+                            acc[j] = fma2(make_float2(cc.z, cc.w), sim[j][q], acc[j]);
+                        }
+                    }
+                    float2 yv = make_float2(acc[0].x + acc[0].y, acc[1].x + acc[1].y);
+#pragma unroll
+                    for (int rp = 0; rp < R; ++rp) yv = fma2(make_float2(kap[r * R + rp], kap[r * R + rp]), xv[rp], yv);
                     if (p.z) {
                         // SiLU(z) = hz + hz tanh(hz), hz = z / 2
-                        const float hz = 0.5f * __bfloat162float(zs[(tt * R + r) * kM3Threads + tid]);
-                        yv *= fmaf(hz, tanh_fast(hz), hz);
+                        const float2 zv = __bfloat1622float2(
+                            *reinterpret_cast<const __nv_bfloat162*>(zs + (tt * R + r) * kM3Threads + cl));
+                        const float2 hz = mul2(make_float2(0.5f, 0.5f), zv);
+                        yv = mul2(yv, fma2(hz, make_float2(tanh_fast(hz.x), tanh_fast(hz.y)), hz));
                     }
-                    yp[r * xr] = __float2bfloat16_rn(yv);
+                    *reinterpret_cast<__nv_bfloat162*>(yp + r * xr) = __floats2bfloat162_rn(yv.x, yv.y);
                 }
             }
         }
@@ -487,13 +527,19 @@ m3_chunk_kernel(const M3Params p)
             // past the last token the tap weight is 0: q is the state s
             float4* hp = reinterpret_cast<float4*>(p.h_last + (static_cast<int64_t>(b) * C + c) * kM3N);
 #pragma unroll
-            for (int q = 0; q < kM3N / 4; ++q) hp[q] = make_float4(sre[q].x, sim[q].x, sre[q].y, sim[q].y);
+            for (int j = 0; j < kM3Cpt; ++j)
+#pragma unroll
+                for (int q = 0; q < kM3N / 4; ++q)
+                    hp[j * (kM3N / 4) + q] = make_float4(sre[j][q].x, sim[j][q].x, sre[j][q].y, sim[j][q].y);
         }
     } else {
         float4* ep = reinterpret_cast<float4*>(
             p.ws_state + ((static_cast<int64_t>(chunk) * gridDim.z + b) * C + c) * kM3N);
 #pragma unroll
-        for (int q = 0; q < kM3N / 4; ++q) ep[q] = make_float4(sre[q].x, sim[q].x, sre[q].y, sim[q].y);
+        for (int j = 0; j < kM3Cpt; ++j)
+#pragma unroll
+            for (int q = 0; q < kM3N / 4; ++q)
+                ep[j * (kM3N / 4) + q] = make_float4(sre[j][q].x, sim[j][q].x, sre[j][q].y, sim[j][q].y);
         if (tid < kM3Heads * kM3Pairs) {
             // (head h0_ + tid / pairs, pair tid % pairs)
             float* pp = p.ws_prod + ((static_cast<int64_t>(chunk) * gridDim.z + b) * p.H + h0_ + tid / kM3Pairs) * kM3N +

@@ -1625,11 +1625,11 @@ cudaError_t launch_m3(const mm::M3Params& p, unsigned cx, int64_t batch, cudaStr
     if (e != cudaSuccess) return e;
     if (p.chunks > 1) {
         mm::m3_chunk_kernel<false, R><<<dim3(cx, static_cast<unsigned>(p.chunks - 1), static_cast<unsigned>(batch)),
-                                        mm::kM3Threads, smem, s>>>(p);
+                                        mm::kM3Block, smem, s>>>(p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     mm::m3_chunk_kernel<true, R><<<dim3(cx, static_cast<unsigned>(p.chunks), static_cast<unsigned>(batch)),
-                                   mm::kM3Threads, smem, s>>>(p);
+                                   mm::kM3Block, smem, s>>>(p);
     return cudaGetLastError();
 }
 
