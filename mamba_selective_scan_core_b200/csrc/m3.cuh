@@ -209,6 +209,9 @@ m3_chunk_kernel(const M3Params p)
     constexpr int kUnroll = R == 1 ? 4 : 2;
     if (FULL && p.status && threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
         p.status[1] = p.status_epoch;
+    // the full pass, launched as a programmatic dependent of this summary
+    // pass, may start its chunk-0 CTAs (which read no summary) at once
+    if (!FULL) launch_dependents();
     const M3Layout lay = m3_layout(R);
     const int tid = threadIdx.x;
     const int cl = kM3Cpt * tid;                                              // first channel, CTA-local
@@ -280,7 +283,9 @@ m3_chunk_kernel(const M3Params p)
                 }
             }
         }
-        // carried through the earlier chunks: q = prod_c' q + e_c'
+        // carried through the earlier chunks: q = prod_c' q + e_c' (their
+        // summaries are complete and visible once the summary grid is)
+        if (chunk > 0) grid_dependency_wait();
         for (int cc = 0; cc < chunk; ++cc) {
             const float4* pp = reinterpret_cast<const float4*>(
                 p.ws_prod + ((static_cast<int64_t>(cc) * gridDim.z + b) * p.H + h) * kM3N);

@@ -1628,8 +1628,20 @@ cudaError_t launch_m3(const mm::M3Params& p, unsigned cx, int64_t batch, cudaStr
                                         mm::kM3Block, smem, s>>>(p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    mm::m3_chunk_kernel<true, R><<<dim3(cx, static_cast<unsigned>(p.chunks), static_cast<unsigned>(batch)),
-                                   mm::kM3Block, smem, s>>>(p);
+    // The full pass is a programmatic dependent of the summary pass: its
+    // chunk-0 CTAs run alongside the summary, the others wait for it in the
+    // kernel before reading the summaries.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cx, static_cast<unsigned>(p.chunks), static_cast<unsigned>(batch));
+    cfg.blockDim = dim3(mm::kM3Block);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.chunks > 1 ? 1 : 0;
+    if ((e = cudaLaunchKernelEx(&cfg, mm::m3_chunk_kernel<true, R>, p)) != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
