@@ -314,6 +314,16 @@ m3_chunk_kernel(const M3Params p)
     float4* fb = reinterpret_cast<float4*>(m3_sm + lay.off_bf());
     float4* fc = reinterpret_cast<float4*>(m3_sm + lay.off_cf());
     float* fk = reinterpret_cast<float*>(m3_sm + lay.off_k());
+    // The per-tile factor loops below stride by the block size, a multiple of
+    // heads x pairs, so each thread's elements there always belong to the same
+    // head (and pair): its per-head parameters are loaded once, here.
+    static_assert(kM3Block % (kM3Heads * kM3Pairs) == 0 && kM3Block % (kM3Heads * 16) == 0, "fixed head per thread");
+    const int hw = h0_ + tid % kM3Heads;                              // tap weights
+    const float bias_w = p.dt_bias ? p.dt_bias[hw] : 0.0f;
+    const int ka = tid % kM3Pairs, ha = h0_ + (tid / kM3Pairs) % kM3Heads;   // a_t
+    const float theta_a = p.theta[ha * kM3Pairs + ka];
+    const float A_a = p.A[ha];
+    const float dskip_k = p.Dskip ? p.Dskip[h0_ + (tid / (R * R)) % kM3Heads] : 0.0f;   // kappa
     int buf = 0;
     for (int64_t ts = t0; ts < t1; ts += T, buf ^= 1) {
         const int n = static_cast<int>(min(static_cast<int64_t>(T), t1 - ts));
@@ -331,10 +341,10 @@ m3_chunk_kernel(const M3Params p)
         // tap weights ((1 - lambda) Delta, lambda Delta) per (token, head), the
         // token after the tile included (zero past the sequence)
         for (int e = tid; e < (T + 1) * kM3Heads; e += kM3Block) {
-            const int tt = e / kM3Heads, hh = e % kM3Heads, hd = h0_ + hh;
+            const int tt = e / kM3Heads;
             float2 w = make_float2(0.0f, 0.0f);
             if (tt < nd) {
-                const float v = __bfloat162float(dts[e]) + (p.dt_bias ? p.dt_bias[hd] : 0.0f);
+                const float v = __bfloat162float(dts[e]) + bias_w;
                 const float dl = fmaxf(v, 0.0f) + log1pf(expf(-fabsf(v)));
                 const float lam = p.trap ? __bfloat162float(trs[e]) : 0.5f;
                 w = make_float2((1.0f - lam) * dl, lam * dl);
@@ -344,12 +354,12 @@ m3_chunk_kernel(const M3Params p)
         __syncthreads();
         // a_t per pair
         for (int e = tid; e < n * kM3Heads * kM3Pairs; e += kM3Block) {
-            const int k = e % kM3Pairs, th = e / kM3Pairs, hd = h0_ + th % kM3Heads;
+            const int k = ka, th = e / kM3Pairs;
             const float2 w = fw[th];
             const float dl = w.x + w.y;
             float sn, cs;
-            m3_sincos(dl * p.theta[hd * kM3Pairs + k], &sn, &cs);
-            const float mag = ex2_fast(dl * p.A[hd] * kLog2e);
+            m3_sincos(dl * theta_a, &sn, &cs);
+            const float mag = ex2_fast(dl * A_a * kLog2e);
             // per (token, head) and pair block q: (re 2q, re 2q+1, im 2q, im 2q+1)
             float* fq = reinterpret_cast<float*>(fa) + th * kM3N + (k >> 1) * 4 + (k & 1);
             fq[0] = mag * cs;
@@ -380,8 +390,7 @@ m3_chunk_kernel(const M3Params p)
                     const float4 bv = m3_widen4(bq[q]), cv = m3_widen4(cq[q]);
                     dot = fmaf(cv.x, bv.x, fmaf(cv.y, bv.y, fmaf(cv.z, bv.z, fmaf(cv.w, bv.w, dot))));
                 }
-                const float dh = p.Dskip ? p.Dskip[h0_ + hh] : 0.0f;
-                fk[e] = (r == rp ? dh : 0.0f) - fw[(tt + 1) * kM3Heads + hh].x * dot;
+                fk[e] = (r == rp ? dskip_k : 0.0f) - fw[(tt + 1) * kM3Heads + hh].x * dot;
             }
         }
         __syncthreads();
