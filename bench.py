@@ -41,6 +41,7 @@ METRIC = "Mamba mixer tokens/s per layer (d_inner 8192) and % of B200 HBM roofli
 PREFILL = CONFIGS["jamba_prefill"]
 DECODE = CONFIGS["decode_28x128"]
 SSD = SSD_CONFIGS["mamba2_prefill"]
+SSD_DEC = SSD_CONFIGS["mamba2_decode"]
 M3 = M3_CONFIGS["mamba3_prefill"]
 M3_MIMO = M3_CONFIGS["mamba3_mimo"]
 
@@ -98,6 +99,7 @@ TRAFFIC_SOURCES = {
     "proj_gemm/dt_proj": ("proj_gemm.cuh", "mixer_common.cuh", API_HEAD),
     "ssd/mamba2_prefill": ("ssd.cuh", "proj_gemm.cuh", "mixer_common.cuh", "mixer_api.cu"),
     "m3/mamba3_prefill": ("m3.cuh", "mixer_common.cuh", "mixer_api.cu"),
+    "ssd/mamba2_decode": ("ssd.cuh", "mixer_common.cuh", "mixer_api.cu"),
 }
 
 
@@ -339,6 +341,7 @@ def run_gpu(args):
 
     # ---- the Mamba-2 form (scalar decay per head, chunked products on the tensor cores)
     ssd = run_ssd(mm, args, world, hbm_peak, hbm_src, peaks)
+    ssd_dec = run_ssd_decode(mm, args, world, hbm_peak, hbm_src)
 
     # ---- the Mamba-3 form (trapezoidal rule, rotating complex state), single input and rank 4
     m3 = {cfg.name: run_m3(mm, args, world, hbm_peak, hbm_src, alu_peak, cfg) for cfg in (M3, M3_MIMO)}
@@ -380,6 +383,7 @@ def run_gpu(args):
             "bc_rmsnorm": normed,
             "projections": proj,
             "mamba2_ssd": ssd,
+            "mamba2_decode": ssd_dec,
             "mamba3": m3,
             **legs,
             "launch_ms": {"mean": round(statistics.mean(launch_ms), 5), "min": round(min(launch_ms), 5),
@@ -773,6 +777,48 @@ def run_ssd(mm, args, world, hbm_peak, hbm_src, peaks):
     }
 
 
+def ssd_decode_bytes(cfg):
+    """Algorithmic HBM bytes of one Mamba-2 decode step: the fp32 state read
+    and written, x, z and y (bf16), dt, B and C (bf16) and the per-head
+    parameters, each moved once."""
+    B, H, P, N, G = cfg.batch, cfg.heads, cfg.headdim, cfg.d_state, cfg.groups
+    return 2 * B * H * P * N * 4 + (3 if cfg.gate else 2) * B * H * P * 2 + B * H * 2 + 2 * B * G * N * 2 + \
+        3 * H * 4
+
+
+def _ssd_decode_setup(mm, cfg):
+    d = {k: (v.cuda() if v is not None else None) for k, v in make_ssd_inputs(cfg).items()}
+    tok = {k: d[k][:, 0].contiguous() for k in ("x", "z", "dt", "Bm", "Cm") if d.get(k) is not None}
+    state = d["h0"]
+    y = torch.empty((cfg.batch, cfg.heads * cfg.headdim), dtype=torch.bfloat16, device="cuda")
+    step = lambda: mm.ssd_state_update(tok["x"], tok.get("z"), tok["dt"], d["dt_bias"], d["A"], tok["Bm"],  # noqa: E731
+                                       tok["Cm"], d["Dskip"], state, y=y)
+    return step, (d, tok, state, y)
+
+
+def run_ssd_decode(mm, args, world, hbm_peak, hbm_src):
+    """One decode token of the Mamba-2 form for 128 sequences at d_inner 8192
+    (128 heads of 64, d_state 128): one launch, in place on a 512 MB fp32
+    state (larger than L2, so no rotation is needed).  Roofline: the state's
+    read and write plus the token's activations against the copy bandwidth."""
+    cfg = SSD_DEC
+    step, keep = _ssd_decode_setup(mm, cfg)
+    K = max(3, min(args.steps, 200))
+    ms = _time_loop(step, K, world)
+    nbytes = ssd_decode_bytes(cfg)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    del keep, step
+    torch.cuda.empty_cache()
+    return {
+        "workload": cfg.name, "batch": cfg.batch, "heads": cfg.heads, "headdim": cfg.headdim,
+        "d_state": cfg.d_state, "groups": cfg.groups, "steps": K, "ms_per_step": round(ms, 5),
+        "value": round(_job_rate(world, cfg.batch, ms), 1), "unit": "tokens/s", "launches_per_call": 1,
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(gbs / hbm_peak, 4), "traffic": _ncu_traffic("ssd/mamba2_decode"),
+                     "algorithmic_bytes": nbytes, "peak_source": hbm_src},
+    }
+
+
 M3_KEYS = ("x", "z", "dt", "trap", "dt_bias", "A", "theta", "Bm", "Cm", "Dskip", "h0", "x_prev", "B_prev")
 
 
@@ -990,6 +1036,8 @@ def run_only(args):
                torch.empty((cfg.batch, cfg.heads, cfg.headdim, cfg.d_state), device="cuda"))
         ws = torch.empty(mm.ssd_workspace_size(cfg.batch, cfg.seqlen, cfg.heads), dtype=torch.uint8, device="cuda")
         step = lambda: _ssd_call(mm, d, out, ws)  # noqa: E731
+    elif args.only == "ssddecode":
+        step, keep = _ssd_decode_setup(mm, SSD_DEC)
     elif args.only in ("m3", "m3mimo"):
         cfg = M3 if args.only == "m3" else M3_MIMO
         d = {k: (v.cuda() if v is not None else None) for k, v in make_m3_inputs(cfg).items()}
@@ -1038,7 +1086,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra-prefill", action="store_true",
                     help="skip the 4 x 32768 and 262,144-token prefill legs")
-    ap.add_argument("--only", choices=["forward", "decode", "xproj", "dtproj", "projected", "ssd", "m3", "m3mimo"],
+    ap.add_argument("--only", choices=["forward", "decode", "xproj", "dtproj", "projected", "ssd", "ssddecode", "m3",
+                                       "m3mimo"],
                     default=None,
                     help="run one kernel's timed loop only (for profiler captures); prints no JSON line")
     ap.add_argument("--decode-layers", type=int, default=None,

@@ -15,6 +15,10 @@
  * the producers either side of the scan, on the tensor cores (tcgen05):
  *   mamba_proj_matmul           out = A W^T, a projection (bf16 operands, fp32 accumulation)
  *   mamba_mixer_fwd_projected   conv -> x_proj -> [dt_low | B | C] (+RMSNorm) -> dt_proj -> scan
+ * the Mamba-2 and Mamba-3 forms of the scan:
+ *   mamba_ssd_fwd            Mamba-2 prefill (scalar decay per head, chunked products on the tensor cores)
+ *   mamba_ssd_state_update   Mamba-2 one-token step (decode), in place on the state
+ *   mamba_m3_fwd             Mamba-3 prefill (trapezoid rule, complex state, 1/2/4 inputs per state)
  *
  * and two status readers:
  *   mamba_check_status       did the last forward on this workspace complete? (per call)
@@ -460,6 +464,39 @@ size_t mamba_ssd_workspace_size(int64_t batch, int64_t seqlen, int64_t heads, in
                                 int64_t groups);
 
 /*
+ * One token of the Mamba-2 form (decode), in place on the state: the
+ * recurrence of mamba_ssd_fwd above for a single token, with the state the
+ * previous call (prefill or decode) left as h_last:
+ *
+ *   Delta    = softplus(dt[h] + dt_bias[h])
+ *   s[p,n]   = exp(Delta A[h]) s[p,n] + Delta B[g,n] x[c]
+ *   y[c]     = (sum_n C[g,n] s[p,n] + D[h] x[c]) * SiLU(z[c])   (no gate if z is NULL)
+ *
+ *   x, z           [batch, heads*headdim]            bf16  (z may be NULL)
+ *   dt             [batch, heads]                    bf16  before dt_bias and softplus
+ *   dt_bias        [heads]                           fp32  or NULL (= 0)
+ *   A              [heads]                           fp32  negative
+ *   Bm, Cm         [batch, groups, d_state]          bf16
+ *   Dskip          [heads]                           fp32  or NULL (= 0)
+ *   state          [batch, heads, headdim, d_state]  fp32  read and overwritten
+ *   y              [batch, heads*headdim]            bf16  output
+ *
+ * The same results as mamba_ssd_fwd with seqlen 1, h0 = state and h_last =
+ * state, up to rounding order.  Supported: headdim == 64, d_state == 128
+ * (MM_ERR_UNSUPPORTED otherwise); heads a multiple of groups, both positive,
+ * batch <= 65535 (MM_ERR_SHAPE).  Every pointer 16-byte aligned
+ * (MM_ERR_ALIGN); state and y may not overlap an input or each other
+ * (MM_ERR_ALIAS).  No workspace and no wait: one launch of one CTA per (head,
+ * sequence) on `stream`.  batch == 0 is a no-op.  Errors otherwise as
+ * mamba_state_update.
+ */
+mm_status mamba_ssd_state_update(const void* x, const void* z, const void* dt, const float* dt_bias,
+                                 const float* A, const void* Bm, const void* Cm, const float* Dskip,
+                                 float* state, void* y,
+                                 int64_t batch, int64_t heads, int64_t headdim, int64_t d_state, int64_t groups,
+                                 void* stream);
+
+/*
  * The Mamba-3 form of the selective scan, prefill (bf16 activations, fp32
  * state and arithmetic).  The Jamba lesson's "Mamba-3" section names three
  * changes over Mamba-2: an exponential-trapezoidal discretisation, whose
@@ -518,7 +555,7 @@ const char* mamba_status_string(mm_status status);
 /* ABI version of this header (incremented on any signature change). */
 int mamba_mixer_abi_version(void);
 
-#define MAMBA_MIXER_ABI_VERSION 7
+#define MAMBA_MIXER_ABI_VERSION 8
 
 #ifdef __cplusplus
 }

@@ -17,7 +17,7 @@ __all__ = [
     "MM_F32", "MM_BF16", "MixerError", "lib", "library_path", "mixer_fwd", "mixer_fwd_noalloc", "mixer_fwd_host",
     "state_update", "workspace_size", "host_workspace_size", "status_string", "abi_version", "fault_status",
     "check_status", "proj_matmul", "proj_matmul_workspace_size", "mixer_fwd_projected",
-    "projected_workspace_size", "ssd_fwd", "ssd_workspace_size", "m3_fwd", "m3_workspace_size", "EXPORTED_SYMBOLS",
+    "projected_workspace_size", "ssd_fwd", "ssd_workspace_size", "ssd_state_update", "m3_fwd", "m3_workspace_size", "EXPORTED_SYMBOLS",
 ]
 
 MM_F32 = 0
@@ -47,6 +47,7 @@ EXPORTED_SYMBOLS = (
     "mamba_mixer_projected_layout",
     "mamba_ssd_fwd",
     "mamba_ssd_workspace_size",
+    "mamba_ssd_state_update",
     "mamba_m3_fwd",
     "mamba_m3_workspace_size",
 )
@@ -113,6 +114,8 @@ def _declare(L):
     L.mamba_ssd_fwd.argtypes = [P] * 11 + [I64] * 6 + [P, ctypes.c_size_t, P]
     L.mamba_ssd_workspace_size.restype = ctypes.c_size_t
     L.mamba_ssd_workspace_size.argtypes = [I64] * 6
+    L.mamba_ssd_state_update.restype = ctypes.c_int
+    L.mamba_ssd_state_update.argtypes = [P] * 10 + [I64] * 5 + [P]
     L.mamba_m3_fwd.restype = ctypes.c_int
     L.mamba_m3_fwd.argtypes = [P] * 15 + [I64] * 7 + [P, ctypes.c_size_t, P]
     L.mamba_m3_workspace_size.restype = ctypes.c_size_t
@@ -612,6 +615,45 @@ def ssd_fwd(x, z, dt, dt_bias, A, Bm, Cm, Dskip, h0=None, *, headdim=64, y=None,
         raise MixerError(st, "mamba_ssd_fwd")
     _keep_alive_on(made, (stream,))
     return y, h_last
+
+
+def ssd_state_update(x, z, dt, dt_bias, A, Bm, Cm, Dskip, state, *, headdim=64, y=None, stream=None):
+    """One token of the Mamba-2 form (mamba_ssd_state_update), in place on
+    state [B,H,P,N] fp32: x, z [B,H*P] bf16 (z may be None: no gate), dt [B,H]
+    bf16, dt_bias/A/Dskip [H] fp32 (dt_bias and Dskip may be None), Bm/Cm
+    [B,G,N] bf16, P = headdim.  Returns y [B,H*P] bf16, allocated if not given."""
+    import torch
+
+    bf, f32 = torch.bfloat16, torch.float32
+    Bsz, HP = x.shape
+    H = A.shape[0]
+    P = int(headdim)
+    G, N = Bm.shape[1], Bm.shape[2]
+    if HP != H * P:
+        raise ValueError(f"x has {HP} channels, expected heads x headdim = {H * P}")
+    dev = x.device
+    made = []
+    _check(x, "x", bf, (Bsz, H * P), dev)
+    _check(z, "z", bf, (Bsz, H * P), dev)
+    _check(dt, "dt", bf, (Bsz, H), dev)
+    _check(dt_bias, "dt_bias", f32, (H,), dev)
+    _check(A, "A", f32, (H,), dev)
+    _check(Bm, "Bm", bf, (Bsz, G, N), dev)
+    _check(Cm, "Cm", bf, (Bsz, G, N), dev)
+    _check(Dskip, "Dskip", f32, (H,), dev)
+    _check(state, "state", f32, (Bsz, H, P, N), dev)
+    if y is None:
+        y = torch.empty((Bsz, H * P), dtype=bf, device=dev)
+        made.append(y)
+    _check(y, "y", bf, (Bsz, H * P), dev)
+    with torch.cuda.device(dev):
+        st = lib().mamba_ssd_state_update(_ptr(x), _ptr(z), _ptr(dt), _ptr(dt_bias), _ptr(A), _ptr(Bm), _ptr(Cm),
+                                          _ptr(Dskip), _ptr(state), _ptr(y), Bsz, H, P, N, G,
+                                          _stream_handle(stream))
+    if st != 0:
+        raise MixerError(st, "mamba_ssd_state_update")
+    _keep_alive_on(made, (stream,))
+    return y
 
 
 def m3_workspace_size(batch, seqlen, heads, rank=1, headdim=64, d_state=16, groups=1) -> int:

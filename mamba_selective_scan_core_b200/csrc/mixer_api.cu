@@ -1585,6 +1585,50 @@ mm_status mamba_ssd_fwd(const void* x, const void* z, const void* dt, const floa
     return MM_OK;
 }
 
+mm_status mamba_ssd_state_update(const void* x, const void* z, const void* dt, const float* dt_bias,
+                                 const float* A, const void* Bm, const void* Cm, const float* Dskip,
+                                 float* state, void* y,
+                                 int64_t batch, int64_t heads, int64_t headdim, int64_t d_state, int64_t groups,
+                                 void* stream)
+{
+    if (batch < 0 || heads <= 0 || groups <= 0 || heads % groups != 0 || batch > 65535 || heads > (1 << 20))
+        return MM_ERR_SHAPE;
+    if (headdim != mm::kSsdP || d_state != mm::kSsdN) return MM_ERR_UNSUPPORTED;
+    if (batch == 0) return MM_OK;
+    if (!x || !dt || !A || !Bm || !Cm || !state || !y) return MM_ERR_NULL;
+    for (const void* q : {x, z, dt, static_cast<const void*>(dt_bias), static_cast<const void*>(A), Bm, Cm,
+                          static_cast<const void*>(Dskip), static_cast<const void*>(state), static_cast<const void*>(y)})
+        if (q && !aligned16(q)) return MM_ERR_ALIGN;
+    const int64_t C = heads * mm::kSsdP;
+    const Span sx = span(x, batch * C * 2), sz = span(z, batch * C * 2), sdt = span(dt, batch * heads * 2),
+               sbias = span(dt_bias, heads * 4), sa = span(A, heads * 4),
+               sb = span(Bm, batch * groups * mm::kSsdN * 2), sc = span(Cm, batch * groups * mm::kSsdN * 2),
+               sd = span(Dskip, heads * 4), sst = span(state, batch * C * mm::kSsdN * 4), sy = span(y, batch * C * 2);
+    const Span ins[] = {sx, sz, sdt, sbias, sa, sb, sc, sd};
+    for (const Span& in : ins)
+        if (overlaps(sy, in) || overlaps(sst, in)) return MM_ERR_ALIAS;
+    if (overlaps(sy, sst)) return MM_ERR_ALIAS;
+    if (mm_status st = check_device(); st != MM_OK) return st;
+
+    mm::SsdDecodeParams p{};
+    p.x = static_cast<const __nv_bfloat16*>(x);
+    p.z = static_cast<const __nv_bfloat16*>(z);
+    p.dt = static_cast<const __nv_bfloat16*>(dt);
+    p.dt_bias = dt_bias;
+    p.A = A;
+    p.Bm = static_cast<const __nv_bfloat16*>(Bm);
+    p.Cm = static_cast<const __nv_bfloat16*>(Cm);
+    p.Dskip = Dskip;
+    p.state = state;
+    p.y = static_cast<__nv_bfloat16*>(y);
+    p.H = static_cast<int>(heads);
+    p.G = static_cast<int>(groups);
+    mm::ssd_state_update_kernel<<<dim3(static_cast<unsigned>(heads), static_cast<unsigned>(batch)),
+                                  mm::kSsdDecThreads, forced_launch_failure() ? (1 << 20) : 0,
+                                  static_cast<cudaStream_t>(stream)>>>(p);
+    return cudaGetLastError() == cudaSuccess ? MM_OK : MM_ERR_CUDA;
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------- Mamba-3 form (chunked fp32 recurrence)

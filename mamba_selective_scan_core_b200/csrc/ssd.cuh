@@ -647,4 +647,88 @@ ssd_chunk_scan_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_
     }
 }
 
+
+// ---------------------------------------------------------------- one-token step (decode)
+// The recurrence above for a single token per (head, sequence), in place on
+// the state: with Delta = softplus(dt[h] + dt_bias[h]),
+//     s[p,n] <- exp(Delta A[h]) s[p,n] + Delta x[p] B[n]
+//     y[p]    = (sum_n C[n] s[p,n] + D[h] x[p]) SiLU(z[p])
+// No product is dense enough for the tensor cores: each state entry is read
+// once, updated and written back, so the step is bound by the state's HBM
+// traffic (2 x 32 KB per head at P = 64, N = 128, fp32).  One CTA of 8 warps
+// per (head, sequence); warp w holds state rows 8w .. 8w+7, lane l entries
+// 4l .. 4l+3 of each (a warp's row is 512 contiguous bytes), all eight rows'
+// loads in flight before the arithmetic.  A row's readout is a warp sum.
+constexpr int kSsdDecThreads = 256;
+constexpr int kSsdDecRows = kSsdP / (kSsdDecThreads / 32);    // state rows per warp
+static_assert(kSsdDecRows == 8 && kSsdN == 4 * 32, "a warp covers 8 rows, a lane 4 entries of each");
+
+struct SsdDecodeParams {
+    const __nv_bfloat16* x;      // [B][H*P]
+    const __nv_bfloat16* z;      // [B][H*P] or null (no gate)
+    const __nv_bfloat16* dt;     // [B][H]
+    const float* dt_bias;        // [H] or null
+    const float* A;              // [H]
+    const __nv_bfloat16* Bm;     // [B][G*N]
+    const __nv_bfloat16* Cm;     // [B][G*N]
+    const float* Dskip;          // [H] or null
+    float* state;                // [B][H][P][N], updated in place
+    __nv_bfloat16* y;            // [B][H*P]
+    int H, G;
+};
+
+__global__ void __launch_bounds__(kSsdDecThreads)
+ssd_state_update_kernel(const SsdDecodeParams p)
+{
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = h / (p.H / p.G);
+    const int64_t C = static_cast<int64_t>(p.H) * kSsdP;
+    float4* st = reinterpret_cast<float4*>(p.state + ((static_cast<int64_t>(b) * p.H + h) * kSsdP +
+                                                      warp * kSsdDecRows) * kSsdN) + lane;
+    float4 s[kSsdDecRows];
+#pragma unroll
+    for (int r = 0; r < kSsdDecRows; ++r) s[r] = st[r * (kSsdN / 4)];
+
+    const float v = __bfloat162float(p.dt[static_cast<int64_t>(b) * p.H + h]) + (p.dt_bias ? p.dt_bias[h] : 0.0f);
+    const float dl = fmaxf(v, 0.0f) + log1pf(expf(-fabsf(v)));
+    const float da = expf(dl * p.A[h]);
+    const int64_t bc = (static_cast<int64_t>(b) * p.G + g) * kSsdN + 4 * lane;
+    const uint2 braw = *reinterpret_cast<const uint2*>(p.Bm + bc);
+    const uint2 craw = *reinterpret_cast<const uint2*>(p.Cm + bc);
+    const float4 bv = make_float4(bf16_lo(braw.x), bf16_hi(braw.x), bf16_lo(braw.y), bf16_hi(braw.y));
+    const float4 cv = make_float4(bf16_lo(craw.x), bf16_hi(craw.x), bf16_lo(craw.y), bf16_hi(craw.y));
+    // x of the warp's 8 rows: one 16-byte load, the same for every lane
+    const int64_t c0 = static_cast<int64_t>(b) * C + static_cast<int64_t>(h) * kSsdP + warp * kSsdDecRows;
+    const uint4 xraw = *reinterpret_cast<const uint4*>(p.x + c0);
+    const float xv[kSsdDecRows] = {bf16_lo(xraw.x), bf16_hi(xraw.x), bf16_lo(xraw.y), bf16_hi(xraw.y),
+                                   bf16_lo(xraw.z), bf16_hi(xraw.z), bf16_lo(xraw.w), bf16_hi(xraw.w)};
+    float mine = 0.0f;    // lane r < 8: the readout of row r
+#pragma unroll
+    for (int r = 0; r < kSsdDecRows; ++r) {
+        const float u = dl * xv[r];
+        s[r].x = fmaf(da, s[r].x, u * bv.x);
+        s[r].y = fmaf(da, s[r].y, u * bv.y);
+        s[r].z = fmaf(da, s[r].z, u * bv.z);
+        s[r].w = fmaf(da, s[r].w, u * bv.w);
+        st[r * (kSsdN / 4)] = s[r];
+        float acc = fmaf(cv.x, s[r].x, fmaf(cv.y, s[r].y, fmaf(cv.z, s[r].z, cv.w * s[r].w)));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+        if (lane == r) mine = acc;
+    }
+    if (lane < kSsdDecRows) {
+        float xr = 0.0f;      // xv[lane], without a dynamic register index
+#pragma unroll
+        for (int r = 0; r < kSsdDecRows; ++r)
+            if (lane == r) xr = xv[r];
+        float yv = mine + (p.Dskip ? p.Dskip[h] : 0.0f) * xr;
+        if (p.z) {
+            const float zv = __bfloat162float(p.z[c0 + lane]);
+            yv *= zv / (1.0f + expf(-zv));
+        }
+        p.y[c0 + lane] = __float2bfloat16_rn(yv);
+    }
+}
+
 }  // namespace mm

@@ -69,7 +69,7 @@ def test_exported_symbols_are_c_linkage():
 
 def test_version_and_strings():
     mmbuild.build()
-    assert mm.abi_version() == 7
+    assert mm.abi_version() == 8
     for code in range(14):
         s = mm.status_string(code)
         assert s and s != "unknown status"
@@ -352,6 +352,33 @@ def test_ssd_validation(L):
     assert L.mamba_ssd_fwd(*ssd_args(ws_bytes=need - 16)) == EWORKSPACE
     assert L.mamba_ssd_fwd(*ssd_args(ws=None)) == EWORKSPACE
     assert L.mamba_ssd_fwd(*ssd_args(ws=WS_ADDR + 8)) == EALIGN
+
+
+def ssd_decode_args(B=2, H=4, P=64, N=128, G=2, **over):
+    """mamba_ssd_state_update arguments on fake addresses, each buffer 2^32 apart."""
+    names = ["x", "z", "dt", "dt_bias", "A", "Bm", "Cm", "Dskip", "state", "y"]
+    addr = {n: BASE + (i << 32) for i, n in enumerate(names)}
+    addr.update(over)
+    return [addr[n] for n in names] + [B, H, P, N, G, None]
+
+
+def test_ssd_decode_validation(L):
+    assert L.mamba_ssd_state_update(*ssd_decode_args()) == EDEVICE
+    assert L.mamba_ssd_state_update(*ssd_decode_args(z=None, dt_bias=None, Dskip=None)) == EDEVICE
+    assert L.mamba_ssd_state_update(*ssd_decode_args(P=32)) == EUNSUP
+    assert L.mamba_ssd_state_update(*ssd_decode_args(N=64)) == EUNSUP
+    assert L.mamba_ssd_state_update(*ssd_decode_args(H=6, G=4)) == ESHAPE
+    assert L.mamba_ssd_state_update(*ssd_decode_args(G=0)) == ESHAPE
+    assert L.mamba_ssd_state_update(*ssd_decode_args(B=-1)) == ESHAPE
+    assert L.mamba_ssd_state_update(*ssd_decode_args(B=70000)) == ESHAPE
+    assert L.mamba_ssd_state_update(*ssd_decode_args(B=0)) == OK
+    for name in ("x", "dt", "A", "Bm", "Cm", "state", "y"):
+        assert L.mamba_ssd_state_update(*ssd_decode_args(**{name: None})) == ENULL, name
+    for name in ("x", "z", "Cm", "state", "y", "Dskip"):
+        assert L.mamba_ssd_state_update(*ssd_decode_args(**{name: BASE + (1 << 40) + 8})) == EALIGN, name
+    assert L.mamba_ssd_state_update(*ssd_decode_args(y=BASE)) == EALIAS                  # y over x
+    assert L.mamba_ssd_state_update(*ssd_decode_args(state=BASE + (5 << 32))) == EALIAS  # state over B
+    assert L.mamba_ssd_state_update(*ssd_decode_args(y=BASE + (8 << 32) + 64)) == EALIAS # y over state
 
 
 # ---------------------------------------------------------------- Mamba-3 form

@@ -203,3 +203,115 @@ def test_ssd_token_by_token_continues_prefill():
         ys.append(y)
     torch.cuda.synchronize()
     check(inp, torch.cat(ys, dim=1), h)
+
+
+# ---------------------------------------------------------------- one-token step (decode)
+def gpu_ssd_decode(d, state=None):
+    """mamba_ssd_state_update on the first token of one-token inputs d, in place
+    on `state` (a copy of d's h0, or zeros, when not given).  Returns y
+    [B,1,H*P] and the state."""
+    B, _, C = d["x"].shape
+    H = d["A"].shape[0]
+    if state is None:
+        state = d["h0"].clone() if d.get("h0") is not None else torch.zeros((B, H, 64, 128), device="cuda")
+    tok = {k: (d[k][:, 0].contiguous() if d.get(k) is not None else None) for k in ("x", "z", "dt", "Bm", "Cm")}
+    y = mm.ssd_state_update(tok["x"], tok["z"], tok["dt"], d.get("dt_bias"), d["A"], tok["Bm"], tok["Cm"],
+                            d.get("Dskip"), state)
+    return y[:, None], state
+
+
+@pytest.mark.parametrize("B,H,G,gate,skip,bias,h0", [(1, 1, 1, True, True, True, True),
+                                                     (2, 4, 2, True, True, True, True),
+                                                     (3, 6, 3, False, False, True, True),
+                                                     (2, 8, 1, True, False, False, True),
+                                                     (5, 2, 2, True, True, True, False)])
+def test_ssd_decode_small(B, H, G, gate, skip, bias, h0):
+    """One token against the oracle's one-token run from the same state."""
+    inp = make_ssd_inputs_custom(B, 1, H, groups=G, seed=300 + B * 11 + H, h0_std=0.3 if h0 else 0.0, gate=gate)
+    if not skip:
+        inp["Dskip"] = None
+    if not bias:
+        inp["dt_bias"] = None
+    y, state = gpu_ssd_decode(to_dev(inp))
+    torch.cuda.synchronize()
+    check(inp, y, state)
+
+
+def test_ssd_decode_large_steps():
+    """Large and small step sizes (softplus on both tails, decays near 0 and 1)."""
+    inp = make_ssd_inputs_custom(2, 1, 4, seed=77, h0_std=0.5, dt_std=4.0)
+    y, state = gpu_ssd_decode(to_dev(inp))
+    torch.cuda.synchronize()
+    check(inp, y, state)
+
+
+def test_ssd_decode_continues_prefill():
+    """Decode use: a prefill of 61 tokens, then three decode steps in place on
+    its h_last, match the oracle's single run of all 64 tokens."""
+    inp = make_ssd_inputs_custom(2, 64, 4, groups=2, seed=45, h0_std=0.2)
+    d = to_dev(inp)
+    c = dict(d)
+    for k in ("x", "z", "dt", "Bm", "Cm"):
+        c[k] = d[k][:, :61].contiguous()
+    y0, state = gpu_ssd(c)
+    ys = [y0]
+    for t in range(61, 64):
+        c = dict(d)
+        for k in ("x", "z", "dt", "Bm", "Cm"):
+            c[k] = d[k][:, t:t + 1].contiguous()
+        y, state = gpu_ssd_decode(c, state)
+        ys.append(y)
+    torch.cuda.synchronize()
+    check(inp, torch.cat(ys, dim=1), state)
+
+
+def test_ssd_decode_matches_one_token_prefill():
+    """The decode step and the chunked prefill of one token agree (the two
+    paths sum in different orders; both within the tolerance of the oracle,
+    and close to each other)."""
+    inp = make_ssd_inputs_custom(2, 1, 4, groups=1, seed=51, h0_std=0.3)
+    d = to_dev(inp)
+    yp, hp = gpu_ssd(d)
+    yd, hd = gpu_ssd_decode(d)
+    torch.cuda.synchronize()
+    check(inp, yd, hd)
+    assert torch.allclose(hd, hp, rtol=1e-4, atol=1e-4)
+
+
+def test_ssd_decode_full_size():
+    """The decode workload at full size (128 sequences x 128 heads of 64,
+    d_state 128: a 512 MB state), as the bench times it: every head of every
+    sequence against the oracle."""
+    cfg = SSD_CONFIGS["mamba2_decode"]
+    inp = make_ssd_inputs(cfg)
+    y, state = gpu_ssd_decode(to_dev(inp))
+    torch.cuda.synchronize()
+    check(inp, y, state)
+
+
+def test_ssd_decode_graph_replay():
+    """Captured in a CUDA graph, two replays from the same state give the
+    bits of two eager calls."""
+    inp = make_ssd_inputs_custom(2, 1, 4, seed=53, h0_std=0.3)
+    d = to_dev(inp)
+    s_eager = d["h0"].clone()
+    ye1, _ = gpu_ssd_decode(d, s_eager)
+    ye2, _ = gpu_ssd_decode(d, s_eager)
+    s_graph = d["h0"].clone()
+    tok = {k: d[k][:, 0].contiguous() for k in ("x", "z", "dt", "Bm", "Cm")}
+    yg = torch.empty_like(ye1[:, 0])
+    mm.ssd_state_update(tok["x"], tok["z"], tok["dt"], d["dt_bias"], d["A"], tok["Bm"], tok["Cm"], d["Dskip"],
+                        s_graph.clone(), y=yg)      # warm-up outside the capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        mm.ssd_state_update(tok["x"], tok["z"], tok["dt"], d["dt_bias"], d["A"], tok["Bm"], tok["Cm"], d["Dskip"],
+                            s_graph, y=yg)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(yg, ye1[:, 0])
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(yg, ye2[:, 0])
+    assert torch.equal(s_graph, s_eager)
+

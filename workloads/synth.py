@@ -206,6 +206,9 @@ SSD_CONFIGS = {
     "mamba2_batched": SsdConfig(
         "mamba2_batched", batch=4, seqlen=8192, heads=128, seed=6, h0_std=0.1,
         desc="Mamba-2 form, 4 x 8192 tokens with an initial state"),
+    "mamba2_decode": SsdConfig(
+        "mamba2_decode", batch=128, seqlen=1, heads=128, seed=8, h0_std=0.3,
+        desc="Mamba-2 form, one decode token for 128 sequences at the Jamba width: a 512 MB fp32 state"),
 }
 
 
