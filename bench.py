@@ -44,6 +44,7 @@ SSD = SSD_CONFIGS["mamba2_prefill"]
 SSD_DEC = SSD_CONFIGS["mamba2_decode"]
 M3 = M3_CONFIGS["mamba3_prefill"]
 M3_MIMO = M3_CONFIGS["mamba3_mimo"]
+M3_DEC = M3_CONFIGS["mamba3_decode"]
 
 SMS = 148
 FP32_LANES_PER_SM = 128
@@ -100,6 +101,7 @@ TRAFFIC_SOURCES = {
     "ssd/mamba2_prefill": ("ssd.cuh", "proj_gemm.cuh", "mixer_common.cuh", "mixer_api.cu"),
     "m3/mamba3_prefill": ("m3.cuh", "mixer_common.cuh", "mixer_api.cu"),
     "ssd/mamba2_decode": ("ssd.cuh", "mixer_common.cuh", "mixer_api.cu"),
+    "m3/mamba3_decode": ("m3.cuh", "mixer_common.cuh", "mixer_api.cu"),
 }
 
 
@@ -345,6 +347,7 @@ def run_gpu(args):
 
     # ---- the Mamba-3 form (trapezoidal rule, rotating complex state), single input and rank 4
     m3 = {cfg.name: run_m3(mm, args, world, hbm_peak, hbm_src, alu_peak, cfg) for cfg in (M3, M3_MIMO)}
+    m3[M3_DEC.name] = run_m3_decode(mm, args, world, hbm_peak, hbm_src)
 
     result = None
     if rank == 0:
@@ -843,6 +846,51 @@ def m3_fp32_ops(cfg):
     return pairs * (8 + 4 * cfg.rank) + 2 * cfg.rank
 
 
+def m3_decode_bytes(cfg):
+    """Algorithmic HBM bytes of one Mamba-3 decode step: the fp32 state read
+    and written, x, z, y and the previous token's x (R x d_inner bf16 each),
+    dt and the trapezoid weight, B, C and the previous B (bf16), and the
+    per-head parameters, each moved once."""
+    B, H, P, N, G, R = cfg.batch, cfg.heads, cfg.headdim, cfg.d_state, cfg.groups, cfg.rank
+    return 2 * B * H * P * N * 4 + (3 + (1 if cfg.prev else 0) + (0 if cfg.gate else -1)) * B * R * H * P * 2 + \
+        2 * B * H * 2 + (3 if cfg.prev else 2) * B * R * G * N * 2 + (3 * H + H * N // 2) * 4
+
+
+def _m3_decode_setup(mm, cfg):
+    d = {k: (v.cuda() if v is not None else None) for k, v in make_m3_inputs(cfg).items()}
+    tok = {k: d[k][:, 0].contiguous() for k in ("x", "z", "dt", "trap", "Bm", "Cm") if d.get(k) is not None}
+    state = d["h0"]
+    y = torch.empty((cfg.batch, cfg.rank, cfg.heads * cfg.headdim), dtype=torch.bfloat16, device="cuda")
+    step = lambda: mm.m3_state_update(tok["x"], tok.get("z"), tok["dt"], tok.get("trap"), d["dt_bias"], d["A"],  # noqa: E731
+                                      d["theta"], tok["Bm"], tok["Cm"], d["Dskip"], state, d.get("x_prev"),
+                                      d.get("B_prev"), y=y)
+    return step, (d, tok, state, y)
+
+
+def run_m3_decode(mm, args, world, hbm_peak, hbm_src):
+    """One decode token of the Mamba-3 form for 512 sequences at d_inner 8192
+    (128 heads of 64, d_state 16, one input, the previous token given): one
+    launch, in place on a 268 MB fp32 state (larger than L2).  Roofline: the
+    state's read and write plus the token's activations against the copy
+    bandwidth."""
+    cfg = M3_DEC
+    step, keep = _m3_decode_setup(mm, cfg)
+    K = max(3, min(args.steps, 200))
+    ms = _time_loop(step, K, world)
+    nbytes = m3_decode_bytes(cfg)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    del keep, step
+    torch.cuda.empty_cache()
+    return {
+        "workload": cfg.name, "batch": cfg.batch, "heads": cfg.heads, "headdim": cfg.headdim,
+        "d_state": cfg.d_state, "rank": cfg.rank, "steps": K, "ms_per_step": round(ms, 5),
+        "value": round(_job_rate(world, cfg.batch, ms), 1), "unit": "tokens/s", "launches_per_call": 1,
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(gbs / hbm_peak, 4), "traffic": _ncu_traffic("m3/mamba3_decode"),
+                     "algorithmic_bytes": nbytes, "peak_source": hbm_src},
+    }
+
+
 def run_m3(mm, args, world, hbm_peak, hbm_src, alu_peak, cfg):
     """The Mamba-3 form on 4096 tokens of 128 heads (d_state 16): a summary
     pass and a full pass per call (fp32 recurrence on the CUDA cores), inputs
@@ -1038,6 +1086,8 @@ def run_only(args):
         step = lambda: _ssd_call(mm, d, out, ws)  # noqa: E731
     elif args.only == "ssddecode":
         step, keep = _ssd_decode_setup(mm, SSD_DEC)
+    elif args.only == "m3decode":
+        step, keep = _m3_decode_setup(mm, M3_DEC)
     elif args.only in ("m3", "m3mimo"):
         cfg = M3 if args.only == "m3" else M3_MIMO
         d = {k: (v.cuda() if v is not None else None) for k, v in make_m3_inputs(cfg).items()}
@@ -1087,7 +1137,7 @@ def main():
     ap.add_argument("--no-extra-prefill", action="store_true",
                     help="skip the 4 x 32768 and 262,144-token prefill legs")
     ap.add_argument("--only", choices=["forward", "decode", "xproj", "dtproj", "projected", "ssd", "ssddecode", "m3",
-                                       "m3mimo"],
+                                       "m3mimo", "m3decode"],
                     default=None,
                     help="run one kernel's timed loop only (for profiler captures); prints no JSON line")
     ap.add_argument("--decode-layers", type=int, default=None,

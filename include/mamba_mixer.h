@@ -19,6 +19,7 @@
  *   mamba_ssd_fwd            Mamba-2 prefill (scalar decay per head, chunked products on the tensor cores)
  *   mamba_ssd_state_update   Mamba-2 one-token step (decode), in place on the state
  *   mamba_m3_fwd             Mamba-3 prefill (trapezoid rule, complex state, 1/2/4 inputs per state)
+ *   mamba_m3_state_update    Mamba-3 one-token step (decode), in place on the state
  *
  * and two status readers:
  *   mamba_check_status       did the last forward on this workspace complete? (per call)
@@ -548,6 +549,40 @@ mm_status mamba_m3_fwd(const void* x, const void* z, const void* dt, const void*
 /* Workspace bytes of mamba_m3_fwd for these sizes (0 if not supported). */
 size_t mamba_m3_workspace_size(int64_t batch, int64_t seqlen, int64_t rank, int64_t heads, int64_t headdim,
                                int64_t d_state, int64_t groups);
+
+/*
+ * One token of the Mamba-3 form (decode), in place on the state: the
+ * recurrence of mamba_m3_fwd above for a single token t, with the state the
+ * previous call left as h_last and the previous token's input:
+ *
+ *   s[k]   = a_t[k] (s[k] + (1 - lambda_t) Delta_t u_prev[k]) + lambda_t Delta_t u_t[k]
+ *   y[r,c] = (sum_k Re(conj(C_t[r,g,k]) s[k]) + D[h] x_t[r,c]) * SiLU(z_t[r,c])
+ *
+ * with a_t, u_t, Delta_t and lambda_t as defined there and u_prev the input
+ * of the token before (x_prev, B_prev; zero when both are NULL).  A decode
+ * loop passes, at each step, the previous step's x and B rows as x_prev and
+ * B_prev.
+ *
+ *   x, z           [batch, rank, heads*headdim]     bf16  (z may be NULL)
+ *   dt, trap       [batch, heads]                   bf16  (trap may be NULL: 1/2)
+ *   dt_bias        [heads] fp32 or NULL;  A [heads] fp32 (negative)
+ *   theta          [heads, d_state/2]               fp32
+ *   Bm, Cm         [batch, rank, groups, d_state]   bf16
+ *   Dskip          [heads] fp32 or NULL
+ *   state          [batch, heads, headdim, d_state] fp32  read and overwritten
+ *   x_prev, B_prev [batch, rank, heads*headdim], [batch, rank, groups, d_state]  bf16  or both NULL
+ *   y              [batch, rank, heads*headdim]     bf16  output
+ *
+ * The same results as mamba_m3_fwd with seqlen 1, h0 = state and h_last =
+ * state, up to rounding order.  Supported sizes and errors as mamba_m3_fwd
+ * (no workspace, no wait); state and y may not overlap an input or each other
+ * (MM_ERR_ALIAS).  One launch on `stream`; batch == 0 is a no-op.
+ */
+mm_status mamba_m3_state_update(const void* x, const void* z, const void* dt, const void* trap, const float* dt_bias,
+                                const float* A, const float* theta, const void* Bm, const void* Cm,
+                                const float* Dskip, float* state, const void* x_prev, const void* B_prev, void* y,
+                                int64_t batch, int64_t rank, int64_t heads, int64_t headdim, int64_t d_state,
+                                int64_t groups, void* stream);
 
 /* A static, human-readable name for a status code. */
 const char* mamba_status_string(mm_status status);

@@ -17,7 +17,7 @@ __all__ = [
     "MM_F32", "MM_BF16", "MixerError", "lib", "library_path", "mixer_fwd", "mixer_fwd_noalloc", "mixer_fwd_host",
     "state_update", "workspace_size", "host_workspace_size", "status_string", "abi_version", "fault_status",
     "check_status", "proj_matmul", "proj_matmul_workspace_size", "mixer_fwd_projected",
-    "projected_workspace_size", "ssd_fwd", "ssd_workspace_size", "ssd_state_update", "m3_fwd", "m3_workspace_size", "EXPORTED_SYMBOLS",
+    "projected_workspace_size", "ssd_fwd", "ssd_workspace_size", "ssd_state_update", "m3_fwd", "m3_state_update", "m3_workspace_size", "EXPORTED_SYMBOLS",
 ]
 
 MM_F32 = 0
@@ -50,6 +50,7 @@ EXPORTED_SYMBOLS = (
     "mamba_ssd_state_update",
     "mamba_m3_fwd",
     "mamba_m3_workspace_size",
+    "mamba_m3_state_update",
 )
 
 
@@ -120,6 +121,8 @@ def _declare(L):
     L.mamba_m3_fwd.argtypes = [P] * 15 + [I64] * 7 + [P, ctypes.c_size_t, P]
     L.mamba_m3_workspace_size.restype = ctypes.c_size_t
     L.mamba_m3_workspace_size.argtypes = [I64] * 7
+    L.mamba_m3_state_update.restype = ctypes.c_int
+    L.mamba_m3_state_update.argtypes = [P] * 14 + [I64] * 6 + [P]
     return L
 
 
@@ -713,3 +716,50 @@ def m3_fwd(x, z, dt, trap, dt_bias, A, theta, Bm, Cm, Dskip, h0=None, x_prev=Non
         raise MixerError(st, "mamba_m3_fwd")
     _keep_alive_on(made, (stream,))
     return y, h_last
+
+
+def m3_state_update(x, z, dt, trap, dt_bias, A, theta, Bm, Cm, Dskip, state, x_prev=None, B_prev=None, *,
+                    headdim=64, y=None, stream=None):
+    """One token of the Mamba-3 form (mamba_m3_state_update), in place on
+    state [B,H,P,N] fp32: x, z [B,R,H*P] bf16 (z may be None: no gate), dt and
+    trap [B,H] bf16 (trap None: 1/2), dt_bias/A/Dskip [H] fp32 (dt_bias and
+    Dskip may be None), theta [H,N/2] fp32, Bm/Cm [B,R,G,N] bf16, x_prev
+    [B,R,H*P] and B_prev [B,R,G,N] bf16 (the previous token's) or None, P =
+    headdim.  Returns y [B,R,H*P] bf16, allocated if not given."""
+    import torch
+
+    bf, f32 = torch.bfloat16, torch.float32
+    Bsz, R, HP = x.shape
+    H = A.shape[0]
+    P = int(headdim)
+    G, N = Bm.shape[2], Bm.shape[3]
+    if HP != H * P:
+        raise ValueError(f"x has {HP} channels, expected heads x headdim = {H * P}")
+    dev = x.device
+    made = []
+    _check(x, "x", bf, (Bsz, R, H * P), dev)
+    _check(z, "z", bf, (Bsz, R, H * P), dev)
+    _check(dt, "dt", bf, (Bsz, H), dev)
+    _check(trap, "trap", bf, (Bsz, H), dev)
+    _check(dt_bias, "dt_bias", f32, (H,), dev)
+    _check(A, "A", f32, (H,), dev)
+    _check(theta, "theta", f32, (H, N // 2), dev)
+    _check(Bm, "Bm", bf, (Bsz, R, G, N), dev)
+    _check(Cm, "Cm", bf, (Bsz, R, G, N), dev)
+    _check(Dskip, "Dskip", f32, (H,), dev)
+    _check(state, "state", f32, (Bsz, H, P, N), dev)
+    _check(x_prev, "x_prev", bf, (Bsz, R, H * P), dev)
+    _check(B_prev, "B_prev", bf, (Bsz, R, G, N), dev)
+    if y is None:
+        y = torch.empty((Bsz, R, H * P), dtype=bf, device=dev)
+        made.append(y)
+    _check(y, "y", bf, (Bsz, R, H * P), dev)
+    with torch.cuda.device(dev):
+        st = lib().mamba_m3_state_update(_ptr(x), _ptr(z), _ptr(dt), _ptr(trap), _ptr(dt_bias), _ptr(A),
+                                         _ptr(theta), _ptr(Bm), _ptr(Cm), _ptr(Dskip), _ptr(state), _ptr(x_prev),
+                                         _ptr(B_prev), _ptr(y), Bsz, R, H, P, N, G, _stream_handle(stream))
+    if st != 0:
+        raise MixerError(st, "mamba_m3_state_update")
+    _keep_alive_on(made, (stream,))
+    return y
+

@@ -143,7 +143,7 @@ __device__ __forceinline__ float4 m3_widen4(uint2 v) {
 // Thread j's channel input u of one token (or of the token before the call):
 // sum_r (B[r, 2k] + i B[r, 2k+1]) x[r], from global rows, as (re, im) pairs.
 template <int R>
-__device__ __forceinline__ void m3_input_global(const M3Params& p, const __nv_bfloat16* xrow,
+__device__ __forceinline__ void m3_input_global(const __nv_bfloat16* xrow,
                                                 const __nv_bfloat16* brow, int64_t x_rstride,
                                                 int64_t b_rstride, float2 (&u)[kM3Pairs]) {
 #pragma unroll
@@ -274,7 +274,7 @@ m3_chunk_kernel(const M3Params p)
 #pragma unroll
             for (int j = 0; j < kM3Cpt; ++j) {
                 float2 up[kM3Pairs];
-                m3_input_global<R>(p, p.x_prev + static_cast<int64_t>(b) * R * C + c + j,
+                m3_input_global<R>(p.x_prev + static_cast<int64_t>(b) * R * C + c + j,
                                 p.B_prev + static_cast<int64_t>(b) * R * br + g * kM3N, xr, br, up);
 #pragma unroll
                 for (int q = 0; q < kM3Pairs / 2; ++q) {
@@ -561,6 +561,168 @@ m3_chunk_kernel(const M3Params p)
             pp[0] = prod.x;
             pp[1] = prod.y;
         }
+    }
+}
+
+
+// ---------------------------------------------------------------- one-token step (decode)
+// One token of the recurrence above per channel, in place on the state s
+// (not the pre-state: the state a prefill leaves as h_last):
+//     s[k] <- a[k] (s[k] + (1 - lambda) Delta u_prev[k]) + lambda Delta u[k]
+//     y[r] = (sum_k Re(conj(C[r,k]) s[k]) + D x[r]) SiLU(z[r])
+// with u_prev the previous token's input (x_prev, B_prev; zero when absent).
+// Each channel's 16 state floats are read and written once: the step is
+// bound by that HBM traffic.  A CTA covers two heads (128 channels, one per
+// thread), a warp 32 channels of one head: each lane computes a[k] for pair
+// k = lane mod 8 and the warp passes them round by shuffles, so no warp waits
+// on another; the head's B and C rows are read by every lane of the warp
+// (the same 16-byte pieces, served by L1).  The warp's 2 KB of state moves
+// through shared memory so that global loads and stores are whole lines.
+struct M3DecodeParams {
+    const __nv_bfloat16* x;        // [B][R][H*P]
+    const __nv_bfloat16* z;        // [B][R][H*P] or null
+    const __nv_bfloat16* dt;       // [B][H]
+    const __nv_bfloat16* trap;     // [B][H] or null (1/2)
+    const float* dt_bias;          // [H] or null
+    const float* A;                // [H]
+    const float* theta;            // [H][N/2]
+    const __nv_bfloat16* Bm;       // [B][R][G][N]
+    const __nv_bfloat16* Cm;       // [B][R][G][N]
+    const float* Dskip;            // [H] or null
+    float* state;                  // [B][H][P][N], updated in place
+    const __nv_bfloat16* x_prev;   // [B][R][H*P] or null
+    const __nv_bfloat16* B_prev;   // [B][R][G][N] or null
+    __nv_bfloat16* y;              // [B][R][H*P]
+    int H, G;
+};
+constexpr int kM3DecThreads = kM3Threads;    // one channel per thread, two heads per CTA
+
+// Position, in a warp's [32 channels][4 pieces] staging area, of 16-byte
+// piece i = 4 channel + piece: XORing the low three bits with bits 3..4 keeps
+// both the coalesced order (i = 32 q + lane) and the per-channel order
+// (i = 4 lane + piece) free of shared-memory bank conflicts.
+__device__ __forceinline__ int m3_dec_slot(int i) { return i ^ ((i >> 3) & 3); }
+
+template <int R>
+__global__ void __launch_bounds__(kM3DecThreads)
+m3_state_update_kernel(const M3DecodeParams p)
+{
+    __shared__ float4 stage[kM3DecThreads / 32][32 * (kM3N / 4)];   // per warp: 32 channels' states
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, b = blockIdx.y;
+    const int h = blockIdx.x * kM3Heads + tid / kM3P;      // a warp's 32 channels share one head
+    const int64_t C = static_cast<int64_t>(p.H) * kM3P;
+    const int64_t c = static_cast<int64_t>(blockIdx.x) * kM3Threads + tid;
+    const int64_t br = static_cast<int64_t>(p.G) * kM3N;
+    const int g = h * p.G / p.H;
+    const bool prev = p.x_prev && p.B_prev;
+    float4* st = stage[warp];
+
+    // every load first.  The warp's 32 channel states are 2 KB of contiguous
+    // memory: loaded as four 512-byte warp-wide pieces and passed through
+    // shared memory, so each load and store instruction moves whole lines.
+    float4* wp = reinterpret_cast<float4*>(p.state) + (static_cast<int64_t>(b) * C + (c - lane)) * (kM3N / 4);
+    float4 lv[kM3N / 4];
+#pragma unroll
+    for (int q = 0; q < kM3N / 4; ++q) lv[q] = wp[32 * q + lane];
+    const int64_t e = static_cast<int64_t>(b) * p.H + h;
+    const float v = __bfloat162float(p.dt[e]) + (p.dt_bias ? p.dt_bias[h] : 0.0f);
+    const float lam = p.trap ? __bfloat162float(p.trap[e]) : 0.5f;
+    const float th = p.theta[h * kM3Pairs + (lane & (kM3Pairs - 1))];
+    const float Ah = p.A[h];
+    const float dh = p.Dskip ? p.Dskip[h] : 0.0f;
+    uint4 bp[R][2], bt[R][2], ct[R][2];
+    float xv[R], xp[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int64_t ro = (static_cast<int64_t>(b) * R + r) * br + g * kM3N;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            bt[r][half] = *reinterpret_cast<const uint4*>(p.Bm + ro + 8 * half);
+            ct[r][half] = *reinterpret_cast<const uint4*>(p.Cm + ro + 8 * half);
+            bp[r][half] = prev ? *reinterpret_cast<const uint4*>(p.B_prev + ro + 8 * half) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        const int64_t xi = (static_cast<int64_t>(b) * R + r) * C + c;
+        xv[r] = __bfloat162float(p.x[xi]);
+        xp[r] = prev ? __bfloat162float(p.x_prev[xi]) : 0.0f;
+    }
+#pragma unroll
+    for (int q = 0; q < kM3N / 4; ++q) st[m3_dec_slot(32 * q + lane)] = lv[q];
+    __syncwarp();
+    float4 sv[kM3N / 4];
+#pragma unroll
+    for (int q = 0; q < kM3N / 4; ++q) sv[q] = st[m3_dec_slot(4 * lane + q)];   // (re, im) of pairs 2q, 2q+1
+
+    // the head's step and tap weights (every lane), and a[k] for pair
+    // k = lane mod 8, passed round the warp
+    const float dl = fmaxf(v, 0.0f) + log1pf(expf(-fabsf(v)));
+    const float2 w = make_float2((1.0f - lam) * dl, lam * dl);
+    float sn, cs;
+    m3_sincos(dl * th, &sn, &cs);
+    const float mag = ex2_fast(dl * Ah * kLog2e);
+    const float ar_mine = mag * cs, ai_mine = mag * sn;
+
+    // u_prev and u: sum_r (B[r,2k] + i B[r,2k+1]) x[r]
+    float2 up[kM3Pairs], u[kM3Pairs];
+#pragma unroll
+    for (int k = 0; k < kM3Pairs; ++k) up[k] = u[k] = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const uint32_t bpw[4] = {bp[r][half].x, bp[r][half].y, bp[r][half].z, bp[r][half].w};
+            const uint32_t btw[4] = {bt[r][half].x, bt[r][half].y, bt[r][half].z, bt[r][half].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {      // pair 4 half + j: (re, im) in one 32-bit word
+                const int k = 4 * half + j;
+                up[k].x = fmaf(__uint_as_float(bpw[j] << 16), xp[r], up[k].x);
+                up[k].y = fmaf(__uint_as_float(bpw[j] & 0xffff0000u), xp[r], up[k].y);
+                u[k].x = fmaf(__uint_as_float(btw[j] << 16), xv[r], u[k].x);
+                u[k].y = fmaf(__uint_as_float(btw[j] & 0xffff0000u), xv[r], u[k].y);
+            }
+        }
+    }
+    // the state's input from the previous token, the rotation-decay, then
+    // this token's input
+    float2 s[kM3Pairs];
+#pragma unroll
+    for (int q = 0; q < kM3N / 4; ++q) {
+        s[2 * q] = make_float2(fmaf(w.x, up[2 * q].x, sv[q].x), fmaf(w.x, up[2 * q].y, sv[q].y));
+        s[2 * q + 1] = make_float2(fmaf(w.x, up[2 * q + 1].x, sv[q].z), fmaf(w.x, up[2 * q + 1].y, sv[q].w));
+    }
+#pragma unroll
+    for (int k = 0; k < kM3Pairs; ++k) {
+        const float ar = __shfl_sync(kFull, ar_mine, k), ai = __shfl_sync(kFull, ai_mine, k);
+        const float re = fmaf(ar, s[k].x, -ai * s[k].y);
+        const float im = fmaf(ar, s[k].y, ai * s[k].x);
+        s[k] = make_float2(fmaf(w.y, u[k].x, re), fmaf(w.y, u[k].y, im));
+    }
+    // back through shared memory to whole-line stores
+#pragma unroll
+    for (int q = 0; q < kM3N / 4; ++q)
+        st[m3_dec_slot(4 * lane + q)] = make_float4(s[2 * q].x, s[2 * q].y, s[2 * q + 1].x, s[2 * q + 1].y);
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < kM3N / 4; ++q) wp[32 * q + lane] = st[m3_dec_slot(32 * q + lane)];
+
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int64_t xi = (static_cast<int64_t>(b) * R + r) * C + c;
+        float yv = 0.0f;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const uint32_t cw[4] = {ct[r][half].x, ct[r][half].y, ct[r][half].z, ct[r][half].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int k = 4 * half + j;
+                yv = fmaf(__uint_as_float(cw[j] << 16), s[k].x, fmaf(__uint_as_float(cw[j] & 0xffff0000u), s[k].y, yv));
+            }
+        }
+        yv = fmaf(dh, xv[r], yv);
+        if (p.z) {
+            const float zv = __bfloat162float(p.z[xi]);
+            yv *= zv / (1.0f + expf(-zv));
+        }
+        p.y[xi] = __float2bfloat16_rn(yv);
     }
 }
 

@@ -1788,4 +1788,61 @@ mm_status mamba_m3_fwd(const void* x, const void* z, const void* dt, const void*
     return MM_OK;
 }
 
+mm_status mamba_m3_state_update(const void* x, const void* z, const void* dt, const void* trap, const float* dt_bias,
+                                const float* A, const float* theta, const void* Bm, const void* Cm,
+                                const float* Dskip, float* state, const void* x_prev, const void* B_prev, void* y,
+                                int64_t batch, int64_t rank, int64_t heads, int64_t headdim, int64_t d_state,
+                                int64_t groups, void* stream)
+{
+    if (headdim != mm::kM3P || d_state != mm::kM3N) return MM_ERR_UNSUPPORTED;
+    if (rank != 1 && rank != 2 && rank != 4) return MM_ERR_UNSUPPORTED;
+    if (heads > 0 && heads % mm::kM3Heads != 0) return MM_ERR_UNSUPPORTED;
+    if (!m3_sizes_ok(batch, 1, rank, heads, groups)) return MM_ERR_SHAPE;
+    if (batch == 0) return MM_OK;
+    if (!x || !dt || !A || !theta || !Bm || !Cm || !state || !y) return MM_ERR_NULL;
+    if ((x_prev == nullptr) != (B_prev == nullptr)) return MM_ERR_NULL;
+    for (const void* q : {x, z, dt, trap, static_cast<const void*>(dt_bias), static_cast<const void*>(A),
+                          static_cast<const void*>(theta), Bm, Cm, static_cast<const void*>(Dskip),
+                          static_cast<const void*>(state), x_prev, B_prev, static_cast<const void*>(y)})
+        if (q && !aligned16(q)) return MM_ERR_ALIGN;
+    const int64_t C = heads * mm::kM3P;
+    const int64_t bc = groups * mm::kM3N;
+    const Span sx = span(x, batch * rank * C * 2), sz = span(z, batch * rank * C * 2),
+               sdt = span(dt, batch * heads * 2), str = span(trap, batch * heads * 2),
+               sbias = span(dt_bias, heads * 4), sa = span(A, heads * 4), sth = span(theta, heads * mm::kM3Pairs * 4),
+               sb = span(Bm, batch * rank * bc * 2), sc = span(Cm, batch * rank * bc * 2), sd = span(Dskip, heads * 4),
+               sxp = span(x_prev, batch * rank * C * 2), sbp = span(B_prev, batch * rank * bc * 2),
+               sst = span(state, batch * C * mm::kM3N * 4), sy = span(y, batch * rank * C * 2);
+    const Span ins[] = {sx, sz, sdt, str, sbias, sa, sth, sb, sc, sd, sxp, sbp};
+    for (const Span& in : ins)
+        if (overlaps(sy, in) || overlaps(sst, in)) return MM_ERR_ALIAS;
+    if (overlaps(sy, sst)) return MM_ERR_ALIAS;
+    if (mm_status st = check_device(); st != MM_OK) return st;
+
+    mm::M3DecodeParams p{};
+    p.x = static_cast<const __nv_bfloat16*>(x);
+    p.z = static_cast<const __nv_bfloat16*>(z);
+    p.dt = static_cast<const __nv_bfloat16*>(dt);
+    p.trap = static_cast<const __nv_bfloat16*>(trap);
+    p.dt_bias = dt_bias;
+    p.A = A;
+    p.theta = theta;
+    p.Bm = static_cast<const __nv_bfloat16*>(Bm);
+    p.Cm = static_cast<const __nv_bfloat16*>(Cm);
+    p.Dskip = Dskip;
+    p.state = state;
+    p.x_prev = static_cast<const __nv_bfloat16*>(x_prev);
+    p.B_prev = static_cast<const __nv_bfloat16*>(B_prev);
+    p.y = static_cast<__nv_bfloat16*>(y);
+    p.H = static_cast<int>(heads);
+    p.G = static_cast<int>(groups);
+    const dim3 grid(static_cast<unsigned>(heads / mm::kM3Heads), static_cast<unsigned>(batch));
+    const size_t smem = forced_launch_failure() ? (size_t(1) << 20) : 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (rank == 1) mm::m3_state_update_kernel<1><<<grid, mm::kM3DecThreads, smem, s>>>(p);
+    else if (rank == 2) mm::m3_state_update_kernel<2><<<grid, mm::kM3DecThreads, smem, s>>>(p);
+    else mm::m3_state_update_kernel<4><<<grid, mm::kM3DecThreads, smem, s>>>(p);
+    return cudaGetLastError() == cudaSuccess ? MM_OK : MM_ERR_CUDA;
+}
+
 }  // extern "C"

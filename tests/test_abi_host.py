@@ -616,3 +616,32 @@ def test_plain_c_program_uses_the_abi(L, tmp_path):
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0, (out.returncode, out.stderr)
     assert out.stdout.strip() == str(ws_bytes(1, 9, 8192))
+
+
+def m3_decode_args(B=2, R=2, H=4, P=64, N=16, G=2, **over):
+    """mamba_m3_state_update arguments on fake addresses, each buffer 2^32 apart."""
+    names = ["x", "z", "dt", "trap", "dt_bias", "A", "theta", "Bm", "Cm", "Dskip", "state", "x_prev", "B_prev", "y"]
+    addr = {n: BASE + (i << 32) for i, n in enumerate(names)}
+    addr.update(over)
+    return [addr[n] for n in names] + [B, R, H, P, N, G, None]
+
+
+def test_m3_decode_validation(L):
+    assert L.mamba_m3_state_update(*m3_decode_args()) == EDEVICE
+    assert L.mamba_m3_state_update(*m3_decode_args(z=None, trap=None, dt_bias=None, Dskip=None, x_prev=None,
+                                                   B_prev=None)) == EDEVICE
+    assert L.mamba_m3_state_update(*m3_decode_args(P=32)) == EUNSUP
+    assert L.mamba_m3_state_update(*m3_decode_args(N=32)) == EUNSUP
+    assert L.mamba_m3_state_update(*m3_decode_args(R=3)) == EUNSUP
+    assert L.mamba_m3_state_update(*m3_decode_args(H=3, G=1)) == EUNSUP
+    assert L.mamba_m3_state_update(*m3_decode_args(H=6, G=4)) == ESHAPE
+    assert L.mamba_m3_state_update(*m3_decode_args(B=-1)) == ESHAPE
+    assert L.mamba_m3_state_update(*m3_decode_args(B=0)) == OK
+    for name in ("x", "dt", "A", "theta", "Bm", "Cm", "state", "y"):
+        assert L.mamba_m3_state_update(*m3_decode_args(**{name: None})) == ENULL, name
+    assert L.mamba_m3_state_update(*m3_decode_args(x_prev=None)) == ENULL      # x_prev and B_prev together
+    for name in ("x", "trap", "theta", "state", "B_prev", "y"):
+        assert L.mamba_m3_state_update(*m3_decode_args(**{name: BASE + (1 << 40) + 8})) == EALIGN, name
+    assert L.mamba_m3_state_update(*m3_decode_args(y=BASE)) == EALIAS                   # y over x
+    assert L.mamba_m3_state_update(*m3_decode_args(state=BASE + (7 << 32))) == EALIAS   # state over B
+    assert L.mamba_m3_state_update(*m3_decode_args(y=BASE + (10 << 32) + 64)) == EALIAS # y over state

@@ -184,3 +184,116 @@ def test_m3_token_by_token_continues_prefill():
         ys.append(y)
     torch.cuda.synchronize()
     check(inp, torch.cat(ys, dim=1), h)
+
+
+# ---------------------------------------------------------------- one-token step (decode)
+def gpu_m3_decode(d, state=None, x_prev=None, B_prev=None, use_prev=True):
+    """mamba_m3_state_update on the first token of one-token inputs d, in
+    place on `state` (a copy of d's h0, or zeros, when not given), with d's
+    x_prev / B_prev unless others are given.  Returns y [B,1,R,H*P] and the
+    state."""
+    B, _, R, C = d["x"].shape
+    H = d["A"].shape[0]
+    if state is None:
+        state = d["h0"].clone() if d.get("h0") is not None else torch.zeros((B, H, 64, 16), device="cuda")
+    if use_prev and x_prev is None:
+        x_prev, B_prev = d.get("x_prev"), d.get("B_prev")
+    tok = {k: (d[k][:, 0].contiguous() if d.get(k) is not None else None)
+           for k in ("x", "z", "dt", "trap", "Bm", "Cm")}
+    y = mm.m3_state_update(tok["x"], tok["z"], tok["dt"], tok["trap"], d.get("dt_bias"), d["A"], d["theta"],
+                           tok["Bm"], tok["Cm"], d.get("Dskip"), state, x_prev, B_prev)
+    return y[:, None], state
+
+
+@pytest.mark.parametrize("B,R,H,G,prev,h0,gate,trap", [(1, 1, 2, 1, False, False, True, True),
+                                                       (2, 1, 4, 2, True, True, True, True),
+                                                       (3, 2, 2, 1, True, True, False, True),
+                                                       (2, 4, 4, 4, True, True, True, False),
+                                                       (5, 4, 2, 2, False, True, True, True)])
+def test_m3_decode_small(B, R, H, G, prev, h0, gate, trap):
+    """One token against the oracle's one-token run from the same state and
+    previous token."""
+    inp = make_m3_inputs_custom(B, 1, H, rank=R, groups=G, seed=500 + B * 13 + R * 7 + H, h0_std=0.3 if h0 else 0.0,
+                                prev=prev, gate=gate, trap=trap)
+    y, state = gpu_m3_decode(to_dev(inp))
+    torch.cuda.synchronize()
+    check(inp, y, state)
+
+
+def test_m3_decode_optional_parameters():
+    """No dt_bias and no skip."""
+    inp = make_m3_inputs_custom(2, 1, 4, rank=2, seed=61, h0_std=0.3, prev=True)
+    inp["dt_bias"] = None
+    inp["Dskip"] = None
+    y, state = gpu_m3_decode(to_dev(inp))
+    torch.cuda.synchronize()
+    check(inp, y, state)
+
+
+def test_m3_decode_large_steps():
+    """Large and small step sizes: softplus on both tails, rotation angles
+    of many turns."""
+    inp = make_m3_inputs_custom(2, 1, 4, rank=1, seed=63, h0_std=0.5, prev=True, dt_std=4.0)
+    y, state = gpu_m3_decode(to_dev(inp))
+    torch.cuda.synchronize()
+    check(inp, y, state)
+
+
+def test_m3_decode_continues_prefill():
+    """Decode use: a prefill of 45 tokens, then three decode steps in place on
+    its h_last, each given the token before as x_prev / B_prev, match the
+    oracle's single run of all 48 tokens."""
+    inp = make_m3_inputs_custom(2, 48, 4, rank=2, groups=2, seed=49, h0_std=0.2, prev=True)
+    d = to_dev(inp)
+    c = dict(d)
+    for k in ("x", "z", "dt", "trap", "Bm", "Cm"):
+        c[k] = d[k][:, :45].contiguous()
+    y0, state = gpu_m3(c)
+    ys = [y0]
+    for t in range(45, 48):
+        c = dict(d)
+        for k in ("x", "z", "dt", "trap", "Bm", "Cm"):
+            c[k] = d[k][:, t:t + 1].contiguous()
+        y, state = gpu_m3_decode(c, state, d["x"][:, t - 1].contiguous(), d["Bm"][:, t - 1].contiguous())
+        ys.append(y)
+    torch.cuda.synchronize()
+    check(inp, torch.cat(ys, dim=1), state)
+
+
+def test_m3_decode_full_size():
+    """The decode workload at full size (512 sequences x 128 heads of 64,
+    d_state 16, one input, the previous token given), as the bench times it:
+    every channel against the oracle."""
+    inp = make_m3_inputs(M3_CONFIGS["mamba3_decode"])
+    y, state = gpu_m3_decode(to_dev(inp))
+    torch.cuda.synchronize()
+    check(inp, y, state)
+
+
+def test_m3_decode_graph_replay():
+    """Captured in a CUDA graph, two replays from the same state give the
+    bits of two eager calls."""
+    inp = make_m3_inputs_custom(2, 1, 4, rank=2, seed=65, h0_std=0.3, prev=True)
+    d = to_dev(inp)
+    s_eager = d["h0"].clone()
+    ye1, _ = gpu_m3_decode(d, s_eager)
+    ye2, _ = gpu_m3_decode(d, s_eager)
+    tok = {k: d[k][:, 0].contiguous() for k in ("x", "z", "dt", "trap", "Bm", "Cm")}
+    args = lambda st, y: mm.m3_state_update(tok["x"], tok["z"], tok["dt"], tok["trap"], d["dt_bias"], d["A"],  # noqa: E731
+                                            d["theta"], tok["Bm"], tok["Cm"], d["Dskip"], st, d["x_prev"],
+                                            d["B_prev"], y=y)
+    yg = torch.empty_like(ye1[:, 0])
+    args(d["h0"].clone(), yg)                     # warm-up outside the capture
+    torch.cuda.synchronize()
+    s_graph = d["h0"].clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        args(s_graph, yg)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(yg, ye1[:, 0])
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(yg, ye2[:, 0])
+    assert torch.equal(s_graph, s_eager)
+

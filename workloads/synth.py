@@ -419,6 +419,10 @@ M3_CONFIGS = {
     "mamba3_mimo": M3Config(
         "mamba3_mimo", batch=1, seqlen=4096, heads=128, rank=4, seed=8, h0_std=0.1, prev=True,
         desc="Mamba-3 form with 4 inputs and outputs per state, an initial state and a previous token"),
+    "mamba3_decode": M3Config(
+        "mamba3_decode", batch=512, seqlen=1, heads=128, seed=9, h0_std=0.3, prev=True,
+        desc="Mamba-3 form, one decode token for 512 sequences at the Jamba width (a 268 MB fp32 state), "
+             "the previous token given"),
 }
 
 
