@@ -598,7 +598,7 @@ struct M3DecodeParams {
 constexpr int kM3DecThreads = kM3Threads;    // one channel per thread, two heads per CTA
 
 // Position, in a warp's [32 channels][4 pieces] staging area, of 16-byte
-// piece i = 4 channel + piece: XORing the low three bits with bits 3..4 keeps
+// piece i = 4 channel + piece: XORing bits 0..1 with bits 3..4 keeps
 // both the coalesced order (i = 32 q + lane) and the per-channel order
 // (i = 4 lane + piece) free of shared-memory bank conflicts.
 __device__ __forceinline__ int m3_dec_slot(int i) { return i ^ ((i >> 3) & 3); }
